@@ -1,0 +1,249 @@
+/*
+ * mxq.h -- C ABI of the B200 (sm_100a) microscaling quantized-linear library.
+ *
+ * The library implements the data-parallel hot path of low-bit diffusion
+ * inference described by these pages:
+ *   - Chameleon article (rit.work, "Chameleon ... format quantization for
+ *     diffusion"): per-output-channel weight format chosen by least
+ *     reconstruction error; per-layer, per-timestep-interval activation
+ *     format table read at run time; MXFP8 forced where channel ranges reach
+ *     163x.
+ *   - Nunchaku / Diffusers article (jiti.kz): svdq_w4a4 -- W4A4 linear layers
+ *     in INT4 and NVFP4 with a 16-bit low-rank branch (SVDQuant).
+ *   - "Bridging the Gap Between Promise and Performance for Microscaling FP4
+ *     Quantization": NVFP4 / MXFP4, block-diagonal Hadamard rotation.
+ * Bit layouts follow the OCP Microscaling (MX) v1.0 definition and NVIDIA's
+ * NVFP4 definition (the pages name the formats without defining them).
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked "device" are caller-owned CUDA device memory; the
+ *     library never allocates or frees on any call (TMEM used by the GEMM
+ *     is allocated and released inside the kernel).  "host" pointers are
+ *     read during the call only.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream) unless stated otherwise.
+ *   - Matrices are row-major.  X is M x K, W is N x K (K contiguous, the
+ *     torch Linear layout), Y = X . W^T is M x N.  Quantization blocks run
+ *     along the contiguous (K) dimension.
+ *   - 4-bit codes are packed two per byte, element 2i in the low nibble.
+ *   - Errors are returned as mxq_status; nothing aborts or throws.  Argument
+ *     errors are detected on the host before any launch.  A device-side
+ *     bounded wait that runs out is latched in a device error word and
+ *     reported by mxq_check().
+ */
+#ifndef MXQ_H
+#define MXQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mxq_status {
+    MXQ_OK = 0,
+    MXQ_EINVAL = 1,         /* bad argument (shape, pointer, size, enum)          */
+    MXQ_EUNSUPPORTED = 2,   /* valid but unsupported combination, or no sm_100 GPU */
+    MXQ_ECUDA = 3,          /* a CUDA runtime/driver call failed                   */
+    MXQ_ETIMEOUT = 4,       /* a bounded device wait ran out (see mxq_check)       */
+    MXQ_ENOSPACE = 5        /* workspace smaller than the *_workspace_bytes query  */
+} mxq_status;
+
+/* Formats.  Block sizes are fixed by the format. */
+typedef enum mxq_fmt {
+    MXQ_MXFP8 = 0,       /* E4M3 codes, 32-element blocks, E8M0 scale (OCP MX)        */
+    MXQ_MXFP4 = 1,       /* E2M1 codes, 32-element blocks, E8M0 scale (OCP MX)        */
+    MXQ_NVFP4 = 2,       /* E2M1 codes, 16-element blocks, E4M3 scale, fp32 tensor scale */
+    MXQ_INT4_G32 = 3,    /* symmetric int4 [-7,7], fp32 scale per 32 elements          */
+    MXQ_INT4_G64 = 4,    /* symmetric int4 [-7,7], fp32 scale per 64 elements          */
+    MXQ_INT8_ROW = 5,    /* symmetric int8 [-127,127], fp32 scale per row (per token / per output channel) */
+    MXQ_FP8_TENSOR = 6,  /* E4M3 codes, one fp32 scale for the whole tensor            */
+    MXQ_NUM_FMT = 7
+} mxq_fmt;
+
+typedef enum mxq_dtype { MXQ_F32 = 0, MXQ_BF16 = 1 } mxq_dtype;
+
+/* Layout of the codes and scales a quantizer writes.
+ *  CANONICAL: codes as above; scales row-major
+ *      MXFP8/MXFP4  uint8 E8M0 [rows][cols/32]
+ *      NVFP4        uint8 E4M3 [rows][cols/16]
+ *      INT4_G32/64  fp32       [rows][cols/g]
+ *      INT8_ROW     fp32       [rows]
+ *      FP8_TENSOR   none (the tensor scale only)
+ *  MMA: the operand layout the qlinear kernels read.
+ *      E8M0/E4M3 scales (MXFP8, MXFP4, NVFP4): rows padded to a multiple of
+ *        128 (R'), scale columns padded to a multiple of 16 (S'); byte of
+ *        (row r, scale column s) at
+ *          ((r/128)*(S'/4) + s/4)*512 + (r%32)*16 + ((r%128)/32)*4 + s%4;
+ *        padding bytes are written as 0.
+ *      INT4_G32/64: codes one signed byte per element [rows][cols]; scales
+ *        fp32 transposed [cols/g][rows].
+ *      INT8_ROW, FP8_TENSOR: identical to CANONICAL.
+ */
+typedef enum mxq_layout { MXQ_LAYOUT_CANONICAL = 0, MXQ_LAYOUT_MMA = 1 } mxq_layout;
+
+/* A quantized matrix (descriptor only; all pointers are device memory). */
+typedef struct mxq_qtensor {
+    int32_t fmt;               /* mxq_fmt                                    */
+    int32_t layout;            /* mxq_layout of codes and scales             */
+    int64_t rows, cols;        /* logical shape (cols = K)                   */
+    const void *codes;         /* device                                     */
+    const void *scales;        /* device; NULL for FP8_TENSOR                */
+    const float *tensor_scale; /* device fp32 scalar for NVFP4 / FP8_TENSOR  */
+} mxq_qtensor;
+
+/* Human-readable name of a status code (static string). */
+const char *mxq_status_string(mxq_status st);
+
+/* 1 if device `device` is an sm_100-family GPU the kernels were built for. */
+int mxq_device_supported(int device);
+
+/* Synchronizes `stream`, then reads and clears the device error word.
+ * Returns MXQ_ETIMEOUT if a bounded wait ran out since the last check,
+ * MXQ_ECUDA if a CUDA error is pending, else MXQ_OK.  Host-blocking. */
+mxq_status mxq_check(void *stream);
+
+/* ---------------------------------------------------------------------- */
+/* Sizes (host only).                                                      */
+/* ---------------------------------------------------------------------- */
+
+/* Bytes of the codes / scales buffers mxq_quantize writes for a rows x cols
+ * input in format `fmt` and `layout`.  MXQ_EINVAL for bad arguments. */
+mxq_status mxq_codes_bytes(int32_t fmt, int64_t rows, int64_t cols, int32_t layout, size_t *bytes);
+mxq_status mxq_scales_bytes(int32_t fmt, int64_t rows, int64_t cols, int32_t layout, size_t *bytes);
+
+/* Scratch bytes mxq_quantize needs (tensor-amax word for NVFP4 and
+ * FP8_TENSOR; 0 otherwise). */
+mxq_status mxq_quantize_workspace_bytes(int32_t fmt, size_t *bytes);
+
+/* ---------------------------------------------------------------------- */
+/* a1-a3: tensor amax, optional Hadamard, block-scaled quantization.       */
+/* ---------------------------------------------------------------------- */
+
+/* Quantize x (rows x cols, fp32 or bf16, device) into `fmt`.
+ * Source: Chameleon article (MXFP8 blocks sharing an exponent; dynamic
+ * scales kept for PixArt), Nunchaku/Diffusers article (INT4 / NVFP4
+ * svdq_w4a4 variants), "Bridging the Gap ..." (NVFP4 groups, MXFP4
+ * power-of-two scales, item 3 Hadamard rotation).  Encodings: OCP MX v1.0,
+ * NVFP4.  Per block: amax, scale, round-to-nearest-even codes (saturating);
+ * NVFP4 and FP8_TENSOR first reduce the tensor amax.
+ *   hadamard_b: 0 (off) or a power of two in [2, 256] dividing cols; the
+ *     rows are rotated by the orthonormal block-diagonal Sylvester Hadamard
+ *     matrix (fp32 butterflies, then one multiply by RN(1/sqrt(b))) before
+ *     quantization.
+ *   codes, scales: device, sizes from mxq_codes_bytes / mxq_scales_bytes
+ *     (scales may be NULL for FP8_TENSOR).
+ *   tensor_scale: device fp32 written for NVFP4 / FP8_TENSOR, else ignored
+ *     (may be NULL).
+ *   workspace: device scratch of mxq_quantize_workspace_bytes (may be NULL
+ *     when that is 0); clobbered.
+ * Constraints: cols % 16 == 0 and cols % block == 0; rows >= 0.
+ * Errors: MXQ_EINVAL (shape / pointer / hadamard_b), MXQ_ENOSPACE,
+ * MXQ_ECUDA (launch failure). */
+mxq_status mxq_quantize(const void *x, int32_t xdtype, int64_t rows, int64_t cols, int32_t fmt,
+                        int32_t hadamard_b, int32_t layout, void *codes, void *scales,
+                        float *tensor_scale, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Dequantize q into y (rows x cols, fp32 or bf16, device).  Each output is
+ * the code value times its scale(s) computed in fp32 (NVFP4: the exact
+ * E2M1 x E4M3 product, then times the tensor scale), rounded to bf16 (RNE)
+ * for bf16 output.  Both layouts are accepted.  MXQ_EINVAL on bad args. */
+mxq_status mxq_dequantize(const mxq_qtensor *q, void *y, int32_t ydtype, void *stream);
+
+/* Block-diagonal Hadamard rotation y = x . blockdiag(H_b)/sqrt(b) along
+ * the rows ("Bridging the Gap ...", item 3).  x, y: rows x cols device
+ * arrays of dtype `dtype` (y may alias x).  bf16 output is the fp32 result
+ * rounded once (RNE).  b: power of two in [2, 256], cols % b == 0 and
+ * cols % 16 == 0. */
+mxq_status mxq_hadamard_block(const void *x, void *y, int32_t dtype, int64_t rows, int64_t cols,
+                              int32_t b, void *stream);
+
+/* Element conversion used by the codec tests: out[i] = E4M3 byte (elem 0)
+ * or E2M1 code in the low nibble (elem 1) of the fp32 x[i], round to
+ * nearest even, saturating.  x, out: device, n elements. */
+mxq_status mxq_cast(const float *x, int64_t n, int32_t elem, uint8_t *out, void *stream);
+
+/* ---------------------------------------------------------------------- */
+/* a4: per-output-channel weight-format selection.                         */
+/* ---------------------------------------------------------------------- */
+
+/* Scratch bytes mxq_select_weight_format needs. */
+mxq_status mxq_select_workspace_bytes(const int32_t *candidates, int32_t ncand, size_t *bytes);
+
+/* Chameleon article, section "the format is chosen by the value
+ * distribution": each output channel (row of w, n x k, fp32/bf16, device)
+ * is quantized under every candidate format (host array of ncand <= 8
+ * mxq_fmt values, no Hadamard); its reconstruction error is the binary64
+ * sum of squared differences from the exact dequantized values; the
+ * channel keeps the candidate with the least error (ties to the lower
+ * candidate index).  Tensor-scaled candidates use the tensor scale of the
+ * whole w.
+ *   fmt_per_channel: device uint8[n], the chosen mxq_fmt.
+ *   sse: device double[n][ncand] or NULL.
+ *   workspace: device scratch of mxq_select_workspace_bytes.
+ * Constraints: k % 64 == 0. */
+mxq_status mxq_select_weight_format(const void *w, int32_t wdtype, int64_t n, int64_t k,
+                                    const int32_t *candidates, int32_t ncand,
+                                    uint8_t *fmt_per_channel, double *sse, void *workspace,
+                                    size_t workspace_bytes, void *stream);
+
+/* ---------------------------------------------------------------------- */
+/* a5-a7: low-rank branch and block-scaled low-bit GEMM.                   */
+/* ---------------------------------------------------------------------- */
+
+/* SVDQuant low-rank down projection (Nunchaku/Diffusers article, "Main
+ * explanation": a 16-bit low-rank part of the weight beside the 4-bit
+ * residual): t = bf16(x) . l1 with fp32 accumulation.
+ *   x: m x k fp32/bf16 device; l1: k x r bf16 device; t: m x r fp32 device.
+ * Constraints: 1 <= r <= 32, k % 16 == 0. */
+mxq_status mxq_lowrank_down(const void *x, int32_t xdtype, int64_t m, int64_t k, const void *l1,
+                            int32_t r, float *t, void *stream);
+
+/* Re-lays the up-projection l2 (r x n bf16, device) as the GEMM operand
+ * l2p (n x 64 bf16, device): row j of l2p holds l2[0..r-1][j], zeros up to
+ * 32, then the same 32 values again (the operand of the split high/low
+ * low-rank product).  Done once per weight. */
+mxq_status mxq_lowrank_pack_l2(const void *l2, int32_t r, int64_t n, void *l2p, void *stream);
+
+/* Scratch bytes mxq_qlinear needs for m rows (the packed low-rank
+ * activation: m x 64 bf16). */
+mxq_status mxq_qlinear_workspace_bytes(int64_t m, size_t *bytes);
+
+/* Block-scaled low-bit GEMM with fused dequantization epilogue and
+ * low-rank branch (Nunchaku/Diffusers article, svdq_w4a4; Chameleon
+ * article, W8A8 formats):
+ *   y[m][n] = sum_k deq(xq)[m][k] * deq(wq)[n][k]  (+ sum_j t[m][j] * l2[j][n])
+ * on tcgen05 tensor cores (fp32 accumulation; int32 for INT8_ROW).
+ *   xq, wq: same fmt, MMA layout, xq->cols == wq->cols == K.
+ *     Supported fmt: NVFP4, MXFP4, MXFP8, FP8_TENSOR, INT8_ROW.
+ *   t: m x r fp32 device (from mxq_lowrank_down) or NULL for no branch;
+ *   l2p: packed up-projection from mxq_lowrank_pack_l2 (n rows); r as there.
+ *     The branch is supported for NVFP4, MXFP4, MXFP8 and FP8_TENSOR.
+ *   y: m x n device, fp32 or bf16 (fp32 result rounded once, RNE).
+ *   workspace: device scratch of mxq_qlinear_workspace_bytes(m) when t is
+ *     given (may be NULL otherwise); clobbered.
+ * Constraints: K % 64 == 0 (4-bit) or K % 32 == 0 (8-bit); K > 0.
+ * Errors: MXQ_EINVAL, MXQ_EUNSUPPORTED (format pair / branch), MXQ_ENOSPACE,
+ * MXQ_ECUDA.  A pipeline wait that runs out is reported by mxq_check(). */
+mxq_status mxq_qlinear(const mxq_qtensor *xq, const mxq_qtensor *wq, const float *t,
+                       const void *l2p, int32_t r, void *y, int32_t ydtype, void *workspace,
+                       size_t workspace_bytes, void *stream);
+
+/* ---------------------------------------------------------------------- */
+/* a8: per-layer, per-timestep-interval format table.                      */
+/* ---------------------------------------------------------------------- */
+
+/* Chameleon article: the denoising trajectory is cut into intervals and a
+ * layer reads its activation format for the current interval from a table
+ * at generation time.  table: host uint8[n_layers][n_intervals] of mxq_fmt;
+ * interval = floor(step * n_intervals / n_steps).  Returns the format, or
+ * -1 for out-of-range arguments.  Host only, no CUDA call. */
+int32_t mxq_route(const uint8_t *table, int32_t n_layers, int32_t n_intervals, int32_t layer,
+                  int32_t step, int32_t n_steps);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXQ_H */

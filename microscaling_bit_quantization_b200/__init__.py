@@ -1,0 +1,273 @@
+"""Python binding of libmxq, the B200 (sm_100a) microscaling quantized-linear
+library.  Argument marshalling only: every step runs in the library's CUDA
+kernels.  torch provides device memory and the current stream.
+
+The C ABI is declared in ``include/mxq.h``; functions here carry the same
+names.  Importing this module loads ``libmxq.so`` from the package directory
+and raises ImportError if it has not been built (``python -m
+microscaling_bit_quantization_b200.build`` or ``__graft_entry__.build()``).
+There is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmxq.so")
+
+MXFP8, MXFP4, NVFP4, INT4_G32, INT4_G64, INT8_ROW, FP8_TENSOR = range(7)
+FORMATS = {"MXFP8": MXFP8, "MXFP4": MXFP4, "NVFP4": NVFP4, "INT4_G32": INT4_G32, "INT4_G64": INT4_G64,
+           "INT8_ROW": INT8_ROW, "FP8_TENSOR": FP8_TENSOR}
+FORMAT_NAMES = {v: k for k, v in FORMATS.items()}
+CANONICAL, MMA = 0, 1
+F32, BF16 = 0, 1
+STATUS = {0: "MXQ_OK", 1: "MXQ_EINVAL", 2: "MXQ_EUNSUPPORTED", 3: "MXQ_ECUDA", 4: "MXQ_ETIMEOUT", 5: "MXQ_ENOSPACE"}
+
+# Every entry point the header declares.
+EXPORTS = ("mxq_status_string", "mxq_device_supported", "mxq_check", "mxq_codes_bytes", "mxq_scales_bytes",
+           "mxq_quantize_workspace_bytes", "mxq_quantize", "mxq_dequantize", "mxq_hadamard_block", "mxq_cast",
+           "mxq_select_workspace_bytes", "mxq_select_weight_format", "mxq_lowrank_down", "mxq_lowrank_pack_l2",
+           "mxq_qlinear_workspace_bytes", "mxq_qlinear", "mxq_route")
+
+
+class MxqError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__("%s failed: %s (%s)" % (what, STATUS.get(status, status), _lib.mxq_status_string(status).decode()))
+        self.status = status
+
+
+class _QTensorC(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("layout", ctypes.c_int32), ("rows", ctypes.c_int64),
+                ("cols", ctypes.c_int64), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("tensor_scale", ctypes.c_void_p)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libmxq.so is not built at %s; run __graft_entry__.build()" % LIB_PATH)
+    L = ctypes.CDLL(LIB_PATH)
+    P, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    psz = ctypes.POINTER(ctypes.c_size_t)
+    sig = {
+        "mxq_status_string": (ctypes.c_char_p, [i32]),
+        "mxq_device_supported": (ctypes.c_int, [ctypes.c_int]),
+        "mxq_check": (i32, [P]),
+        "mxq_codes_bytes": (i32, [i32, i64, i64, i32, psz]),
+        "mxq_scales_bytes": (i32, [i32, i64, i64, i32, psz]),
+        "mxq_quantize_workspace_bytes": (i32, [i32, psz]),
+        "mxq_quantize": (i32, [P, i32, i64, i64, i32, i32, i32, P, P, P, P, sz, P]),
+        "mxq_dequantize": (i32, [ctypes.POINTER(_QTensorC), P, i32, P]),
+        "mxq_hadamard_block": (i32, [P, P, i32, i64, i64, i32, P]),
+        "mxq_cast": (i32, [P, i64, i32, P, P]),
+        "mxq_select_workspace_bytes": (i32, [P, i32, psz]),
+        "mxq_select_weight_format": (i32, [P, i32, i64, i64, P, i32, P, P, P, sz, P]),
+        "mxq_lowrank_down": (i32, [P, i32, i64, i64, P, i32, P, P]),
+        "mxq_lowrank_pack_l2": (i32, [P, i32, i64, P, P]),
+        "mxq_qlinear_workspace_bytes": (i32, [i64, psz]),
+        "mxq_qlinear": (i32, [ctypes.POINTER(_QTensorC), ctypes.POINTER(_QTensorC), P, P, i32, P, i32, P, sz, P]),
+        "mxq_route": (i32, [P, i32, i32, i32, i32, i32]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype, f.argtypes = res, args
+    return L
+
+
+_lib = _load()
+
+
+def lib():
+    return _lib
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None and t.numel() > 0 else None
+
+
+def _ok(st: int, what: str):
+    if st != 0:
+        raise MxqError(st, what)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError("expected float32 or bfloat16, got %s" % t.dtype)
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("tensors must be on a CUDA device (there is no CPU path)")
+
+
+def _size(fn, *args) -> int:
+    out = ctypes.c_size_t(0)
+    _ok(fn(*args, ctypes.byref(out)), fn.__name__)
+    return out.value
+
+
+@dataclass
+class QTensor:
+    """A quantized matrix: device tensors for codes, scales, tensor scale."""
+    fmt: int
+    layout: int
+    rows: int
+    cols: int
+    codes: torch.Tensor
+    scales: Optional[torch.Tensor]
+    tensor_scale: Optional[torch.Tensor]
+
+    def c(self) -> _QTensorC:
+        return _QTensorC(self.fmt, self.layout, self.rows, self.cols, _ptr(self.codes), _ptr(self.scales),
+                         _ptr(self.tensor_scale))
+
+
+def codes_bytes(fmt, rows, cols, layout=CANONICAL) -> int:
+    return _size(_lib.mxq_codes_bytes, fmt, rows, cols, layout)
+
+
+def scales_bytes(fmt, rows, cols, layout=CANONICAL) -> int:
+    return _size(_lib.mxq_scales_bytes, fmt, rows, cols, layout)
+
+
+def alloc_qtensor(fmt, rows, cols, layout=CANONICAL, device="cuda") -> QTensor:
+    cb = codes_bytes(fmt, rows, cols, layout)
+    sb = scales_bytes(fmt, rows, cols, layout)
+    codes = torch.empty(cb, dtype=torch.uint8, device=device)
+    scales = torch.empty(max(sb, 1), dtype=torch.uint8, device=device) if sb else None
+    ts = torch.empty(1, dtype=torch.float32, device=device) if fmt in (NVFP4, FP8_TENSOR) else None
+    return QTensor(fmt, layout, rows, cols, codes, scales, ts)
+
+
+def quantize_workspace_bytes(fmt) -> int:
+    return _size(_lib.mxq_quantize_workspace_bytes, fmt)
+
+
+def quantize(x: torch.Tensor, fmt: int, hadamard_b: int = 0, layout: int = CANONICAL, out: QTensor = None,
+             workspace: torch.Tensor = None, stream=None) -> QTensor:
+    """Block-scaled quantization of a 2-D CUDA tensor (fp32 or bf16)."""
+    _require_cuda(x)
+    x = x.contiguous()
+    rows, cols = x.shape
+    q = out if out is not None else alloc_qtensor(fmt, rows, cols, layout, x.device)
+    wsb = quantize_workspace_bytes(fmt)
+    if wsb and workspace is None:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=x.device)
+    _ok(_lib.mxq_quantize(_ptr(x), _dtype_code(x), rows, cols, fmt, hadamard_b, layout, _ptr(q.codes),
+                          _ptr(q.scales), _ptr(q.tensor_scale), _ptr(workspace), wsb, _stream(stream)),
+        "mxq_quantize")
+    return q
+
+
+def dequantize(q: QTensor, dtype=torch.float32, stream=None) -> torch.Tensor:
+    y = torch.empty((q.rows, q.cols), dtype=dtype, device=q.codes.device)
+    qc = q.c()
+    _ok(_lib.mxq_dequantize(ctypes.byref(qc), _ptr(y), _dtype_code(y), _stream(stream)), "mxq_dequantize")
+    return y
+
+
+def hadamard_block(x: torch.Tensor, b: int, out: torch.Tensor = None, stream=None) -> torch.Tensor:
+    _require_cuda(x)
+    x = x.contiguous()
+    y = out if out is not None else torch.empty_like(x)
+    rows, cols = x.shape
+    _ok(_lib.mxq_hadamard_block(_ptr(x), _ptr(y), _dtype_code(x), rows, cols, b, _stream(stream)),
+        "mxq_hadamard_block")
+    return y
+
+
+def cast(x: torch.Tensor, elem: str, out: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """Element conversion of fp32 values: 'e4m3' byte or 'e2m1' nibble per element."""
+    _require_cuda(x)
+    assert x.dtype == torch.float32 and x.is_contiguous()
+    y = out if out is not None else torch.empty(x.numel(), dtype=torch.uint8, device=x.device)
+    _ok(_lib.mxq_cast(_ptr(x), x.numel(), 0 if elem == "e4m3" else 1, _ptr(y), _stream(stream)), "mxq_cast")
+    return y
+
+
+def select_weight_format(w: torch.Tensor, candidates: Sequence[int], want_sse: bool = True, stream=None):
+    """Per-output-channel format choice; returns (uint8 formats, float64 errors or None)."""
+    _require_cuda(w)
+    w = w.contiguous()
+    n, k = w.shape
+    cands = (ctypes.c_int32 * len(candidates))(*candidates)
+    wsb = _size(_lib.mxq_select_workspace_bytes, cands, len(candidates))
+    ws = torch.empty(wsb, dtype=torch.uint8, device=w.device)
+    choice = torch.empty(n, dtype=torch.uint8, device=w.device)
+    sse = torch.empty((n, len(candidates)), dtype=torch.float64, device=w.device) if want_sse else None
+    _ok(_lib.mxq_select_weight_format(_ptr(w), _dtype_code(w), n, k, cands, len(candidates), _ptr(choice),
+                                      _ptr(sse), _ptr(ws), wsb, _stream(stream)), "mxq_select_weight_format")
+    return choice, sse
+
+
+def lowrank_down(x: torch.Tensor, l1: torch.Tensor, out: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """t = bf16(x) . l1 in fp32 (l1: k x r bf16)."""
+    _require_cuda(x, l1)
+    x, l1 = x.contiguous(), l1.contiguous()
+    assert l1.dtype == torch.bfloat16
+    m, k = x.shape
+    r = l1.shape[1]
+    t = out if out is not None else torch.empty((m, r), dtype=torch.float32, device=x.device)
+    _ok(_lib.mxq_lowrank_down(_ptr(x), _dtype_code(x), m, k, _ptr(l1), r, _ptr(t), _stream(stream)),
+        "mxq_lowrank_down")
+    return t
+
+
+def lowrank_pack_l2(l2: torch.Tensor, stream=None) -> torch.Tensor:
+    """Packs the up-projection (r x n bf16) as the GEMM operand (n x 64 bf16)."""
+    _require_cuda(l2)
+    l2 = l2.contiguous()
+    assert l2.dtype == torch.bfloat16
+    r, n = l2.shape
+    l2p = torch.empty((n, 64), dtype=torch.bfloat16, device=l2.device)
+    _ok(_lib.mxq_lowrank_pack_l2(_ptr(l2), r, n, _ptr(l2p), _stream(stream)), "mxq_lowrank_pack_l2")
+    return l2p
+
+
+def qlinear_workspace_bytes(m: int) -> int:
+    return _size(_lib.mxq_qlinear_workspace_bytes, m)
+
+
+def qlinear(xq: QTensor, wq: QTensor, t: torch.Tensor = None, l2p: torch.Tensor = None, r: int = 0,
+            out_dtype=torch.bfloat16, out: torch.Tensor = None, workspace: torch.Tensor = None,
+            stream=None) -> torch.Tensor:
+    """y = deq(xq) . deq(wq)^T (+ t . l2) on tcgen05 tensor cores."""
+    m, n = xq.rows, wq.rows
+    y = out if out is not None else torch.empty((m, n), dtype=out_dtype, device=xq.codes.device)
+    wsb = 0
+    if t is not None:
+        wsb = qlinear_workspace_bytes(m)
+        if workspace is None:
+            workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=y.device)
+        t = t.contiguous()
+    xc, wc = xq.c(), wq.c()
+    _ok(_lib.mxq_qlinear(ctypes.byref(xc), ctypes.byref(wc), _ptr(t), _ptr(l2p), r, _ptr(y), _dtype_code(y),
+                         _ptr(workspace), wsb, _stream(stream)), "mxq_qlinear")
+    return y
+
+
+def route(table, layer: int, step: int, n_steps: int) -> int:
+    """Format id of `layer` at denoising `step` from a host uint8 table [layers][intervals]."""
+    import numpy as np
+    tab = np.ascontiguousarray(np.asarray(table, dtype=np.uint8))
+    n_layers, n_int = tab.shape
+    return _lib.mxq_route(tab.ctypes.data_as(ctypes.c_void_p), n_layers, n_int, layer, step, n_steps)
+
+
+def check(stream=None) -> int:
+    """Synchronizes and returns the status of bounded device waits (0 = ok)."""
+    return _lib.mxq_check(_stream(stream))

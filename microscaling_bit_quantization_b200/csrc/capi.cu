@@ -1,0 +1,245 @@
+// capi.cu -- the extern "C" boundary declared in include/mxq.h: argument
+// validation (all on the host, before any launch), buffer-size queries,
+// format routing, and dispatch to the kernel launchers.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/mxq.h"
+#include "mxq_formats.cuh"
+#include "mxq_internal.h"
+
+using namespace mxq;
+
+namespace {
+
+bool valid_fmt(int32_t f) { return f >= 0 && f < MXQ_NUM_FMT; }
+bool valid_dtype(int32_t d) { return d == MXQ_F32 || d == MXQ_BF16; }
+bool valid_layout(int32_t l) { return l == MXQ_LAYOUT_CANONICAL || l == MXQ_LAYOUT_MMA; }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_hadamard(int32_t b, int64_t cols) {
+    if (b == 0) return true;
+    return b >= 2 && b <= 256 && (b & (b - 1)) == 0 && cols % b == 0;
+}
+
+// Shape rule shared by the quantizers: 16-element chunks and whole blocks.
+bool valid_shape(int32_t fmt, int64_t rows, int64_t cols) {
+    if (rows < 0 || cols < 0 || cols % 16) return false;
+    int blk = fmt_block(fmt);
+    if (blk && cols % blk) return false;
+    if (rows > (int64_t)1 << 31 || cols > (int64_t)1 << 31) return false;
+    return true;
+}
+
+mxq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MXQ_OK : MXQ_ECUDA; }
+
+int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+
+}  // namespace
+
+extern "C" {
+
+const char *mxq_status_string(mxq_status st) {
+    switch (st) {
+    case MXQ_OK: return "ok";
+    case MXQ_EINVAL: return "invalid argument";
+    case MXQ_EUNSUPPORTED: return "unsupported format, combination or device";
+    case MXQ_ECUDA: return "CUDA error";
+    case MXQ_ETIMEOUT: return "a bounded device wait ran out";
+    case MXQ_ENOSPACE: return "workspace too small";
+    }
+    return "unknown status";
+}
+
+int mxq_device_supported(int device) {
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device) != cudaSuccess) return 0;
+    return major == 10;
+}
+
+mxq_status mxq_check(void *stream) {
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return MXQ_ECUDA;
+    unsigned int w = 0;
+    if (read_and_clear_error(&w) != cudaSuccess) return MXQ_ECUDA;
+    return w ? MXQ_ETIMEOUT : MXQ_OK;
+}
+
+mxq_status mxq_codes_bytes(int32_t fmt, int64_t rows, int64_t cols, int32_t layout, size_t *bytes) {
+    if (!valid_fmt(fmt) || !valid_layout(layout) || !bytes || !valid_shape(fmt, rows, cols)) return MXQ_EINVAL;
+    const bool int4_unpacked = (fmt == MXQ_INT4_G32 || fmt == MXQ_INT4_G64) && layout == MXQ_LAYOUT_MMA;
+    *bytes = (size_t)(rows * cols / ((fmt_is4(fmt) && !int4_unpacked) ? 2 : 1));
+    return MXQ_OK;
+}
+
+mxq_status mxq_scales_bytes(int32_t fmt, int64_t rows, int64_t cols, int32_t layout, size_t *bytes) {
+    if (!valid_fmt(fmt) || !valid_layout(layout) || !bytes || !valid_shape(fmt, rows, cols)) return MXQ_EINVAL;
+    switch (fmt) {
+    case MXQ_MXFP8:
+    case MXQ_MXFP4:
+    case MXQ_NVFP4: {
+        int64_t S = cols / fmt_block(fmt);
+        *bytes = layout == MXQ_LAYOUT_CANONICAL ? (size_t)(rows * S) : (size_t)(round_up(rows, 128) * round_up(S, 16));
+        break;
+    }
+    case MXQ_INT4_G32:
+    case MXQ_INT4_G64: *bytes = (size_t)(rows * (cols / fmt_block(fmt)) * 4); break;
+    case MXQ_INT8_ROW: *bytes = (size_t)(rows * 4); break;
+    default: *bytes = 0;
+    }
+    return MXQ_OK;
+}
+
+mxq_status mxq_quantize_workspace_bytes(int32_t fmt, size_t *bytes) {
+    if (!valid_fmt(fmt) || !bytes) return MXQ_EINVAL;
+    *bytes = fmt_tensor_scaled(fmt) ? 16 : 0;
+    return MXQ_OK;
+}
+
+mxq_status mxq_quantize(const void *x, int32_t xdtype, int64_t rows, int64_t cols, int32_t fmt, int32_t hadamard_b,
+                        int32_t layout, void *codes, void *scales, float *tensor_scale, void *workspace,
+                        size_t workspace_bytes, void *stream) {
+    if (!valid_fmt(fmt) || !valid_dtype(xdtype) || !valid_layout(layout) || !valid_shape(fmt, rows, cols) ||
+        !valid_hadamard(hadamard_b, cols))
+        return MXQ_EINVAL;
+    const int64_t n = rows * cols;
+    if (n > 0 && (!x || !codes || !aligned16(x) || !aligned16(codes))) return MXQ_EINVAL;
+    if (n > 0 && fmt != MXQ_FP8_TENSOR && !scales) return MXQ_EINVAL;
+    if (fmt_tensor_scaled(fmt) && !tensor_scale) return MXQ_EINVAL;
+    size_t ws = 0, sb = 0;
+    mxq_quantize_workspace_bytes(fmt, &ws);
+    if (ws && (!workspace || workspace_bytes < ws)) return workspace ? MXQ_ENOSPACE : MXQ_EINVAL;
+    mxq_scales_bytes(fmt, rows, cols, layout, &sb);
+    return from_cuda(launch_quantize(x, xdtype == MXQ_BF16, rows, cols, fmt, hadamard_b, layout, codes, scales, sb,
+                                     tensor_scale, (unsigned int *)workspace, (cudaStream_t)stream));
+}
+
+mxq_status mxq_dequantize(const mxq_qtensor *q, void *y, int32_t ydtype, void *stream) {
+    if (!q || !valid_fmt(q->fmt) || !valid_layout(q->layout) || !valid_dtype(ydtype) ||
+        !valid_shape(q->fmt, q->rows, q->cols))
+        return MXQ_EINVAL;
+    if (q->rows * q->cols > 0) {
+        if (!q->codes || !y || !aligned16(q->codes) || !aligned16(y)) return MXQ_EINVAL;
+        if (q->fmt != MXQ_FP8_TENSOR && !q->scales) return MXQ_EINVAL;
+        if (fmt_tensor_scaled(q->fmt) && !q->tensor_scale) return MXQ_EINVAL;
+    }
+    return from_cuda(launch_dequantize(q->fmt, q->layout, q->rows, q->cols, q->codes, q->scales, q->tensor_scale, y,
+                                       ydtype == MXQ_BF16, (cudaStream_t)stream));
+}
+
+mxq_status mxq_hadamard_block(const void *x, void *y, int32_t dtype, int64_t rows, int64_t cols, int32_t b,
+                              void *stream) {
+    if (!valid_dtype(dtype) || rows < 0 || cols < 0 || cols % 16 || b == 0 || !valid_hadamard(b, cols))
+        return MXQ_EINVAL;
+    if (rows * cols > 0 && (!x || !y || !aligned16(x) || !aligned16(y))) return MXQ_EINVAL;
+    return from_cuda(launch_hadamard(x, y, dtype == MXQ_BF16, rows, cols, b, (cudaStream_t)stream));
+}
+
+mxq_status mxq_cast(const float *x, int64_t n, int32_t elem, uint8_t *out, void *stream) {
+    if (n < 0 || (elem != 0 && elem != 1)) return MXQ_EINVAL;
+    if (n > 0 && (!x || !out)) return MXQ_EINVAL;
+    return from_cuda(launch_cast(x, n, elem, out, (cudaStream_t)stream));
+}
+
+mxq_status mxq_select_workspace_bytes(const int32_t *candidates, int32_t ncand, size_t *bytes) {
+    if (!candidates || ncand < 1 || ncand > kMaxCandidates || !bytes) return MXQ_EINVAL;
+    *bytes = 16;
+    return MXQ_OK;
+}
+
+mxq_status mxq_select_weight_format(const void *w, int32_t wdtype, int64_t n, int64_t k, const int32_t *candidates,
+                                    int32_t ncand, uint8_t *fmt_per_channel, double *sse, void *workspace,
+                                    size_t workspace_bytes, void *stream) {
+    if (!valid_dtype(wdtype) || !candidates || ncand < 1 || ncand > kMaxCandidates || n < 0 || k < 0 || k % 16)
+        return MXQ_EINVAL;
+    int cands[kMaxCandidates];
+    for (int j = 0; j < ncand; j++) {
+        if (!valid_fmt(candidates[j]) || !valid_shape(candidates[j], n, k)) return MXQ_EINVAL;
+        cands[j] = candidates[j];
+    }
+    if (n > 0 && (!w || !fmt_per_channel || !aligned16(w))) return MXQ_EINVAL;
+    if (!workspace) return MXQ_EINVAL;
+    if (workspace_bytes < 16) return MXQ_ENOSPACE;
+    return from_cuda(launch_select(w, wdtype == MXQ_BF16, n, k, cands, ncand, fmt_per_channel, sse,
+                                   (unsigned int *)workspace, (cudaStream_t)stream));
+}
+
+mxq_status mxq_lowrank_down(const void *x, int32_t xdtype, int64_t m, int64_t k, const void *l1, int32_t r, float *t,
+                            void *stream) {
+    if (!valid_dtype(xdtype) || m < 0 || k <= 0 || k % 16 || r < 1 || r > 32) return MXQ_EINVAL;
+    if (m > 0 && (!x || !l1 || !t || !aligned16(x))) return MXQ_EINVAL;
+    return from_cuda(launch_lowrank_down(x, xdtype == MXQ_BF16, m, k, l1, r, t, (cudaStream_t)stream));
+}
+
+mxq_status mxq_lowrank_pack_l2(const void *l2, int32_t r, int64_t n, void *l2p, void *stream) {
+    if (r < 1 || r > 32 || n < 0) return MXQ_EINVAL;
+    if (n > 0 && (!l2 || !l2p || !aligned16(l2p))) return MXQ_EINVAL;
+    return from_cuda(launch_pack_l2(l2, r, n, l2p, (cudaStream_t)stream));
+}
+
+mxq_status mxq_qlinear_workspace_bytes(int64_t m, size_t *bytes) {
+    if (m < 0 || !bytes) return MXQ_EINVAL;
+    *bytes = (size_t)(m * 64 * 2);
+    return MXQ_OK;
+}
+
+mxq_status mxq_qlinear(const mxq_qtensor *xq, const mxq_qtensor *wq, const float *t, const void *l2p, int32_t r,
+                       void *y, int32_t ydtype, void *workspace, size_t workspace_bytes, void *stream) {
+    if (!xq || !wq || !valid_dtype(ydtype) || !y) return MXQ_EINVAL;
+    if (!valid_fmt(xq->fmt) || xq->fmt != wq->fmt) return MXQ_EUNSUPPORTED;
+    const int fmt = xq->fmt;
+    if (fmt == MXQ_INT4_G32 || fmt == MXQ_INT4_G64) return MXQ_EUNSUPPORTED;
+    if (xq->layout != MXQ_LAYOUT_MMA || wq->layout != MXQ_LAYOUT_MMA) return MXQ_EINVAL;
+    const int64_t m = xq->rows, n = wq->rows, k = xq->cols;
+    if (wq->cols != k || k <= 0 || m < 0 || n < 0) return MXQ_EINVAL;
+    if (k % (fmt_is4(fmt) ? 64 : 32)) return MXQ_EINVAL;
+    if (!valid_shape(fmt, m, k) || !valid_shape(fmt, n, k)) return MXQ_EINVAL;
+    if (m > 0 && n > 0) {
+        if (!xq->codes || !wq->codes || !aligned16(xq->codes) || !aligned16(wq->codes) || !aligned16(y))
+            return MXQ_EINVAL;
+        if (fmt != MXQ_FP8_TENSOR && (!xq->scales || !wq->scales)) return MXQ_EINVAL;
+        if (fmt_tensor_scaled(fmt) && (!xq->tensor_scale || !wq->tensor_scale)) return MXQ_EINVAL;
+    }
+    if (t) {
+        if (fmt == MXQ_INT8_ROW) return MXQ_EUNSUPPORTED;
+        if (r < 1 || r > 32 || !l2p || !aligned16(l2p)) return MXQ_EINVAL;
+        size_t need = 0;
+        mxq_qlinear_workspace_bytes(m, &need);
+        if (!workspace) return MXQ_EINVAL;
+        if (workspace_bytes < need) return MXQ_ENOSPACE;
+        if (!aligned16(workspace)) return MXQ_EINVAL;
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    if (t) {
+        const bool ts = fmt_tensor_scaled(fmt);
+        cudaError_t e = launch_pack_t(t, r, m, ts ? xq->tensor_scale : nullptr, ts ? wq->tensor_scale : nullptr,
+                                      workspace, s);
+        if (e != cudaSuccess) return MXQ_ECUDA;
+    }
+    GemmOperands op;
+    op.fmt = fmt;
+    op.m = m;
+    op.n = n;
+    op.k = k;
+    op.a_codes = xq->codes;
+    op.b_codes = wq->codes;
+    op.a_scales = xq->scales;
+    op.b_scales = wq->scales;
+    op.a_tensor_scale = xq->tensor_scale;
+    op.b_tensor_scale = wq->tensor_scale;
+    op.tp = t ? workspace : nullptr;
+    op.l2p = l2p;
+    op.y = y;
+    op.y_bf16 = ydtype == MXQ_BF16;
+    return from_cuda(launch_qlinear(op, s));
+}
+
+int32_t mxq_route(const uint8_t *table, int32_t n_layers, int32_t n_intervals, int32_t layer, int32_t step,
+                  int32_t n_steps) {
+    if (!table || n_layers <= 0 || n_intervals <= 0 || n_steps <= 0) return -1;
+    if (layer < 0 || layer >= n_layers || step < 0 || step >= n_steps) return -1;
+    const int64_t interval = (int64_t)step * n_intervals / n_steps;
+    return table[(int64_t)layer * n_intervals + interval];
+}
+
+}  // extern "C"

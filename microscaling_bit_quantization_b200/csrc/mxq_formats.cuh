@@ -1,0 +1,230 @@
+// mxq_formats.cuh -- device-side element codecs and per-block scale rules.
+//
+// Encodings follow the OCP Microscaling (MX) v1.0 definition (E2M1, E4M3
+// "fn", E8M0, 32-element blocks) and NVIDIA's NVFP4 definition (E2M1 in
+// 16-element blocks with an E4M3 block scale and an fp32 tensor scale); the
+// pages name these formats (Chameleon article: MXFP8 blocks sharing an
+// exponent; Nunchaku/Diffusers article: INT4 and NVFP4 svdq_w4a4 variants;
+// "Bridging the Gap ... Microscaling FP4 Quantization": NVFP4 groups, MXFP4
+// power-of-two scales) but do not define them.
+//
+// Encoding uses the hardware conversions (cvt.rn.satfinite.{e4m3x2,e2m1x2})
+// through the CUDA intrinsics; every fp32 division or multiply that feeds a
+// code uses the IEEE round-to-nearest intrinsics so no contraction or
+// approximate division can change a code.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp4.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+namespace mxq {
+
+enum Fmt : int {
+    kMXFP8 = 0, kMXFP4 = 1, kNVFP4 = 2, kINT4G32 = 3, kINT4G64 = 4, kINT8Row = 5, kFP8Tensor = 6,
+    kNumFmt = 7
+};
+
+__host__ __device__ constexpr int fmt_block(int f) {
+    return (f == kMXFP8 || f == kMXFP4 || f == kINT4G32) ? 32 : f == kNVFP4 ? 16 : f == kINT4G64 ? 64 : 0;
+}
+__host__ __device__ constexpr bool fmt_is4(int f) {
+    return f == kMXFP4 || f == kNVFP4 || f == kINT4G32 || f == kINT4G64;
+}
+__host__ __device__ constexpr bool fmt_tensor_scaled(int f) { return f == kNVFP4 || f == kFP8Tensor; }
+__host__ __device__ constexpr bool fmt_byte_scales(int f) { return f == kMXFP8 || f == kMXFP4 || f == kNVFP4; }
+
+// ----------------------------------------------------------------- encode
+
+__device__ __forceinline__ uint8_t enc_e4m3(float v) {
+    return (uint8_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
+}
+
+// Two E2M1 codes in one byte: `lo` in bits 0..3, `hi` in bits 4..7.
+__device__ __forceinline__ uint8_t enc_e2m1x2(float lo, float hi) {
+    return (uint8_t)__nv_cvt_float2_to_fp4x2(make_float2(lo, hi), __NV_E2M1, cudaRoundNearest);
+}
+
+// ----------------------------------------------------------------- decode
+
+// E4M3: exponent field e (bias 7), mantissa m; e == 0 is subnormal m * 2^-9;
+// S.1111.111 is NaN.
+__device__ __forceinline__ float dec_e4m3(uint32_t c) {
+    uint32_t e = (c >> 3) & 15u, m = c & 7u;
+    float mag;
+    if ((c & 0x7Fu) == 0x7Fu) mag = __int_as_float(0x7FC00000);
+    else if (e == 0) mag = __fmul_rn((float)m, 0.001953125f);          // m * 2^-9, exact
+    else mag = __int_as_float((int)(((e + 120u) << 23) | (m << 20)));  // (1 + m/8) * 2^(e-7)
+    return (c & 0x80u) ? -mag : mag;
+}
+
+// E2M1: exponent field e (bias 1), mantissa bit m; e == 0 is m * 0.5.
+__device__ __forceinline__ float dec_e2m1(uint32_t c) {
+    uint32_t e = (c >> 1) & 3u, m = c & 1u;
+    float mag = e == 0 ? (m ? 0.5f : 0.0f) : __int_as_float((int)(((e + 126u) << 23) | (m << 22)));
+    return (c & 8u) ? -mag : mag;
+}
+
+// 2^n as fp32 for n in [-127, 127] (2^-127 is the subnormal 0x00400000).
+__device__ __forceinline__ float exp2i_f32(int n) {
+    return n >= -126 ? __int_as_float((n + 127) << 23) : __int_as_float(0x00400000);
+}
+
+// E8M0 scale byte b -> 2^(b - 127); 0xFF is NaN.
+__device__ __forceinline__ float dec_e8m0(uint32_t b) {
+    return b == 255u ? __int_as_float(0x7FC00000) : exp2i_f32((int)b - 127);
+}
+
+__device__ __forceinline__ double exp2i_f64(int n) {   // n in [-1022, 1023]
+    return __longlong_as_double((long long)(n + 1023) << 52);
+}
+
+// floor(log2(a)) for finite a > 0, from the binary32 fields.
+__device__ __forceinline__ int floor_log2_pos(float a) {
+    uint32_t u = __float_as_uint(a);
+    int e = (int)((u >> 23) & 0xFFu);
+    if (e) return e - 127;
+    return (31 - __clz((int)(u & 0x7FFFFFu))) - 149;
+}
+
+// ----------------------------------------------------------------- scale rules
+
+// OCP MX shared scale: e = floor(log2 amax) - emax_elem, clamped to [-127,127];
+// scale byte e + 127.  Returns the byte; `inv` gets 2^-e.  amax must be > 0.
+__device__ __forceinline__ uint32_t mx_scale(float amax, int emax_elem, float &inv) {
+    int e = floor_log2_pos(amax) - emax_elem;
+    e = e < -127 ? -127 : (e > 127 ? 127 : e);
+    inv = exp2i_f32(-e);
+    return (uint32_t)(e + 127);
+}
+
+// NVFP4 tensor scale s_t = RN(amax_T / (6 * 448)); 1 when that is 0.
+__device__ __forceinline__ float nvfp4_tensor_scale(float amax_t) {
+    float s = __fdiv_rn(amax_t, 2688.0f);
+    return s == 0.0f ? 1.0f : s;
+}
+
+// FP8 per-tensor scale s = RN(amax_T / 448); 1 when that is 0.
+__device__ __forceinline__ float fp8_tensor_scale(float amax_t) {
+    float s = __fdiv_rn(amax_t, 448.0f);
+    return s == 0.0f ? 1.0f : s;
+}
+
+// NVFP4 block: E4M3 block scale of RN(RN(amax_b / 6) / s_t); decode scale
+// d = RN(value(e4) * s_t) (0 when e4 == 0).
+__device__ __forceinline__ uint32_t nvfp4_block_scale(float amax_b, float s_t, float &d) {
+    float raw = __fdiv_rn(__fdiv_rn(amax_b, 6.0f), s_t);
+    uint32_t e4 = enc_e4m3(raw);
+    d = e4 ? __fmul_rn(dec_e4m3(e4), s_t) : 0.0f;
+    return e4;
+}
+
+// Symmetric integer code: clamp(RNE(RN(v / s)), -qmax, qmax); 0 when s == 0.
+__device__ __forceinline__ int int_code(float v, float s, int qmax) {
+    if (s == 0.0f) return 0;
+    int q = __float2int_rn(__fdiv_rn(v, s));
+    return q > qmax ? qmax : (q < -qmax ? -qmax : q);
+}
+
+// ----------------------------------------------------------------- loads
+
+// 16 consecutive elements as fp32 (bf16 widened exactly).
+__device__ __forceinline__ void load16(const float *p, float v[16]) {
+    const float4 *q = reinterpret_cast<const float4 *>(p);
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        float4 t = __ldg(q + i);
+        v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
+    }
+}
+__device__ __forceinline__ void load16(const __nv_bfloat16 *p, float v[16]) {
+    const uint4 *q = reinterpret_cast<const uint4 *>(p);
+#pragma unroll
+    for (int i = 0; i < 2; i++) {
+        uint4 t = __ldg(q + i);
+        uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+            v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+    }
+}
+
+__device__ __forceinline__ void store16(float *p, const float v[16]) {
+    float4 *q = reinterpret_cast<float4 *>(p);
+#pragma unroll
+    for (int i = 0; i < 4; i++) q[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);   // RNE; .x (low half) = lo
+    return *reinterpret_cast<uint32_t *>(&t);
+}
+__device__ __forceinline__ void store16(__nv_bfloat16 *p, const float v[16]) {
+    uint4 *q = reinterpret_cast<uint4 *>(p);
+#pragma unroll
+    for (int i = 0; i < 2; i++)
+        q[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                          pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+}
+
+__device__ __forceinline__ float amax16(const float v[16]) {
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; i++) m = fmaxf(m, fabsf(v[i]));
+    return m;
+}
+
+// Max over aligned groups of G lanes (G a power of two <= 32).
+template <int G>
+__device__ __forceinline__ float group_max(float a) {
+#pragma unroll
+    for (int o = 1; o < G; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+    return a;
+}
+
+// ----------------------------------------------------------------- Hadamard
+
+// Block-diagonal Hadamard rotation of size b ("Bridging the Gap ...",
+// item 3) over 16-element chunks, one chunk per lane, consecutive chunks of
+// a row in consecutive lanes.  Butterfly stage h pairs elements i and i+h
+// (bit h of i clear) into (a+c, a-c); stages h < 16 stay inside the lane,
+// stages h >= 16 pair lanes that differ in bit h/16.  Then every element is
+// multiplied by RN(1/sqrt(b)).  All lanes of the warp must call this.
+__device__ __forceinline__ void hadamard_chunk(float v[16], int b, int lane) {
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1) {
+        if (h < b) {
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                if (!(i & h)) {
+                    float a = v[i], c = v[i + h];
+                    v[i] = __fadd_rn(a, c);
+                    v[i + h] = __fsub_rn(a, c);
+                }
+            }
+        }
+    }
+    for (int h = 16; h < b; h <<= 1) {
+        int lm = h >> 4;
+        bool upper = (lane & lm) != 0;
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+            float p = __shfl_xor_sync(0xFFFFFFFFu, v[i], lm);
+            v[i] = upper ? __fsub_rn(p, v[i]) : __fadd_rn(v[i], p);
+        }
+    }
+    float norm = __frsqrt_rn((float)b);
+#pragma unroll
+    for (int i = 0; i < 16; i++) v[i] = __fmul_rn(v[i], norm);
+}
+
+// Byte offset of scale (row r, scale column s) in the MMA scale layout:
+// 128-row x 4-column atoms of 512 bytes, row r%32 at 16-byte pitch, the four
+// 32-row quarters side by side in each 16-byte line.
+__host__ __device__ __forceinline__ int64_t mma_scale_offset(int64_t r, int64_t s, int64_t s_pad) {
+    return ((r >> 7) * (s_pad >> 2) + (s >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (s & 3);
+}
+
+}  // namespace mxq

@@ -1,0 +1,49 @@
+// mxq_internal.h -- host-side launchers shared between the kernel files and
+// the C ABI layer.  Arguments are validated by the C ABI before any call.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace mxq {
+
+constexpr int kMaxCandidates = 8;
+
+cudaError_t launch_amax(const void *x, bool bf16, int64_t rows, int64_t cols, int hadamard_b,
+                        unsigned int *amax_word, cudaStream_t s);
+cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols, int fmt, int hadamard_b,
+                            int layout, void *codes, void *scales, size_t scales_bytes, float *tensor_scale,
+                            unsigned int *amax_word, cudaStream_t s);
+cudaError_t launch_dequantize(int fmt, int layout, int64_t rows, int64_t cols, const void *codes,
+                              const void *scales, const float *tensor_scale, void *y, bool bf16_out,
+                              cudaStream_t s);
+cudaError_t launch_hadamard(const void *x, void *y, bool bf16, int64_t rows, int64_t cols, int b,
+                            cudaStream_t s);
+cudaError_t launch_cast(const float *x, int64_t n, int elem, uint8_t *out, cudaStream_t s);
+cudaError_t launch_select(const void *w, bool bf16, int64_t n, int64_t k, const int *cands, int ncand,
+                          uint8_t *choice, double *sse, unsigned int *amax_word, cudaStream_t s);
+
+cudaError_t launch_lowrank_down(const void *x, bool bf16, int64_t m, int64_t k, const void *l1, int r,
+                                float *t, cudaStream_t s);
+cudaError_t launch_pack_l2(const void *l2, int r, int64_t n, void *l2p, cudaStream_t s);
+cudaError_t launch_pack_t(const float *t, int r, int64_t m, const float *xs, const float *ws, void *tp,
+                          cudaStream_t s);
+
+struct GemmOperands {
+    int fmt;
+    int64_t m, n, k;
+    const void *a_codes, *b_codes;         // MMA layout
+    const void *a_scales, *b_scales;       // byte scales (MMA layout) or fp32 row scales (INT8)
+    const float *a_tensor_scale, *b_tensor_scale;
+    const void *tp;                        // packed low-rank activation (m x 64 bf16) or null
+    const void *l2p;                       // packed up-projection (n x 64 bf16)
+    void *y;
+    bool y_bf16;
+};
+cudaError_t launch_qlinear(const GemmOperands &op, cudaStream_t s);
+
+// Device error word (bounded waits that ran out); read-and-clear.
+cudaError_t read_and_clear_error(unsigned int *value);
+
+}  // namespace mxq

@@ -1,0 +1,106 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/mxq.h declares, sizes and routing agree with the
+documented formulas, and bad arguments are rejected before any launch."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def mxq():
+    from microscaling_bit_quantization_b200 import build
+    build.build()
+    import microscaling_bit_quantization_b200 as m
+    return m
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "mxq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mxq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(mxq):
+    names = _declared()
+    assert len(names) >= 15
+    lib = ctypes.CDLL(mxq.LIB_PATH)
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(names) == set(mxq.EXPORTS)
+
+
+def test_status_strings(mxq):
+    for code in range(6):
+        assert mxq.lib().mxq_status_string(code)
+
+
+def test_sizes(mxq):
+    M = mxq
+    assert M.codes_bytes(M.NVFP4, 64, 256) == 64 * 128
+    assert M.codes_bytes(M.MXFP8, 64, 256) == 64 * 256
+    assert M.codes_bytes(M.INT4_G64, 64, 256, M.MMA) == 64 * 256
+    assert M.scales_bytes(M.NVFP4, 64, 256) == 64 * 16
+    assert M.scales_bytes(M.NVFP4, 64, 256, M.MMA) == 128 * 16
+    assert M.scales_bytes(M.MXFP4, 300, 96, M.MMA) == 384 * 16
+    assert M.scales_bytes(M.MXFP8, 4096, 3072, M.MMA) == 4096 * 96
+    assert M.scales_bytes(M.INT4_G32, 10, 64) == 10 * 2 * 4
+    assert M.scales_bytes(M.INT8_ROW, 10, 64) == 40
+    assert M.scales_bytes(M.FP8_TENSOR, 10, 64) == 0
+    assert M.quantize_workspace_bytes(M.NVFP4) >= 4 and M.quantize_workspace_bytes(M.MXFP8) == 0
+    assert M.qlinear_workspace_bytes(4096) == 4096 * 128
+
+
+def test_bad_shapes_rejected_on_host(mxq):
+    L, P = mxq.lib(), ctypes.c_void_p
+    size = ctypes.c_size_t(0)
+    assert L.mxq_codes_bytes(mxq.MXFP8, 4, 48, 0, ctypes.byref(size)) == 1          # 48 % 32
+    assert L.mxq_codes_bytes(mxq.INT4_G64, 4, 96, 0, ctypes.byref(size)) == 1       # 96 % 64
+    assert L.mxq_codes_bytes(9, 4, 64, 0, ctypes.byref(size)) == 1                  # bad fmt
+    dummy = P(256)
+    # cols not a multiple of 16, hadamard not a power of two, null pointers
+    assert L.mxq_quantize(dummy, 1, 4, 40, mxq.INT8_ROW, 0, 0, dummy, dummy, None, None, 0, None) == 1
+    assert L.mxq_quantize(dummy, 1, 4, 64, mxq.MXFP8, 48, 0, dummy, dummy, None, None, 0, None) == 1
+    assert L.mxq_quantize(None, 1, 4, 64, mxq.MXFP8, 0, 0, dummy, dummy, None, None, 0, None) == 1
+    # NVFP4 needs a tensor-scale pointer and workspace
+    assert L.mxq_quantize(dummy, 1, 4, 64, mxq.NVFP4, 0, 0, dummy, dummy, None, dummy, 16, None) == 1
+    assert L.mxq_quantize(dummy, 1, 4, 64, mxq.NVFP4, 0, 0, dummy, dummy, dummy, dummy, 2, None) == 5
+    assert L.mxq_hadamard_block(dummy, dummy, 1, 4, 64, 3, None) == 1
+    assert L.mxq_hadamard_block(dummy, dummy, 1, 4, 64, 512, None) == 1
+    assert L.mxq_lowrank_down(dummy, 1, 4, 64, dummy, 33, dummy, None) == 1
+    assert L.mxq_cast(dummy, 10, 2, dummy, None) == 1
+
+
+def test_qlinear_argument_checks(mxq):
+    L = mxq.lib()
+    Q = mxq._QTensorC
+    a = Q(mxq.NVFP4, mxq.MMA, 64, 256, 256, 256, 256)
+    b = Q(mxq.MXFP4, mxq.MMA, 128, 256, 256, 256, 256)
+    y = ctypes.c_void_p(256)
+    assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(b), None, None, 0, y, 0, None, 0, None) == 2   # format pair
+    b = Q(mxq.NVFP4, mxq.CANONICAL, 128, 256, 256, 256, 256)
+    assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(b), None, None, 0, y, 0, None, 0, None) == 1   # layout
+    b = Q(mxq.NVFP4, mxq.MMA, 128, 192, 256, 256, 256)
+    assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(b), None, None, 0, y, 0, None, 0, None) == 1   # K mismatch
+    a = Q(mxq.INT4_G64, mxq.MMA, 64, 256, 256, 256, 0)
+    b = Q(mxq.INT4_G64, mxq.MMA, 64, 256, 256, 256, 0)
+    assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(b), None, None, 0, y, 0, None, 0, None) == 2
+    a = Q(mxq.NVFP4, mxq.MMA, 64, 256, 256, 256, 256)
+    b = Q(mxq.NVFP4, mxq.MMA, 128, 256, 256, 256, 256)
+    t = ctypes.c_void_p(256)
+    # low-rank branch needs workspace of m x 128 bytes
+    assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(b), t, t, 8, y, 0, t, 100, None) == 5
+    assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(b), t, t, 40, y, 0, t, 64 * 128, None) == 1
+
+
+def test_route_matches_oracle(mxq, orc):
+    rng = np.random.default_rng(3)
+    for n_layers, n_int, n_steps in ((112, 10, 20), (7, 3, 11), (1, 1, 1)):
+        table = rng.integers(0, 7, size=(n_layers, n_int)).astype(np.uint8)
+        for layer in range(n_layers):
+            for step in range(-1, n_steps + 1):
+                assert mxq.route(table, layer, step, n_steps) == orc.route(table, n_layers, n_int, layer, step, n_steps)

@@ -1,0 +1,167 @@
+"""GPU parity of the low-rank branch and the tcgen05 block-scaled GEMM
+against the oracle's binary64 GEMM over exactly dequantized operands.
+
+Tolerance (stated by the benchmark spec for fp32 output): relative Frobenius error
+<= 1e-4 and max abs error <= 1e-4 * max|Y_ref|; bf16 output also allows the
+final bf16 rounding (see gpu_util.gemm_close).  Quantized operands are
+produced by the library and checked bit-exact against the oracle's in
+test_gpu_quantize; here the oracle re-derives every operand (codes, scales,
+T = bf16(X) . L1) from the same seeded inputs itself."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from gpu_util import assert_qtensor_equal, dev, gemm_close, host_values
+
+pytestmark = pytest.mark.gpu
+
+GEMM_FMTS = (2, 1, 0, 6, 5)   # NVFP4, MXFP4, MXFP8, FP8_TENSOR, INT8_ROW
+LOWRANK_FMTS = (2, 1, 0, 6)
+
+
+@pytest.fixture(scope="module")
+def mxq():
+    import microscaling_bit_quantization_b200 as m
+    assert torch.cuda.is_available() and m.lib().mxq_device_supported(0) == 1
+    return m
+
+
+def _inputs(seed, m, n, k, r=0):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_t(4, size=(m, k)).astype(np.float32)
+    x[:, rng.choice(k, max(1, k // 64), replace=False)] *= 30
+    w = (rng.standard_normal((n, k)) * 0.02).astype(np.float32)
+    out = {"x": workloads.to_bf16_values(x), "w": workloads.to_bf16_values(w)}
+    if r:
+        out["l1"] = workloads.to_bf16_values((rng.standard_normal((k, r)) * 0.05).astype(np.float32))
+        out["l2"] = workloads.to_bf16_values((rng.standard_normal((r, n)) * 0.05).astype(np.float32))
+    return out
+
+
+def _run(mxq, fmt, d, r, out_dtype, hadamard_b=0, x_dtype="bf16"):
+    xq = mxq.quantize(dev(d["x"], x_dtype), fmt, hadamard_b, mxq.MMA)
+    wq = mxq.quantize(dev(d["w"], "bf16"), fmt, hadamard_b, mxq.MMA)
+    t = l2p = None
+    if r:
+        t = mxq.lowrank_down(dev(d["x"], x_dtype), dev(d["l1"], "bf16"))
+        l2p = mxq.lowrank_pack_l2(dev(d["l2"], "bf16"))
+    y = mxq.qlinear(xq, wq, t, l2p, r, out_dtype=out_dtype)
+    assert mxq.check() == 0
+    return y, xq, wq
+
+
+def _ref(orc, fmt, d, r, rows=None, hadamard_b=0):
+    oxq = orc.quantize(d["x"], fmt, hadamard_b)
+    owq = orc.quantize(d["w"], fmt, hadamard_b)
+    t = None
+    if r:
+        t = orc.lowrank_down(d["x"], d["l1"]) if rows is None else orc.lowrank_down_rows(d["x"], d["l1"], rows)
+    return orc.qlinear(oxq, owq, t, d.get("l2"), rows=rows), oxq, owq
+
+
+@pytest.mark.parametrize("fmt", GEMM_FMTS)
+@pytest.mark.parametrize("shape", [(200, 384, 512), (64, 128, 256), (130, 520, 320), (257, 256, 1024)])
+def test_qlinear_shapes(mxq, orc, fmt, shape):
+    m, n, k = shape
+    if k % 64 and fmt in (1, 2):
+        pytest.skip("4-bit K must be a multiple of 64")
+    d = _inputs(10 + fmt, m, n, k)
+    ref, oxq, owq = _ref(orc, fmt, d, 0)
+    for out_dtype in (torch.float32, torch.bfloat16):
+        y, xq, wq = _run(mxq, fmt, d, 0, out_dtype)
+        gemm_close(y.float().cpu().numpy(), ref, bf16_out=out_dtype == torch.bfloat16)
+    assert_qtensor_equal(xq, oxq, layout_mma=True)
+    assert_qtensor_equal(wq, owq, layout_mma=True)
+
+
+@pytest.mark.parametrize("fmt", GEMM_FMTS)
+def test_qlinear_short_k(mxq, orc, fmt):
+    k = 64 if fmt in (1, 2) else 96
+    d = _inputs(20 + fmt, 70, 300, k)
+    ref, _, _ = _ref(orc, fmt, d, 0)
+    y, _, _ = _run(mxq, fmt, d, 0, torch.float32)
+    gemm_close(y.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("fmt", LOWRANK_FMTS)
+@pytest.mark.parametrize("r", [8, 32])
+def test_qlinear_lowrank(mxq, orc, fmt, r):
+    d = _inputs(30 + fmt, 150, 384, 512, r)
+    ref, _, _ = _ref(orc, fmt, d, r)
+    for out_dtype in (torch.float32, torch.bfloat16):
+        y, _, _ = _run(mxq, fmt, d, r, out_dtype)
+        gemm_close(y.float().cpu().numpy(), ref, bf16_out=out_dtype == torch.bfloat16)
+
+
+def test_lowrank_down(mxq, orc):
+    d = workloads.svdquant_mlp_up(draw_weights=False)
+    t = mxq.lowrank_down(dev(d["x"], "bf16"), dev(d["l1"], "bf16")).cpu().numpy().astype(np.float64)
+    ref = orc.lowrank_down(d["x"], d["l1"])
+    err = np.abs(t - ref)
+    assert err.max() <= 1e-5 * np.abs(ref).max()
+    w1 = workloads.tiny_nvfp4_linear()
+    t = mxq.lowrank_down(dev(w1["x"], "f32"), dev(w1["l1"], "bf16")).cpu().numpy()
+    ref = orc.lowrank_down(w1["x"], w1["l1"])
+    assert np.abs(t - ref).max() <= 1e-5 * np.abs(ref).max()
+
+
+def test_tiny_nvfp4_linear_full(mxq, orc):
+    """Workload 1 end to end, every output: fp32 X, NVFP4, rank-8 branch."""
+    w1 = workloads.tiny_nvfp4_linear()
+    d = {"x": w1["x"], "w": w1["w"], "l1": w1["l1"], "l2": w1["l2"]}
+    ref, oxq, owq = _ref(orc, 2, d, 8)
+    xq = mxq.quantize(dev(d["x"], "f32"), 2, 0, mxq.MMA)
+    wq = mxq.quantize(dev(d["w"], "f32"), 2, 0, mxq.MMA)
+    assert_qtensor_equal(xq, oxq, layout_mma=True)
+    assert_qtensor_equal(wq, owq, layout_mma=True)
+    t = mxq.lowrank_down(dev(d["x"], "f32"), dev(d["l1"], "bf16"))
+    l2p = mxq.lowrank_pack_l2(dev(d["l2"], "bf16"))
+    y = mxq.qlinear(xq, wq, t, l2p, 8, out_dtype=torch.float32)
+    assert mxq.check() == 0
+    gemm_close(y.cpu().numpy(), ref)
+
+
+def _sample_rows(m, seed, count=256):
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(m, size=count, replace=False))
+    rows[-1] = m - 1
+    return rows
+
+
+@pytest.mark.parametrize("fmt", [2, 1])
+def test_svdquant_mlp_up_full_size(mxq, orc, fmt):
+    """Workload 3 at full size (4096 x 12288 x 3072, rank 32) in the launch
+    configuration the benchmark times; 256 sampled rows x all columns."""
+    d = workloads.svdquant_mlp_up()
+    rows = _sample_rows(4096, 3)
+    ref, _, _ = _ref(orc, fmt, d, 32, rows=rows)
+    for out_dtype in (torch.bfloat16, torch.float32):
+        y, _, _ = _run(mxq, fmt, d, 32, out_dtype)
+        gemm_close(y[torch.from_numpy(rows).cuda()].float().cpu().numpy(), ref,
+                   bf16_out=out_dtype == torch.bfloat16)
+        del y
+
+
+@pytest.mark.parametrize("hadamard_b", [0, 128])
+def test_mxfp4_hadamard_full_size(mxq, orc, hadamard_b):
+    """Workload 4: 8192 x 4096 x 4096 MXFP4, with and without the b=128 rotation."""
+    d = workloads.mxfp4_hadamard_gemm()
+    rows = _sample_rows(8192, 4)
+    ref, _, _ = _ref(orc, 1, d, 0, rows=rows, hadamard_b=hadamard_b)
+    y, _, _ = _run(mxq, 1, d, 0, torch.float32, hadamard_b=hadamard_b)
+    gemm_close(y[torch.from_numpy(rows).cuda()].cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("fmt", [5, 6, 0])
+def test_dit_layers_full_size(mxq, orc, fmt):
+    """Workload 5 linears at M = 8192 in each routed format."""
+    seed = 5
+    for (name, kin, nout), step in zip(workloads.DIT_LINEARS, (0, 7, 13, 19)):
+        x = workloads.dit_activation(seed, step, kin)
+        w = workloads.dit_weight(seed, 0, kin, nout)
+        d = {"x": x, "w": w}
+        rows = _sample_rows(workloads.DIT_TOKENS, step, 128)
+        ref, _, _ = _ref(orc, fmt, d, 0, rows=rows)
+        y, _, _ = _run(mxq, fmt, d, 0, torch.float32)
+        gemm_close(y[torch.from_numpy(rows).cuda()].cpu().numpy(), ref)

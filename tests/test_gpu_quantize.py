@@ -1,0 +1,200 @@
+"""GPU parity of the HBM-bound kernels against the oracle: quantize (every
+format, fp32/bf16 input, both layouts, with and without Hadamard),
+dequantize, the Hadamard rotation, the element casts (exhaustively over all
+2^32 fp32 bit patterns) and the per-channel format selection.  Codes,
+scales and choices must match bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from gpu_util import assert_qtensor_equal, dev, host_values, nasty_matrix
+
+pytestmark = pytest.mark.gpu
+
+ALL_FMTS = (0, 1, 2, 3, 4, 5, 6)
+
+
+@pytest.fixture(scope="module")
+def mxq():
+    import microscaling_bit_quantization_b200 as m
+    assert torch.cuda.is_available() and m.lib().mxq_device_supported(0) == 1
+    return m
+
+
+def _moderate(x):
+    x = x.copy()
+    x[3, :] = np.clip(x[3, :], -1e4, 1e4)   # keep Hadamard sums finite
+    return x
+
+
+@pytest.mark.parametrize("fmt", ALL_FMTS)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("hadamard_b", [0, 2, 32, 128, 256])
+def test_quantize_small_ragged(mxq, orc, fmt, dtype, hadamard_b):
+    rows, cols = 37, 512
+    x = nasty_matrix(100 + fmt, rows, cols)
+    if hadamard_b:
+        x = _moderate(x)
+    xv = host_values(x, dtype)
+    ref = orc.quantize(xv, fmt, hadamard_b)
+    for layout in (mxq.CANONICAL, mxq.MMA):
+        q = mxq.quantize(dev(x, dtype), fmt, hadamard_b, layout)
+        torch.cuda.synchronize()
+        assert_qtensor_equal(q, ref, layout_mma=layout == mxq.MMA)
+
+
+@pytest.mark.parametrize("fmt", ALL_FMTS)
+def test_quantize_edge_shapes(mxq, orc, fmt):
+    blk = {0: 32, 1: 32, 2: 16, 3: 32, 4: 64, 5: 16, 6: 16}[fmt]
+    for rows, cols in ((0, 64), (1, 64), (129, blk), (3, 1024 + 64)):
+        x = nasty_matrix(7, max(rows, 1), cols)[:rows]
+        ref = orc.quantize(x, fmt) if rows else None
+        for layout in (mxq.CANONICAL, mxq.MMA):
+            q = mxq.quantize(dev(x, "f32"), fmt, 0, layout)
+            torch.cuda.synchronize()
+            if rows:
+                assert_qtensor_equal(q, ref, layout_mma=layout == mxq.MMA)
+            elif fmt in (2, 6):
+                assert q.tensor_scale.item() == 1.0
+    # all-zero tensor
+    z = np.zeros((8, 128), np.float32)
+    q = mxq.quantize(dev(z, "bf16"), fmt)
+    assert_qtensor_equal(q, orc.quantize(z, fmt))
+
+
+def test_quantize_full_size_workloads(mxq, orc):
+    """Each workload's activations (and weights) at full size, every element."""
+    w2 = workloads.chameleon_selection()
+    q = mxq.quantize(dev(w2["x"], "bf16"), mxq.MXFP8, 0, mxq.MMA)
+    assert_qtensor_equal(q, orc.quantize(w2["x"], mxq.MXFP8), layout_mma=True)
+    del w2
+    w3 = workloads.svdquant_mlp_up()
+    for fmt in (mxq.NVFP4, mxq.INT4_G64):
+        for name in ("x", "w"):
+            q = mxq.quantize(dev(w3[name], "bf16"), fmt, 0, mxq.MMA)
+            assert_qtensor_equal(q, orc.quantize(w3[name], fmt), layout_mma=True)
+    del w3
+    w4 = workloads.mxfp4_hadamard_gemm()
+    for hb in (0, 128):
+        q = mxq.quantize(dev(w4["x"], "bf16"), mxq.MXFP4, hb, mxq.MMA)
+        assert_qtensor_equal(q, orc.quantize(w4["x"], mxq.MXFP4, hb), layout_mma=True)
+    w1 = workloads.tiny_nvfp4_linear()
+    q = mxq.quantize(dev(w1["x"], "f32"), mxq.NVFP4)
+    assert_qtensor_equal(q, orc.quantize(w1["x"], mxq.NVFP4))
+
+
+def test_quantize_dit_activations(mxq, orc):
+    """Workload 5 activations: every step's tail index, the three formats, a
+    forced layer's 163x column spread."""
+    seed = 5
+    for step in (0, 9, 19):
+        x = workloads.dit_activation(seed, step, workloads.DIT_HIDDEN, m=1024)
+        for fmt in (mxq.INT8_ROW, mxq.FP8_TENSOR, mxq.MXFP8):
+            q = mxq.quantize(dev(x, "bf16"), fmt, 0, mxq.MMA)
+            assert_qtensor_equal(q, orc.quantize(x, fmt), layout_mma=True)
+    f = workloads.dit_forced_column_factors(seed, 3, workloads.DIT_MLP)
+    x = workloads.to_bf16_values(workloads.dit_activation(seed, 4, workloads.DIT_MLP, m=512) * f[None, :])
+    q = mxq.quantize(dev(x, "bf16"), mxq.MXFP8, 0, mxq.MMA)
+    assert_qtensor_equal(q, orc.quantize(x, mxq.MXFP8), layout_mma=True)
+
+
+@pytest.mark.parametrize("fmt", ALL_FMTS)
+@pytest.mark.parametrize("layout", [0, 1])
+def test_dequantize(mxq, orc, fmt, layout):
+    x = nasty_matrix(200 + fmt, 29, 256)
+    oq = orc.quantize(x, fmt)
+    q = mxq.quantize(dev(x, "f32"), fmt, 0, layout)
+    want = orc.dequantize_f32(oq)
+    y32 = mxq.dequantize(q, torch.float32).cpu().numpy()
+    np.testing.assert_array_equal(y32.view(np.uint32), want.view(np.uint32))
+    y16 = mxq.dequantize(q, torch.bfloat16).cpu()
+    want16 = torch.from_numpy(want).to(torch.bfloat16)
+    assert torch.equal(y16.view(torch.int16), want16.view(torch.int16))
+
+
+@pytest.mark.parametrize("b", [2, 4, 8, 16, 32, 64, 128, 256])
+def test_hadamard_block(mxq, orc, b):
+    x = _moderate(nasty_matrix(300 + b, 45, 512))
+    y = mxq.hadamard_block(dev(x, "f32"), b).cpu().numpy()
+    np.testing.assert_array_equal(y.view(np.uint32), orc.hadamard(x, b).view(np.uint32))
+    xb = host_values(x, "bf16")
+    yb = mxq.hadamard_block(dev(x, "bf16"), b).cpu()
+    want = torch.from_numpy(orc.hadamard(xb, b)).to(torch.bfloat16)
+    assert torch.equal(yb.view(torch.int16), want.view(torch.int16))
+
+
+def test_hadamard_full_size(mxq, orc):
+    w4 = workloads.mxfp4_hadamard_gemm()
+    x = w4["w"]
+    y = mxq.hadamard_block(dev(x, "f32"), 128).cpu().numpy()
+    np.testing.assert_array_equal(y.view(np.uint32), orc.hadamard(x, 128).view(np.uint32))
+
+
+@pytest.mark.parametrize("elem", ["e4m3", "e2m1"])
+def test_cast_exhaustive(mxq, orc, elem):
+    """Every fp32 bit pattern (NaN inputs excluded for E2M1, which has no NaN)."""
+    chunk = 1 << 27
+    bad = 0
+    for start in range(0, 1 << 32, chunk):
+        bits = torch.arange(start, start + chunk, dtype=torch.int64, device="cuda")
+        x = bits.to(torch.int32).view(torch.float32) if start < (1 << 31) else \
+            (bits - (1 << 32)).to(torch.int32).view(torch.float32)
+        got = mxq.cast(x.contiguous(), elem)
+        want = torch.from_numpy(orc.cast_range(start, chunk, elem)).cuda()
+        if elem == "e2m1":
+            keep = ~torch.isnan(x)
+            bad += int((got[keep] != want[keep]).sum())
+        else:
+            bad += int((got != want).sum())
+        del bits, x, got, want
+    assert bad == 0
+
+
+def _near_tie_ok(choice_gpu, choice_ref, sse_ref, cands):
+    """Rows may differ only where the oracle's best two errors are within 1e-12 relative."""
+    diff = np.nonzero(choice_gpu != choice_ref)[0]
+    for r in diff:
+        s = np.sort(sse_ref[r])
+        assert s[1] - s[0] <= 1e-12 * max(s[0], 1e-300), (r, sse_ref[r])
+    return len(diff)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_select_small(mxq, orc, dtype):
+    x = nasty_matrix(400, 40, 256)
+    x = host_values(_moderate(x), dtype)
+    cands = [mxq.INT4_G32, mxq.NVFP4, mxq.MXFP4, mxq.MXFP8, mxq.INT8_ROW, mxq.FP8_TENSOR, mxq.INT4_G64]
+    ch, sse = mxq.select_weight_format(dev(x, dtype), cands)
+    ref_ch, ref_sse = orc.select_weight_format(x, cands)
+    np.testing.assert_allclose(sse.cpu().numpy(), ref_sse, rtol=1e-12, atol=0)
+    _near_tie_ok(ch.cpu().numpy(), ref_ch, ref_sse, cands)
+
+
+def test_select_constructed_rows(mxq, orc):
+    """The oracle's constructed rows (exact ties, strict winners) choose identically."""
+    grid = np.array([0, .5, 1, 1.5, 2, 3, 4, 6], np.float32)
+    rng = np.random.default_rng(23)
+    w = np.zeros((4, 64), np.float32)
+    w[0] = rng.choice(grid, 64) * 448
+    w[0, ::16] = 2688
+    w[1] = rng.choice(grid, 64) * rng.choice([-1, 1], 64)
+    w[1, ::16] = 6
+    w[2] = w[1] * np.float32(2.0 ** -20)
+    w[3] = rng.integers(-7, 8, 64) * np.float32(0.25)
+    w[3, 0], w[3, 32] = 1.75, -1.75
+    for cands in ([mxq.INT4_G32, mxq.NVFP4, mxq.MXFP4], [mxq.INT4_G32, mxq.MXFP4, mxq.NVFP4]):
+        ch, sse = mxq.select_weight_format(dev(w, "f32"), cands)
+        ref_ch, ref_sse = orc.select_weight_format(w, cands)
+        np.testing.assert_array_equal(ch.cpu().numpy(), ref_ch)
+        np.testing.assert_array_equal(sse.cpu().numpy() == 0, ref_sse == 0)
+
+
+def test_select_full_size(mxq, orc):
+    """Workload 2: W 3072 x 3072 bf16 Student-t, candidates {INT4-g32, NVFP4, MXFP4}."""
+    w = workloads.chameleon_selection()["w"]
+    cands = [mxq.INT4_G32, mxq.NVFP4, mxq.MXFP4]
+    ch, sse = mxq.select_weight_format(dev(w, "bf16"), cands)
+    ref_ch, ref_sse = orc.select_weight_format(w, cands)
+    np.testing.assert_allclose(sse.cpu().numpy(), ref_sse, rtol=1e-12, atol=0)
+    assert _near_tie_ok(ch.cpu().numpy(), ref_ch, ref_sse, cands) <= 3
