@@ -1,0 +1,381 @@
+#!/usr/bin/env python
+"""Benchmark of the W4A4 quantized linear layer (SVDQuant MLP up-projection,
+NVFP4, rank-32 low-rank branch): X 4096 x 3072 bf16, residual weight
+12288 x 3072, L1 3072 x 32, L2 32 x 12288, output bf16.
+
+One step is one inference pass of the layer's hot path on one batch:
+  tensor amax of X -> NVFP4 quantization of X (MMA layout) -> low-rank down
+  projection T = bf16(X) . L1 -> packing of T for the GEMM -> tcgen05
+  block-scaled GEMM with the fused epilogue and low-rank up projection.
+The weight (quantized to NVFP4, L2 packed) is prepared once, before timing,
+as a deployed layer's weights are.
+
+Contract: `python bench.py --gpus N --steps K --warmup W` prints one JSON line
+on rank 0.  N > 1 runs under torchrun, one process per GPU; each rank runs the
+same layer on its own batch (data parallel over tokens, no collective on the
+data path: weak scaling); the timed region is bracketed by a barrier and a
+device synchronize, and the time is the max over ranks.  Inputs rotate over
+4 device-resident sets (~190 MB > 126 MB L2), so every step reads its
+operands from HBM.
+
+`--impl reference` times the CPU oracle (oracle/, plain C + numpy binary64
+GEMM) on the host cores on a bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+M, K, N, RANK = 4096, 3072, 12288, 32
+FLOP_MAIN = 2 * M * N * K                       # 309,237,645,312
+FLOP_LR_UP = 2 * M * N * RANK                   # inside the GEMM kernel
+FLOP_LR_DOWN = 2 * M * K * RANK
+FLOP_STEP = FLOP_MAIN + FLOP_LR_UP + FLOP_LR_DOWN
+N_SETS = 4
+WORKLOAD = "svdquant_mlp_up_nvfp4_w4a4_lowrank32"
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "src": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.th = threading.Thread(target=self._read, daemon=True)
+            self.th.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist_init():
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def _max_over_ranks(value, world):
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ oracle
+
+class OracleSample:
+    """The oracle as it stands, on `rows` token rows of the workload per step:
+    NVFP4 quantization (C), low-rank down projection (C), binary64 GEMM over
+    exactly dequantized operands (numpy matmul, one BLAS thread), which
+    dequantizes the whole 12288 x 3072 weight each call."""
+
+    def __init__(self, rows=64):
+        import oracle
+        import workloads
+        d = workloads.svdquant_mlp_up()
+        self.rows = rows
+        self.x = d["x"][:rows].copy()
+        self.l1, self.l2 = d["l1"], d["l2"]
+        self.wq = oracle.quantize(d["w"], oracle.NVFP4)
+        self.flops = 2 * rows * N * K + 2 * rows * N * RANK + 2 * rows * K * RANK
+        self.desc = ("%d of %d token rows per step: NVFP4 quantize, low-rank down projection, binary64 GEMM "
+                     "over exactly dequantized operands (incl. dequantizing the 12288 x 3072 weight); "
+                     "1 thread" % (rows, M))
+
+    def step(self):
+        import oracle
+        xq = oracle.quantize(self.x, oracle.NVFP4)
+        t = oracle.lowrank_down(self.x, self.l1)
+        return oracle.qlinear(xq, self.wq, t, self.l2)
+
+    def timed(self, steps):
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(1):
+            t0 = time.perf_counter()
+            for _ in range(steps):
+                self.step()
+            return (time.perf_counter() - t0) / steps
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    o = OracleSample()
+    o.timed(args.warmup)
+    sec = o.timed(args.steps)
+    value = o.flops / sec / 1e12
+    line = {"impl": "reference", "metric": "qlinear TFLOPS (NVFP4 W4A4 + rank-32 low-rank), whole step",
+            "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sec, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "m": M, "k": K, "n": N, "rank": RANK, "sample_rows": o.rows},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": o.desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_ours(args, world, rank, local):
+    import numpy as np
+    import torch
+
+    import microscaling_bit_quantization_b200 as mxq
+    import workloads
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if mxq.lib().mxq_device_supported(local) != 1:
+        raise RuntimeError("this benchmark needs an sm_100 GPU")
+    stream = torch.cuda.current_stream()
+
+    d = workloads.svdquant_mlp_up()
+    x_host = torch.from_numpy(d["x"]).to(torch.bfloat16)
+    w = torch.from_numpy(d["w"]).to(torch.bfloat16).to(dev)
+    l1 = torch.from_numpy(d["l1"]).to(torch.bfloat16).to(dev)
+    l2 = torch.from_numpy(d["l2"]).to(torch.bfloat16).to(dev)
+    del d
+
+    # Offline weight preparation (once): NVFP4 codes + scales, packed L2.
+    wq0 = mxq.quantize(w, mxq.NVFP4, 0, mxq.MMA)
+    l2p = mxq.lowrank_pack_l2(l2)
+    sets = []
+    for i in range(N_SETS):
+        wq = mxq.alloc_qtensor(mxq.NVFP4, N, K, mxq.MMA, dev)
+        wq.codes.copy_(wq0.codes)
+        wq.scales.copy_(wq0.scales)
+        wq.tensor_scale.copy_(wq0.tensor_scale)
+        s = {"x": x_host.to(dev), "wq": wq, "l2p": l2p.clone(),
+             "xq": mxq.alloc_qtensor(mxq.NVFP4, M, K, mxq.MMA, dev),
+             "tp": torch.empty((M, 64), dtype=torch.bfloat16, device=dev),
+             "qws": torch.empty(16, dtype=torch.uint8, device=dev),
+             "y": torch.empty((M, N), dtype=torch.bfloat16, device=dev)}
+        sets.append(s)
+    del w, wq0
+
+    def step(i):
+        s = sets[i % N_SETS]
+        mxq.quantize(s["x"], mxq.NVFP4, 0, mxq.MMA, out=s["xq"], workspace=s["qws"])
+        mxq.lowrank_down_packed(s["x"], l1, s["xq"], s["wq"], out=s["tp"])
+        mxq.qlinear(s["xq"], s["wq"], s["tp"], s["l2p"], out=s["y"])
+
+    launches_per_step = 4      # k_amax, k_quantize, k_lowrank_down (packed), k_gemm
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert mxq.check() == 0
+
+    # ---- timed region
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    _barrier(world)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        step(i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    _barrier(world)
+    clocks = sampler.stop()
+    ms_local = start.elapsed_time(end) / args.steps
+    ms = _max_over_ranks(ms_local, world)
+    assert mxq.check() == 0
+
+    # ---- per-kernel durations of the dominant kernel (GEMM) and the quantizer, on the launch stream
+    def time_kernel(fn, reps):
+        evs = []
+        for i in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn(i)
+            b.record(stream)
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+    def gemm_only(i):
+        s = sets[i % N_SETS]
+        mxq.qlinear(s["xq"], s["wq"], s["tp"], s["l2p"], out=s["y"])
+
+    def quant_only(i):
+        s = sets[i % N_SETS]
+        mxq.quantize(s["x"], mxq.NVFP4, 0, mxq.MMA, out=s["xq"], workspace=s["qws"])
+
+    reps = max(args.steps, 10)
+    gemm_ms = time_kernel(gemm_only, reps)
+    quant_ms = time_kernel(quant_only, reps)
+
+    peaks = _peaks()
+    fp4_peak = peaks["bf16_tflops"] * 4.0          # nominal dense FP4 : BF16 ratio 9 : 2.25
+    gemm_flops = FLOP_MAIN + FLOP_LR_UP
+    gemm_tflops = gemm_flops / (gemm_ms * 1e-3) / 1e12
+    quant_bytes = M * K * 2 + M * K // 2 + (M * K // 16)    # read bf16 X, write codes, write scales
+    quant_gbs = quant_bytes / (quant_ms * 1e-3) / 1e9
+    profiles_traffic = None
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            profiles_traffic = json.load(f).get("k_gemm_nvfp4")
+    except Exception:
+        pass
+
+    # ---- end to end through the public API with host buffers
+    x_pin = x_host.pin_memory()
+    y_pin = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    e_steps = max(3, min(args.steps, 10))
+    for i in range(2):
+        s = sets[i % N_SETS]
+        s["x"].copy_(x_pin, non_blocking=True)
+        step(i)
+        y_pin.copy_(s["y"], non_blocking=True)
+    torch.cuda.synchronize()
+    _barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e_steps):
+        s = sets[i % N_SETS]
+        s["x"].copy_(x_pin, non_blocking=True)
+        step(i)
+        y_pin.copy_(s["y"], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / e_steps, world)
+    _barrier(world)
+
+    cpu = None
+    if rank == 0:
+        o = OracleSample()
+        o.timed(1)
+        sec = o.timed(10)
+        cpu = {"value": o.flops / sec / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+               "sample": o.desc + "; 10 steps"}
+
+    if rank == 0:
+        value = world * FLOP_STEP / (ms * 1e-3) / 1e12
+        line = {
+            "metric": "qlinear TFLOPS (NVFP4 W4A4 + rank-32 low-rank), whole step",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "nvfp4(e2m1+ue4m3)xnvfp4->f32 acc, bf16 out", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "m": M, "k": K, "n": N, "rank": RANK, "out": "bf16",
+                       "l2": "4 rotating input sets (~190 MB > 126 MB L2), no flush",
+                       "parallelism": "dp%d (independent batch per GPU)" % world},
+            "roofline": {"bound": "tensor", "kernel": "k_gemm<NVFP4> (main + low-rank up MMAs, fused epilogue)",
+                         "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
+                         "frac": gemm_tflops / fp4_peak, "traffic": profiles_traffic,
+                         "peak_note": "measured bf16 burst %.1f TF/s x 4 (nominal dense FP4:BF16), of %s"
+                                      % (peaks["bf16_tflops"], peaks["src"]),
+                         "gemm_ms": gemm_ms, "flops_per_launch": gemm_flops},
+            "quantize": {"kernel": "k_amax + k_quantize<NVFP4> (X 4096 x 3072 bf16)", "ms": quant_ms,
+                         "achieved": quant_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": quant_gbs / peaks["hbm_gbs"], "bytes_per_launch": quant_bytes},
+            "e2e": {"value": world * FLOP_STEP / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "ms_per_step": e2e_ms},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = _dist_init()
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -193,12 +193,31 @@ mxq_status mxq_select_weight_format(const void *w, int32_t wdtype, int64_t n, in
 /* ---------------------------------------------------------------------- */
 
 /* SVDQuant low-rank down projection (Nunchaku/Diffusers article, "Main
- * explanation": a 16-bit low-rank part of the weight beside the 4-bit
- * residual): t = bf16(x) . l1 with fp32 accumulation.
+ * explanation": a 16-bit low-rank part of the weight is kept beside the
+ * 4-bit residual): t = bf16(x) . l1 with fp32 accumulation.
  *   x: m x k fp32/bf16 device; l1: k x r bf16 device; t: m x r fp32 device.
  * Constraints: 1 <= r <= 32, k % 16 == 0. */
 mxq_status mxq_lowrank_down(const void *x, int32_t xdtype, int64_t m, int64_t k, const void *l1,
                             int32_t r, float *t, void *stream);
+
+/* Bytes of the packed low-rank activation for m rows (m x 64 bf16). */
+mxq_status mxq_lowrank_packed_bytes(int64_t m, size_t *bytes);
+
+/* Packed low-rank activation, the operand mxq_qlinear reads:
+ *   tp: m x 64 bf16 device; row i = [hi_0 .. hi_31, lo_0 .. lo_31] with
+ *   u_j = t[i][j] / (xs * ws) rounded to fp32, hi_j = bf16(u_j),
+ *   lo_j = bf16(u_j - hi_j), and zeros for j >= r.  xs, ws are the device
+ *   tensor scales of the quantized activation and weight (NVFP4,
+ *   FP8_TENSOR), both NULL for formats without one (then the divisor is 1).
+ * The GEMM epilogue multiplies its accumulator by xs * ws, so the split
+ * high/low product restores t . l2 to about 2^-16 relative.
+ * mxq_lowrank_down_packed computes t as mxq_lowrank_down does and writes
+ * tp directly; mxq_lowrank_pack_t packs a given t (m x r fp32 device). */
+mxq_status mxq_lowrank_down_packed(const void *x, int32_t xdtype, int64_t m, int64_t k, const void *l1,
+                                   int32_t r, const float *x_tensor_scale, const float *w_tensor_scale,
+                                   void *tp, void *stream);
+mxq_status mxq_lowrank_pack_t(const float *t, int32_t r, int64_t m, const float *x_tensor_scale,
+                              const float *w_tensor_scale, void *tp, void *stream);
 
 /* Re-lays the up-projection l2 (r x n bf16, device) as the GEMM operand
  * l2p (n x 64 bf16, device): row j of l2p holds l2[0..r-1][j], zeros up to
@@ -206,29 +225,26 @@ mxq_status mxq_lowrank_down(const void *x, int32_t xdtype, int64_t m, int64_t k,
  * low-rank product).  Done once per weight. */
 mxq_status mxq_lowrank_pack_l2(const void *l2, int32_t r, int64_t n, void *l2p, void *stream);
 
-/* Scratch bytes mxq_qlinear needs for m rows (the packed low-rank
- * activation: m x 64 bf16). */
-mxq_status mxq_qlinear_workspace_bytes(int64_t m, size_t *bytes);
-
 /* Block-scaled low-bit GEMM with fused dequantization epilogue and
  * low-rank branch (Nunchaku/Diffusers article, svdq_w4a4; Chameleon
- * article, W8A8 formats):
+ * article, W8A8 formats), one kernel launch:
  *   y[m][n] = sum_k deq(xq)[m][k] * deq(wq)[n][k]  (+ sum_j t[m][j] * l2[j][n])
- * on tcgen05 tensor cores (fp32 accumulation; int32 for INT8_ROW).
+ * on tcgen05 tensor cores (fp32 accumulation; int32 for INT8_ROW), the
+ * per-block scales applied by the tensor cores, tensor / row scales in the
+ * epilogue.
  *   xq, wq: same fmt, MMA layout, xq->cols == wq->cols == K.
  *     Supported fmt: NVFP4, MXFP4, MXFP8, FP8_TENSOR, INT8_ROW.
- *   t: m x r fp32 device (from mxq_lowrank_down) or NULL for no branch;
- *   l2p: packed up-projection from mxq_lowrank_pack_l2 (n rows); r as there.
- *     The branch is supported for NVFP4, MXFP4, MXFP8 and FP8_TENSOR.
+ *   tp: packed low-rank activation (m x 64 bf16, from
+ *     mxq_lowrank_down_packed / mxq_lowrank_pack_t with the same tensor
+ *     scales as xq, wq) or NULL for no branch; l2p: packed up-projection
+ *     (n rows).  The branch is supported for NVFP4, MXFP4, MXFP8, FP8_TENSOR.
  *   y: m x n device, fp32 or bf16 (fp32 result rounded once, RNE).
- *   workspace: device scratch of mxq_qlinear_workspace_bytes(m) when t is
- *     given (may be NULL otherwise); clobbered.
- * Constraints: K % 64 == 0 (4-bit) or K % 32 == 0 (8-bit); K > 0.
- * Errors: MXQ_EINVAL, MXQ_EUNSUPPORTED (format pair / branch), MXQ_ENOSPACE,
- * MXQ_ECUDA.  A pipeline wait that runs out is reported by mxq_check(). */
-mxq_status mxq_qlinear(const mxq_qtensor *xq, const mxq_qtensor *wq, const float *t,
-                       const void *l2p, int32_t r, void *y, int32_t ydtype, void *workspace,
-                       size_t workspace_bytes, void *stream);
+ * Constraints: K % 64 == 0 (4-bit) or K % 32 == 0 (8-bit); K > 0; device
+ * pointers 16-byte aligned.
+ * Errors: MXQ_EINVAL, MXQ_EUNSUPPORTED (format pair / branch), MXQ_ECUDA.
+ * A pipeline wait that runs out is reported by mxq_check(). */
+mxq_status mxq_qlinear(const mxq_qtensor *xq, const mxq_qtensor *wq, const void *tp, const void *l2p,
+                       void *y, int32_t ydtype, void *stream);
 
 /* ---------------------------------------------------------------------- */
 /* a8: per-layer, per-timestep-interval format table.                      */

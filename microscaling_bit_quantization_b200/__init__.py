@@ -31,8 +31,8 @@ STATUS = {0: "MXQ_OK", 1: "MXQ_EINVAL", 2: "MXQ_EUNSUPPORTED", 3: "MXQ_ECUDA", 4
 # Every entry point the header declares.
 EXPORTS = ("mxq_status_string", "mxq_device_supported", "mxq_check", "mxq_codes_bytes", "mxq_scales_bytes",
            "mxq_quantize_workspace_bytes", "mxq_quantize", "mxq_dequantize", "mxq_hadamard_block", "mxq_cast",
-           "mxq_select_workspace_bytes", "mxq_select_weight_format", "mxq_lowrank_down", "mxq_lowrank_pack_l2",
-           "mxq_qlinear_workspace_bytes", "mxq_qlinear", "mxq_route")
+           "mxq_select_workspace_bytes", "mxq_select_weight_format", "mxq_lowrank_down", "mxq_lowrank_packed_bytes",
+           "mxq_lowrank_down_packed", "mxq_lowrank_pack_t", "mxq_lowrank_pack_l2", "mxq_qlinear", "mxq_route")
 
 
 class MxqError(RuntimeError):
@@ -67,9 +67,11 @@ def _load():
         "mxq_select_workspace_bytes": (i32, [P, i32, psz]),
         "mxq_select_weight_format": (i32, [P, i32, i64, i64, P, i32, P, P, P, sz, P]),
         "mxq_lowrank_down": (i32, [P, i32, i64, i64, P, i32, P, P]),
+        "mxq_lowrank_packed_bytes": (i32, [i64, psz]),
+        "mxq_lowrank_down_packed": (i32, [P, i32, i64, i64, P, i32, P, P, P, P]),
+        "mxq_lowrank_pack_t": (i32, [P, i32, i64, P, P, P, P]),
         "mxq_lowrank_pack_l2": (i32, [P, i32, i64, P, P]),
-        "mxq_qlinear_workspace_bytes": (i32, [i64, psz]),
-        "mxq_qlinear": (i32, [ctypes.POINTER(_QTensorC), ctypes.POINTER(_QTensorC), P, P, i32, P, i32, P, sz, P]),
+        "mxq_qlinear": (i32, [ctypes.POINTER(_QTensorC), ctypes.POINTER(_QTensorC), P, P, P, i32, P]),
         "mxq_route": (i32, [P, i32, i32, i32, i32, i32]),
     }
     for name, (res, args) in sig.items():
@@ -238,25 +240,50 @@ def lowrank_pack_l2(l2: torch.Tensor, stream=None) -> torch.Tensor:
     return l2p
 
 
-def qlinear_workspace_bytes(m: int) -> int:
-    return _size(_lib.mxq_qlinear_workspace_bytes, m)
+def lowrank_packed_bytes(m: int) -> int:
+    return _size(_lib.mxq_lowrank_packed_bytes, m)
 
 
-def qlinear(xq: QTensor, wq: QTensor, t: torch.Tensor = None, l2p: torch.Tensor = None, r: int = 0,
-            out_dtype=torch.bfloat16, out: torch.Tensor = None, workspace: torch.Tensor = None,
-            stream=None) -> torch.Tensor:
-    """y = deq(xq) . deq(wq)^T (+ t . l2) on tcgen05 tensor cores."""
+def _scales_of(xq: Optional[QTensor], wq: Optional[QTensor]):
+    if xq is None or xq.tensor_scale is None:
+        return None, None
+    return _ptr(xq.tensor_scale), _ptr(wq.tensor_scale)
+
+
+def lowrank_down_packed(x: torch.Tensor, l1: torch.Tensor, xq: QTensor = None, wq: QTensor = None,
+                        out: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """Packed low-rank activation (m x 64 bf16) for qlinear, divided by the
+    tensor scales of xq and wq when their format has them."""
+    _require_cuda(x, l1)
+    x, l1 = x.contiguous(), l1.contiguous()
+    m, k = x.shape
+    r = l1.shape[1]
+    tp = out if out is not None else torch.empty((m, 64), dtype=torch.bfloat16, device=x.device)
+    xs, ws = _scales_of(xq, wq)
+    _ok(_lib.mxq_lowrank_down_packed(_ptr(x), _dtype_code(x), m, k, _ptr(l1), r, xs, ws, _ptr(tp), _stream(stream)),
+        "mxq_lowrank_down_packed")
+    return tp
+
+
+def lowrank_pack_t(t: torch.Tensor, xq: QTensor = None, wq: QTensor = None, out: torch.Tensor = None,
+                   stream=None) -> torch.Tensor:
+    _require_cuda(t)
+    t = t.contiguous()
+    m, r = t.shape
+    tp = out if out is not None else torch.empty((m, 64), dtype=torch.bfloat16, device=t.device)
+    xs, ws = _scales_of(xq, wq)
+    _ok(_lib.mxq_lowrank_pack_t(_ptr(t), r, m, xs, ws, _ptr(tp), _stream(stream)), "mxq_lowrank_pack_t")
+    return tp
+
+
+def qlinear(xq: QTensor, wq: QTensor, tp: torch.Tensor = None, l2p: torch.Tensor = None,
+            out_dtype=torch.bfloat16, out: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """y = deq(xq) . deq(wq)^T (+ t . l2 from the packed operands) on tcgen05 tensor cores."""
     m, n = xq.rows, wq.rows
     y = out if out is not None else torch.empty((m, n), dtype=out_dtype, device=xq.codes.device)
-    wsb = 0
-    if t is not None:
-        wsb = qlinear_workspace_bytes(m)
-        if workspace is None:
-            workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=y.device)
-        t = t.contiguous()
     xc, wc = xq.c(), wq.c()
-    _ok(_lib.mxq_qlinear(ctypes.byref(xc), ctypes.byref(wc), _ptr(t), _ptr(l2p), r, _ptr(y), _dtype_code(y),
-                         _ptr(workspace), wsb, _stream(stream)), "mxq_qlinear")
+    _ok(_lib.mxq_qlinear(ctypes.byref(xc), ctypes.byref(wc), _ptr(tp), _ptr(l2p), _ptr(y), _dtype_code(y),
+                         _stream(stream)), "mxq_qlinear")
     return y
 
 

@@ -168,7 +168,30 @@ mxq_status mxq_lowrank_down(const void *x, int32_t xdtype, int64_t m, int64_t k,
                             void *stream) {
     if (!valid_dtype(xdtype) || m < 0 || k <= 0 || k % 16 || r < 1 || r > 32) return MXQ_EINVAL;
     if (m > 0 && (!x || !l1 || !t || !aligned16(x))) return MXQ_EINVAL;
-    return from_cuda(launch_lowrank_down(x, xdtype == MXQ_BF16, m, k, l1, r, t, (cudaStream_t)stream));
+    return from_cuda(launch_lowrank_down(x, xdtype == MXQ_BF16, m, k, l1, r, t, nullptr, nullptr, nullptr,
+                                         (cudaStream_t)stream));
+}
+
+mxq_status mxq_lowrank_packed_bytes(int64_t m, size_t *bytes) {
+    if (m < 0 || !bytes) return MXQ_EINVAL;
+    *bytes = (size_t)(m * 64 * 2);
+    return MXQ_OK;
+}
+
+mxq_status mxq_lowrank_down_packed(const void *x, int32_t xdtype, int64_t m, int64_t k, const void *l1, int32_t r,
+                                   const float *x_tensor_scale, const float *w_tensor_scale, void *tp, void *stream) {
+    if (!valid_dtype(xdtype) || m < 0 || k <= 0 || k % 16 || r < 1 || r > 32) return MXQ_EINVAL;
+    if (!x_tensor_scale != !w_tensor_scale) return MXQ_EINVAL;
+    if (m > 0 && (!x || !l1 || !tp || !aligned16(x) || !aligned16(tp))) return MXQ_EINVAL;
+    return from_cuda(launch_lowrank_down(x, xdtype == MXQ_BF16, m, k, l1, r, nullptr, x_tensor_scale,
+                                         w_tensor_scale, tp, (cudaStream_t)stream));
+}
+
+mxq_status mxq_lowrank_pack_t(const float *t, int32_t r, int64_t m, const float *x_tensor_scale,
+                              const float *w_tensor_scale, void *tp, void *stream) {
+    if (r < 1 || r > 32 || m < 0 || (!x_tensor_scale != !w_tensor_scale)) return MXQ_EINVAL;
+    if (m > 0 && (!t || !tp || !aligned16(tp))) return MXQ_EINVAL;
+    return from_cuda(launch_pack_t(t, r, m, x_tensor_scale, w_tensor_scale, tp, (cudaStream_t)stream));
 }
 
 mxq_status mxq_lowrank_pack_l2(const void *l2, int32_t r, int64_t n, void *l2p, void *stream) {
@@ -177,14 +200,8 @@ mxq_status mxq_lowrank_pack_l2(const void *l2, int32_t r, int64_t n, void *l2p, 
     return from_cuda(launch_pack_l2(l2, r, n, l2p, (cudaStream_t)stream));
 }
 
-mxq_status mxq_qlinear_workspace_bytes(int64_t m, size_t *bytes) {
-    if (m < 0 || !bytes) return MXQ_EINVAL;
-    *bytes = (size_t)(m * 64 * 2);
-    return MXQ_OK;
-}
-
-mxq_status mxq_qlinear(const mxq_qtensor *xq, const mxq_qtensor *wq, const float *t, const void *l2p, int32_t r,
-                       void *y, int32_t ydtype, void *workspace, size_t workspace_bytes, void *stream) {
+mxq_status mxq_qlinear(const mxq_qtensor *xq, const mxq_qtensor *wq, const void *tp, const void *l2p, void *y,
+                       int32_t ydtype, void *stream) {
     if (!xq || !wq || !valid_dtype(ydtype) || !y) return MXQ_EINVAL;
     if (!valid_fmt(xq->fmt) || xq->fmt != wq->fmt) return MXQ_EUNSUPPORTED;
     const int fmt = xq->fmt;
@@ -200,21 +217,9 @@ mxq_status mxq_qlinear(const mxq_qtensor *xq, const mxq_qtensor *wq, const float
         if (fmt != MXQ_FP8_TENSOR && (!xq->scales || !wq->scales)) return MXQ_EINVAL;
         if (fmt_tensor_scaled(fmt) && (!xq->tensor_scale || !wq->tensor_scale)) return MXQ_EINVAL;
     }
-    if (t) {
+    if (tp) {
         if (fmt == MXQ_INT8_ROW) return MXQ_EUNSUPPORTED;
-        if (r < 1 || r > 32 || !l2p || !aligned16(l2p)) return MXQ_EINVAL;
-        size_t need = 0;
-        mxq_qlinear_workspace_bytes(m, &need);
-        if (!workspace) return MXQ_EINVAL;
-        if (workspace_bytes < need) return MXQ_ENOSPACE;
-        if (!aligned16(workspace)) return MXQ_EINVAL;
-    }
-    cudaStream_t s = (cudaStream_t)stream;
-    if (t) {
-        const bool ts = fmt_tensor_scaled(fmt);
-        cudaError_t e = launch_pack_t(t, r, m, ts ? xq->tensor_scale : nullptr, ts ? wq->tensor_scale : nullptr,
-                                      workspace, s);
-        if (e != cudaSuccess) return MXQ_ECUDA;
+        if (!l2p || !aligned16(l2p) || !aligned16(tp)) return MXQ_EINVAL;
     }
     GemmOperands op;
     op.fmt = fmt;
@@ -227,11 +232,11 @@ mxq_status mxq_qlinear(const mxq_qtensor *xq, const mxq_qtensor *wq, const float
     op.b_scales = wq->scales;
     op.a_tensor_scale = xq->tensor_scale;
     op.b_tensor_scale = wq->tensor_scale;
-    op.tp = t ? workspace : nullptr;
+    op.tp = tp;
     op.l2p = l2p;
     op.y = y;
     op.y_bf16 = ydtype == MXQ_BF16;
-    return from_cuda(launch_qlinear(op, s));
+    return from_cuda(launch_qlinear(op, (cudaStream_t)stream));
 }
 
 int32_t mxq_route(const uint8_t *table, int32_t n_layers, int32_t n_intervals, int32_t layer, int32_t step,

@@ -24,8 +24,10 @@ cudaError_t launch_cast(const float *x, int64_t n, int elem, uint8_t *out, cudaS
 cudaError_t launch_select(const void *w, bool bf16, int64_t n, int64_t k, const int *cands, int ncand,
                           uint8_t *choice, double *sse, unsigned int *amax_word, cudaStream_t s);
 
+// t (m x r fp32) when tp is null; else the packed GEMM operand tp (m x 64
+// bf16, [hi | lo] of t / (xs * ws), xs = ws = null meaning 1).
 cudaError_t launch_lowrank_down(const void *x, bool bf16, int64_t m, int64_t k, const void *l1, int r,
-                                float *t, cudaStream_t s);
+                                float *t, const float *xs, const float *ws, void *tp, cudaStream_t s);
 cudaError_t launch_pack_l2(const void *l2, int r, int64_t n, void *l2p, cudaStream_t s);
 cudaError_t launch_pack_t(const float *t, int r, int64_t m, const float *xs, const float *ws, void *tp,
                           cudaStream_t s);

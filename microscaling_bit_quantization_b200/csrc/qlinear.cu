@@ -446,10 +446,12 @@ __device__ __forceinline__ void mma_m16n8k16_bf16(float (&c)[4], const uint32_t 
 
 // t = bf16(x) . l1 (fp32 accumulate).  CTA = 4 warps over 16 rows; warp w
 // takes the k16 steps w, w+4, ...; the four partial tiles are summed in a
-// fixed order through shared memory.  HBM-bound on reading x.
-template <typename T>
+// fixed order through shared memory.  HBM-bound on reading x.  With PACKED
+// the result is written as the GEMM operand instead (see k_pack_t).
+template <typename T, bool PACKED>
 __global__ void __launch_bounds__(128) k_lowrank_down(const T *__restrict__ x, int64_t m, int64_t k,
-                                                     const __nv_bfloat16 *__restrict__ l1, int r, float *__restrict__ t) {
+                                                     const __nv_bfloat16 *__restrict__ l1, int r, float *__restrict__ t,
+                                                     const float *xs, const float *ws, __nv_bfloat16 *__restrict__ tp) {
     __shared__ float red[4][16][33];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, tq = lane & 3;
@@ -486,12 +488,20 @@ __global__ void __launch_bounds__(128) k_lowrank_down(const T *__restrict__ x, i
         red[warp][g + 8][nt * 8 + tq * 2 + 1] = acc[nt][3];
     }
     __syncthreads();
+    float alpha = 1.0f;
+    if (PACKED && xs) alpha = __fmul_rn(*xs, *ws);
     for (int i = threadIdx.x; i < 16 * 32; i += 128) {
         const int rr = i >> 5, cc = i & 31;
         const int64_t row = row0 + rr;
-        if (row < m && cc < r) {
-            float s = __fadd_rn(__fadd_rn(red[0][rr][cc], red[1][rr][cc]), __fadd_rn(red[2][rr][cc], red[3][rr][cc]));
-            t[row * r + cc] = s;
+        if (row >= m) continue;
+        float sum = __fadd_rn(__fadd_rn(red[0][rr][cc], red[1][rr][cc]), __fadd_rn(red[2][rr][cc], red[3][rr][cc]));
+        if (!PACKED) {
+            if (cc < r) t[row * r + cc] = sum;
+        } else {
+            const float u = cc < r ? (xs ? __fdiv_rn(sum, alpha) : sum) : 0.0f;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(u);
+            tp[row * 64 + cc] = hi;
+            tp[row * 64 + 32 + cc] = __float2bfloat16_rn(__fsub_rn(u, __bfloat162float(hi)));
         }
     }
 }
@@ -568,13 +578,20 @@ cudaError_t launch_kind(const GemmParams &p, dim3 grid, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_lowrank_down(const void *x, bool bf16, int64_t m, int64_t k, const void *l1, int r, float *t,
-                                cudaStream_t s) {
+                                const float *xs, const float *ws, void *tp, cudaStream_t s) {
     if (m == 0) return cudaSuccess;
     const int grid = (int)((m + 15) / 16);
-    if (bf16)
-        k_lowrank_down<__nv_bfloat16><<<grid, 128, 0, s>>>((const __nv_bfloat16 *)x, m, k, (const __nv_bfloat16 *)l1, r, t);
-    else
-        k_lowrank_down<float><<<grid, 128, 0, s>>>((const float *)x, m, k, (const __nv_bfloat16 *)l1, r, t);
+    const __nv_bfloat16 *l = (const __nv_bfloat16 *)l1;
+    __nv_bfloat16 *tpb = (__nv_bfloat16 *)tp;
+    if (bf16) {
+        const __nv_bfloat16 *xb = (const __nv_bfloat16 *)x;
+        if (tp) k_lowrank_down<__nv_bfloat16, true><<<grid, 128, 0, s>>>(xb, m, k, l, r, t, xs, ws, tpb);
+        else k_lowrank_down<__nv_bfloat16, false><<<grid, 128, 0, s>>>(xb, m, k, l, r, t, xs, ws, tpb);
+    } else {
+        const float *xf = (const float *)x;
+        if (tp) k_lowrank_down<float, true><<<grid, 128, 0, s>>>(xf, m, k, l, r, t, xs, ws, tpb);
+        else k_lowrank_down<float, false><<<grid, 128, 0, s>>>(xf, m, k, l, r, t, xs, ws, tpb);
+    }
     return cudaGetLastError();
 }
 

@@ -52,7 +52,7 @@ def test_sizes(mxq):
     assert M.scales_bytes(M.INT8_ROW, 10, 64) == 40
     assert M.scales_bytes(M.FP8_TENSOR, 10, 64) == 0
     assert M.quantize_workspace_bytes(M.NVFP4) >= 4 and M.quantize_workspace_bytes(M.MXFP8) == 0
-    assert M.qlinear_workspace_bytes(4096) == 4096 * 128
+    assert M.lowrank_packed_bytes(4096) == 4096 * 128
 
 
 def test_bad_shapes_rejected_on_host(mxq):
@@ -78,23 +78,24 @@ def test_bad_shapes_rejected_on_host(mxq):
 def test_qlinear_argument_checks(mxq):
     L = mxq.lib()
     Q = mxq._QTensorC
+    y = ctypes.c_void_p(256)
     a = Q(mxq.NVFP4, mxq.MMA, 64, 256, 256, 256, 256)
     b = Q(mxq.MXFP4, mxq.MMA, 128, 256, 256, 256, 256)
-    y = ctypes.c_void_p(256)
-    assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(b), None, None, 0, y, 0, None, 0, None) == 2   # format pair
+    assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(b), None, None, y, 0, None) == 2   # format pair
     b = Q(mxq.NVFP4, mxq.CANONICAL, 128, 256, 256, 256, 256)
-    assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(b), None, None, 0, y, 0, None, 0, None) == 1   # layout
+    assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(b), None, None, y, 0, None) == 1   # layout
     b = Q(mxq.NVFP4, mxq.MMA, 128, 192, 256, 256, 256)
-    assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(b), None, None, 0, y, 0, None, 0, None) == 1   # K mismatch
-    a = Q(mxq.INT4_G64, mxq.MMA, 64, 256, 256, 256, 0)
-    b = Q(mxq.INT4_G64, mxq.MMA, 64, 256, 256, 256, 0)
-    assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(b), None, None, 0, y, 0, None, 0, None) == 2
-    a = Q(mxq.NVFP4, mxq.MMA, 64, 256, 256, 256, 256)
-    b = Q(mxq.NVFP4, mxq.MMA, 128, 256, 256, 256, 256)
+    assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(b), None, None, y, 0, None) == 1   # K mismatch
+    i4 = Q(mxq.INT4_G64, mxq.MMA, 64, 256, 256, 256, 0)
+    assert L.mxq_qlinear(ctypes.byref(i4), ctypes.byref(i4), None, None, y, 0, None) == 2
+    a = Q(mxq.NVFP4, mxq.MMA, 64, 96, 256, 256, 256)
+    assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(a), None, None, y, 0, None) == 1   # K % 64
+    i8 = Q(mxq.INT8_ROW, mxq.MMA, 64, 256, 256, 256, 0)
     t = ctypes.c_void_p(256)
-    # low-rank branch needs workspace of m x 128 bytes
-    assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(b), t, t, 8, y, 0, t, 100, None) == 5
-    assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(b), t, t, 40, y, 0, t, 64 * 128, None) == 1
+    assert L.mxq_qlinear(ctypes.byref(i8), ctypes.byref(i8), t, t, y, 0, None) == 2       # branch on INT8
+    a = Q(mxq.NVFP4, mxq.MMA, 64, 256, 256, 256, 256)
+    assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(a), t, None, y, 0, None) == 1      # branch without l2p
+    assert L.mxq_lowrank_down_packed(t, 1, 4, 64, t, 8, t, None, t, None) == 1             # one tensor scale
 
 
 def test_route_matches_oracle(mxq, orc):

@@ -1,7 +1,7 @@
 """GPU parity of the low-rank branch and the tcgen05 block-scaled GEMM
 against the oracle's binary64 GEMM over exactly dequantized operands.
 
-Tolerance (stated by the benchmark spec for fp32 output): relative Frobenius error
+Tolerance for fp32 output: relative Frobenius error
 <= 1e-4 and max abs error <= 1e-4 * max|Y_ref|; bf16 output also allows the
 final bf16 rounding (see gpu_util.gemm_close).  Quantized operands are
 produced by the library and checked bit-exact against the oracle's in
@@ -42,11 +42,11 @@ def _inputs(seed, m, n, k, r=0):
 def _run(mxq, fmt, d, r, out_dtype, hadamard_b=0, x_dtype="bf16"):
     xq = mxq.quantize(dev(d["x"], x_dtype), fmt, hadamard_b, mxq.MMA)
     wq = mxq.quantize(dev(d["w"], "bf16"), fmt, hadamard_b, mxq.MMA)
-    t = l2p = None
+    tp = l2p = None
     if r:
-        t = mxq.lowrank_down(dev(d["x"], x_dtype), dev(d["l1"], "bf16"))
+        tp = mxq.lowrank_down_packed(dev(d["x"], x_dtype), dev(d["l1"], "bf16"), xq, wq)
         l2p = mxq.lowrank_pack_l2(dev(d["l2"], "bf16"))
-    y = mxq.qlinear(xq, wq, t, l2p, r, out_dtype=out_dtype)
+    y = mxq.qlinear(xq, wq, tp, l2p, out_dtype=out_dtype)
     assert mxq.check() == 0
     return y, xq, wq
 
@@ -115,9 +115,13 @@ def test_tiny_nvfp4_linear_full(mxq, orc):
     wq = mxq.quantize(dev(d["w"], "f32"), 2, 0, mxq.MMA)
     assert_qtensor_equal(xq, oxq, layout_mma=True)
     assert_qtensor_equal(wq, owq, layout_mma=True)
-    t = mxq.lowrank_down(dev(d["x"], "f32"), dev(d["l1"], "bf16"))
     l2p = mxq.lowrank_pack_l2(dev(d["l2"], "bf16"))
-    y = mxq.qlinear(xq, wq, t, l2p, 8, out_dtype=torch.float32)
+    # both routes to the packed branch operand: fused, and fp32 t then pack
+    tp_fused = mxq.lowrank_down_packed(dev(d["x"], "f32"), dev(d["l1"], "bf16"), xq, wq)
+    t = mxq.lowrank_down(dev(d["x"], "f32"), dev(d["l1"], "bf16"))
+    tp_split = mxq.lowrank_pack_t(t, xq, wq)
+    assert torch.equal(tp_fused.view(torch.int16), tp_split.view(torch.int16))
+    y = mxq.qlinear(xq, wq, tp_fused, l2p, out_dtype=torch.float32)
     assert mxq.check() == 0
     gemm_close(y.cpu().numpy(), ref)
 
