@@ -219,6 +219,28 @@ mxq_status mxq_lowrank_down_packed(const void *x, int32_t xdtype, int64_t m, int
 mxq_status mxq_lowrank_pack_t(const float *t, int32_t r, int64_t m, const float *x_tensor_scale,
                               const float *w_tensor_scale, void *tp, void *stream);
 
+/* Scratch bytes mxq_quantize_lowrank needs for m rows and rank r. */
+mxq_status mxq_quantize_lowrank_workspace_bytes(int64_t m, int32_t r, size_t *bytes);
+
+/* Activation side of one W4A4 + low-rank linear in one call: quantizes x
+ * (as mxq_quantize, MMA layout) and writes the packed low-rank operand tp
+ * (as mxq_lowrank_down_packed with the new tensor scale of x and
+ * w_tensor_scale).  For tensor-scaled formats without rotation the tensor
+ * amax and t = bf16(x) . l1 come from one read of x, and the encoding pass
+ * re-reads x from L2.
+ *   fmt: NVFP4, MXFP4, MXFP8 or FP8_TENSOR (the formats whose GEMM takes
+ *     the branch); w_tensor_scale: device scalar of the weight (NVFP4,
+ *     FP8_TENSOR), else ignored.
+ *   workspace: device scratch of mxq_quantize_lowrank_workspace_bytes,
+ *     256-byte aligned; clobbered.
+ * Other arguments, constraints and errors as mxq_quantize and
+ * mxq_lowrank_down. */
+mxq_status mxq_quantize_lowrank(const void *x, int32_t xdtype, int64_t m, int64_t k, int32_t fmt,
+                                int32_t hadamard_b, const void *l1, int32_t r,
+                                const float *w_tensor_scale, void *codes, void *scales,
+                                float *tensor_scale, void *tp, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
 /* Re-lays the up-projection l2 (r x n bf16, device) as the GEMM operand
  * l2p (n x 64 bf16, device): row j of l2p holds l2[0..r-1][j], zeros up to
  * 32, then the same 32 values again (the operand of the split high/low

@@ -32,7 +32,8 @@ STATUS = {0: "MXQ_OK", 1: "MXQ_EINVAL", 2: "MXQ_EUNSUPPORTED", 3: "MXQ_ECUDA", 4
 EXPORTS = ("mxq_status_string", "mxq_device_supported", "mxq_check", "mxq_codes_bytes", "mxq_scales_bytes",
            "mxq_quantize_workspace_bytes", "mxq_quantize", "mxq_dequantize", "mxq_hadamard_block", "mxq_cast",
            "mxq_select_workspace_bytes", "mxq_select_weight_format", "mxq_lowrank_down", "mxq_lowrank_packed_bytes",
-           "mxq_lowrank_down_packed", "mxq_lowrank_pack_t", "mxq_lowrank_pack_l2", "mxq_qlinear", "mxq_route")
+           "mxq_lowrank_down_packed", "mxq_lowrank_pack_t", "mxq_lowrank_pack_l2", "mxq_qlinear", "mxq_route",
+           "mxq_quantize_lowrank_workspace_bytes", "mxq_quantize_lowrank")
 
 
 class MxqError(RuntimeError):
@@ -73,6 +74,8 @@ def _load():
         "mxq_lowrank_pack_l2": (i32, [P, i32, i64, P, P]),
         "mxq_qlinear": (i32, [ctypes.POINTER(_QTensorC), ctypes.POINTER(_QTensorC), P, P, P, i32, P]),
         "mxq_route": (i32, [P, i32, i32, i32, i32, i32]),
+        "mxq_quantize_lowrank_workspace_bytes": (i32, [i64, i32, psz]),
+        "mxq_quantize_lowrank": (i32, [P, i32, i64, i64, i32, i32, P, i32, P, P, P, P, P, P, sz, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -274,6 +277,30 @@ def lowrank_pack_t(t: torch.Tensor, xq: QTensor = None, wq: QTensor = None, out:
     xs, ws = _scales_of(xq, wq)
     _ok(_lib.mxq_lowrank_pack_t(_ptr(t), r, m, xs, ws, _ptr(tp), _stream(stream)), "mxq_lowrank_pack_t")
     return tp
+
+
+def quantize_lowrank_workspace_bytes(m: int, r: int) -> int:
+    return _size(_lib.mxq_quantize_lowrank_workspace_bytes, m, r)
+
+
+def quantize_lowrank(x: torch.Tensor, fmt: int, l1: torch.Tensor, wq: QTensor, hadamard_b: int = 0,
+                     out: QTensor = None, tp: torch.Tensor = None, workspace: torch.Tensor = None, stream=None):
+    """Quantized activation (MMA layout) and packed low-rank operand in one call; returns (xq, tp)."""
+    _require_cuda(x, l1)
+    x, l1 = x.contiguous(), l1.contiguous()
+    m, k = x.shape
+    r = l1.shape[1]
+    q = out if out is not None else alloc_qtensor(fmt, m, k, MMA, x.device)
+    if tp is None:
+        tp = torch.empty((m, 64), dtype=torch.bfloat16, device=x.device)
+    wsb = quantize_lowrank_workspace_bytes(m, r)
+    if workspace is None:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=x.device)
+    _ok(_lib.mxq_quantize_lowrank(_ptr(x), _dtype_code(x), m, k, fmt, hadamard_b, _ptr(l1), r,
+                                  _ptr(wq.tensor_scale) if wq is not None else None, _ptr(q.codes), _ptr(q.scales),
+                                  _ptr(q.tensor_scale), _ptr(tp), _ptr(workspace), wsb, _stream(stream)),
+        "mxq_quantize_lowrank")
+    return q, tp
 
 
 def qlinear(xq: QTensor, wq: QTensor, tp: torch.Tensor = None, l2p: torch.Tensor = None,

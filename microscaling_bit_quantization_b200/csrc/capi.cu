@@ -194,6 +194,51 @@ mxq_status mxq_lowrank_pack_t(const float *t, int32_t r, int64_t m, const float 
     return from_cuda(launch_pack_t(t, r, m, x_tensor_scale, w_tensor_scale, tp, (cudaStream_t)stream));
 }
 
+mxq_status mxq_quantize_lowrank_workspace_bytes(int64_t m, int32_t r, size_t *bytes) {
+    if (m < 0 || r < 1 || r > 32 || !bytes) return MXQ_EINVAL;
+    *bytes = 256 + (size_t)(m * r * 4);
+    return MXQ_OK;
+}
+
+mxq_status mxq_quantize_lowrank(const void *x, int32_t xdtype, int64_t m, int64_t k, int32_t fmt, int32_t hadamard_b,
+                                const void *l1, int32_t r, const float *w_tensor_scale, void *codes, void *scales,
+                                float *tensor_scale, void *tp, void *workspace, size_t workspace_bytes,
+                                void *stream) {
+    if (!valid_fmt(fmt) || !valid_dtype(xdtype) || !valid_shape(fmt, m, k) || !valid_hadamard(hadamard_b, k))
+        return MXQ_EINVAL;
+    if (fmt != MXQ_NVFP4 && fmt != MXQ_MXFP4 && fmt != MXQ_MXFP8 && fmt != MXQ_FP8_TENSOR) return MXQ_EUNSUPPORTED;
+    if (k <= 0 || r < 1 || r > 32) return MXQ_EINVAL;
+    const bool ts = fmt_tensor_scaled(fmt);
+    if (ts && (!tensor_scale || !w_tensor_scale)) return MXQ_EINVAL;
+    if (m > 0 && (!x || !codes || !tp || !l1 || !aligned16(x) || !aligned16(codes) || !aligned16(tp)))
+        return MXQ_EINVAL;
+    if (m > 0 && fmt != MXQ_FP8_TENSOR && !scales) return MXQ_EINVAL;
+    size_t need = 0, sb = 0;
+    mxq_quantize_lowrank_workspace_bytes(m, r, &need);
+    if (!workspace) return MXQ_EINVAL;
+    if (workspace_bytes < need) return MXQ_ENOSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MXQ_EINVAL;
+    mxq_scales_bytes(fmt, m, k, MXQ_LAYOUT_MMA, &sb);
+    cudaStream_t s = (cudaStream_t)stream;
+    unsigned int *amax = (unsigned int *)workspace;
+    float *t = (float *)((char *)workspace + 256);
+    const bool bf = xdtype == MXQ_BF16;
+    cudaError_t e = cudaSuccess;
+    bool amax_ready = false;
+    if (ts && hadamard_b == 0) {
+        // one read of x from HBM gives both the tensor amax and t
+        e = cudaMemsetAsync(amax, 0, sizeof(unsigned int), s);
+        if (e == cudaSuccess) e = launch_lowrank_down(x, bf, m, k, l1, r, t, nullptr, nullptr, nullptr, s, amax);
+        amax_ready = true;
+    } else {
+        e = launch_lowrank_down(x, bf, m, k, l1, r, t, nullptr, nullptr, nullptr, s);
+    }
+    if (e != cudaSuccess) return MXQ_ECUDA;
+    PackT pack{t, r, w_tensor_scale, tp};
+    return from_cuda(launch_quantize(x, bf, m, k, fmt, hadamard_b, MXQ_LAYOUT_MMA, codes, scales, sb, tensor_scale,
+                                     amax, s, &pack, amax_ready));
+}
+
 mxq_status mxq_lowrank_pack_l2(const void *l2, int32_t r, int64_t n, void *l2p, void *stream) {
     if (r < 1 || r > 32 || n < 0) return MXQ_EINVAL;
     if (n > 0 && (!l2 || !l2p || !aligned16(l2p))) return MXQ_EINVAL;

@@ -12,9 +12,20 @@ constexpr int kMaxCandidates = 8;
 
 cudaError_t launch_amax(const void *x, bool bf16, int64_t rows, int64_t cols, int hadamard_b,
                         unsigned int *amax_word, cudaStream_t s);
+// Optional duty of the quantizer: pack the low-rank activation t (rows x r
+// fp32) into tp (rows x 64 bf16) divided by s_x * *w_ts (tensor-scaled
+// formats) or by 1.
+struct PackT {
+    const float *t;
+    int r;
+    const float *w_ts;
+    void *tp;
+};
+// amax_ready: the tensor amax is already in *amax_word (skip the amax pass).
 cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols, int fmt, int hadamard_b,
                             int layout, void *codes, void *scales, size_t scales_bytes, float *tensor_scale,
-                            unsigned int *amax_word, cudaStream_t s);
+                            unsigned int *amax_word, cudaStream_t s, const PackT *pack = nullptr,
+                            bool amax_ready = false);
 cudaError_t launch_dequantize(int fmt, int layout, int64_t rows, int64_t cols, const void *codes,
                               const void *scales, const float *tensor_scale, void *y, bool bf16_out,
                               cudaStream_t s);
@@ -25,9 +36,12 @@ cudaError_t launch_select(const void *w, bool bf16, int64_t n, int64_t k, const 
                           uint8_t *choice, double *sse, unsigned int *amax_word, cudaStream_t s);
 
 // t (m x r fp32) when tp is null; else the packed GEMM operand tp (m x 64
-// bf16, [hi | lo] of t / (xs * ws), xs = ws = null meaning 1).
+// bf16, [hi | lo] of t / (xs * ws), xs = ws = null meaning 1).  With
+// amax_word (and tp null) the max |x| of the whole tensor is also
+// atomically folded into *amax_word (which must be zeroed beforehand).
 cudaError_t launch_lowrank_down(const void *x, bool bf16, int64_t m, int64_t k, const void *l1, int r,
-                                float *t, const float *xs, const float *ws, void *tp, cudaStream_t s);
+                                float *t, const float *xs, const float *ws, void *tp, cudaStream_t s,
+                                unsigned int *amax_word = nullptr);
 cudaError_t launch_pack_l2(const void *l2, int r, int64_t n, void *l2p, cudaStream_t s);
 cudaError_t launch_pack_t(const float *t, int r, int64_t m, const float *xs, const float *ws, void *tp,
                           cudaStream_t s);

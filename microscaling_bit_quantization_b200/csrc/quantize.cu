@@ -30,6 +30,31 @@ inline int grid_for(int64_t warp_tiles, int sm_count) {
 
 // ------------------------------------------------------------------ amax
 
+// Max over the CTA, then one atomicMax on the word (non-negative floats
+// order like their bit patterns).  All threads of the CTA must call this.
+__device__ __forceinline__ void cta_max_to_word(float m, unsigned int *word) {
+    __shared__ float wmax[kThreads / 32];
+    m = group_max<32>(m);
+    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float v = threadIdx.x < kThreads / 32 ? wmax[threadIdx.x] : 0.0f;
+        v = group_max<32>(v);
+        if (threadIdx.x == 0 && v > 0.0f) atomicMax(word, __float_as_uint(v));
+    }
+}
+
+// Bytes of four consecutive scale columns s..s+3 (held by lanes lane,
+// lane+L, lane+2L, lane+3L) as one little-endian word, for the lane whose
+// scale column is a multiple of 4.  All lanes must call this.
+template <int L>
+__device__ __forceinline__ uint32_t gather4(uint32_t byte) {
+    uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, byte, L);
+    uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, byte, 2 * L);
+    uint32_t b3 = __shfl_down_sync(0xFFFFFFFFu, byte, 3 * L);
+    return (byte & 0xFFu) | ((b1 & 0xFFu) << 8) | ((b2 & 0xFFu) << 16) | ((b3 & 0xFFu) << 24);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) k_amax(const T *__restrict__ x, int64_t total_chunks,
                                                   int hadamard_b, unsigned int *__restrict__ amax_word) {
@@ -49,9 +74,7 @@ __global__ void __launch_bounds__(kThreads) k_amax(const T *__restrict__ x, int6
         if (hadamard_b) hadamard_chunk(v, hadamard_b, lane);
         m = fmaxf(m, amax16(v));
     }
-    m = group_max<32>(m);
-    // non-negative floats order like their bit patterns
-    if (lane == 0 && m > 0.0f) atomicMax(amax_word, __float_as_uint(m));
+    cta_max_to_word(m, amax_word);
 }
 
 // ------------------------------------------------------------------ quantize
@@ -65,7 +88,38 @@ struct QuantArgs {
     void *scales;
     float *tensor_scale;     // written by chunk 0 (NVFP4, FP8_TENSOR)
     const unsigned int *amax_word;
+    int combine;             // scale bytes stored as 32-bit words (scale columns per row % 4 == 0)
+    // optional packed low-rank operand: tp[row] = [hi | lo] of t[row] / (s_x * *w_ts)
+    const float *t;
+    int r;
+    const float *w_ts;
+    __nv_bfloat16 *tp;
 };
+
+// Packs one row of the low-rank activation: u_j = t_j / alpha (alpha = 1
+// when `divide` is false), hi = bf16(u), lo = bf16(u - hi), zeros past r.
+__device__ __forceinline__ void pack_t_row(const float *t, int r, bool divide, float alpha, __nv_bfloat16 *tp) {
+    uint32_t hi[16], lo[16];
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+        float u0 = j < r ? t[j] : 0.0f, u1 = j + 1 < r ? t[j + 1] : 0.0f;
+        if (divide) {
+            u0 = __fdiv_rn(u0, alpha);
+            u1 = __fdiv_rn(u1, alpha);
+        }
+        __nv_bfloat162 h = __floats2bfloat162_rn(u0, u1);
+        float2 hf = __bfloat1622float2(h);
+        __nv_bfloat162 l = __floats2bfloat162_rn(__fsub_rn(u0, hf.x), __fsub_rn(u1, hf.y));
+        hi[j >> 1] = *reinterpret_cast<uint32_t *>(&h);
+        lo[j >> 1] = *reinterpret_cast<uint32_t *>(&l);
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(tp);
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        dst[i] = make_uint4(hi[4 * i], hi[4 * i + 1], hi[4 * i + 2], hi[4 * i + 3]);
+        dst[4 + i] = make_uint4(lo[4 * i], lo[4 * i + 1], lo[4 * i + 2], lo[4 * i + 3]);
+    }
+}
 
 template <typename T, int F>
 __global__ void __launch_bounds__(kThreads) k_quantize(const T *__restrict__ x, QuantArgs a) {
@@ -98,6 +152,10 @@ __global__ void __launch_bounds__(kThreads) k_quantize(const T *__restrict__ x, 
         const int64_t col0 = (c - row * chunks_per_row) << 4;
         float amax = amax16(v);
         if (G > 1) amax = group_max<G>(amax);
+        if (a.tp && valid && col0 == 0) {
+            const bool ts = F == kNVFP4 || F == kFP8Tensor;
+            pack_t_row(a.t + row * a.r, a.r, ts, ts ? __fmul_rn(s_t, *a.w_ts) : 1.0f, a.tp + row * 64);
+        }
 
         if (F == kMXFP8 || F == kMXFP4) {
             float inv = 0.0f;
@@ -134,11 +192,16 @@ __global__ void __launch_bounds__(kThreads) k_quantize(const T *__restrict__ x, 
                     }
                     *reinterpret_cast<uint2 *>(a.codes + c * 8) = make_uint2(w[0], w[1]);
                 }
-                if ((lane & 1) == 0) {
-                    int64_t s = col0 >> 5;
-                    uint8_t *sc = reinterpret_cast<uint8_t *>(a.scales);
-                    if (a.layout == 0) sc[row * (a.cols >> 5) + s] = (uint8_t)sb;
-                    else sc[mma_scale_offset(row, s, a.s_pad)] = (uint8_t)sb;
+            }
+            const uint32_t word = gather4<2>(sb);
+            if (valid) {
+                const int64_t s = col0 >> 5;
+                uint8_t *sc = reinterpret_cast<uint8_t *>(a.scales);
+                const int64_t off = a.layout == 0 ? row * (a.cols >> 5) + s : mma_scale_offset(row, s, a.s_pad);
+                if (a.combine) {
+                    if ((lane & 7) == 0) *reinterpret_cast<uint32_t *>(sc + off) = word;
+                } else if ((lane & 1) == 0) {
+                    sc[off] = (uint8_t)sb;
                 }
             }
         } else if (F == kNVFP4) {
@@ -159,10 +222,17 @@ __global__ void __launch_bounds__(kThreads) k_quantize(const T *__restrict__ x, 
                     w[j] = acc;
                 }
                 *reinterpret_cast<uint2 *>(a.codes + c * 8) = make_uint2(w[0], w[1]);
-                int64_t s = col0 >> 4;
+            }
+            const uint32_t word = gather4<1>(e4);
+            if (valid) {
+                const int64_t s = col0 >> 4;
                 uint8_t *sc = reinterpret_cast<uint8_t *>(a.scales);
-                if (a.layout == 0) sc[c] = (uint8_t)e4;
-                else sc[mma_scale_offset(row, s, a.s_pad)] = (uint8_t)e4;
+                const int64_t off = a.layout == 0 ? c : mma_scale_offset(row, s, a.s_pad);
+                if (a.combine) {
+                    if ((lane & 3) == 0) *reinterpret_cast<uint32_t *>(sc + off) = word;
+                } else {
+                    sc[off] = (uint8_t)e4;
+                }
             }
         } else if (F == kINT4G32 || F == kINT4G64) {
             float s = __fdiv_rn(amax, 7.0f);
@@ -548,9 +618,9 @@ static void launch_q(int fmt, int grid, const T *x, const QuantArgs &a, cudaStre
 
 cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols, int fmt, int hadamard_b,
                             int layout, void *codes, void *scales, size_t scales_bytes, float *tensor_scale,
-                            unsigned int *amax_word, cudaStream_t s) {
+                            unsigned int *amax_word, cudaStream_t s, const PackT *pack, bool amax_ready) {
     cudaError_t e;
-    if (fmt_tensor_scaled(fmt)) {
+    if (fmt_tensor_scaled(fmt) && !amax_ready) {
         e = launch_amax(x, bf16, rows, cols, hadamard_b, amax_word, s);
         if (e != cudaSuccess) return e;
     }
@@ -565,6 +635,11 @@ cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols
     a.scales = scales;
     a.tensor_scale = tensor_scale;
     a.amax_word = amax_word;
+    a.combine = fmt_byte_scales(fmt) && (cols / fmt_block(fmt)) % 4 == 0;
+    a.t = pack ? pack->t : nullptr;
+    a.r = pack ? pack->r : 0;
+    a.w_ts = pack ? pack->w_ts : nullptr;
+    a.tp = pack ? (__nv_bfloat16 *)pack->tp : nullptr;
     if (layout == 1 && fmt_byte_scales(fmt)) {
         int64_t S = cols / fmt_block(fmt);
         a.s_pad = (S + 15) / 16 * 16;

@@ -169,3 +169,37 @@ def test_dit_layers_full_size(mxq, orc, fmt):
         ref, _, _ = _ref(orc, fmt, d, 0, rows=rows)
         y, _, _ = _run(mxq, fmt, d, 0, torch.float32)
         gemm_close(y[torch.from_numpy(rows).cuda()].cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("fmt", LOWRANK_FMTS)
+@pytest.mark.parametrize("hadamard_b", [0, 64])
+@pytest.mark.parametrize("x_dtype", ["bf16", "f32"])
+def test_quantize_lowrank_fused(mxq, orc, fmt, hadamard_b, x_dtype):
+    """The fused activation path equals quantize + lowrank_down_packed bit for
+    bit, and its codes/scales equal the oracle's."""
+    d = _inputs(40 + fmt, 77, 300, 512, 24)
+    x = dev(d["x"], x_dtype)
+    wq = mxq.quantize(dev(d["w"], "bf16"), fmt, hadamard_b, mxq.MMA)
+    l1 = dev(d["l1"], "bf16")
+    xq, tp = mxq.quantize_lowrank(x, fmt, l1, wq, hadamard_b)
+    xq2 = mxq.quantize(x, fmt, hadamard_b, mxq.MMA)
+    tp2 = mxq.lowrank_down_packed(x, l1, xq2, wq)
+    torch.cuda.synchronize()
+    assert torch.equal(xq.codes, xq2.codes)
+    if xq.scales is not None:
+        assert torch.equal(xq.scales, xq2.scales)
+    assert torch.equal(tp.view(torch.int16), tp2.view(torch.int16))
+    assert_qtensor_equal(xq, orc.quantize(host_values(d["x"], x_dtype), fmt, hadamard_b), layout_mma=True)
+
+
+def test_svdquant_fused_path_full_size(mxq, orc):
+    """Workload 3 through the fused activation path, as the benchmark runs it."""
+    d = workloads.svdquant_mlp_up()
+    rows = _sample_rows(4096, 33)
+    ref, _, _ = _ref(orc, 2, d, 32, rows=rows)
+    wq = mxq.quantize(dev(d["w"], "bf16"), 2, 0, mxq.MMA)
+    xq, tp = mxq.quantize_lowrank(dev(d["x"], "bf16"), 2, dev(d["l1"], "bf16"), wq)
+    l2p = mxq.lowrank_pack_l2(dev(d["l2"], "bf16"))
+    y = mxq.qlinear(xq, wq, tp, l2p, out_dtype=torch.bfloat16)
+    assert mxq.check() == 0
+    gemm_close(y[torch.from_numpy(rows).cuda()].float().cpu().numpy(), ref, bf16_out=True)
