@@ -45,10 +45,13 @@ constexpr int A_STAGE = BM * BKB;                          // 16 KB
 constexpr int B_STAGE = BN * BKB;                          // 32 KB
 constexpr int SF_STAGE = 6144;                             // SFA 2 KB + SFB 2 x 2 KB
 constexpr int STAGE_BYTES = A_STAGE + B_STAGE + SF_STAGE;  // 54 KB (multiple of 1 KB)
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;   // ring + barriers + alignment slack
 constexpr int kGemmThreads = 192;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TMEM_SFA = 256, TMEM_SFB = 272;
+// TMEM columns: accumulator stage 0 at [0, 256), stage 1 at [192, 448)
+// (the stages share 64 columns), scale factors at [448, 512).
+constexpr uint32_t ACC_STAGE1 = 192, OVL_COLS = 64;
+constexpr uint32_t TMEM_SFA = 448, TMEM_SFB = 464;
 
 enum Kind : int { kKindNVFP4 = 0, kKindMXFP4 = 1, kKindMXFP8 = 2, kKindFP8 = 3, kKindINT8 = 4 };
 
@@ -60,7 +63,7 @@ struct GemmParams {
     const float *a_row_scale, *b_row_scale;
     const float *a_ts, *b_ts;
     void *y;
-    int m, n, kbytes, num_k_tiles, s4, has_lowrank, y_bf16;
+    int m, n, kbytes, num_k_tiles, s4, has_lowrank, y_bf16, m_tiles, n_tiles;
     unsigned long long wait_ns;
 };
 
@@ -212,27 +215,61 @@ __device__ __forceinline__ void latch_error(unsigned int code) { atomicOr(&g_err
 
 // ------------------------------------------------------------------ GEMM
 
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Epilogue value of accumulator column j of a chunk: alpha * acc (fp32
+// accumulators) or acc * sa * sb[n] (s32 accumulators of INT8_ROW).
+template <int KIND>
+__device__ __forceinline__ void scale_chunk(const uint32_t (&r)[32], float (&v)[32], float alpha, float ra,
+                                            const float *sbn, int nvalid) {
+    if (KIND == kKindINT8) {
+#pragma unroll
+        for (int j = 0; j < 32; j++) {
+            const float sb = j < nvalid ? __ldg(sbn + j) : 0.0f;
+            v[j] = __fmul_rn(__fmul_rn((float)(int)r[j], ra), sb);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; j++) v[j] = __fmul_rn(__uint_as_float(r[j]), alpha);
+    }
+}
+
+// Persistent GEMM: gridDim.x CTAs (one per SM) walk the output tiles
+// blockIdx.x, blockIdx.x + gridDim.x, ...  The TMA ring runs continuously
+// across tiles, so the next tile's operands stream in while the current
+// tile finishes.  Tiles alternate between two TMEM accumulator stages that
+// share 64 columns (512 columns hold two 256-column stages only that way,
+// beside the scale factors); the epilogue drains the shared columns first,
+// so the next tile's MMAs wait only for those, not for the whole epilogue.
 template <int KIND>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant__ GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
     uint64_t *empty = full + STAGES;
-    uint64_t *accf = empty + STAGES;
-    uint64_t *drain = accf + 1;
+    uint64_t *accf = empty + STAGES;      // [2] accumulator stage full
+    uint64_t *acce = accf + 2;            // [2] accumulator stage drained
+    uint64_t *ovlf = acce + 2;            // shared 64 columns drained
+    uint64_t *drain = ovlf + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
     constexpr int NSF = sf_atoms<KIND>();
+    const int num_tiles = p.m_tiles * p.n_tiles;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; s++) {
             mbar_init(full + s, 1);
             mbar_init(empty + s, 1);
         }
-        mbar_init(accf, 1);
+        for (int i = 0; i < 2; i++) {
+            mbar_init(accf + i, 1);
+            mbar_init(acce + i, 4);   // one arrival per epilogue warp
+        }
+        mbar_init(ovlf, 4);
         mbar_init(drain, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -252,165 +289,190 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm(const __grid_constant_
     if (warp == 0) {
         // ---------------------------------------------------------- producer
         if (lane == 0) {
-            int issued = 0;
-            for (int it = 0; it < nsteps; it++) {
-                const int s = it % STAGES;
-                const uint32_t ph = (it / STAGES) & 1;
-                if (!mbar_wait(empty + s, ph ^ 1, p.wait_ns)) {
-                    latch_error(kErrTimeoutProducer);
-                    *abort_flag = 1;
-                    break;
-                }
-                if (*abort_flag) break;
-                uint8_t *sa = smem + s * STAGE_BYTES;
-                uint8_t *sb = sa + A_STAGE;
-                uint8_t *sf = sb + B_STAGE;
-                if (it < p.num_k_tiles) {
-                    uint32_t bytes = A_STAGE + B_STAGE;
-                    const int rt_a = m0 >> 7;
-                    const bool b_hi = (n0 + 128) < p.n;
-                    if (NSF) bytes += NSF * 512 * (b_hi ? 3 : 2);
-                    mbar_arrive_expect_tx(full + s, bytes);
-                    tma_load_2d(&p.tma_a, sa, full + s, it * BKB, m0);
-                    tma_load_2d(&p.tma_b, sb, full + s, it * BKB, n0);
-                    if (NSF) {
-                        bulk_load(sf, p.sfa + ((int64_t)rt_a * p.s4 + it * NSF) * 512, NSF * 512, full + s);
-                        const int rt_b = n0 >> 7;
-                        bulk_load(sf + 2048, p.sfb + ((int64_t)rt_b * p.s4 + it * NSF) * 512, NSF * 512, full + s);
-                        if (b_hi)
-                            bulk_load(sf + 4096, p.sfb + ((int64_t)(rt_b + 1) * p.s4 + it * NSF) * 512, NSF * 512,
-                                      full + s);
+            int it = 0, issued = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
+                const int m0 = (tile / p.n_tiles) * BM, n0 = (tile % p.n_tiles) * BN;
+                const int rt_a = m0 >> 7, rt_b = n0 >> 7;
+                const bool b_hi = (n0 + 128) < p.n;
+                for (int kt = 0; kt < nsteps; kt++, it++) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!mbar_wait(empty + s, ph ^ 1, p.wait_ns)) {
+                        latch_error(kErrTimeoutProducer);
+                        *abort_flag = 1;
+                        break;
                     }
-                } else {
-                    mbar_arrive_expect_tx(full + s, A_STAGE + B_STAGE);
-                    tma_load_2d(&p.tma_t, sa, full + s, 0, m0);
-                    tma_load_2d(&p.tma_l2, sb, full + s, 0, n0);
+                    if (*abort_flag) break;
+                    uint8_t *sa = smem + s * STAGE_BYTES;
+                    uint8_t *sb = sa + A_STAGE;
+                    uint8_t *sf = sb + B_STAGE;
+                    if (kt < p.num_k_tiles) {
+                        uint32_t bytes = A_STAGE + B_STAGE;
+                        if (NSF) bytes += NSF * 512 * (b_hi ? 3 : 2);
+                        mbar_arrive_expect_tx(full + s, bytes);
+                        tma_load_2d(&p.tma_a, sa, full + s, kt * BKB, m0);
+                        tma_load_2d(&p.tma_b, sb, full + s, kt * BKB, n0);
+                        if (NSF) {
+                            bulk_load(sf, p.sfa + ((int64_t)rt_a * p.s4 + kt * NSF) * 512, NSF * 512, full + s);
+                            bulk_load(sf + 2048, p.sfb + ((int64_t)rt_b * p.s4 + kt * NSF) * 512, NSF * 512, full + s);
+                            if (b_hi)
+                                bulk_load(sf + 4096, p.sfb + ((int64_t)(rt_b + 1) * p.s4 + kt * NSF) * 512, NSF * 512,
+                                          full + s);
+                        }
+                    } else {
+                        mbar_arrive_expect_tx(full + s, A_STAGE + B_STAGE);
+                        tma_load_2d(&p.tma_t, sa, full + s, 0, m0);
+                        tma_load_2d(&p.tma_l2, sb, full + s, 0, n0);
+                    }
+                    issued = it + 1;
                 }
-                issued = it + 1;
             }
             if (*abort_flag) {
-                // drain: wait (bounded) for every load this thread issued
-                for (int it = (issued > STAGES ? issued - STAGES : 0); it < issued; it++)
-                    mbar_wait(full + (it % STAGES), (it / STAGES) & 1, p.wait_ns);
+                // drain: wait (bounded) for the loads this thread may still have in flight
+                for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; i++)
+                    mbar_wait(full + (i % STAGES), (i / STAGES) & 1, p.wait_ns);
             }
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            const uint32_t acc_addr = tmem;
             const uint32_t sfa_addr = tmem + TMEM_SFA, sfb_addr = tmem + TMEM_SFB;
-            const bool b_hi = (n0 + 128) < p.n;
             bool issued_any = false;
-            for (int it = 0; it < nsteps; it++) {
-                const int s = it % STAGES;
-                const uint32_t ph = (it / STAGES) & 1;
-                if (!mbar_wait(full + s, ph, p.wait_ns)) {
+            int it = 0, tcount = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x, tcount++) {
+                const int n0 = (tile % p.n_tiles) * BN;
+                const bool b_hi = (n0 + 128) < p.n;
+                const int st = tcount & 1;
+                const uint32_t acc_addr = tmem + (st ? ACC_STAGE1 : 0u);
+                // this stage drained by tile tcount-2, shared columns by tile tcount-1
+                bool ok = mbar_wait(acce + st, ((tcount >> 1) & 1) ^ 1, p.wait_ns);
+                if (ok && tcount > 0) ok = mbar_wait(ovlf, (tcount - 1) & 1, p.wait_ns);
+                if (!ok) {
                     latch_error(kErrTimeoutMma);
                     *abort_flag = 1;
                     break;
                 }
-                if (*abort_flag) break;
                 tc_fence_after();
-                uint8_t *sa = smem + s * STAGE_BYTES;
-                uint8_t *sb = sa + A_STAGE;
-                uint8_t *sf = sb + B_STAGE;
-                if (it < p.num_k_tiles) {
-                    const int rem = (p.kbytes - it * BKB) >> 5;
-                    const int nks = rem < 4 ? rem : 4;
-                    if (NSF) {
-#pragma unroll
-                        for (int i = 0; i < NSF; i++) {
-                            tc_cp_32x128b_warpx4(sfa_addr + 4 * i, sdesc_sf(sf + 512 * i));
-                            tc_cp_32x128b_warpx4(sfb_addr + 8 * i, sdesc_sf(sf + 2048 + 512 * i));
-                            if (b_hi) tc_cp_32x128b_warpx4(sfb_addr + 8 * i + 4, sdesc_sf(sf + 4096 + 512 * i));
-                        }
+                for (int kt = 0; kt < nsteps; kt++, it++) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!mbar_wait(full + s, ph, p.wait_ns)) {
+                        latch_error(kErrTimeoutMma);
+                        *abort_flag = 1;
+                        break;
                     }
-                    for (int ks = 0; ks < nks; ks++) {
-                        const uint64_t ad = sdesc_sw128(sa + ks * 32), bd = sdesc_sw128(sb + ks * 32);
-                        const uint32_t accum = (it > 0 || ks > 0) ? 1u : 0u;
-                        if (KIND == kKindNVFP4) {
-                            mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>(), accum, sfa_addr + 4 * ks,
-                                                   sfb_addr + 8 * ks);
-                        } else if (KIND == kKindMXFP4) {
-                            const uint32_t id = (uint32_t)((ks & 1) * 2);
-                            mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>() | (id << 29) | (id << 4), accum,
-                                                   sfa_addr + 4 * (ks >> 1), sfb_addr + 8 * (ks >> 1));
-                        } else if (KIND == kKindMXFP8) {
-                            const uint32_t id = (uint32_t)ks;
-                            mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>() | (id << 29) | (id << 4), accum,
-                                                   sfa_addr, sfb_addr);
-                        } else {
-                            mma_plain<KIND>(acc_addr, ad, bd, idesc_main<KIND>(), accum);
-                        }
-                    }
-                } else {
+                    if (*abort_flag) break;
+                    tc_fence_after();
+                    uint8_t *sa = smem + s * STAGE_BYTES;
+                    uint8_t *sb = sa + A_STAGE;
+                    uint8_t *sf = sb + B_STAGE;
+                    if (kt < p.num_k_tiles) {
+                        const int rem = (p.kbytes - kt * BKB) >> 5;
+                        const int nks = rem < 4 ? rem : 4;
+                        if (NSF) {
 #pragma unroll
-                    for (int ks = 0; ks < 4; ks++)
-                        mma_bf16(acc_addr, sdesc_sw128(sa + ks * 32), sdesc_sw128(sb + ks * 32), idesc_bf16(), 1u);
+                            for (int i = 0; i < NSF; i++) {
+                                tc_cp_32x128b_warpx4(sfa_addr + 4 * i, sdesc_sf(sf + 512 * i));
+                                tc_cp_32x128b_warpx4(sfb_addr + 8 * i, sdesc_sf(sf + 2048 + 512 * i));
+                                if (b_hi) tc_cp_32x128b_warpx4(sfb_addr + 8 * i + 4, sdesc_sf(sf + 4096 + 512 * i));
+                            }
+                        }
+                        for (int ks = 0; ks < nks; ks++) {
+                            const uint64_t ad = sdesc_sw128(sa + ks * 32), bd = sdesc_sw128(sb + ks * 32);
+                            const uint32_t accum = (kt > 0 || ks > 0) ? 1u : 0u;
+                            if (KIND == kKindNVFP4) {
+                                mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>(), accum, sfa_addr + 4 * ks,
+                                                       sfb_addr + 8 * ks);
+                            } else if (KIND == kKindMXFP4) {
+                                const uint32_t id = (uint32_t)((ks & 1) * 2);
+                                mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>() | (id << 29) | (id << 4),
+                                                       accum, sfa_addr + 4 * (ks >> 1), sfb_addr + 8 * (ks >> 1));
+                            } else if (KIND == kKindMXFP8) {
+                                const uint32_t id = (uint32_t)ks;
+                                mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>() | (id << 29) | (id << 4),
+                                                       accum, sfa_addr, sfb_addr);
+                            } else {
+                                mma_plain<KIND>(acc_addr, ad, bd, idesc_main<KIND>(), accum);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int ks = 0; ks < 4; ks++)
+                            mma_bf16(acc_addr, sdesc_sw128(sa + ks * 32), sdesc_sw128(sb + ks * 32), idesc_bf16(), 1u);
+                    }
+                    issued_any = true;
+                    tc_commit(empty + s);
                 }
-                issued_any = true;
-                tc_commit(empty + s);
+                if (*abort_flag) break;
+                tc_commit(accf + st);
             }
-            if (!*abort_flag) {
-                tc_commit(accf);
-            } else if (issued_any) {
+            if (*abort_flag && issued_any) {
                 tc_commit(drain);
                 mbar_wait(drain, 0, p.wait_ns);
             }
         }
     } else {
         // ---------------------------------------------------------- epilogue
-        const int q = warp & 3;                 // TMEM lane quarter this warp may access
-        const int row = m0 + q * 32 + lane;
-        bool ok = mbar_wait(accf, 0, p.wait_ns);
-        if (!ok) {
-            latch_error(kErrTimeoutEpilogue);
-            *abort_flag = 1;
-        }
-        __syncwarp();
-        ok = __all_sync(0xFFFFFFFFu, ok);
-        if (ok) {
+        const int q = warp & 3;   // TMEM lane quarter this warp may access
+        const bool vec = p.y_bf16 ? (p.n % 8 == 0) : (p.n % 4 == 0);
+        int tcount = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, tcount++) {
+            const int m0 = (tile / p.n_tiles) * BM, n0 = (tile % p.n_tiles) * BN;
+            const int row = m0 + q * 32 + lane;
+            const int st = tcount & 1;
+            bool ok = !*abort_flag && mbar_wait(accf + st, (tcount >> 1) & 1, p.wait_ns);
+            ok = __all_sync(0xFFFFFFFFu, ok);
+            if (!ok) {
+                if (lane == 0 && !*abort_flag) latch_error(kErrTimeoutEpilogue);
+                *abort_flag = 1;
+                break;
+            }
             tc_fence_after();
+            const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + (st ? ACC_STAGE1 : 0u);
             float alpha = 1.0f, ra = 0.0f;
-            if (KIND == kKindNVFP4 || KIND == kKindFP8) alpha = __fmul_rn(*p.a_ts, *p.b_ts);
-            if (KIND == kKindINT8 && row < p.m) ra = p.a_row_scale[row];
-            const bool vec = p.y_bf16 ? (p.n % 8 == 0) : (p.n % 4 == 0);
-            for (int c = 0; c < BN / 32; c++) {
+            if (KIND == kKindNVFP4 || KIND == kKindFP8) alpha = __fmul_rn(__ldg(p.a_ts), __ldg(p.b_ts));
+            const bool row_ok = row < p.m;
+            if (KIND == kKindINT8 && row_ok) ra = __ldg(p.a_row_scale + row);
+            // the 64 shared columns first: the last two chunks of stage 0, the first two of stage 1
+#pragma unroll 1
+            for (int i = 0; i < BN / 32; i++) {
+                const int c = st ? i : (i + 6) & 7;
                 uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), r);
-                const int nb = n0 + c * 32;
-                if (row >= p.m || nb >= p.n) continue;
-                float v[32];
-                if (KIND == kKindINT8) {
-#pragma unroll
-                    for (int j = 0; j < 32; j++) {
-                        const float sb = (nb + j < p.n) ? p.b_row_scale[nb + j] : 0.0f;
-                        v[j] = __fmul_rn(__fmul_rn((float)(int)r[j], ra), sb);
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 32; j++) v[j] = __fmul_rn(__uint_as_float(r[j]), alpha);
+                tmem_ld_32x32b_x32(lane_base + (uint32_t)(c * 32), r);
+                if (i == 1 || i == 7) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(i == 1 ? ovlf : acce + st);
                 }
-                const int64_t off = (int64_t)row * p.n + nb;
-                if (vec && nb + 32 <= p.n) {
-                    if (p.y_bf16) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.y) + off);
+                const int nb = n0 + c * 32;
+                if (!row_ok || nb >= p.n) continue;
+                float v[32];
+                scale_chunk<KIND>(r, v, alpha, ra, p.b_row_scale + nb, p.n - nb);
+                if (p.y_bf16) {
+                    __nv_bfloat16 *yrow = reinterpret_cast<__nv_bfloat16 *>(p.y) + (int64_t)row * p.n;
+                    if (vec && nb + 32 <= p.n) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(yrow + nb);
 #pragma unroll
-                        for (int i = 0; i < 4; i++)
-                            dst[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
-                                                pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+                        for (int k4 = 0; k4 < 4; k4++)
+                            dst[k4] = make_uint4(pack_bf16x2(v[8 * k4], v[8 * k4 + 1]), pack_bf16x2(v[8 * k4 + 2], v[8 * k4 + 3]),
+                                                 pack_bf16x2(v[8 * k4 + 4], v[8 * k4 + 5]),
+                                                 pack_bf16x2(v[8 * k4 + 6], v[8 * k4 + 7]));
                     } else {
-                        float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.y) + off);
 #pragma unroll
-                        for (int i = 0; i < 8; i++) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                        for (int j = 0; j < 32; j++)
+                            if (nb + j < p.n) yrow[nb + j] = __float2bfloat16_rn(v[j]);
                     }
                 } else {
+                    float *yrow = reinterpret_cast<float *>(p.y) + (int64_t)row * p.n;
+                    if (vec && nb + 32 <= p.n) {
+                        float4 *dst = reinterpret_cast<float4 *>(yrow + nb);
 #pragma unroll
-                    for (int j = 0; j < 32; j++) {
-                        if (nb + j < p.n) {
-                            if (p.y_bf16) reinterpret_cast<__nv_bfloat16 *>(p.y)[off + j] = __float2bfloat16_rn(v[j]);
-                            else reinterpret_cast<float *>(p.y)[off + j] = v[j];
-                        }
+                        for (int k4 = 0; k4 < 8; k4++)
+                            dst[k4] = make_float4(v[4 * k4], v[4 * k4 + 1], v[4 * k4 + 2], v[4 * k4 + 3]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; j++)
+                            if (nb + j < p.n) yrow[nb + j] = v[j];
                     }
                 }
             }
@@ -686,7 +748,17 @@ cudaError_t launch_qlinear(const GemmOperands &op, cudaStream_t s) {
     p.has_lowrank = op.tp != nullptr;
     p.y_bf16 = op.y_bf16;
     p.wait_ns = 2000000000ull;   // 2 s
-    dim3 grid((unsigned)((op.n + BN - 1) / BN), (unsigned)((op.m + BM - 1) / BM));
+    p.m_tiles = (int)((op.m + BM - 1) / BM);
+    p.n_tiles = (int)((op.n + BN - 1) / BN);
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0) sms = 148;
+    }
+    const int tiles = p.m_tiles * p.n_tiles;
+    dim3 grid((unsigned)(tiles < sms ? tiles : sms));
     switch (op.fmt) {
     case kNVFP4: return launch_kind<kKindNVFP4>(p, grid, s);
     case kMXFP4: return launch_kind<kKindMXFP4>(p, grid, s);
