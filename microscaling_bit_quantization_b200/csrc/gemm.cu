@@ -1,0 +1,711 @@
+// gemm.cu -- block-scaled low-bit GEMM on 5th-generation tensor cores
+// (tcgen05, CTA pairs) with the dequantization epilogue and the SVDQuant
+// low-rank branch fused.
+//
+// Sources: Nunchaku/Diffusers article -- svdq_w4a4 runs attention and MLP
+// linears with 4-bit weights and activations (INT4 and NVFP4 variants) and
+// keeps a 16-bit low-rank part of each weight beside the 4-bit residual
+// (sections "Main explanation", "Kernels and supported hardware");
+// Chameleon article -- W8A8 formats per layer and timestep interval;
+// MixDiT article section 1 -- with shared block exponents a multiply is a
+// mantissa multiply plus an exponent add, which the block-scaled MMA does in
+// hardware.
+//
+// Structure.  Clusters of two CTAs (one per SM) compute 256 x 256 output
+// tiles with cta_group::2 MMAs: each CTA stages its own 128 rows of A, its
+// 128-row half of B, the scale factors of its A rows and of all 256 B rows,
+// and holds its 128 x 256 part of the accumulator in its own TMEM.  Per CTA:
+//   warp 0      TMA producer into a 5-stage ring (128-byte rows, 128B
+//               swizzle); the second CTA's loads complete on the first
+//               CTA's barriers (TMA .cta_group::2, no multicast)
+//   warp 1      TMEM allocation; in the first CTA also the single thread
+//               that copies scale factors to TMEM (tcgen05.cp) and issues
+//               the MMAs, committing to both CTAs' barriers
+//   warps 2-5   epilogue: TMEM -> registers -> scaling -> swizzled shared
+//               staging -> TMA bulk stores
+// The kernel is persistent: clusters walk the tiles, the TMA ring runs on
+// across tiles, and tiles alternate between two TMEM accumulator stages
+// that share 64 columns (two 256-column stages fit beside the scale factors
+// only that way); the epilogue drains the shared columns first, so the next
+// tile's MMAs wait only for those.
+// The low-rank branch is one extra pipeline stage: a bf16 kind::f16 MMA of
+// the packed activation [hi | lo] (m x 64) against the packed up-projection
+// [L2^T | L2^T] (n x 64) into the same accumulator, the activation having
+// been divided by the epilogue scale so that alpha * acc adds t . l2.
+// Every mbarrier wait is bounded; a wait that runs out latches the device
+// error word (read by mxq_check) and the CTA drains and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+
+#include "mxq_formats.cuh"
+#include "mxq_internal.h"
+
+namespace mxq {
+
+__device__ unsigned int g_error_word;
+
+namespace {
+
+constexpr int BM = 128;                 // accumulator rows per CTA (a pair covers 256)
+constexpr int BN = 256;                 // output columns per tile
+constexpr int BNH = 128;                // B rows staged per CTA
+constexpr int BKB = 128;                // bytes of K per stage row
+constexpr int STAGES = 5;
+constexpr int A_STAGE = BM * BKB;       // 16 KB
+constexpr int B_STAGE = BNH * BKB;      // 16 KB
+constexpr int SF_STAGE = 6144;          // SFA (<= 4 atoms) at 0, SFB halves at 2048 and 4096
+constexpr int STAGE_BYTES = A_STAGE + B_STAGE + SF_STAGE;   // 38 KB, a multiple of 1 KB
+constexpr int EPI_BUF = 4096;           // one 32-row x 128-byte staging buffer
+constexpr int EPI_BYTES = 4 * 2 * EPI_BUF;                  // 4 warps x 2 buffers
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
+constexpr int kGemmThreads = 192;
+constexpr uint32_t TMEM_COLS = 512;
+// TMEM columns: accumulator stage 0 at [0, 256), stage 1 at [192, 448)
+// (the stages share 64 columns), scale factors at [448, 512).
+constexpr uint32_t ACC_STAGE1 = 192;
+constexpr uint32_t TMEM_SFA = 448, TMEM_SFB = 464;
+
+enum Kind : int { kKindNVFP4 = 0, kKindMXFP4 = 1, kKindMXFP8 = 2, kKindFP8 = 3, kKindINT8 = 4 };
+
+constexpr unsigned int kErrTimeoutProducer = 1u, kErrTimeoutMma = 2u, kErrTimeoutEpilogue = 4u;
+
+struct GemmParams {
+    CUtensorMap tma_a, tma_b, tma_sfa, tma_sfb, tma_t, tma_l2, tma_y;
+    const float *a_row_scale, *b_row_scale;
+    const float *a_ts, *b_ts;
+    void *y;
+    int m, n, kbytes, num_k_tiles, s4, has_lowrank, y_bf16, y_tma;
+    int m_tiles, n_tiles;         // 256 x 256 tiles
+    int sfa_tiles;                // 128-row scale tiles of A (rows padded to 128)
+    unsigned long long wait_ns;
+};
+
+// ------------------------------------------------------------------ PTX
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_id() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_count() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+// Address of this CTA's shared variable `p` in the shared window of cluster rank `rank`.
+__device__ __forceinline__ uint32_t map_to_rank(const void *p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+// Arrival on a barrier of a CTA of the cluster (cluster-scope release).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+template <bool CLUSTER>
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    if (CLUSTER)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Bounded wait for the phase of parity `parity` to complete.
+template <bool CLUSTER = false>
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned long long limit_ns) {
+    if (mbar_try_wait<CLUSTER>(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if (mbar_try_wait<CLUSTER>(bar, parity)) return true;
+        if (global_ns() - t0 > limit_ns) return false;
+    }
+}
+
+// 2-D tiled TMA load into this CTA's shared memory, completing on the
+// barrier at cluster address `bar` (either CTA of the pair).
+__device__ __forceinline__ void tma_load_pair(const CUtensorMap *map, void *dst, uint32_t bar, int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int c0, int c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map), "r"(c0),
+                 "r"(c1), "r"(smem_u32(src))
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Arrive on the barrier at this offset in both CTAs once the issued MMAs complete.
+__device__ __forceinline__ void tc_commit_pair(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"((uint16_t)3)
+        : "memory");
+}
+__device__ __forceinline__ void tc_cp_pair(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Shared-memory matrix descriptor, K-major, 128-byte swizzle: 8-row x 128 B
+// core groups 1024 B apart (stride byte offset), descriptor version 1.
+__device__ __forceinline__ uint64_t sdesc_sw128(const void *p) {
+    uint64_t a = (smem_u32(p) >> 4) & 0x3FFFu;
+    return a | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+// Descriptor of one 512-byte scale-factor atom for tcgen05.cp (no swizzle,
+// 8 rows of 16 B per core matrix, core matrices 128 B apart).
+__device__ __forceinline__ uint64_t sdesc_sf(const void *p) {
+    uint64_t a = (smem_u32(p) >> 4) & 0x3FFFu;
+    return a | (8ull << 32) | (1ull << 46);
+}
+
+template <int KIND>
+__device__ __forceinline__ void mma_block_scaled(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc,
+                                                 uint32_t sfa, uint32_t sfb) {
+    if (KIND == kKindNVFP4)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+            ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb));
+    else if (KIND == kKindMXFP4)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+            ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb));
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale.scale_vec::1X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+            ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb));
+}
+
+template <int KIND>
+__device__ __forceinline__ void mma_plain(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    if (KIND == kKindFP8)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+            ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc));
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+            ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+
+// 32 lanes x 32 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Instruction descriptors (M = 256 over the pair, N = 256, K-major A and B).
+__host__ __device__ constexpr uint32_t idesc_common() { return ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(256 >> 4) << 24); }
+template <int KIND>
+__host__ __device__ constexpr uint32_t idesc_main() {
+    return KIND == kKindNVFP4 ? idesc_common() | (1u << 7) | (1u << 10)                 // E2M1 x E2M1, UE4M3 scales
+         : KIND == kKindMXFP4 ? idesc_common() | (1u << 7) | (1u << 10) | (1u << 23)   // E2M1 x E2M1, UE8M0 scales
+         : KIND == kKindMXFP8 ? idesc_common() | (1u << 23)                           // E4M3 x E4M3, UE8M0 scales
+         : KIND == kKindFP8   ? idesc_common() | (1u << 4)                            // E4M3 x E4M3 -> f32
+                              : idesc_common() | (2u << 4) | (1u << 7) | (1u << 10);  // s8 x s8 -> s32
+}
+__host__ __device__ constexpr uint32_t idesc_bf16() { return idesc_common() | (1u << 4) | (1u << 7) | (1u << 10); }
+
+// Scale-factor atoms (512 B) per stage for 128 rows.
+template <int KIND>
+__host__ __device__ constexpr int sf_atoms() { return KIND == kKindNVFP4 ? 4 : KIND == kKindMXFP4 ? 2 : KIND == kKindMXFP8 ? 1 : 0; }
+
+__device__ __forceinline__ void latch_error(unsigned int code) { atomicOr(&g_error_word, code); }
+
+// Epilogue value of accumulator column j of a chunk: alpha * acc (fp32
+// accumulators) or acc * sa * sb[n] (s32 accumulators of INT8_ROW).
+template <int KIND>
+__device__ __forceinline__ void scale_chunk(const uint32_t (&r)[32], float (&v)[32], float alpha, float ra,
+                                            const float *sbn, int nvalid) {
+    if (KIND == kKindINT8) {
+#pragma unroll
+        for (int j = 0; j < 32; j++) {
+            const float sb = j < nvalid ? __ldg(sbn + j) : 0.0f;
+            v[j] = __fmul_rn(__fmul_rn((float)(int)r[j], ra), sb);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; j++) v[j] = __fmul_rn(__uint_as_float(r[j]), alpha);
+    }
+}
+
+template <int KIND>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    k_gemm(const __grid_constant__ GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t *epi = smem + STAGES * STAGE_BYTES;
+    uint64_t *full = reinterpret_cast<uint64_t *>(epi + EPI_BYTES);   // [STAGES] (used in the first CTA)
+    uint64_t *empty = full + STAGES;                                   // [STAGES]
+    uint64_t *accf = empty + STAGES;                                   // [2] accumulator stage full
+    uint64_t *acce = accf + 2;                                         // [2] stage drained (first CTA)
+    uint64_t *ovlf = acce + 2;                                         // shared columns drained (first CTA)
+    uint64_t *drain = ovlf + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const int cid = (int)cluster_id(), ncl = (int)cluster_count();
+    constexpr int NSF = sf_atoms<KIND>();
+    const int num_tiles = p.m_tiles * p.n_tiles;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; s++) {
+            mbar_init(full + s, 1);
+            mbar_init(empty + s, 1);
+        }
+        for (int i = 0; i < 2; i++) {
+            mbar_init(accf + i, 1);
+            mbar_init(acce + i, 8);   // 4 epilogue warps x 2 CTAs
+        }
+        mbar_init(ovlf, 8);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int nsteps = p.num_k_tiles + p.has_lowrank;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- producer (both CTAs)
+        if (lane == 0) {
+            int it = 0, issued = 0;
+            for (int tile = cid; tile < num_tiles && !*abort_flag; tile += ncl) {
+                const int pm0 = (tile / p.n_tiles) * 256, n0 = (tile % p.n_tiles) * BN;
+                const int m0 = pm0 + (int)rank * BM, nb0 = n0 + (int)rank * BNH;
+                const int rt_a = (pm0 >> 7) + (int)rank;
+                const bool sfa_mine = rt_a < p.sfa_tiles;
+                const bool sfa_peer = (pm0 >> 7) + 1 < p.sfa_tiles;
+                const bool b_hi = (n0 + 128) < p.n;
+                const int rt_b = n0 >> 7;
+                for (int kt = 0; kt < nsteps; kt++, it++) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!mbar_wait(empty + s, ph ^ 1, p.wait_ns)) {
+                        latch_error(kErrTimeoutProducer);
+                        *abort_flag = 1;
+                        break;
+                    }
+                    if (*abort_flag) break;
+                    uint8_t *sa = smem + s * STAGE_BYTES;
+                    uint8_t *sb = sa + A_STAGE;
+                    uint8_t *sf = sb + B_STAGE;
+                    const uint32_t bar = map_to_rank(full + s, 0);
+                    if (kt < p.num_k_tiles) {
+                        if (rank == 0) {
+                            uint32_t bytes = 2 * (A_STAGE + B_STAGE);
+                            if (NSF) bytes += NSF * 512 * (1 + (sfa_peer ? 1 : 0) + 2 * (b_hi ? 2 : 1));
+                            mbar_arrive_expect_tx(full + s, bytes);
+                        }
+                        tma_load_pair(&p.tma_a, sa, bar, kt * BKB, m0);
+                        tma_load_pair(&p.tma_b, sb, bar, kt * BKB, nb0);
+                        if (NSF) {
+                            if (sfa_mine) tma_load_pair(&p.tma_sfa, sf, bar, 0, rt_a * p.s4 + kt * NSF);
+                            tma_load_pair(&p.tma_sfb, sf + 2048, bar, 0, rt_b * p.s4 + kt * NSF);
+                            if (b_hi) tma_load_pair(&p.tma_sfb, sf + 4096, bar, 0, (rt_b + 1) * p.s4 + kt * NSF);
+                        }
+                    } else {
+                        if (rank == 0) mbar_arrive_expect_tx(full + s, 2 * (A_STAGE + B_STAGE));
+                        tma_load_pair(&p.tma_t, sa, bar, 0, m0);
+                        tma_load_pair(&p.tma_l2, sb, bar, 0, nb0);
+                    }
+                    issued = it + 1;
+                }
+            }
+            if (*abort_flag && rank == 0) {
+                // drain: wait (bounded) for the loads that may still be in flight
+                for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; i++)
+                    mbar_wait(full + (i % STAGES), (i / STAGES) & 1, p.wait_ns);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer (first CTA)
+        if (lane == 0 && rank == 0) {
+            const uint32_t sfa_addr = tmem + TMEM_SFA, sfb_addr = tmem + TMEM_SFB;
+            bool issued_any = false;
+            int it = 0, tcount = 0;
+            for (int tile = cid; tile < num_tiles && !*abort_flag; tile += ncl, tcount++) {
+                const int n0 = (tile % p.n_tiles) * BN;
+                const bool b_hi = (n0 + 128) < p.n;
+                const int st = tcount & 1;
+                const uint32_t acc_addr = tmem + (st ? ACC_STAGE1 : 0u);
+                // this stage drained (tile tcount-2) and the shared columns (tile tcount-1), in both CTAs
+                bool ok = mbar_wait<true>(acce + st, ((tcount >> 1) & 1) ^ 1, p.wait_ns);
+                if (ok && tcount > 0) ok = mbar_wait<true>(ovlf, (tcount - 1) & 1, p.wait_ns);
+                if (!ok) {
+                    latch_error(kErrTimeoutMma);
+                    *abort_flag = 1;
+                    break;
+                }
+                tc_fence_after();
+                for (int kt = 0; kt < nsteps; kt++, it++) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!mbar_wait(full + s, ph, p.wait_ns)) {
+                        latch_error(kErrTimeoutMma);
+                        *abort_flag = 1;
+                        break;
+                    }
+                    if (*abort_flag) break;
+                    tc_fence_after();
+                    uint8_t *sa = smem + s * STAGE_BYTES;
+                    uint8_t *sb = sa + A_STAGE;
+                    uint8_t *sf = sb + B_STAGE;
+                    if (kt < p.num_k_tiles) {
+                        const int rem = (p.kbytes - kt * BKB) >> 5;
+                        const int nks = rem < 4 ? rem : 4;
+                        if (NSF) {
+#pragma unroll
+                            for (int i = 0; i < NSF; i++) {
+                                tc_cp_pair(sfa_addr + 4 * i, sdesc_sf(sf + 512 * i));
+                                tc_cp_pair(sfb_addr + 8 * i, sdesc_sf(sf + 2048 + 512 * i));
+                                if (b_hi) tc_cp_pair(sfb_addr + 8 * i + 4, sdesc_sf(sf + 4096 + 512 * i));
+                            }
+                        }
+                        for (int ks = 0; ks < nks; ks++) {
+                            const uint64_t ad = sdesc_sw128(sa + ks * 32), bd = sdesc_sw128(sb + ks * 32);
+                            const uint32_t accum = (kt > 0 || ks > 0) ? 1u : 0u;
+                            if (KIND == kKindNVFP4) {
+                                mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>(), accum, sfa_addr + 4 * ks,
+                                                       sfb_addr + 8 * ks);
+                            } else if (KIND == kKindMXFP4) {
+                                const uint32_t id = (uint32_t)((ks & 1) * 2);
+                                mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>() | (id << 29) | (id << 4),
+                                                       accum, sfa_addr + 4 * (ks >> 1), sfb_addr + 8 * (ks >> 1));
+                            } else if (KIND == kKindMXFP8) {
+                                const uint32_t id = (uint32_t)ks;
+                                mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>() | (id << 29) | (id << 4),
+                                                       accum, sfa_addr, sfb_addr);
+                            } else {
+                                mma_plain<KIND>(acc_addr, ad, bd, idesc_main<KIND>(), accum);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int ks = 0; ks < 4; ks++)
+                            mma_bf16(acc_addr, sdesc_sw128(sa + ks * 32), sdesc_sw128(sb + ks * 32), idesc_bf16(), 1u);
+                    }
+                    issued_any = true;
+                    tc_commit_pair(empty + s);
+                }
+                if (*abort_flag) break;
+                tc_commit_pair(accf + st);
+            }
+            if (*abort_flag && issued_any) {
+                tc_commit_pair(drain);
+                mbar_wait(drain, 0, p.wait_ns);
+            }
+        }
+    } else {
+        // ---------------------------------------------------------- epilogue (both CTAs)
+        const int q = warp & 3;   // TMEM lane quarter this warp may access
+        const uint32_t ovl_leader = map_to_rank(ovlf, 0);
+        const uint32_t acce_leader0 = map_to_rank(acce, 0), acce_leader1 = map_to_rank(acce + 1, 0);
+        uint8_t *stage_buf = epi + q * 2 * EPI_BUF;
+        const bool vec = p.y_bf16 ? (p.n % 8 == 0) : (p.n % 4 == 0);
+        int tcount = 0, sub = 0;
+        for (int tile = cid; tile < num_tiles; tile += ncl, tcount++) {
+            const int pm0 = (tile / p.n_tiles) * 256, n0 = (tile % p.n_tiles) * BN;
+            const int row0 = pm0 + (int)rank * BM + q * 32;
+            const int row = row0 + lane;
+            const int st = tcount & 1;
+            bool ok = !*abort_flag && mbar_wait(accf + st, (tcount >> 1) & 1, p.wait_ns);
+            ok = __all_sync(0xFFFFFFFFu, ok);
+            if (!ok) {
+                if (lane == 0 && !*abort_flag) latch_error(kErrTimeoutEpilogue);
+                *abort_flag = 1;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + (st ? ACC_STAGE1 : 0u);
+            float alpha = 1.0f, ra = 0.0f;
+            if (KIND == kKindNVFP4 || KIND == kKindFP8) alpha = __fmul_rn(__ldg(p.a_ts), __ldg(p.b_ts));
+            const bool row_ok = row < p.m;
+            if (KIND == kKindINT8 && row_ok) ra = __ldg(p.a_row_scale + row);
+            // the 64 shared columns first: the last two chunks of stage 0, the first two of stage 1
+#pragma unroll 1
+            for (int i = 0; i < BN / 32; i++) {
+                const int c = st ? i : (i + 6) & 7;
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(lane_base + (uint32_t)(c * 32), r);
+                if (i == 1 || i == 7) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_remote(i == 1 ? ovl_leader : (st ? acce_leader1 : acce_leader0));
+                }
+                const int nb = n0 + c * 32;
+                float v[32];
+                scale_chunk<KIND>(r, v, alpha, ra, p.b_row_scale + nb, p.n - nb);
+                if (p.y_tma) {
+                    // swizzled staging (16-byte chunk j of row t at t*128 + (j ^ (t & 7))*16),
+                    // then one TMA store per 32 rows x 128 bytes
+                    const bool bf = p.y_bf16 != 0;
+                    const bool first_half = !bf || (c & 1) == 0;
+                    uint8_t *buf = stage_buf + (sub & 1) * EPI_BUF;
+                    if (first_half) {
+                        if (lane == 0) bulk_wait_read1();
+                        __syncwarp();
+                    }
+                    uint4 *rowp = reinterpret_cast<uint4 *>(buf + lane * 128);
+                    if (bf) {
+                        const int j0 = (c & 1) * 4;
+#pragma unroll
+                        for (int k4 = 0; k4 < 4; k4++)
+                            rowp[(j0 + k4) ^ (lane & 7)] =
+                                make_uint4(pack_bf16x2(v[8 * k4], v[8 * k4 + 1]), pack_bf16x2(v[8 * k4 + 2], v[8 * k4 + 3]),
+                                           pack_bf16x2(v[8 * k4 + 4], v[8 * k4 + 5]),
+                                           pack_bf16x2(v[8 * k4 + 6], v[8 * k4 + 7]));
+                    } else {
+#pragma unroll
+                        for (int k4 = 0; k4 < 8; k4++)
+                            rowp[k4 ^ (lane & 7)] = make_uint4(__float_as_uint(v[4 * k4]), __float_as_uint(v[4 * k4 + 1]),
+                                                               __float_as_uint(v[4 * k4 + 2]), __float_as_uint(v[4 * k4 + 3]));
+                    }
+                    if (!bf || (c & 1) == 1) {
+                        fence_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&p.tma_y, buf, bf ? n0 + (c >> 1) * 64 : nb, row0);
+                            bulk_commit();
+                        }
+                        sub++;
+                    }
+                } else if (row_ok && nb < p.n) {
+                    if (p.y_bf16) {
+                        __nv_bfloat16 *yrow = reinterpret_cast<__nv_bfloat16 *>(p.y) + (int64_t)row * p.n;
+                        if (vec && nb + 32 <= p.n) {
+                            uint4 *dst = reinterpret_cast<uint4 *>(yrow + nb);
+#pragma unroll
+                            for (int k4 = 0; k4 < 4; k4++)
+                                dst[k4] = make_uint4(pack_bf16x2(v[8 * k4], v[8 * k4 + 1]),
+                                                     pack_bf16x2(v[8 * k4 + 2], v[8 * k4 + 3]),
+                                                     pack_bf16x2(v[8 * k4 + 4], v[8 * k4 + 5]),
+                                                     pack_bf16x2(v[8 * k4 + 6], v[8 * k4 + 7]));
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; j++)
+                                if (nb + j < p.n) yrow[nb + j] = __float2bfloat16_rn(v[j]);
+                        }
+                    } else {
+                        float *yrow = reinterpret_cast<float *>(p.y) + (int64_t)row * p.n;
+                        if (vec && nb + 32 <= p.n) {
+                            float4 *dst = reinterpret_cast<float4 *>(yrow + nb);
+#pragma unroll
+                            for (int k4 = 0; k4 < 8; k4++)
+                                dst[k4] = make_float4(v[4 * k4], v[4 * k4 + 1], v[4 * k4 + 2], v[4 * k4 + 3]);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; j++)
+                                if (nb + j < p.n) yrow[nb + j] = v[j];
+                        }
+                    }
+                }
+            }
+        }
+        if (lane == 0) bulk_wait_all();
+    }
+
+    tc_fence_before();
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+    }
+}
+
+// ------------------------------------------------------------------ host
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+    auto fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int KIND>
+cudaError_t launch_kind(const GemmParams &p, int grid, cudaStream_t s) {
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(k_gemm<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    k_gemm<KIND><<<grid, kGemmThreads, SMEM_BYTES, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_qlinear(const GemmOperands &op, cudaStream_t s) {
+    if (op.m == 0 || op.n == 0) return cudaSuccess;
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    const bool is4 = op.fmt == kMXFP4 || op.fmt == kNVFP4;
+    const int64_t kbytes = is4 ? op.k / 2 : op.k;
+    const auto SW128 = CU_TENSOR_MAP_SWIZZLE_128B, NOSW = CU_TENSOR_MAP_SWIZZLE_NONE;
+    if (!encode_2d(&p.tma_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, op.a_codes, kbytes, op.m, kbytes, BKB, BM, SW128) ||
+        !encode_2d(&p.tma_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, op.b_codes, kbytes, op.n, kbytes, BKB, BNH, SW128))
+        return cudaErrorInvalidValue;
+    const int blk = fmt_block(op.fmt);
+    const bool byte_sf = fmt_byte_scales(op.fmt);
+    if (byte_sf) {
+        // scale atoms as rows of 64 x 8-byte elements: (row tile, scale-column group) -> atom index
+        const int64_t s_pad = ((op.k / blk) + 15) / 16 * 16;
+        const int64_t atoms_a = ((op.m + 127) / 128) * (s_pad / 4), atoms_b = ((op.n + 127) / 128) * (s_pad / 4);
+        const int nsf = op.fmt == kNVFP4 ? 4 : op.fmt == kMXFP4 ? 2 : 1;
+        if (!encode_2d(&p.tma_sfa, CU_TENSOR_MAP_DATA_TYPE_UINT64, op.a_scales, 64, atoms_a, 512, 64, nsf, NOSW) ||
+            !encode_2d(&p.tma_sfb, CU_TENSOR_MAP_DATA_TYPE_UINT64, op.b_scales, 64, atoms_b, 512, 64, nsf, NOSW))
+            return cudaErrorInvalidValue;
+        p.s4 = (int)(s_pad / 4);
+    }
+    if (op.tp) {
+        if (!encode_2d(&p.tma_t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, op.tp, 64, op.m, 128, 64, BM, SW128) ||
+            !encode_2d(&p.tma_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, op.l2p, 64, op.n, 128, 64, BNH, SW128))
+            return cudaErrorInvalidValue;
+    }
+    const int esz = op.y_bf16 ? 2 : 4;
+    p.y_tma = ((op.n * esz) % 16 == 0) && ((reinterpret_cast<uintptr_t>(op.y) & 15u) == 0);
+    if (p.y_tma &&
+        !encode_2d(&p.tma_y, op.y_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, op.y,
+                   op.n, op.m, op.n * esz, op.y_bf16 ? 64 : 32, 32, SW128))
+        p.y_tma = 0;
+    p.a_row_scale = (const float *)op.a_scales;
+    p.b_row_scale = (const float *)op.b_scales;
+    p.a_ts = op.a_tensor_scale;
+    p.b_ts = op.b_tensor_scale;
+    p.y = op.y;
+    p.m = (int)op.m;
+    p.n = (int)op.n;
+    p.kbytes = (int)kbytes;
+    p.num_k_tiles = (int)((kbytes + BKB - 1) / BKB);
+    p.has_lowrank = op.tp != nullptr;
+    p.y_bf16 = op.y_bf16;
+    p.m_tiles = (int)((op.m + 255) / 256);
+    p.n_tiles = (int)((op.n + BN - 1) / BN);
+    p.sfa_tiles = (int)((op.m + 127) / 128);
+    p.wait_ns = 2000000000ull;   // 2 s
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0) sms = 148;
+    }
+    const int tiles = p.m_tiles * p.n_tiles;
+    const int clusters = tiles < sms / 2 ? tiles : sms / 2;
+    const int grid = 2 * clusters;
+    switch (op.fmt) {
+    case kNVFP4: return launch_kind<kKindNVFP4>(p, grid, s);
+    case kMXFP4: return launch_kind<kKindMXFP4>(p, grid, s);
+    case kMXFP8: return launch_kind<kKindMXFP8>(p, grid, s);
+    case kFP8Tensor: return launch_kind<kKindFP8>(p, grid, s);
+    case kINT8Row: return launch_kind<kKindINT8>(p, grid, s);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t read_and_clear_error(unsigned int *value) {
+    unsigned int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(value, g_error_word, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    return cudaMemcpyToSymbol(g_error_word, &zero, sizeof(unsigned int));
+}
+
+}  // namespace mxq
