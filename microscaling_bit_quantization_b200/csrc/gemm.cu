@@ -25,9 +25,9 @@
 //               staging -> TMA bulk stores
 // The kernel is persistent: clusters walk the tiles, the TMA ring runs on
 // across tiles, and tiles alternate between two TMEM accumulator stages
-// that share 64 columns (two 256-column stages fit beside the scale factors
-// only that way); the epilogue drains the shared columns first, so the next
-// tile's MMAs wait only for those.
+// that share 96 columns (two 256-column stages fit beside the scale-factor
+// ring only that way); the epilogue drains the shared columns first, so the
+// next tile's MMAs wait only for those.
 // The low-rank branch is one extra pipeline stage: a bf16 kind::f16 MMA of
 // the packed activation [hi | lo] (m x 64) against the packed up-projection
 // [L2^T | L2^T] (n x 64) into the same accumulator, the activation having
@@ -65,10 +65,13 @@ constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
 constexpr int kGemmThreads = 192;
 constexpr uint32_t TMEM_COLS = 512;
-// TMEM columns: accumulator stage 0 at [0, 256), stage 1 at [192, 448)
-// (the stages share 64 columns), scale factors at [448, 512).
-constexpr uint32_t ACC_STAGE1 = 192;
-constexpr uint32_t TMEM_SFA = 448, TMEM_SFB = 464;
+// TMEM columns: accumulator stage 0 at [0, 256), stage 1 at [160, 416)
+// (the stages share 96 columns), then a ring of 8 scale-factor slots of 12
+// columns at [416, 512): SFA (4 columns) and the two SFB halves (4 + 4).
+// Each copy of scale factors goes to the next slot, so it never overwrites
+// columns that one of the last seven MMA groups reads.
+constexpr uint32_t ACC_STAGE1 = 160, OVL_CHUNKS = 3;
+constexpr uint32_t TMEM_SF = 416, SF_SLOT_COLS = 12, SF_SLOTS = 8;
 
 enum Kind : int { kKindNVFP4 = 0, kKindMXFP4 = 1, kKindMXFP8 = 2, kKindFP8 = 3, kKindINT8 = 4 };
 
@@ -400,9 +403,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer (first CTA)
         if (lane == 0 && rank == 0) {
-            const uint32_t sfa_addr = tmem + TMEM_SFA, sfb_addr = tmem + TMEM_SFB;
             bool issued_any = false;
             int it = 0, tcount = 0;
+            uint32_t sf_slot = 0;
             for (int tile = cid; tile < num_tiles && !*abort_flag; tile += ncl, tcount++) {
                 const int n0 = (tile % p.n_tiles) * BN;
                 const bool b_hi = (n0 + 128) < p.n;
@@ -433,28 +436,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                     if (kt < p.num_k_tiles) {
                         const int rem = (p.kbytes - kt * BKB) >> 5;
                         const int nks = rem < 4 ? rem : 4;
-                        if (NSF) {
-#pragma unroll
-                            for (int i = 0; i < NSF; i++) {
-                                tc_cp_pair(sfa_addr + 4 * i, sdesc_sf(sf + 512 * i));
-                                tc_cp_pair(sfb_addr + 8 * i, sdesc_sf(sf + 2048 + 512 * i));
-                                if (b_hi) tc_cp_pair(sfb_addr + 8 * i + 4, sdesc_sf(sf + 4096 + 512 * i));
-                            }
+                        // scale-factor atoms of this stage (an NVFP4 atom serves one k-step,
+                        // an MXFP4 atom two, an MXFP8 atom four), each into the next ring slot
+                        const int natoms = NSF == 4 ? nks : NSF == 2 ? (nks + 1) >> 1 : (NSF ? 1 : 0);
+                        const uint32_t slot0 = sf_slot;
+                        for (int a = 0; a < natoms; a++) {
+                            const uint32_t base = tmem + TMEM_SF + SF_SLOT_COLS * ((slot0 + a) % SF_SLOTS);
+                            tc_cp_pair(base, sdesc_sf(sf + 512 * a));
+                            tc_cp_pair(base + 4, sdesc_sf(sf + 2048 + 512 * a));
+                            if (b_hi) tc_cp_pair(base + 8, sdesc_sf(sf + 4096 + 512 * a));
                         }
+                        sf_slot = (slot0 + natoms) % SF_SLOTS;
                         for (int ks = 0; ks < nks; ks++) {
                             const uint64_t ad = sdesc_sw128(sa + ks * 32), bd = sdesc_sw128(sb + ks * 32);
                             const uint32_t accum = (kt > 0 || ks > 0) ? 1u : 0u;
+                            const int a = NSF == 4 ? ks : NSF == 2 ? (ks >> 1) : 0;
+                            const uint32_t base = tmem + TMEM_SF + SF_SLOT_COLS * ((slot0 + a) % SF_SLOTS);
                             if (KIND == kKindNVFP4) {
-                                mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>(), accum, sfa_addr + 4 * ks,
-                                                       sfb_addr + 8 * ks);
+                                mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>(), accum, base, base + 4);
                             } else if (KIND == kKindMXFP4) {
                                 const uint32_t id = (uint32_t)((ks & 1) * 2);
                                 mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>() | (id << 29) | (id << 4),
-                                                       accum, sfa_addr + 4 * (ks >> 1), sfb_addr + 8 * (ks >> 1));
+                                                       accum, base, base + 4);
                             } else if (KIND == kKindMXFP8) {
                                 const uint32_t id = (uint32_t)ks;
                                 mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>() | (id << 29) | (id << 4),
-                                                       accum, sfa_addr, sfb_addr);
+                                                       accum, base, base + 4);
                             } else {
                                 mma_plain<KIND>(acc_addr, ad, bd, idesc_main<KIND>(), accum);
                             }
@@ -501,54 +508,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             if (KIND == kKindNVFP4 || KIND == kKindFP8) alpha = __fmul_rn(__ldg(p.a_ts), __ldg(p.b_ts));
             const bool row_ok = row < p.m;
             if (KIND == kKindINT8 && row_ok) ra = __ldg(p.a_row_scale + row);
-            // the 64 shared columns first: the last two chunks of stage 0, the first two of stage 1
+            // the 96 shared columns first: the last three chunks of stage 0, the first three of stage 1
 #pragma unroll 1
             for (int i = 0; i < BN / 32; i++) {
-                const int c = st ? i : (i + 6) & 7;
+                const int c = st ? i : (i + 8 - (int)OVL_CHUNKS) & 7;
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(lane_base + (uint32_t)(c * 32), r);
-                if (i == 1 || i == 7) {
+                if (i == (int)OVL_CHUNKS - 1 || i == 7) {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive_remote(i == 1 ? ovl_leader : (st ? acce_leader1 : acce_leader0));
+                    if (lane == 0)
+                        mbar_arrive_remote(i == (int)OVL_CHUNKS - 1 ? ovl_leader : (st ? acce_leader1 : acce_leader0));
                 }
                 const int nb = n0 + c * 32;
                 float v[32];
                 scale_chunk<KIND>(r, v, alpha, ra, p.b_row_scale + nb, p.n - nb);
                 if (p.y_tma) {
-                    // swizzled staging (16-byte chunk j of row t at t*128 + (j ^ (t & 7))*16),
-                    // then one TMA store per 32 rows x 128 bytes
-                    const bool bf = p.y_bf16 != 0;
-                    const bool first_half = !bf || (c & 1) == 0;
+                    // swizzled staging of this 32-column chunk, then one TMA store of 32 rows:
+                    // bf16 rows of 64 B (64B swizzle: 16-byte unit j of row t at t*64 + (j ^ ((t >> 1) & 3))*16),
+                    // fp32 rows of 128 B (128B swizzle: unit j at t*128 + (j ^ (t & 7))*16)
                     uint8_t *buf = stage_buf + (sub & 1) * EPI_BUF;
-                    if (first_half) {
-                        if (lane == 0) bulk_wait_read1();
-                        __syncwarp();
-                    }
-                    uint4 *rowp = reinterpret_cast<uint4 *>(buf + lane * 128);
-                    if (bf) {
-                        const int j0 = (c & 1) * 4;
+                    if (lane == 0) bulk_wait_read1();
+                    __syncwarp();
+                    if (p.y_bf16) {
+                        uint4 *rowp = reinterpret_cast<uint4 *>(buf + lane * 64);
 #pragma unroll
                         for (int k4 = 0; k4 < 4; k4++)
-                            rowp[(j0 + k4) ^ (lane & 7)] =
+                            rowp[k4 ^ ((lane >> 1) & 3)] =
                                 make_uint4(pack_bf16x2(v[8 * k4], v[8 * k4 + 1]), pack_bf16x2(v[8 * k4 + 2], v[8 * k4 + 3]),
                                            pack_bf16x2(v[8 * k4 + 4], v[8 * k4 + 5]),
                                            pack_bf16x2(v[8 * k4 + 6], v[8 * k4 + 7]));
                     } else {
+                        uint4 *rowp = reinterpret_cast<uint4 *>(buf + lane * 128);
 #pragma unroll
                         for (int k4 = 0; k4 < 8; k4++)
                             rowp[k4 ^ (lane & 7)] = make_uint4(__float_as_uint(v[4 * k4]), __float_as_uint(v[4 * k4 + 1]),
                                                                __float_as_uint(v[4 * k4 + 2]), __float_as_uint(v[4 * k4 + 3]));
                     }
-                    if (!bf || (c & 1) == 1) {
-                        fence_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_store_2d(&p.tma_y, buf, bf ? n0 + (c >> 1) * 64 : nb, row0);
-                            bulk_commit();
-                        }
-                        sub++;
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&p.tma_y, buf, nb, row0);
+                        bulk_commit();
                     }
+                    sub++;
                 } else if (row_ok && nb < p.n) {
                     if (p.y_bf16) {
                         __nv_bfloat16 *yrow = reinterpret_cast<__nv_bfloat16 *>(p.y) + (int64_t)row * p.n;
@@ -664,7 +667,7 @@ cudaError_t launch_qlinear(const GemmOperands &op, cudaStream_t s) {
     p.y_tma = ((op.n * esz) % 16 == 0) && ((reinterpret_cast<uintptr_t>(op.y) & 15u) == 0);
     if (p.y_tma &&
         !encode_2d(&p.tma_y, op.y_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, op.y,
-                   op.n, op.m, op.n * esz, op.y_bf16 ? 64 : 32, 32, SW128))
+                   op.n, op.m, op.n * esz, 32, 32, op.y_bf16 ? CU_TENSOR_MAP_SWIZZLE_64B : SW128))
         p.y_tma = 0;
     p.a_row_scale = (const float *)op.a_scales;
     p.b_row_scale = (const float *)op.b_scales;
