@@ -19,10 +19,11 @@
 //               swizzle); the second CTA's loads complete on the first
 //               CTA's barriers (TMA .cta_group::2, no multicast)
 //   warp 1      TMEM allocation; in the first CTA also the single thread
-//               that copies scale factors to TMEM (tcgen05.cp) and issues
-//               the MMAs, committing to both CTAs' barriers
+//               that issues the MMAs, committing to both CTAs' barriers
 //   warps 2-5   epilogue: TMEM -> registers -> scaling -> swizzled shared
 //               staging -> TMA bulk stores
+//   warp 6      in the first CTA, the thread that copies each stage's scale
+//               factors to TMEM (tcgen05.cp) and signals the MMA thread
 // The kernel is persistent: clusters walk the tiles, the TMA ring runs on
 // across tiles, and tiles alternate between two TMEM accumulator stages
 // that share 96 columns (two 256-column stages fit beside the scale-factor
@@ -63,15 +64,15 @@ constexpr int EPI_BUF = 4096;           // one 32-row x 128-byte staging buffer
 constexpr int EPI_BYTES = 4 * 2 * EPI_BUF;                  // 4 warps x 2 buffers
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 224;   // 7 warps
 constexpr uint32_t TMEM_COLS = 512;
 // TMEM columns: accumulator stage 0 at [0, 256), stage 1 at [160, 416)
-// (the stages share 96 columns), then a ring of 8 scale-factor slots of 12
-// columns at [416, 512): SFA (4 columns) and the two SFB halves (4 + 4).
-// Each copy of scale factors goes to the next slot, so it never overwrites
-// columns that one of the last seven MMA groups reads.
+// (the stages share 96 columns), then two groups of four 12-column
+// scale-factor slots at [416, 512) (SFA 4 columns, the two SFB halves 4 + 4
+// per atom).  K-tile i uses group i % 2, so a group is rewritten only after
+// the MMAs of k-tile i - 2 have completed.
 constexpr uint32_t ACC_STAGE1 = 160, OVL_CHUNKS = 3;
-constexpr uint32_t TMEM_SF = 416, SF_SLOT_COLS = 12, SF_SLOTS = 8;
+constexpr uint32_t TMEM_SF = 416, SF_SLOT_COLS = 12, SF_GROUP_COLS = 48;
 
 enum Kind : int { kKindNVFP4 = 0, kKindMXFP4 = 1, kKindMXFP8 = 2, kKindFP8 = 3, kKindINT8 = 4 };
 
@@ -195,6 +196,14 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t *bar) {
         "h"((uint16_t)3)
         : "memory");
 }
+// Arrive on this CTA's barrier once this thread's issued tcgen05 operations complete.
+__device__ __forceinline__ void tc_commit_self(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_local(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 __device__ __forceinline__ void tc_cp_pair(uint32_t taddr, uint64_t sdesc) {
     asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
@@ -314,7 +323,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     uint64_t *acce = accf + 2;                                         // [2] stage drained (first CTA)
     uint64_t *ovlf = acce + 2;                                         // shared columns drained (first CTA)
     uint64_t *drain = ovlf + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *sfready = drain + 1;                                     // [STAGES] scale factors in TMEM (first CTA)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sfready + STAGES);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -334,6 +344,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
         mbar_init(ovlf, 8);
         mbar_init(drain, 1);
+        for (int i = 0; i < STAGES; i++) mbar_init(sfready + i, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -405,10 +416,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         if (lane == 0 && rank == 0) {
             bool issued_any = false;
             int it = 0, tcount = 0;
-            uint32_t sf_slot = 0;
             for (int tile = cid; tile < num_tiles && !*abort_flag; tile += ncl, tcount++) {
-                const int n0 = (tile % p.n_tiles) * BN;
-                const bool b_hi = (n0 + 128) < p.n;
                 const int st = tcount & 1;
                 const uint32_t acc_addr = tmem + (st ? ACC_STAGE1 : 0u);
                 // this stage drained (tile tcount-2) and the shared columns (tile tcount-1), in both CTAs
@@ -423,7 +431,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 for (int kt = 0; kt < nsteps; kt++, it++) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
-                    if (!mbar_wait(full + s, ph, p.wait_ns)) {
+                    // block-scaled kinds: the scale-factor warp has copied this stage's atoms to TMEM
+                    // (and seen the stage full); other kinds wait for the stage itself
+                    if (!mbar_wait(NSF ? sfready + s : full + s, ph, p.wait_ns)) {
                         latch_error(kErrTimeoutMma);
                         *abort_flag = 1;
                         break;
@@ -432,26 +442,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                     tc_fence_after();
                     uint8_t *sa = smem + s * STAGE_BYTES;
                     uint8_t *sb = sa + A_STAGE;
-                    uint8_t *sf = sb + B_STAGE;
                     if (kt < p.num_k_tiles) {
                         const int rem = (p.kbytes - kt * BKB) >> 5;
                         const int nks = rem < 4 ? rem : 4;
-                        // scale-factor atoms of this stage (an NVFP4 atom serves one k-step,
-                        // an MXFP4 atom two, an MXFP8 atom four), each into the next ring slot
-                        const int natoms = NSF == 4 ? nks : NSF == 2 ? (nks + 1) >> 1 : (NSF ? 1 : 0);
-                        const uint32_t slot0 = sf_slot;
-                        for (int a = 0; a < natoms; a++) {
-                            const uint32_t base = tmem + TMEM_SF + SF_SLOT_COLS * ((slot0 + a) % SF_SLOTS);
-                            tc_cp_pair(base, sdesc_sf(sf + 512 * a));
-                            tc_cp_pair(base + 4, sdesc_sf(sf + 2048 + 512 * a));
-                            if (b_hi) tc_cp_pair(base + 8, sdesc_sf(sf + 4096 + 512 * a));
-                        }
-                        sf_slot = (slot0 + natoms) % SF_SLOTS;
+                        const uint32_t group = tmem + TMEM_SF + SF_GROUP_COLS * (uint32_t)(it & 1);
                         for (int ks = 0; ks < nks; ks++) {
                             const uint64_t ad = sdesc_sw128(sa + ks * 32), bd = sdesc_sw128(sb + ks * 32);
                             const uint32_t accum = (kt > 0 || ks > 0) ? 1u : 0u;
+                            // an NVFP4 atom serves one k-step, an MXFP4 atom two, an MXFP8 atom four
                             const int a = NSF == 4 ? ks : NSF == 2 ? (ks >> 1) : 0;
-                            const uint32_t base = tmem + TMEM_SF + SF_SLOT_COLS * ((slot0 + a) % SF_SLOTS);
+                            const uint32_t base = group + SF_SLOT_COLS * (uint32_t)a;
                             if (KIND == kKindNVFP4) {
                                 mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>(), accum, base, base + 4);
                             } else if (KIND == kKindMXFP4) {
@@ -479,6 +479,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             }
             if (*abort_flag && issued_any) {
                 tc_commit_pair(drain);
+                mbar_wait(drain, 0, p.wait_ns);
+            }
+        }
+    } else if (warp == 6) {
+        // ---------------------------------------------------------- scale-factor copies (first CTA)
+        // Issued apart from the MMA thread: a tcgen05.cp stalls the thread that
+        // issues it, but runs alongside the MMAs in the tensor pipe.
+        if (NSF && lane == 0 && rank == 0) {
+            int it = 0;
+            bool ok = true;
+            for (int tile = cid; tile < num_tiles && ok && !*abort_flag; tile += ncl) {
+                const int n0 = (tile % p.n_tiles) * BN;
+                const bool b_hi = (n0 + 128) < p.n;
+                for (int kt = 0; kt < nsteps; kt++, it++) {
+                    const int s = it % STAGES;
+                    ok = mbar_wait(full + s, (it / STAGES) & 1, p.wait_ns);
+                    // slot group it % 2 was last read by the MMAs of k-tile it - 2
+                    if (ok && it >= 2) ok = mbar_wait(empty + ((it - 2) % STAGES), ((it - 2) / STAGES) & 1, p.wait_ns);
+                    if (!ok || *abort_flag) {
+                        if (!ok) latch_error(kErrTimeoutMma);
+                        *abort_flag = 1;
+                        break;
+                    }
+                    if (kt < p.num_k_tiles) {
+                        const int rem = (p.kbytes - kt * BKB) >> 5;
+                        const int nks = rem < 4 ? rem : 4;
+                        const int natoms = NSF == 4 ? nks : NSF == 2 ? (nks + 1) >> 1 : 1;
+                        const uint8_t *sf = smem + s * STAGE_BYTES + A_STAGE + B_STAGE;
+                        const uint32_t group = tmem + TMEM_SF + SF_GROUP_COLS * (uint32_t)(it & 1);
+                        tc_fence_after();
+                        for (int a = 0; a < natoms; a++) {
+                            const uint32_t base = group + SF_SLOT_COLS * (uint32_t)a;
+                            tc_cp_pair(base, sdesc_sf(sf + 512 * a));
+                            tc_cp_pair(base + 4, sdesc_sf(sf + 2048 + 512 * a));
+                            if (b_hi) tc_cp_pair(base + 8, sdesc_sf(sf + 4096 + 512 * a));
+                        }
+                        tc_commit_self(sfready + s);
+                    } else {
+                        mbar_arrive_local(sfready + s);
+                    }
+                }
+            }
+            if (*abort_flag) {
+                tc_commit_self(drain);
                 mbar_wait(drain, 0, p.wait_ns);
             }
         }
