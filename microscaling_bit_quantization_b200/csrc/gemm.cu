@@ -22,8 +22,9 @@
 //               that issues the MMAs, committing to both CTAs' barriers
 //   warps 2-5   epilogue: TMEM -> registers -> scaling -> swizzled shared
 //               staging -> TMA bulk stores
-//   warp 6      in the first CTA, the thread that copies each stage's scale
-//               factors to TMEM (tcgen05.cp) and signals the MMA thread
+//   warps 6-7   in the first CTA, two threads that copy each stage's scale
+//               factors to TMEM (tcgen05.cp, even / odd atoms) and signal
+//               the MMA thread
 // The kernel is persistent: clusters walk the tiles, the TMA ring runs on
 // across tiles, and tiles alternate between two TMEM accumulator stages
 // that share 96 columns (two 256-column stages fit beside the scale-factor
@@ -64,7 +65,7 @@ constexpr int EPI_BUF = 4096;           // one 32-row x 128-byte staging buffer
 constexpr int EPI_BYTES = 4 * 2 * EPI_BUF;                  // 4 warps x 2 buffers
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
-constexpr int kGemmThreads = 224;   // 7 warps
+constexpr int kGemmThreads = 256;   // 8 warps
 constexpr uint32_t TMEM_COLS = 512;
 // TMEM columns: accumulator stage 0 at [0, 256), stage 1 at [160, 416)
 // (the stages share 96 columns), then two groups of four 12-column
@@ -344,7 +345,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
         mbar_init(ovlf, 8);
         mbar_init(drain, 1);
-        for (int i = 0; i < STAGES; i++) mbar_init(sfready + i, 1);
+        for (int i = 0; i < STAGES; i++) mbar_init(sfready + i, 2);   // one arrival per scale-factor warp
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -482,10 +483,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 mbar_wait(drain, 0, p.wait_ns);
             }
         }
-    } else if (warp == 6) {
+    } else if (warp >= 6) {
         // ---------------------------------------------------------- scale-factor copies (first CTA)
         // Issued apart from the MMA thread: a tcgen05.cp stalls the thread that
-        // issues it, but runs alongside the MMAs in the tensor pipe.
+        // issues it, but runs alongside the MMAs in the tensor pipe.  Two warps
+        // share the atoms of a stage (even / odd atoms).
+        const int par = warp - 6;
         if (NSF && lane == 0 && rank == 0) {
             int it = 0;
             bool ok = true;
@@ -509,7 +512,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                         const uint8_t *sf = smem + s * STAGE_BYTES + A_STAGE + B_STAGE;
                         const uint32_t group = tmem + TMEM_SF + SF_GROUP_COLS * (uint32_t)(it & 1);
                         tc_fence_after();
-                        for (int a = 0; a < natoms; a++) {
+                        for (int a = par; a < natoms; a += 2) {
                             const uint32_t base = group + SF_SLOT_COLS * (uint32_t)a;
                             tc_cp_pair(base, sdesc_sf(sf + 512 * a));
                             tc_cp_pair(base + 4, sdesc_sf(sf + 2048 + 512 * a));
