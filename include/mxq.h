@@ -241,6 +241,30 @@ mxq_status mxq_quantize_lowrank(const void *x, int32_t xdtype, int64_t m, int64_
                                 float *tensor_scale, void *tp, void *workspace,
                                 size_t workspace_bytes, void *stream);
 
+/* Same as mxq_quantize_lowrank, but without a workspace argument: the
+ * scratch it needs (the tensor-amax word and the m x r fp32 low-rank
+ * activation, 256 + 4*m*r bytes) lives in a 4 MiB array that the library
+ * keeps in device memory, one per GPU that loads it, until the process
+ * exits.  The pages describe no such call; it exists for callers that
+ * cannot allocate device memory themselves: code embedded in a host
+ * application that owns every device buffer and hands the library only its
+ * inputs and outputs, and latency-bound callers for whom a cudaMalloc,
+ * which may synchronize the device, is not acceptable.
+ *   Limit: 256 + 4*m*r <= 4 MiB (m*r <= 1,048,512, e.g. m <= 32,767 rows
+ *     at rank 32); larger calls return MXQ_ENOSPACE and launch nothing.
+ *   The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   All calls share the array: calls whose work overlaps on the GPU (other
+ *     streams, other host threads) race on it and must be ordered by the
+ *     caller.  The amax word is cleared on every call; nothing else in the
+ *     array needs to start at zero.
+ *   The call itself allocates and frees nothing.
+ * Other arguments, results and errors as mxq_quantize_lowrank. */
+mxq_status mxq_quantize_lowrank_noalloc(const void *x, int32_t xdtype, int64_t m, int64_t k,
+                                        int32_t fmt, int32_t hadamard_b, const void *l1, int32_t r,
+                                        const float *w_tensor_scale, void *codes, void *scales,
+                                        float *tensor_scale, void *tp, void *stream);
+
 /* Re-lays the up-projection l2 (r x n bf16, device) as the GEMM operand
  * l2p (n x 64 bf16, device): row j of l2p holds l2[0..r-1][j], zeros up to
  * 32, then the same 32 values again (the operand of the split high/low

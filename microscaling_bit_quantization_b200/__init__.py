@@ -33,7 +33,7 @@ EXPORTS = ("mxq_status_string", "mxq_device_supported", "mxq_check", "mxq_codes_
            "mxq_quantize_workspace_bytes", "mxq_quantize", "mxq_dequantize", "mxq_hadamard_block", "mxq_cast",
            "mxq_select_workspace_bytes", "mxq_select_weight_format", "mxq_lowrank_down", "mxq_lowrank_packed_bytes",
            "mxq_lowrank_down_packed", "mxq_lowrank_pack_t", "mxq_lowrank_pack_l2", "mxq_qlinear", "mxq_route",
-           "mxq_quantize_lowrank_workspace_bytes", "mxq_quantize_lowrank")
+           "mxq_quantize_lowrank_workspace_bytes", "mxq_quantize_lowrank", "mxq_quantize_lowrank_noalloc")
 
 
 class MxqError(RuntimeError):
@@ -76,6 +76,7 @@ def _load():
         "mxq_route": (i32, [P, i32, i32, i32, i32, i32]),
         "mxq_quantize_lowrank_workspace_bytes": (i32, [i64, i32, psz]),
         "mxq_quantize_lowrank": (i32, [P, i32, i64, i64, i32, i32, P, i32, P, P, P, P, P, P, sz, P]),
+        "mxq_quantize_lowrank_noalloc": (i32, [P, i32, i64, i64, i32, i32, P, i32, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -300,6 +301,24 @@ def quantize_lowrank(x: torch.Tensor, fmt: int, l1: torch.Tensor, wq: QTensor, h
                                   _ptr(wq.tensor_scale) if wq is not None else None, _ptr(q.codes), _ptr(q.scales),
                                   _ptr(q.tensor_scale), _ptr(tp), _ptr(workspace), wsb, _stream(stream)),
         "mxq_quantize_lowrank")
+    return q, tp
+
+
+def quantize_lowrank_noalloc(x: torch.Tensor, fmt: int, l1: torch.Tensor, wq: QTensor, hadamard_b: int = 0,
+                             out: QTensor = None, tp: torch.Tensor = None, stream=None):
+    """quantize_lowrank without a workspace: the library's own 4 MiB device
+    scratch array is used (see mxq_quantize_lowrank_noalloc in mxq.h)."""
+    _require_cuda(x, l1)
+    x, l1 = x.contiguous(), l1.contiguous()
+    m, k = x.shape
+    r = l1.shape[1]
+    q = out if out is not None else alloc_qtensor(fmt, m, k, MMA, x.device)
+    if tp is None:
+        tp = torch.empty((m, 64), dtype=torch.bfloat16, device=x.device)
+    _ok(_lib.mxq_quantize_lowrank_noalloc(_ptr(x), _dtype_code(x), m, k, fmt, hadamard_b, _ptr(l1), r,
+                                          _ptr(wq.tensor_scale) if wq is not None else None, _ptr(q.codes),
+                                          _ptr(q.scales), _ptr(q.tensor_scale), _ptr(tp), _stream(stream)),
+        "mxq_quantize_lowrank_noalloc")
     return q, tp
 
 

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/mxq.h"
 #include "mxq_formats.cuh"
 #include "mxq_internal.h"
@@ -282,6 +284,53 @@ mxq_status mxq_qlinear(const mxq_qtensor *xq, const mxq_qtensor *wq, const void 
     op.y = y;
     op.y_bf16 = ydtype == MXQ_BF16;
     return from_cuda(launch_qlinear(op, (cudaStream_t)stream));
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of mxq_quantize_lowrank: its scratch (the tensor-amax
+// word and the fp32 low-rank activation) lives in this file-scope device
+// array, which every GPU that loads the library holds until the process ends.
+// In host code the array's name is only a stand-in for the device object, so
+// the device address is looked up once per device (with that device current)
+// and cached.
+namespace {
+constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;   // 4 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+constexpr int kNoAllocMaxDevices = 64;
+void *g_noalloc_addr[kNoAllocMaxDevices];
+std::mutex g_noalloc_lock;
+
+mxq_status noalloc_scratch(void **ptr) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MXQ_ECUDA;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return MXQ_EUNSUPPORTED;
+    std::lock_guard<std::mutex> guard(g_noalloc_lock);
+    if (!g_noalloc_addr[dev]) {
+        void *a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_noalloc_scratch) != cudaSuccess || !a) return MXQ_ECUDA;
+        g_noalloc_addr[dev] = a;
+    }
+    *ptr = g_noalloc_addr[dev];
+    return MXQ_OK;
+}
+}  // namespace
+
+extern "C" {
+
+mxq_status mxq_quantize_lowrank_noalloc(const void *x, int32_t xdtype, int64_t m, int64_t k, int32_t fmt,
+                                        int32_t hadamard_b, const void *l1, int32_t r,
+                                        const float *w_tensor_scale, void *codes, void *scales,
+                                        float *tensor_scale, void *tp, void *stream) {
+    size_t need = 0;
+    if (mxq_quantize_lowrank_workspace_bytes(m, r, &need) != MXQ_OK) return MXQ_EINVAL;
+    if (need > kNoAllocScratchBytes) return MXQ_ENOSPACE;
+    void *scratch = nullptr;
+    const mxq_status st = noalloc_scratch(&scratch);
+    if (st != MXQ_OK) return st;
+    return mxq_quantize_lowrank(x, xdtype, m, k, fmt, hadamard_b, l1, r, w_tensor_scale, codes, scales, tensor_scale,
+                                tp, scratch, kNoAllocScratchBytes, stream);
 }
 
 int32_t mxq_route(const uint8_t *table, int32_t n_layers, int32_t n_intervals, int32_t layer, int32_t step,
