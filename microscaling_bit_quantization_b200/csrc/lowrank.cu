@@ -167,6 +167,145 @@ __global__ void k_pack_t(const float *__restrict__ t, int r, int64_t m, const fl
     tp[row * 64 + 32 + j] = lo;
 }
 
+// ---------------------------------------------------------------------------
+// Staged variant for bf16 x (k % 64 == 0, r % 8 == 0): a CTA of 4 warps
+// owns a 16-row strip and walks K in 64-wide chunks that cp.async stages into
+// shared memory, kLsStages chunks in flight; warp w takes the chunk's k16 step
+// w.  Fragments come from shared memory through ldmatrix (A) and
+// ldmatrix.trans (B, straight from L1's k x r rows); rows are stored with an
+// XOR swizzle of their 16-byte pieces so the eight rows an ldmatrix reads hit
+// distinct banks.  max |x| comes from each thread's own staged piece.
+constexpr int kLsStages = 12, kLsThreads = 128;
+constexpr int kLsX = 16 * 128;            // 16 rows x 64 bf16
+constexpr int kLsL1 = 64 * 64;            // 64 k-rows x 32 bf16 (zero-padded past r)
+constexpr int kLsStage = kLsX + kLsL1;
+constexpr int kLsSmem = kLsStages * kLsStage;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
+    const int n = valid ? 16 : 0;   // zero-fill rows past m
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+// byte offset of 16-byte piece p of row `row` in a 128-byte-row tile (x) / 64-byte-row tile (L1)
+__device__ __forceinline__ uint32_t xs_off(int row, int p) { return row * 128 + ((p ^ (row & 7)) << 4); }
+__device__ __forceinline__ uint32_t ls_off(int row, int p) { return row * 64 + ((p ^ ((row >> 1) & 3)) << 4); }
+
+template <int MODE>
+__global__ void __launch_bounds__(kLsThreads) k_lowrank_staged(const __nv_bfloat16 *__restrict__ x, int64_t m, int64_t k,
+                                                              const __nv_bfloat16 *__restrict__ l1, int r,
+                                                              float *__restrict__ t, const float *xs, const float *ws,
+                                                              __nv_bfloat16 *__restrict__ tp, unsigned int *amax_word) {
+    extern __shared__ __align__(128) uint8_t ls_smem[];
+    __shared__ float red[4][16][33];
+    __shared__ float wmax[4];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t row0 = (int64_t)blockIdx.x * 16;
+    const int nchunks = (int)(k >> 6);
+    const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(ls_smem);
+    const int pieces_l1 = r >> 3;   // 16-byte pieces per L1 row
+    // L1 tiles: columns past r stay zero
+    for (int i = tid; i < kLsStages * kLsL1 / 16; i += kLsThreads) {
+        const int st = i / (kLsL1 / 16), q = i % (kLsL1 / 16);
+        *reinterpret_cast<uint4 *>(ls_smem + st * kLsStage + kLsX + q * 16) = make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();
+    // thread tid stages x piece (row tid / 8, piece tid % 8) and L1 pieces tid, tid + 128
+    const int xr = tid >> 3, xp = tid & 7;
+    const bool xrow_ok = row0 + xr < m;
+    const __nv_bfloat16 *xsrc = x + (row0 + (xrow_ok ? xr : 0)) * k + xp * 8;
+    auto issue = [&](int c) {
+        const uint32_t st = sbase + (uint32_t)((c % kLsStages) * kLsStage);
+        cp_async16(st + xs_off(xr, xp), xsrc + (int64_t)c * 64, xrow_ok);
+        for (int i = tid; i < 64 * pieces_l1; i += kLsThreads) {
+            const int kr = i / pieces_l1, pc = i % pieces_l1;
+            cp_async16(st + kLsX + ls_off(kr, pc), l1 + ((int64_t)c * 64 + kr) * r + pc * 8, true);
+        }
+    };
+#pragma unroll 1
+    for (int c = 0; c < kLsStages - 1; c++) {
+        if (c < nchunks) issue(c);
+        cp_async_commit();
+    }
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; i++)
+#pragma unroll
+        for (int j = 0; j < 4; j++) acc[i][j] = 0.0f;
+    float am = 0.0f;
+    // ldmatrix row addresses (lane supplies row lane % 8 of matrix lane / 8)
+    const int mi = lane >> 3, mr = lane & 7;
+    const int a_row = mr + 8 * (mi & 1), a_piece = 2 * warp + (mi >> 1);
+    const int b_row = 16 * warp + mr + 8 * (mi & 1);
+#pragma unroll 1
+    for (int c = 0; c < nchunks; c++) {
+        cp_async_wait<kLsStages - 2>();
+        __syncthreads();
+        if (c + kLsStages - 1 < nchunks) issue(c + kLsStages - 1);
+        cp_async_commit();
+        const uint32_t st = sbase + (uint32_t)((c % kLsStages) * kLsStage);
+        if (MODE == kLrTAmax) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(ls_smem + (c % kLsStages) * kLsStage + xs_off(xr, xp));
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; j++)
+                am = fmaxf(am, fmaxf(fabsf(__uint_as_float(w4[j] << 16)), fabsf(__uint_as_float(w4[j] & 0xFFFF0000u))));
+        }
+        uint32_t a[4], b01[4], b23[4];
+        ldsm_x4(st + xs_off(a_row, a_piece), a);
+        ldsm_x4_trans(st + kLsX + ls_off(b_row, mi >> 1), b01);
+        ldsm_x4_trans(st + kLsX + ls_off(b_row, 2 + (mi >> 1)), b23);
+        mma_m16n8k16_bf16(acc[0], a, b01[0], b01[1]);
+        mma_m16n8k16_bf16(acc[1], a, b01[2], b01[3]);
+        mma_m16n8k16_bf16(acc[2], a, b23[0], b23[1]);
+        mma_m16n8k16_bf16(acc[3], a, b23[2], b23[3]);
+    }
+    cp_async_wait<0>();
+    const int g = lane >> 2, tq = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 4; nt++) {
+        red[warp][g][nt * 8 + tq * 2] = acc[nt][0];
+        red[warp][g][nt * 8 + tq * 2 + 1] = acc[nt][1];
+        red[warp][g + 8][nt * 8 + tq * 2] = acc[nt][2];
+        red[warp][g + 8][nt * 8 + tq * 2 + 1] = acc[nt][3];
+    }
+    if (MODE == kLrTAmax) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
+        if (lane == 0) wmax[warp] = am;
+    }
+    __syncthreads();
+    if (MODE == kLrTAmax && tid == 0) {
+        const float v = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+        if (v > 0.0f) atomicMax(amax_word, __float_as_uint(v));
+    }
+    float alpha = 1.0f;
+    if (MODE == kLrPacked && xs) alpha = __fmul_rn(*xs, *ws);
+    for (int i = tid; i < 16 * 32; i += kLsThreads) {
+        const int rr = i >> 5, cc = i & 31;
+        const int64_t row = row0 + rr;
+        if (row >= m) continue;
+        const float sum = __fadd_rn(__fadd_rn(red[0][rr][cc], red[1][rr][cc]), __fadd_rn(red[2][rr][cc], red[3][rr][cc]));
+        if (MODE != kLrPacked) {
+            if (cc < r) t[row * r + cc] = sum;
+        } else {
+            const float u = cc < r ? (xs ? __fdiv_rn(sum, alpha) : sum) : 0.0f;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(u);
+            tp[row * 64 + cc] = hi;
+            tp[row * 64 + 32 + cc] = __float2bfloat16_rn(__fsub_rn(u, __bfloat162float(hi)));
+        }
+    }
+}
+
 }  // namespace
 
 template <typename T>
@@ -185,6 +324,21 @@ cudaError_t launch_lowrank_down(const void *x, bool bf16, int64_t m, int64_t k, 
     const int mode = tp ? kLrPacked : (amax_word ? kLrTAmax : kLrT);
     const __nv_bfloat16 *l = (const __nv_bfloat16 *)l1;
     __nv_bfloat16 *tpb = (__nv_bfloat16 *)tp;
+    if (bf16 && k % 64 == 0 && r % 8 == 0 && (reinterpret_cast<uintptr_t>(l1) & 15u) == 0) {
+        static bool configured = false;
+        if (!configured) {
+            cudaFuncSetAttribute(k_lowrank_staged<kLrT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kLsSmem);
+            cudaFuncSetAttribute(k_lowrank_staged<kLrPacked>, cudaFuncAttributeMaxDynamicSharedMemorySize, kLsSmem);
+            cudaFuncSetAttribute(k_lowrank_staged<kLrTAmax>, cudaFuncAttributeMaxDynamicSharedMemorySize, kLsSmem);
+            configured = true;
+        }
+        const __nv_bfloat16 *xb = (const __nv_bfloat16 *)x;
+        if (mode == kLrT) k_lowrank_staged<kLrT><<<grid, kLsThreads, kLsSmem, s>>>(xb, m, k, l, r, t, xs, ws, tpb, amax_word);
+        else if (mode == kLrPacked)
+            k_lowrank_staged<kLrPacked><<<grid, kLsThreads, kLsSmem, s>>>(xb, m, k, l, r, t, xs, ws, tpb, amax_word);
+        else k_lowrank_staged<kLrTAmax><<<grid, kLsThreads, kLsSmem, s>>>(xb, m, k, l, r, t, xs, ws, tpb, amax_word);
+        return cudaGetLastError();
+    }
     if (bf16) launch_lr(mode, grid, (const __nv_bfloat16 *)x, m, k, l, r, t, xs, ws, tpb, amax_word, s);
     else launch_lr(mode, grid, (const float *)x, m, k, l, r, t, xs, ws, tpb, amax_word, s);
     return cudaGetLastError();

@@ -96,31 +96,6 @@ struct QuantArgs {
     __nv_bfloat16 *tp;
 };
 
-// Packs one row of the low-rank activation: u_j = t_j / alpha (alpha = 1
-// when `divide` is false), hi = bf16(u), lo = bf16(u - hi), zeros past r.
-__device__ __forceinline__ void pack_t_row(const float *t, int r, bool divide, float alpha, __nv_bfloat16 *tp) {
-    uint32_t hi[16], lo[16];
-#pragma unroll
-    for (int j = 0; j < 32; j += 2) {
-        float u0 = j < r ? t[j] : 0.0f, u1 = j + 1 < r ? t[j + 1] : 0.0f;
-        if (divide) {
-            u0 = __fdiv_rn(u0, alpha);
-            u1 = __fdiv_rn(u1, alpha);
-        }
-        __nv_bfloat162 h = __floats2bfloat162_rn(u0, u1);
-        float2 hf = __bfloat1622float2(h);
-        __nv_bfloat162 l = __floats2bfloat162_rn(__fsub_rn(u0, hf.x), __fsub_rn(u1, hf.y));
-        hi[j >> 1] = *reinterpret_cast<uint32_t *>(&h);
-        lo[j >> 1] = *reinterpret_cast<uint32_t *>(&l);
-    }
-    uint4 *dst = reinterpret_cast<uint4 *>(tp);
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-        dst[i] = make_uint4(hi[4 * i], hi[4 * i + 1], hi[4 * i + 2], hi[4 * i + 3]);
-        dst[4 + i] = make_uint4(lo[4 * i], lo[4 * i + 1], lo[4 * i + 2], lo[4 * i + 3]);
-    }
-}
-
 template <typename T, int F>
 __global__ void __launch_bounds__(kThreads) k_quantize(const T *__restrict__ x, QuantArgs a) {
     constexpr int BLK = fmt_block(F) ? fmt_block(F) : 16;
@@ -152,10 +127,6 @@ __global__ void __launch_bounds__(kThreads) k_quantize(const T *__restrict__ x, 
         const int64_t col0 = (c - row * chunks_per_row) << 4;
         float amax = amax16(v);
         if (G > 1) amax = group_max<G>(amax);
-        if (a.tp && valid && col0 == 0) {
-            const bool ts = F == kNVFP4 || F == kFP8Tensor;
-            pack_t_row(a.t + row * a.r, a.r, ts, ts ? __fmul_rn(s_t, *a.w_ts) : 1.0f, a.tp + row * 64);
-        }
 
         if (F == kMXFP8 || F == kMXFP4) {
             float inv = 0.0f;
@@ -277,6 +248,19 @@ __global__ void __launch_bounds__(kThreads) k_quantize(const T *__restrict__ x, 
                 }
                 *reinterpret_cast<uint4 *>(a.codes + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
             }
+        }
+    }
+    if (a.tp) {
+        // packed low-rank operand, one row per warp, one value per lane:
+        // u = t / alpha, hi = bf16(u), lo = bf16(u - hi), zeros past r
+        const bool ts = F == kNVFP4 || F == kFP8Tensor;
+        const float alpha = ts ? __fmul_rn(s_t, *a.w_ts) : 1.0f;
+        for (int64_t row = warp; row < a.rows; row += nwarps) {
+            float u = lane < a.r ? a.t[row * a.r + lane] : 0.0f;
+            if (ts) u = __fdiv_rn(u, alpha);
+            const __nv_bfloat16 hi = __float2bfloat16_rn(u);
+            a.tp[row * 64 + lane] = hi;
+            a.tp[row * 64 + 32 + lane] = __float2bfloat16_rn(__fsub_rn(u, __bfloat162float(hi)));
         }
     }
 }
