@@ -129,13 +129,22 @@ def _dist_init():
 
 
 def _max_over_ranks(value, world):
+    """Max of a per-rank scalar over all ranks (the job's time is its slowest rank)."""
     if world == 1:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(ms_local, world, flop_per_rank):
+    """(max ms over ranks, whole-job TFLOP/s): every rank runs the same layer on
+    its own batch, so the job does world * flop_per_rank per step."""
+    ms = _max_over_ranks(ms_local, world)
+    return ms, world * flop_per_rank / (ms * 1e-3) / 1e12
 
 
 def _barrier(world):
@@ -262,7 +271,7 @@ def run_ours(args, world, rank, local):
     _barrier(world)
     clocks = sampler.stop()
     ms_local = start.elapsed_time(end) / args.steps
-    ms = _max_over_ranks(ms_local, world)
+    ms, value = job_throughput(ms_local, world, FLOP_STEP)
     assert mxq.check() == 0
 
     # ---- per-kernel durations of the dominant kernel (GEMM) and the quantizer, on the launch stream
@@ -335,7 +344,6 @@ def run_ours(args, world, rank, local):
                "sample": o.desc + "; 10 steps"}
 
     if rank == 0:
-        value = world * FLOP_STEP / (ms * 1e-3) / 1e12
         line = {
             "metric": "qlinear TFLOPS (NVFP4 W4A4 + rank-32 low-rank), whole step",
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

@@ -127,6 +127,75 @@ __device__ __forceinline__ int int_code(float v, float s, int qmax) {
     return q > qmax ? qmax : (q < -qmax ? -qmax : q);
 }
 
+// ----------------------------------------------------------------- codes of quotients
+//
+// Codes of RN(v / d) for many v and one divisor d, without an IEEE division
+// per element.  y = RN(1/d) (correctly rounded reciprocal) and q = RN(|v| y)
+// give q within a relative 2^-23 + 2^-48 of |v|/d, so RN(|v|/d) lies in
+// [q (1 - 2^-22), q (1 + 2^-22)].  Every code function used here is a
+// monotone function of the magnitude, so when the codes of the bracket ends
+// RN(q (1 - 2^-20)) and RN(q (1 + 2^-20)) (which enclose that interval)
+// agree, the code of RN(|v|/d) is that code; otherwise a code boundary (or an
+// exact tie) lies inside the bracket and the quotient is computed by exact
+// division.  Signs are applied afterwards (RN(-x) = -RN(x)).  When q is an
+// fp32 subnormal (|v|/d < 2^-126) the relative bound does not hold, but both
+// ends and the true quotient are then far below the smallest nonzero code.
+struct Recip {
+    float d, y;
+    bool fast;   // d in [2^-120, 2^120]: y finite and normal, no overflow in q
+};
+__device__ __forceinline__ Recip recip_of(float d) {
+    Recip r;
+    r.d = d;
+    r.fast = d >= 7.52316384526264e-37f && d <= 1.329227995784916e36f;
+    r.y = r.fast ? __frcp_rn(d) : 0.0f;
+    return r;
+}
+constexpr float kBracketLo = 0.99999904632568359375f;   // 1 - 2^-20
+constexpr float kBracketHi = 1.00000095367431640625f;   // 1 + 2^-20
+
+// E2M1 codes of RN(v0/d), RN(v1/d) as one byte (v0 in the low nibble).
+__device__ __forceinline__ uint32_t e2m1x2_quot(float v0, float v1, const Recip &r) {
+    const uint32_t sign = ((__float_as_uint(v0) >> 31) << 3) | ((__float_as_uint(v1) >> 31) << 7);
+    const float a0 = fabsf(v0), a1 = fabsf(v1);
+    if (r.fast) {
+        const float q0 = __fmul_rn(a0, r.y), q1 = __fmul_rn(a1, r.y);
+        const uint32_t lo = enc_e2m1x2(__fmul_rn(q0, kBracketLo), __fmul_rn(q1, kBracketLo));
+        const uint32_t hi = enc_e2m1x2(__fmul_rn(q0, kBracketHi), __fmul_rn(q1, kBracketHi));
+        if (lo == hi) return lo | sign;
+    }
+    return enc_e2m1x2(__fdiv_rn(a0, r.d), __fdiv_rn(a1, r.d)) | sign;
+}
+
+// E4M3 code of RN(v/d).
+__device__ __forceinline__ uint32_t e4m3_quot(float v, const Recip &r) {
+    const uint32_t sign = (__float_as_uint(v) >> 31) << 7;
+    const float a = fabsf(v);
+    if (r.fast) {
+        const float q = __fmul_rn(a, r.y);
+        const uint32_t lo = enc_e4m3(__fmul_rn(q, kBracketLo)), hi = enc_e4m3(__fmul_rn(q, kBracketHi));
+        if (lo == hi) return lo | sign;
+    }
+    return (uint32_t)enc_e4m3(__fdiv_rn(a, r.d)) | sign;
+}
+
+// Symmetric integer code clamp(RNE(RN(v/s)), -qmax, qmax); 0 when s == 0.
+__device__ __forceinline__ int int_code_quot(float v, const Recip &r, int qmax) {
+    if (r.d == 0.0f) return 0;
+    const float a = fabsf(v);
+    int c;
+    bool done = false;
+    if (r.fast) {
+        const float q = __fmul_rn(a, r.y);
+        const int lo = __float2int_rn(__fmul_rn(q, kBracketLo)), hi = __float2int_rn(__fmul_rn(q, kBracketHi));
+        c = lo;
+        done = lo == hi;
+    }
+    if (!done) c = __float2int_rn(__fdiv_rn(a, r.d));
+    c = c > qmax ? qmax : c;
+    return v < 0.0f ? -c : c;
+}
+
 // ----------------------------------------------------------------- loads
 
 // 16 consecutive elements as fp32 (bf16 widened exactly).

@@ -179,6 +179,7 @@ __global__ void __launch_bounds__(kThreads) k_quantize(const T *__restrict__ x, 
             float d;
             uint32_t e4 = nvfp4_block_scale(amax, s_t, d);
             if (valid) {
+                const Recip rd = recip_of(d);
                 uint32_t w[2];
 #pragma unroll
                 for (int j = 0; j < 2; j++) {
@@ -186,8 +187,7 @@ __global__ void __launch_bounds__(kThreads) k_quantize(const T *__restrict__ x, 
 #pragma unroll
                     for (int k = 0; k < 4; k++) {
                         uint32_t byte = 0;
-                        if (e4)
-                            byte = enc_e2m1x2(__fdiv_rn(v[8 * j + 2 * k], d), __fdiv_rn(v[8 * j + 2 * k + 1], d));
+                        if (e4) byte = e2m1x2_quot(v[8 * j + 2 * k], v[8 * j + 2 * k + 1], rd);
                         acc |= byte << (8 * k);
                     }
                     w[j] = acc;
@@ -207,6 +207,7 @@ __global__ void __launch_bounds__(kThreads) k_quantize(const T *__restrict__ x, 
             }
         } else if (F == kINT4G32 || F == kINT4G64) {
             float s = __fdiv_rn(amax, 7.0f);
+            const Recip rs = recip_of(s);
             if (valid) {
                 if (a.layout == 0) {
                     uint32_t w[2];
@@ -214,7 +215,7 @@ __global__ void __launch_bounds__(kThreads) k_quantize(const T *__restrict__ x, 
                     for (int j = 0; j < 2; j++) {
                         uint32_t acc = 0;
 #pragma unroll
-                        for (int k = 0; k < 8; k++) acc |= ((uint32_t)int_code(v[8 * j + k], s, 7) & 0xFu) << (4 * k);
+                        for (int k = 0; k < 8; k++) acc |= ((uint32_t)int_code_quot(v[8 * j + k], rs, 7) & 0xFu) << (4 * k);
                         w[j] = acc;
                     }
                     *reinterpret_cast<uint2 *>(a.codes + c * 8) = make_uint2(w[0], w[1]);
@@ -224,7 +225,7 @@ __global__ void __launch_bounds__(kThreads) k_quantize(const T *__restrict__ x, 
                     for (int j = 0; j < 4; j++) {
                         uint32_t acc = 0;
 #pragma unroll
-                        for (int k = 0; k < 4; k++) acc |= ((uint32_t)int_code(v[4 * j + k], s, 7) & 0xFFu) << (8 * k);
+                        for (int k = 0; k < 4; k++) acc |= ((uint32_t)int_code_quot(v[4 * j + k], rs, 7) & 0xFFu) << (8 * k);
                         w[j] = acc;
                     }
                     *reinterpret_cast<uint4 *>(a.codes + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -238,12 +239,13 @@ __global__ void __launch_bounds__(kThreads) k_quantize(const T *__restrict__ x, 
             }
         } else if (F == kFP8Tensor) {
             if (valid) {
+                const Recip rs = recip_of(s_t);
                 uint32_t w[4];
 #pragma unroll
                 for (int j = 0; j < 4; j++) {
                     uint32_t acc = 0;
 #pragma unroll
-                    for (int k = 0; k < 4; k++) acc |= (uint32_t)enc_e4m3(__fdiv_rn(v[4 * j + k], s_t)) << (8 * k);
+                    for (int k = 0; k < 4; k++) acc |= e4m3_quot(v[4 * j + k], rs) << (8 * k);
                     w[j] = acc;
                 }
                 *reinterpret_cast<uint4 *>(a.codes + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -288,6 +290,7 @@ __global__ void __launch_bounds__(kThreads) k_quantize_int8_row(const T *__restr
         }
         m = group_max<32>(m);
         const float s = __fdiv_rn(m, 127.0f);
+        const Recip rs = recip_of(s);
         for (int64_t c0 = 0; c0 < cpr; c0 += 32) {
             int64_t c = c0 + lane;
             float v[16];
@@ -303,7 +306,7 @@ __global__ void __launch_bounds__(kThreads) k_quantize_int8_row(const T *__restr
                 for (int j = 0; j < 4; j++) {
                     uint32_t acc = 0;
 #pragma unroll
-                    for (int k = 0; k < 4; k++) acc |= ((uint32_t)int_code(v[4 * j + k], s, 127) & 0xFFu) << (8 * k);
+                    for (int k = 0; k < 4; k++) acc |= ((uint32_t)int_code_quot(v[4 * j + k], rs, 127) & 0xFFu) << (8 * k);
                     w[j] = acc;
                 }
                 *reinterpret_cast<uint4 *>(a.codes + (row * cpr + c) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
