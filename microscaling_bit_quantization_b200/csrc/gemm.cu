@@ -751,6 +751,22 @@ cudaError_t launch_qlinear(const GemmOperands &op, cudaStream_t s) {
     }
 }
 
+cudaError_t error_word_address(unsigned int **ptr) {
+    static unsigned int *addr[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_error_word);
+        if (e != cudaSuccess) return e;
+        addr[dev] = reinterpret_cast<unsigned int *>(p);
+    }
+    *ptr = addr[dev];
+    return cudaSuccess;
+}
+
 cudaError_t read_and_clear_error(unsigned int *value) {
     unsigned int zero = 0;
     cudaError_t e = cudaMemcpyFromSymbol(value, g_error_word, sizeof(unsigned int));

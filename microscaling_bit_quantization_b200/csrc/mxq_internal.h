@@ -59,7 +59,9 @@ struct GemmOperands {
 };
 cudaError_t launch_qlinear(const GemmOperands &op, cudaStream_t s);
 
-// Device error word (bounded waits that ran out); read-and-clear.
+// Device error word (bounded waits that ran out); read-and-clear, and its
+// device address on the current device (for kernels of other files).
 cudaError_t read_and_clear_error(unsigned int *value);
+cudaError_t error_word_address(unsigned int **ptr);
 
 }  // namespace mxq

@@ -10,6 +10,8 @@
 // Loads are 16-byte vectors; codes are stored as 8- or 16-byte vectors.
 #include <cuda_runtime.h>
 
+#include <cstring>
+
 #include "mxq_formats.cuh"
 #include "mxq_internal.h"
 
@@ -55,28 +57,6 @@ __device__ __forceinline__ uint32_t gather4(uint32_t byte) {
     return (byte & 0xFFu) | ((b1 & 0xFFu) << 8) | ((b2 & 0xFFu) << 16) | ((b3 & 0xFFu) << 24);
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kThreads) k_amax(const T *__restrict__ x, int64_t total_chunks,
-                                                  int hadamard_b, unsigned int *__restrict__ amax_word) {
-    const int lane = lane_id();
-    const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * kThreads) >> 5;
-    const int64_t tiles = (total_chunks + 31) >> 5;
-    float m = 0.0f;
-    for (int64_t t = warp; t < tiles; t += nwarps) {
-        int64_t c = (t << 5) + lane;
-        float v[16];
-        if (c < total_chunks) load16(x + c * 16, v);
-        else {
-#pragma unroll
-            for (int i = 0; i < 16; i++) v[i] = 0.0f;
-        }
-        if (hadamard_b) hadamard_chunk(v, hadamard_b, lane);
-        m = fmaxf(m, amax16(v));
-    }
-    cta_max_to_word(m, amax_word);
-}
-
 // ------------------------------------------------------------------ quantize
 
 struct QuantArgs {
@@ -94,17 +74,88 @@ struct QuantArgs {
     int r;
     const float *w_ts;
     __nv_bfloat16 *tp;
+    unsigned int *err;       // device error word (a bounded wait that ran out)
 };
+
+// Staged input: persistent CTAs bring 16 KB tiles of x into a ring of
+// kQStages shared-memory buffers with one cp.async.bulk each (completion on
+// an mbarrier), then encode from shared memory.
+constexpr int kQStages = 4, kQTileBytes = 16384, kQSmem = kQStages * kQTileBytes;
+constexpr unsigned int kErrTimeoutQuant = 8u;
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void q_bar_init(uint64_t *bar) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(bar)));
+}
+__device__ __forceinline__ void q_bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_addr(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
+}
+// Bounded wait (about 2 s of polling) for phase `parity` of the barrier.
+__device__ __forceinline__ bool q_bar_wait(uint64_t *bar, uint32_t parity) {
+    for (long long i = 0; i < (1ll << 26); i++) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_addr(bar)), "r"(parity)
+            : "memory");
+        if (ok) return true;
+    }
+    return false;
+}
+
+__device__ __forceinline__ void load16_shared(const float *p, float v[16]) {
+    const float4 *q = reinterpret_cast<const float4 *>(p);
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        float4 t = q[i];
+        v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
+    }
+}
+__device__ __forceinline__ void load16_shared(const __nv_bfloat16 *p, float v[16]) {
+    const uint4 *q = reinterpret_cast<const uint4 *>(p);
+#pragma unroll
+    for (int i = 0; i < 2; i++) {
+        uint4 t = q[i];
+        uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+            v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+    }
+}
 
 template <typename T, int F>
 __global__ void __launch_bounds__(kThreads) k_quantize(const T *__restrict__ x, QuantArgs a) {
     constexpr int BLK = fmt_block(F) ? fmt_block(F) : 16;
     constexpr int G = BLK ? BLK / 16 : 1;   // lanes per quantization block
+    constexpr int CPT = kQTileBytes / (16 * (int)sizeof(T));   // chunks per staged tile
+    extern __shared__ __align__(128) uint8_t q_smem[];
+    __shared__ uint64_t q_bars[kQStages];
     const int lane = lane_id();
     const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * kThreads) >> 5;
-    const int64_t tiles = (a.total_chunks + 31) >> 5;
+    const int64_t ntiles = (a.total_chunks + CPT - 1) / CPT;
     const int64_t chunks_per_row = a.cols >> 4;
+    auto issue = [&](int64_t tile, int stage) {
+        const int64_t n = a.total_chunks - tile * CPT;
+        const uint32_t bytes = (uint32_t)((n < CPT ? n : CPT) * 16 * (int64_t)sizeof(T));
+        q_bulk_load(q_smem + stage * kQTileBytes, x + tile * CPT * 16, bytes, &q_bars[stage]);
+    };
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kQStages; i++) q_bar_init(&q_bars[i]);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (int i = 0; i < kQStages; i++) {
+            const int64_t tile = blockIdx.x + (int64_t)i * gridDim.x;
+            if (tile < ntiles) issue(tile, i);
+        }
+    }
+    __syncthreads();
 
     float s_t = 1.0f;
     if (F == kNVFP4 || F == kFP8Tensor) {
@@ -113,11 +164,23 @@ __global__ void __launch_bounds__(kThreads) k_quantize(const T *__restrict__ x, 
         if (blockIdx.x == 0 && threadIdx.x == 0) *a.tensor_scale = s_t;
     }
 
-    for (int64_t t = warp; t < tiles; t += nwarps) {
-        const int64_t c = (t << 5) + lane;
+    bool failed = false;
+    float tensor_max = 0.0f;
+    int64_t it = 0;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, it++) {
+      const int stage = (int)(it % kQStages);
+      if (!q_bar_wait(&q_bars[stage], (uint32_t)((it / kQStages) & 1))) {
+          failed = true;
+          break;
+      }
+      const T *tx = reinterpret_cast<const T *>(q_smem + stage * kQTileBytes);
+#pragma unroll 1
+      for (int jc = 0; jc < CPT / kThreads; jc++) {
+        const int cit = threadIdx.x + jc * kThreads;   // chunk within the tile
+        const int64_t c = tile * CPT + cit;
         const bool valid = c < a.total_chunks;
         float v[16];
-        if (valid) load16(x + c * 16, v);
+        if (valid) load16_shared(tx + cit * 16, v);
         else {
 #pragma unroll
             for (int i = 0; i < 16; i++) v[i] = 0.0f;
@@ -126,6 +189,10 @@ __global__ void __launch_bounds__(kThreads) k_quantize(const T *__restrict__ x, 
         const int64_t row = c / chunks_per_row;
         const int64_t col0 = (c - row * chunks_per_row) << 4;
         float amax = amax16(v);
+        if (F == kNumFmt) {   // tensor-amax pass only
+            tensor_max = fmaxf(tensor_max, amax);
+            continue;
+        }
         if (G > 1) amax = group_max<G>(amax);
 
         if (F == kMXFP8 || F == kMXFP4) {
@@ -251,6 +318,20 @@ __global__ void __launch_bounds__(kThreads) k_quantize(const T *__restrict__ x, 
                 *reinterpret_cast<uint4 *>(a.codes + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
             }
         }
+      }
+      __syncthreads();   // the stage is free again
+      if (threadIdx.x == 0) {
+          const int64_t next = tile + (int64_t)kQStages * gridDim.x;
+          if (next < ntiles) issue(next, stage);
+      }
+    }
+    if (failed) {
+        if (threadIdx.x == 0) atomicOr(a.err, kErrTimeoutQuant);
+        return;
+    }
+    if (F == kNumFmt) {
+        cta_max_to_word(tensor_max, const_cast<unsigned int *>(a.amax_word));
+        return;
     }
     if (a.tp) {
         // packed low-rank operand, one row per warp, one value per lane:
@@ -574,27 +655,52 @@ static int sm_count_cached() {
     return count;
 }
 
+template <typename T, int F>
+static void launch_qf(const T *x, const QuantArgs &a, cudaStream_t s);
+
 cudaError_t launch_amax(const void *x, bool bf16, int64_t rows, int64_t cols, int hadamard_b,
                         unsigned int *amax_word, cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(amax_word, 0, sizeof(unsigned int), s);
     if (e != cudaSuccess) return e;
     int64_t chunks = rows * cols / 16;
     if (chunks == 0) return cudaSuccess;
-    int grid = grid_for((chunks + 31) / 32, sm_count_cached());
-    if (bf16) k_amax<__nv_bfloat16><<<grid, kThreads, 0, s>>>((const __nv_bfloat16 *)x, chunks, hadamard_b, amax_word);
-    else k_amax<float><<<grid, kThreads, 0, s>>>((const float *)x, chunks, hadamard_b, amax_word);
+    QuantArgs a;
+    memset(&a, 0, sizeof(a));
+    a.rows = rows;
+    a.cols = cols;
+    a.total_chunks = chunks;
+    a.hadamard_b = hadamard_b;
+    a.amax_word = amax_word;
+    e = error_word_address(&a.err);
+    if (e != cudaSuccess) return e;
+    if (bf16) launch_qf<__nv_bfloat16, kNumFmt>((const __nv_bfloat16 *)x, a, s);
+    else launch_qf<float, kNumFmt>((const float *)x, a, s);
     return cudaGetLastError();
+}
+
+template <typename T, int F>
+static void launch_qf(const T *x, const QuantArgs &a, cudaStream_t s) {
+    static bool configured = false;
+    if (!configured) {
+        cudaFuncSetAttribute(k_quantize<T, F>, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem);
+        configured = true;
+    }
+    constexpr int CPT = kQTileBytes / (16 * (int)sizeof(T));
+    const int64_t ntiles = (a.total_chunks + CPT - 1) / CPT;
+    const int64_t cap = (int64_t)sm_count_cached() * 3;   // 3 x 64 KB of ring per SM
+    const int grid = (int)(ntiles < cap ? ntiles : cap);
+    k_quantize<T, F><<<grid, kThreads, kQSmem, s>>>(x, a);
 }
 
 template <typename T>
 static void launch_q(int fmt, int grid, const T *x, const QuantArgs &a, cudaStream_t s) {
     switch (fmt) {
-    case kMXFP8: k_quantize<T, kMXFP8><<<grid, kThreads, 0, s>>>(x, a); break;
-    case kMXFP4: k_quantize<T, kMXFP4><<<grid, kThreads, 0, s>>>(x, a); break;
-    case kNVFP4: k_quantize<T, kNVFP4><<<grid, kThreads, 0, s>>>(x, a); break;
-    case kINT4G32: k_quantize<T, kINT4G32><<<grid, kThreads, 0, s>>>(x, a); break;
-    case kINT4G64: k_quantize<T, kINT4G64><<<grid, kThreads, 0, s>>>(x, a); break;
-    case kFP8Tensor: k_quantize<T, kFP8Tensor><<<grid, kThreads, 0, s>>>(x, a); break;
+    case kMXFP8: launch_qf<T, kMXFP8>(x, a, s); break;
+    case kMXFP4: launch_qf<T, kMXFP4>(x, a, s); break;
+    case kNVFP4: launch_qf<T, kNVFP4>(x, a, s); break;
+    case kINT4G32: launch_qf<T, kINT4G32>(x, a, s); break;
+    case kINT4G64: launch_qf<T, kINT4G64>(x, a, s); break;
+    case kFP8Tensor: launch_qf<T, kFP8Tensor>(x, a, s); break;
     case kINT8Row: {
         int g = grid_for(a.rows, sm_count_cached());
         k_quantize_int8_row<T><<<g, kThreads, 0, s>>>(x, a);
@@ -627,6 +733,8 @@ cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols
     a.r = pack ? pack->r : 0;
     a.w_ts = pack ? pack->w_ts : nullptr;
     a.tp = pack ? (__nv_bfloat16 *)pack->tp : nullptr;
+    e = error_word_address(&a.err);
+    if (e != cudaSuccess) return e;
     if (layout == 1 && fmt_byte_scales(fmt)) {
         int64_t S = cols / fmt_block(fmt);
         a.s_pad = (S + 15) / 16 * 16;
