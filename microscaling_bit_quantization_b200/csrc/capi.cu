@@ -30,6 +30,7 @@ bool valid_shape(int32_t fmt, int64_t rows, int64_t cols) {
     int blk = fmt_block(fmt);
     if (blk && cols % blk) return false;
     if (rows > (int64_t)1 << 31 || cols > (int64_t)1 << 31) return false;
+    if (rows * (cols / 16) >= ((int64_t)1 << 31)) return false;   // chunk indices are 31-bit
     return true;
 }
 

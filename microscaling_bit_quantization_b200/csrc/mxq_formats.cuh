@@ -15,6 +15,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <stdint.h>
@@ -88,6 +89,29 @@ __device__ __forceinline__ int floor_log2_pos(float a) {
     return (31 - __clz((int)(u & 0x7FFFFFu))) - 149;
 }
 
+// ----------------------------------------------------------------- integer division
+
+// floor(n / d) for n < 2^31 and 1 <= d < 2^31 by one multiply-high
+// (Granlund & Montgomery, "Division by invariant integers using
+// multiplication", 1994): with l = ceil(log2 d) and m = floor(2^(31+l)/d) + 1,
+// m*d - 2^(31+l) <= 2^l, so floor(n/d) = floor(m n / 2^(31+l)) for all 31-bit
+// n; m fits 32 bits when d is not a power of two (powers of two shift).
+struct FastDiv {
+    uint32_t d, m;
+    int l;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+    FastDiv f;
+    f.d = d;
+    f.l = 0;
+    while ((1u << f.l) < d) f.l++;
+    f.m = (d & (d - 1)) == 0 ? 0u : (uint32_t)((((uint64_t)1) << (31 + f.l)) / d + 1);
+    return f;
+}
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv &f) {
+    return f.m == 0 ? (n >> f.l) : (__umulhi(n, f.m) >> (f.l - 1));
+}
+
 // ----------------------------------------------------------------- scale rules
 
 // OCP MX shared scale: e = floor(log2 amax) - emax_elem, clamped to [-127,127];
@@ -127,73 +151,177 @@ __device__ __forceinline__ int int_code(float v, float s, int qmax) {
     return q > qmax ? qmax : (q < -qmax ? -qmax : q);
 }
 
+// ----------------------------------------------------------------- packed conversions
+
+// E2M1 codes of eight fp32 values (RN, satfinite), two per byte, element
+// 2i in the low nibble of byte i.  The conversion keeps the sign of zero.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(float v0, float v1, float v2, float v3, float v4, float v5,
+                                               float v6, float v7) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
+    return r;
+}
+
+// E4M3 codes of four fp32 values (RN, satfinite), element i in byte i.
+__device__ __forceinline__ uint32_t cvt_e4m3x4(float v0, float v1, float v2, float v3) {
+    uint32_t r;
+    asm("{\n\t.reg .b16 h0, h1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 h0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 h1, %4, %3;\n\t"
+        "mov.b32 %0, {h0, h1};\n\t}"
+        : "=r"(r)
+        : "f"(v0), "f"(v1), "f"(v2), "f"(v3));
+    return r;
+}
+
+// Value of a positive E4M3 code (exact: every E4M3 value is an fp16 value).
+// The code is placed in both bytes, so either half of the result holds it.
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+    uint32_t h2;
+    asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}" : "=r"(h2) : "r"(code * 0x101u));
+    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
 // ----------------------------------------------------------------- codes of quotients
 //
 // Codes of RN(v / d) for many v and one divisor d, without an IEEE division
-// per element.  y = RN(1/d) (correctly rounded reciprocal) and q = RN(|v| y)
-// give q within a relative 2^-23 + 2^-48 of |v|/d, so RN(|v|/d) lies in
-// [q (1 - 2^-22), q (1 + 2^-22)].  Every code function used here is a
-// monotone function of the magnitude, so when the codes of the bracket ends
-// RN(q (1 - 2^-20)) and RN(q (1 + 2^-20)) (which enclose that interval)
-// agree, the code of RN(|v|/d) is that code; otherwise a code boundary (or an
-// exact tie) lies inside the bracket and the quotient is computed by exact
-// division.  Signs are applied afterwards (RN(-x) = -RN(x)).  When q is an
-// fp32 subnormal (|v|/d < 2^-126) the relative bound does not hold, but both
-// ends and the true quotient are then far below the smallest nonzero code.
+// per element.  With y = RN(1/d) (correctly rounded reciprocal) and the
+// bracket multipliers y_lo = RN(y (1 - 2^-20)), y_hi = RN(y (1 + 2^-20)), the
+// products L = v y_lo and H = v y_hi (exact reals, or rounded once) satisfy
+// |L| < |v/d|(1 - 13 * 2^-24) and |H| > |v/d|(1 + 13 * 2^-24), so RN(v/d),
+// which is within 2^-24 of v/d, lies strictly between them.  Every code
+// function used here (E2M1, E4M3, round-to-integer) is monotone, so when the
+// codes of L and H agree the code of RN(v/d) is that code; otherwise a code
+// boundary or an exact tie lies inside the bracket and that group of values
+// is coded from exact divisions.  Signs need no special handling: the codes
+// are odd functions and the bracket ends keep the sign of v.  When products
+// fall into the fp32 subnormal range the relative bound fails, but the ends
+// and the true quotient are then far below the smallest nonzero code.
 struct Recip {
-    float d, y;
-    bool fast;   // d in [2^-120, 2^120]: y finite and normal, no overflow in q
+    float d, lo, hi;
+    bool fast;   // d in [2^-120, 2^120]: y finite and normal, no overflow in the products
 };
+constexpr float kBracketLo = 0.99999904632568359375f;   // 1 - 2^-20
+constexpr float kBracketHi = 1.00000095367431640625f;   // 1 + 2^-20
 __device__ __forceinline__ Recip recip_of(float d) {
     Recip r;
     r.d = d;
     r.fast = d >= 7.52316384526264e-37f && d <= 1.329227995784916e36f;
-    r.y = r.fast ? __frcp_rn(d) : 0.0f;
+    const float y = r.fast ? __frcp_rn(d) : 0.0f;
+    r.lo = __fmul_rn(y, kBracketLo);
+    r.hi = __fmul_rn(y, kBracketHi);
     return r;
 }
-constexpr float kBracketLo = 0.99999904632568359375f;   // 1 - 2^-20
-constexpr float kBracketHi = 1.00000095367431640625f;   // 1 + 2^-20
 
-// E2M1 codes of RN(v0/d), RN(v1/d) as one byte (v0 in the low nibble).
-__device__ __forceinline__ uint32_t e2m1x2_quot(float v0, float v1, const Recip &r) {
-    const uint32_t sign = ((__float_as_uint(v0) >> 31) << 3) | ((__float_as_uint(v1) >> 31) << 7);
-    const float a0 = fabsf(v0), a1 = fabsf(v1);
+// E2M1 codes of RN(v[i] / d) for eight values, packed like cvt_e2m1x8.
+__device__ __forceinline__ uint32_t e2m1x8_quot(const float *v, const Recip &r) {
     if (r.fast) {
-        const float q0 = __fmul_rn(a0, r.y), q1 = __fmul_rn(a1, r.y);
-        const uint32_t lo = enc_e2m1x2(__fmul_rn(q0, kBracketLo), __fmul_rn(q1, kBracketLo));
-        const uint32_t hi = enc_e2m1x2(__fmul_rn(q0, kBracketHi), __fmul_rn(q1, kBracketHi));
-        if (lo == hi) return lo | sign;
+        const uint32_t lo = cvt_e2m1x8(__fmul_rn(v[0], r.lo), __fmul_rn(v[1], r.lo), __fmul_rn(v[2], r.lo),
+                                       __fmul_rn(v[3], r.lo), __fmul_rn(v[4], r.lo), __fmul_rn(v[5], r.lo),
+                                       __fmul_rn(v[6], r.lo), __fmul_rn(v[7], r.lo));
+        const uint32_t hi = cvt_e2m1x8(__fmul_rn(v[0], r.hi), __fmul_rn(v[1], r.hi), __fmul_rn(v[2], r.hi),
+                                       __fmul_rn(v[3], r.hi), __fmul_rn(v[4], r.hi), __fmul_rn(v[5], r.hi),
+                                       __fmul_rn(v[6], r.hi), __fmul_rn(v[7], r.hi));
+        if (lo == hi) return lo;
     }
-    return enc_e2m1x2(__fdiv_rn(a0, r.d), __fdiv_rn(a1, r.d)) | sign;
+    return cvt_e2m1x8(__fdiv_rn(v[0], r.d), __fdiv_rn(v[1], r.d), __fdiv_rn(v[2], r.d), __fdiv_rn(v[3], r.d),
+                      __fdiv_rn(v[4], r.d), __fdiv_rn(v[5], r.d), __fdiv_rn(v[6], r.d), __fdiv_rn(v[7], r.d));
 }
 
-// E4M3 code of RN(v/d).
-__device__ __forceinline__ uint32_t e4m3_quot(float v, const Recip &r) {
-    const uint32_t sign = (__float_as_uint(v) >> 31) << 7;
-    const float a = fabsf(v);
+// E4M3 codes of RN(v[i] / d) for four values, packed like cvt_e4m3x4.
+__device__ __forceinline__ uint32_t e4m3x4_quot(const float *v, const Recip &r) {
     if (r.fast) {
-        const float q = __fmul_rn(a, r.y);
-        const uint32_t lo = enc_e4m3(__fmul_rn(q, kBracketLo)), hi = enc_e4m3(__fmul_rn(q, kBracketHi));
-        if (lo == hi) return lo | sign;
+        const uint32_t lo = cvt_e4m3x4(__fmul_rn(v[0], r.lo), __fmul_rn(v[1], r.lo), __fmul_rn(v[2], r.lo),
+                                       __fmul_rn(v[3], r.lo));
+        const uint32_t hi = cvt_e4m3x4(__fmul_rn(v[0], r.hi), __fmul_rn(v[1], r.hi), __fmul_rn(v[2], r.hi),
+                                       __fmul_rn(v[3], r.hi));
+        if (lo == hi) return lo;
     }
-    return (uint32_t)enc_e4m3(__fdiv_rn(a, r.d)) | sign;
+    return cvt_e4m3x4(__fdiv_rn(v[0], r.d), __fdiv_rn(v[1], r.d), __fdiv_rn(v[2], r.d), __fdiv_rn(v[3], r.d));
 }
 
-// Symmetric integer code clamp(RNE(RN(v/s)), -qmax, qmax); 0 when s == 0.
-__device__ __forceinline__ int int_code_quot(float v, const Recip &r, int qmax) {
-    if (r.d == 0.0f) return 0;
-    const float a = fabsf(v);
-    int c;
+// Symmetric integer codes clamp(RNE(RN(v[i]/s)), -qmax, qmax) of four values,
+// as bytes (two's complement, element i in byte i); all 0 when s == 0.
+// Rounding to an integer is one FMA: for |t| < 2^22, RN(t + 1.5 * 2^23) is
+// 1.5 * 2^23 + RNE(t) with no intermediate rounding of t, and the low byte of
+// its bit pattern is RNE(t) in two's complement.  The fast path needs no
+// clamp when s comes from the block's own maximum: |v| <= amax and
+// s = RN(amax / qmax) give |v/s| <= qmax (1 + 2^-23), which rounds to qmax.
+constexpr float kRoundMagic = 12582912.0f;   // 1.5 * 2^23
+__device__ __forceinline__ uint32_t int_x4_quot(const float *v, const Recip &r, int qmax) {
+    if (r.d == 0.0f) return 0u;
+    if (r.fast) {
+        uint32_t b[4];
+        bool same = true;
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const float l = __fmaf_rn(v[i], r.lo, kRoundMagic), h = __fmaf_rn(v[i], r.hi, kRoundMagic);
+            same = same && l == h;
+            b[i] = __float_as_uint(l);
+        }
+        if (same) return __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+    }
+    uint32_t out = 0;
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        int q = __float2int_rn(__fdiv_rn(v[i], r.d));
+        q = q > qmax ? qmax : (q < -qmax ? -qmax : q);
+        out |= ((uint32_t)q & 0xFFu) << (8 * i);
+    }
+    return out;
+}
+
+// Low nibbles of the four bytes of two words, as eight packed nibbles
+// (byte i of w0 -> nibble i, byte i of w1 -> nibble 4 + i).
+__device__ __forceinline__ uint32_t nibbles_of_bytes(uint32_t w0, uint32_t w1) {
+    uint32_t t0 = w0 & 0x0F0F0F0Fu, t1 = w1 & 0x0F0F0F0Fu;
+    t0 |= t0 >> 4;   // byte 0: n0 | n1 << 4, byte 2: n2 | n3 << 4
+    t1 |= t1 >> 4;
+    return __byte_perm(t0, t1, 0x6420);
+}
+
+// ----------------------------------------------------------------- NVFP4 block scale
+
+// Reciprocal of the tensor scale, for the division-free block-scale path.
+struct TensorRecip {
+    float s, inv;
+    bool fast;   // s in [2^-100, 2^100]
+};
+__device__ __forceinline__ TensorRecip tensor_recip_of(float s) {
+    TensorRecip t;
+    t.s = s;
+    t.fast = s >= 7.888609052210118e-31f && s <= 1.2676506002282294e30f;
+    t.inv = t.fast ? __frcp_rn(s) : 0.0f;
+    return t;
+}
+
+// The NVFP4 block scale of nvfp4_block_scale without the two divisions in
+// the common case.  q = RN(RN(amax_b c6) inv), c6 = RN(1/6), is within
+// 4 * 2^-24 of amax_b / (6 s_t) and the exact RN(RN(amax_b / 6) / s_t) within
+// 2 * 2^-24, so the E4M3 codes of RN(q (1 -+ 2^-20)) enclose the exact code
+// (the argument of the quotient codes above); on disagreement, divide.  With
+// s_t in [2^-100, 2^100] a subnormal RN(amax_b c6) only occurs when both ends
+// and the exact value are below 2^-26, where every code is 0.
+constexpr float kInvSix = 0.16666667163372039794921875f;   // RN(1/6)
+__device__ __forceinline__ uint32_t nvfp4_block_scale_fast(float amax_b, const TensorRecip &t, float &d) {
+    uint32_t e4 = 0;
     bool done = false;
-    if (r.fast) {
-        const float q = __fmul_rn(a, r.y);
-        const int lo = __float2int_rn(__fmul_rn(q, kBracketLo)), hi = __float2int_rn(__fmul_rn(q, kBracketHi));
-        c = lo;
-        done = lo == hi;
+    if (t.fast) {
+        const float q = __fmul_rn(__fmul_rn(amax_b, kInvSix), t.inv);
+        const uint32_t two = cvt_e4m3x4(__fmul_rn(q, kBracketLo), __fmul_rn(q, kBracketHi), 0.0f, 0.0f);
+        e4 = two & 0xFFu;
+        done = e4 == ((two >> 8) & 0xFFu);
     }
-    if (!done) c = __float2int_rn(__fdiv_rn(a, r.d));
-    c = c > qmax ? qmax : c;
-    return v < 0.0f ? -c : c;
+    if (!done) e4 = enc_e4m3(__fdiv_rn(__fdiv_rn(amax_b, 6.0f), t.s));
+    d = e4 ? __fmul_rn(e4m3_to_f32(e4), t.s) : 0.0f;
+    return e4;
 }
 
 // ----------------------------------------------------------------- loads

@@ -33,14 +33,15 @@ inline int grid_for(int64_t warp_tiles, int sm_count) {
 // ------------------------------------------------------------------ amax
 
 // Max over the CTA, then one atomicMax on the word (non-negative floats
-// order like their bit patterns).  All threads of the CTA must call this.
+// order like their bit patterns).  All NT threads of the CTA must call this.
+template <int NT = kThreads>
 __device__ __forceinline__ void cta_max_to_word(float m, unsigned int *word) {
-    __shared__ float wmax[kThreads / 32];
+    __shared__ float wmax[NT / 32];
     m = group_max<32>(m);
     if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
     __syncthreads();
     if (threadIdx.x < 32) {
-        float v = threadIdx.x < kThreads / 32 ? wmax[threadIdx.x] : 0.0f;
+        float v = threadIdx.x < NT / 32 ? wmax[threadIdx.x] : 0.0f;
         v = group_max<32>(v);
         if (threadIdx.x == 0 && v > 0.0f) atomicMax(word, __float_as_uint(v));
     }
@@ -60,7 +61,8 @@ __device__ __forceinline__ uint32_t gather4(uint32_t byte) {
 // ------------------------------------------------------------------ quantize
 
 struct QuantArgs {
-    int64_t rows, cols, total_chunks;
+    int64_t rows, cols, total_chunks;   // total_chunks < 2^31
+    FastDiv cpr;                        // chunks per row
     int hadamard_b;
     int layout;              // 0 canonical, 1 MMA
     int64_t s_pad;           // padded scale columns (MMA layout)
@@ -77,117 +79,97 @@ struct QuantArgs {
     unsigned int *err;       // device error word (a bounded wait that ran out)
 };
 
-// Staged input: persistent CTAs bring 16 KB tiles of x into a ring of
-// kQStages shared-memory buffers with one cp.async.bulk each (completion on
-// an mbarrier), then encode from shared memory.
-constexpr int kQStages = 4, kQTileBytes = 16384, kQSmem = kQStages * kQTileBytes;
+// Streaming structure of the quantize kernels: each CTA owns a contiguous,
+// warp-aligned range of chunks; every thread encodes one chunk per step, the
+// CTA's 512 threads covering 512 consecutive chunks, and keeps the raw bytes
+// of its next 64 bytes of input (two bf16 chunks or one fp32 chunk) in flight
+// in registers, 64 KB per SM with two CTAs, so warps never wait on each
+// other and loads overlap the encoding.
+constexpr int kQThreads = 512;
 constexpr unsigned int kErrTimeoutQuant = 8u;
 
-__device__ __forceinline__ uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
-__device__ __forceinline__ void q_bar_init(uint64_t *bar) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(bar)));
+// Raw bytes of one 16-element chunk (32 B of bf16 or 64 B of fp32).
+template <typename T>
+struct RawChunk {
+    uint4 q[sizeof(T) * 16 / 16];
+};
+template <typename T>
+__device__ __forceinline__ void raw_load(RawChunk<T> &r, const T *p) {
+    const uint4 *g = reinterpret_cast<const uint4 *>(p);
+#pragma unroll
+    for (int i = 0; i < (int)(sizeof(r.q) / 16); i++) r.q[i] = __ldg(g + i);
 }
-__device__ __forceinline__ void q_bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     smem_addr(dst)),
-                 "l"(src), "r"(bytes), "r"(smem_addr(bar))
-                 : "memory");
-}
-// Bounded wait (about 2 s of polling) for phase `parity` of the barrier.
-__device__ __forceinline__ bool q_bar_wait(uint64_t *bar, uint32_t parity) {
-    for (long long i = 0; i < (1ll << 26); i++) {
-        uint32_t ok;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(smem_addr(bar)), "r"(parity)
-            : "memory");
-        if (ok) return true;
+__device__ __forceinline__ void raw_unpack(const RawChunk<__nv_bfloat16> &r, float v[16]) {
+    const uint32_t w[8] = {r.q[0].x, r.q[0].y, r.q[0].z, r.q[0].w, r.q[1].x, r.q[1].y, r.q[1].z, r.q[1].w};
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+        v[2 * j] = __uint_as_float(w[j] << 16);
+        v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
     }
-    return false;
 }
-
-__device__ __forceinline__ void load16_shared(const float *p, float v[16]) {
-    const float4 *q = reinterpret_cast<const float4 *>(p);
+__device__ __forceinline__ void raw_unpack(const RawChunk<float> &r, float v[16]) {
 #pragma unroll
     for (int i = 0; i < 4; i++) {
-        float4 t = q[i];
-        v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
-    }
-}
-__device__ __forceinline__ void load16_shared(const __nv_bfloat16 *p, float v[16]) {
-    const uint4 *q = reinterpret_cast<const uint4 *>(p);
-#pragma unroll
-    for (int i = 0; i < 2; i++) {
-        uint4 t = q[i];
-        uint32_t w[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-            v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
-            v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-        }
+        v[4 * i] = __uint_as_float(r.q[i].x);
+        v[4 * i + 1] = __uint_as_float(r.q[i].y);
+        v[4 * i + 2] = __uint_as_float(r.q[i].z);
+        v[4 * i + 3] = __uint_as_float(r.q[i].w);
     }
 }
 
 template <typename T, int F>
-__global__ void __launch_bounds__(kThreads) k_quantize(const T *__restrict__ x, QuantArgs a) {
+__global__ void __launch_bounds__(kQThreads, 2) k_quantize(const T *__restrict__ x, QuantArgs a) {
+    constexpr int kQDepth = 64 / (16 * (int)sizeof(T));   // chunks in flight per thread
     constexpr int BLK = fmt_block(F) ? fmt_block(F) : 16;
-    constexpr int G = BLK ? BLK / 16 : 1;   // lanes per quantization block
-    constexpr int CPT = kQTileBytes / (16 * (int)sizeof(T));   // chunks per staged tile
-    extern __shared__ __align__(128) uint8_t q_smem[];
-    __shared__ uint64_t q_bars[kQStages];
+    constexpr int G = BLK / 16;   // lanes per quantization block
     const int lane = lane_id();
-    const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * kThreads) >> 5;
-    const int64_t ntiles = (a.total_chunks + CPT - 1) / CPT;
-    const int64_t chunks_per_row = a.cols >> 4;
-    auto issue = [&](int64_t tile, int stage) {
-        const int64_t n = a.total_chunks - tile * CPT;
-        const uint32_t bytes = (uint32_t)((n < CPT ? n : CPT) * 16 * (int64_t)sizeof(T));
-        q_bulk_load(q_smem + stage * kQTileBytes, x + tile * CPT * 16, bytes, &q_bars[stage]);
-    };
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < kQStages; i++) q_bar_init(&q_bars[i]);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        for (int i = 0; i < kQStages; i++) {
-            const int64_t tile = blockIdx.x + (int64_t)i * gridDim.x;
-            if (tile < ntiles) issue(tile, i);
-        }
-    }
-    __syncthreads();
+    // this CTA's chunks [c_begin, c_end), boundaries on multiples of 32 chunks
+    const uint32_t total = (uint32_t)a.total_chunks;
+    const uint32_t units = (total + 31) >> 5;
+    const uint32_t c_begin = (uint32_t)(((uint64_t)blockIdx.x * units / gridDim.x) << 5);
+    uint32_t c_end = (uint32_t)(((uint64_t)(blockIdx.x + 1) * units / gridDim.x) << 5);
+    c_end = c_end < total ? c_end : total;
+    const int steps = (int)((c_end - c_begin + kQThreads - 1) / kQThreads);
+    const uint32_t cpr = (uint32_t)(a.cols >> 4);
 
     float s_t = 1.0f;
+    TensorRecip tr;
+    Recip rt;
     if (F == kNVFP4 || F == kFP8Tensor) {
         float amax_t = __uint_as_float(*a.amax_word);
         s_t = F == kNVFP4 ? nvfp4_tensor_scale(amax_t) : fp8_tensor_scale(amax_t);
         if (blockIdx.x == 0 && threadIdx.x == 0) *a.tensor_scale = s_t;
+        if (F == kNVFP4) tr = tensor_recip_of(s_t);
+        else rt = recip_of(s_t);
     }
 
-    bool failed = false;
+    RawChunk<T> pre[kQDepth];
+#pragma unroll
+    for (int i = 0; i < kQDepth; i++) {
+        const uint32_t c = c_begin + (uint32_t)i * kQThreads + threadIdx.x;
+        if (c < c_end) raw_load(pre[i], x + (int64_t)c * 16);
+    }
     float tensor_max = 0.0f;
-    int64_t it = 0;
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, it++) {
-      const int stage = (int)(it % kQStages);
-      if (!q_bar_wait(&q_bars[stage], (uint32_t)((it / kQStages) & 1))) {
-          failed = true;
-          break;
-      }
-      const T *tx = reinterpret_cast<const T *>(q_smem + stage * kQTileBytes);
 #pragma unroll 1
-      for (int jc = 0; jc < CPT / kThreads; jc++) {
-        const int cit = threadIdx.x + jc * kThreads;   // chunk within the tile
-        const int64_t c = tile * CPT + cit;
-        const bool valid = c < a.total_chunks;
+    for (int it = 0; it < steps; it++) {
+        const uint32_t c = c_begin + (uint32_t)it * kQThreads + threadIdx.x;
+        const bool valid = c < c_end;
         float v[16];
-        if (valid) load16_shared(tx + cit * 16, v);
+        if (valid) raw_unpack(pre[0], v);
         else {
 #pragma unroll
             for (int i = 0; i < 16; i++) v[i] = 0.0f;
         }
+#pragma unroll
+        for (int i = 0; i + 1 < kQDepth; i++) pre[i] = pre[i + 1];
+        {
+            const uint32_t cn = c + (uint32_t)kQDepth * kQThreads;
+            if (cn < c_end) raw_load(pre[kQDepth - 1], x + (int64_t)cn * 16);
+        }
+
         if (a.hadamard_b) hadamard_chunk(v, a.hadamard_b, lane);
-        const int64_t row = c / chunks_per_row;
-        const int64_t col0 = (c - row * chunks_per_row) << 4;
+        const uint32_t row = fdiv(c, a.cpr);
+        const uint32_t colc = c - row * cpr;   // chunk index within the row
         float amax = amax16(v);
         if (F == kNumFmt) {   // tensor-amax pass only
             tensor_max = fmaxf(tensor_max, amax);
@@ -200,137 +182,89 @@ __global__ void __launch_bounds__(kThreads) k_quantize(const T *__restrict__ x, 
             uint32_t sb = 127;
             if (amax > 0.0f) sb = mx_scale(amax, F == kMXFP8 ? 8 : 2, inv);
             if (valid) {
+                // inv is a power of two: v * inv is exact (or far below the smallest code)
+                float u[16];
+#pragma unroll
+                for (int i = 0; i < 16; i++) u[i] = __fmul_rn(v[i], inv);
+                const bool zero = !(amax > 0.0f);   // all-zero block: +0 codes
                 if (F == kMXFP8) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int j = 0; j < 4; j++) {
-                        uint32_t b0 = 0, b1 = 0, b2 = 0, b3 = 0;
-                        if (amax > 0.0f) {
-                            b0 = enc_e4m3(__fmul_rn(v[4 * j], inv));
-                            b1 = enc_e4m3(__fmul_rn(v[4 * j + 1], inv));
-                            b2 = enc_e4m3(__fmul_rn(v[4 * j + 2], inv));
-                            b3 = enc_e4m3(__fmul_rn(v[4 * j + 3], inv));
-                        }
-                        w[j] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
-                    }
-                    *reinterpret_cast<uint4 *>(a.codes + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+                    uint4 w;
+                    w.x = zero ? 0u : cvt_e4m3x4(u[0], u[1], u[2], u[3]);
+                    w.y = zero ? 0u : cvt_e4m3x4(u[4], u[5], u[6], u[7]);
+                    w.z = zero ? 0u : cvt_e4m3x4(u[8], u[9], u[10], u[11]);
+                    w.w = zero ? 0u : cvt_e4m3x4(u[12], u[13], u[14], u[15]);
+                    *reinterpret_cast<uint4 *>(a.codes + (int64_t)c * 16) = w;
                 } else {
-                    uint32_t w[2];
-#pragma unroll
-                    for (int j = 0; j < 2; j++) {
-                        uint32_t acc = 0;
-#pragma unroll
-                        for (int k = 0; k < 4; k++) {
-                            uint32_t byte = 0;
-                            if (amax > 0.0f)
-                                byte = enc_e2m1x2(__fmul_rn(v[8 * j + 2 * k], inv), __fmul_rn(v[8 * j + 2 * k + 1], inv));
-                            acc |= byte << (8 * k);
-                        }
-                        w[j] = acc;
-                    }
-                    *reinterpret_cast<uint2 *>(a.codes + c * 8) = make_uint2(w[0], w[1]);
+                    uint2 w;
+                    w.x = zero ? 0u : cvt_e2m1x8(u[0], u[1], u[2], u[3], u[4], u[5], u[6], u[7]);
+                    w.y = zero ? 0u : cvt_e2m1x8(u[8], u[9], u[10], u[11], u[12], u[13], u[14], u[15]);
+                    *reinterpret_cast<uint2 *>(a.codes + (int64_t)c * 8) = w;
                 }
             }
             const uint32_t word = gather4<2>(sb);
             if (valid) {
-                const int64_t s = col0 >> 5;
-                uint8_t *sc = reinterpret_cast<uint8_t *>(a.scales);
-                const int64_t off = a.layout == 0 ? row * (a.cols >> 5) + s : mma_scale_offset(row, s, a.s_pad);
+                const uint32_t sc = colc >> 1;
+                uint8_t *scb = reinterpret_cast<uint8_t *>(a.scales);
+                const int64_t off = a.layout == 0 ? (int64_t)row * (cpr >> 1) + sc : mma_scale_offset(row, sc, a.s_pad);
                 if (a.combine) {
-                    if ((lane & 7) == 0) *reinterpret_cast<uint32_t *>(sc + off) = word;
+                    if ((lane & 7) == 0) *reinterpret_cast<uint32_t *>(scb + off) = word;
                 } else if ((lane & 1) == 0) {
-                    sc[off] = (uint8_t)sb;
+                    scb[off] = (uint8_t)sb;
                 }
             }
         } else if (F == kNVFP4) {
             float d;
-            uint32_t e4 = nvfp4_block_scale(amax, s_t, d);
+            const uint32_t e4 = nvfp4_block_scale_fast(amax, tr, d);
             if (valid) {
-                const Recip rd = recip_of(d);
-                uint32_t w[2];
-#pragma unroll
-                for (int j = 0; j < 2; j++) {
-                    uint32_t acc = 0;
-#pragma unroll
-                    for (int k = 0; k < 4; k++) {
-                        uint32_t byte = 0;
-                        if (e4) byte = e2m1x2_quot(v[8 * j + 2 * k], v[8 * j + 2 * k + 1], rd);
-                        acc |= byte << (8 * k);
-                    }
-                    w[j] = acc;
+                uint2 w = make_uint2(0u, 0u);   // e4 == 0: +0 codes
+                if (e4) {
+                    const Recip rd = recip_of(d);
+                    w.x = e2m1x8_quot(v, rd);
+                    w.y = e2m1x8_quot(v + 8, rd);
                 }
-                *reinterpret_cast<uint2 *>(a.codes + c * 8) = make_uint2(w[0], w[1]);
+                *reinterpret_cast<uint2 *>(a.codes + (int64_t)c * 8) = w;
             }
             const uint32_t word = gather4<1>(e4);
             if (valid) {
-                const int64_t s = col0 >> 4;
-                uint8_t *sc = reinterpret_cast<uint8_t *>(a.scales);
-                const int64_t off = a.layout == 0 ? c : mma_scale_offset(row, s, a.s_pad);
+                uint8_t *scb = reinterpret_cast<uint8_t *>(a.scales);
+                const int64_t off = a.layout == 0 ? (int64_t)c : mma_scale_offset(row, colc, a.s_pad);
                 if (a.combine) {
-                    if ((lane & 3) == 0) *reinterpret_cast<uint32_t *>(sc + off) = word;
+                    if ((lane & 3) == 0) *reinterpret_cast<uint32_t *>(scb + off) = word;
                 } else {
-                    sc[off] = (uint8_t)e4;
+                    scb[off] = (uint8_t)e4;
                 }
             }
         } else if (F == kINT4G32 || F == kINT4G64) {
-            float s = __fdiv_rn(amax, 7.0f);
+            const float s = __fdiv_rn(amax, 7.0f);
             const Recip rs = recip_of(s);
             if (valid) {
-                if (a.layout == 0) {
-                    uint32_t w[2];
-#pragma unroll
-                    for (int j = 0; j < 2; j++) {
-                        uint32_t acc = 0;
-#pragma unroll
-                        for (int k = 0; k < 8; k++) acc |= ((uint32_t)int_code_quot(v[8 * j + k], rs, 7) & 0xFu) << (4 * k);
-                        w[j] = acc;
-                    }
-                    *reinterpret_cast<uint2 *>(a.codes + c * 8) = make_uint2(w[0], w[1]);
-                } else {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int j = 0; j < 4; j++) {
-                        uint32_t acc = 0;
-#pragma unroll
-                        for (int k = 0; k < 4; k++) acc |= ((uint32_t)int_code_quot(v[4 * j + k], rs, 7) & 0xFFu) << (8 * k);
-                        w[j] = acc;
-                    }
-                    *reinterpret_cast<uint4 *>(a.codes + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-                }
+                const uint32_t b0 = int_x4_quot(v, rs, 7), b1 = int_x4_quot(v + 4, rs, 7);
+                const uint32_t b2 = int_x4_quot(v + 8, rs, 7), b3 = int_x4_quot(v + 12, rs, 7);
+                if (a.layout == 0)
+                    *reinterpret_cast<uint2 *>(a.codes + (int64_t)c * 8) =
+                        make_uint2(nibbles_of_bytes(b0, b1), nibbles_of_bytes(b2, b3));
+                else
+                    *reinterpret_cast<uint4 *>(a.codes + (int64_t)c * 16) = make_uint4(b0, b1, b2, b3);
                 if ((lane & (G - 1)) == 0) {
                     float *sc = reinterpret_cast<float *>(a.scales);
-                    int64_t g = col0 / BLK;
-                    if (a.layout == 0) sc[row * (a.cols / BLK) + g] = s;
-                    else sc[g * a.rows + row] = s;
+                    const uint32_t g = colc / G;
+                    if (a.layout == 0) sc[(int64_t)row * (cpr / G) + g] = s;
+                    else sc[(int64_t)g * a.rows + row] = s;
                 }
             }
         } else if (F == kFP8Tensor) {
             if (valid) {
-                const Recip rs = recip_of(s_t);
-                uint32_t w[4];
-#pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    uint32_t acc = 0;
-#pragma unroll
-                    for (int k = 0; k < 4; k++) acc |= e4m3_quot(v[4 * j + k], rs) << (8 * k);
-                    w[j] = acc;
-                }
-                *reinterpret_cast<uint4 *>(a.codes + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+                uint4 w;
+                w.x = e4m3x4_quot(v, rt);
+                w.y = e4m3x4_quot(v + 4, rt);
+                w.z = e4m3x4_quot(v + 8, rt);
+                w.w = e4m3x4_quot(v + 12, rt);
+                *reinterpret_cast<uint4 *>(a.codes + (int64_t)c * 16) = w;
             }
         }
-      }
-      __syncthreads();   // the stage is free again
-      if (threadIdx.x == 0) {
-          const int64_t next = tile + (int64_t)kQStages * gridDim.x;
-          if (next < ntiles) issue(next, stage);
-      }
-    }
-    if (failed) {
-        if (threadIdx.x == 0) atomicOr(a.err, kErrTimeoutQuant);
-        return;
     }
     if (F == kNumFmt) {
-        cta_max_to_word(tensor_max, const_cast<unsigned int *>(a.amax_word));
+        cta_max_to_word<kQThreads>(tensor_max, const_cast<unsigned int *>(a.amax_word));
         return;
     }
     if (a.tp) {
@@ -338,6 +272,8 @@ __global__ void __launch_bounds__(kThreads) k_quantize(const T *__restrict__ x, 
         // u = t / alpha, hi = bf16(u), lo = bf16(u - hi), zeros past r
         const bool ts = F == kNVFP4 || F == kFP8Tensor;
         const float alpha = ts ? __fmul_rn(s_t, *a.w_ts) : 1.0f;
+        const int64_t warp = ((int64_t)blockIdx.x * kQThreads + threadIdx.x) >> 5;
+        const int64_t nwarps = ((int64_t)gridDim.x * kQThreads) >> 5;
         for (int64_t row = warp; row < a.rows; row += nwarps) {
             float u = lane < a.r ? a.t[row * a.r + lane] : 0.0f;
             if (ts) u = __fdiv_rn(u, alpha);
@@ -381,17 +317,10 @@ __global__ void __launch_bounds__(kThreads) k_quantize_int8_row(const T *__restr
                 for (int i = 0; i < 16; i++) v[i] = 0.0f;
             }
             if (a.hadamard_b) hadamard_chunk(v, a.hadamard_b, lane);
-            if (c < cpr) {
-                uint32_t w[4];
-#pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    uint32_t acc = 0;
-#pragma unroll
-                    for (int k = 0; k < 4; k++) acc |= ((uint32_t)int_code_quot(v[4 * j + k], rs, 127) & 0xFFu) << (8 * k);
-                    w[j] = acc;
-                }
-                *reinterpret_cast<uint4 *>(a.codes + (row * cpr + c) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
+            if (c < cpr)
+                *reinterpret_cast<uint4 *>(a.codes + (row * cpr + c) * 16) =
+                    make_uint4(int_x4_quot(v, rs, 127), int_x4_quot(v + 4, rs, 127), int_x4_quot(v + 8, rs, 127),
+                               int_x4_quot(v + 12, rs, 127));
         }
         if (lane == 0) reinterpret_cast<float *>(a.scales)[row] = s;
     }
@@ -401,6 +330,7 @@ __global__ void __launch_bounds__(kThreads) k_quantize_int8_row(const T *__restr
 
 struct DequantArgs {
     int64_t rows, cols, total_chunks;
+    FastDiv cpr;
     int layout;
     int64_t s_pad;
     const uint8_t *codes;
@@ -412,7 +342,7 @@ template <int F>
 __device__ __forceinline__ void dequant_chunk(const DequantArgs &a, int64_t c, float out[16]) {
     constexpr int BLK = fmt_block(F) ? fmt_block(F) : 16;
     const int64_t cpr = a.cols >> 4;
-    const int64_t row = c / cpr;
+    const int64_t row = fdiv((uint32_t)c, a.cpr);
     const int64_t col0 = (c - row * cpr) << 4;
     uint32_t code[16];
     const bool unpacked_int4 = (F == kINT4G32 || F == kINT4G64) && a.layout == 1;
@@ -669,6 +599,7 @@ cudaError_t launch_amax(const void *x, bool bf16, int64_t rows, int64_t cols, in
     a.rows = rows;
     a.cols = cols;
     a.total_chunks = chunks;
+    a.cpr = make_fastdiv((uint32_t)(cols / 16 > 0 ? cols / 16 : 1));
     a.hadamard_b = hadamard_b;
     a.amax_word = amax_word;
     e = error_word_address(&a.err);
@@ -680,16 +611,10 @@ cudaError_t launch_amax(const void *x, bool bf16, int64_t rows, int64_t cols, in
 
 template <typename T, int F>
 static void launch_qf(const T *x, const QuantArgs &a, cudaStream_t s) {
-    static bool configured = false;
-    if (!configured) {
-        cudaFuncSetAttribute(k_quantize<T, F>, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem);
-        configured = true;
-    }
-    constexpr int CPT = kQTileBytes / (16 * (int)sizeof(T));
-    const int64_t ntiles = (a.total_chunks + CPT - 1) / CPT;
-    const int64_t cap = (int64_t)sm_count_cached() * 3;   // 3 x 64 KB of ring per SM
-    const int grid = (int)(ntiles < cap ? ntiles : cap);
-    k_quantize<T, F><<<grid, kThreads, kQSmem, s>>>(x, a);
+    const int64_t steps = (a.total_chunks + kQThreads - 1) / kQThreads;
+    const int64_t cap = (int64_t)sm_count_cached() * 2;   // two 512-thread CTAs per SM
+    const int grid = (int)(steps < cap ? steps : cap);
+    k_quantize<T, F><<<grid, kQThreads, 0, s>>>(x, a);
 }
 
 template <typename T>
@@ -721,6 +646,7 @@ cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols
     a.rows = rows;
     a.cols = cols;
     a.total_chunks = rows * cols / 16;
+    a.cpr = make_fastdiv((uint32_t)(cols / 16 > 0 ? cols / 16 : 1));
     a.hadamard_b = hadamard_b;
     a.layout = layout;
     a.s_pad = 0;
@@ -776,6 +702,7 @@ cudaError_t launch_dequantize(int fmt, int layout, int64_t rows, int64_t cols, c
     a.rows = rows;
     a.cols = cols;
     a.total_chunks = rows * cols / 16;
+    a.cpr = make_fastdiv((uint32_t)(cols / 16 > 0 ? cols / 16 : 1));
     a.layout = layout;
     a.s_pad = fmt_byte_scales(fmt) ? (cols / fmt_block(fmt) + 15) / 16 * 16 : 0;
     a.codes = (const uint8_t *)codes;
