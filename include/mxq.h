@@ -77,8 +77,10 @@ typedef enum mxq_dtype { MXQ_F32 = 0, MXQ_BF16 = 1 } mxq_dtype;
  *        (row r, scale column s) at
  *          ((r/128)*(S'/4) + s/4)*512 + (r%32)*16 + ((r%128)/32)*4 + s%4;
  *        padding bytes are written as 0.
- *      INT4_G32/64: codes one signed byte per element [rows][cols]; scales
- *        fp32 transposed [cols/g][rows].
+ *      INT4_G32/64: codes one byte per element [rows][cols] holding the
+ *        E4M3 encoding of the integer code (every integer in [-7, 7] is an
+ *        E4M3 value; zero is encoded +0), so that the tensor cores form the
+ *        exact integer products in fp32; scales fp32 transposed [cols/g][rows].
  *      INT8_ROW, FP8_TENSOR: identical to CANONICAL.
  */
 typedef enum mxq_layout { MXQ_LAYOUT_CANONICAL = 0, MXQ_LAYOUT_MMA = 1 } mxq_layout;
@@ -228,9 +230,10 @@ mxq_status mxq_quantize_lowrank_workspace_bytes(int64_t m, int32_t r, size_t *by
  * w_tensor_scale).  For tensor-scaled formats without rotation the tensor
  * amax and t = bf16(x) . l1 come from one read of x, and the encoding pass
  * re-reads x from L2.
- *   fmt: NVFP4, MXFP4, MXFP8 or FP8_TENSOR (the formats whose GEMM takes
- *     the branch); w_tensor_scale: device scalar of the weight (NVFP4,
- *     FP8_TENSOR), else ignored.
+ *   fmt: NVFP4, MXFP4, MXFP8, FP8_TENSOR, INT4_G32 or INT4_G64 (the
+ *     formats whose GEMM takes the branch; INT8_ROW gives
+ *     MXQ_EUNSUPPORTED); w_tensor_scale: device scalar of the weight
+ *     (NVFP4, FP8_TENSOR), else ignored.
  *   workspace: device scratch of mxq_quantize_lowrank_workspace_bytes,
  *     256-byte aligned; clobbered.
  * Other arguments, constraints and errors as mxq_quantize and
@@ -277,16 +280,19 @@ mxq_status mxq_lowrank_pack_l2(const void *l2, int32_t r, int64_t n, void *l2p, 
  *   y[m][n] = sum_k deq(xq)[m][k] * deq(wq)[n][k]  (+ sum_j t[m][j] * l2[j][n])
  * on tcgen05 tensor cores (fp32 accumulation; int32 for INT8_ROW), the
  * per-block scales applied by the tensor cores, tensor / row scales in the
- * epilogue.
+ * epilogue.  INT4_G32 / INT4_G64 (fp32 group scales, which the tensor
+ * cores cannot apply) form each group's exact integer dot product on the
+ * tensor cores and add it, times sx * sw, to fp32 sums in the epilogue.
  *   xq, wq: same fmt, MMA layout, xq->cols == wq->cols == K.
- *     Supported fmt: NVFP4, MXFP4, MXFP8, FP8_TENSOR, INT8_ROW.
+ *     Supported fmt: NVFP4, MXFP4, MXFP8, FP8_TENSOR, INT8_ROW, INT4_G32,
+ *     INT4_G64.
  *   tp: packed low-rank activation (m x 64 bf16, from
  *     mxq_lowrank_down_packed / mxq_lowrank_pack_t with the same tensor
  *     scales as xq, wq) or NULL for no branch; l2p: packed up-projection
- *     (n rows).  The branch is supported for NVFP4, MXFP4, MXFP8, FP8_TENSOR.
+ *     (n rows).  The branch is supported for every fmt but INT8_ROW.
  *   y: m x n device, fp32 or bf16 (fp32 result rounded once, RNE).
- * Constraints: K % 64 == 0 (4-bit) or K % 32 == 0 (8-bit); K > 0; device
- * pointers 16-byte aligned.
+ * Constraints: K % 64 == 0 (NVFP4, MXFP4), K % g == 0 (INT4_Gg) or
+ * K % 32 == 0 (8-bit); K > 0; device pointers 16-byte aligned.
  * Errors: MXQ_EINVAL, MXQ_EUNSUPPORTED (format pair / branch), MXQ_ECUDA.
  * A pipeline wait that runs out is reported by mxq_check(). */
 mxq_status mxq_qlinear(const mxq_qtensor *xq, const mxq_qtensor *wq, const void *tp, const void *l2p,

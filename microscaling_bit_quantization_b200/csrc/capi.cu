@@ -209,7 +209,7 @@ mxq_status mxq_quantize_lowrank(const void *x, int32_t xdtype, int64_t m, int64_
                                 void *stream) {
     if (!valid_fmt(fmt) || !valid_dtype(xdtype) || !valid_shape(fmt, m, k) || !valid_hadamard(hadamard_b, k))
         return MXQ_EINVAL;
-    if (fmt != MXQ_NVFP4 && fmt != MXQ_MXFP4 && fmt != MXQ_MXFP8 && fmt != MXQ_FP8_TENSOR) return MXQ_EUNSUPPORTED;
+    if (fmt == MXQ_INT8_ROW) return MXQ_EUNSUPPORTED;   // its GEMM takes no branch
     if (k <= 0 || r < 1 || r > 32) return MXQ_EINVAL;
     const bool ts = fmt_tensor_scaled(fmt);
     if (ts && (!tensor_scale || !w_tensor_scale)) return MXQ_EINVAL;
@@ -253,11 +253,11 @@ mxq_status mxq_qlinear(const mxq_qtensor *xq, const mxq_qtensor *wq, const void 
     if (!xq || !wq || !valid_dtype(ydtype) || !y) return MXQ_EINVAL;
     if (!valid_fmt(xq->fmt) || xq->fmt != wq->fmt) return MXQ_EUNSUPPORTED;
     const int fmt = xq->fmt;
-    if (fmt == MXQ_INT4_G32 || fmt == MXQ_INT4_G64) return MXQ_EUNSUPPORTED;
+    const bool igroup = fmt == MXQ_INT4_G32 || fmt == MXQ_INT4_G64;
     if (xq->layout != MXQ_LAYOUT_MMA || wq->layout != MXQ_LAYOUT_MMA) return MXQ_EINVAL;
     const int64_t m = xq->rows, n = wq->rows, k = xq->cols;
     if (wq->cols != k || k <= 0 || m < 0 || n < 0) return MXQ_EINVAL;
-    if (k % (fmt_is4(fmt) ? 64 : 32)) return MXQ_EINVAL;
+    if (k % (igroup ? fmt_block(fmt) : fmt_is4(fmt) ? 64 : 32)) return MXQ_EINVAL;
     if (!valid_shape(fmt, m, k) || !valid_shape(fmt, n, k)) return MXQ_EINVAL;
     if (m > 0 && n > 0) {
         if (!xq->codes || !wq->codes || !aligned16(xq->codes) || !aligned16(wq->codes) || !aligned16(y))
@@ -284,7 +284,7 @@ mxq_status mxq_qlinear(const mxq_qtensor *xq, const mxq_qtensor *wq, const void 
     op.l2p = l2p;
     op.y = y;
     op.y_bf16 = ydtype == MXQ_BF16;
-    return from_cuda(launch_qlinear(op, (cudaStream_t)stream));
+    return from_cuda(igroup ? launch_qlinear_igroup(op, (cudaStream_t)stream) : launch_qlinear(op, (cudaStream_t)stream));
 }
 
 }  // extern "C"

@@ -278,6 +278,32 @@ __device__ __forceinline__ uint32_t int_x4_quot(const float *v, const Recip &r, 
     return out;
 }
 
+// The same integer codes as E4M3 bytes (element i in byte i).  Every integer
+// of magnitude <= 7 is an E4M3 value, so the conversion is exact; a zero code
+// is +0 (RN(1.5 * 2^23 - 1.5 * 2^23) = +0).
+__device__ __forceinline__ uint32_t int_x4_quot_e4m3(const float *v, const Recip &r, int qmax) {
+    if (r.d == 0.0f) return 0u;
+    if (r.fast) {
+        float q[4];
+        bool same = true;
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const float l = __fmaf_rn(v[i], r.lo, kRoundMagic), h = __fmaf_rn(v[i], r.hi, kRoundMagic);
+            same = same && l == h;
+            q[i] = __fsub_rn(l, kRoundMagic);
+        }
+        if (same) return cvt_e4m3x4(q[0], q[1], q[2], q[3]);
+    }
+    float q[4];
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        int c = __float2int_rn(__fdiv_rn(v[i], r.d));
+        c = c > qmax ? qmax : (c < -qmax ? -qmax : c);
+        q[i] = (float)c;
+    }
+    return cvt_e4m3x4(q[0], q[1], q[2], q[3]);
+}
+
 // Low nibbles of the four bytes of two words, as eight packed nibbles
 // (byte i of w0 -> nibble i, byte i of w1 -> nibble 4 + i).
 __device__ __forceinline__ uint32_t nibbles_of_bytes(uint32_t w0, uint32_t w1) {

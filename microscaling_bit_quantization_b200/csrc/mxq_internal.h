@@ -2,6 +2,7 @@
 // the C ABI layer.  Arguments are validated by the C ABI before any call.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -58,6 +59,13 @@ struct GemmOperands {
     bool y_bf16;
 };
 cudaError_t launch_qlinear(const GemmOperands &op, cudaStream_t s);
+// INT4_G32 / INT4_G64 operands (E4M3 code bytes, transposed fp32 group scales).
+cudaError_t launch_qlinear_igroup(const GemmOperands &op, cudaStream_t s);
+
+// 2-D tiled tensor map (row-major, `row_bytes` between rows) through the
+// driver entry point; false when the driver rejects it.
+bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
 
 // Device error word (bounded waits that ran out); read-and-clear, and its
 // device address on the current device (for kernels of other files).

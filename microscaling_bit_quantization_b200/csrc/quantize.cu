@@ -76,7 +76,6 @@ struct QuantArgs {
     int r;
     const float *w_ts;
     __nv_bfloat16 *tp;
-    unsigned int *err;       // device error word (a bounded wait that ran out)
 };
 
 // Streaming structure of the quantize kernels: each CTA owns a contiguous,
@@ -86,7 +85,6 @@ struct QuantArgs {
 // in registers, 64 KB per SM with two CTAs, so warps never wait on each
 // other and loads overlap the encoding.
 constexpr int kQThreads = 512;
-constexpr unsigned int kErrTimeoutQuant = 8u;
 
 // Raw bytes of one 16-element chunk (32 B of bf16 or 64 B of fp32).
 template <typename T>
@@ -238,13 +236,16 @@ __global__ void __launch_bounds__(kQThreads, 2) k_quantize(const T *__restrict__
             const float s = __fdiv_rn(amax, 7.0f);
             const Recip rs = recip_of(s);
             if (valid) {
-                const uint32_t b0 = int_x4_quot(v, rs, 7), b1 = int_x4_quot(v + 4, rs, 7);
-                const uint32_t b2 = int_x4_quot(v + 8, rs, 7), b3 = int_x4_quot(v + 12, rs, 7);
-                if (a.layout == 0)
+                if (a.layout == 0) {
+                    const uint32_t b0 = int_x4_quot(v, rs, 7), b1 = int_x4_quot(v + 4, rs, 7);
+                    const uint32_t b2 = int_x4_quot(v + 8, rs, 7), b3 = int_x4_quot(v + 12, rs, 7);
                     *reinterpret_cast<uint2 *>(a.codes + (int64_t)c * 8) =
                         make_uint2(nibbles_of_bytes(b0, b1), nibbles_of_bytes(b2, b3));
-                else
-                    *reinterpret_cast<uint4 *>(a.codes + (int64_t)c * 16) = make_uint4(b0, b1, b2, b3);
+                } else {   // MMA layout: E4M3 bytes of the integer codes
+                    *reinterpret_cast<uint4 *>(a.codes + (int64_t)c * 16) =
+                        make_uint4(int_x4_quot_e4m3(v, rs, 7), int_x4_quot_e4m3(v + 4, rs, 7),
+                                   int_x4_quot_e4m3(v + 8, rs, 7), int_x4_quot_e4m3(v + 12, rs, 7));
+                }
                 if ((lane & (G - 1)) == 0) {
                     float *sc = reinterpret_cast<float *>(a.scales);
                     const uint32_t g = colc / G;
@@ -375,8 +376,10 @@ __device__ __forceinline__ void dequant_chunk(const DequantArgs &a, int64_t c, f
         float s = a.layout == 0 ? sf[row * (a.cols / BLK) + g] : sf[g * a.rows + row];
 #pragma unroll
         for (int i = 0; i < 16; i++) {
-            int q = unpacked_int4 ? (int)(int8_t)code[i] : ((code[i] & 8u) ? (int)code[i] - 16 : (int)code[i]);
-            out[i] = __fmul_rn((float)q, s);
+            // MMA layout: E4M3 byte of the integer code; canonical: two's-complement nibble
+            const float q = unpacked_int4 ? dec_e4m3(code[i])
+                                          : (float)((code[i] & 8u) ? (int)code[i] - 16 : (int)code[i]);
+            out[i] = __fmul_rn(q, s);
         }
     } else if (F == kINT8Row) {
         float s = sf[row];
@@ -602,8 +605,6 @@ cudaError_t launch_amax(const void *x, bool bf16, int64_t rows, int64_t cols, in
     a.cpr = make_fastdiv((uint32_t)(cols / 16 > 0 ? cols / 16 : 1));
     a.hadamard_b = hadamard_b;
     a.amax_word = amax_word;
-    e = error_word_address(&a.err);
-    if (e != cudaSuccess) return e;
     if (bf16) launch_qf<__nv_bfloat16, kNumFmt>((const __nv_bfloat16 *)x, a, s);
     else launch_qf<float, kNumFmt>((const float *)x, a, s);
     return cudaGetLastError();
@@ -659,8 +660,6 @@ cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols
     a.r = pack ? pack->r : 0;
     a.w_ts = pack ? pack->w_ts : nullptr;
     a.tp = pack ? (__nv_bfloat16 *)pack->tp : nullptr;
-    e = error_word_address(&a.err);
-    if (e != cudaSuccess) return e;
     if (layout == 1 && fmt_byte_scales(fmt)) {
         int64_t S = cols / fmt_block(fmt);
         a.s_pad = (S + 15) / 16 * 16;

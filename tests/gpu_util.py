@@ -67,8 +67,11 @@ def assert_qtensor_equal(gq, oq, layout_mma=False):
     fmt, rows, cols = oq.fmt, oq.rows, oq.cols
     codes = gq.codes.cpu().numpy()
     if layout_mma and fmt in (INT4_G32, INT4_G64):
-        want = unpack4(oq.codes, rows).astype(np.uint8)
-        want = np.where(want & 8, want | 0xF0, want).astype(np.uint8)   # sign-extend nibbles
+        # MMA layout: the E4M3 byte of each integer code (exact for |q| <= 7, zero as +0)
+        q = unpack4(oq.codes, rows).astype(np.int32)
+        q = np.where(q & 8, q - 16, q).astype(np.float32)
+        want = torch.from_numpy(q).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        want = np.where(q == 0, 0, want).astype(np.uint8)
         np.testing.assert_array_equal(codes.reshape(rows, cols), want)
     else:
         np.testing.assert_array_equal(codes.reshape(oq.codes.shape), oq.codes)

@@ -86,8 +86,10 @@ def test_qlinear_argument_checks(mxq):
     assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(b), None, None, y, 0, None) == 1   # layout
     b = Q(mxq.NVFP4, mxq.MMA, 128, 192, 256, 256, 256)
     assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(b), None, None, y, 0, None) == 1   # K mismatch
-    i4 = Q(mxq.INT4_G64, mxq.MMA, 64, 256, 256, 256, 0)
-    assert L.mxq_qlinear(ctypes.byref(i4), ctypes.byref(i4), None, None, y, 0, None) == 2
+    i4 = Q(mxq.INT4_G64, mxq.MMA, 64, 96, 256, 256, 0)
+    assert L.mxq_qlinear(ctypes.byref(i4), ctypes.byref(i4), None, None, y, 0, None) == 1   # K % 64 (group)
+    i4 = Q(mxq.INT4_G32, mxq.CANONICAL, 64, 96, 256, 256, 0)
+    assert L.mxq_qlinear(ctypes.byref(i4), ctypes.byref(i4), None, None, y, 0, None) == 1   # layout
     a = Q(mxq.NVFP4, mxq.MMA, 64, 96, 256, 256, 256)
     assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(a), None, None, y, 0, None) == 1   # K % 64
     i8 = Q(mxq.INT8_ROW, mxq.MMA, 64, 256, 256, 256, 0)

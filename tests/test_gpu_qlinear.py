@@ -16,8 +16,8 @@ from gpu_util import assert_qtensor_equal, dev, gemm_close, host_values
 
 pytestmark = pytest.mark.gpu
 
-GEMM_FMTS = (2, 1, 0, 6, 5)   # NVFP4, MXFP4, MXFP8, FP8_TENSOR, INT8_ROW
-LOWRANK_FMTS = (2, 1, 0, 6)
+GEMM_FMTS = (2, 1, 0, 6, 5, 4, 3)   # NVFP4, MXFP4, MXFP8, FP8_TENSOR, INT8_ROW, INT4_G64, INT4_G32
+LOWRANK_FMTS = (2, 1, 0, 6, 4, 3)
 
 
 @pytest.fixture(scope="module")
@@ -64,8 +64,8 @@ def _ref(orc, fmt, d, r, rows=None, hadamard_b=0):
 @pytest.mark.parametrize("shape", [(200, 384, 512), (64, 128, 256), (130, 520, 320), (257, 256, 1024)])
 def test_qlinear_shapes(mxq, orc, fmt, shape):
     m, n, k = shape
-    if k % 64 and fmt in (1, 2):
-        pytest.skip("4-bit K must be a multiple of 64")
+    if k % 64 and fmt in (1, 2, 4):
+        pytest.skip("K must be a multiple of 64")
     d = _inputs(10 + fmt, m, n, k)
     ref, oxq, owq = _ref(orc, fmt, d, 0)
     for out_dtype in (torch.float32, torch.bfloat16):
@@ -77,7 +77,7 @@ def test_qlinear_shapes(mxq, orc, fmt, shape):
 
 @pytest.mark.parametrize("fmt", GEMM_FMTS)
 def test_qlinear_short_k(mxq, orc, fmt):
-    k = 64 if fmt in (1, 2) else 96
+    k = 64 if fmt in (1, 2, 4) else 96
     d = _inputs(20 + fmt, 70, 300, k)
     ref, _, _ = _ref(orc, fmt, d, 0)
     y, _, _ = _run(mxq, fmt, d, 0, torch.float32)
@@ -133,10 +133,11 @@ def _sample_rows(m, seed, count=256):
     return rows
 
 
-@pytest.mark.parametrize("fmt", [2, 1])
+@pytest.mark.parametrize("fmt", [2, 1, 4])
 def test_svdquant_mlp_up_full_size(mxq, orc, fmt):
     """Workload 3 at full size (4096 x 12288 x 3072, rank 32) in the launch
-    configuration the benchmark times; 256 sampled rows x all columns."""
+    configuration the benchmark times (NVFP4 and the INT4-g64 variant, plus
+    MXFP4); 256 sampled rows x all columns."""
     d = workloads.svdquant_mlp_up()
     rows = _sample_rows(4096, 3)
     ref, _, _ = _ref(orc, fmt, d, 32, rows=rows)
@@ -203,3 +204,22 @@ def test_svdquant_fused_path_full_size(mxq, orc):
     y = mxq.qlinear(xq, wq, tp, l2p, out_dtype=torch.bfloat16)
     assert mxq.check() == 0
     gemm_close(y[torch.from_numpy(rows).cuda()].float().cpu().numpy(), ref, bf16_out=True)
+
+
+@pytest.mark.parametrize("fmt", [4, 3])
+def test_igroup_ragged_and_degenerate(mxq, orc, fmt):
+    """INT4 group GEMM: ragged M and N (not multiples of the 128 x 128 tile),
+    a K that leaves half a pipeline stage, all-zero activation rows and weight
+    rows (group scale 0), and more tiles than SMs."""
+    g = 64 if fmt == 4 else 32
+    for m, n, k in ((1, 8, g), (129, 136, 3 * g), (300, 1000, 5 * g)):
+        d = _inputs(50 + fmt, m, n, k, 16)
+        d["x"][m // 2] = 0.0
+        d["w"][n // 3] = 0.0
+        ref, _, _ = _ref(orc, fmt, d, 16)
+        y, _, _ = _run(mxq, fmt, d, 16, torch.float32)
+        gemm_close(y.cpu().numpy(), ref)
+    d = _inputs(60 + fmt, 1100, 2400, 256)   # 9 x 19 tiles > 148 SMs: persistent CTAs take several
+    ref, _, _ = _ref(orc, fmt, d, 0, rows=_sample_rows(1100, 7))
+    y, _, _ = _run(mxq, fmt, d, 0, torch.float32)
+    gemm_close(y[torch.from_numpy(_sample_rows(1100, 7)).cuda()].cpu().numpy(), ref)
