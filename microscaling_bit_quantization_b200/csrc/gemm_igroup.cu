@@ -25,7 +25,10 @@
 //               thread that issues the MMAs (cta_group::1)
 //   warps 2-9   epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 (its 32
 //               rows) and one half of the 128 columns ((w - 2) / 4), keeps
-//               64 running sums per thread and stores its rows of Y
+//               64 running sums per thread and stores its rows of Y.  TMEM
+//               loads run one half-group (32 columns) ahead of the arithmetic,
+//               and each warp's group scales arrive by cp.async in a ring of
+//               shared-memory slots IG_SCALE_AHEAD groups ahead of their use
 // The low-rank branch is one more group with scale 1: a bf16 kind::f16 MMA
 // of the packed activation [T_hi | T_lo] against [L2^T | L2^T].
 // Every wait is bounded; a wait that runs out latches the error word and
@@ -50,8 +53,11 @@ constexpr int IG_STAGE = IG_A + IG_B;
 constexpr int IG_NBUF = 4;                                    // TMEM group buffers
 constexpr uint32_t IG_TMEM_COLS = IG_NBUF * IG_BN;            // 512
 constexpr int IG_EPI_WARPS = 8;
+constexpr int IG_EPI_COLS = IG_BN / (IG_EPI_WARPS / 4);        // 64 columns per epilogue warp
 constexpr int IG_THREADS = 64 + 32 * IG_EPI_WARPS;            // 320
-constexpr int IG_WSCALE_BYTES = IG_EPI_WARPS * 2 * 64 * 4;    // per epilogue warp: two buffers of 64 column scales
+constexpr int IG_SCALE_SLOTS = 8, IG_SCALE_AHEAD = 6;          // per-warp scale ring: slots, groups in flight
+constexpr int IG_SLOT_FLOATS = 32 + IG_EPI_COLS;              // sx of the warp's 32 rows, sw of its columns
+constexpr int IG_WSCALE_BYTES = IG_EPI_WARPS * IG_SCALE_SLOTS * IG_SLOT_FLOATS * 4;
 constexpr int IG_BAR_BYTES = 256;
 constexpr int IG_SMEM = IG_STAGES * IG_STAGE + IG_WSCALE_BYTES + IG_BAR_BYTES + 1024;
 
@@ -90,6 +96,15 @@ __device__ __forceinline__ void mma_bf16_1(uint32_t d, uint64_t a, uint64_t b, u
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
         "l"(a), "l"(b), "r"(kIdescBF16), "r"(acc));
 }
+// 4-byte asynchronous copy global -> shared; src_bytes 0 writes a zero.
+__device__ __forceinline__ void cp_async4(void *dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 // Arrive on this CTA's barrier once this thread's issued MMAs complete.
 __device__ __forceinline__ void tc_commit_1(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -104,7 +119,7 @@ __global__ void __launch_bounds__(IG_THREADS, 1) k_gemm_igroup(const __grid_cons
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + IG_STAGES * IG_STAGE + IG_WSCALE_BYTES);
     uint64_t *empty = full + IG_STAGES;
     uint64_t *bfull = empty + IG_STAGES;   // group buffer written (MMA commit)
-    uint64_t *bempty = bfull + IG_NBUF;    // group buffer read (8 epilogue warps)
+    uint64_t *bempty = bfull + IG_NBUF;    // group buffer read (all epilogue warps)
     uint64_t *drain = bempty + IG_NBUF;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -220,89 +235,94 @@ __global__ void __launch_bounds__(IG_THREADS, 1) k_gemm_igroup(const __grid_cons
         }
     } else {
         // ---------------------------------------------------------- epilogue
-        const int e = warp - 2, q = warp & 3, h = e >> 2;
-        float *wbuf = wscale + e * 128;   // two buffers of 64 column scales
-        const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * 64);
+        const int e = warp - 2, q = warp & 3, cq = e >> 2;
+        float *ring = wscale + e * IG_SCALE_SLOTS * IG_SLOT_FLOATS;
+        const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(cq * IG_EPI_COLS);
         uint32_t gc = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
             const int m0 = (tile / p.n_tiles) * IG_BM, n0 = (tile % p.n_tiles) * IG_BN;
             const int row = m0 + q * 32 + lane;
-            const int col0 = n0 + h * 64;
+            const int col0 = n0 + cq * IG_EPI_COLS;
             const bool row_ok = row < p.m;
-            // this thread's part of the next group's scales: sx of its row, sw of columns col0 + 2 lane (+1)
-            float sx_next = 0.0f;
-            float2 sw_next = make_float2(0.0f, 0.0f);
-            auto load_scales = [&](int g) {
-                sx_next = row_ok ? __ldg(p.sx + (int64_t)g * p.m + row) : 0.0f;
-                const int c = col0 + 2 * lane;
-                sw_next.x = c < p.n ? __ldg(p.sw + (int64_t)g * p.n + c) : 0.0f;
-                sw_next.y = c + 1 < p.n ? __ldg(p.sw + (int64_t)g * p.n + c + 1) : 0.0f;
-            };
-            if (p.groups > 0) load_scales(0);
-            float acc[64];
-#pragma unroll
-            for (int j = 0; j < 64; j++) acc[j] = 0.0f;
-            bool ok = true;
-#pragma unroll 1
-            for (int gi = 0; gi < ngroups; gi++, gc++) {
-                const bool lr = gi >= p.groups;
-                const float sxv = sx_next;
-                float *buf = wbuf + (gi & 1) * 64;
-                if (!lr) {
-                    reinterpret_cast<float2 *>(buf)[lane] = sw_next;
-                    if (gi + 1 < p.groups) load_scales(gi + 1);
+            // group g's scales into slot g % IG_SCALE_SLOTS: sx of this lane's row, sw of columns
+            // col0 + lane and col0 + 32 + lane (zeros past the matrix); one commit group per group
+            auto fetch_scales = [&](int g) {
+                if (g < p.groups) {
+                    float *slot = ring + (g % IG_SCALE_SLOTS) * IG_SLOT_FLOATS;
+                    const int c0 = col0 + lane, c1 = col0 + 32 + lane;
+                    cp_async4(slot + lane, p.sx + (int64_t)g * p.m + (row_ok ? row : 0), row_ok ? 4u : 0u);
+                    cp_async4(slot + 32 + lane, p.sw + (int64_t)g * p.n + (c0 < p.n ? c0 : 0), c0 < p.n ? 4u : 0u);
+                    cp_async4(slot + 64 + lane, p.sw + (int64_t)g * p.n + (c1 < p.n ? c1 : 0), c1 < p.n ? 4u : 0u);
                 }
-                const uint32_t b = gc % IG_NBUF;
-                bool w = !*abort_flag && mbar_wait(bfull + b, (gc / IG_NBUF) & 1, p.wait_ns);
+                cp_async_commit();
+            };
+            auto wait_group = [&](uint32_t g) {
+                bool w = !*abort_flag && mbar_wait(bfull + g % IG_NBUF, (g / IG_NBUF) & 1, p.wait_ns);
                 w = __all_sync(0xFFFFFFFFu, w);
                 if (!w) {
                     if (lane == 0 && !*abort_flag) atomicOr(p.err, kErrIgEpilogue);
                     *abort_flag = 1;
-                    ok = false;
-                    break;
                 }
                 tc_fence_after();
-                uint32_t r0[32], r1[32];
-                tmem_ld_32x32b_x32(lane_base + b * IG_BN, r0);
-                tmem_ld_32x32b_x32(lane_base + b * IG_BN + 32, r1);
-                tc_fence_before();
-                __syncwarp();   // also orders this group's scale stores before the loads below
-                if (lane == 0) mbar_arrive_local(bempty + b);
+                return w;
+            };
+            // acc[j] += P[j] * (sx * sw[j]) for the 32 columns of one half; factor 1 for the branch
+            float acc[IG_EPI_COLS];
+#pragma unroll
+            for (int j = 0; j < IG_EPI_COLS; j++) acc[j] = 0.0f;
+            auto fold = [&](const uint32_t (&r)[32], float *accp, const float *sw, float sxv, bool lr) {
                 if (lr) {
 #pragma unroll
-                    for (int j = 0; j < 32; j++) {
-                        acc[j] = __fadd_rn(acc[j], __uint_as_float(r0[j]));
-                        acc[32 + j] = __fadd_rn(acc[32 + j], __uint_as_float(r1[j]));
-                    }
+                    for (int j = 0; j < 32; j++) accp[j] = __fadd_rn(accp[j], __uint_as_float(r[j]));
                 } else {
-                    const float4 *sw4 = reinterpret_cast<const float4 *>(buf);
+                    const float4 *sw4 = reinterpret_cast<const float4 *>(sw);
 #pragma unroll
                     for (int jj = 0; jj < 8; jj++) {
                         const float4 w4 = sw4[jj];
-                        acc[4 * jj] = __fmaf_rn(__uint_as_float(r0[4 * jj]), __fmul_rn(sxv, w4.x), acc[4 * jj]);
-                        acc[4 * jj + 1] = __fmaf_rn(__uint_as_float(r0[4 * jj + 1]), __fmul_rn(sxv, w4.y), acc[4 * jj + 1]);
-                        acc[4 * jj + 2] = __fmaf_rn(__uint_as_float(r0[4 * jj + 2]), __fmul_rn(sxv, w4.z), acc[4 * jj + 2]);
-                        acc[4 * jj + 3] = __fmaf_rn(__uint_as_float(r0[4 * jj + 3]), __fmul_rn(sxv, w4.w), acc[4 * jj + 3]);
-                    }
-#pragma unroll
-                    for (int jj = 0; jj < 8; jj++) {
-                        const float4 w4 = sw4[8 + jj];
-                        acc[32 + 4 * jj] = __fmaf_rn(__uint_as_float(r1[4 * jj]), __fmul_rn(sxv, w4.x), acc[32 + 4 * jj]);
-                        acc[33 + 4 * jj] =
-                            __fmaf_rn(__uint_as_float(r1[4 * jj + 1]), __fmul_rn(sxv, w4.y), acc[33 + 4 * jj]);
-                        acc[34 + 4 * jj] =
-                            __fmaf_rn(__uint_as_float(r1[4 * jj + 2]), __fmul_rn(sxv, w4.z), acc[34 + 4 * jj]);
-                        acc[35 + 4 * jj] =
-                            __fmaf_rn(__uint_as_float(r1[4 * jj + 3]), __fmul_rn(sxv, w4.w), acc[35 + 4 * jj]);
+                        accp[4 * jj] = __fmaf_rn(__uint_as_float(r[4 * jj]), __fmul_rn(sxv, w4.x), accp[4 * jj]);
+                        accp[4 * jj + 1] = __fmaf_rn(__uint_as_float(r[4 * jj + 1]), __fmul_rn(sxv, w4.y), accp[4 * jj + 1]);
+                        accp[4 * jj + 2] = __fmaf_rn(__uint_as_float(r[4 * jj + 2]), __fmul_rn(sxv, w4.z), accp[4 * jj + 2]);
+                        accp[4 * jj + 3] = __fmaf_rn(__uint_as_float(r[4 * jj + 3]), __fmul_rn(sxv, w4.w), accp[4 * jj + 3]);
                     }
                 }
+            };
+            for (int g = 0; g < IG_SCALE_AHEAD; g++) fetch_scales(g);
+            bool ok = wait_group(gc);
+            uint32_t ra[32], rb[32];
+#pragma unroll
+            for (int j = 0; j < 32; j++) ra[j] = 0u;
+            if (ok) tmem_ld_32x32b_x32_async(lane_base + (gc % IG_NBUF) * IG_BN, ra);
+            tmem_ld_wait(ra);
+#pragma unroll 1
+            for (int gi = 0; ok && gi < ngroups; gi++, gc++) {
+                const bool lr = gi >= p.groups;
+                // slot gi + AHEAD was last read by group gi + AHEAD - SLOTS < gi, before the previous __syncwarp
+                fetch_scales(gi + IG_SCALE_AHEAD);
+                cp_async_wait<IG_SCALE_AHEAD>();   // this group's copies (all but the newest AHEAD) have landed
+                __syncwarp();                      // ... for every lane of the warp
+                const float *slot = ring + (gi % IG_SCALE_SLOTS) * IG_SLOT_FLOATS;
+                const float sxv = lr ? 1.0f : slot[lane];
+                const uint32_t b = gc % IG_NBUF;
+                tmem_ld_32x32b_x32_async(lane_base + b * IG_BN + 32, rb);   // second half, in flight
+                fold(ra, acc, slot + 32, sxv, lr);
+                tmem_ld_wait(rb);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_local(bempty + b);   // the MMAs may reuse this buffer
+                if (gi + 1 < ngroups) {
+                    ok = wait_group(gc + 1);
+                    if (ok) tmem_ld_32x32b_x32_async(lane_base + ((gc + 1) % IG_NBUF) * IG_BN, ra);   // next first half
+                }
+                fold(rb, acc + 32, slot + 64, sxv, lr);
+                tmem_ld_wait(ra);
             }
+            cp_async_wait<0>();
             if (!ok) break;
             if (row_ok) {
                 if (p.y_bf16) {
                     __nv_bfloat16 *yr = reinterpret_cast<__nv_bfloat16 *>(p.y) + (int64_t)row * p.n + col0;
 #pragma unroll
-                    for (int jj = 0; jj < 8; jj++) {
+                    for (int jj = 0; jj < IG_EPI_COLS / 8; jj++) {
                         const int c = col0 + 8 * jj;
                         if (p.y_vec && c + 8 <= p.n) {
                             reinterpret_cast<uint4 *>(yr)[jj] =
@@ -319,7 +339,7 @@ __global__ void __launch_bounds__(IG_THREADS, 1) k_gemm_igroup(const __grid_cons
                 } else {
                     float *yr = reinterpret_cast<float *>(p.y) + (int64_t)row * p.n + col0;
 #pragma unroll
-                    for (int jj = 0; jj < 16; jj++) {
+                    for (int jj = 0; jj < IG_EPI_COLS / 4; jj++) {
                         const int c = col0 + 4 * jj;
                         if (p.y_vec && c + 4 <= p.n) {
                             reinterpret_cast<float4 *>(yr)[jj] =
