@@ -43,6 +43,13 @@ cudaError_t launch_select(const void *w, bool bf16, int64_t n, int64_t k, const 
 cudaError_t launch_lowrank_down(const void *x, bool bf16, int64_t m, int64_t k, const void *l1, int r,
                                 float *t, const float *xs, const float *ws, void *tp, cudaStream_t s,
                                 unsigned int *amax_word = nullptr);
+// Tensor-core down-projection of bf16 x (one pass over x): writes t (m x r
+// fp32) or, when t is null, the packed operand tp (as launch_lowrank_down);
+// with amax_word (zeroed beforehand) also folds in max |x|.  Returns
+// cudaErrorNotSupported, launching nothing, for shapes it does not take
+// (k % 8, unaligned x, a K slice that does not fit in shared memory).
+cudaError_t launch_lowrank_tc(const void *x, int64_t m, int64_t k, const void *l1, int r, float *t, void *tp,
+                              const float *xs, const float *ws, unsigned int *amax_word, cudaStream_t s);
 cudaError_t launch_pack_l2(const void *l2, int r, int64_t n, void *l2p, cudaStream_t s);
 cudaError_t launch_pack_t(const float *t, int r, int64_t m, const float *xs, const float *ws, void *tp,
                           cudaStream_t s);
