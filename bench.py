@@ -68,7 +68,7 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), "--query-gpu=" + self.FIELDS,
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.th = threading.Thread(target=self._read, daemon=True)
             self.th.start()
@@ -90,7 +90,7 @@ class ClockSampler:
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.15)
+        time.sleep(0.08)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -156,23 +156,24 @@ def _barrier(world):
 # ------------------------------------------------------------------ oracle
 
 class OracleSample:
-    """The oracle as it stands, on `rows` token rows of the workload per step:
-    NVFP4 quantization (C), low-rank down projection (C), binary64 GEMM over
-    exactly dequantized operands (numpy matmul, one BLAS thread), which
-    dequantizes the whole 12288 x 3072 weight each call."""
+    """The oracle as it stands, on a bounded sample of the workload per step:
+    `rows` token rows of X against the first `cols` output channels of the
+    weight -- NVFP4 quantization (C), low-rank down projection (C), binary64
+    GEMM over exactly dequantized operands (numpy matmul, one BLAS thread),
+    which dequantizes its weight slice on every call."""
 
-    def __init__(self, rows=64):
+    def __init__(self, rows=64, cols=N):
         import oracle
         import workloads
         d = workloads.svdquant_mlp_up()
-        self.rows = rows
+        self.rows, self.cols = rows, cols
         self.x = d["x"][:rows].copy()
-        self.l1, self.l2 = d["l1"], d["l2"]
-        self.wq = oracle.quantize(d["w"], oracle.NVFP4)
-        self.flops = 2 * rows * N * K + 2 * rows * N * RANK + 2 * rows * K * RANK
-        self.desc = ("%d of %d token rows per step: NVFP4 quantize, low-rank down projection, binary64 GEMM "
-                     "over exactly dequantized operands (incl. dequantizing the 12288 x 3072 weight); "
-                     "1 thread" % (rows, M))
+        self.l1, self.l2 = d["l1"], d["l2"][:, :cols].copy()
+        self.wq = oracle.quantize(d["w"][:cols].copy(), oracle.NVFP4)
+        self.flops = 2 * rows * cols * K + 2 * rows * cols * RANK + 2 * rows * K * RANK
+        self.desc = ("%d of %d token rows x %d of %d output channels per step: NVFP4 quantize, low-rank down "
+                     "projection, binary64 GEMM over exactly dequantized operands (incl. dequantizing the "
+                     "%d x %d weight slice); 1 thread" % (rows, M, cols, N, cols, K))
 
     def step(self):
         import oracle
@@ -192,7 +193,7 @@ class OracleSample:
 def run_reference(args, world, rank):
     if rank != 0:
         return
-    o = OracleSample()
+    o = OracleSample(rows=8, cols=512)   # ~40 ms per step: --steps in the thousands still ends in minutes
     o.timed(args.warmup)
     sec = o.timed(args.steps)
     value = o.flops / sec / 1e12
@@ -200,7 +201,8 @@ def run_reference(args, world, rank):
             "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * sec, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "m": M, "k": K, "n": N, "rank": RANK, "sample_rows": o.rows},
+            "config": {"workload": WORKLOAD, "m": M, "k": K, "n": N, "rank": RANK, "sample_rows": o.rows,
+                       "sample_cols": o.cols},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": o.desc},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -244,28 +246,41 @@ def run_ours(args, world, rank, local):
         sets.append(s)
     del w, wq0
 
-    def step(i):
+    def quant(i):
         s = sets[i % N_SETS]
         mxq.quantize_lowrank(s["x"], mxq.NVFP4, l1, s["wq"], 0, out=s["xq"], tp=s["tp"], workspace=s["qws"])
+
+    def gemm(i):
+        s = sets[i % N_SETS]
         mxq.qlinear(s["xq"], s["wq"], s["tp"], s["l2p"], out=s["y"])
 
-    launches_per_step = 3      # k_lowrank (t + tensor amax), k_quantize (codes, scales, packed t), k_gemm
+    def step(i):
+        quant(i)
+        gemm(i)
 
-    for i in range(args.warmup):
+    launches_per_step = 3      # k_lowrank_tc (T + tensor amax), k_quantize (codes, scales, packed T), k_gemm
+
+    for i in range(max(args.warmup, N_SETS)):   # every input set has been through the path once
         step(i)
     torch.cuda.synchronize()
     assert mxq.check() == 0
 
-    # ---- timed region
+    # ---- timed region: events around each kernel group on the launching stream (the queue
+    # stays full, so each interval is device time); step time from the outer pair
     sampler = ClockSampler(local)
     sampler.start()
     sampler.wait_ready()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     _barrier(world)
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for i in range(args.steps):
-        step(i)
+        ev[i][0].record(stream)
+        quant(i)
+        ev[i][1].record(stream)
+        gemm(i)
+        ev[i][2].record(stream)
     end.record(stream)
     torch.cuda.synchronize()
     _barrier(world)
@@ -273,33 +288,12 @@ def run_ours(args, world, rank, local):
     ms_local = start.elapsed_time(end) / args.steps
     ms, value = job_throughput(ms_local, world, FLOP_STEP)
     assert mxq.check() == 0
-
-    # ---- per-kernel durations of the dominant kernel (GEMM) and the quantizer, on the launch stream
-    def time_kernel(fn, reps):
-        evs = []
-        for i in range(reps):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            fn(i)
-            b.record(stream)
-            evs.append((a, b))
-        torch.cuda.synchronize()
-        return statistics.mean(a.elapsed_time(b) for a, b in evs)
-
-    def gemm_only(i):
-        s = sets[i % N_SETS]
-        mxq.qlinear(s["xq"], s["wq"], s["tp"], s["l2p"], out=s["y"])
-
-    def quant_only(i):
-        s = sets[i % N_SETS]
-        mxq.quantize_lowrank(s["x"], mxq.NVFP4, l1, s["wq"], 0, out=s["xq"], tp=s["tp"], workspace=s["qws"])
-
-    reps = max(args.steps, 10)
-    gemm_ms = time_kernel(gemm_only, reps)
-    quant_ms = time_kernel(quant_only, reps)
+    quant_ms = statistics.median(e[0].elapsed_time(e[1]) for e in ev)
+    gemm_ms = statistics.median(e[1].elapsed_time(e[2]) for e in ev)
 
     peaks = _peaks()
     fp4_peak = peaks["bf16_tflops"] * 4.0          # nominal dense FP4 : BF16 ratio 9 : 2.25
+    int8_peak = peaks["bf16_tflops"] * 2.0         # nominal dense INT8/FP8 : BF16 ratio 4.5 : 2.25
     gemm_flops = FLOP_MAIN + FLOP_LR_UP
     gemm_tflops = gemm_flops / (gemm_ms * 1e-3) / 1e12
     # algorithmic bytes of the activation side: read bf16 X once, write codes, scales, packed T
@@ -311,6 +305,54 @@ def run_ours(args, world, rank, local):
             profiles_traffic = json.load(f).get("k_gemm_nvfp4")
     except Exception:
         pass
+
+    # ---- the other rows of the measurement table, timed alone by CUDA-graph replay
+    def graph_ms(fn, n=12, reps=5):
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            fn(0)
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(n):
+                fn(i)
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        del g
+        return a.elapsed_time(b) / (reps * n)
+
+    qws = torch.empty(16, dtype=torch.uint8, device=dev)
+    formats = {}
+    for name, fmt, had in (("NVFP4", mxq.NVFP4, 0), ("MXFP4", mxq.MXFP4, 0), ("MXFP4+hadamard128", mxq.MXFP4, 128),
+                           ("MXFP8", mxq.MXFP8, 0), ("INT4_G64", mxq.INT4_G64, 0), ("INT8_ROW", mxq.INT8_ROW, 0),
+                           ("FP8_TENSOR", mxq.FP8_TENSOR, 0)):
+        outs = [mxq.alloc_qtensor(fmt, M, K, mxq.MMA, dev) for _ in range(N_SETS)]
+        t_ms = graph_ms(lambda i: mxq.quantize(sets[i % N_SETS]["x"], fmt, had, mxq.MMA, out=outs[i % N_SETS],
+                                               workspace=qws))
+        nbytes = M * K * 2 + mxq.codes_bytes(fmt, M, K, mxq.CANONICAL) + mxq.scales_bytes(fmt, M, K, mxq.CANONICAL)
+        formats[name] = {"us": 1e3 * t_ms, "GB/s": nbytes / (t_ms * 1e-3) / 1e9,
+                         "frac": nbytes / (t_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+        del outs
+    w4 = workloads.svdquant_mlp_up()["w"]
+    wq4 = mxq.quantize(torch.from_numpy(w4).to(torch.bfloat16).to(dev), mxq.INT4_G64, 0, mxq.MMA)
+    del w4
+    xq4 = mxq.quantize(sets[0]["x"], mxq.INT4_G64, 0, mxq.MMA)
+    tp4 = mxq.lowrank_down_packed(sets[0]["x"], l1, xq4, wq4)
+    i4_ms = graph_ms(lambda i: mxq.qlinear(xq4, wq4, tp4, sets[0]["l2p"], out=sets[i % N_SETS]["y"]), n=4, reps=3)
+    i4_tf = gemm_flops / (i4_ms * 1e-3) / 1e12
+    int4 = {"kernel": "k_gemm_igroup<64> (E4M3-coded INT4 groups on kind::f8f6f4, fp32 group rescale in the epilogue)",
+            "us": 1e3 * i4_ms, "TFLOP/s": i4_tf, "frac_of_int8_peak": i4_tf / int8_peak,
+            "int8_peak": int8_peak}
+    del wq4, xq4, tp4
+    assert mxq.check() == 0
 
     # ---- end to end through the public API with host buffers
     x_pin = x_host.pin_memory()
@@ -358,10 +400,14 @@ def run_ours(args, world, rank, local):
                          "peak_note": "measured bf16 burst %.1f TF/s x 4 (nominal dense FP4:BF16), of %s"
                                       % (peaks["bf16_tflops"], peaks["src"]),
                          "gemm_ms": gemm_ms, "flops_per_launch": gemm_flops},
-            "quantize": {"kernel": "k_lowrank (T + tensor amax) + k_quantize<NVFP4> (codes, scales, packed T), "
+            "quantize": {"kernel": "k_lowrank_tc (T + tensor amax) + k_quantize<NVFP4> (codes, scales, packed T), "
                                    "X 4096 x 3072 bf16", "ms": quant_ms,
                          "achieved": quant_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": quant_gbs / peaks["hbm_gbs"], "bytes_per_launch": quant_bytes},
+            "quantize_formats": {"shape": "4096 x 3072 bf16, MMA layout, alone (graph replay)",
+                                 "bytes": "read 2 B/element + canonical codes and scales", "peak_GB/s": peaks["hbm_gbs"],
+                                 "rows": formats},
+            "int4_g64_qlinear": int4,
             "e2e": {"value": world * FLOP_STEP / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "ms_per_step": e2e_ms},
             "gpu_launches": launches_per_step * args.steps,
@@ -374,8 +420,8 @@ def run_ours(args, world, rank, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=2000)   # ~0.3 s timed: a few clock samples
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     args = ap.parse_args()
     if args.warmup < 3:
