@@ -68,13 +68,23 @@ constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
 constexpr int kGemmThreads = 256;   // 8 warps
 constexpr uint32_t TMEM_COLS = 512;
-// TMEM columns: accumulator stage 0 at [0, 256), stage 1 at [160, 416)
-// (the stages share 96 columns), then two groups of four 12-column
-// scale-factor slots at [416, 512) (SFA 4 columns, the two SFB halves 4 + 4
-// per atom).  K-tile i uses group i % 2, so a group is rewritten only after
-// the MMAs of k-tile i - 2 have completed.
-constexpr uint32_t ACC_STAGE1 = 160, OVL_CHUNKS = 3;
-constexpr uint32_t TMEM_SF = 416, SF_SLOT_COLS = 12, SF_GROUP_COLS = 48;
+// TMEM columns: accumulator stage 0 at [0, 256), stage 1 at
+// [ACC_STAGE1, ACC_STAGE1 + 256) (the two stages share 256 - ACC_STAGE1
+// columns), then SF_GROUPS groups of four 12-column scale-factor slots (SFA 4
+// columns, the two SFB halves 4 + 4 per atom) up to column 512.  K-tile i uses
+// group i % SF_GROUPS, so the scale factors of k-tile i are copied once the
+// MMAs of k-tile i - SF_GROUPS have completed: more groups let the copies run
+// further ahead of the MMAs, at the price of more shared accumulator columns
+// (which the epilogue drains first, before the next tile's MMAs may start).
+#ifndef MXQ_SF_GROUPS
+#define MXQ_SF_GROUPS 2
+#endif
+constexpr uint32_t SF_GROUPS = MXQ_SF_GROUPS;
+constexpr uint32_t SF_SLOT_COLS = 12, SF_GROUP_COLS = 48;
+constexpr uint32_t TMEM_SF = TMEM_COLS - SF_GROUPS * SF_GROUP_COLS;
+constexpr uint32_t ACC_STAGE1 = (TMEM_SF - 256) & ~31u;    // 32-column aligned
+constexpr uint32_t OVL_CHUNKS = (256 - ACC_STAGE1) / 32;   // shared 32-column chunks
+static_assert(ACC_STAGE1 + 256 <= TMEM_SF && OVL_CHUNKS >= 1 && OVL_CHUNKS <= 8, "TMEM budget");
 
 enum Kind : int { kKindNVFP4 = 0, kKindMXFP4 = 1, kKindMXFP8 = 2, kKindFP8 = 3, kKindINT8 = 4 };
 
@@ -339,7 +349,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                     if (kt < p.num_k_tiles) {
                         const int rem = (p.kbytes - kt * BKB) >> 5;
                         const int nks = rem < 4 ? rem : 4;
-                        const uint32_t group = tmem + TMEM_SF + SF_GROUP_COLS * (uint32_t)(it & 1);
+                        const uint32_t group = tmem + TMEM_SF + SF_GROUP_COLS * ((uint32_t)it % SF_GROUPS);
                         for (int ks = 0; ks < nks; ks++) {
                             const uint64_t ad = sdesc_sw128(sa + ks * 32), bd = sdesc_sw128(sb + ks * 32);
                             const uint32_t accum = (kt > 0 || ks > 0) ? 1u : 0u;
@@ -391,8 +401,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 for (int kt = 0; kt < nsteps; kt++, it++) {
                     const int s = it % STAGES;
                     ok = mbar_wait(full + s, (it / STAGES) & 1, p.wait_ns);
-                    // slot group it % 2 was last read by the MMAs of k-tile it - 2
-                    if (ok && it >= 2) ok = mbar_wait(empty + ((it - 2) % STAGES), ((it - 2) / STAGES) & 1, p.wait_ns);
+                    // slot group it % SF_GROUPS was last read by the MMAs of k-tile it - SF_GROUPS
+                    const int prev = it - (int)SF_GROUPS;
+                    if (ok && prev >= 0) ok = mbar_wait(empty + (prev % STAGES), (prev / STAGES) & 1, p.wait_ns);
                     if (!ok || *abort_flag) {
                         if (!ok) latch_error(kErrTimeoutMma);
                         *abort_flag = 1;
@@ -403,7 +414,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                         const int nks = rem < 4 ? rem : 4;
                         const int natoms = NSF == 4 ? nks : NSF == 2 ? (nks + 1) >> 1 : 1;
                         const uint8_t *sf = smem + s * STAGE_BYTES + A_STAGE + B_STAGE;
-                        const uint32_t group = tmem + TMEM_SF + SF_GROUP_COLS * (uint32_t)(it & 1);
+                        const uint32_t group = tmem + TMEM_SF + SF_GROUP_COLS * ((uint32_t)it % SF_GROUPS);
                         tc_fence_after();
                         for (int a = par; a < natoms; a += 2) {
                             const uint32_t base = group + SF_SLOT_COLS * (uint32_t)a;
@@ -448,80 +459,96 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             if (KIND == kKindNVFP4 || KIND == kKindFP8) alpha = __fmul_rn(__ldg(p.a_ts), __ldg(p.b_ts));
             const bool row_ok = row < p.m;
             if (KIND == kKindINT8 && row_ok) ra = __ldg(p.a_row_scale + row);
-            // the 96 shared columns first: the last three chunks of stage 0, the first three of stage 1
-#pragma unroll 1
-            for (int i = 0; i < BN / 32; i++) {
-                const int c = st ? i : (i + 8 - (int)OVL_CHUNKS) & 7;
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(lane_base + (uint32_t)(c * 32), r);
-                if (i == (int)OVL_CHUNKS - 1 || i == 7) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive_remote(i == (int)OVL_CHUNKS - 1 ? ovl_leader : (st ? acce_leader1 : acce_leader0));
-                }
-                const int nb = n0 + c * 32;
-                float v[32];
-                scale_chunk<KIND>(r, v, alpha, ra, p.b_row_scale + nb, p.n - nb);
-                if (p.y_tma) {
-                    // swizzled staging of this 32-column chunk, then one TMA store of 32 rows:
-                    // bf16 rows of 64 B (64B swizzle: 16-byte unit j of row t at t*64 + (j ^ ((t >> 1) & 3))*16),
-                    // fp32 rows of 128 B (128B swizzle: unit j at t*128 + (j ^ (t & 7))*16)
-                    uint8_t *buf = stage_buf + (sub & 1) * EPI_BUF;
-                    if (lane == 0) bulk_wait_read1();
-                    __syncwarp();
-                    if (p.y_bf16) {
-                        uint4 *rowp = reinterpret_cast<uint4 *>(buf + lane * 64);
-#pragma unroll
-                        for (int k4 = 0; k4 < 4; k4++)
-                            rowp[k4 ^ ((lane >> 1) & 3)] =
-                                make_uint4(pack_bf16x2(v[8 * k4], v[8 * k4 + 1]), pack_bf16x2(v[8 * k4 + 2], v[8 * k4 + 3]),
-                                           pack_bf16x2(v[8 * k4 + 4], v[8 * k4 + 5]),
-                                           pack_bf16x2(v[8 * k4 + 6], v[8 * k4 + 7]));
-                    } else {
-                        uint4 *rowp = reinterpret_cast<uint4 *>(buf + lane * 128);
-#pragma unroll
-                        for (int k4 = 0; k4 < 8; k4++)
-                            rowp[k4 ^ (lane & 7)] = make_uint4(__float_as_uint(v[4 * k4]), __float_as_uint(v[4 * k4 + 1]),
-                                                               __float_as_uint(v[4 * k4 + 2]), __float_as_uint(v[4 * k4 + 3]));
-                    }
-                    fence_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&p.tma_y, buf, nb, row0);
-                        bulk_commit();
-                    }
-                    sub++;
-                } else if (row_ok && nb < p.n) {
-                    if (p.y_bf16) {
-                        __nv_bfloat16 *yrow = reinterpret_cast<__nv_bfloat16 *>(p.y) + (int64_t)row * p.n;
-                        if (vec && nb + 32 <= p.n) {
-                            uint4 *dst = reinterpret_cast<uint4 *>(yrow + nb);
+            // The shared columns (the last OVL_CHUNKS chunks of stage 0, the first OVL_CHUNKS of
+            // stage 1) go to registers first and are released at once, so the next tile's MMAs
+            // wait only for these loads; then every chunk is scaled, staged and stored.
+            auto process = [&](const int c, const uint32_t (&r)[32]) {
+                    const int nb = n0 + c * 32;
+                    float v[32];
+                    scale_chunk<KIND>(r, v, alpha, ra, p.b_row_scale + nb, p.n - nb);
+                    if (p.y_tma) {
+                        // swizzled staging of this 32-column chunk, then one TMA store of 32 rows:
+                        // bf16 rows of 64 B (64B swizzle: 16-byte unit j of row t at t*64 + (j ^ ((t >> 1) & 3))*16),
+                        // fp32 rows of 128 B (128B swizzle: unit j at t*128 + (j ^ (t & 7))*16)
+                        uint8_t *buf = stage_buf + (sub & 1) * EPI_BUF;
+                        if (lane == 0) bulk_wait_read1();
+                        __syncwarp();
+                        if (p.y_bf16) {
+                            uint4 *rowp = reinterpret_cast<uint4 *>(buf + lane * 64);
 #pragma unroll
                             for (int k4 = 0; k4 < 4; k4++)
-                                dst[k4] = make_uint4(pack_bf16x2(v[8 * k4], v[8 * k4 + 1]),
-                                                     pack_bf16x2(v[8 * k4 + 2], v[8 * k4 + 3]),
-                                                     pack_bf16x2(v[8 * k4 + 4], v[8 * k4 + 5]),
-                                                     pack_bf16x2(v[8 * k4 + 6], v[8 * k4 + 7]));
+                                rowp[k4 ^ ((lane >> 1) & 3)] =
+                                    make_uint4(pack_bf16x2(v[8 * k4], v[8 * k4 + 1]), pack_bf16x2(v[8 * k4 + 2], v[8 * k4 + 3]),
+                                               pack_bf16x2(v[8 * k4 + 4], v[8 * k4 + 5]),
+                                               pack_bf16x2(v[8 * k4 + 6], v[8 * k4 + 7]));
                         } else {
-#pragma unroll
-                            for (int j = 0; j < 32; j++)
-                                if (nb + j < p.n) yrow[nb + j] = __float2bfloat16_rn(v[j]);
-                        }
-                    } else {
-                        float *yrow = reinterpret_cast<float *>(p.y) + (int64_t)row * p.n;
-                        if (vec && nb + 32 <= p.n) {
-                            float4 *dst = reinterpret_cast<float4 *>(yrow + nb);
+                            uint4 *rowp = reinterpret_cast<uint4 *>(buf + lane * 128);
 #pragma unroll
                             for (int k4 = 0; k4 < 8; k4++)
-                                dst[k4] = make_float4(v[4 * k4], v[4 * k4 + 1], v[4 * k4 + 2], v[4 * k4 + 3]);
-                        } else {
+                                rowp[k4 ^ (lane & 7)] = make_uint4(__float_as_uint(v[4 * k4]), __float_as_uint(v[4 * k4 + 1]),
+                                                                   __float_as_uint(v[4 * k4 + 2]), __float_as_uint(v[4 * k4 + 3]));
+                        }
+                        fence_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&p.tma_y, buf, nb, row0);
+                            bulk_commit();
+                        }
+                        sub++;
+                    } else if (row_ok && nb < p.n) {
+                        if (p.y_bf16) {
+                            __nv_bfloat16 *yrow = reinterpret_cast<__nv_bfloat16 *>(p.y) + (int64_t)row * p.n;
+                            if (vec && nb + 32 <= p.n) {
+                                uint4 *dst = reinterpret_cast<uint4 *>(yrow + nb);
 #pragma unroll
-                            for (int j = 0; j < 32; j++)
-                                if (nb + j < p.n) yrow[nb + j] = v[j];
+                                for (int k4 = 0; k4 < 4; k4++)
+                                    dst[k4] = make_uint4(pack_bf16x2(v[8 * k4], v[8 * k4 + 1]),
+                                                         pack_bf16x2(v[8 * k4 + 2], v[8 * k4 + 3]),
+                                                         pack_bf16x2(v[8 * k4 + 4], v[8 * k4 + 5]),
+                                                         pack_bf16x2(v[8 * k4 + 6], v[8 * k4 + 7]));
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < 32; j++)
+                                    if (nb + j < p.n) yrow[nb + j] = __float2bfloat16_rn(v[j]);
+                            }
+                        } else {
+                            float *yrow = reinterpret_cast<float *>(p.y) + (int64_t)row * p.n;
+                            if (vec && nb + 32 <= p.n) {
+                                float4 *dst = reinterpret_cast<float4 *>(yrow + nb);
+#pragma unroll
+                                for (int k4 = 0; k4 < 8; k4++)
+                                    dst[k4] = make_float4(v[4 * k4], v[4 * k4 + 1], v[4 * k4 + 2], v[4 * k4 + 3]);
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < 32; j++)
+                                    if (nb + j < p.n) yrow[nb + j] = v[j];
+                            }
                         }
                     }
+            };
+            uint32_t ro[OVL_CHUNKS][32];
+#pragma unroll
+            for (int i = 0; i < (int)OVL_CHUNKS; i++)
+                tmem_ld_32x32b_x32_async(lane_base + (uint32_t)((st ? i : 8 - (int)OVL_CHUNKS + i) * 32), ro[i]);
+            tmem_ld_wait(ro[OVL_CHUNKS - 1]);
+#pragma unroll
+            for (int i = 0; i + 1 < (int)OVL_CHUNKS; i++) tmem_reg_tie(ro[i]);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(ovl_leader);
+#pragma unroll
+            for (int i = 0; i < (int)OVL_CHUNKS; i++) process(st ? i : 8 - (int)OVL_CHUNKS + i, ro[i]);
+#pragma unroll 1
+            for (int i = (int)OVL_CHUNKS; i < BN / 32; i++) {
+                const int c = st ? i : i - (int)OVL_CHUNKS;
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(lane_base + (uint32_t)(c * 32), r);
+                if (i == BN / 32 - 1) {   // the whole stage is drained
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_remote(st ? acce_leader1 : acce_leader0);
                 }
+                process(c, r);
             }
         }
         if (lane == 0) bulk_wait_all();
