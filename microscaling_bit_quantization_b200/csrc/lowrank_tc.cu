@@ -59,7 +59,7 @@ struct LrTcParams {
     const float *xs, *ws;      // packed output divisor s_x * s_w; null: 1
     unsigned int *amax_word;   // null: no amax
     unsigned int *err;
-    int m, k, r, kb_total, kb_max, row_tiles, S, red_count;
+    int m, k, r, kb_total, kb_max, row_tiles, S;
     unsigned long long wait_ns;
 };
 
@@ -80,8 +80,13 @@ __device__ __forceinline__ void commit_lt(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                  : "memory");
 }
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+// Asynchronous 16-byte store into a cluster peer's shared memory that counts
+// its bytes on the peer's mbarrier (complete_tx): no fence, no separate arrival.
+__device__ __forceinline__ void st_async_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                            uint32_t bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     addr),
+                 "r"(a), "r"(b), "r"(c), "r"(d), "r"(bar)
                  : "memory");
 }
 
@@ -97,6 +102,7 @@ __device__ __forceinline__ float amax_bf16x8(uint4 a, uint4 b) {
     return m;
 }
 
+template <int S>
 __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_constant__ LrTcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -107,7 +113,7 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
     uint64_t *empty = full + LT_STAGES;
     uint64_t *accf = empty + LT_STAGES;
     uint64_t *acce = accf + 2;
-    uint64_t *redf = acce + 2;      // my reduce buffer filled (remote arrivals)
+    uint64_t *redf = acce + 2;      // my reduce buffer filled (bytes of remote st.async)
     uint64_t *redfree = redf + 2;   // every receiver has consumed buffer (remote arrivals)
     uint64_t *sumdone = redfree + 2;   // the four reducing warps are done with my buffer
     uint64_t *drain = sumdone + 2;
@@ -115,7 +121,8 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int S = p.S, R = 128 / S;
+    constexpr int R = 128 / S;
+    constexpr uint32_t kRedBytes = S * R * 32 * 4;   // bytes each CTA receives per row tile
     const uint32_t rank = cluster_rank();
     const int cid = (int)cluster_id(), ncl = (int)cluster_count();
     const int kb0 = (int)(rank * (uint32_t)p.kb_total / (uint32_t)S);
@@ -132,13 +139,19 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
         for (int i = 0; i < 2; i++) {
             mbar_init(accf + i, 1);
             mbar_init(acce + i, 4);
-            mbar_init(redf + i, (uint32_t)p.red_count);
+            // S > 1: its own expect_tx, completed by the senders' st.async bytes;
+            // S == 1: one arrival per warp after plain local stores
+            mbar_init(redf + i, S > 1 ? 1 : 4);
             mbar_init(redfree + i, (uint32_t)S);
             mbar_init(sumdone + i, 4);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        if (S > 1) {   // the bytes of the first two row tiles are expected before any sender may start
+            mbar_arrive_expect_tx(redf + 0, kRedBytes);
+            mbar_arrive_expect_tx(redf + 1, kRedBytes);
+        }
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -162,27 +175,27 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
     // B tile j, row n, 16-byte unit c holds L1[(kb0 + j) 64 + 8 c + t][n], t = 0..7 (128B swizzle)
     if (p.r % 8 == 0 && (reinterpret_cast<uintptr_t>(p.l1) & 15u) == 0) {
         // 8 x 8 blocks: eight independent 16-byte row loads, a transpose by byte permutes, eight stores
-        for (int idx = threadIdx.x; idx < nkb * 32; idx += LT_THREADS) {
+        auto load_block = [&](int idx, uint4 (&rv)[8]) {
             const int j = idx >> 5, c = (idx >> 2) & 7, n0 = 8 * (idx & 3);
             const int kk0 = (kb0 + j) * 64 + 8 * c;
-            uint4 rv[8];
 #pragma unroll
             for (int t = 0; t < 8; t++)
-                rv[t] = (n0 < p.r && kk0 + t < p.k)
+                rv[t] = (idx < nkb * 32 && n0 < p.r && kk0 + t < p.k)
                             ? __ldg(reinterpret_cast<const uint4 *>(p.l1 + (int64_t)(kk0 + t) * p.r + n0))
                             : make_uint4(0u, 0u, 0u, 0u);
-            uint32_t w[8][4];
-#pragma unroll
-            for (int t = 0; t < 8; t++) {
-                w[t][0] = rv[t].x; w[t][1] = rv[t].y; w[t][2] = rv[t].z; w[t][3] = rv[t].w;
-            }
+        };
+        auto store_block = [&](int idx, const uint4 (&rv)[8]) {
+            if (idx >= nkb * 32) return;
+            const int j = idx >> 5, c = (idx >> 2) & 7, n0 = 8 * (idx & 3);
 #pragma unroll
             for (int i = 0; i < 4; i++) {   // columns n0 + 2i (low halves) and n0 + 2i + 1 (high halves)
                 uint32_t lo[4], hi[4];
 #pragma unroll
                 for (int jj = 0; jj < 4; jj++) {
-                    lo[jj] = __byte_perm(w[2 * jj][i], w[2 * jj + 1][i], 0x5410);
-                    hi[jj] = __byte_perm(w[2 * jj][i], w[2 * jj + 1][i], 0x7632);
+                    const uint32_t *wa = reinterpret_cast<const uint32_t *>(&rv[2 * jj]);
+                    const uint32_t *wb = reinterpret_cast<const uint32_t *>(&rv[2 * jj + 1]);
+                    lo[jj] = __byte_perm(wa[i], wb[i], 0x5410);
+                    hi[jj] = __byte_perm(wa[i], wb[i], 0x7632);
                 }
                 const int na = n0 + 2 * i, nb = na + 1;
                 *reinterpret_cast<uint4 *>(btile + j * LT_B + na * 128 + ((c ^ (na & 7)) << 4)) =
@@ -190,6 +203,14 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
                 *reinterpret_cast<uint4 *>(btile + j * LT_B + nb * 128 + ((c ^ (nb & 7)) << 4)) =
                     make_uint4(hi[0], hi[1], hi[2], hi[3]);
             }
+        };
+        // two blocks per thread per round, all sixteen loads in flight before any transpose
+        for (int idx = threadIdx.x; idx < nkb * 32; idx += 2 * LT_THREADS) {
+            uint4 ra[8], rb[8];
+            load_block(idx, ra);
+            load_block(idx + LT_THREADS, rb);
+            store_block(idx, ra);
+            store_block(idx + LT_THREADS, rb);
         }
     } else {
         for (int idx = threadIdx.x; idx < nkb * 256; idx += LT_THREADS) {
@@ -307,13 +328,19 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
                 break;
             }
             const int row_t = q * 32 + lane, dst = row_t / R, lr = row_t % R;
-            const uint32_t raddr = map_to_rank(red + pb * (128 * 32) + ((int)rank * R + lr) * 32, (uint32_t)dst);
+            float *mine = red + pb * (128 * 32) + ((int)rank * R + lr) * 32;
+            if (S > 1) {
+                const uint32_t raddr = map_to_rank(mine, (uint32_t)dst), rbar = map_to_rank(redf + pb, (uint32_t)dst);
 #pragma unroll
-            for (int i = 0; i < 8; i++) st_cluster_v4(raddr + 16 * i, v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-            asm volatile("fence.acq_rel.cluster;" ::: "memory");
-            __syncwarp();
-            if (lane == 0)
-                for (int d = (q * 32) / R; d <= (q * 32 + 31) / R; d++) mbar_arrive_remote(map_to_rank(redf + pb, (uint32_t)d));
+                for (int i = 0; i < 8; i++)
+                    st_async_v4(raddr + 16 * i, v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3], rbar);
+            } else {   // the whole tile stays in this CTA
+#pragma unroll
+                for (int i = 0; i < 8; i++)
+                    reinterpret_cast<uint4 *>(mine)[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive_local(redf + pb);
+            }
 
             // receive rows [rank R, rank R + R) from every CTA, add in rank order, write
             w = mbar_wait<true>(redf + pb, (tc >> 1) & 1, p.wait_ns);
@@ -322,10 +349,15 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
                 break;
             }
             const float *buf = red + pb * (128 * 32);
+#pragma unroll
             for (int pos = te; pos < R * 32; pos += 128) {
                 const int row = pos >> 5, col = pos & 31;
+                float part[S];
+#pragma unroll
+                for (int jj = 0; jj < S; jj++) part[jj] = buf[(jj * R + row) * 32 + col];
                 float sum = 0.0f;
-                for (int jj = 0; jj < S; jj++) sum = __fadd_rn(sum, buf[(jj * R + row) * 32 + col]);
+#pragma unroll
+                for (int jj = 0; jj < S; jj++) sum = __fadd_rn(sum, part[jj]);
                 const int64_t grow = (int64_t)rt * 128 + (int)rank * R + row;
                 if (grow < p.m) {
                     if (p.t) {
@@ -344,6 +376,7 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
             if (lane == 0) mbar_arrive_local(sumdone + pb);
             if (te == 0) {
                 if (mbar_wait(sumdone + pb, (tc >> 1) & 1, p.wait_ns)) {
+                    if (S > 1) mbar_arrive_expect_tx(redf + pb, kRedBytes);   // the bytes of row tile tc + 2
                     for (int d = 0; d < S; d++) mbar_arrive_remote(map_to_rank(redfree + pb, (uint32_t)d));
                 } else {
                     ok = false;
@@ -385,8 +418,10 @@ cudaError_t launch_lowrank_tc(const void *x, int64_t m, int64_t k, const void *l
     p.kb_total = (int)((k + 63) / 64);
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(k_lowrank_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, LT_SMEM_MAX);
-        if (e != cudaSuccess) return e;
+        for (auto fn : {k_lowrank_tc<1>, k_lowrank_tc<2>, k_lowrank_tc<4>, k_lowrank_tc<8>}) {
+            cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, LT_SMEM_MAX);
+            if (e != cudaSuccess) return e;
+        }
         configured = true;
     }
     // cluster size: fewest rounds x k-blocks per CTA, then the smaller cluster; the
@@ -412,7 +447,11 @@ cudaError_t launch_lowrank_tc(const void *x, int64_t m, int64_t k, const void *l
             q.attrs = &a;
             q.numAttrs = 1;
             int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, k_lowrank_tc, &q) != cudaSuccess) {
+            const cudaError_t oe = S == 1 ? cudaOccupancyMaxActiveClusters(&n, k_lowrank_tc<1>, &q)
+                                 : S == 2 ? cudaOccupancyMaxActiveClusters(&n, k_lowrank_tc<2>, &q)
+                                 : S == 4 ? cudaOccupancyMaxActiveClusters(&n, k_lowrank_tc<4>, &q)
+                                          : cudaOccupancyMaxActiveClusters(&n, k_lowrank_tc<8>, &q);
+            if (oe != cudaSuccess) {
                 cudaGetLastError();
                 n = 0;
             }
@@ -430,7 +469,6 @@ cudaError_t launch_lowrank_tc(const void *x, int64_t m, int64_t k, const void *l
     if (!best_s) return cudaErrorNotSupported;
     p.S = best_s;
     p.kb_max = (p.kb_total + best_s - 1) / best_s;
-    p.red_count = best_s * (128 / best_s >= 32 ? (128 / best_s) / 32 : 1);
     p.l1 = (const __nv_bfloat16 *)l1;
     p.t = t;
     p.tp = (__nv_bfloat16 *)tp;
@@ -457,7 +495,12 @@ cudaError_t launch_lowrank_tc(const void *x, int64_t m, int64_t k, const void *l
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_lowrank_tc, p);
+    switch (best_s) {
+    case 1: return cudaLaunchKernelEx(&cfg, k_lowrank_tc<1>, p);
+    case 2: return cudaLaunchKernelEx(&cfg, k_lowrank_tc<2>, p);
+    case 4: return cudaLaunchKernelEx(&cfg, k_lowrank_tc<4>, p);
+    default: return cudaLaunchKernelEx(&cfg, k_lowrank_tc<8>, p);
+    }
 }
 
 }  // namespace mxq
