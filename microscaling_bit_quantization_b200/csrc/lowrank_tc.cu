@@ -163,15 +163,19 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // the first tiles of X are in flight while the B tiles are built
+    // The first tiles of X are in flight while the B tiles are built; the L1
+    // loads of the first round are issued before them, so they are not queued
+    // behind the prefetch of X.
     const int pre = total < LT_STAGES ? total : LT_STAGES;
-    if (warp == 0 && lane == 0) {
-        for (int u = 0; u < pre; u++) {
-            const int rt = cid + (u / nkb) * ncl, kb = kb0 + u % nkb;
-            mbar_arrive_expect_tx(full + u, LT_X);
-            tma_load_x(&p.tma_x, xst + u * LT_X, full + u, kb * 64, rt * 128);
+    auto prefetch_x = [&]() {
+        if (warp == 0 && lane == 0) {
+            for (int u = 0; u < pre; u++) {
+                const int rt = cid + (u / nkb) * ncl, kb = kb0 + u % nkb;
+                mbar_arrive_expect_tx(full + u, LT_X);
+                tma_load_x(&p.tma_x, xst + u * LT_X, full + u, kb * 64, rt * 128);
+            }
         }
-    }
+    };
     // B tile j, row n, 16-byte unit c holds L1[(kb0 + j) 64 + 8 c + t][n], t = 0..7 (128B swizzle)
     if (p.r % 8 == 0 && (reinterpret_cast<uintptr_t>(p.l1) & 15u) == 0) {
         // 8 x 8 blocks: eight independent 16-byte row loads, a transpose by byte permutes, eight stores
@@ -209,10 +213,13 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
             uint4 ra[8], rb[8];
             load_block(idx, ra);
             load_block(idx + LT_THREADS, rb);
+            if (idx == (int)threadIdx.x) prefetch_x();
             store_block(idx, ra);
             store_block(idx + LT_THREADS, rb);
         }
+        if (nkb * 32 <= (int)threadIdx.x) prefetch_x();   // a thread without blocks
     } else {
+        prefetch_x();
         for (int idx = threadIdx.x; idx < nkb * 256; idx += LT_THREADS) {
             const int j = idx >> 8, n = (idx >> 3) & 31, c = idx & 7;
             const int kk0 = (kb0 + j) * 64 + 8 * c;
@@ -372,6 +379,8 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
                 }
             }
             // buffer pb is free again once all four warps are done with it: tell every sender
+            // (not after this cluster's last row tile: nothing is sent into it again)
+            if (tc + 1 == ntiles) continue;
             __syncwarp();
             if (lane == 0) mbar_arrive_local(sumdone + pb);
             if (te == 0) {
