@@ -220,15 +220,26 @@ __device__ __forceinline__ Recip recip_of(float d) {
     return r;
 }
 
+// Products of eight values with one factor, as four packed two-wide multiplies
+// (each lane of a pair rounded exactly like __fmul_rn).
+__device__ __forceinline__ void mul8(const float *v, float f, float *o) {
+    const float2 ff = make_float2(f, f);
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const float2 p = __fmul2_rn(make_float2(v[2 * i], v[2 * i + 1]), ff);
+        o[2 * i] = p.x;
+        o[2 * i + 1] = p.y;
+    }
+}
+
 // E2M1 codes of RN(v[i] / d) for eight values, packed like cvt_e2m1x8.
 __device__ __forceinline__ uint32_t e2m1x8_quot(const float *v, const Recip &r) {
     if (r.fast) {
-        const uint32_t lo = cvt_e2m1x8(__fmul_rn(v[0], r.lo), __fmul_rn(v[1], r.lo), __fmul_rn(v[2], r.lo),
-                                       __fmul_rn(v[3], r.lo), __fmul_rn(v[4], r.lo), __fmul_rn(v[5], r.lo),
-                                       __fmul_rn(v[6], r.lo), __fmul_rn(v[7], r.lo));
-        const uint32_t hi = cvt_e2m1x8(__fmul_rn(v[0], r.hi), __fmul_rn(v[1], r.hi), __fmul_rn(v[2], r.hi),
-                                       __fmul_rn(v[3], r.hi), __fmul_rn(v[4], r.hi), __fmul_rn(v[5], r.hi),
-                                       __fmul_rn(v[6], r.hi), __fmul_rn(v[7], r.hi));
+        float l[8], h[8];
+        mul8(v, r.lo, l);
+        mul8(v, r.hi, h);
+        const uint32_t lo = cvt_e2m1x8(l[0], l[1], l[2], l[3], l[4], l[5], l[6], l[7]);
+        const uint32_t hi = cvt_e2m1x8(h[0], h[1], h[2], h[3], h[4], h[5], h[6], h[7]);
         if (lo == hi) return lo;
     }
     return cvt_e2m1x8(__fdiv_rn(v[0], r.d), __fdiv_rn(v[1], r.d), __fdiv_rn(v[2], r.d), __fdiv_rn(v[3], r.d),

@@ -182,8 +182,8 @@ __global__ void __launch_bounds__(kQThreads, 2) k_quantize(const T *__restrict__
             if (valid) {
                 // inv is a power of two: v * inv is exact (or far below the smallest code)
                 float u[16];
-#pragma unroll
-                for (int i = 0; i < 16; i++) u[i] = __fmul_rn(v[i], inv);
+                mul8(v, inv, u);
+                mul8(v + 8, inv, u + 8);
                 const bool zero = !(amax > 0.0f);   // all-zero block: +0 codes
                 if (F == kMXFP8) {
                     uint4 w;
