@@ -98,6 +98,10 @@ typedef struct mxq_qtensor {
 /* Human-readable name of a status code (static string). */
 const char *mxq_status_string(mxq_status st);
 
+/* Text of the CUDA error behind the last MXQ_ECUDA that a call made from
+ * this host thread returned ("no error" if none yet); static string. */
+const char *mxq_last_cuda_error_string(void);
+
 /* 1 if device `device` is an sm_100-family GPU the kernels were built for. */
 int mxq_device_supported(int device);
 

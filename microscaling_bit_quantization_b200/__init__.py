@@ -29,7 +29,7 @@ F32, BF16 = 0, 1
 STATUS = {0: "MXQ_OK", 1: "MXQ_EINVAL", 2: "MXQ_EUNSUPPORTED", 3: "MXQ_ECUDA", 4: "MXQ_ETIMEOUT", 5: "MXQ_ENOSPACE"}
 
 # Every entry point the header declares.
-EXPORTS = ("mxq_status_string", "mxq_device_supported", "mxq_check", "mxq_codes_bytes", "mxq_scales_bytes",
+EXPORTS = ("mxq_status_string", "mxq_last_cuda_error_string", "mxq_device_supported", "mxq_check", "mxq_codes_bytes", "mxq_scales_bytes",
            "mxq_quantize_workspace_bytes", "mxq_quantize", "mxq_dequantize", "mxq_hadamard_block", "mxq_cast",
            "mxq_select_workspace_bytes", "mxq_select_weight_format", "mxq_lowrank_down", "mxq_lowrank_packed_bytes",
            "mxq_lowrank_down_packed", "mxq_lowrank_pack_t", "mxq_lowrank_pack_l2", "mxq_qlinear", "mxq_route",
@@ -38,7 +38,10 @@ EXPORTS = ("mxq_status_string", "mxq_device_supported", "mxq_check", "mxq_codes_
 
 class MxqError(RuntimeError):
     def __init__(self, status: int, what: str):
-        super().__init__("%s failed: %s (%s)" % (what, STATUS.get(status, status), _lib.mxq_status_string(status).decode()))
+        detail = _lib.mxq_status_string(status).decode()
+        if status == 3:   # MXQ_ECUDA: name the CUDA error
+            detail += ": " + _lib.mxq_last_cuda_error_string().decode()
+        super().__init__("%s failed: %s (%s)" % (what, STATUS.get(status, status), detail))
         self.status = status
 
 
@@ -56,6 +59,7 @@ def _load():
     psz = ctypes.POINTER(ctypes.c_size_t)
     sig = {
         "mxq_status_string": (ctypes.c_char_p, [i32]),
+        "mxq_last_cuda_error_string": (ctypes.c_char_p, []),
         "mxq_device_supported": (ctypes.c_int, [ctypes.c_int]),
         "mxq_check": (i32, [P]),
         "mxq_codes_bytes": (i32, [i32, i64, i64, i32, psz]),

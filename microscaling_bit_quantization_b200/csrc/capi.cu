@@ -34,13 +34,21 @@ bool valid_shape(int32_t fmt, int64_t rows, int64_t cols) {
     return true;
 }
 
-mxq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MXQ_OK : MXQ_ECUDA; }
+// The last CUDA error a call of this host thread returned as MXQ_ECUDA.
+thread_local cudaError_t g_last_cuda = cudaSuccess;
+mxq_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return MXQ_OK;
+    g_last_cuda = e;
+    return MXQ_ECUDA;
+}
 
 int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 
 }  // namespace
 
 extern "C" {
+
+const char *mxq_last_cuda_error_string(void) { return cudaGetErrorString(g_last_cuda); }
 
 const char *mxq_status_string(mxq_status st) {
     switch (st) {
@@ -62,9 +70,10 @@ int mxq_device_supported(int device) {
 
 mxq_status mxq_check(void *stream) {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
-    if (e != cudaSuccess) return MXQ_ECUDA;
+    if (e != cudaSuccess) return from_cuda(e);
     unsigned int w = 0;
-    if (read_and_clear_error(&w) != cudaSuccess) return MXQ_ECUDA;
+    e = read_and_clear_error(&w);
+    if (e != cudaSuccess) return from_cuda(e);
     return w ? MXQ_ETIMEOUT : MXQ_OK;
 }
 
@@ -236,7 +245,7 @@ mxq_status mxq_quantize_lowrank(const void *x, int32_t xdtype, int64_t m, int64_
     } else {
         e = launch_lowrank_down(x, bf, m, k, l1, r, t, nullptr, nullptr, nullptr, s);
     }
-    if (e != cudaSuccess) return MXQ_ECUDA;
+    if (e != cudaSuccess) return from_cuda(e);
     PackT pack{t, r, w_tensor_scale, tp};
     return from_cuda(launch_quantize(x, bf, m, k, fmt, hadamard_b, MXQ_LAYOUT_MMA, codes, scales, sb, tensor_scale,
                                      amax, s, &pack, amax_ready));
@@ -305,12 +314,15 @@ std::mutex g_noalloc_lock;
 
 mxq_status noalloc_scratch(void **ptr) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return MXQ_ECUDA;
+    const cudaError_t de = cudaGetDevice(&dev);
+    if (de != cudaSuccess) return from_cuda(de);
     if (dev < 0 || dev >= kNoAllocMaxDevices) return MXQ_EUNSUPPORTED;
     std::lock_guard<std::mutex> guard(g_noalloc_lock);
     if (!g_noalloc_addr[dev]) {
         void *a = nullptr;
-        if (cudaGetSymbolAddress(&a, g_noalloc_scratch) != cudaSuccess || !a) return MXQ_ECUDA;
+        const cudaError_t se = cudaGetSymbolAddress(&a, g_noalloc_scratch);
+        if (se != cudaSuccess) return from_cuda(se);
+        if (!a) return MXQ_ECUDA;
         g_noalloc_addr[dev] = a;
     }
     *ptr = g_noalloc_addr[dev];

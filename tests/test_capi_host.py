@@ -107,3 +107,11 @@ def test_route_matches_oracle(mxq, orc):
         for layer in range(n_layers):
             for step in range(-1, n_steps + 1):
                 assert mxq.route(table, layer, step, n_steps) == orc.route(table, n_layers, n_int, layer, step, n_steps)
+
+
+def test_last_cuda_error_string(mxq):
+    """Before any CUDA failure the thread's last error reads as no error; the
+    Python error for MXQ_ECUDA names the CUDA error through it."""
+    s = mxq.lib().mxq_last_cuda_error_string()
+    assert isinstance(s, bytes) and len(s) > 0
+    assert b"no error" in s.lower()
