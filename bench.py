@@ -341,6 +341,20 @@ def run_ours(args, world, rank, local):
         formats[name] = {"us": 1e3 * t_ms, "GB/s": nbytes / (t_ms * 1e-3) / 1e9,
                          "frac": nbytes / (t_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
         del outs
+    # per-channel format selection (workload 2 weights) and the low-rank down projection alone
+    wsel = torch.from_numpy(workloads.chameleon_selection(m=1)["w"]).to(torch.bfloat16).to(dev)
+    sel_ms = graph_ms(lambda i: mxq.select_weight_format(wsel, (mxq.INT4_G32, mxq.NVFP4, mxq.MXFP4), want_sse=False),
+                      n=8, reps=5)
+    sel_bytes = wsel.numel() * 2 + wsel.shape[0]
+    select = {"kernel": "k_select over INT4-g32, NVFP4, MXFP4 (+ tensor amax pass), W 3072 x 3072 bf16",
+              "us": 1e3 * sel_ms, "GB/s": sel_bytes / (sel_ms * 1e-3) / 1e9,
+              "frac": sel_bytes / (sel_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    del wsel
+    t_buf = torch.empty((M, RANK), dtype=torch.float32, device=dev)
+    lr_ms = graph_ms(lambda i: mxq.lowrank_down(sets[i % N_SETS]["x"], l1, out=t_buf))
+    lowrank = {"kernel": "k_lowrank_tc (T = bf16(X) L1 alone), X 4096 x 3072 bf16, rank 32", "us": 1e3 * lr_ms,
+               "GB/s": M * K * 2 / (lr_ms * 1e-3) / 1e9, "frac": M * K * 2 / (lr_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    del t_buf
     w4 = workloads.svdquant_mlp_up()["w"]
     wq4 = mxq.quantize(torch.from_numpy(w4).to(torch.bfloat16).to(dev), mxq.INT4_G64, 0, mxq.MMA)
     del w4
@@ -408,6 +422,8 @@ def run_ours(args, world, rank, local):
                                  "bytes": "read 2 B/element + canonical codes and scales", "peak_GB/s": peaks["hbm_gbs"],
                                  "rows": formats},
             "int4_g64_qlinear": int4,
+            "select_weight_format": select,
+            "lowrank_down": lowrank,
             "e2e": {"value": world * FLOP_STEP / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "ms_per_step": e2e_ms},
             "gpu_launches": launches_per_step * args.steps,
