@@ -83,6 +83,8 @@ def lib():
         L.orc_dequantize.argtypes = [P, P, P, i64, i64, i32, P]
         L.orc_select.restype = i32
         L.orc_select.argtypes = [P, i64, i64, P, i32, P, P, P, P, P]
+        L.orc_quantize_mse_nvfp4.restype = i32
+        L.orc_quantize_mse_nvfp4.argtypes = [P, i64, i64, i32, P, P, P, P]
         L.orc_lowrank_down.restype = i32
         L.orc_lowrank_down.argtypes = [P, P, i64, i64, i32, P]
         L.orc_route.restype = i32
@@ -233,6 +235,23 @@ def select_weight_format(w, candidates):
     if st != 0:
         raise OracleError("bad select arguments")
     return choice, sse
+
+
+# ---------------------------------------------------------------- MSE-fitted NVFP4 scales
+
+def quantize_mse_nvfp4(x, iters: int):
+    """NVFP4 with block and tensor scales fitted to the squared error
+    (mxq_oracle.c, orc_quantize_mse_nvfp4).  Returns (QTensor, total error)."""
+    x = _f32(x)
+    rows, cols = x.shape
+    codes = np.zeros(codes_shape(NVFP4, rows, cols), dtype=np.uint8)
+    scales = np.zeros((rows, cols // 16), dtype=np.uint8)
+    ts = np.zeros(1, dtype=np.float32)
+    sse = np.zeros(1, dtype=np.float64)
+    st = lib().orc_quantize_mse_nvfp4(_ptr(x), rows, cols, iters, _ptr(codes), _ptr(scales), _ptr(ts), _ptr(sse))
+    if st != 0:
+        raise OracleError("bad quantize_mse_nvfp4 arguments")
+    return QTensor(NVFP4, rows, cols, codes, scales, float(ts[0])), float(sse[0])
 
 
 # ---------------------------------------------------------------- low rank + GEMM

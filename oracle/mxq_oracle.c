@@ -501,6 +501,122 @@ int orc_select(const float *w, int64_t n, int64_t k, const int *cands, int ncand
 }
 
 /* ------------------------------------------------------------------ */
+/* NVFP4 scales fitted to the squared error ("Bridging the Gap Between */
+/* Promise and Performance for Microscaling FP4 Quantization", MR-GPTQ */
+/* modification 1: the quantization grid is chosen for the MSE by      */
+/* optimizing the per-block scales and the tensor scale in turn; the   */
+/* page reports the gain for NVFP4 without rotations).  The page gives */
+/* no candidate set, round count or summation order; the readings:     */
+/*  - Block step (tensor scale s_t fixed).  e0 = the usual block code   */
+/*    (quant_nvfp4_block).  Candidates, scored in this order: e0, then  */
+/*    e0 + 1, e0 - 1, e0 - 2, ..., e0 - 6, keeping codes in [1, 126]    */
+/*    (for e0 = 0: 0 then 1).  A candidate e codes the block as usual   */
+/*    under it: d = RN(value(e) s_t), q_i = E2M1(RN(v_i / d)) (e = 0:   */
+/*    all +0).  Its error is sum_i (v_i - value(q_i) value(e) s_t)^2    */
+/*    with the dequantized value exact in binary64 and the sum taken    */
+/*    in binary64 in element order.  The first least error wins.        */
+/*  - Tensor step (block codes fixed).  Least squares for the common    */
+/*    factor: s_t = RN32(RN64(A / B)), A = sum v_i u_i, B = sum u_i^2,  */
+/*    u_i = value(q_i) value(e); binary64 sums within a block in        */
+/*    element order, within a row in block order, over rows in row      */
+/*    order.  B = 0 keeps s_t.                                          */
+/*  - Start from the usual tensor scale; `iters` rounds of (block step, */
+/*    tensor step); a final block step gives codes and scales.  The     */
+/*    total error of the result (same summation order) goes to *sse.    */
+/* Output layout as orc_quantize's canonical NVFP4.                     */
+/* ------------------------------------------------------------------ */
+
+/* error of block v under block code e (codes into q[16] when q != NULL) */
+static double mse_block_error(const float *v, float s_t, uint8_t e, uint8_t *q)
+{
+    double err = 0.0;
+    float d = e ? (float)orc_e4m3_value(e) * s_t : 0.0f;
+    for (int i = 0; i < 16; i++) {
+        uint8_t c = e ? orc_to_e2m1(v[i] / d) : 0;
+        if (q) q[i] = c;
+        double w_hat = orc_e2m1_value(c) * orc_e4m3_value(e) * (double)s_t;
+        double diff = (double)v[i] - w_hat;
+        err += diff * diff;
+    }
+    return err;
+}
+
+/* block step for one block: chosen code, its element codes and error */
+static uint8_t mse_block_choose(const float *v, float s_t, uint8_t *q, double *err_out)
+{
+    float raw = (amax_of(v, 16) / 6.0f) / s_t;
+    int e0 = orc_to_e4m3(raw);
+    int order[8];
+    int n = 0;
+    order[n++] = e0;
+    if (e0 == 0) {
+        order[n++] = 1;
+    } else {
+        if (e0 + 1 <= 126) order[n++] = e0 + 1;
+        for (int j = 1; j <= 6; j++)
+            if (e0 - j >= 1) order[n++] = e0 - j;
+    }
+    int best = order[0];
+    double best_err = mse_block_error(v, s_t, (uint8_t)best, NULL);
+    for (int i = 1; i < n; i++) {
+        double err = mse_block_error(v, s_t, (uint8_t)order[i], NULL);
+        if (err < best_err) {
+            best_err = err;
+            best = order[i];
+        }
+    }
+    mse_block_error(v, s_t, (uint8_t)best, q);
+    *err_out = best_err;
+    return (uint8_t)best;
+}
+
+int orc_quantize_mse_nvfp4(const float *x, int64_t rows, int64_t cols, int iters, uint8_t *codes,
+                           uint8_t *scales, float *tensor_scale, double *sse)
+{
+    if (rows < 0 || cols < 0 || cols % 16 || iters < 0) return ORC_EINVAL;
+    float amax_t = amax_of(x, rows * cols);
+    float s_t = nvfp4_tensor_scale(amax_t);
+    int64_t nb = cols / 16;
+    uint8_t q[16];
+    double err;
+    for (int it = 0; it < iters; it++) {
+        double a_sum = 0.0, b_sum = 0.0;
+        for (int64_t r = 0; r < rows; r++) {
+            double a_row = 0.0, b_row = 0.0;
+            for (int64_t b = 0; b < nb; b++) {
+                const float *v = x + r * cols + b * 16;
+                uint8_t e = mse_block_choose(v, s_t, q, &err);
+                double a_blk = 0.0, b_blk = 0.0;
+                for (int i = 0; i < 16; i++) {
+                    double u = orc_e2m1_value(q[i]) * orc_e4m3_value(e);
+                    a_blk += (double)v[i] * u;
+                    b_blk += u * u;
+                }
+                a_row += a_blk;
+                b_row += b_blk;
+            }
+            a_sum += a_row;
+            b_sum += b_row;
+        }
+        if (b_sum > 0.0) s_t = (float)(a_sum / b_sum);
+    }
+    *tensor_scale = s_t;
+    double total = 0.0;
+    for (int64_t r = 0; r < rows; r++) {
+        double row_err = 0.0;
+        for (int64_t b = 0; b < nb; b++) {
+            uint8_t e = mse_block_choose(x + r * cols + b * 16, s_t, q, &err);
+            scales[r * nb + b] = e;
+            for (int i = 0; i < 16; i++) put_code(codes, r * cols + b * 16 + i, 1, q[i]);
+            row_err += err;
+        }
+        total += row_err;
+    }
+    if (sse) *sse = total;
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
 /* SVDQuant low-rank branch, down projection (Nunchaku/Diffusers       */
 /* article, section "Main explanation": a 16-bit low-rank part of the  */
 /* weight is kept beside the 4-bit residual).                          */

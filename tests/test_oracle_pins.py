@@ -442,6 +442,149 @@ def test_fp_grid_wins_on_heavy_tails(orc):
     assert (c_heavy == orc.MXFP4).mean() > (c_flat == orc.MXFP4).mean()
 
 
+# ------------------------------------------------------------------ MSE-fitted NVFP4 scales
+
+_E2M1_GRID = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def _e2m1_nearest(t: float) -> float:
+    """E2M1 value nearest to t (ties to the even grid index), saturating at 6;
+    written here from the grid, independently of the oracle's rounding."""
+    a = abs(t)
+    best = 0
+    for i, g in enumerate(_E2M1_GRID):
+        da, db = abs(a - g), abs(a - _E2M1_GRID[best])
+        if da < db or (da == db and i % 2 == 0 and best % 2 == 1):
+            best = i
+    return math.copysign(_E2M1_GRID[best], t)
+
+
+def _block_values_under(orc, v, e, s_t):
+    """Decoded element values of block v coded under block code e: the
+    quotient RN32(v / RN32(value(e) s_t)) by torch's IEEE fp32 division."""
+    if e == 0:
+        return [0.0] * len(v)
+    d = torch.tensor(orc.e4m3_value(e), dtype=torch.float32) * torch.tensor(s_t, dtype=torch.float32)
+    t = torch.tensor(v, dtype=torch.float32) / d
+    return [_e2m1_nearest(float(z)) for z in t]
+
+
+def _exact_block_error(v, vals, e_value, s_t):
+    from fractions import Fraction
+    s = Fraction(s_t) * Fraction(e_value)
+    return sum((Fraction(float(a)) - Fraction(b) * s) ** 2 for a, b in zip(v, vals))
+
+
+def _window(e0):
+    if e0 == 0:
+        return [0, 1]
+    return [e0] + ([e0 + 1] if e0 + 1 <= 126 else []) + [e0 - j for j in range(1, 7) if e0 - j >= 1]
+
+
+def test_mse_nvfp4_block_choice_brute_force(orc):
+    # every block's chosen code has the least exact (rational) error over its
+    # candidate window, the first one in scoring order on exact ties, and its
+    # element codes are those the scale gives
+    rng = np.random.default_rng(31)
+    x = (rng.standard_t(3, size=(6, 64)) * 0.02).astype(np.float32)
+    q_usual = orc.quantize(x, orc.NVFP4)
+    q, _ = orc.quantize_mse_nvfp4(x, 0)
+    assert q.tensor_scale == q_usual.tensor_scale
+    s_t = q.tensor_scale
+    deq = q.dequantize()
+    for r in range(x.shape[0]):
+        for b in range(x.shape[1] // 16):
+            v = [float(z) for z in x[r, 16 * b:16 * b + 16]]
+            e0 = int(q_usual.scales[r, b])
+            errs = []
+            for e in _window(e0):
+                vals = _block_values_under(orc, v, e, s_t)
+                errs.append((_exact_block_error(v, vals, orc.e4m3_value(e) if e else 0.0, s_t), e, vals))
+            best = min(t[0] for t in errs)
+            first = next(t for t in errs if t[0] == best)
+            chosen = int(q.scales[r, b])
+            err_chosen = next(t[0] for t in errs if t[1] == chosen)
+            # binary64 scoring may only differ from exact rationals at rounding level
+            assert float(err_chosen) <= float(best) * (1 + 1e-12)
+            if chosen != first[1]:
+                assert float(err_chosen - best) <= float(best) * 1e-12
+            vals = next(t[2] for t in errs if t[1] == chosen)
+            e_val = orc.e4m3_value(chosen) if chosen else 0.0
+            assert list(deq[r, 16 * b:16 * b + 16]) == [a * e_val * s_t for a in vals]
+
+
+def test_mse_nvfp4_never_worse_per_block(orc):
+    rng = np.random.default_rng(32)
+    x = (rng.standard_t(2.5, size=(16, 128)) * 0.05).astype(np.float32)
+    xd = x.astype(np.float64)
+    e_usual = ((orc.quantize(x, orc.NVFP4).dequantize() - xd) ** 2).reshape(16, 8, 16).sum(-1)
+    q, sse = orc.quantize_mse_nvfp4(x, 0)
+    e_mse = ((q.dequantize() - xd) ** 2).reshape(16, 8, 16).sum(-1)
+    assert np.all(e_mse <= e_usual * (1 + 1e-12))
+    assert e_mse.sum() < e_usual.sum()
+    assert sse == pytest.approx(e_mse.sum(), rel=1e-12)
+
+
+def test_mse_nvfp4_tensor_step_is_least_squares(orc):
+    # one round = block step under the usual s_t (exactly the iters=0 result),
+    # then s_t = RN32 of the least-squares factor sum(v u) / sum(u^2) for those
+    # codes; recomputed here in exact rationals
+    from fractions import Fraction
+    rng = np.random.default_rng(33)
+    x = (rng.standard_t(3, size=(8, 96)) * 0.03).astype(np.float32)
+    q0, _ = orc.quantize_mse_nvfp4(x, 0)
+    codes = _unpack4(q0.codes)
+    num = den = Fraction(0)
+    for r in range(x.shape[0]):
+        for c in range(x.shape[1]):
+            u = Fraction(orc.e2m1_value(int(codes[r, c]))) * Fraction(orc.e4m3_value(int(q0.scales[r, c // 16])))
+            num += Fraction(float(x[r, c])) * u
+            den += u * u
+    exact = float(np.float32(num / den))   # RN to fp32 via the nearest binary64 first
+    q1, _ = orc.quantize_mse_nvfp4(x, 1)
+    assert abs(q1.tensor_scale - exact) <= np.spacing(np.float32(exact))
+    assert q1.tensor_scale != q0.tensor_scale
+
+
+def test_mse_nvfp4_power_of_two_equivariance(orc):
+    rng = np.random.default_rng(34)
+    x = (rng.standard_t(3, size=(8, 64)) * 0.02).astype(np.float32)
+    for iters in (0, 2):
+        q, sse = orc.quantize_mse_nvfp4(x, iters)
+        for j in (6, -5):
+            xs = (x * np.float32(2.0 ** j)).astype(np.float32)
+            qs, sses = orc.quantize_mse_nvfp4(xs, iters)
+            assert np.array_equal(qs.codes, q.codes) and np.array_equal(qs.scales, q.scales)
+            assert qs.tensor_scale == q.tensor_scale * 2.0 ** j
+            assert sses == sse * 4.0 ** j
+
+
+def test_mse_nvfp4_degenerate_cases(orc):
+    z = np.zeros((3, 32), np.float32)
+    q, sse = orc.quantize_mse_nvfp4(z, 2)
+    assert q.tensor_scale == 1.0 and sse == 0.0
+    assert not q.codes.any() and not q.scales.any()
+    # E2M1 grid values with 6 and the tensor max 2688 in every block: the
+    # usual code reproduces them exactly, is scored first and kept
+    grid = np.array(_E2M1_GRID, np.float32)
+    rng = np.random.default_rng(35)
+    w = (rng.choice(grid, (2, 64)) * 448).astype(np.float32)
+    w[:, ::16] = 2688
+    q, sse = orc.quantize_mse_nvfp4(w, 0)
+    u = orc.quantize(w, orc.NVFP4)
+    assert sse == 0.0 and np.array_equal(q.codes, u.codes) and np.array_equal(q.scales, u.scales)
+
+
+def test_mse_nvfp4_rounds_lower_the_error(orc):
+    # the page's claim for NVFP4 without rotations, on heavy-tailed weights:
+    # a sanity check, not parity
+    rng = np.random.default_rng(36)
+    w = (rng.standard_t(4, size=(64, 256)) * 0.0141).astype(np.float32)
+    usual = ((orc.quantize(w, orc.NVFP4).dequantize() - w.astype(np.float64)) ** 2).sum()
+    errs = [orc.quantize_mse_nvfp4(w, it)[1] for it in (0, 1, 3)]
+    assert errs[0] < usual and errs[2] <= errs[0]
+
+
 # ------------------------------------------------------------------ low rank + GEMM
 
 def test_lowrank_down_brute_force(orc):
