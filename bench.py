@@ -356,8 +356,25 @@ def run_ours(args, world, rank, local):
                "GB/s": M * K * 2 / (lr_ms * 1e-3) / 1e9, "frac": M * K * 2 / (lr_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
     del t_buf
     w4 = workloads.svdquant_mlp_up()["w"]
-    wq4 = mxq.quantize(torch.from_numpy(w4).to(torch.bfloat16).to(dev), mxq.INT4_G64, 0, mxq.MMA)
+    w4d = torch.from_numpy(w4).to(torch.bfloat16).to(dev)
     del w4
+    # NVFP4 weight scales fitted to the squared error (two rounds), workload 3's R
+    mse_ws = torch.empty(mxq.quantize_mse_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
+    mse_q = mxq.alloc_qtensor(mxq.NVFP4, N, K, mxq.MMA, dev)
+    mse_ms = graph_ms(lambda i: mxq.quantize_mse(w4d, 2, mxq.MMA, out=mse_q, workspace=mse_ws, want_sse=False),
+                      n=2, reps=3)
+    _, mse_sse = mxq.quantize_mse(w4d, 2, mxq.MMA, out=mse_q, workspace=mse_ws)
+    w64 = w4d.double()
+    usual_sse = ((mxq.dequantize(mxq.quantize(w4d, mxq.NVFP4), torch.float32).double() - w64) ** 2).sum().item()
+    mse_bytes = N * K * 2 + N * K // 2 + N * K // 16
+    mse_row = {"kernel": "k_mse_block (8 scale candidates per block, binary64 errors) x 3 passes + amax and "
+                         "ordered sums, R 12288 x 3072 bf16, 2 rounds",
+               "us": 1e3 * mse_ms, "GB/s": mse_bytes / (mse_ms * 1e-3) / 1e9,
+               "frac": mse_bytes / (mse_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+               "sse_vs_usual_nvfp4": mse_sse.item() / usual_sse}
+    del mse_ws, mse_q, w64
+    wq4 = mxq.quantize(w4d, mxq.INT4_G64, 0, mxq.MMA)
+    del w4d
     xq4 = mxq.quantize(sets[0]["x"], mxq.INT4_G64, 0, mxq.MMA)
     tp4 = mxq.lowrank_down_packed(sets[0]["x"], l1, xq4, wq4)
     i4_ms = graph_ms(lambda i: mxq.qlinear(xq4, wq4, tp4, sets[0]["l2p"], out=sets[i % N_SETS]["y"]), n=4, reps=3)
@@ -423,6 +440,7 @@ def run_ours(args, world, rank, local):
                                  "rows": formats},
             "int4_g64_qlinear": int4,
             "select_weight_format": select,
+            "quantize_mse_nvfp4": mse_row,
             "lowrank_down": lowrank,
             "e2e": {"value": world * FLOP_STEP / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "ms_per_step": e2e_ms},

@@ -194,6 +194,41 @@ mxq_status mxq_select_weight_format(const void *w, int32_t wdtype, int64_t n, in
                                     uint8_t *fmt_per_channel, double *sse, void *workspace,
                                     size_t workspace_bytes, void *stream);
 
+/* Scratch bytes mxq_quantize_mse needs for a rows x cols tensor:
+ * 256 + 16 * rows * cols / 16 + 16 * rows. */
+mxq_status mxq_quantize_mse_workspace_bytes(int64_t rows, int64_t cols, size_t *bytes);
+
+/* NVFP4 quantization with the block and tensor scales fitted to the squared
+ * error ("Bridging the Gap Between Promise and Performance for Microscaling
+ * FP4 Quantization", MR-GPTQ modification 1: the grid is chosen for the MSE
+ * by optimizing the per-block scales and the tensor scale in turn), meant
+ * for weights, which are quantized once.
+ *   Block step, s_t fixed: per 16-element block the E4M3 codes e0, e0 + 1,
+ *     e0 - 1, ..., e0 - 6 (e0 = the usual code; codes in [1, 126]; for
+ *     e0 = 0: 0, 1) are scored in that order by the binary64 sum, in element
+ *     order, of (v - exact dequantized value)^2 with the elements coded as
+ *     usual under each; the first least error wins.
+ *   Tensor step, codes fixed: s_t = fp32(A / B), A = sum v u, B = sum u^2,
+ *     u = E2M1 value x E4M3 value, binary64 sums within a block in element
+ *     order, within a row in block order, over rows in order; B = 0 keeps s_t.
+ *   Start from the usual s_t; `iters` >= 0 rounds of (block step, tensor
+ *   step); a final block step writes codes and scales.
+ * The result is the output layout of mxq_quantize for NVFP4 (codes,
+ * scales, tensor_scale) and dequantizes with mxq_dequantize / feeds
+ * mxq_qlinear unchanged.
+ *   w: rows x cols fp32/bf16 device; fmt: MXQ_NVFP4 (others
+ *     MXQ_EUNSUPPORTED); layout: MXQ_LAYOUT_CANONICAL or MXQ_LAYOUT_MMA.
+ *   sse: device double receiving the total squared error of the result
+ *     (same summation order), or NULL.
+ *   workspace: device scratch of mxq_quantize_mse_workspace_bytes, 256-byte
+ *     aligned; clobbered.
+ * Constraints as mxq_quantize (cols % 16 == 0, 16-byte aligned w and
+ * codes); rows * cols / 16 < 2^31.  Bit-identical from run to run. */
+mxq_status mxq_quantize_mse(const void *w, int32_t wdtype, int64_t rows, int64_t cols, int32_t fmt,
+                            int32_t iters, int32_t layout, void *codes, void *scales,
+                            float *tensor_scale, double *sse, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
 /* ---------------------------------------------------------------------- */
 /* a5-a7: low-rank branch and block-scaled low-bit GEMM.                   */
 /* ---------------------------------------------------------------------- */

@@ -31,7 +31,8 @@ STATUS = {0: "MXQ_OK", 1: "MXQ_EINVAL", 2: "MXQ_EUNSUPPORTED", 3: "MXQ_ECUDA", 4
 # Every entry point the header declares.
 EXPORTS = ("mxq_status_string", "mxq_last_cuda_error_string", "mxq_device_supported", "mxq_check", "mxq_codes_bytes", "mxq_scales_bytes",
            "mxq_quantize_workspace_bytes", "mxq_quantize", "mxq_dequantize", "mxq_hadamard_block", "mxq_cast",
-           "mxq_select_workspace_bytes", "mxq_select_weight_format", "mxq_lowrank_down", "mxq_lowrank_packed_bytes",
+           "mxq_select_workspace_bytes", "mxq_select_weight_format", "mxq_quantize_mse_workspace_bytes",
+           "mxq_quantize_mse", "mxq_lowrank_down", "mxq_lowrank_packed_bytes",
            "mxq_lowrank_down_packed", "mxq_lowrank_pack_t", "mxq_lowrank_pack_l2", "mxq_qlinear", "mxq_route",
            "mxq_quantize_lowrank_workspace_bytes", "mxq_quantize_lowrank", "mxq_quantize_lowrank_noalloc")
 
@@ -71,6 +72,8 @@ def _load():
         "mxq_cast": (i32, [P, i64, i32, P, P]),
         "mxq_select_workspace_bytes": (i32, [P, i32, psz]),
         "mxq_select_weight_format": (i32, [P, i32, i64, i64, P, i32, P, P, P, sz, P]),
+        "mxq_quantize_mse_workspace_bytes": (i32, [i64, i64, psz]),
+        "mxq_quantize_mse": (i32, [P, i32, i64, i64, i32, i32, i32, P, P, P, P, P, sz, P]),
         "mxq_lowrank_down": (i32, [P, i32, i64, i64, P, i32, P, P]),
         "mxq_lowrank_packed_bytes": (i32, [i64, psz]),
         "mxq_lowrank_down_packed": (i32, [P, i32, i64, i64, P, i32, P, P, P, P]),
@@ -222,6 +225,27 @@ def select_weight_format(w: torch.Tensor, candidates: Sequence[int], want_sse: b
     _ok(_lib.mxq_select_weight_format(_ptr(w), _dtype_code(w), n, k, cands, len(candidates), _ptr(choice),
                                       _ptr(sse), _ptr(ws), wsb, _stream(stream)), "mxq_select_weight_format")
     return choice, sse
+
+
+def quantize_mse_workspace_bytes(rows: int, cols: int) -> int:
+    return _size(_lib.mxq_quantize_mse_workspace_bytes, rows, cols)
+
+
+def quantize_mse(w: torch.Tensor, iters: int = 2, layout: int = CANONICAL, out: QTensor = None,
+                 workspace: torch.Tensor = None, want_sse: bool = True, stream=None):
+    """NVFP4 with block and tensor scales fitted to the squared error;
+    returns (QTensor, device float64 total error or None)."""
+    _require_cuda(w)
+    w = w.contiguous()
+    rows, cols = w.shape
+    q = out if out is not None else alloc_qtensor(NVFP4, rows, cols, layout, w.device)
+    wsb = quantize_mse_workspace_bytes(rows, cols)
+    ws = workspace if workspace is not None else torch.empty(wsb, dtype=torch.uint8, device=w.device)
+    sse = torch.empty(1, dtype=torch.float64, device=w.device) if want_sse else None
+    _ok(_lib.mxq_quantize_mse(_ptr(w), _dtype_code(w), rows, cols, NVFP4, iters, layout, _ptr(q.codes),
+                              _ptr(q.scales), _ptr(q.tensor_scale), _ptr(sse), _ptr(ws), ws.numel(), _stream(stream)),
+        "mxq_quantize_mse")
+    return q, sse
 
 
 def lowrank_down(x: torch.Tensor, l1: torch.Tensor, out: torch.Tensor = None, stream=None) -> torch.Tensor:

@@ -176,6 +176,30 @@ mxq_status mxq_select_weight_format(const void *w, int32_t wdtype, int64_t n, in
                                    (unsigned int *)workspace, (cudaStream_t)stream));
 }
 
+mxq_status mxq_quantize_mse_workspace_bytes(int64_t rows, int64_t cols, size_t *bytes) {
+    if (rows < 0 || cols < 0 || cols % 16 || !bytes) return MXQ_EINVAL;
+    *bytes = mse_workspace_bytes(rows, cols);
+    return MXQ_OK;
+}
+
+mxq_status mxq_quantize_mse(const void *w, int32_t wdtype, int64_t rows, int64_t cols, int32_t fmt,
+                            int32_t iters, int32_t layout, void *codes, void *scales, float *tensor_scale,
+                            double *sse, void *workspace, size_t workspace_bytes, void *stream) {
+    if (!valid_fmt(fmt) || !valid_dtype(wdtype) || !valid_layout(layout) || iters < 0) return MXQ_EINVAL;
+    if (fmt != MXQ_NVFP4) return MXQ_EUNSUPPORTED;
+    if (!valid_shape(fmt, rows, cols) || !tensor_scale) return MXQ_EINVAL;
+    const int64_t n = rows * cols;
+    if (n > 0 && (!w || !codes || !scales || !aligned16(w) || !aligned16(codes))) return MXQ_EINVAL;
+    size_t need = 0, sb = 0;
+    mxq_quantize_mse_workspace_bytes(rows, cols, &need);
+    if (!workspace) return MXQ_EINVAL;
+    if (workspace_bytes < need) return MXQ_ENOSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MXQ_EINVAL;
+    mxq_scales_bytes(fmt, rows, cols, layout, &sb);
+    return from_cuda(launch_quantize_mse(w, wdtype == MXQ_BF16, rows, cols, iters, layout, codes, scales, sb,
+                                         tensor_scale, sse, workspace, (cudaStream_t)stream));
+}
+
 mxq_status mxq_lowrank_down(const void *x, int32_t xdtype, int64_t m, int64_t k, const void *l1, int32_t r, float *t,
                             void *stream) {
     if (!valid_dtype(xdtype) || m < 0 || k <= 0 || k % 16 || r < 1 || r > 32) return MXQ_EINVAL;

@@ -1,0 +1,248 @@
+// mse.cu -- NVFP4 weights with the block and tensor scales fitted to the
+// squared error ("Bridging the Gap Between Promise and Performance for
+// Microscaling FP4 Quantization", MR-GPTQ modification 1: the quantization
+// grid is chosen for the MSE by optimizing the per-block scales and the
+// tensor scale in turn).
+//
+// The readings the page leaves open, and which every kernel below follows:
+//  - Block step (tensor scale s_t fixed): e0 is the usual block code;
+//    candidates are scored in the order e0, e0 + 1, e0 - 1, ..., e0 - 6
+//    (codes in [1, 126]; for e0 = 0 the order is 0, 1).  Candidate e codes
+//    the block as usual under it (d = RN(value(e) s_t), q = E2M1(RN(v / d)))
+//    and scores sum_i (v_i - value(q_i) value(e) s_t)^2, the dequantized value
+//    exact in binary64, the sum in binary64 in element order, no fused
+//    multiply-add.  The first least error wins.
+//  - Tensor step (block codes fixed): s_t = RN32(RN64(A / B)) with
+//    A = sum v u, B = sum u^2, u = value(q) value(e), summed in binary64
+//    within a block in element order, within a row in block order and over
+//    rows in row order (B = 0 keeps s_t).
+//  - The usual tensor scale to start, `iters` rounds of (block step, tensor
+//    step), then a final block step writes codes and scales; the total error
+//    of the result is summed in the same order.
+// Fixed summation orders make the result a function of the input alone
+// (bit-identical from run to run and to any other implementation that keeps
+// them).  The per-block work is ALU-bound (8 candidates, binary64 errors);
+// each row's sum runs on lane 0 of a warp that stages the row, the sum over
+// rows on one thread.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "mxq_formats.cuh"
+#include "mxq_internal.h"
+
+namespace mxq {
+
+namespace {
+
+constexpr int kMseThreads = 256;
+enum MseMode : int { kMsePartial = 0, kMseEncode = 1 };
+
+// E2M1 value of a 4-bit code (sign in bit 3) as binary64, assembled from
+// bits: the high 16 bits of the double for magnitudes 0, .5, 1, 1.5, 2, 3, 4,
+// 6 are 0x0000, 0x3FE0, 0x3FF0, 0x3FF8, 0x4000, 0x4008, 0x4010, 0x4018 (the
+// high and low bytes picked from two words each); the low 48 bits are 0.
+__device__ __forceinline__ double e2m1_value_f64(uint32_t code) {
+    const uint32_t m = code & 7u;
+    const uint32_t hi = __byte_perm(0x3F3F3F00u, 0x40404040u, m);
+    const uint32_t lo = __byte_perm(0xF8F0E000u, 0x18100800u, m);
+    return __hiloint2double((int)((hi << 24) | (lo << 16) | ((code & 8u) << 28)), 0);
+}
+
+// Squared error of block v (vd: the same values in binary64) coded under
+// block code e (codes into w0, w1).  The dequantized value is q * (e * s_t):
+// the product of three numbers with 3, 4 and 24 significant bits, exact in
+// binary64 in any order.
+__device__ __forceinline__ double block_error(const float (&v)[16], const double (&vd)[16], uint32_t e, float s_t,
+                                              uint32_t &w0, uint32_t &w1) {
+    w0 = w1 = 0u;
+    double es = 0.0;
+    if (e) {
+        const float ev = dec_e4m3(e);
+        const Recip rd = recip_of(__fmul_rn(ev, s_t));
+        w0 = e2m1x8_quot(v, rd);
+        w1 = e2m1x8_quot(v + 8, rd);
+        es = __dmul_rn((double)ev, (double)s_t);   // exact
+    }
+    double err = 0.0;
+#pragma unroll
+    for (int i = 0; i < 16; i++) {
+        const uint32_t code = ((i < 8 ? w0 : w1) >> (4 * (i & 7))) & 0xFu;
+        const double diff = __dsub_rn(vd[i], __dmul_rn(e2m1_value_f64(code), es));
+        err = __dadd_rn(err, __dmul_rn(diff, diff));
+    }
+    return err;
+}
+
+struct MseArgs {
+    int64_t rows, cols, blocks;   // blocks = rows * cols / 16 < 2^31
+    int layout;
+    uint32_t s_pad4;              // MMA layout: padded scale columns / 4
+    const float *s_t;             // current tensor scale (device)
+    uint8_t *codes;               // kMseEncode
+    uint8_t *scales;              // kMseEncode
+    double *blk;                  // per block: (A, B) for kMsePartial, error for kMseEncode
+};
+
+// One thread per 16-element block: the block step, then the block's
+// least-squares sums (kMsePartial) or its codes, scale byte and error
+// (kMseEncode).
+template <typename T, int MODE>
+__global__ void __launch_bounds__(kMseThreads) k_mse_block(const T *__restrict__ x, MseArgs a) {
+    const int64_t b = (int64_t)blockIdx.x * kMseThreads + threadIdx.x;
+    if (b >= a.blocks) return;
+    float v[16];
+    load16(x + b * 16, v);
+    double vd[16];
+#pragma unroll
+    for (int i = 0; i < 16; i++) vd[i] = (double)v[i];
+    const float s_t = *a.s_t;
+    float d0;
+    const uint32_t e0 = nvfp4_block_scale(amax16(v), s_t, d0);
+    // scoring order e0, e0 + 1, e0 - 1, ..., e0 - 6 (e0 = 0: 0, 1)
+    uint32_t best = e0, bw0, bw1;
+    double best_err = block_error(v, vd, e0, s_t, bw0, bw1);
+    const int n_cand = e0 == 0 ? 2 : 8;
+#pragma unroll 1
+    for (int j = 1; j < n_cand; j++) {
+        const int e = e0 == 0 ? 1 : (j == 1 ? (int)e0 + 1 : (int)e0 - (j - 1));
+        if (e < 1 || e > 126) continue;
+        uint32_t w0, w1;
+        const double err = block_error(v, vd, (uint32_t)e, s_t, w0, w1);
+        if (err < best_err) {
+            best_err = err;
+            best = (uint32_t)e;
+            bw0 = w0;
+            bw1 = w1;
+        }
+    }
+    if (MODE == kMsePartial) {
+        const double ev = best ? (double)dec_e4m3(best) : 0.0;
+        double sa = 0.0, sb = 0.0;
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+            const uint32_t code = ((i < 8 ? bw0 : bw1) >> (4 * (i & 7))) & 0xFu;
+            const double u = __dmul_rn(e2m1_value_f64(code), ev);   // exact
+            sa = __dadd_rn(sa, __dmul_rn(vd[i], u));                // product exact
+            sb = __dadd_rn(sb, __dmul_rn(u, u));
+        }
+        a.blk[2 * b] = sa;
+        a.blk[2 * b + 1] = sb;
+    } else {
+        *reinterpret_cast<uint2 *>(a.codes + b * 8) = make_uint2(bw0, bw1);
+        const uint32_t nb = (uint32_t)(a.cols >> 4);
+        const uint32_t row = (uint32_t)(b / nb), col = (uint32_t)(b - (int64_t)row * nb);
+        a.scales[a.layout == 0 ? (uint32_t)b : mma_scale_offset32(row, col, a.s_pad4)] = (uint8_t)best;
+        a.blk[b] = best_err;
+    }
+}
+
+// One warp per row: the lanes stage the row's block values (W per block: 2
+// for (A, B), 1 for the error) through shared memory 32 blocks at a time,
+// and lane 0 adds them in block order.
+template <int W>
+__global__ void __launch_bounds__(kMseThreads) k_mse_rows(const double *__restrict__ blk, int64_t rows, int64_t nb,
+                                                          double *__restrict__ row_sums) {
+    __shared__ double stage[kMseThreads / 32][32 * W];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t r = (int64_t)blockIdx.x * (kMseThreads / 32) + warp;
+    if (r >= rows) return;
+    const double *p = blk + r * nb * W;
+    double s0 = 0.0, s1 = 0.0;
+    for (int64_t i0 = 0; i0 < nb; i0 += 32) {
+        const int n = nb - i0 < 32 ? (int)(nb - i0) : 32;
+        for (int j = lane; j < n * W; j += 32) stage[warp][j] = p[i0 * W + j];
+        __syncwarp();
+        if (lane == 0) {
+            for (int j = 0; j < n; j++) {
+                s0 = __dadd_rn(s0, stage[warp][j * W]);
+                if (W == 2) s1 = __dadd_rn(s1, stage[warp][j * W + 1]);
+            }
+        }
+        __syncwarp();
+    }
+    if (lane == 0) {
+        row_sums[r * W] = s0;
+        if (W == 2) row_sums[r * W + 1] = s1;
+    }
+}
+
+// One thread: rows summed in order.  W == 2: the least-squares tensor scale
+// replaces *s_t (kept when B == 0); W == 1: the total error into *sse.
+template <int W>
+__global__ void k_mse_tensor(const double *__restrict__ row_sums, int64_t rows, float *s_t, double *sse) {
+    double s0 = 0.0, s1 = 0.0;
+#pragma unroll 8
+    for (int64_t r = 0; r < rows; r++) {
+        s0 = __dadd_rn(s0, row_sums[r * W]);
+        if (W == 2) s1 = __dadd_rn(s1, row_sums[r * W + 1]);
+    }
+    if (W == 2) {
+        if (s1 > 0.0) *s_t = __double2float_rn(__ddiv_rn(s0, s1));
+    } else if (sse) {
+        *sse = s0;
+    }
+}
+
+// The usual tensor scale from the amax word.
+__global__ void k_mse_init(const unsigned int *amax_word, float *s_t) {
+    *s_t = nvfp4_tensor_scale(__uint_as_float(*amax_word));
+}
+
+template <typename T>
+cudaError_t run_mse(const T *x, const MseArgs &base, int iters, double *row_sums, double *sse, cudaStream_t s) {
+    const int64_t nb = base.cols >> 4;
+    const int gb = (int)((base.blocks + kMseThreads - 1) / kMseThreads);
+    const int gr = (int)((base.rows + kMseThreads / 32 - 1) / (kMseThreads / 32));
+    for (int it = 0; it < iters; it++) {
+        k_mse_block<T, kMsePartial><<<gb, kMseThreads, 0, s>>>(x, base);
+        k_mse_rows<2><<<gr, kMseThreads, 0, s>>>(base.blk, base.rows, nb, row_sums);
+        k_mse_tensor<2><<<1, 1, 0, s>>>(row_sums, base.rows, const_cast<float *>(base.s_t), nullptr);
+    }
+    k_mse_block<T, kMseEncode><<<gb, kMseThreads, 0, s>>>(x, base);
+    k_mse_rows<1><<<gr, kMseThreads, 0, s>>>(base.blk, base.rows, nb, row_sums);
+    k_mse_tensor<1><<<1, 1, 0, s>>>(row_sums, base.rows, nullptr, sse);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t mse_workspace_bytes(int64_t rows, int64_t cols) {
+    return 256 + (size_t)(rows * (cols / 16)) * 16 + (size_t)rows * 16;
+}
+
+cudaError_t launch_quantize_mse(const void *w, bool bf16, int64_t rows, int64_t cols, int iters, int layout,
+                                void *codes, void *scales, size_t scales_bytes, float *tensor_scale, double *sse,
+                                void *workspace, cudaStream_t s) {
+    if (rows == 0 || cols == 0) {   // empty tensor: s_t = 1, no error
+        static const float one = 1.0f;
+        static const double zero = 0.0;
+        cudaError_t e = cudaMemcpyAsync(tensor_scale, &one, sizeof(float), cudaMemcpyHostToDevice, s);
+        if (e == cudaSuccess && sse) e = cudaMemcpyAsync(sse, &zero, sizeof(double), cudaMemcpyHostToDevice, s);
+        return e;
+    }
+    unsigned int *amax = (unsigned int *)workspace;
+    double *blk = (double *)((char *)workspace + 256);
+    double *row_sums = blk + 2 * rows * (cols / 16);
+    cudaError_t e = launch_amax(w, bf16, rows, cols, 0, amax, s);
+    if (e != cudaSuccess) return e;
+    k_mse_init<<<1, 1, 0, s>>>(amax, tensor_scale);
+    MseArgs a;
+    a.rows = rows;
+    a.cols = cols;
+    a.blocks = rows * (cols / 16);
+    a.layout = layout;
+    const int64_t S = cols / 16, s_pad = (S + 15) / 16 * 16;
+    a.s_pad4 = (uint32_t)(s_pad >> 2);
+    if (layout == 1 && (s_pad != S || rows % 128)) {   // padding bytes must read as 0
+        e = cudaMemsetAsync(scales, 0, scales_bytes, s);
+        if (e != cudaSuccess) return e;
+    }
+    a.s_t = tensor_scale;
+    a.codes = (uint8_t *)codes;
+    a.scales = (uint8_t *)scales;
+    a.blk = blk;
+    if (bf16) return run_mse((const __nv_bfloat16 *)w, a, iters, row_sums, sse, s);
+    return run_mse((const float *)w, a, iters, row_sums, sse, s);
+}
+
+}  // namespace mxq

@@ -27,6 +27,12 @@ cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols
                             int layout, void *codes, void *scales, size_t scales_bytes, float *tensor_scale,
                             unsigned int *amax_word, cudaStream_t s, const PackT *pack = nullptr,
                             bool amax_ready = false);
+// NVFP4 with block and tensor scales fitted to the squared error (mse.cu);
+// workspace of mse_workspace_bytes, 256-byte aligned.
+size_t mse_workspace_bytes(int64_t rows, int64_t cols);
+cudaError_t launch_quantize_mse(const void *w, bool bf16, int64_t rows, int64_t cols, int iters, int layout,
+                                void *codes, void *scales, size_t scales_bytes, float *tensor_scale, double *sse,
+                                void *workspace, cudaStream_t s);
 cudaError_t launch_dequantize(int fmt, int layout, int64_t rows, int64_t cols, const void *codes,
                               const void *scales, const float *tensor_scale, void *y, bool bf16_out,
                               cudaStream_t s);

@@ -85,6 +85,8 @@ def lib():
         L.orc_select.argtypes = [P, i64, i64, P, i32, P, P, P, P, P]
         L.orc_quantize_mse_nvfp4.restype = i32
         L.orc_quantize_mse_nvfp4.argtypes = [P, i64, i64, i32, P, P, P, P]
+        L.orc_mse_nvfp4_blocks.restype = i32
+        L.orc_mse_nvfp4_blocks.argtypes = [P, i64, i64, ctypes.c_float, P, P, P]
         L.orc_lowrank_down.restype = i32
         L.orc_lowrank_down.argtypes = [P, P, i64, i64, i32, P]
         L.orc_route.restype = i32
@@ -252,6 +254,20 @@ def quantize_mse_nvfp4(x, iters: int):
     if st != 0:
         raise OracleError("bad quantize_mse_nvfp4 arguments")
     return QTensor(NVFP4, rows, cols, codes, scales, float(ts[0])), float(sse[0])
+
+
+def mse_nvfp4_blocks(x, s_t: float):
+    """Block step of quantize_mse_nvfp4 under a given tensor scale: (QTensor,
+    per-row errors)."""
+    x = _f32(x)
+    rows, cols = x.shape
+    codes = np.zeros(codes_shape(NVFP4, rows, cols), dtype=np.uint8)
+    scales = np.zeros((rows, cols // 16), dtype=np.uint8)
+    row_err = np.zeros(rows, dtype=np.float64)
+    st = lib().orc_mse_nvfp4_blocks(_ptr(x), rows, cols, float(s_t), _ptr(codes), _ptr(scales), _ptr(row_err))
+    if st != 0:
+        raise OracleError("bad mse_nvfp4_blocks arguments")
+    return QTensor(NVFP4, rows, cols, codes, scales, float(s_t)), row_err
 
 
 # ---------------------------------------------------------------- low rank + GEMM

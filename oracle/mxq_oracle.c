@@ -570,6 +570,29 @@ static uint8_t mse_block_choose(const float *v, float s_t, uint8_t *q, double *e
     return (uint8_t)best;
 }
 
+/* The block step alone under a given tensor scale (the last step of       */
+/* orc_quantize_mse_nvfp4): codes, scale bytes, and each row's error       */
+/* summed in block order.                                                   */
+int orc_mse_nvfp4_blocks(const float *x, int64_t rows, int64_t cols, float s_t, uint8_t *codes,
+                         uint8_t *scales, double *row_err)
+{
+    if (rows < 0 || cols < 0 || cols % 16) return ORC_EINVAL;
+    int64_t nb = cols / 16;
+    uint8_t q[16];
+    double err;
+    for (int64_t r = 0; r < rows; r++) {
+        double acc = 0.0;
+        for (int64_t b = 0; b < nb; b++) {
+            uint8_t e = mse_block_choose(x + r * cols + b * 16, s_t, q, &err);
+            scales[r * nb + b] = e;
+            for (int i = 0; i < 16; i++) put_code(codes, r * cols + b * 16 + i, 1, q[i]);
+            acc += err;
+        }
+        row_err[r] = acc;
+    }
+    return ORC_OK;
+}
+
 int orc_quantize_mse_nvfp4(const float *x, int64_t rows, int64_t cols, int iters, uint8_t *codes,
                            uint8_t *scales, float *tensor_scale, double *sse)
 {
@@ -603,13 +626,8 @@ int orc_quantize_mse_nvfp4(const float *x, int64_t rows, int64_t cols, int iters
     *tensor_scale = s_t;
     double total = 0.0;
     for (int64_t r = 0; r < rows; r++) {
-        double row_err = 0.0;
-        for (int64_t b = 0; b < nb; b++) {
-            uint8_t e = mse_block_choose(x + r * cols + b * 16, s_t, q, &err);
-            scales[r * nb + b] = e;
-            for (int i = 0; i < 16; i++) put_code(codes, r * cols + b * 16 + i, 1, q[i]);
-            row_err += err;
-        }
+        double row_err;
+        orc_mse_nvfp4_blocks(x + r * cols, 1, cols, s_t, codes + r * (cols / 2), scales + r * nb, &row_err);
         total += row_err;
     }
     if (sse) *sse = total;

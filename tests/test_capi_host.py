@@ -13,8 +13,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def mxq():
-    from microscaling_bit_quantization_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__.build()   # loads build.py by path, so a stale library cannot get in the way
     import microscaling_bit_quantization_b200 as m
     return m
 
@@ -73,6 +73,26 @@ def test_bad_shapes_rejected_on_host(mxq):
     assert L.mxq_hadamard_block(dummy, dummy, 1, 4, 64, 512, None) == 1
     assert L.mxq_lowrank_down(dummy, 1, 4, 64, dummy, 33, dummy, None) == 1
     assert L.mxq_cast(dummy, 10, 2, dummy, None) == 1
+
+
+def test_quantize_mse_argument_checks(mxq):
+    L, P = mxq.lib(), ctypes.c_void_p
+    size = ctypes.c_size_t(0)
+    assert L.mxq_quantize_mse_workspace_bytes(4, 64, ctypes.byref(size)) == 0
+    assert size.value == 256 + 4 * 4 * 16 + 4 * 16
+    assert L.mxq_quantize_mse_workspace_bytes(4, 40, ctypes.byref(size)) == 1
+    d = P(256)
+
+    def call(fmt=mxq.NVFP4, iters=2, cols=64, ts=d, ws=d, wsb=1 << 20):
+        return L.mxq_quantize_mse(d, 1, 4, cols, fmt, iters, 0, d, d, ts, None, ws, wsb, None)
+
+    assert call(fmt=mxq.MXFP4) == 2          # NVFP4 only
+    assert call(iters=-1) == 1
+    assert call(cols=40) == 1
+    assert call(ts=None) == 1
+    assert call(ws=None) == 1
+    assert call(wsb=64) == 5                 # workspace too small
+    assert call(ws=P(256 + 8)) == 1          # workspace not 256-byte aligned
 
 
 def test_qlinear_argument_checks(mxq):

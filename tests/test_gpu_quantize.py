@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import workloads
-from gpu_util import assert_qtensor_equal, dev, host_values, nasty_matrix
+from gpu_util import assert_qtensor_equal, byte_scales_from_mma, dev, host_values, nasty_matrix
 
 pytestmark = pytest.mark.gpu
 
@@ -198,3 +198,66 @@ def test_select_full_size(mxq, orc):
     ref_ch, ref_sse = orc.select_weight_format(w, cands)
     np.testing.assert_allclose(sse.cpu().numpy(), ref_sse, rtol=1e-12, atol=0)
     assert _near_tie_ok(ch.cpu().numpy(), ref_ch, ref_sse, cands) <= 3
+
+
+# ------------------------------------------------------------------ MSE-fitted NVFP4 scales
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("iters", [0, 1, 3])
+def test_quantize_mse_small(mxq, orc, dtype, iters):
+    rows, cols = 37, 512   # ragged rows (padded MMA scale tiles), 32 blocks per row
+    x = nasty_matrix(300 + iters, rows, cols)
+    xv = host_values(x, dtype)
+    ref, ref_sse = orc.quantize_mse_nvfp4(xv, iters)
+    for layout in (mxq.CANONICAL, mxq.MMA):
+        q, sse = mxq.quantize_mse(dev(x, dtype), iters, layout)
+        torch.cuda.synchronize()
+        assert_qtensor_equal(q, ref, layout_mma=layout == mxq.MMA)
+        assert sse.item() == ref_sse
+
+
+def test_quantize_mse_edge_shapes(mxq, orc):
+    for rows, cols in ((1, 16), (129, 16), (3, 1024 + 64), (300, 48)):
+        x = nasty_matrix(11, rows, cols)
+        ref, ref_sse = orc.quantize_mse_nvfp4(x, 2)
+        for layout in (mxq.CANONICAL, mxq.MMA):
+            q, sse = mxq.quantize_mse(dev(x, "f32"), 2, layout)
+            torch.cuda.synchronize()
+            assert_qtensor_equal(q, ref, layout_mma=layout == mxq.MMA)
+            assert sse.item() == ref_sse
+    q, sse = mxq.quantize_mse(torch.empty((0, 64), device="cuda"), 2)
+    assert q.tensor_scale.item() == 1.0 and sse.item() == 0.0
+    z = np.zeros((8, 128), np.float32)
+    q, sse = mxq.quantize_mse(dev(z, "bf16"), 2)
+    ref, _ = orc.quantize_mse_nvfp4(z, 2)
+    assert_qtensor_equal(q, ref)
+    assert sse.item() == 0.0
+
+
+def test_quantize_mse_full_size(mxq, orc):
+    """Workload 3's residual weight R (12288 x 3072 bf16), two rounds, MMA
+    layout: sampled rows against the oracle's block step under the device's
+    final tensor scale; run-to-run identity; the reported error against the
+    dequantized result; lower error than the usual NVFP4 scales."""
+    w = workloads.svdquant_mlp_up()["w"]
+    n, k = w.shape
+    wd = dev(w, "bf16")
+    q, sse = mxq.quantize_mse(wd, 2, mxq.MMA)
+    q2, sse2 = mxq.quantize_mse(wd, 2, mxq.MMA)
+    torch.cuda.synchronize()
+    assert torch.equal(q.codes, q2.codes) and torch.equal(q.scales, q2.scales)
+    assert q.tensor_scale.item() == q2.tensor_scale.item() and sse.item() == sse2.item()
+    s_t = q.tensor_scale.item()
+    rows = np.sort(np.random.default_rng(37).choice(n, 48, replace=False))
+    ref, _ = orc.mse_nvfp4_blocks(w[rows], s_t)
+    codes = q.codes.cpu().numpy().reshape(n, k // 2)
+    np.testing.assert_array_equal(codes[rows], ref.codes)
+    canon, pad = byte_scales_from_mma(q.scales.cpu().numpy(), n, k // 16)
+    np.testing.assert_array_equal(canon[rows], ref.scales)
+    assert (pad == 0).all()
+    wt = torch.from_numpy(w).cuda().double()
+    err = ((mxq.dequantize(q, torch.float32).double() - wt) ** 2).sum().item()
+    assert err == pytest.approx(sse.item(), rel=1e-5)
+    u = mxq.quantize(wd, mxq.NVFP4)
+    usual = ((mxq.dequantize(u, torch.float32).double() - wt) ** 2).sum().item()
+    assert sse.item() < usual
