@@ -192,10 +192,11 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
 // ----------------------------------------------------------------- codes of quotients
 //
 // Codes of RN(v / d) for many v and one divisor d, without an IEEE division
-// per element.  With y = RN(1/d) (correctly rounded reciprocal) and the
+// per element.  With y within one ulp of 1/d (rcp.approx.ftz.f32, whose
+// maximum error the PTX ISA gives as 1 ulp over the full range) and the
 // bracket multipliers y_lo = RN(y (1 - 2^-20)), y_hi = RN(y (1 + 2^-20)), the
 // products L = v y_lo and H = v y_hi (exact reals, or rounded once) satisfy
-// |L| < |v/d|(1 - 13 * 2^-24) and |H| > |v/d|(1 + 13 * 2^-24), so RN(v/d),
+// |L| < |v/d|(1 - 11 * 2^-24) and |H| > |v/d|(1 + 11 * 2^-24), so RN(v/d),
 // which is within 2^-24 of v/d, lies strictly between them.  Every code
 // function used here (E2M1, E4M3, round-to-integer) is monotone, so when the
 // codes of L and H agree the code of RN(v/d) is that code; otherwise a code
@@ -214,7 +215,8 @@ __device__ __forceinline__ Recip recip_of(float d) {
     Recip r;
     r.d = d;
     r.fast = d >= 7.52316384526264e-37f && d <= 1.329227995784916e36f;
-    const float y = r.fast ? __frcp_rn(d) : 0.0f;
+    float y = 0.0f;
+    if (r.fast) asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(d));
     r.lo = __fmul_rn(y, kBracketLo);
     r.hi = __fmul_rn(y, kBracketHi);
     return r;
@@ -459,6 +461,11 @@ __device__ __forceinline__ void hadamard_chunk(float v[16], int b, int lane) {
 // 32-row quarters side by side in each 16-byte line.
 __host__ __device__ __forceinline__ int64_t mma_scale_offset(int64_t r, int64_t s, int64_t s_pad) {
     return ((r >> 7) * (s_pad >> 2) + (s >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (s & 3);
+}
+// The same offset in 32-bit arithmetic (scale arrays below 2^32 bytes);
+// s_pad4 = s_pad / 4.
+__device__ __forceinline__ uint32_t mma_scale_offset32(uint32_t r, uint32_t s, uint32_t s_pad4) {
+    return ((r >> 7) * s_pad4 + (s >> 2)) * 512u + (r & 31u) * 16u + ((r >> 5) & 3u) * 4u + (s & 3u);
 }
 
 }  // namespace mxq

@@ -47,17 +47,6 @@ __device__ __forceinline__ void cta_max_to_word(float m, unsigned int *word) {
     }
 }
 
-// Bytes of four consecutive scale columns s..s+3 (held by lanes lane,
-// lane+L, lane+2L, lane+3L) as one little-endian word, for the lane whose
-// scale column is a multiple of 4.  All lanes must call this.
-template <int L>
-__device__ __forceinline__ uint32_t gather4(uint32_t byte) {
-    uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, byte, L);
-    uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, byte, 2 * L);
-    uint32_t b3 = __shfl_down_sync(0xFFFFFFFFu, byte, 3 * L);
-    return (byte & 0xFFu) | ((b1 & 0xFFu) << 8) | ((b2 & 0xFFu) << 16) | ((b3 & 0xFFu) << 24);
-}
-
 // ------------------------------------------------------------------ quantize
 
 struct QuantArgs {
@@ -70,7 +59,6 @@ struct QuantArgs {
     void *scales;
     float *tensor_scale;     // written by chunk 0 (NVFP4, FP8_TENSOR)
     const unsigned int *amax_word;
-    int combine;             // scale bytes stored as 32-bit words (scale columns per row % 4 == 0)
     // optional packed low-rank operand: tp[row] = [hi | lo] of t[row] / (s_x * *w_ts)
     const float *t;
     int r;
@@ -115,6 +103,88 @@ __device__ __forceinline__ void raw_unpack(const RawChunk<float> &r, float v[16]
     }
 }
 
+// Codes and scale of chunk c (row `row`, chunk column `colc`) from its 16
+// values v and the block amax (already the max over the block's G lanes).
+// All lanes of the warp must call this (no per-lane early exit), but only
+// lanes with `valid` store.
+template <int F>
+__device__ __forceinline__ void encode_chunk(const float (&v)[16], float amax, uint32_t c, uint32_t row, uint32_t colc,
+                                             bool valid, int lane, const QuantArgs &a, uint32_t s_pad4,
+                                             const TensorRecip &tr, const Recip &rt) {
+    constexpr int BLK = fmt_block(F) ? fmt_block(F) : 16;
+    constexpr int G = BLK / 16;
+    const uint32_t cpr = (uint32_t)(a.cols >> 4);
+    uint8_t *scb = reinterpret_cast<uint8_t *>(a.scales);
+    if (F == kMXFP8 || F == kMXFP4) {
+        float inv = 0.0f;
+        uint32_t sb = 127;
+        if (amax > 0.0f) sb = mx_scale(amax, F == kMXFP8 ? 8 : 2, inv);
+        if (!valid) return;
+        // inv is a power of two: v * inv is exact (or far below the smallest code)
+        float u[16];
+        mul8(v, inv, u);
+        mul8(v + 8, inv, u + 8);
+        const bool zero = !(amax > 0.0f);   // all-zero block: +0 codes
+        if (F == kMXFP8) {
+            uint4 w;
+            w.x = zero ? 0u : cvt_e4m3x4(u[0], u[1], u[2], u[3]);
+            w.y = zero ? 0u : cvt_e4m3x4(u[4], u[5], u[6], u[7]);
+            w.z = zero ? 0u : cvt_e4m3x4(u[8], u[9], u[10], u[11]);
+            w.w = zero ? 0u : cvt_e4m3x4(u[12], u[13], u[14], u[15]);
+            *reinterpret_cast<uint4 *>(a.codes + (int64_t)c * 16) = w;
+        } else {
+            uint2 w;
+            w.x = zero ? 0u : cvt_e2m1x8(u[0], u[1], u[2], u[3], u[4], u[5], u[6], u[7]);
+            w.y = zero ? 0u : cvt_e2m1x8(u[8], u[9], u[10], u[11], u[12], u[13], u[14], u[15]);
+            *reinterpret_cast<uint2 *>(a.codes + (int64_t)c * 8) = w;
+        }
+        if ((lane & 1) == 0) {
+            const uint32_t sc = colc >> 1;
+            scb[a.layout == 0 ? row * (cpr >> 1) + sc : mma_scale_offset32(row, sc, s_pad4)] = (uint8_t)sb;
+        }
+    } else if (F == kNVFP4) {
+        float d;
+        const uint32_t e4 = nvfp4_block_scale_fast(amax, tr, d);
+        if (!valid) return;
+        uint2 w = make_uint2(0u, 0u);   // e4 == 0: +0 codes
+        if (e4) {
+            const Recip rd = recip_of(d);
+            w.x = e2m1x8_quot(v, rd);
+            w.y = e2m1x8_quot(v + 8, rd);
+        }
+        *reinterpret_cast<uint2 *>(a.codes + (int64_t)c * 8) = w;
+        scb[a.layout == 0 ? c : mma_scale_offset32(row, colc, s_pad4)] = (uint8_t)e4;
+    } else if (F == kINT4G32 || F == kINT4G64) {
+        const float s = __fdiv_rn(amax, 7.0f);
+        const Recip rs = recip_of(s);
+        if (!valid) return;
+        if (a.layout == 0) {
+            const uint32_t b0 = int_x4_quot(v, rs, 7), b1 = int_x4_quot(v + 4, rs, 7);
+            const uint32_t b2 = int_x4_quot(v + 8, rs, 7), b3 = int_x4_quot(v + 12, rs, 7);
+            *reinterpret_cast<uint2 *>(a.codes + (int64_t)c * 8) =
+                make_uint2(nibbles_of_bytes(b0, b1), nibbles_of_bytes(b2, b3));
+        } else {   // MMA layout: E4M3 bytes of the integer codes
+            *reinterpret_cast<uint4 *>(a.codes + (int64_t)c * 16) =
+                make_uint4(int_x4_quot_e4m3(v, rs, 7), int_x4_quot_e4m3(v + 4, rs, 7),
+                           int_x4_quot_e4m3(v + 8, rs, 7), int_x4_quot_e4m3(v + 12, rs, 7));
+        }
+        if ((lane & (G - 1)) == 0) {
+            float *sc = reinterpret_cast<float *>(a.scales);
+            const uint32_t g = colc / G;
+            if (a.layout == 0) sc[row * (cpr / G) + g] = s;
+            else sc[g * (uint32_t)a.rows + row] = s;
+        }
+    } else if (F == kFP8Tensor) {
+        if (!valid) return;
+        uint4 w;
+        w.x = e4m3x4_quot(v, rt);
+        w.y = e4m3x4_quot(v + 4, rt);
+        w.z = e4m3x4_quot(v + 8, rt);
+        w.w = e4m3x4_quot(v + 12, rt);
+        *reinterpret_cast<uint4 *>(a.codes + (int64_t)c * 16) = w;
+    }
+}
+
 template <typename T, int F>
 __global__ void __launch_bounds__(kQThreads, 2) k_quantize(const T *__restrict__ x, QuantArgs a) {
     constexpr int kQDepth = 64 / (16 * (int)sizeof(T));   // chunks in flight per thread
@@ -129,6 +199,7 @@ __global__ void __launch_bounds__(kQThreads, 2) k_quantize(const T *__restrict__
     c_end = c_end < total ? c_end : total;
     const int steps = (int)((c_end - c_begin + kQThreads - 1) / kQThreads);
     const uint32_t cpr = (uint32_t)(a.cols >> 4);
+    const uint32_t s_pad4 = (uint32_t)(a.s_pad >> 2);
 
     float s_t = 1.0f;
     TensorRecip tr;
@@ -141,126 +212,67 @@ __global__ void __launch_bounds__(kQThreads, 2) k_quantize(const T *__restrict__
         else rt = recip_of(s_t);
     }
 
+    // this thread's chunk c = (row, colc), advanced by kQThreads chunks a step
+    uint32_t c = c_begin + threadIdx.x;
+    uint32_t row = fdiv(c, a.cpr);
+    uint32_t colc = c - row * cpr;
+    const uint32_t drow = fdiv((uint32_t)kQThreads, a.cpr);
+    const uint32_t dcol = (uint32_t)kQThreads - drow * cpr;
+
+    float tensor_max = 0.0f;
     RawChunk<T> pre[kQDepth];
 #pragma unroll
     for (int i = 0; i < kQDepth; i++) {
-        const uint32_t c = c_begin + (uint32_t)i * kQThreads + threadIdx.x;
-        if (c < c_end) raw_load(pre[i], x + (int64_t)c * 16);
+        const uint32_t ci = c + (uint32_t)i * kQThreads;
+        if (ci < c_end) raw_load(pre[i], x + (int64_t)ci * 16);
     }
-    float tensor_max = 0.0f;
+    // The integer formats keep their register budget for the codes: one
+    // chunk per loop turn, the prefetch buffers moved down each turn and the
+    // chunk position recomputed.  The others take kQDepth steps a turn with
+    // buffer j always holding step it0 + j (no buffer moves) and advance the
+    // position incrementally.
+    constexpr bool kRotate = F == kINT4G32 || F == kINT4G64;
+    constexpr int kTurn = kRotate ? 1 : kQDepth;
 #pragma unroll 1
-    for (int it = 0; it < steps; it++) {
-        const uint32_t c = c_begin + (uint32_t)it * kQThreads + threadIdx.x;
-        const bool valid = c < c_end;
-        float v[16];
-        if (valid) raw_unpack(pre[0], v);
-        else {
+    for (int it0 = 0; it0 < steps; it0 += kTurn) {
 #pragma unroll
-            for (int i = 0; i < 16; i++) v[i] = 0.0f;
-        }
+        for (int j = 0; j < kTurn; j++) {
+            if (it0 + j < steps) {
+                const bool valid = c < c_end;
+                float v[16];
+                if (valid) raw_unpack(pre[j], v);
+                else {
 #pragma unroll
-        for (int i = 0; i + 1 < kQDepth; i++) pre[i] = pre[i + 1];
-        {
-            const uint32_t cn = c + (uint32_t)kQDepth * kQThreads;
-            if (cn < c_end) raw_load(pre[kQDepth - 1], x + (int64_t)cn * 16);
-        }
-
-        if (a.hadamard_b) hadamard_chunk(v, a.hadamard_b, lane);
-        const uint32_t row = fdiv(c, a.cpr);
-        const uint32_t colc = c - row * cpr;   // chunk index within the row
-        float amax = amax16(v);
-        if (F == kNumFmt) {   // tensor-amax pass only
-            tensor_max = fmaxf(tensor_max, amax);
-            continue;
-        }
-        if (G > 1) amax = group_max<G>(amax);
-
-        if (F == kMXFP8 || F == kMXFP4) {
-            float inv = 0.0f;
-            uint32_t sb = 127;
-            if (amax > 0.0f) sb = mx_scale(amax, F == kMXFP8 ? 8 : 2, inv);
-            if (valid) {
-                // inv is a power of two: v * inv is exact (or far below the smallest code)
-                float u[16];
-                mul8(v, inv, u);
-                mul8(v + 8, inv, u + 8);
-                const bool zero = !(amax > 0.0f);   // all-zero block: +0 codes
-                if (F == kMXFP8) {
-                    uint4 w;
-                    w.x = zero ? 0u : cvt_e4m3x4(u[0], u[1], u[2], u[3]);
-                    w.y = zero ? 0u : cvt_e4m3x4(u[4], u[5], u[6], u[7]);
-                    w.z = zero ? 0u : cvt_e4m3x4(u[8], u[9], u[10], u[11]);
-                    w.w = zero ? 0u : cvt_e4m3x4(u[12], u[13], u[14], u[15]);
-                    *reinterpret_cast<uint4 *>(a.codes + (int64_t)c * 16) = w;
+                    for (int i = 0; i < 16; i++) v[i] = 0.0f;
+                }
+                const uint32_t cn = c + (uint32_t)kQDepth * kQThreads;
+                if constexpr (kRotate) {
+#pragma unroll
+                    for (int i = 0; i + 1 < kQDepth; i++) pre[i] = pre[i + 1];
+                    if (cn < c_end) raw_load(pre[kQDepth - 1], x + (int64_t)cn * 16);
                 } else {
-                    uint2 w;
-                    w.x = zero ? 0u : cvt_e2m1x8(u[0], u[1], u[2], u[3], u[4], u[5], u[6], u[7]);
-                    w.y = zero ? 0u : cvt_e2m1x8(u[8], u[9], u[10], u[11], u[12], u[13], u[14], u[15]);
-                    *reinterpret_cast<uint2 *>(a.codes + (int64_t)c * 8) = w;
+                    if (cn < c_end) raw_load(pre[j], x + (int64_t)cn * 16);
                 }
-            }
-            const uint32_t word = gather4<2>(sb);
-            if (valid) {
-                const uint32_t sc = colc >> 1;
-                uint8_t *scb = reinterpret_cast<uint8_t *>(a.scales);
-                const int64_t off = a.layout == 0 ? (int64_t)row * (cpr >> 1) + sc : mma_scale_offset(row, sc, a.s_pad);
-                if (a.combine) {
-                    if ((lane & 7) == 0) *reinterpret_cast<uint32_t *>(scb + off) = word;
-                } else if ((lane & 1) == 0) {
-                    scb[off] = (uint8_t)sb;
-                }
-            }
-        } else if (F == kNVFP4) {
-            float d;
-            const uint32_t e4 = nvfp4_block_scale_fast(amax, tr, d);
-            if (valid) {
-                uint2 w = make_uint2(0u, 0u);   // e4 == 0: +0 codes
-                if (e4) {
-                    const Recip rd = recip_of(d);
-                    w.x = e2m1x8_quot(v, rd);
-                    w.y = e2m1x8_quot(v + 8, rd);
-                }
-                *reinterpret_cast<uint2 *>(a.codes + (int64_t)c * 8) = w;
-            }
-            const uint32_t word = gather4<1>(e4);
-            if (valid) {
-                uint8_t *scb = reinterpret_cast<uint8_t *>(a.scales);
-                const int64_t off = a.layout == 0 ? (int64_t)c : mma_scale_offset(row, colc, a.s_pad);
-                if (a.combine) {
-                    if ((lane & 3) == 0) *reinterpret_cast<uint32_t *>(scb + off) = word;
+                if (a.hadamard_b) hadamard_chunk(v, a.hadamard_b, lane);
+                float amax = amax16(v);
+                if (F == kNumFmt) {   // tensor-amax pass only
+                    tensor_max = fmaxf(tensor_max, amax);
                 } else {
-                    scb[off] = (uint8_t)e4;
+                    if (G > 1) amax = group_max<G>(amax);
+                    encode_chunk<F>(v, amax, c, row, colc, valid, lane, a, s_pad4, tr, rt);
                 }
-            }
-        } else if (F == kINT4G32 || F == kINT4G64) {
-            const float s = __fdiv_rn(amax, 7.0f);
-            const Recip rs = recip_of(s);
-            if (valid) {
-                if (a.layout == 0) {
-                    const uint32_t b0 = int_x4_quot(v, rs, 7), b1 = int_x4_quot(v + 4, rs, 7);
-                    const uint32_t b2 = int_x4_quot(v + 8, rs, 7), b3 = int_x4_quot(v + 12, rs, 7);
-                    *reinterpret_cast<uint2 *>(a.codes + (int64_t)c * 8) =
-                        make_uint2(nibbles_of_bytes(b0, b1), nibbles_of_bytes(b2, b3));
-                } else {   // MMA layout: E4M3 bytes of the integer codes
-                    *reinterpret_cast<uint4 *>(a.codes + (int64_t)c * 16) =
-                        make_uint4(int_x4_quot_e4m3(v, rs, 7), int_x4_quot_e4m3(v + 4, rs, 7),
-                                   int_x4_quot_e4m3(v + 8, rs, 7), int_x4_quot_e4m3(v + 12, rs, 7));
+                c += kQThreads;
+                if constexpr (kRotate) {
+                    row = fdiv(c, a.cpr);
+                    colc = c - row * cpr;
+                } else {
+                    row += drow;
+                    colc += dcol;
+                    if (colc >= cpr) {
+                        colc -= cpr;
+                        row++;
+                    }
                 }
-                if ((lane & (G - 1)) == 0) {
-                    float *sc = reinterpret_cast<float *>(a.scales);
-                    const uint32_t g = colc / G;
-                    if (a.layout == 0) sc[(int64_t)row * (cpr / G) + g] = s;
-                    else sc[(int64_t)g * a.rows + row] = s;
-                }
-            }
-        } else if (F == kFP8Tensor) {
-            if (valid) {
-                uint4 w;
-                w.x = e4m3x4_quot(v, rt);
-                w.y = e4m3x4_quot(v + 4, rt);
-                w.z = e4m3x4_quot(v + 8, rt);
-                w.w = e4m3x4_quot(v + 12, rt);
-                *reinterpret_cast<uint4 *>(a.codes + (int64_t)c * 16) = w;
             }
         }
     }
@@ -275,12 +287,12 @@ __global__ void __launch_bounds__(kQThreads, 2) k_quantize(const T *__restrict__
         const float alpha = ts ? __fmul_rn(s_t, *a.w_ts) : 1.0f;
         const int64_t warp = ((int64_t)blockIdx.x * kQThreads + threadIdx.x) >> 5;
         const int64_t nwarps = ((int64_t)gridDim.x * kQThreads) >> 5;
-        for (int64_t row = warp; row < a.rows; row += nwarps) {
-            float u = lane < a.r ? a.t[row * a.r + lane] : 0.0f;
+        for (int64_t r = warp; r < a.rows; r += nwarps) {
+            float u = lane < a.r ? a.t[r * a.r + lane] : 0.0f;
             if (ts) u = __fdiv_rn(u, alpha);
             const __nv_bfloat16 hi = __float2bfloat16_rn(u);
-            a.tp[row * 64 + lane] = hi;
-            a.tp[row * 64 + 32 + lane] = __float2bfloat16_rn(__fsub_rn(u, __bfloat162float(hi)));
+            a.tp[r * 64 + lane] = hi;
+            a.tp[r * 64 + 32 + lane] = __float2bfloat16_rn(__fsub_rn(u, __bfloat162float(hi)));
         }
     }
 }
@@ -655,7 +667,6 @@ cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols
     a.scales = scales;
     a.tensor_scale = tensor_scale;
     a.amax_word = amax_word;
-    a.combine = fmt_byte_scales(fmt) && (cols / fmt_block(fmt)) % 4 == 0;
     a.t = pack ? pack->t : nullptr;
     a.r = pack ? pack->r : 0;
     a.w_ts = pack ? pack->w_ts : nullptr;
