@@ -195,7 +195,7 @@ mxq_status mxq_select_weight_format(const void *w, int32_t wdtype, int64_t n, in
                                     size_t workspace_bytes, void *stream);
 
 /* Scratch bytes mxq_quantize_mse needs for a rows x cols tensor:
- * 256 + 16 * rows * cols / 16 + 16 * rows. */
+ * 256 + 16 * (rows * cols / 16) + 16 * rows + 16 * ceil(rows / 128). */
 mxq_status mxq_quantize_mse_workspace_bytes(int64_t rows, int64_t cols, size_t *bytes);
 
 /* NVFP4 quantization with the block and tensor scales fitted to the squared
@@ -210,7 +210,9 @@ mxq_status mxq_quantize_mse_workspace_bytes(int64_t rows, int64_t cols, size_t *
  *     usual under each; the first least error wins.
  *   Tensor step, codes fixed: s_t = fp32(A / B), A = sum v u, B = sum u^2,
  *     u = E2M1 value x E4M3 value, binary64 sums within a block in element
- *     order, within a row in block order, over rows in order; B = 0 keeps s_t.
+ *     order, within a row in block order, over each group of 128
+ *     consecutive rows in row order, over the groups in order; B = 0 keeps
+ *     s_t.  The total error below is summed in the same order.
  *   Start from the usual s_t; `iters` >= 0 rounds of (block step, tensor
  *   step); a final block step writes codes and scales.
  * The result is the output layout of mxq_quantize for NVFP4 (codes,

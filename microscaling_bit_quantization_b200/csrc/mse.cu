@@ -14,16 +14,16 @@
 //    multiply-add.  The first least error wins.
 //  - Tensor step (block codes fixed): s_t = RN32(RN64(A / B)) with
 //    A = sum v u, B = sum u^2, u = value(q) value(e), summed in binary64
-//    within a block in element order, within a row in block order and over
-//    rows in row order (B = 0 keeps s_t).
+//    within a block in element order, within a row in block order, over
+//    each group of 128 consecutive rows in row order and over the groups in
+//    order (B = 0 keeps s_t).
 //  - The usual tensor scale to start, `iters` rounds of (block step, tensor
 //    step), then a final block step writes codes and scales; the total error
 //    of the result is summed in the same order.
 // Fixed summation orders make the result a function of the input alone
 // (bit-identical from run to run and to any other implementation that keeps
 // them).  The per-block work is ALU-bound (8 candidates, binary64 errors);
-// each row's sum runs on lane 0 of a warp that stages the row, the sum over
-// rows on one thread.
+// each ordered sum runs on lane 0 of a warp that stages its entries.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -35,6 +35,7 @@ namespace mxq {
 namespace {
 
 constexpr int kMseThreads = 256;
+constexpr int64_t kMseGroup = 128;   // rows per group of the tensor-level sums
 enum MseMode : int { kMsePartial = 0, kMseEncode = 1 };
 
 // E2M1 value of a 4-bit code (sign in bit 3) as binary64, assembled from
@@ -136,21 +137,27 @@ __global__ void __launch_bounds__(kMseThreads) k_mse_block(const T *__restrict__
     }
 }
 
-// One warp per row: the lanes stage the row's block values (W per block: 2
-// for (A, B), 1 for the error) through shared memory 32 blocks at a time,
-// and lane 0 adds them in block order.
-template <int W>
-__global__ void __launch_bounds__(kMseThreads) k_mse_rows(const double *__restrict__ blk, int64_t rows, int64_t nb,
-                                                          double *__restrict__ row_sums) {
+// Ordered sums, one warp per output: output o adds entries
+// [o * per, min((o + 1) * per, total)) of `in` (W values per entry: 2 for
+// (A, B), 1 for the error) in index order; the lanes stage 32 entries at a
+// time through shared memory and lane 0 adds them.  Applied level by level:
+// blocks -> rows (per = blocks per row), rows -> groups of kMseGroup rows,
+// groups -> tensor.  FINAL (one output): W == 2 replaces *s_t by the
+// least-squares scale RN32(RN64(A / B)) (kept when B == 0); W == 1 writes the
+// total error to *sse.
+template <int W, bool FINAL>
+__global__ void __launch_bounds__(kMseThreads) k_mse_sum(const double *__restrict__ in, int64_t total, int64_t per,
+                                                         double *__restrict__ out, float *s_t, double *sse) {
     __shared__ double stage[kMseThreads / 32][32 * W];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t r = (int64_t)blockIdx.x * (kMseThreads / 32) + warp;
-    if (r >= rows) return;
-    const double *p = blk + r * nb * W;
+    const int64_t o = (int64_t)blockIdx.x * (kMseThreads / 32) + warp;
+    const int64_t begin = o * per;
+    if (begin >= total && !(FINAL && o == 0)) return;
+    const int64_t end = begin + per < total ? begin + per : total;
     double s0 = 0.0, s1 = 0.0;
-    for (int64_t i0 = 0; i0 < nb; i0 += 32) {
-        const int n = nb - i0 < 32 ? (int)(nb - i0) : 32;
-        for (int j = lane; j < n * W; j += 32) stage[warp][j] = p[i0 * W + j];
+    for (int64_t i0 = begin; i0 < end; i0 += 32) {
+        const int n = end - i0 < 32 ? (int)(end - i0) : 32;
+        for (int j = lane; j < n * W; j += 32) stage[warp][j] = in[i0 * W + j];
         __syncwarp();
         if (lane == 0) {
             for (int j = 0; j < n; j++) {
@@ -160,23 +167,11 @@ __global__ void __launch_bounds__(kMseThreads) k_mse_rows(const double *__restri
         }
         __syncwarp();
     }
-    if (lane == 0) {
-        row_sums[r * W] = s0;
-        if (W == 2) row_sums[r * W + 1] = s1;
-    }
-}
-
-// One thread: rows summed in order.  W == 2: the least-squares tensor scale
-// replaces *s_t (kept when B == 0); W == 1: the total error into *sse.
-template <int W>
-__global__ void k_mse_tensor(const double *__restrict__ row_sums, int64_t rows, float *s_t, double *sse) {
-    double s0 = 0.0, s1 = 0.0;
-#pragma unroll 8
-    for (int64_t r = 0; r < rows; r++) {
-        s0 = __dadd_rn(s0, row_sums[r * W]);
-        if (W == 2) s1 = __dadd_rn(s1, row_sums[r * W + 1]);
-    }
-    if (W == 2) {
+    if (lane != 0) return;
+    if (!FINAL) {
+        out[o * W] = s0;
+        if (W == 2) out[o * W + 1] = s1;
+    } else if (W == 2) {
         if (s1 > 0.0) *s_t = __double2float_rn(__ddiv_rn(s0, s1));
     } else if (sse) {
         *sse = s0;
@@ -188,26 +183,37 @@ __global__ void k_mse_init(const unsigned int *amax_word, float *s_t) {
     *s_t = nvfp4_tensor_scale(__uint_as_float(*amax_word));
 }
 
+template <int W>
+void launch_sums(const double *blk, int64_t blocks, int64_t nb, int64_t rows, double *row_sums, double *grp_sums,
+                 float *s_t, double *sse, cudaStream_t s) {
+    constexpr int kWarps = kMseThreads / 32;
+    const int64_t groups = (rows + kMseGroup - 1) / kMseGroup;
+    k_mse_sum<W, false><<<(int)((rows + kWarps - 1) / kWarps), kMseThreads, 0, s>>>(blk, blocks, nb, row_sums,
+                                                                                    nullptr, nullptr);
+    k_mse_sum<W, false><<<(int)((groups + kWarps - 1) / kWarps), kMseThreads, 0, s>>>(row_sums, rows, kMseGroup,
+                                                                                      grp_sums, nullptr, nullptr);
+    k_mse_sum<W, true><<<1, 32, 0, s>>>(grp_sums, groups, groups, nullptr, s_t, sse);
+}
+
 template <typename T>
-cudaError_t run_mse(const T *x, const MseArgs &base, int iters, double *row_sums, double *sse, cudaStream_t s) {
+cudaError_t run_mse(const T *x, const MseArgs &base, int iters, double *row_sums, double *grp_sums, double *sse,
+                    cudaStream_t s) {
     const int64_t nb = base.cols >> 4;
     const int gb = (int)((base.blocks + kMseThreads - 1) / kMseThreads);
-    const int gr = (int)((base.rows + kMseThreads / 32 - 1) / (kMseThreads / 32));
     for (int it = 0; it < iters; it++) {
         k_mse_block<T, kMsePartial><<<gb, kMseThreads, 0, s>>>(x, base);
-        k_mse_rows<2><<<gr, kMseThreads, 0, s>>>(base.blk, base.rows, nb, row_sums);
-        k_mse_tensor<2><<<1, 1, 0, s>>>(row_sums, base.rows, const_cast<float *>(base.s_t), nullptr);
+        launch_sums<2>(base.blk, base.blocks, nb, base.rows, row_sums, grp_sums, const_cast<float *>(base.s_t),
+                       nullptr, s);
     }
     k_mse_block<T, kMseEncode><<<gb, kMseThreads, 0, s>>>(x, base);
-    k_mse_rows<1><<<gr, kMseThreads, 0, s>>>(base.blk, base.rows, nb, row_sums);
-    k_mse_tensor<1><<<1, 1, 0, s>>>(row_sums, base.rows, nullptr, sse);
+    launch_sums<1>(base.blk, base.blocks, nb, base.rows, row_sums, grp_sums, nullptr, sse, s);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 size_t mse_workspace_bytes(int64_t rows, int64_t cols) {
-    return 256 + (size_t)(rows * (cols / 16)) * 16 + (size_t)rows * 16;
+    return 256 + (size_t)(rows * (cols / 16)) * 16 + (size_t)rows * 16 + (size_t)((rows + kMseGroup - 1) / kMseGroup) * 16;
 }
 
 cudaError_t launch_quantize_mse(const void *w, bool bf16, int64_t rows, int64_t cols, int iters, int layout,
@@ -223,6 +229,7 @@ cudaError_t launch_quantize_mse(const void *w, bool bf16, int64_t rows, int64_t 
     unsigned int *amax = (unsigned int *)workspace;
     double *blk = (double *)((char *)workspace + 256);
     double *row_sums = blk + 2 * rows * (cols / 16);
+    double *grp_sums = row_sums + 2 * rows;
     cudaError_t e = launch_amax(w, bf16, rows, cols, 0, amax, s);
     if (e != cudaSuccess) return e;
     k_mse_init<<<1, 1, 0, s>>>(amax, tensor_scale);
@@ -241,8 +248,8 @@ cudaError_t launch_quantize_mse(const void *w, bool bf16, int64_t rows, int64_t 
     a.codes = (uint8_t *)codes;
     a.scales = (uint8_t *)scales;
     a.blk = blk;
-    if (bf16) return run_mse((const __nv_bfloat16 *)w, a, iters, row_sums, sse, s);
-    return run_mse((const float *)w, a, iters, row_sums, sse, s);
+    if (bf16) return run_mse((const __nv_bfloat16 *)w, a, iters, row_sums, grp_sums, sse, s);
+    return run_mse((const float *)w, a, iters, row_sums, grp_sums, sse, s);
 }
 
 }  // namespace mxq

@@ -518,13 +518,17 @@ int orc_select(const float *w, int64_t n, int64_t k, const int *cands, int ncand
 /*  - Tensor step (block codes fixed).  Least squares for the common    */
 /*    factor: s_t = RN32(RN64(A / B)), A = sum v_i u_i, B = sum u_i^2,  */
 /*    u_i = value(q_i) value(e); binary64 sums within a block in        */
-/*    element order, within a row in block order, over rows in row      */
-/*    order.  B = 0 keeps s_t.                                          */
+/*    element order, within a row in block order, over each group of    */
+/*    128 consecutive rows in row order, then over the groups in order  */
+/*    (a fixed order whose longest chain of additions is short enough   */
+/*    to run in parallel).  B = 0 keeps s_t.                            */
 /*  - Start from the usual tensor scale; `iters` rounds of (block step, */
 /*    tensor step); a final block step gives codes and scales.  The     */
 /*    total error of the result (same summation order) goes to *sse.    */
 /* Output layout as orc_quantize's canonical NVFP4.                     */
 /* ------------------------------------------------------------------ */
+
+#define ORC_MSE_GROUP 128   /* rows per group of the tensor-level sums */
 
 /* error of block v under block code e (codes into q[16] when q != NULL) */
 static double mse_block_error(const float *v, float s_t, uint8_t e, uint8_t *q)
@@ -604,31 +608,40 @@ int orc_quantize_mse_nvfp4(const float *x, int64_t rows, int64_t cols, int iters
     double err;
     for (int it = 0; it < iters; it++) {
         double a_sum = 0.0, b_sum = 0.0;
-        for (int64_t r = 0; r < rows; r++) {
-            double a_row = 0.0, b_row = 0.0;
-            for (int64_t b = 0; b < nb; b++) {
-                const float *v = x + r * cols + b * 16;
-                uint8_t e = mse_block_choose(v, s_t, q, &err);
-                double a_blk = 0.0, b_blk = 0.0;
-                for (int i = 0; i < 16; i++) {
-                    double u = orc_e2m1_value(q[i]) * orc_e4m3_value(e);
-                    a_blk += (double)v[i] * u;
-                    b_blk += u * u;
+        for (int64_t g0 = 0; g0 < rows; g0 += ORC_MSE_GROUP) {
+            double a_grp = 0.0, b_grp = 0.0;
+            for (int64_t r = g0; r < rows && r < g0 + ORC_MSE_GROUP; r++) {
+                double a_row = 0.0, b_row = 0.0;
+                for (int64_t b = 0; b < nb; b++) {
+                    const float *v = x + r * cols + b * 16;
+                    uint8_t e = mse_block_choose(v, s_t, q, &err);
+                    double a_blk = 0.0, b_blk = 0.0;
+                    for (int i = 0; i < 16; i++) {
+                        double u = orc_e2m1_value(q[i]) * orc_e4m3_value(e);
+                        a_blk += (double)v[i] * u;
+                        b_blk += u * u;
+                    }
+                    a_row += a_blk;
+                    b_row += b_blk;
                 }
-                a_row += a_blk;
-                b_row += b_blk;
+                a_grp += a_row;
+                b_grp += b_row;
             }
-            a_sum += a_row;
-            b_sum += b_row;
+            a_sum += a_grp;
+            b_sum += b_grp;
         }
         if (b_sum > 0.0) s_t = (float)(a_sum / b_sum);
     }
     *tensor_scale = s_t;
     double total = 0.0;
-    for (int64_t r = 0; r < rows; r++) {
-        double row_err;
-        orc_mse_nvfp4_blocks(x + r * cols, 1, cols, s_t, codes + r * (cols / 2), scales + r * nb, &row_err);
-        total += row_err;
+    for (int64_t g0 = 0; g0 < rows; g0 += ORC_MSE_GROUP) {
+        double grp = 0.0;
+        for (int64_t r = g0; r < rows && r < g0 + ORC_MSE_GROUP; r++) {
+            double row_err;
+            orc_mse_nvfp4_blocks(x + r * cols, 1, cols, s_t, codes + r * (cols / 2), scales + r * nb, &row_err);
+            grp += row_err;
+        }
+        total += grp;
     }
     if (sse) *sse = total;
     return ORC_OK;

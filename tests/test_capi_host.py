@@ -79,7 +79,9 @@ def test_quantize_mse_argument_checks(mxq):
     L, P = mxq.lib(), ctypes.c_void_p
     size = ctypes.c_size_t(0)
     assert L.mxq_quantize_mse_workspace_bytes(4, 64, ctypes.byref(size)) == 0
-    assert size.value == 256 + 4 * 4 * 16 + 4 * 16
+    assert size.value == 256 + 4 * 4 * 16 + 4 * 16 + 16
+    assert L.mxq_quantize_mse_workspace_bytes(300, 32, ctypes.byref(size)) == 0
+    assert size.value == 256 + 600 * 16 + 300 * 16 + 3 * 16
     assert L.mxq_quantize_mse_workspace_bytes(4, 40, ctypes.byref(size)) == 1
     d = P(256)
 
