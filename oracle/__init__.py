@@ -87,6 +87,10 @@ def lib():
         L.orc_quantize_mse_nvfp4.argtypes = [P, i64, i64, i32, P, P, P, P]
         L.orc_mse_nvfp4_blocks.restype = i32
         L.orc_mse_nvfp4_blocks.argtypes = [P, i64, i64, ctypes.c_float, P, P, P]
+        L.orc_quantize_mx_grid.restype = i32
+        L.orc_quantize_mx_grid.argtypes = [P, i64, i64, i32, i32, ctypes.c_float, P, P, P]
+        L.orc_mx_grid_sse.restype = i32
+        L.orc_mx_grid_sse.argtypes = [P, i64, i64, i32, i32, P, i32, P, P, P, P]
         L.orc_lowrank_down.restype = i32
         L.orc_lowrank_down.argtypes = [P, P, i64, i64, i32, P]
         L.orc_route.restype = i32
@@ -268,6 +272,39 @@ def mse_nvfp4_blocks(x, s_t: float):
     if st != 0:
         raise OracleError("bad mse_nvfp4_blocks arguments")
     return QTensor(NVFP4, rows, cols, codes, scales, float(s_t)), row_err
+
+
+# ---------------------------------------------------------------- MX fixed grid scale
+
+def quantize_mx_grid(x, fmt: int, g: float, hadamard_b: int = 0) -> QTensor:
+    """MXFP4 / MXFP8 with the exponent taken from RN32(g amax) (mxq_oracle.c,
+    orc_quantize_mx_grid)."""
+    x = _f32(x)
+    rows, cols = x.shape
+    codes = np.zeros(codes_shape(fmt, rows, cols), dtype=np.uint8)
+    scales = np.zeros((rows, cols // 32), dtype=np.uint8)
+    work = np.empty_like(x) if hadamard_b else np.empty(1, np.float32)
+    st = lib().orc_quantize_mx_grid(_ptr(x), rows, cols, fmt, hadamard_b, float(g), _ptr(work), _ptr(codes),
+                                    _ptr(scales))
+    if st != 0:
+        raise OracleError("bad quantize_mx_grid arguments")
+    return QTensor(fmt, rows, cols, codes, scales, 0.0)
+
+
+def mx_grid_sse(x, fmt: int, grid_scales, hadamard_b: int = 0) -> np.ndarray:
+    """Squared error of the (rotated) tensor for each candidate grid scale."""
+    x = _f32(x)
+    rows, cols = x.shape
+    gs = np.ascontiguousarray(np.asarray(grid_scales, dtype=np.float32))
+    codes = np.zeros(codes_shape(fmt, rows, cols), dtype=np.uint8)
+    scales = np.zeros((rows, cols // 32), dtype=np.uint8)
+    work = np.empty_like(x) if hadamard_b else np.empty(1, np.float32)
+    sse = np.zeros(len(gs), dtype=np.float64)
+    st = lib().orc_mx_grid_sse(_ptr(x), rows, cols, fmt, hadamard_b, _ptr(gs), len(gs), _ptr(work), _ptr(codes),
+                               _ptr(scales), _ptr(sse))
+    if st != 0:
+        raise OracleError("bad mx_grid_sse arguments")
+    return sse
 
 
 # ---------------------------------------------------------------- low rank + GEMM

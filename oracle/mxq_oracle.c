@@ -278,7 +278,8 @@ static float amax_of(const float *v, int64_t n)
  * clamped to the E8M0 range [-127, 127]; element = RNE_sat(v / X), the
  * division by a power of two done as an fp32 multiply by 2^-e.
  * Reading: an all-zero block gets scale byte 127 (X = 1) and +0 codes. */
-static void quant_mx_block(const float *v, int n, int fp4, uint8_t *codes, int64_t base,
+/* g: grid scale (see orc_quantize_mx_grid); 1 gives the OCP rule. */
+static void quant_mx_block(const float *v, int n, int fp4, float g, uint8_t *codes, int64_t base,
                            uint8_t *scale)
 {
     float amax = amax_of(v, n);
@@ -287,7 +288,9 @@ static void quant_mx_block(const float *v, int n, int fp4, uint8_t *codes, int64
         for (int i = 0; i < n; i++) put_code(codes, base + i, fp4, 0);
         return;
     }
-    int e = floor_log2_f32(amax) - (fp4 ? 2 : 8);
+    int fl = floor_log2_f32(amax);
+    double m = ldexp((double)amax, -fl);               /* significand in [1, 2), exact */
+    int e = fl + ((double)g * m >= 2.0 ? 1 : 0) - (fp4 ? 2 : 8);   /* product exact */
     if (e < -127) e = -127;
     if (e > 127) e = 127;
     *scale = (uint8_t)(e + 127);
@@ -394,7 +397,7 @@ int orc_quantize(const float *x, int64_t rows, int64_t cols, int fmt, int hadama
         case ORC_MXFP8:
         case ORC_MXFP4:
             for (int64_t c = 0; c < cols; c += 32)
-                quant_mx_block(row + c, 32, fmt == ORC_MXFP4, codes, base + c,
+                quant_mx_block(row + c, 32, fmt == ORC_MXFP4, 1.0f, codes, base + c,
                                (uint8_t *)scales + r * (cols / 32) + c / 32);
             break;
         case ORC_NVFP4:
@@ -644,6 +647,78 @@ int orc_quantize_mse_nvfp4(const float *x, int64_t rows, int64_t cols, int iters
         total += grp;
     }
     if (sse) *sse = total;
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Fixed grid scale for MX formats after rotation ("Bridging the Gap   */
+/* Between Promise and Performance for Microscaling FP4 Quantization", */
+/* MR-GPTQ modification 1: for MXFP4 with Hadamard rotations one fixed */
+/* grid scale serves every model).  Readings: the grid scale g in      */
+/* [1, 2] scales the block amax before the power-of-two exponent is    */
+/* taken: e = floor(log2(g amax)) - emax, computed exactly as           */
+/* floor(log2 amax) + [g m >= 2] - emax with m the significand of amax  */
+/* in [1, 2) (g = 1: the OCP rule; g = 4/3: the exponent rises exactly */
+/* when amax / 2^e would land in [6, 8), so E2M1 never clips; g and 2g */
+/* differ by one exponent step, so [1, 2] spans every such rule); the   */
+/* block is rotated first when hadamard_b > 0.  The                    */
+/* fit scores each candidate g by the squared error of the rotated     */
+/* tensor, sum (h - value(code) 2^e)^2 with the dequantized value exact */
+/* in binary64, summed in binary64 in element order within a block, in */
+/* block order within a row, over each group of 128 consecutive rows   */
+/* in row order, and over the groups in order; the caller keeps the    */
+/* least (a constant of the method, found once).                       */
+/* ------------------------------------------------------------------ */
+
+int orc_quantize_mx_grid(const float *x, int64_t rows, int64_t cols, int fmt, int hadamard_b, float g,
+                         float *work, uint8_t *codes, uint8_t *scales)
+{
+    if ((fmt != ORC_MXFP4 && fmt != ORC_MXFP8) || rows < 0 || cols < 0 || cols % 32) return ORC_EINVAL;
+    if (!(g >= 1.0f && g <= 2.0f)) return ORC_EINVAL;
+    if (!all_finite(x, rows * cols)) return ORC_EINVAL;
+    const float *src = x;
+    if (hadamard_b) {
+        if (orc_hadamard(x, work, rows, cols, hadamard_b) != ORC_OK) return ORC_EINVAL;
+        src = work;
+    }
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t c = 0; c < cols; c += 32)
+            quant_mx_block(src + r * cols + c, 32, fmt == ORC_MXFP4, g, codes, r * cols + c,
+                           scales + r * (cols / 32) + c / 32);
+    return ORC_OK;
+}
+
+int orc_mx_grid_sse(const float *x, int64_t rows, int64_t cols, int fmt, int hadamard_b, const float *gs, int n,
+                    float *work, uint8_t *codes, uint8_t *scales, double *sse)
+{
+    int fp4 = fmt == ORC_MXFP4;
+    for (int j = 0; j < n; j++) {
+        int st = orc_quantize_mx_grid(x, rows, cols, fmt, hadamard_b, gs[j], work, codes, scales);
+        if (st != ORC_OK) return st;
+        const float *h = hadamard_b ? work : x;
+        double total = 0.0;
+        for (int64_t g0 = 0; g0 < rows; g0 += ORC_MSE_GROUP) {
+            double grp = 0.0;
+            for (int64_t r = g0; r < rows && r < g0 + ORC_MSE_GROUP; r++) {
+                double row_err = 0.0;
+                for (int64_t b = 0; b < cols / 32; b++) {
+                    double scale = ldexp(1.0, (int)scales[r * (cols / 32) + b] - 127);
+                    double err = 0.0;
+                    for (int i = 0; i < 32; i++) {
+                        int64_t idx = r * cols + b * 32 + i;
+                        uint8_t c = fp4 ? (uint8_t)((codes[idx >> 1] >> (4 * (idx & 1))) & 0xF) : codes[idx];
+                        double w_hat = (fp4 ? orc_e2m1_value(c) : orc_e4m3_value(c)) * scale;
+                        double diff = (double)h[idx] - w_hat;
+                        err += diff * diff;
+                    }
+                    row_err += err;
+                }
+                grp += row_err;
+            }
+            total += grp;
+        }
+        sse[j] = total;
+    }
     return ORC_OK;
 }
 

@@ -585,6 +585,81 @@ def test_mse_nvfp4_rounds_lower_the_error(orc):
     assert errs[0] < usual and errs[2] <= errs[0]
 
 
+# ------------------------------------------------------------------ MX fixed grid scale
+
+@pytest.mark.parametrize("fmt_name", ["MXFP4", "MXFP8"])
+@pytest.mark.parametrize("hadamard_b", [0, 128])
+def test_mx_grid_one_is_the_ocp_rule(orc, fmt_name, hadamard_b):
+    fmt = getattr(orc, fmt_name)
+    rng = np.random.default_rng(41)
+    x = (rng.standard_t(3, size=(12, 256)) * 0.03).astype(np.float32)
+    q = orc.quantize_mx_grid(x, fmt, 1.0, hadamard_b)
+    u = orc.quantize(x, fmt, hadamard_b)
+    assert np.array_equal(q.codes, u.codes) and np.array_equal(q.scales, u.scales)
+
+
+def test_mx_grid_exponent_closed_form(orc):
+    # one nonzero element per 32-block with significand m and exponent k:
+    # e = k + [g m >= 2] - 2 (E2M1's largest exponent), scale byte e + 127
+    ms = [1.0, 1.25, 1.4999999, 1.5, 1.75, 1.9999999]
+    ks = [-3, 0, 5]
+    x = np.zeros((len(ks), 32 * len(ms)), np.float32)
+    for i, k in enumerate(ks):
+        for j, m in enumerate(ms):
+            x[i, 32 * j + 7] = np.float32(m) * np.float32(2.0 ** k)
+    for g in (1.0, 4.0 / 3.0, 1.125, 2.0):
+        q = orc.quantize_mx_grid(x, orc.MXFP4, g)
+        for i, k in enumerate(ks):
+            for j, m in enumerate(ms):
+                raise_ = float(np.float32(g)) * float(np.float32(m)) >= 2.0
+                assert q.scales[i, j] == k + int(raise_) - 2 + 127
+
+
+def test_mx_grid_four_thirds_never_clips(orc):
+    # g = 4/3: the scale is the least power of two with amax / 2^e < 6
+    rng = np.random.default_rng(42)
+    x = (rng.standard_t(2, size=(16, 512)) * 0.05).astype(np.float32)
+    q = orc.quantize_mx_grid(x, orc.MXFP4, 4.0 / 3.0)
+    amax = np.abs(x.astype(np.float64)).reshape(16, 16, 32).max(-1)
+    e = q.scales.astype(np.int64) - 127
+    assert np.all(amax / 2.0 ** e < 6) and np.all(amax / 2.0 ** (e - 1) >= 6)
+
+
+def test_mx_grid_sse_recomputed(orc):
+    rng = np.random.default_rng(43)
+    x = (rng.standard_t(4, size=(140, 256)) * 0.02).astype(np.float32)   # two 128-row groups
+    gs = [1.0, 1.125, 1.25, 1.5, 2.0]
+    for fmt, had in ((orc.MXFP4, 128), (orc.MXFP4, 0), (orc.MXFP8, 32)):
+        sse = orc.mx_grid_sse(x, fmt, gs, had)
+        h = orc.hadamard(x, had).astype(np.float64) if had else x.astype(np.float64)
+        for j, g in enumerate(gs):
+            deq = orc.quantize_mx_grid(x, fmt, g, had).dequantize()
+            assert sse[j] == pytest.approx(((h - deq) ** 2).sum(), rel=1e-12)
+
+
+def test_mx_grid_power_of_two_equivariance(orc):
+    rng = np.random.default_rng(44)
+    x = (rng.standard_t(3, size=(8, 128)) * 0.02).astype(np.float32)
+    gs = [1.0, 1.125, 4.0 / 3.0]
+    base = orc.mx_grid_sse(x, orc.MXFP4, gs, 32)
+    q = orc.quantize_mx_grid(x, orc.MXFP4, 1.125, 32)
+    for j in (4, -6):
+        xs = (x * np.float32(2.0 ** j)).astype(np.float32)
+        assert np.array_equal(orc.mx_grid_sse(xs, orc.MXFP4, gs, 32), base * 4.0 ** j)
+        qs = orc.quantize_mx_grid(xs, orc.MXFP4, 1.125, 32)
+        assert np.array_equal(qs.codes, q.codes)
+        assert np.array_equal(qs.scales.astype(np.int64), q.scales.astype(np.int64) + j)
+
+
+def test_mx_grid_fit_beats_ocp_after_rotation(orc):
+    # the page's claim (one fixed grid scale for rotated MXFP4) on heavy-tailed
+    # weights: some g > 1 lowers the error below the OCP rule -- a sanity check
+    rng = np.random.default_rng(45)
+    w = (rng.standard_t(4, size=(64, 512)) * 0.02).astype(np.float32)
+    sse = orc.mx_grid_sse(w, orc.MXFP4, [1.0, 1.0625, 1.125, 1.1875, 1.25], 128)
+    assert sse[1:].min() < sse[0]
+
+
 # ------------------------------------------------------------------ low rank + GEMM
 
 def test_lowrank_down_brute_force(orc):
