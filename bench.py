@@ -373,6 +373,19 @@ def run_ours(args, world, rank, local):
                "frac": mse_bytes / (mse_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                "sse_vs_usual_nvfp4": mse_sse.item() / usual_sse}
     del mse_ws, mse_q, w64
+    # MX fixed grid scale: squared error of workload 4's W after the 128-wide rotation for 8 grid scales
+    wg = torch.from_numpy(workloads.mxfp4_hadamard_gemm(m=1)["w"]).to(torch.bfloat16).to(dev)
+    grid = [1.0, 1.0625, 1.125, 1.25, 4.0 / 3.0, 1.5, 1.75, 2.0]
+    g_ws = torch.empty(mxq.fit_mx_grid_workspace_bytes(*wg.shape, len(grid)), dtype=torch.uint8, device=dev)
+    g_sse = torch.empty(len(grid), dtype=torch.float64, device=dev)
+    fit_ms = graph_ms(lambda i: mxq.fit_mx_grid(wg, mxq.MXFP4, grid, 128, workspace=g_ws, sse=g_sse), n=2, reps=3)
+    g_best, g_sse = mxq.fit_mx_grid(wg, mxq.MXFP4, grid, 128, workspace=g_ws, sse=g_sse)
+    grid_row = {"kernel": "k_mx_grid_err (MXFP4, 8 grid scales, Hadamard 128, binary64 errors) + ordered sums, "
+                          "W 4096 x 4096 bf16",
+                "us": 1e3 * fit_ms, "GB/s": wg.numel() * 2 / (fit_ms * 1e-3) / 1e9,
+                "frac": wg.numel() * 2 / (fit_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                "best_grid_scale": g_best, "sse_best_vs_ocp": g_sse.min().item() / g_sse[0].item()}
+    del wg, g_ws
     wq4 = mxq.quantize(w4d, mxq.INT4_G64, 0, mxq.MMA)
     del w4d
     xq4 = mxq.quantize(sets[0]["x"], mxq.INT4_G64, 0, mxq.MMA)
@@ -441,6 +454,7 @@ def run_ours(args, world, rank, local):
             "int4_g64_qlinear": int4,
             "select_weight_format": select,
             "quantize_mse_nvfp4": mse_row,
+            "fit_mx_grid": grid_row,
             "lowrank_down": lowrank,
             "e2e": {"value": world * FLOP_STEP / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "ms_per_step": e2e_ms},

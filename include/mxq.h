@@ -231,6 +231,40 @@ mxq_status mxq_quantize_mse(const void *w, int32_t wdtype, int64_t rows, int64_t
                             float *tensor_scale, double *sse, void *workspace,
                             size_t workspace_bytes, void *stream);
 
+/* MX quantization with a fixed grid scale ("Bridging the Gap Between
+ * Promise and Performance for Microscaling FP4 Quantization", MR-GPTQ
+ * modification 1: for MXFP4 with Hadamard rotations one fixed grid scale
+ * serves every model).  The grid scale g in [1, 2] scales the block amax
+ * before the power-of-two exponent is taken: e = floor(log2 amax) +
+ * [g m >= 2] - emax, m the significand of amax in [1, 2) (the product
+ * exact); g = 1 is mxq_quantize's OCP rule, g = 4/3 the rule under which
+ * E2M1 never clips.  Elements, scales and layouts as mxq_quantize.
+ *   fmt: MXQ_MXFP4 or MXQ_MXFP8 (others MXQ_EUNSUPPORTED); g outside [1, 2]:
+ *     MXQ_EINVAL.  Other arguments and constraints as mxq_quantize. */
+mxq_status mxq_quantize_mx_grid(const void *x, int32_t xdtype, int64_t rows, int64_t cols, int32_t fmt,
+                                int32_t hadamard_b, float grid_scale, int32_t layout, void *codes,
+                                void *scales, void *stream);
+
+/* Scratch bytes mxq_fit_mx_grid needs for n candidates:
+ * 256 + 8 * n * (rows * cols / 32) + 8 * rows + 8 * ceil(rows / 128). */
+mxq_status mxq_fit_mx_grid_workspace_bytes(int64_t rows, int64_t cols, int32_t n, size_t *bytes);
+
+/* Squared error of w (after the block-diagonal Hadamard rotation when
+ * hadamard_b > 0) under mxq_quantize_mx_grid with each candidate grid
+ * scale: sse[j] = sum (h - value(code) 2^e)^2 over the rotated tensor h, the
+ * dequantized value exact in binary64, summed in binary64 in element order
+ * within a block, in block order within a row, over each group of 128
+ * consecutive rows in row order and over the groups in order (bit-identical
+ * from run to run).  The least entry names the grid scale to fix.
+ *   grid_scales: host float[n], 1 <= n <= 8, each in [1, 2].
+ *   sse: device double[n].
+ *   workspace: device scratch of mxq_fit_mx_grid_workspace_bytes, 256-byte
+ *     aligned; clobbered.
+ * Other arguments and constraints as mxq_quantize_mx_grid. */
+mxq_status mxq_fit_mx_grid(const void *w, int32_t wdtype, int64_t rows, int64_t cols, int32_t fmt,
+                           int32_t hadamard_b, const float *grid_scales, int32_t n, double *sse,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
 /* ---------------------------------------------------------------------- */
 /* a5-a7: low-rank branch and block-scaled low-bit GEMM.                   */
 /* ---------------------------------------------------------------------- */

@@ -32,7 +32,8 @@ STATUS = {0: "MXQ_OK", 1: "MXQ_EINVAL", 2: "MXQ_EUNSUPPORTED", 3: "MXQ_ECUDA", 4
 EXPORTS = ("mxq_status_string", "mxq_last_cuda_error_string", "mxq_device_supported", "mxq_check", "mxq_codes_bytes", "mxq_scales_bytes",
            "mxq_quantize_workspace_bytes", "mxq_quantize", "mxq_dequantize", "mxq_hadamard_block", "mxq_cast",
            "mxq_select_workspace_bytes", "mxq_select_weight_format", "mxq_quantize_mse_workspace_bytes",
-           "mxq_quantize_mse", "mxq_lowrank_down", "mxq_lowrank_packed_bytes",
+           "mxq_quantize_mse", "mxq_quantize_mx_grid", "mxq_fit_mx_grid_workspace_bytes", "mxq_fit_mx_grid",
+           "mxq_lowrank_down", "mxq_lowrank_packed_bytes",
            "mxq_lowrank_down_packed", "mxq_lowrank_pack_t", "mxq_lowrank_pack_l2", "mxq_qlinear", "mxq_route",
            "mxq_quantize_lowrank_workspace_bytes", "mxq_quantize_lowrank", "mxq_quantize_lowrank_noalloc")
 
@@ -74,6 +75,9 @@ def _load():
         "mxq_select_weight_format": (i32, [P, i32, i64, i64, P, i32, P, P, P, sz, P]),
         "mxq_quantize_mse_workspace_bytes": (i32, [i64, i64, psz]),
         "mxq_quantize_mse": (i32, [P, i32, i64, i64, i32, i32, i32, P, P, P, P, P, sz, P]),
+        "mxq_quantize_mx_grid": (i32, [P, i32, i64, i64, i32, i32, ctypes.c_float, i32, P, P, P]),
+        "mxq_fit_mx_grid_workspace_bytes": (i32, [i64, i64, i32, psz]),
+        "mxq_fit_mx_grid": (i32, [P, i32, i64, i64, i32, i32, P, i32, P, P, sz, P]),
         "mxq_lowrank_down": (i32, [P, i32, i64, i64, P, i32, P, P]),
         "mxq_lowrank_packed_bytes": (i32, [i64, psz]),
         "mxq_lowrank_down_packed": (i32, [P, i32, i64, i64, P, i32, P, P, P, P]),
@@ -246,6 +250,39 @@ def quantize_mse(w: torch.Tensor, iters: int = 2, layout: int = CANONICAL, out: 
                               _ptr(q.scales), _ptr(q.tensor_scale), _ptr(sse), _ptr(ws), ws.numel(), _stream(stream)),
         "mxq_quantize_mse")
     return q, sse
+
+
+def quantize_mx_grid(x: torch.Tensor, fmt: int, grid_scale: float, hadamard_b: int = 0, layout: int = CANONICAL,
+                     out: QTensor = None, stream=None) -> QTensor:
+    """MXFP4 / MXFP8 with a fixed grid scale g in [1, 2] (g = 1: mxq_quantize)."""
+    _require_cuda(x)
+    x = x.contiguous()
+    rows, cols = x.shape
+    q = out if out is not None else alloc_qtensor(fmt, rows, cols, layout, x.device)
+    _ok(_lib.mxq_quantize_mx_grid(_ptr(x), _dtype_code(x), rows, cols, fmt, hadamard_b, float(grid_scale), layout,
+                                  _ptr(q.codes), _ptr(q.scales), _stream(stream)), "mxq_quantize_mx_grid")
+    return q
+
+
+def fit_mx_grid_workspace_bytes(rows: int, cols: int, n: int) -> int:
+    return _size(_lib.mxq_fit_mx_grid_workspace_bytes, rows, cols, n)
+
+
+def fit_mx_grid(w: torch.Tensor, fmt: int, grid_scales: Sequence[float], hadamard_b: int = 0,
+                workspace: torch.Tensor = None, sse: torch.Tensor = None, stream=None):
+    """Squared error of w under each candidate grid scale; returns (the
+    least-error grid scale, device float64 errors)."""
+    _require_cuda(w)
+    w = w.contiguous()
+    rows, cols = w.shape
+    n = len(grid_scales)
+    gs = (ctypes.c_float * n)(*grid_scales)
+    ws = workspace if workspace is not None else torch.empty(fit_mx_grid_workspace_bytes(rows, cols, n),
+                                                             dtype=torch.uint8, device=w.device)
+    sse = sse if sse is not None else torch.empty(n, dtype=torch.float64, device=w.device)
+    _ok(_lib.mxq_fit_mx_grid(_ptr(w), _dtype_code(w), rows, cols, fmt, hadamard_b, gs, n, _ptr(sse), _ptr(ws),
+                             ws.numel(), _stream(stream)), "mxq_fit_mx_grid")
+    return None if torch.cuda.is_current_stream_capturing() else grid_scales[int(torch.argmin(sse).item())], sse
 
 
 def lowrank_down(x: torch.Tensor, l1: torch.Tensor, out: torch.Tensor = None, stream=None) -> torch.Tensor:

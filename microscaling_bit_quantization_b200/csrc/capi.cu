@@ -200,6 +200,48 @@ mxq_status mxq_quantize_mse(const void *w, int32_t wdtype, int64_t rows, int64_t
                                          tensor_scale, sse, workspace, (cudaStream_t)stream));
 }
 
+static bool valid_grid(float g) { return g >= 1.0f && g <= 2.0f; }
+
+mxq_status mxq_quantize_mx_grid(const void *x, int32_t xdtype, int64_t rows, int64_t cols, int32_t fmt,
+                                int32_t hadamard_b, float grid_scale, int32_t layout, void *codes, void *scales,
+                                void *stream) {
+    if (!valid_fmt(fmt) || !valid_dtype(xdtype) || !valid_layout(layout)) return MXQ_EINVAL;
+    if (fmt != MXQ_MXFP4 && fmt != MXQ_MXFP8) return MXQ_EUNSUPPORTED;
+    if (!valid_shape(fmt, rows, cols) || !valid_hadamard(hadamard_b, cols) || !valid_grid(grid_scale))
+        return MXQ_EINVAL;
+    const int64_t n = rows * cols;
+    if (n > 0 && (!x || !codes || !scales || !aligned16(x) || !aligned16(codes))) return MXQ_EINVAL;
+    size_t sb = 0;
+    mxq_scales_bytes(fmt, rows, cols, layout, &sb);
+    return from_cuda(launch_quantize(x, xdtype == MXQ_BF16, rows, cols, fmt, hadamard_b, layout, codes, scales, sb,
+                                     nullptr, nullptr, (cudaStream_t)stream, nullptr, false, grid_scale));
+}
+
+mxq_status mxq_fit_mx_grid_workspace_bytes(int64_t rows, int64_t cols, int32_t n, size_t *bytes) {
+    if (rows < 0 || cols < 0 || cols % 32 || n < 1 || n > kMaxCandidates || !bytes) return MXQ_EINVAL;
+    *bytes = mx_grid_workspace_bytes(rows, cols, n);
+    return MXQ_OK;
+}
+
+mxq_status mxq_fit_mx_grid(const void *w, int32_t wdtype, int64_t rows, int64_t cols, int32_t fmt,
+                           int32_t hadamard_b, const float *grid_scales, int32_t n, double *sse, void *workspace,
+                           size_t workspace_bytes, void *stream) {
+    if (!valid_fmt(fmt) || !valid_dtype(wdtype)) return MXQ_EINVAL;
+    if (fmt != MXQ_MXFP4 && fmt != MXQ_MXFP8) return MXQ_EUNSUPPORTED;
+    if (!valid_shape(fmt, rows, cols) || !valid_hadamard(hadamard_b, cols)) return MXQ_EINVAL;
+    if (n < 1 || n > kMaxCandidates || !grid_scales || !sse) return MXQ_EINVAL;
+    for (int j = 0; j < n; j++)
+        if (!valid_grid(grid_scales[j])) return MXQ_EINVAL;
+    if (rows * cols > 0 && (!w || !aligned16(w))) return MXQ_EINVAL;
+    size_t need = 0;
+    mxq_fit_mx_grid_workspace_bytes(rows, cols, n, &need);
+    if (!workspace) return MXQ_EINVAL;
+    if (workspace_bytes < need) return MXQ_ENOSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MXQ_EINVAL;
+    return from_cuda(launch_fit_mx_grid(w, wdtype == MXQ_BF16, rows, cols, fmt, hadamard_b, grid_scales, n, sse,
+                                        workspace, (cudaStream_t)stream));
+}
+
 mxq_status mxq_lowrank_down(const void *x, int32_t xdtype, int64_t m, int64_t k, const void *l1, int32_t r, float *t,
                             void *stream) {
     if (!valid_dtype(xdtype) || m < 0 || k <= 0 || k % 16 || r < 1 || r > 32) return MXQ_EINVAL;

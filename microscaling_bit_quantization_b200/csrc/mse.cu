@@ -210,10 +210,133 @@ cudaError_t run_mse(const T *x, const MseArgs &base, int iters, double *row_sums
     return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Fixed grid scale for MX formats ("Bridging the Gap ...", MR-GPTQ
+// modification 1: for MXFP4 with Hadamard rotations one fixed grid scale
+// serves every model).  The fit scores candidate grid scales g in [1, 2]
+// (mx_scale_grid) by the squared error of the rotated tensor, the
+// dequantized value exact in binary64, summed in element order within a
+// block, then rows, groups of kMseGroup rows and groups as above.
+
+struct MxFitArgs {
+    int64_t rows, cols, chunks;   // chunks = rows * cols / 16 < 2^31
+    int hadamard_b;
+    int n;                        // candidate grid scales
+    float g[kMaxCandidates];
+    double *blk;                  // [n][chunks / 2] block errors
+};
+
+// Signed E4M3 element code -> value.
+__device__ __forceinline__ double e4m3_value_f64(uint32_t code) {
+    const double mag = (double)dec_e4m3(code & 0x7Fu);
+    return (code & 0x80u) ? -mag : mag;
+}
+
+// One lane per 16-element chunk, 32 consecutive chunks per warp (a 32-element
+// MX block is two lanes; a Hadamard block of b <= 256 elements lies in one
+// warp).  Per grid scale: the block's scale and codes as the quantizer makes
+// them, each lane's 16 squared differences, then the block's sum in element
+// order: the first lane of the pair adds its terms and hands the sum to the
+// second, which adds its own and stores the block error.
+template <typename T, bool FP4>
+__global__ void __launch_bounds__(kMseThreads) k_mx_grid_err(const T *__restrict__ x, MxFitArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int64_t c = (int64_t)blockIdx.x * kMseThreads + threadIdx.x;
+    const bool valid = c < a.chunks;
+    float v[16];
+    if (valid) load16(x + c * 16, v);
+    else {
+#pragma unroll
+        for (int i = 0; i < 16; i++) v[i] = 0.0f;
+    }
+    if (a.hadamard_b) hadamard_chunk(v, a.hadamard_b, lane);
+    double vd[16];
+#pragma unroll
+    for (int i = 0; i < 16; i++) vd[i] = (double)v[i];
+    const float amax = group_max<2>(amax16(v));
+    const int64_t blocks = a.chunks >> 1;
+#pragma unroll 1
+    for (int j = 0; j < a.n; j++) {
+        float inv = 0.0f;
+        uint32_t sb = 127;
+        if (amax > 0.0f) sb = mx_scale_grid(amax, FP4 ? 2 : 8, a.g[j], inv);
+        const double sc = exp2i_f64((int)sb - 127);
+        float u[16];
+        mul8(v, inv, u);
+        mul8(v + 8, inv, u + 8);
+        double t[16];
+        if (FP4) {
+            const uint32_t w0 = cvt_e2m1x8(u[0], u[1], u[2], u[3], u[4], u[5], u[6], u[7]);
+            const uint32_t w1 = cvt_e2m1x8(u[8], u[9], u[10], u[11], u[12], u[13], u[14], u[15]);
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                const uint32_t code = ((i < 8 ? w0 : w1) >> (4 * (i & 7))) & 0xFu;
+                const double d = __dsub_rn(vd[i], __dmul_rn(e2m1_value_f64(code), sc));
+                t[i] = __dmul_rn(d, d);
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+                const uint32_t w = cvt_e4m3x4(u[4 * q], u[4 * q + 1], u[4 * q + 2], u[4 * q + 3]);
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    const double d = __dsub_rn(vd[4 * q + i], __dmul_rn(e4m3_value_f64((w >> (8 * i)) & 0xFFu), sc));
+                    t[4 * q + i] = __dmul_rn(d, d);
+                }
+            }
+        }
+        double acc = 0.0;
+        if (!(lane & 1)) {
+#pragma unroll
+            for (int i = 0; i < 16; i++) acc = __dadd_rn(acc, t[i]);
+        }
+        const double first = __shfl_up_sync(0xFFFFFFFFu, acc, 1);
+        if ((lane & 1) && valid) {
+            acc = first;
+#pragma unroll
+            for (int i = 0; i < 16; i++) acc = __dadd_rn(acc, t[i]);
+            a.blk[j * blocks + (c >> 1)] = acc;
+        }
+    }
+}
+
+template <typename T>
+void launch_mx_grid_err(const T *x, int fmt, const MxFitArgs &a, cudaStream_t s) {
+    const int grid = (int)((a.chunks + kMseThreads - 1) / kMseThreads);
+    if (fmt == kMXFP4) k_mx_grid_err<T, true><<<grid, kMseThreads, 0, s>>>(x, a);
+    else k_mx_grid_err<T, false><<<grid, kMseThreads, 0, s>>>(x, a);
+}
+
 }  // namespace
 
 size_t mse_workspace_bytes(int64_t rows, int64_t cols) {
     return 256 + (size_t)(rows * (cols / 16)) * 16 + (size_t)rows * 16 + (size_t)((rows + kMseGroup - 1) / kMseGroup) * 16;
+}
+
+size_t mx_grid_workspace_bytes(int64_t rows, int64_t cols, int n) {
+    return 256 + (size_t)n * (size_t)(rows * (cols / 32)) * 8 + (size_t)rows * 8 +
+           (size_t)((rows + kMseGroup - 1) / kMseGroup) * 8;
+}
+
+cudaError_t launch_fit_mx_grid(const void *w, bool bf16, int64_t rows, int64_t cols, int fmt, int hadamard_b,
+                               const float *grid_scales, int n, double *sse, void *workspace, cudaStream_t s) {
+    if (rows == 0 || cols == 0) return cudaMemsetAsync(sse, 0, sizeof(double) * n, s);
+    MxFitArgs a;
+    a.rows = rows;
+    a.cols = cols;
+    a.chunks = rows * (cols / 16);
+    a.hadamard_b = hadamard_b;
+    a.n = n;
+    for (int j = 0; j < kMaxCandidates; j++) a.g[j] = j < n ? grid_scales[j] : 1.0f;
+    a.blk = (double *)((char *)workspace + 256);
+    const int64_t blocks = a.chunks / 2;
+    double *row_sums = a.blk + (int64_t)n * blocks;
+    double *grp_sums = row_sums + rows;
+    if (bf16) launch_mx_grid_err((const __nv_bfloat16 *)w, fmt, a, s);
+    else launch_mx_grid_err((const float *)w, fmt, a, s);
+    for (int j = 0; j < n; j++)
+        launch_sums<1>(a.blk + (int64_t)j * blocks, blocks, cols / 32, rows, row_sums, grp_sums, nullptr, sse + j, s);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_quantize_mse(const void *w, bool bf16, int64_t rows, int64_t cols, int iters, int layout,

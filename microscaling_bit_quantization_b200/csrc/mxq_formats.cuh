@@ -123,6 +123,20 @@ __device__ __forceinline__ uint32_t mx_scale(float amax, int emax_elem, float &i
     return (uint32_t)(e + 127);
 }
 
+// MX shared scale with a fixed grid scale g in [1, 2] ("Bridging the Gap
+// ...", MR-GPTQ modification 1: one fixed grid scale for rotated MXFP4): the
+// exponent of g * amax, e = floor(log2 amax) + [g m >= 2] - emax_elem with m
+// the significand of amax in [1, 2), the product exact in binary64; g = 1
+// gives mx_scale.  amax must be > 0.
+__device__ __forceinline__ uint32_t mx_scale_grid(float amax, int emax_elem, float g, float &inv) {
+    const int fl = floor_log2_pos(amax);
+    const double m = __dmul_rn((double)amax, exp2i_f64(-fl));   // exact
+    int e = fl + (__dmul_rn((double)g, m) >= 2.0 ? 1 : 0) - emax_elem;
+    e = e < -127 ? -127 : (e > 127 ? 127 : e);
+    inv = exp2i_f32(-e);
+    return (uint32_t)(e + 127);
+}
+
 // NVFP4 tensor scale s_t = RN(amax_T / (6 * 448)); 1 when that is 0.
 __device__ __forceinline__ float nvfp4_tensor_scale(float amax_t) {
     float s = __fdiv_rn(amax_t, 2688.0f);

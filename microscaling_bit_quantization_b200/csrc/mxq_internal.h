@@ -26,7 +26,12 @@ struct PackT {
 cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols, int fmt, int hadamard_b,
                             int layout, void *codes, void *scales, size_t scales_bytes, float *tensor_scale,
                             unsigned int *amax_word, cudaStream_t s, const PackT *pack = nullptr,
-                            bool amax_ready = false);
+                            bool amax_ready = false, float mx_grid = 1.0f);
+// Squared error of the (rotated) tensor under MX quantization with each of
+// n <= kMaxCandidates grid scales (mse.cu); sse: device double[n].
+size_t mx_grid_workspace_bytes(int64_t rows, int64_t cols, int n);
+cudaError_t launch_fit_mx_grid(const void *w, bool bf16, int64_t rows, int64_t cols, int fmt, int hadamard_b,
+                               const float *grid_scales, int n, double *sse, void *workspace, cudaStream_t s);
 // NVFP4 with block and tensor scales fitted to the squared error (mse.cu);
 // workspace of mse_workspace_bytes, 256-byte aligned.
 size_t mse_workspace_bytes(int64_t rows, int64_t cols);

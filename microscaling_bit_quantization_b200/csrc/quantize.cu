@@ -59,6 +59,7 @@ struct QuantArgs {
     void *scales;
     float *tensor_scale;     // written by chunk 0 (NVFP4, FP8_TENSOR)
     const unsigned int *amax_word;
+    float mx_grid;           // MX grid scale g in [1, 2] (1: the OCP rule)
     // optional packed low-rank operand: tp[row] = [hi | lo] of t[row] / (s_x * *w_ts)
     const float *t;
     int r;
@@ -118,7 +119,9 @@ __device__ __forceinline__ void encode_chunk(const float (&v)[16], float amax, u
     if (F == kMXFP8 || F == kMXFP4) {
         float inv = 0.0f;
         uint32_t sb = 127;
-        if (amax > 0.0f) sb = mx_scale(amax, F == kMXFP8 ? 8 : 2, inv);
+        if (amax > 0.0f)
+            sb = a.mx_grid == 1.0f ? mx_scale(amax, F == kMXFP8 ? 8 : 2, inv)
+                                   : mx_scale_grid(amax, F == kMXFP8 ? 8 : 2, a.mx_grid, inv);
         if (!valid) return;
         // inv is a power of two: v * inv is exact (or far below the smallest code)
         float u[16];
@@ -649,7 +652,8 @@ static void launch_q(int fmt, int grid, const T *x, const QuantArgs &a, cudaStre
 
 cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols, int fmt, int hadamard_b,
                             int layout, void *codes, void *scales, size_t scales_bytes, float *tensor_scale,
-                            unsigned int *amax_word, cudaStream_t s, const PackT *pack, bool amax_ready) {
+                            unsigned int *amax_word, cudaStream_t s, const PackT *pack, bool amax_ready,
+                            float mx_grid) {
     cudaError_t e;
     if (fmt_tensor_scaled(fmt) && !amax_ready) {
         e = launch_amax(x, bf16, rows, cols, hadamard_b, amax_word, s);
@@ -667,6 +671,7 @@ cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols
     a.scales = scales;
     a.tensor_scale = tensor_scale;
     a.amax_word = amax_word;
+    a.mx_grid = mx_grid;
     a.t = pack ? pack->t : nullptr;
     a.r = pack ? pack->r : 0;
     a.w_ts = pack ? pack->w_ts : nullptr;

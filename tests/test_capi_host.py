@@ -97,6 +97,28 @@ def test_quantize_mse_argument_checks(mxq):
     assert call(ws=P(256 + 8)) == 1          # workspace not 256-byte aligned
 
 
+def test_mx_grid_argument_checks(mxq):
+    L, P = mxq.lib(), ctypes.c_void_p
+    size = ctypes.c_size_t(0)
+    assert L.mxq_fit_mx_grid_workspace_bytes(300, 64, 3, ctypes.byref(size)) == 0
+    assert size.value == 256 + 8 * 3 * 600 + 8 * 300 + 8 * 3
+    assert L.mxq_fit_mx_grid_workspace_bytes(4, 48, 1, ctypes.byref(size)) == 1     # 48 % 32
+    assert L.mxq_fit_mx_grid_workspace_bytes(4, 64, 9, ctypes.byref(size)) == 1     # more than 8 candidates
+    d = P(256)
+    q = L.mxq_quantize_mx_grid
+    assert q(d, 1, 4, 64, mxq.NVFP4, 0, ctypes.c_float(1.0), 0, d, d, None) == 2   # MX formats only
+    assert q(d, 1, 4, 64, mxq.MXFP4, 0, ctypes.c_float(0.75), 0, d, d, None) == 1  # g outside [1, 2]
+    assert q(d, 1, 4, 64, mxq.MXFP4, 0, ctypes.c_float(2.5), 0, d, d, None) == 1
+    assert q(d, 1, 4, 64, mxq.MXFP4, 48, ctypes.c_float(1.0), 0, d, d, None) == 1  # bad Hadamard size
+    gs = (ctypes.c_float * 2)(1.0, 3.0)
+    fit = L.mxq_fit_mx_grid
+    assert fit(d, 1, 4, 64, mxq.MXFP4, 0, gs, 2, d, d, 1 << 20, None) == 1         # 3.0 outside [1, 2]
+    gs[1] = 1.5
+    assert fit(d, 1, 4, 64, mxq.MXFP4, 0, gs, 0, d, d, 1 << 20, None) == 1         # no candidates
+    assert fit(d, 1, 4, 64, mxq.MXFP4, 0, gs, 2, d, d, 16, None) == 5              # workspace too small
+    assert fit(d, 1, 4, 64, mxq.INT4_G32, 0, gs, 2, d, d, 1 << 20, None) == 2
+
+
 def test_qlinear_argument_checks(mxq):
     L = mxq.lib()
     Q = mxq._QTensorC

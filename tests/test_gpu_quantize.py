@@ -261,3 +261,58 @@ def test_quantize_mse_full_size(mxq, orc):
     u = mxq.quantize(wd, mxq.NVFP4)
     usual = ((mxq.dequantize(u, torch.float32).double() - wt) ** 2).sum().item()
     assert sse.item() < usual
+
+
+# ------------------------------------------------------------------ MX fixed grid scale
+
+GRID = [1.0, 1.0625, 1.125, 1.25, 4.0 / 3.0, 1.5, 1.75, 2.0]
+
+
+@pytest.mark.parametrize("fmt", [1, 0])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("hadamard_b", [0, 32, 128])
+def test_mx_grid_small(mxq, orc, fmt, dtype, hadamard_b):
+    rows, cols = 37, 512
+    x = nasty_matrix(400 + fmt, rows, cols)
+    if hadamard_b:
+        x = _moderate(x)
+    xv = host_values(x, dtype)
+    for g in (1.0, 1.125, 4.0 / 3.0, 2.0):
+        ref = orc.quantize_mx_grid(xv, fmt, g, hadamard_b)
+        for layout in (mxq.CANONICAL, mxq.MMA):
+            q = mxq.quantize_mx_grid(dev(x, dtype), fmt, g, hadamard_b, layout)
+            torch.cuda.synchronize()
+            assert_qtensor_equal(q, ref, layout_mma=layout == mxq.MMA)
+    best, sse = mxq.fit_mx_grid(dev(x, dtype), fmt, GRID, hadamard_b)
+    ref_sse = orc.mx_grid_sse(xv, fmt, GRID, hadamard_b)
+    np.testing.assert_array_equal(sse.cpu().numpy(), ref_sse)
+    assert best == GRID[int(np.argmin(ref_sse))]
+
+
+def test_mx_grid_fit_ragged_groups(mxq, orc):
+    # 300 rows: three row groups, the last one ragged; 1 and 8 candidates
+    x = nasty_matrix(12, 300, 96)
+    for gs in ([1.125], GRID):
+        _, sse = mxq.fit_mx_grid(dev(x, "f32"), mxq.MXFP4, gs, 32)
+        np.testing.assert_array_equal(sse.cpu().numpy(), orc.mx_grid_sse(x, mxq.MXFP4, gs, 32))
+    _, sse = mxq.fit_mx_grid(torch.empty((0, 64), device="cuda"), mxq.MXFP4, GRID[:2])
+    assert sse.cpu().tolist() == [0.0, 0.0]
+
+
+def test_mx_grid_full_size(mxq, orc):
+    """Workload 4's weight W (4096 x 4096 bf16) after the 128-wide rotation:
+    run-to-run identity, the g = 1 error against the usual quantizer's
+    dequantized result, and a fitted grid scale at least as good as g = 1."""
+    w = workloads.mxfp4_hadamard_gemm()["w"]
+    wd = dev(w, "bf16")
+    best, sse = mxq.fit_mx_grid(wd, mxq.MXFP4, GRID, 128)
+    _, sse2 = mxq.fit_mx_grid(wd, mxq.MXFP4, GRID, 128)
+    torch.cuda.synchronize()
+    assert torch.equal(sse, sse2)
+    h = mxq.hadamard_block(wd.float(), 128).double()
+    deq = mxq.dequantize(mxq.quantize(wd, mxq.MXFP4, 128), torch.float32).double()
+    assert sse[0].item() == pytest.approx(((h - deq) ** 2).sum().item(), rel=1e-9)
+    assert sse.min().item() <= sse[0].item() and best == GRID[int(torch.argmin(sse).item())]
+    q = mxq.quantize_mx_grid(wd, mxq.MXFP4, best, 128, mxq.MMA)
+    u = mxq.quantize(wd, mxq.MXFP4, 128, mxq.MMA)
+    assert torch.equal(q.codes, u.codes) == (best == 1.0)
