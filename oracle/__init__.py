@@ -91,6 +91,8 @@ def lib():
         L.orc_quantize_mx_grid.argtypes = [P, i64, i64, i32, i32, ctypes.c_float, P, P, P]
         L.orc_mx_grid_sse.restype = i32
         L.orc_mx_grid_sse.argtypes = [P, i64, i64, i32, i32, P, i32, P, P, P, P]
+        L.orc_calibrate_activation.restype = i32
+        L.orc_calibrate_activation.argtypes = [P, i64, i64, P, i32, P, P, P, P, P, P, P]
         L.orc_lowrank_down.restype = i32
         L.orc_lowrank_down.argtypes = [P, P, i64, i64, i32, P]
         L.orc_route.restype = i32
@@ -305,6 +307,35 @@ def mx_grid_sse(x, fmt: int, grid_scales, hadamard_b: int = 0) -> np.ndarray:
     if st != 0:
         raise OracleError("bad mx_grid_sse arguments")
     return sse
+
+
+# ---------------------------------------------------------------- activation-format calibration
+
+def calibrate_activation(x, candidates, sse_accum: np.ndarray, moments_accum: np.ndarray):
+    """Adds x's per-candidate squared error and (sum x^2, sum x^4) to the
+    accumulators (mxq_oracle.c, orc_calibrate_activation)."""
+    x = _f32(x)
+    n, k = x.shape
+    cands = np.ascontiguousarray(np.asarray(candidates, dtype=np.int32))
+    codes = np.empty(max(n * k, 1), np.uint8)
+    scales = np.empty(max(n * k * 4, 1), np.uint8)
+    deq = np.empty(max(n * k, 1), np.float64)
+    choice = np.empty(max(n, 1), np.uint8)
+    sse_rows = np.empty(max(n * len(cands), 1), np.float64)
+    assert sse_accum.dtype == np.float64 and moments_accum.dtype == np.float64
+    st = lib().orc_calibrate_activation(_ptr(x), n, k, _ptr(cands), len(cands), _ptr(codes), _ptr(scales),
+                                        _ptr(deq), _ptr(choice), _ptr(sse_rows), _ptr(sse_accum),
+                                        _ptr(moments_accum))
+    if st != 0:
+        raise OracleError("bad calibrate_activation arguments")
+
+
+def calibrate_pick(sse_accum, candidates, forced_fmt: int = -1) -> int:
+    """Table entry: forced_fmt if >= 0, else the candidate with the least
+    accumulated error (ties to the lower candidate index)."""
+    if forced_fmt >= 0:
+        return forced_fmt
+    return int(candidates[int(np.argmin(np.asarray(sse_accum)))])
 
 
 # ---------------------------------------------------------------- low rank + GEMM

@@ -723,6 +723,64 @@ int orc_mx_grid_sse(const float *x, int64_t rows, int64_t cols, int fmt, int had
 }
 
 /* ------------------------------------------------------------------ */
+/* Activation-format calibration (Chameleon article, section "the      */
+/* format is chosen by the value distribution": per layer and per      */
+/* interval of the trajectory, activations are calibrated in advance   */
+/* into the table read at generation time).  The page gives no         */
+/* decision rule; the reading mirrors its rule for weights: an entry   */
+/* takes the candidate with the least squared quantization error       */
+/* accumulated over its calibration activations (orc_select's per-row  */
+/* errors, rows summed over each group of 128 consecutive rows in      */
+/* order, then the groups in order, then added to the accumulator);   */
+/* the tail moments sum x^2 and sum x^4 are accumulated beside it      */
+/* (binary64, element order within 16-element chunks, chunks in order  */
+/* within a row, rows and groups as above).                            */
+/* ------------------------------------------------------------------ */
+
+int orc_calibrate_activation(const float *x, int64_t rows, int64_t cols, const int *cands, int ncand,
+                             uint8_t *codes_work, void *scales_work, double *deq_work, uint8_t *choice_work,
+                             double *sse_rows, double *sse_accum, double *moments_accum)
+{
+    if (rows < 0 || cols < 0 || cols % 16) return ORC_EINVAL;
+    if (rows == 0 || cols == 0) return ORC_OK;
+    int st = orc_select(x, rows, cols, cands, ncand, codes_work, scales_work, deq_work, choice_work, sse_rows);
+    if (st != ORC_OK) return st;
+    for (int j = 0; j < ncand; j++) {
+        double total = 0.0;
+        for (int64_t g0 = 0; g0 < rows; g0 += ORC_MSE_GROUP) {
+            double grp = 0.0;
+            for (int64_t r = g0; r < rows && r < g0 + ORC_MSE_GROUP; r++) grp += sse_rows[r * ncand + j];
+            total += grp;
+        }
+        sse_accum[j] += total;
+    }
+    double t2 = 0.0, t4 = 0.0;
+    for (int64_t g0 = 0; g0 < rows; g0 += ORC_MSE_GROUP) {
+        double g2 = 0.0, g4 = 0.0;
+        for (int64_t r = g0; r < rows && r < g0 + ORC_MSE_GROUP; r++) {
+            double r2 = 0.0, r4 = 0.0;
+            for (int64_t c = 0; c < cols; c += 16) {
+                double c2 = 0.0, c4 = 0.0;
+                for (int i = 0; i < 16; i++) {
+                    double q = (double)x[r * cols + c + i] * (double)x[r * cols + c + i];
+                    c2 += q;
+                    c4 += q * q;
+                }
+                r2 += c2;
+                r4 += c4;
+            }
+            g2 += r2;
+            g4 += r4;
+        }
+        t2 += g2;
+        t4 += g4;
+    }
+    moments_accum[0] += t2;
+    moments_accum[1] += t4;
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
 /* SVDQuant low-rank branch, down projection (Nunchaku/Diffusers       */
 /* article, section "Main explanation": a 16-bit low-rank part of the  */
 /* weight is kept beside the 4-bit residual).                          */

@@ -660,6 +660,52 @@ def test_mx_grid_fit_beats_ocp_after_rotation(orc):
     assert sse[1:].min() < sse[0]
 
 
+# ------------------------------------------------------------------ activation-format calibration
+
+def test_calibration_errors_are_selection_row_sums(orc):
+    rng = np.random.default_rng(51)
+    cands = [orc.INT8_ROW, orc.FP8_TENSOR, orc.MXFP8]
+    xs = [(rng.standard_t(nu, size=(150, 128))).astype(np.float32) for nu in (2.5, 30.0)]
+    sse = np.zeros(3)
+    mom = np.zeros(2)
+    totals = []
+    for x in xs:
+        _, rows = orc.select_weight_format(x, cands)
+        totals.append(rows.sum(0))
+        before = sse.copy()
+        orc.calibrate_activation(x, cands, sse, mom)
+        np.testing.assert_allclose(sse - before, totals[-1], rtol=1e-12)
+    np.testing.assert_allclose(sse, totals[0] + totals[1], rtol=1e-12)
+
+
+def test_calibration_moments_exact(orc):
+    # dyadic values k/4 (|k| <= 40): every partial sum is exact, so the
+    # accumulated moments equal the integer sums
+    rng = np.random.default_rng(52)
+    k = rng.integers(-40, 41, size=(260, 64))
+    x = (k / 4.0).astype(np.float32)
+    mom = np.zeros(2)
+    orc.calibrate_activation(x, [orc.MXFP8], np.zeros(1), mom)
+    k2 = int((k.astype(object) ** 2).sum())
+    k4 = int((k.astype(object) ** 4).sum())
+    assert mom[0] == k2 / 16.0 and mom[1] == k4 / 256.0
+
+
+def test_calibration_pick_is_least_recomputed_error(orc):
+    # heavy tails vs near-Gaussian activations: the entry is the candidate
+    # whose quantize/dequantize error is least (recomputed independently)
+    rng = np.random.default_rng(53)
+    cands = [orc.INT8_ROW, orc.FP8_TENSOR, orc.MXFP8, orc.MXFP4]
+    for nu in (1.5, 3.0, 50.0):
+        x = rng.standard_t(nu, size=(96, 256)).astype(np.float32)
+        x[:, :4] *= 40.0   # outlier channels
+        sse = np.zeros(len(cands))
+        orc.calibrate_activation(x, cands, sse, np.zeros(2))
+        ref = [((orc.quantize(x, f).dequantize() - x.astype(np.float64)) ** 2).sum() for f in cands]
+        assert orc.calibrate_pick(sse, cands) == cands[int(np.argmin(ref))]
+        assert orc.calibrate_pick(sse, cands, orc.MXFP8) == orc.MXFP8
+
+
 # ------------------------------------------------------------------ low rank + GEMM
 
 def test_lowrank_down_brute_force(orc):
