@@ -386,6 +386,18 @@ def run_ours(args, world, rank, local):
                 "frac": wg.numel() * 2 / (fit_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                 "best_grid_scale": g_best, "sse_best_vs_ocp": g_sse.min().item() / g_sse[0].item()}
     del wg, g_ws
+    # activation-format calibration: workload 5's fc1 input at step 0 against {INT8 row, FP8 tensor, MXFP8}
+    xc = torch.from_numpy(workloads.dit_activation(5, 0, 1152)).to(torch.bfloat16).to(dev)
+    calib = [mxq.INT8_ROW, mxq.FP8_TENSOR, mxq.MXFP8]
+    c_ws = torch.empty(mxq.calibrate_workspace_bytes(*xc.shape, len(calib)), dtype=torch.uint8, device=dev)
+    c_sse = torch.zeros(len(calib), dtype=torch.float64, device=dev)
+    c_mom = torch.zeros(2, dtype=torch.float64, device=dev)
+    cal_ms = graph_ms(lambda i: mxq.calibrate_activation(xc, calib, c_sse, c_mom, workspace=c_ws), n=4, reps=3)
+    calib_row = {"kernel": "k_select (3 candidates, per-row binary64 errors) + k_moments + ordered sums, "
+                           "X 8192 x 1152 bf16",
+                 "us": 1e3 * cal_ms, "GB/s": xc.numel() * 2 / (cal_ms * 1e-3) / 1e9,
+                 "frac": xc.numel() * 2 / (cal_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    del xc, c_ws
     wq4 = mxq.quantize(w4d, mxq.INT4_G64, 0, mxq.MMA)
     del w4d
     xq4 = mxq.quantize(sets[0]["x"], mxq.INT4_G64, 0, mxq.MMA)
@@ -455,6 +467,7 @@ def run_ours(args, world, rank, local):
             "select_weight_format": select,
             "quantize_mse_nvfp4": mse_row,
             "fit_mx_grid": grid_row,
+            "calibrate_activation": calib_row,
             "lowrank_down": lowrank,
             "e2e": {"value": world * FLOP_STEP / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "ms_per_step": e2e_ms},

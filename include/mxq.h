@@ -265,6 +265,39 @@ mxq_status mxq_fit_mx_grid(const void *w, int32_t wdtype, int64_t rows, int64_t 
                            int32_t hadamard_b, const float *grid_scales, int32_t n, double *sse,
                            void *workspace, size_t workspace_bytes, void *stream);
 
+/* Activation-format calibration (Chameleon article, section "the format is
+ * chosen by the value distribution": the trajectory is cut into ten
+ * intervals, activations are calibrated in advance and the per-layer,
+ * per-interval result is the table mxq_route reads).  The page gives no
+ * decision rule; this library's reading mirrors its rule for weights: an
+ * entry takes the candidate with the least squared quantization error
+ * accumulated over the calibration activations of its layer and interval,
+ * and the tail moments are accumulated beside it (excess kurtosis
+ * n * sum x^4 / (sum x^2)^2 - 3 over n elements).
+ *
+ * mxq_calibrate_activation adds, for one calibration activation x
+ * (rows x cols fp32/bf16, device): to sse_accum[j] (device double[ncand])
+ * the squared error of x under candidate j as mxq_select_weight_format
+ * measures it per row, the rows summed in binary64 over each group of 128
+ * consecutive rows in order and then over the groups in order; to
+ * moments_accum[0..1] (device double[2]) sum x^2 and sum x^4 in binary64
+ * (element order within 16-element chunks, then chunks, rows, groups as
+ * above).  Zero the accumulators before an entry's first activation.
+ *   candidates: host array of 1..8 mxq_fmt values; cols % 64 == 0.
+ *   workspace: device scratch of mxq_calibrate_workspace_bytes, 256-byte
+ *     aligned; clobbered. */
+mxq_status mxq_calibrate_workspace_bytes(int64_t rows, int64_t cols, int32_t ncand, size_t *bytes);
+mxq_status mxq_calibrate_activation(const void *x, int32_t xdtype, int64_t rows, int64_t cols,
+                                    const int32_t *candidates, int32_t ncand, double *sse_accum,
+                                    double *moments_accum, void *workspace, size_t workspace_bytes,
+                                    void *stream);
+
+/* Writes one table entry (device uint8): forced_fmt when >= 0 (layers the
+ * article pins to MXFP8), else the candidate with the least sse_accum
+ * (device double[ncand]), ties to the lower candidate index. */
+mxq_status mxq_calibrate_pick(const double *sse_accum, const int32_t *candidates, int32_t ncand,
+                              int32_t forced_fmt, uint8_t *entry, void *stream);
+
 /* ---------------------------------------------------------------------- */
 /* a5-a7: low-rank branch and block-scaled low-bit GEMM.                   */
 /* ---------------------------------------------------------------------- */

@@ -33,6 +33,7 @@ EXPORTS = ("mxq_status_string", "mxq_last_cuda_error_string", "mxq_device_suppor
            "mxq_quantize_workspace_bytes", "mxq_quantize", "mxq_dequantize", "mxq_hadamard_block", "mxq_cast",
            "mxq_select_workspace_bytes", "mxq_select_weight_format", "mxq_quantize_mse_workspace_bytes",
            "mxq_quantize_mse", "mxq_quantize_mx_grid", "mxq_fit_mx_grid_workspace_bytes", "mxq_fit_mx_grid",
+           "mxq_calibrate_workspace_bytes", "mxq_calibrate_activation", "mxq_calibrate_pick",
            "mxq_lowrank_down", "mxq_lowrank_packed_bytes",
            "mxq_lowrank_down_packed", "mxq_lowrank_pack_t", "mxq_lowrank_pack_l2", "mxq_qlinear", "mxq_route",
            "mxq_quantize_lowrank_workspace_bytes", "mxq_quantize_lowrank", "mxq_quantize_lowrank_noalloc")
@@ -78,6 +79,9 @@ def _load():
         "mxq_quantize_mx_grid": (i32, [P, i32, i64, i64, i32, i32, ctypes.c_float, i32, P, P, P]),
         "mxq_fit_mx_grid_workspace_bytes": (i32, [i64, i64, i32, psz]),
         "mxq_fit_mx_grid": (i32, [P, i32, i64, i64, i32, i32, P, i32, P, P, sz, P]),
+        "mxq_calibrate_workspace_bytes": (i32, [i64, i64, i32, psz]),
+        "mxq_calibrate_activation": (i32, [P, i32, i64, i64, P, i32, P, P, P, sz, P]),
+        "mxq_calibrate_pick": (i32, [P, P, i32, i32, P, P]),
         "mxq_lowrank_down": (i32, [P, i32, i64, i64, P, i32, P, P]),
         "mxq_lowrank_packed_bytes": (i32, [i64, psz]),
         "mxq_lowrank_down_packed": (i32, [P, i32, i64, i64, P, i32, P, P, P, P]),
@@ -283,6 +287,35 @@ def fit_mx_grid(w: torch.Tensor, fmt: int, grid_scales: Sequence[float], hadamar
     _ok(_lib.mxq_fit_mx_grid(_ptr(w), _dtype_code(w), rows, cols, fmt, hadamard_b, gs, n, _ptr(sse), _ptr(ws),
                              ws.numel(), _stream(stream)), "mxq_fit_mx_grid")
     return None if torch.cuda.is_current_stream_capturing() else grid_scales[int(torch.argmin(sse).item())], sse
+
+
+def calibrate_workspace_bytes(rows: int, cols: int, ncand: int) -> int:
+    return _size(_lib.mxq_calibrate_workspace_bytes, rows, cols, ncand)
+
+
+def calibrate_activation(x: torch.Tensor, candidates: Sequence[int], sse_accum: torch.Tensor,
+                         moments_accum: torch.Tensor, workspace: torch.Tensor = None, stream=None):
+    """Adds x's per-candidate squared error to sse_accum (float64[ncand]) and
+    (sum x^2, sum x^4) to moments_accum (float64[2])."""
+    _require_cuda(x)
+    x = x.contiguous()
+    rows, cols = x.shape
+    n = len(candidates)
+    cands = (ctypes.c_int32 * n)(*candidates)
+    ws = workspace if workspace is not None else torch.empty(calibrate_workspace_bytes(rows, cols, n),
+                                                             dtype=torch.uint8, device=x.device)
+    _ok(_lib.mxq_calibrate_activation(_ptr(x), _dtype_code(x), rows, cols, cands, n, _ptr(sse_accum),
+                                      _ptr(moments_accum), _ptr(ws), ws.numel(), _stream(stream)),
+        "mxq_calibrate_activation")
+
+
+def calibrate_pick(sse_accum: torch.Tensor, candidates: Sequence[int], entry: torch.Tensor, forced_fmt: int = -1,
+                   stream=None):
+    """Writes the table entry (a device uint8 view) for the accumulated errors."""
+    n = len(candidates)
+    cands = (ctypes.c_int32 * n)(*candidates)
+    _ok(_lib.mxq_calibrate_pick(_ptr(sse_accum), cands, n, forced_fmt, _ptr(entry), _stream(stream)),
+        "mxq_calibrate_pick")
 
 
 def lowrank_down(x: torch.Tensor, l1: torch.Tensor, out: torch.Tensor = None, stream=None) -> torch.Tensor:

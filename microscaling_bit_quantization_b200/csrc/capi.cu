@@ -242,6 +242,47 @@ mxq_status mxq_fit_mx_grid(const void *w, int32_t wdtype, int64_t rows, int64_t 
                                         workspace, (cudaStream_t)stream));
 }
 
+static bool copy_candidates(const int32_t *candidates, int32_t ncand, int *out) {
+    if (!candidates || ncand < 1 || ncand > kMaxCandidates) return false;
+    for (int j = 0; j < ncand; j++) {
+        if (!valid_fmt(candidates[j])) return false;
+        out[j] = candidates[j];
+    }
+    return true;
+}
+
+mxq_status mxq_calibrate_workspace_bytes(int64_t rows, int64_t cols, int32_t ncand, size_t *bytes) {
+    if (rows < 0 || cols < 0 || cols % 64 || ncand < 1 || ncand > kMaxCandidates || !bytes) return MXQ_EINVAL;
+    *bytes = calib_workspace_bytes(rows, cols, ncand);
+    return MXQ_OK;
+}
+
+mxq_status mxq_calibrate_activation(const void *x, int32_t xdtype, int64_t rows, int64_t cols,
+                                    const int32_t *candidates, int32_t ncand, double *sse_accum,
+                                    double *moments_accum, void *workspace, size_t workspace_bytes, void *stream) {
+    int cands[kMaxCandidates];
+    if (!valid_dtype(xdtype) || !copy_candidates(candidates, ncand, cands)) return MXQ_EINVAL;
+    if (rows < 0 || cols < 0 || cols % 64 || rows * (cols / 16) >= ((int64_t)1 << 31)) return MXQ_EINVAL;
+    if (!sse_accum || !moments_accum) return MXQ_EINVAL;
+    if (rows * cols > 0 && (!x || !aligned16(x))) return MXQ_EINVAL;
+    size_t need = 0;
+    mxq_calibrate_workspace_bytes(rows, cols, ncand, &need);
+    if (!workspace) return MXQ_EINVAL;
+    if (workspace_bytes < need) return MXQ_ENOSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MXQ_EINVAL;
+    return from_cuda(launch_calibrate(x, xdtype == MXQ_BF16, rows, cols, cands, ncand, sse_accum, moments_accum,
+                                      workspace, (cudaStream_t)stream));
+}
+
+mxq_status mxq_calibrate_pick(const double *sse_accum, const int32_t *candidates, int32_t ncand, int32_t forced_fmt,
+                              uint8_t *entry, void *stream) {
+    int cands[kMaxCandidates];
+    if (!copy_candidates(candidates, ncand, cands) || !sse_accum || !entry) return MXQ_EINVAL;
+    if (forced_fmt >= 0 && !valid_fmt(forced_fmt)) return MXQ_EINVAL;
+    return from_cuda(launch_calib_pick(sse_accum, cands, ncand, forced_fmt < 0 ? -1 : forced_fmt, entry,
+                                       (cudaStream_t)stream));
+}
+
 mxq_status mxq_lowrank_down(const void *x, int32_t xdtype, int64_t m, int64_t k, const void *l1, int32_t r, float *t,
                             void *stream) {
     if (!valid_dtype(xdtype) || m < 0 || k <= 0 || k % 16 || r < 1 || r > 32) return MXQ_EINVAL;

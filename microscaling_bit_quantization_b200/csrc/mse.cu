@@ -138,26 +138,30 @@ __global__ void __launch_bounds__(kMseThreads) k_mse_block(const T *__restrict__
 }
 
 // Ordered sums, one warp per output: output o adds entries
-// [o * per, min((o + 1) * per, total)) of `in` (W values per entry: 2 for
-// (A, B), 1 for the error) in index order; the lanes stage 32 entries at a
-// time through shared memory and lane 0 adds them.  Applied level by level:
-// blocks -> rows (per = blocks per row), rows -> groups of kMseGroup rows,
-// groups -> tensor.  FINAL (one output): W == 2 replaces *s_t by the
-// least-squares scale RN32(RN64(A / B)) (kept when B == 0); W == 1 writes the
-// total error to *sse.
-template <int W, bool FINAL>
+// [o * per, min((o + 1) * per, total)) of `in` in index order, entry i being
+// the W values at in[i * stride ...] (W = 2 for (A, B), 1 otherwise); the
+// lanes stage 32 entries at a time through shared memory and lane 0 adds
+// them.  Applied level by level: blocks -> rows (per = blocks per row), rows
+// -> groups of kMseGroup rows, groups -> tensor.  The last level (one
+// output) by FIN: kFinLsq (W == 2) replaces *s_t by the least-squares scale
+// RN32(RN64(A / B)) (kept when B == 0); kFinStore writes the W sums to
+// acc[0..W); kFinAccumulate adds them to acc[0..W).
+enum SumFinal : int { kFinNone = 0, kFinLsq = 1, kFinStore = 2, kFinAccumulate = 3 };
+
+template <int W, int FIN>
 __global__ void __launch_bounds__(kMseThreads) k_mse_sum(const double *__restrict__ in, int64_t total, int64_t per,
-                                                         double *__restrict__ out, float *s_t, double *sse) {
+                                                         int64_t stride, double *__restrict__ out, float *s_t,
+                                                         double *acc) {
     __shared__ double stage[kMseThreads / 32][32 * W];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t o = (int64_t)blockIdx.x * (kMseThreads / 32) + warp;
     const int64_t begin = o * per;
-    if (begin >= total && !(FINAL && o == 0)) return;
+    if (begin >= total && !(FIN != kFinNone && o == 0)) return;
     const int64_t end = begin + per < total ? begin + per : total;
     double s0 = 0.0, s1 = 0.0;
     for (int64_t i0 = begin; i0 < end; i0 += 32) {
         const int n = end - i0 < 32 ? (int)(end - i0) : 32;
-        for (int j = lane; j < n * W; j += 32) stage[warp][j] = in[i0 * W + j];
+        for (int j = lane; j < n * W; j += 32) stage[warp][j] = in[(i0 + j / W) * stride + j % W];
         __syncwarp();
         if (lane == 0) {
             for (int j = 0; j < n; j++) {
@@ -168,13 +172,17 @@ __global__ void __launch_bounds__(kMseThreads) k_mse_sum(const double *__restric
         __syncwarp();
     }
     if (lane != 0) return;
-    if (!FINAL) {
+    if (FIN == kFinNone) {
         out[o * W] = s0;
         if (W == 2) out[o * W + 1] = s1;
-    } else if (W == 2) {
+    } else if (FIN == kFinLsq) {
         if (s1 > 0.0) *s_t = __double2float_rn(__ddiv_rn(s0, s1));
-    } else if (sse) {
-        *sse = s0;
+    } else if (FIN == kFinStore) {
+        acc[0] = s0;
+        if (W == 2) acc[1] = s1;
+    } else {
+        acc[0] = __dadd_rn(acc[0], s0);
+        if (W == 2) acc[1] = __dadd_rn(acc[1], s1);
     }
 }
 
@@ -183,16 +191,23 @@ __global__ void k_mse_init(const unsigned int *amax_word, float *s_t) {
     *s_t = nvfp4_tensor_scale(__uint_as_float(*amax_word));
 }
 
-template <int W>
-void launch_sums(const double *blk, int64_t blocks, int64_t nb, int64_t rows, double *row_sums, double *grp_sums,
-                 float *s_t, double *sse, cudaStream_t s) {
+// blocks -> rows -> groups -> tensor over `blk` (entry i at blk[i * stride],
+// nb entries per row), the last level as FIN.
+template <int W, int FIN>
+void launch_sums(const double *blk, int64_t stride, int64_t blocks, int64_t nb, int64_t rows, double *row_sums,
+                 double *grp_sums, float *s_t, double *acc, cudaStream_t s) {
     constexpr int kWarps = kMseThreads / 32;
     const int64_t groups = (rows + kMseGroup - 1) / kMseGroup;
-    k_mse_sum<W, false><<<(int)((rows + kWarps - 1) / kWarps), kMseThreads, 0, s>>>(blk, blocks, nb, row_sums,
-                                                                                    nullptr, nullptr);
-    k_mse_sum<W, false><<<(int)((groups + kWarps - 1) / kWarps), kMseThreads, 0, s>>>(row_sums, rows, kMseGroup,
-                                                                                      grp_sums, nullptr, nullptr);
-    k_mse_sum<W, true><<<1, 32, 0, s>>>(grp_sums, groups, groups, nullptr, s_t, sse);
+    if (nb > 1) {
+        k_mse_sum<W, kFinNone><<<(int)((rows + kWarps - 1) / kWarps), kMseThreads, 0, s>>>(
+            blk, blocks, nb, stride, row_sums, nullptr, nullptr);
+    }
+    // with one entry per row the entries are the row sums (0 + x = x exactly)
+    const double *rs = nb > 1 ? row_sums : blk;
+    const int64_t rs_stride = nb > 1 ? W : stride;
+    k_mse_sum<W, kFinNone><<<(int)((groups + kWarps - 1) / kWarps), kMseThreads, 0, s>>>(
+        rs, rows, kMseGroup, rs_stride, grp_sums, nullptr, nullptr);
+    k_mse_sum<W, FIN><<<1, 32, 0, s>>>(grp_sums, groups, groups, W, nullptr, s_t, acc);
 }
 
 template <typename T>
@@ -202,11 +217,11 @@ cudaError_t run_mse(const T *x, const MseArgs &base, int iters, double *row_sums
     const int gb = (int)((base.blocks + kMseThreads - 1) / kMseThreads);
     for (int it = 0; it < iters; it++) {
         k_mse_block<T, kMsePartial><<<gb, kMseThreads, 0, s>>>(x, base);
-        launch_sums<2>(base.blk, base.blocks, nb, base.rows, row_sums, grp_sums, const_cast<float *>(base.s_t),
-                       nullptr, s);
+        launch_sums<2, kFinLsq>(base.blk, 2, base.blocks, nb, base.rows, row_sums, grp_sums,
+                                const_cast<float *>(base.s_t), nullptr, s);
     }
     k_mse_block<T, kMseEncode><<<gb, kMseThreads, 0, s>>>(x, base);
-    launch_sums<1>(base.blk, base.blocks, nb, base.rows, row_sums, grp_sums, nullptr, sse, s);
+    if (sse) launch_sums<1, kFinStore>(base.blk, 1, base.blocks, nb, base.rows, row_sums, grp_sums, nullptr, sse, s);
     return cudaGetLastError();
 }
 
@@ -307,6 +322,48 @@ void launch_mx_grid_err(const T *x, int fmt, const MxFitArgs &a, cudaStream_t s)
     else k_mx_grid_err<T, false><<<grid, kMseThreads, 0, s>>>(x, a);
 }
 
+// ---------------------------------------------------------------------------
+// Activation-format calibration (Chameleon article, section "the format is
+// chosen by the value distribution": per layer and per interval of the
+// denoising trajectory, activations are calibrated in advance and the
+// result is a table read at generation time).  Per calibration activation:
+// each candidate's squared quantization error (the selection kernel's
+// per-row errors, rows summed in groups of kMseGroup, groups in order) and
+// the tail moments sum x^2, sum x^4 (element order within a 16-element
+// chunk, chunks, rows, groups) are added to the entry's accumulators; the
+// entry then takes the candidate with the least accumulated error.
+
+// Per 16-element chunk: (sum x^2, sum x^4) in element order (x^2 exact).
+template <typename T>
+__global__ void __launch_bounds__(kMseThreads) k_moments(const T *__restrict__ x, int64_t chunks, double *blk) {
+    const int64_t c = (int64_t)blockIdx.x * kMseThreads + threadIdx.x;
+    if (c >= chunks) return;
+    float v[16];
+    load16(x + c * 16, v);
+    double s2 = 0.0, s4 = 0.0;
+#pragma unroll
+    for (int i = 0; i < 16; i++) {
+        const double q = __dmul_rn((double)v[i], (double)v[i]);
+        s2 = __dadd_rn(s2, q);
+        s4 = __dadd_rn(s4, __dmul_rn(q, q));
+    }
+    blk[2 * c] = s2;
+    blk[2 * c + 1] = s4;
+}
+
+struct PickArgs {
+    int ncand;
+    int cand[kMaxCandidates];
+    int forced;   // >= 0: the entry takes this format
+};
+
+__global__ void k_calib_pick(const double *sse, PickArgs a, uint8_t *entry) {
+    int best = 0;
+    for (int j = 1; j < a.ncand; j++)
+        if (sse[j] < sse[best]) best = j;
+    *entry = (uint8_t)(a.forced >= 0 ? a.forced : a.cand[best]);
+}
+
 }  // namespace
 
 size_t mse_workspace_bytes(int64_t rows, int64_t cols) {
@@ -335,7 +392,45 @@ cudaError_t launch_fit_mx_grid(const void *w, bool bf16, int64_t rows, int64_t c
     if (bf16) launch_mx_grid_err((const __nv_bfloat16 *)w, fmt, a, s);
     else launch_mx_grid_err((const float *)w, fmt, a, s);
     for (int j = 0; j < n; j++)
-        launch_sums<1>(a.blk + (int64_t)j * blocks, blocks, cols / 32, rows, row_sums, grp_sums, nullptr, sse + j, s);
+        launch_sums<1, kFinStore>(a.blk + (int64_t)j * blocks, 1, blocks, cols / 32, rows, row_sums, grp_sums, nullptr,
+                                  sse + j, s);
+    return cudaGetLastError();
+}
+
+size_t calib_workspace_bytes(int64_t rows, int64_t cols, int ncand) {
+    return 256 + (size_t)rows * ncand * 8 + (size_t)rows + 15 + (size_t)(rows * (cols / 16)) * 16 +
+           (size_t)rows * 16 + (size_t)((rows + kMseGroup - 1) / kMseGroup) * 16 + 64;
+}
+
+cudaError_t launch_calibrate(const void *x, bool bf16, int64_t rows, int64_t cols, const int *cands, int ncand,
+                             double *sse_accum, double *moments_accum, void *workspace, cudaStream_t s) {
+    if (rows == 0 || cols == 0) return cudaSuccess;   // nothing to add
+    unsigned int *amax = (unsigned int *)workspace;
+    double *sse_rows = (double *)((char *)workspace + 256);
+    uint8_t *choice = (uint8_t *)(sse_rows + rows * ncand);
+    double *mom = (double *)(((uintptr_t)(choice + rows) + 15) & ~(uintptr_t)15);
+    const int64_t chunks = rows * (cols / 16);
+    double *row_sums = mom + 2 * chunks;
+    double *grp_sums = row_sums + 2 * rows;
+    cudaError_t e = launch_select(x, bf16, rows, cols, cands, ncand, choice, sse_rows, amax, s);
+    if (e != cudaSuccess) return e;
+    for (int j = 0; j < ncand; j++)
+        launch_sums<1, kFinAccumulate>(sse_rows + j, ncand, rows, 1, rows, row_sums, grp_sums, nullptr,
+                                       sse_accum + j, s);
+    const int g = (int)((chunks + kMseThreads - 1) / kMseThreads);
+    if (bf16) k_moments<<<g, kMseThreads, 0, s>>>((const __nv_bfloat16 *)x, chunks, mom);
+    else k_moments<<<g, kMseThreads, 0, s>>>((const float *)x, chunks, mom);
+    launch_sums<2, kFinAccumulate>(mom, 2, chunks, cols / 16, rows, row_sums, grp_sums, nullptr, moments_accum, s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_calib_pick(const double *sse_accum, const int *cands, int ncand, int forced, uint8_t *entry,
+                              cudaStream_t s) {
+    PickArgs a;
+    a.ncand = ncand;
+    for (int j = 0; j < kMaxCandidates; j++) a.cand[j] = j < ncand ? cands[j] : 0;
+    a.forced = forced;
+    k_calib_pick<<<1, 1, 0, s>>>(sse_accum, a, entry);
     return cudaGetLastError();
 }
 

@@ -30,6 +30,13 @@ cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols
 // Squared error of the (rotated) tensor under MX quantization with each of
 // n <= kMaxCandidates grid scales (mse.cu); sse: device double[n].
 size_t mx_grid_workspace_bytes(int64_t rows, int64_t cols, int n);
+// Activation-format calibration (mse.cu): adds each candidate's squared
+// error to sse_accum[j] and (sum x^2, sum x^4) to moments_accum[0..1].
+size_t calib_workspace_bytes(int64_t rows, int64_t cols, int ncand);
+cudaError_t launch_calibrate(const void *x, bool bf16, int64_t rows, int64_t cols, const int *cands, int ncand,
+                             double *sse_accum, double *moments_accum, void *workspace, cudaStream_t s);
+cudaError_t launch_calib_pick(const double *sse_accum, const int *cands, int ncand, int forced, uint8_t *entry,
+                              cudaStream_t s);
 cudaError_t launch_fit_mx_grid(const void *w, bool bf16, int64_t rows, int64_t cols, int fmt, int hadamard_b,
                                const float *grid_scales, int n, double *sse, void *workspace, cudaStream_t s);
 // NVFP4 with block and tensor scales fitted to the squared error (mse.cu);

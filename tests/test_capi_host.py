@@ -119,6 +119,24 @@ def test_mx_grid_argument_checks(mxq):
     assert fit(d, 1, 4, 64, mxq.INT4_G32, 0, gs, 2, d, d, 1 << 20, None) == 2
 
 
+def test_calibration_argument_checks(mxq):
+    L, P = mxq.lib(), ctypes.c_void_p
+    size = ctypes.c_size_t(0)
+    assert L.mxq_calibrate_workspace_bytes(300, 1152, 3, ctypes.byref(size)) == 0 and size.value > 300 * 3 * 8
+    assert L.mxq_calibrate_workspace_bytes(4, 48, 3, ctypes.byref(size)) == 1      # 48 % 64
+    d = P(256)
+    c3 = (ctypes.c_int32 * 3)(5, 6, 0)
+    cal = L.mxq_calibrate_activation
+    assert cal(d, 1, 4, 64, c3, 0, d, d, d, 1 << 20, None) == 1                  # no candidates
+    assert cal(d, 1, 4, 64, c3, 3, None, d, d, 1 << 20, None) == 1               # no accumulator
+    assert cal(d, 1, 4, 64, c3, 3, d, d, d, 16, None) == 5                       # workspace too small
+    bad = (ctypes.c_int32 * 1)(9)
+    assert cal(d, 1, 4, 64, bad, 1, d, d, d, 1 << 20, None) == 1                 # bad format id
+    pick = L.mxq_calibrate_pick
+    assert pick(d, c3, 3, 9, d, None) == 1                                       # bad forced format
+    assert pick(None, c3, 3, -1, d, None) == 1
+
+
 def test_qlinear_argument_checks(mxq):
     L = mxq.lib()
     Q = mxq._QTensorC

@@ -316,3 +316,82 @@ def test_mx_grid_full_size(mxq, orc):
     q = mxq.quantize_mx_grid(wd, mxq.MXFP4, best, 128, mxq.MMA)
     u = mxq.quantize(wd, mxq.MXFP4, 128, mxq.MMA)
     assert torch.equal(q.codes, u.codes) == (best == 1.0)
+
+
+# ------------------------------------------------------------------ activation-format calibration
+
+CALIB = [5, 6, 0]   # INT8 per row, FP8 per tensor, MXFP8 (workload 5's palette)
+
+
+def _pick_ok(gpu_entry, ref_sse, cands, forced=-1):
+    if forced >= 0:
+        return gpu_entry == forced
+    s = np.sort(ref_sse)
+    return gpu_entry == cands[int(np.argmin(ref_sse))] or s[1] - s[0] <= 1e-12 * s[0]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_calibrate_small(mxq, orc, dtype):
+    rng = np.random.default_rng(61)
+    xs = []
+    for nu in (2.2, 20.0):
+        x = rng.standard_t(nu, size=(300, 1152)).astype(np.float32)   # three row groups, the last ragged
+        x[:, rng.choice(1152, 8, replace=False)] *= 60.0
+        xs.append(host_values(x, dtype))
+    sse = torch.zeros(3, dtype=torch.float64, device="cuda")
+    mom = torch.zeros(2, dtype=torch.float64, device="cuda")
+    ref_sse, ref_mom = np.zeros(3), np.zeros(2)
+    for x in xs:
+        mxq.calibrate_activation(dev(x, dtype), CALIB, sse, mom)
+        orc.calibrate_activation(x, CALIB, ref_sse, ref_mom)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(sse.cpu().numpy(), ref_sse, rtol=1e-12)   # per-row order differs
+    np.testing.assert_array_equal(mom.cpu().numpy(), ref_mom)            # same order: bit-exact
+    entry = torch.zeros(1, dtype=torch.uint8, device="cuda")
+    mxq.calibrate_pick(sse, CALIB, entry)
+    assert _pick_ok(int(entry.item()), ref_sse, CALIB)
+    mxq.calibrate_pick(sse, CALIB, entry, forced_fmt=mxq.MXFP8)
+    assert entry.item() == mxq.MXFP8
+
+
+def test_calibrate_table(mxq, orc):
+    """A 3-layer x 4-interval table from seeded activations whose tails
+    thin out along the trajectory; layer 2 forced to MXFP8; then routed."""
+    n_layers, n_int, per = 3, 4, 2
+    table = torch.zeros((n_layers, n_int), dtype=torch.uint8, device="cuda")
+    ref = np.zeros((n_layers, n_int), np.uint8)
+    for layer in range(n_layers):
+        for it in range(n_int):
+            sse = torch.zeros(3, dtype=torch.float64, device="cuda")
+            mom = torch.zeros(2, dtype=torch.float64, device="cuda")
+            ref_sse, ref_mom = np.zeros(3), np.zeros(2)
+            for s in range(per):
+                x = workloads.student_t(70 + layer, "calib.%d.%d" % (it, s), (256, 1152), 2.0 + 10.0 * it)
+                if layer == 1:
+                    x = x * workloads.dit_forced_column_factors(7, layer, 1152)[None, :]
+                x = host_values(x, "bf16")
+                mxq.calibrate_activation(dev(x, "bf16"), CALIB, sse, mom)
+                orc.calibrate_activation(x, CALIB, ref_sse, ref_mom)
+            forced = mxq.MXFP8 if layer == 2 else -1
+            mxq.calibrate_pick(sse, CALIB, table[layer, it:it + 1], forced_fmt=forced)
+            ref[layer, it] = orc.calibrate_pick(ref_sse, CALIB, forced)
+            np.testing.assert_array_equal(mom.cpu().numpy(), ref_mom)
+            assert _pick_ok(int(table[layer, it].item()), ref_sse, CALIB, forced)
+    tab = table.cpu().numpy()
+    assert (tab[2] == mxq.MXFP8).all()
+    for layer in range(n_layers):
+        for step in range(20):
+            assert mxq.route(tab, layer, step, 20) == orc.route(tab, n_layers, n_int, layer, step, 20)
+
+
+def test_calibrate_full_size(mxq, orc):
+    """Workload 5's fc1 input at step 0 (8192 x 1152 bf16), the benchmark's call."""
+    x = workloads.dit_activation(5, 0, 1152)
+    sse = torch.zeros(3, dtype=torch.float64, device="cuda")
+    mom = torch.zeros(2, dtype=torch.float64, device="cuda")
+    mxq.calibrate_activation(dev(x, "bf16"), CALIB, sse, mom)
+    ref_sse, ref_mom = np.zeros(3), np.zeros(2)
+    orc.calibrate_activation(x, CALIB, ref_sse, ref_mom)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(sse.cpu().numpy(), ref_sse, rtol=1e-12)
+    np.testing.assert_array_equal(mom.cpu().numpy(), ref_mom)
