@@ -354,14 +354,14 @@ mxq_status mxq_quantize_lowrank(const void *x, int32_t xdtype, int64_t m, int64_
 
 /* Same as mxq_quantize_lowrank, but without a workspace argument: the
  * scratch it needs (the tensor-amax word and the m x r fp32 low-rank
- * activation, 256 + 4*m*r bytes) lives in a 4 MiB array that the library
+ * activation, 4096 + 4*m*r bytes) lives in a 4 MiB array that the library
  * keeps in device memory, one per GPU that loads it, until the process
  * exits.  The pages describe no such call; it exists for callers that
  * cannot allocate device memory themselves: code embedded in a host
  * application that owns every device buffer and hands the library only its
  * inputs and outputs, and latency-bound callers for whom a cudaMalloc,
  * which may synchronize the device, is not acceptable.
- *   Limit: 256 + 4*m*r <= 4 MiB (m*r <= 1,048,512, e.g. m <= 32,767 rows
+ *   Limit: 4096 + 4*m*r <= 4 MiB (m*r <= 1,047,552, e.g. m <= 32,736 rows
  *     at rank 32); larger calls return MXQ_ENOSPACE and launch nothing.
  *   The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.

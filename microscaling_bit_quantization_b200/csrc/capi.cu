@@ -315,7 +315,7 @@ mxq_status mxq_lowrank_pack_t(const float *t, int32_t r, int64_t m, const float 
 
 mxq_status mxq_quantize_lowrank_workspace_bytes(int64_t m, int32_t r, size_t *bytes) {
     if (m < 0 || r < 1 || r > 32 || !bytes) return MXQ_EINVAL;
-    *bytes = 256 + (size_t)(m * r * 4);
+    *bytes = kLrHeader + (size_t)(m * r * 4);
     return MXQ_OK;
 }
 
@@ -340,14 +340,24 @@ mxq_status mxq_quantize_lowrank(const void *x, int32_t xdtype, int64_t m, int64_
     mxq_scales_bytes(fmt, m, k, MXQ_LAYOUT_MMA, &sb);
     cudaStream_t s = (cudaStream_t)stream;
     unsigned int *amax = (unsigned int *)workspace;
-    float *t = (float *)((char *)workspace + 256);
+    float *slots = (float *)((char *)workspace + 256);
+    float *t = (float *)((char *)workspace + kLrHeader);
     const bool bf = xdtype == MXQ_BF16;
     cudaError_t e = cudaSuccess;
     bool amax_ready = false;
+    int n_slots = 0;
     if (ts && hadamard_b == 0) {
-        // one read of x from HBM gives both the tensor amax and t
-        e = cudaMemsetAsync(amax, 0, sizeof(unsigned int), s);
-        if (e == cudaSuccess) e = launch_lowrank_down(x, bf, m, k, l1, r, t, nullptr, nullptr, nullptr, s, amax);
+        // one read of x from HBM gives both the tensor amax and t: the
+        // tensor-core kernel writes per-warp maxima (no clearing needed, so
+        // the three kernels follow each other with no memset between); the
+        // other kernels fold into a zeroed word
+        e = bf ? launch_lowrank_tc(x, m, k, l1, r, t, nullptr, nullptr, nullptr, slots, &n_slots, s)
+               : cudaErrorNotSupported;
+        if (e == cudaErrorNotSupported) {
+            n_slots = 0;
+            e = cudaMemsetAsync(amax, 0, sizeof(unsigned int), s);
+            if (e == cudaSuccess) e = launch_lowrank_down(x, bf, m, k, l1, r, t, nullptr, nullptr, nullptr, s, amax);
+        }
         amax_ready = true;
     } else {
         e = launch_lowrank_down(x, bf, m, k, l1, r, t, nullptr, nullptr, nullptr, s);
@@ -355,7 +365,7 @@ mxq_status mxq_quantize_lowrank(const void *x, int32_t xdtype, int64_t m, int64_
     if (e != cudaSuccess) return from_cuda(e);
     PackT pack{t, r, w_tensor_scale, tp};
     return from_cuda(launch_quantize(x, bf, m, k, fmt, hadamard_b, MXQ_LAYOUT_MMA, codes, scales, sb, tensor_scale,
-                                     amax, s, &pack, amax_ready));
+                                     amax, s, &pack, amax_ready, 1.0f, slots, n_slots));
 }
 
 mxq_status mxq_lowrank_pack_l2(const void *l2, int32_t r, int64_t n, void *l2p, void *stream) {

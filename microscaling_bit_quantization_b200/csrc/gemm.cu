@@ -262,6 +262,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int nsteps = p.num_k_tiles + p.has_lowrank;
+    // the setup above overlaps the previous kernel (the quantizer); operands
+    // are read and Y written only after it has completed
+    pdl_wait();
+    pdl_launch_dependents();
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer (both CTAs)
@@ -601,8 +605,16 @@ cudaError_t launch_kind(const GemmParams &p, int grid, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    k_gemm<KIND><<<grid, kGemmThreads, SMEM_BYTES, s>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);   // clusters of 2 from __cluster_dims__
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1] = {pdl_attribute()};
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_gemm<KIND>, p);
 }
 
 }  // namespace

@@ -320,8 +320,8 @@ static void launch_lr(int mode, int grid, const T *x, int64_t m, int64_t k, cons
 cudaError_t launch_lowrank_down(const void *x, bool bf16, int64_t m, int64_t k, const void *l1, int r, float *t,
                                 const float *xs, const float *ws, void *tp, cudaStream_t s, unsigned int *amax_word) {
     if (m == 0) return cudaSuccess;
-    if (bf16) {   // the tensor-core path when it takes the shape
-        const cudaError_t e = launch_lowrank_tc(x, m, k, l1, r, tp ? nullptr : t, tp, xs, ws, amax_word, s);
+    if (bf16 && !amax_word) {   // the tensor-core path when it takes the shape (its amax goes to slots)
+        const cudaError_t e = launch_lowrank_tc(x, m, k, l1, r, tp ? nullptr : t, tp, xs, ws, nullptr, nullptr, s);
         if (e != cudaErrorNotSupported) return e;
     }
     const int grid = (int)((m + 15) / 16);

@@ -57,7 +57,7 @@ struct LrTcParams {
     float *t;                  // m x r (T output) or null
     __nv_bfloat16 *tp;         // m x 64 (packed output) or null
     const float *xs, *ws;      // packed output divisor s_x * s_w; null: 1
-    unsigned int *amax_word;   // null: no amax
+    float *amax_slots;         // null: no amax; else warp w (2-5) of CTA b writes slot 4 b + w - 2
     unsigned int *err;
     int m, k, r, kb_total, kb_max, row_tiles, S;
     unsigned long long wait_ns;
@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
     const int nkb = (int)((rank + 1) * (uint32_t)p.kb_total / (uint32_t)S) - kb0;
     const int ntiles = cid < p.row_tiles ? (p.row_tiles - cid + ncl - 1) / ncl : 0;
     const int total = ntiles * nkb;
-    const bool want_amax = p.amax_word != nullptr;
+    const bool want_amax = p.amax_slots != nullptr;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < LT_STAGES; s++) {
@@ -162,6 +162,10 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
     cluster_sync();   // barriers of every CTA initialized before any remote arrival
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // setup above overlaps the previous kernel; X, L1 and the scales are read,
+    // and T and the maxima written, only after it has completed
+    pdl_wait();
+    pdl_launch_dependents();
 
     // The first tiles of X are in flight while the B tiles are built; the L1
     // loads of the first round are issued before them, so they are not queued
@@ -397,9 +401,9 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
             if (lane == 0 && !*abort_flag) atomicOr(p.err, kErrLt);
             *abort_flag = 1;
         }
-        if (want_amax) {   // non-negative floats order like their bit patterns
+        if (want_amax) {   // every slot is written, so the slots need no clearing
             mx = group_max<32>(mx);
-            if (lane == 0 && mx > 0.0f) atomicMax(p.amax_word, __float_as_uint(mx));
+            if (lane == 0) p.amax_slots[4 * blockIdx.x + e] = mx;
         }
     }
 
@@ -414,7 +418,8 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
 }  // namespace
 
 cudaError_t launch_lowrank_tc(const void *x, int64_t m, int64_t k, const void *l1, int r, float *t, void *tp,
-                              const float *xs, const float *ws, unsigned int *amax_word, cudaStream_t s) {
+                              const float *xs, const float *ws, float *amax_slots, int *n_slots,
+                              cudaStream_t s) {
     if (m <= 0 || k <= 0 || r < 1 || r > 32 || k % 8 || m >= ((int64_t)1 << 31) || k >= ((int64_t)1 << 31) ||
         (reinterpret_cast<uintptr_t>(x) & 15u))
         return cudaErrorNotSupported;
@@ -483,7 +488,9 @@ cudaError_t launch_lowrank_tc(const void *x, int64_t m, int64_t k, const void *l
     p.tp = (__nv_bfloat16 *)tp;
     p.xs = xs;
     p.ws = ws;
-    p.amax_word = amax_word;
+    p.amax_slots = amax_slots;
+    if (4 * best_clusters * best_s > kAmaxSlots) return cudaErrorNotSupported;
+    if (n_slots) *n_slots = 4 * best_clusters * best_s;
     p.wait_ns = 2000000000ull;
     cudaError_t e = error_word_address(&p.err);
     if (e != cudaSuccess) return e;
@@ -497,13 +504,14 @@ cudaError_t launch_lowrank_tc(const void *x, int64_t m, int64_t k, const void *l
     cfg.blockDim = dim3(LT_THREADS, 1, 1);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)best_s;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1] = pdl_attribute();
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     switch (best_s) {
     case 1: return cudaLaunchKernelEx(&cfg, k_lowrank_tc<1>, p);
     case 2: return cudaLaunchKernelEx(&cfg, k_lowrank_tc<2>, p);

@@ -11,6 +11,23 @@ namespace mxq {
 
 constexpr int kMaxCandidates = 8;
 
+// Launch attribute of the kernels on the activation -> GEMM chain
+// (k_lowrank_tc, k_quantize, k_gemm): the kernel may be scheduled while
+// the previous kernel in the stream finishes; it overlaps only its setup
+// (barriers, TMEM, launch latency) and waits (pdl_wait) before touching
+// global memory.
+inline cudaLaunchAttribute pdl_attribute() {
+    cudaLaunchAttribute a;
+    a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a.val.programmaticStreamSerializationAllowed = 1;
+    return a;
+}
+
+// Workspace of mxq_quantize_lowrank: the amax word at 0, the per-warp maxima
+// of k_lowrank_tc from byte 256 (at most kAmaxSlots), T from kLrHeader.
+constexpr size_t kLrHeader = 4096;
+constexpr int kAmaxSlots = (int)((kLrHeader - 256) / 4);
+
 cudaError_t launch_amax(const void *x, bool bf16, int64_t rows, int64_t cols, int hadamard_b,
                         unsigned int *amax_word, cudaStream_t s);
 // Optional duty of the quantizer: pack the low-rank activation t (rows x r
@@ -26,7 +43,8 @@ struct PackT {
 cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols, int fmt, int hadamard_b,
                             int layout, void *codes, void *scales, size_t scales_bytes, float *tensor_scale,
                             unsigned int *amax_word, cudaStream_t s, const PackT *pack = nullptr,
-                            bool amax_ready = false, float mx_grid = 1.0f);
+                            bool amax_ready = false, float mx_grid = 1.0f, const float *amax_slots = nullptr,
+                            int n_slots = 0);
 // Squared error of the (rotated) tensor under MX quantization with each of
 // n <= kMaxCandidates grid scales (mse.cu); sse: device double[n].
 size_t mx_grid_workspace_bytes(int64_t rows, int64_t cols, int n);
@@ -66,8 +84,11 @@ cudaError_t launch_lowrank_down(const void *x, bool bf16, int64_t m, int64_t k, 
 // with amax_word (zeroed beforehand) also folds in max |x|.  Returns
 // cudaErrorNotSupported, launching nothing, for shapes it does not take
 // (k % 8, unaligned x, a K slice that does not fit in shared memory).
+// amax_slots: null, or room for kAmaxSlots floats receiving per-warp maxima
+// of |x| (*n_slots of them, every one written).  cudaErrorNotSupported: a
+// shape this kernel does not take (nothing launched).
 cudaError_t launch_lowrank_tc(const void *x, int64_t m, int64_t k, const void *l1, int r, float *t, void *tp,
-                              const float *xs, const float *ws, unsigned int *amax_word, cudaStream_t s);
+                              const float *xs, const float *ws, float *amax_slots, int *n_slots, cudaStream_t s);
 cudaError_t launch_pack_l2(const void *l2, int r, int64_t n, void *l2p, cudaStream_t s);
 cudaError_t launch_pack_t(const float *t, int r, int64_t m, const float *xs, const float *ws, void *tp,
                           cudaStream_t s);

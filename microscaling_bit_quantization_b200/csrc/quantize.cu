@@ -14,6 +14,7 @@
 
 #include "mxq_formats.cuh"
 #include "mxq_internal.h"
+#include "tc_ptx.cuh"
 
 namespace mxq {
 
@@ -47,6 +48,22 @@ __device__ __forceinline__ void cta_max_to_word(float m, unsigned int *word) {
     }
 }
 
+// Max of n non-negative values, reduced by the whole CTA (all NT threads call
+// this).
+template <int NT>
+__device__ __forceinline__ float cta_max_of(const float *v, int n) {
+    __shared__ float wm[NT / 32];
+    float m = 0.0f;
+    for (int i = threadIdx.x; i < n; i += NT) m = fmaxf(m, v[i]);
+    m = group_max<32>(m);
+    if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+    __syncthreads();
+    float r = 0.0f;
+#pragma unroll
+    for (int w = 0; w < NT / 32; w++) r = fmaxf(r, wm[w]);
+    return r;
+}
+
 // ------------------------------------------------------------------ quantize
 
 struct QuantArgs {
@@ -59,6 +76,8 @@ struct QuantArgs {
     void *scales;
     float *tensor_scale;     // written by chunk 0 (NVFP4, FP8_TENSOR)
     const unsigned int *amax_word;
+    const float *amax_slots;  // n_slots > 0: the tensor amax is the max of these (else *amax_word)
+    int n_slots;
     float mx_grid;           // MX grid scale g in [1, 2] (1: the OCP rule)
     // optional packed low-rank operand: tp[row] = [hi | lo] of t[row] / (s_x * *w_ts)
     const float *t;
@@ -204,11 +223,15 @@ __global__ void __launch_bounds__(kQThreads, 2) k_quantize(const T *__restrict__
     const uint32_t cpr = (uint32_t)(a.cols >> 4);
     const uint32_t s_pad4 = (uint32_t)(a.s_pad >> 2);
 
+    // nothing global is touched before the previous kernel has completed
+    pdl_wait();
+    pdl_launch_dependents();
     float s_t = 1.0f;
     TensorRecip tr;
     Recip rt;
     if (F == kNVFP4 || F == kFP8Tensor) {
-        float amax_t = __uint_as_float(*a.amax_word);
+        const float amax_t = a.n_slots > 0 ? cta_max_of<kQThreads>(a.amax_slots, a.n_slots)
+                                           : __uint_as_float(*a.amax_word);
         s_t = F == kNVFP4 ? nvfp4_tensor_scale(amax_t) : fp8_tensor_scale(amax_t);
         if (blockIdx.x == 0 && threadIdx.x == 0) *a.tensor_scale = s_t;
         if (F == kNVFP4) tr = tensor_recip_of(s_t);
@@ -630,7 +653,15 @@ static void launch_qf(const T *x, const QuantArgs &a, cudaStream_t s) {
     const int64_t steps = (a.total_chunks + kQThreads - 1) / kQThreads;
     const int64_t cap = (int64_t)sm_count_cached() * 2;   // two 512-thread CTAs per SM
     const int grid = (int)(steps < cap ? steps : cap);
-    k_quantize<T, F><<<grid, kQThreads, 0, s>>>(x, a);
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(kQThreads, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1] = {pdl_attribute()};
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, k_quantize<T, F>, x, a);
 }
 
 template <typename T>
@@ -653,7 +684,7 @@ static void launch_q(int fmt, int grid, const T *x, const QuantArgs &a, cudaStre
 cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols, int fmt, int hadamard_b,
                             int layout, void *codes, void *scales, size_t scales_bytes, float *tensor_scale,
                             unsigned int *amax_word, cudaStream_t s, const PackT *pack, bool amax_ready,
-                            float mx_grid) {
+                            float mx_grid, const float *amax_slots, int n_slots) {
     cudaError_t e;
     if (fmt_tensor_scaled(fmt) && !amax_ready) {
         e = launch_amax(x, bf16, rows, cols, hadamard_b, amax_word, s);
@@ -671,6 +702,8 @@ cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols
     a.scales = scales;
     a.tensor_scale = tensor_scale;
     a.amax_word = amax_word;
+    a.amax_slots = amax_slots;
+    a.n_slots = n_slots;
     a.mx_grid = mx_grid;
     a.t = pack ? pack->t : nullptr;
     a.r = pack ? pack->r : 0;

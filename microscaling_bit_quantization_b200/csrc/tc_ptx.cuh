@@ -167,5 +167,15 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Programmatic dependent launch.  pdl_wait: returns once the preceding grid
+// in the stream has completed and its memory operations are visible (at
+// once when there is none); a kernel launched with the programmatic
+// serialization attribute calls it before its first global read of data
+// another kernel may produce and before its first global write.
+// pdl_launch_dependents: the next such grid may be scheduled (it still
+// waits in pdl_wait for this grid to complete).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 }  // namespace
 }  // namespace mxq

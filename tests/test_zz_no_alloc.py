@@ -78,7 +78,7 @@ def test_noalloc_rejects_sizes_beyond_the_array(mxq):
     wq = mxq.quantize(w, 2, 0, mxq.MMA)
     P = ctypes.c_void_p
     dummy = P(x.data_ptr())
-    # 256 + 4 * m * r bytes must fit in 4 MiB: m = 40000 rows at rank 32 does not
+    # 4096 + 4 * m * r bytes must fit in 4 MiB: m = 40000 rows at rank 32 does not
     st = mxq.lib().mxq_quantize_lowrank_noalloc(dummy, mxq.BF16, 40000, 512, 2, 0, P(l1.data_ptr()), 32,
                                                 P(wq.tensor_scale.data_ptr()), dummy, dummy, dummy, dummy, None)
     assert st == 5   # MXQ_ENOSPACE, nothing launched
