@@ -335,7 +335,7 @@ def run_ours(args, world, rank, local):
         del g
         return a.elapsed_time(b) / (reps * n)
 
-    qws = torch.empty(16, dtype=torch.uint8, device=dev)
+    qws = torch.empty(mxq.quantize_workspace_bytes(mxq.NVFP4), dtype=torch.uint8, device=dev)
     formats = {}
     for name, fmt, had in (("NVFP4", mxq.NVFP4, 0), ("MXFP4", mxq.MXFP4, 0), ("MXFP4+hadamard128", mxq.MXFP4, 128),
                            ("MXFP8", mxq.MXFP8, 0), ("INT4_G64", mxq.INT4_G64, 0), ("INT8_ROW", mxq.INT8_ROW, 0),

@@ -119,8 +119,8 @@ mxq_status mxq_check(void *stream);
 mxq_status mxq_codes_bytes(int32_t fmt, int64_t rows, int64_t cols, int32_t layout, size_t *bytes);
 mxq_status mxq_scales_bytes(int32_t fmt, int64_t rows, int64_t cols, int32_t layout, size_t *bytes);
 
-/* Scratch bytes mxq_quantize needs (tensor-amax word for NVFP4 and
- * FP8_TENSOR; 0 otherwise). */
+/* Scratch bytes mxq_quantize needs (4096 for NVFP4 and FP8_TENSOR: the
+ * per-CTA maxima of the tensor-amax pass; 0 otherwise). */
 mxq_status mxq_quantize_workspace_bytes(int32_t fmt, size_t *bytes);
 
 /* ---------------------------------------------------------------------- */

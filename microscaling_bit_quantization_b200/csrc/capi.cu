@@ -104,7 +104,7 @@ mxq_status mxq_scales_bytes(int32_t fmt, int64_t rows, int64_t cols, int32_t lay
 
 mxq_status mxq_quantize_workspace_bytes(int32_t fmt, size_t *bytes) {
     if (!valid_fmt(fmt) || !bytes) return MXQ_EINVAL;
-    *bytes = fmt_tensor_scaled(fmt) ? 16 : 0;
+    *bytes = fmt_tensor_scaled(fmt) ? kLrHeader : 0;   // the amax word and per-CTA maxima
     return MXQ_OK;
 }
 

@@ -64,6 +64,19 @@ __device__ __forceinline__ float cta_max_of(const float *v, int n) {
     return r;
 }
 
+// Max over the CTA of one value per thread (all NT threads call this).
+template <int NT>
+__device__ __forceinline__ float cta_reduce_max(float m) {
+    __shared__ float wr[NT / 32];
+    m = group_max<32>(m);
+    if ((threadIdx.x & 31) == 0) wr[threadIdx.x >> 5] = m;
+    __syncthreads();
+    float r = 0.0f;
+#pragma unroll
+    for (int w = 0; w < NT / 32; w++) r = fmaxf(r, wr[w]);
+    return r;
+}
+
 // ------------------------------------------------------------------ quantize
 
 struct QuantArgs {
@@ -78,6 +91,7 @@ struct QuantArgs {
     const unsigned int *amax_word;
     const float *amax_slots;  // n_slots > 0: the tensor amax is the max of these (else *amax_word)
     int n_slots;
+    float *amax_out;          // amax-only pass: CTA b writes its max to amax_out[b] (null: atomicMax into the word)
     float mx_grid;           // MX grid scale g in [1, 2] (1: the OCP rule)
     // optional packed low-rank operand: tp[row] = [hi | lo] of t[row] / (s_x * *w_ts)
     const float *t;
@@ -303,7 +317,12 @@ __global__ void __launch_bounds__(kQThreads, 2) k_quantize(const T *__restrict__
         }
     }
     if (F == kNumFmt) {
-        cta_max_to_word<kQThreads>(tensor_max, const_cast<unsigned int *>(a.amax_word));
+        if (a.amax_out) {   // every CTA writes its slot, so the slots need no clearing
+            const float m = cta_reduce_max<kQThreads>(tensor_max);
+            if (threadIdx.x == 0) a.amax_out[blockIdx.x] = m;
+        } else {
+            cta_max_to_word<kQThreads>(tensor_max, const_cast<unsigned int *>(a.amax_word));
+        }
         return;
     }
     if (a.tp) {
@@ -648,6 +667,29 @@ cudaError_t launch_amax(const void *x, bool bf16, int64_t rows, int64_t cols, in
     return cudaGetLastError();
 }
 
+// The tensor amax as per-CTA maxima (no clearing, no atomics): slots must
+// hold 2 x SM-count floats; *n_slots gets the count written.
+static cudaError_t launch_amax_slots(const void *x, bool bf16, int64_t rows, int64_t cols, int hadamard_b,
+                                     float *slots, int *n_slots, cudaStream_t s) {
+    *n_slots = 0;
+    int64_t chunks = rows * cols / 16;
+    if (chunks == 0) return cudaSuccess;
+    QuantArgs a;
+    memset(&a, 0, sizeof(a));
+    a.rows = rows;
+    a.cols = cols;
+    a.total_chunks = chunks;
+    a.cpr = make_fastdiv((uint32_t)(cols / 16 > 0 ? cols / 16 : 1));
+    a.hadamard_b = hadamard_b;
+    a.amax_out = slots;
+    const int64_t steps = (chunks + kQThreads - 1) / kQThreads;
+    const int64_t cap = (int64_t)sm_count_cached() * 2;
+    *n_slots = (int)(steps < cap ? steps : cap);
+    if (bf16) launch_qf<__nv_bfloat16, kNumFmt>((const __nv_bfloat16 *)x, a, s);
+    else launch_qf<float, kNumFmt>((const float *)x, a, s);
+    return cudaGetLastError();
+}
+
 template <typename T, int F>
 static void launch_qf(const T *x, const QuantArgs &a, cudaStream_t s) {
     const int64_t steps = (a.total_chunks + kQThreads - 1) / kQThreads;
@@ -687,8 +729,11 @@ cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols
                             float mx_grid, const float *amax_slots, int n_slots) {
     cudaError_t e;
     if (fmt_tensor_scaled(fmt) && !amax_ready) {
-        e = launch_amax(x, bf16, rows, cols, hadamard_b, amax_word, s);
+        // per-CTA maxima in the scratch behind the amax word (kLrHeader bytes)
+        float *slots = reinterpret_cast<float *>(reinterpret_cast<char *>(amax_word) + 256);
+        e = launch_amax_slots(x, bf16, rows, cols, hadamard_b, slots, &n_slots, s);
         if (e != cudaSuccess) return e;
+        amax_slots = slots;
     }
     QuantArgs a;
     a.rows = rows;

@@ -223,3 +223,38 @@ def test_igroup_ragged_and_degenerate(mxq, orc, fmt):
     ref, _, _ = _ref(orc, fmt, d, 0, rows=_sample_rows(1100, 7))
     y, _, _ = _run(mxq, fmt, d, 0, torch.float32)
     gemm_close(y[torch.from_numpy(_sample_rows(1100, 7)).cuda()].cpu().numpy(), ref)
+
+
+def test_launch_chain_reused_buffers(mxq):
+    """Workload 3's step twice per round, both steps sharing the quantized
+    activation, packed T and workspace, with no synchronization between them:
+    the kernels overlap their setup with the previous kernel but must not read
+    or write global memory before it completes, so every output equals the
+    same step run alone."""
+    d = workloads.svdquant_mlp_up()
+    wq = mxq.quantize(dev(d["w"], "bf16"), 2, 0, mxq.MMA)
+    l1 = dev(d["l1"], "bf16")
+    l2p = mxq.lowrank_pack_l2(dev(d["l2"], "bf16"))
+    m, k = d["x"].shape
+    xs = [dev(d["x"], "bf16"), dev(workloads.svdquant_mlp_up(seed=9, draw_weights=False)["x"], "bf16")]
+    xq = mxq.alloc_qtensor(2, m, k, mxq.MMA)
+    tp = torch.empty((m, 64), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(mxq.quantize_lowrank_workspace_bytes(m, 32), dtype=torch.uint8, device="cuda")
+
+    def step(x, y):
+        mxq.quantize_lowrank(x, 2, l1, wq, 0, out=xq, tp=tp, workspace=ws)
+        mxq.qlinear(xq, wq, tp, l2p, out=y)
+
+    alone = []
+    for x in xs:
+        y = torch.empty((m, wq.rows), dtype=torch.bfloat16, device="cuda")
+        step(x, y)
+        torch.cuda.synchronize()
+        alone.append(y)
+    outs = [torch.empty_like(alone[0]) for _ in range(6)]
+    for i, y in enumerate(outs):
+        step(xs[i % 2], y)
+    torch.cuda.synchronize()
+    assert mxq.check() == 0
+    for i, y in enumerate(outs):
+        assert torch.equal(y, alone[i % 2]), i
