@@ -84,6 +84,21 @@ def test_qlinear_short_k(mxq, orc, fmt):
     gemm_close(y.cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("fmt", GEMM_FMTS)
+def test_qlinear_partial_last_round(mxq, orc, fmt):
+    """81 output tiles of 256 x 256 on 74 clusters (a partly filled last round
+    of the persistent walk), ragged M and N (the last tiles are 152 rows and
+    152 columns), with the low-rank branch where the format takes it; every
+    output element checked."""
+    m, n, k = 2200, 2200, 512
+    r = 32 if fmt in LOWRANK_FMTS else 0
+    d = _inputs(60 + fmt, m, n, k, r)
+    ref, _, _ = _ref(orc, fmt, d, r)
+    for out_dtype in (torch.float32, torch.bfloat16):
+        y, _, _ = _run(mxq, fmt, d, r, out_dtype)
+        gemm_close(y.float().cpu().numpy(), ref, bf16_out=out_dtype == torch.bfloat16)
+
+
 @pytest.mark.parametrize("fmt", LOWRANK_FMTS)
 @pytest.mark.parametrize("r", [8, 32])
 def test_qlinear_lowrank(mxq, orc, fmt, r):
