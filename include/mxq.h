@@ -30,6 +30,11 @@
  *     errors are detected on the host before any launch.  A device-side
  *     bounded wait that runs out is latched in a device error word and
  *     reported by mxq_check().
+ *   - Stream order holds as usual.  The kernels of the activation -> GEMM
+ *     chain (low-rank down projection, quantizer, GEMM) are launched with
+ *     programmatic dependent launch: each may start its setup while the
+ *     previous kernel in the stream finishes, and waits for that kernel to
+ *     complete before its first global read or write.
  */
 #ifndef MXQ_H
 #define MXQ_H
@@ -109,6 +114,14 @@ int mxq_device_supported(int device);
  * Returns MXQ_ETIMEOUT if a bounded wait ran out since the last check,
  * MXQ_ECUDA if a CUDA error is pending, else MXQ_OK.  Host-blocking. */
 mxq_status mxq_check(void *stream);
+
+/* Diagnostics of the error path: launches one thread that waits, for at
+ * most wait_us microseconds (1 .. 1,000,000), on a barrier whose phase never
+ * completes; the bound runs out and the thread latches the device error word
+ * exactly as a stuck wait in the library's kernels would, then returns, so
+ * the next mxq_check returns MXQ_ETIMEOUT and the context stays usable.
+ * Asynchronous on `stream`. */
+mxq_status mxq_selftest_wait_timeout(uint32_t wait_us, void *stream);
 
 /* ---------------------------------------------------------------------- */
 /* Sizes (host only).                                                      */

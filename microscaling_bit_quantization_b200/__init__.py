@@ -29,7 +29,8 @@ F32, BF16 = 0, 1
 STATUS = {0: "MXQ_OK", 1: "MXQ_EINVAL", 2: "MXQ_EUNSUPPORTED", 3: "MXQ_ECUDA", 4: "MXQ_ETIMEOUT", 5: "MXQ_ENOSPACE"}
 
 # Every entry point the header declares.
-EXPORTS = ("mxq_status_string", "mxq_last_cuda_error_string", "mxq_device_supported", "mxq_check", "mxq_codes_bytes", "mxq_scales_bytes",
+EXPORTS = ("mxq_status_string", "mxq_last_cuda_error_string", "mxq_device_supported", "mxq_check",
+           "mxq_selftest_wait_timeout", "mxq_codes_bytes", "mxq_scales_bytes",
            "mxq_quantize_workspace_bytes", "mxq_quantize", "mxq_dequantize", "mxq_hadamard_block", "mxq_cast",
            "mxq_select_workspace_bytes", "mxq_select_weight_format", "mxq_quantize_mse_workspace_bytes",
            "mxq_quantize_mse", "mxq_quantize_mx_grid", "mxq_fit_mx_grid_workspace_bytes", "mxq_fit_mx_grid",
@@ -69,6 +70,7 @@ def _load():
         "mxq_scales_bytes": (i32, [i32, i64, i64, i32, psz]),
         "mxq_quantize_workspace_bytes": (i32, [i32, psz]),
         "mxq_quantize": (i32, [P, i32, i64, i64, i32, i32, i32, P, P, P, P, sz, P]),
+        "mxq_selftest_wait_timeout": (i32, [ctypes.c_uint32, P]),
         "mxq_dequantize": (i32, [ctypes.POINTER(_QTensorC), P, i32, P]),
         "mxq_hadamard_block": (i32, [P, P, i32, i64, i64, i32, P]),
         "mxq_cast": (i32, [P, i64, i32, P, P]),

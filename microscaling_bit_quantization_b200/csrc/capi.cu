@@ -77,6 +77,11 @@ mxq_status mxq_check(void *stream) {
     return w ? MXQ_ETIMEOUT : MXQ_OK;
 }
 
+mxq_status mxq_selftest_wait_timeout(uint32_t wait_us, void *stream) {
+    if (wait_us < 1 || wait_us > 1000000) return MXQ_EINVAL;
+    return from_cuda(launch_wait_selftest(1000ull * wait_us, (cudaStream_t)stream));
+}
+
 mxq_status mxq_codes_bytes(int32_t fmt, int64_t rows, int64_t cols, int32_t layout, size_t *bytes) {
     if (!valid_fmt(fmt) || !valid_layout(layout) || !bytes || !valid_shape(fmt, rows, cols)) return MXQ_EINVAL;
     const bool int4_unpacked = (fmt == MXQ_INT4_G32 || fmt == MXQ_INT4_G64) && layout == MXQ_LAYOUT_MMA;

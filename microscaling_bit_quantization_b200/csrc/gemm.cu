@@ -687,6 +687,26 @@ cudaError_t launch_qlinear(const GemmOperands &op, cudaStream_t s) {
     }
 }
 
+namespace {
+constexpr unsigned int kErrSelfTest = 64u;
+
+// Self-test of the bounded waits and the error word: one thread waits on an
+// mbarrier that nothing arrives on (its first phase never completes); when
+// the bound runs out it latches the error word as every bounded wait of the
+// library's kernels does, and the kernel returns.
+__global__ void k_wait_selftest(unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    if (!mbar_wait(&bar, 0, limit_ns)) latch_error(kErrSelfTest);
+}
+}  // namespace
+
+cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t s) {
+    k_wait_selftest<<<1, 32, 0, s>>>(limit_ns);
+    return cudaGetLastError();
+}
+
 cudaError_t error_word_address(unsigned int **ptr) {
     static unsigned int *addr[64] = {};
     int dev = 0;

@@ -116,6 +116,8 @@ bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint6
 // Device error word (bounded waits that ran out); read-and-clear, and its
 // device address on the current device (for kernels of other files).
 cudaError_t read_and_clear_error(unsigned int *value);
+// One bounded wait that runs out (gemm.cu): latches the error word.
+cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t s);
 cudaError_t error_word_address(unsigned int **ptr);
 
 }  // namespace mxq

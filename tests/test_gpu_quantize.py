@@ -395,3 +395,20 @@ def test_calibrate_full_size(mxq, orc):
     torch.cuda.synchronize()
     np.testing.assert_allclose(sse.cpu().numpy(), ref_sse, rtol=1e-12)
     np.testing.assert_array_equal(mom.cpu().numpy(), ref_mom)
+
+
+# ------------------------------------------------------------------ error path
+
+def test_bounded_wait_reports_timeout(mxq, orc):
+    """A bounded device wait that runs out is latched in the error word and
+    reported by mxq_check (MXQ_ETIMEOUT = 4), which clears it; the context
+    stays usable (no trap, fault or unbounded loop is involved)."""
+    assert mxq.check() == 0
+    assert mxq.lib().mxq_selftest_wait_timeout(20000, None) == 0   # 20 ms
+    assert mxq.check() == 4
+    assert mxq.check() == 0
+    x = nasty_matrix(71, 37, 512)
+    q = mxq.quantize(dev(x, "f32"), mxq.NVFP4)
+    torch.cuda.synchronize()
+    assert_qtensor_equal(q, orc.quantize(x, mxq.NVFP4))
+    assert mxq.lib().mxq_selftest_wait_timeout(0, None) == 1        # bound outside 1 us .. 1 s
