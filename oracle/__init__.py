@@ -93,6 +93,8 @@ def lib():
         L.orc_mx_grid_sse.argtypes = [P, i64, i64, i32, i32, P, i32, P, P, P, P]
         L.orc_calibrate_activation.restype = i32
         L.orc_calibrate_activation.argtypes = [P, i64, i64, P, i32, P, P, P, P, P, P, P]
+        L.orc_w4a16_weights.restype = i32
+        L.orc_w4a16_weights.argtypes = [P, P, i64, i64, i32, P]
         L.orc_lowrank_down.restype = i32
         L.orc_lowrank_down.argtypes = [P, P, i64, i64, i32, P]
         L.orc_route.restype = i32
@@ -366,6 +368,26 @@ def qlinear(xq: QTensor, wq: QTensor, t=None, l2=None, rows=None) -> np.ndarray:
     if t is not None:
         y = y + np.asarray(t, np.float64) @ np.asarray(l2, np.float64)
     return y
+
+
+def w4a16_weights(wq: QTensor) -> np.ndarray:
+    """bf16(RN32(q s)) of every weight of an INT4-g32/g64 tensor (mxq_oracle.c,
+    orc_w4a16_weights), as fp32 values."""
+    g = BLOCK[wq.fmt]
+    w = np.empty((wq.rows, wq.cols), np.float32)
+    st = lib().orc_w4a16_weights(_ptr(wq.codes), _ptr(np.ascontiguousarray(wq.scales, np.float32)), wq.rows, wq.cols,
+                                 g, _ptr(w))
+    if st != 0:
+        raise OracleError("bad w4a16 arguments")
+    return w
+
+
+def w4a16(x, wq: QTensor, rows=None) -> np.ndarray:
+    """Y = bf16(X) . W16^T in binary64, W16 = w4a16_weights(wq)."""
+    xb = round_bf16_array(x).astype(np.float64)
+    if rows is not None:
+        xb = xb[np.asarray(rows)]
+    return xb @ w4a16_weights(wq).astype(np.float64).T
 
 
 # ---------------------------------------------------------------- routing

@@ -781,6 +781,29 @@ int orc_calibrate_activation(const float *x, int64_t rows, int64_t cols, const i
 }
 
 /* ------------------------------------------------------------------ */
+/* W4A16 weights (Nunchaku/Diffusers article, awq_w4a16: 4-bit         */
+/* per-group weights against 16-bit activations).  Reading: a weight   */
+/* is dequantized the way a kernel feeding 16-bit tensor cores does    */
+/* it, w = bf16(RN32(q * s)) with q the signed INT4 code and s the     */
+/* group's fp32 scale (canonical INT4 layout); the product with        */
+/* bf16(x) is then summed (binary64 here, by the caller).               */
+/* ------------------------------------------------------------------ */
+
+int orc_w4a16_weights(const uint8_t *codes, const float *scales, int64_t n, int64_t k, int g, float *w)
+{
+    if (n < 0 || k < 0 || (g != 32 && g != 64) || k % g) return ORC_EINVAL;
+    for (int64_t r = 0; r < n; r++)
+        for (int64_t c = 0; c < k; c++) {
+            int64_t idx = r * k + c;
+            int q = get_code(codes, idx, 1);
+            if (q & 8) q -= 16;
+            float prod = (float)q * scales[r * (k / g) + c / g];
+            w[idx] = orc_round_bf16(prod);
+        }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
 /* SVDQuant low-rank branch, down projection (Nunchaku/Diffusers       */
 /* article, section "Main explanation": a 16-bit low-rank part of the  */
 /* weight is kept beside the 4-bit residual).                          */

@@ -706,6 +706,41 @@ def test_calibration_pick_is_least_recomputed_error(orc):
         assert orc.calibrate_pick(sse, cands, orc.MXFP8) == orc.MXFP8
 
 
+# ------------------------------------------------------------------ W4A16
+
+def test_w4a16_weights_against_torch(orc):
+    # every INT4 code against many scales: bf16(RN32(q s)) by torch's own
+    # fp32 multiply and bf16 cast
+    rng = np.random.default_rng(81)
+    k, g = 64, 32
+    q = np.tile(np.arange(-7, 8), 30)[: 7 * k].reshape(7, k)
+    s = (np.exp(rng.uniform(-30, 30, size=(7, k // g))) * rng.choice([1, 1.0 + 2 ** -20], (7, k // g))).astype(np.float32)
+    s[0, 0] = np.float32(1.0 / 3.0)
+    nib = (q & 0xF).astype(np.uint8)
+    codes = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+    wq = orc.QTensor(orc.INT4_G32, 7, k, codes, s, 0.0)
+    w = orc.w4a16_weights(wq)
+    ref = (torch.from_numpy(q.astype(np.float32)) * torch.from_numpy(np.repeat(s, g, axis=1))).to(torch.bfloat16)
+    assert np.array_equal(w.view(np.uint32), ref.float().numpy().view(np.uint32))
+
+
+def test_w4a16_brute_force_tiny(orc):
+    rng = np.random.default_rng(82)
+    x = rng.standard_normal((3, 128)).astype(np.float32)
+    w = (rng.standard_normal((5, 128)) * 0.05).astype(np.float32)
+    for fmt in (orc.INT4_G32, orc.INT4_G64):
+        wq = orc.quantize(w, fmt)
+        y = orc.w4a16(x, wq)
+        w16 = orc.w4a16_weights(wq)
+        for i in range(3):
+            for j in range(5):
+                acc = math.fsum(float(orc.round_bf16(float(x[i, c]))) * float(w16[j, c]) for c in range(128))
+                assert y[i, j] == pytest.approx(acc, rel=1e-14, abs=1e-300)
+        # the bf16 weights stay within half a bf16 ulp (plus the fp32 step) of the exact dequantization
+        exact = wq.dequantize()
+        assert np.all(np.abs(w16 - exact) <= np.abs(exact) * (2.0 ** -8 + 2.0 ** -24) + 1e-45)   # 8-bit significand
+
+
 # ------------------------------------------------------------------ low rank + GEMM
 
 def test_lowrank_down_brute_force(orc):
