@@ -404,6 +404,16 @@ def run_ours(args, world, rank, local):
                  "us": 1e3 * cal_ms, "GB/s": xc.numel() * 2 / (cal_ms * 1e-3) / 1e9,
                  "frac": xc.numel() * 2 / (cal_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
     del xc, c_ws
+    # W4A16: the same weight as canonical INT4-g64, dequantized to bf16 in shared memory, bf16 activations
+    wq16 = mxq.quantize(w4d, mxq.INT4_G64)
+    y16 = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    w16_ms = graph_ms(lambda i: mxq.qlinear_w4a16(sets[i % N_SETS]["x"], wq16, out=y16), n=4, reps=3)
+    w16_tf = FLOP_MAIN / (w16_ms * 1e-3) / 1e12
+    w4a16_row = {"kernel": "k_w4a16 (INT4-g64 weights dequantized to bf16 in shared memory, kind::f16, "
+                           "X 4096 x 3072 bf16, W 12288 x 3072)",
+                 "us": 1e3 * w16_ms, "TFLOP/s": w16_tf, "frac_of_bf16_peak": w16_tf / peaks["bf16_tflops"],
+                 "bf16_peak": peaks["bf16_tflops"]}
+    del wq16, y16
     wq4 = mxq.quantize(w4d, mxq.INT4_G64, 0, mxq.MMA)
     del w4d
     xq4 = mxq.quantize(sets[0]["x"], mxq.INT4_G64, 0, mxq.MMA)
@@ -473,6 +483,7 @@ def run_ours(args, world, rank, local):
             "select_weight_format": select,
             "quantize_mse_nvfp4": mse_row,
             "fit_mx_grid": grid_row,
+            "w4a16_qlinear": w4a16_row,
             "calibrate_activation": calib_row,
             "lowrank_down": lowrank,
             "e2e": {"value": world * FLOP_STEP / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",

@@ -389,6 +389,18 @@ mxq_status mxq_quantize_lowrank_noalloc(const void *x, int32_t xdtype, int64_t m
                                         const float *w_tensor_scale, void *codes, void *scales,
                                         float *tensor_scale, void *tp, void *stream);
 
+/* W4A16 linear (Nunchaku/Diffusers article, awq_w4a16: 4-bit per-group
+ * weights against 16-bit activations): y = bf16(x) . W16^T with
+ * W16 = bf16(RN32(q s)), q the signed INT4 code and s its group's fp32
+ * scale, fp32 accumulation on tcgen05 tensor cores; the weights are
+ * dequantized in shared memory, stage by stage, never written out.
+ *   x: m x k bf16 device (16-byte aligned); wq: INT4_G32 or INT4_G64 in the
+ *   canonical layout (mxq_quantize), wq->cols == k; y: m x wq->rows device,
+ *   ydtype MXQ_BF16 or MXQ_F32.
+ * Constraints: k % 64 == 0.  Other formats: MXQ_EUNSUPPORTED. */
+mxq_status mxq_qlinear_w4a16(const void *x, int64_t m, int64_t k, const mxq_qtensor *wq, void *y,
+                             int32_t ydtype, void *stream);
+
 /* Re-lays the up-projection l2 (r x n bf16, device) as the GEMM operand
  * l2p (n x 64 bf16, device): row j of l2p holds l2[0..r-1][j], zeros up to
  * 32, then the same 32 values again (the operand of the split high/low

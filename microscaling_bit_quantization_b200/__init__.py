@@ -36,7 +36,7 @@ EXPORTS = ("mxq_status_string", "mxq_last_cuda_error_string", "mxq_device_suppor
            "mxq_quantize_mse", "mxq_quantize_mx_grid", "mxq_fit_mx_grid_workspace_bytes", "mxq_fit_mx_grid",
            "mxq_calibrate_workspace_bytes", "mxq_calibrate_activation", "mxq_calibrate_pick",
            "mxq_lowrank_down", "mxq_lowrank_packed_bytes",
-           "mxq_lowrank_down_packed", "mxq_lowrank_pack_t", "mxq_lowrank_pack_l2", "mxq_qlinear", "mxq_route",
+           "mxq_lowrank_down_packed", "mxq_lowrank_pack_t", "mxq_lowrank_pack_l2", "mxq_qlinear", "mxq_qlinear_w4a16", "mxq_route",
            "mxq_quantize_lowrank_workspace_bytes", "mxq_quantize_lowrank", "mxq_quantize_lowrank_noalloc")
 
 
@@ -90,6 +90,7 @@ def _load():
         "mxq_lowrank_pack_t": (i32, [P, i32, i64, P, P, P, P]),
         "mxq_lowrank_pack_l2": (i32, [P, i32, i64, P, P]),
         "mxq_qlinear": (i32, [ctypes.POINTER(_QTensorC), ctypes.POINTER(_QTensorC), P, P, P, i32, P]),
+        "mxq_qlinear_w4a16": (i32, [P, i64, i64, ctypes.POINTER(_QTensorC), P, i32, P]),
         "mxq_route": (i32, [P, i32, i32, i32, i32, i32]),
         "mxq_quantize_lowrank_workspace_bytes": (i32, [i64, i32, psz]),
         "mxq_quantize_lowrank": (i32, [P, i32, i64, i64, i32, i32, P, i32, P, P, P, P, P, P, sz, P]),
@@ -430,6 +431,20 @@ def qlinear(xq: QTensor, wq: QTensor, tp: torch.Tensor = None, l2p: torch.Tensor
     xc, wc = xq.c(), wq.c()
     _ok(_lib.mxq_qlinear(ctypes.byref(xc), ctypes.byref(wc), _ptr(tp), _ptr(l2p), _ptr(y), _dtype_code(y),
                          _stream(stream)), "mxq_qlinear")
+    return y
+
+
+def qlinear_w4a16(x: torch.Tensor, wq: QTensor, out_dtype=torch.bfloat16, out: torch.Tensor = None,
+                  stream=None) -> torch.Tensor:
+    """y = bf16(x) . bf16(q s)^T for an INT4-g32/g64 weight in the canonical layout."""
+    _require_cuda(x)
+    assert x.dtype == torch.bfloat16
+    x = x.contiguous()
+    m, k = x.shape
+    y = out if out is not None else torch.empty((m, wq.rows), dtype=out_dtype, device=x.device)
+    wc = wq.c()
+    _ok(_lib.mxq_qlinear_w4a16(_ptr(x), m, k, ctypes.byref(wc), _ptr(y), _dtype_code(y), _stream(stream)),
+        "mxq_qlinear_w4a16")
     return y
 
 

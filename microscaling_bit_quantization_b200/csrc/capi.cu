@@ -373,6 +373,18 @@ mxq_status mxq_quantize_lowrank(const void *x, int32_t xdtype, int64_t m, int64_
                                      amax, s, &pack, amax_ready, 1.0f, slots, n_slots));
 }
 
+mxq_status mxq_qlinear_w4a16(const void *x, int64_t m, int64_t k, const mxq_qtensor *wq, void *y, int32_t ydtype,
+                             void *stream) {
+    if (!wq || !valid_dtype(ydtype) || m < 0 || k <= 0 || k % 64) return MXQ_EINVAL;
+    if (wq->fmt != MXQ_INT4_G32 && wq->fmt != MXQ_INT4_G64) return MXQ_EUNSUPPORTED;
+    if (wq->layout != MXQ_LAYOUT_CANONICAL || wq->cols != k || wq->rows < 0) return MXQ_EINVAL;
+    if (m >= ((int64_t)1 << 31) || wq->rows >= ((int64_t)1 << 31) || k >= ((int64_t)1 << 31)) return MXQ_EINVAL;
+    if (m > 0 && wq->rows > 0 && (!x || !y || !wq->codes || !wq->scales || !aligned16(x) || !aligned16(wq->codes)))
+        return MXQ_EINVAL;
+    return from_cuda(launch_w4a16(x, m, k, (const uint8_t *)wq->codes, (const float *)wq->scales, wq->rows,
+                                  wq->fmt == MXQ_INT4_G32 ? 32 : 64, y, ydtype == MXQ_BF16, (cudaStream_t)stream));
+}
+
 mxq_status mxq_lowrank_pack_l2(const void *l2, int32_t r, int64_t n, void *l2p, void *stream) {
     if (r < 1 || r > 32 || n < 0) return MXQ_EINVAL;
     if (n > 0 && (!l2 || !l2p || !aligned16(l2p))) return MXQ_EINVAL;

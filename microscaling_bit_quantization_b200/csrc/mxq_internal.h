@@ -116,6 +116,10 @@ bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint6
 // Device error word (bounded waits that ran out); read-and-clear, and its
 // device address on the current device (for kernels of other files).
 cudaError_t read_and_clear_error(unsigned int *value);
+// W4A16 linear (w4a16.cu): y = bf16(x) . bf16(RN32(q s))^T, x m x k bf16,
+// codes n x k/2 canonical INT4, scales n x k/g fp32; k % 64 == 0.
+cudaError_t launch_w4a16(const void *x, int64_t m, int64_t k, const uint8_t *codes, const float *scales, int64_t n,
+                         int g, void *y, bool y_bf16, cudaStream_t s);
 // One bounded wait that runs out (gemm.cu): latches the error word.
 cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t s);
 cudaError_t error_word_address(unsigned int **ptr);

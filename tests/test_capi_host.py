@@ -137,6 +137,22 @@ def test_calibration_argument_checks(mxq):
     assert pick(None, c3, 3, -1, d, None) == 1
 
 
+def test_w4a16_argument_checks(mxq):
+    L = mxq.lib()
+    P = ctypes.c_void_p
+    d = P(256)
+
+    def qt(fmt, layout, rows, cols):
+        return mxq._QTensorC(fmt, layout, rows, cols, 256, 256, None)
+
+    call = lambda q, k=128, yd=1: L.mxq_qlinear_w4a16(d, 4, k, ctypes.byref(q), d, yd, None)
+    assert call(qt(mxq.NVFP4, 0, 8, 128)) == 2            # INT4 groups only
+    assert call(qt(mxq.INT4_G64, 1, 8, 128)) == 1         # canonical layout only
+    assert call(qt(mxq.INT4_G64, 0, 8, 96), k=96) == 1    # k % 64
+    assert call(qt(mxq.INT4_G64, 0, 8, 192), k=128) == 1  # cols != k
+    assert call(qt(mxq.INT4_G32, 0, 8, 128), yd=7) == 1   # bad output dtype
+
+
 def test_qlinear_argument_checks(mxq):
     L = mxq.lib()
     Q = mxq._QTensorC

@@ -273,3 +273,36 @@ def test_launch_chain_reused_buffers(mxq):
     assert mxq.check() == 0
     for i, y in enumerate(outs):
         assert torch.equal(y, alone[i % 2]), i
+
+
+# ------------------------------------------------------------------ W4A16
+
+@pytest.mark.parametrize("fmt", [4, 3])
+@pytest.mark.parametrize("shape", [(37, 200, 512), (300, 260, 192), (129, 128, 64), (1, 8, 128)])
+def test_w4a16_small(mxq, orc, fmt, shape):
+    """bf16 activations x INT4-g64 / g32 weights (canonical layout), ragged M
+    and N, one K stage up to eight; every element against the oracle."""
+    m, n, k = shape
+    d = _inputs(90 + fmt, m, n, k)
+    xv = host_values(d["x"], "bf16")
+    wq = mxq.quantize(dev(d["w"], "bf16"), fmt)
+    owq = orc.quantize(host_values(d["w"], "bf16"), fmt)
+    assert_qtensor_equal(wq, owq)
+    ref = orc.w4a16(xv, owq)
+    for out_dtype in (torch.float32, torch.bfloat16):
+        y = mxq.qlinear_w4a16(dev(d["x"], "bf16"), wq, out_dtype=out_dtype)
+        assert mxq.check() == 0
+        gemm_close(y.float().cpu().numpy(), ref, bf16_out=out_dtype == torch.bfloat16)
+
+
+def test_w4a16_full_size(mxq, orc):
+    """Workload 3's shape with its residual weight as INT4-g64: 256 sampled
+    rows (all 12288 columns) against the oracle."""
+    d = workloads.svdquant_mlp_up()
+    wq = mxq.quantize(dev(d["w"], "bf16"), 4)
+    owq = orc.quantize(d["w"], 4)
+    rows = _sample_rows(4096, 91)
+    ref = orc.w4a16(d["x"], owq, rows=rows)
+    y = mxq.qlinear_w4a16(dev(d["x"], "bf16"), wq)
+    assert mxq.check() == 0
+    gemm_close(y[torch.from_numpy(rows).cuda()].float().cpu().numpy(), ref, bf16_out=True)
