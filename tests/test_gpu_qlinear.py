@@ -306,3 +306,42 @@ def test_w4a16_full_size(mxq, orc):
     y = mxq.qlinear_w4a16(dev(d["x"], "bf16"), wq)
     assert mxq.check() == 0
     gemm_close(y[torch.from_numpy(rows).cuda()].float().cpu().numpy(), ref, bf16_out=True)
+
+
+def test_launch_chain_in_cuda_graph(mxq):
+    """The fused activation path and the GEMM captured in a CUDA graph (the
+    programmatic launches become programmatic graph edges) give, on replay,
+    exactly the outputs of the same calls run eagerly."""
+    d = workloads.svdquant_mlp_up(m=1024, n=2048)
+    wq = mxq.quantize(dev(d["w"], "bf16"), 2, 0, mxq.MMA)
+    l1 = dev(d["l1"], "bf16")
+    l2p = mxq.lowrank_pack_l2(dev(d["l2"], "bf16"))
+    x = dev(d["x"], "bf16")
+    m, k = x.shape
+    xq = mxq.alloc_qtensor(2, m, k, mxq.MMA)
+    tp = torch.empty((m, 64), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(mxq.quantize_lowrank_workspace_bytes(m, 32), dtype=torch.uint8, device="cuda")
+    y_eager = torch.empty((m, wq.rows), dtype=torch.bfloat16, device="cuda")
+    y_graph = torch.empty_like(y_eager)
+
+    def step(y):
+        mxq.quantize_lowrank(x, 2, l1, wq, 0, out=xq, tp=tp, workspace=ws)
+        mxq.qlinear(xq, wq, tp, l2p, out=y)
+
+    step(y_eager)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step(y_graph)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(3):
+            step(y_graph)
+    y_graph.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert mxq.check() == 0
+    assert torch.equal(y_graph, y_eager)
