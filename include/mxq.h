@@ -397,7 +397,8 @@ mxq_status mxq_quantize_lowrank_noalloc(const void *x, int32_t xdtype, int64_t m
  *   x: m x k bf16 device (16-byte aligned); wq: INT4_G32 or INT4_G64 in the
  *   canonical layout (mxq_quantize), wq->cols == k; y: m x wq->rows device,
  *   ydtype MXQ_BF16 or MXQ_F32.
- * Constraints: k % 64 == 0.  Other formats: MXQ_EUNSUPPORTED. */
+ * Constraints: k % 64 == 0; ceil(m/128) * ceil(n/128) * k/64 < 2^31.
+ * Other formats: MXQ_EUNSUPPORTED. */
 mxq_status mxq_qlinear_w4a16(const void *x, int64_t m, int64_t k, const mxq_qtensor *wq, void *y,
                              int32_t ydtype, void *stream);
 
@@ -425,7 +426,8 @@ mxq_status mxq_lowrank_pack_l2(const void *l2, int32_t r, int64_t n, void *l2p, 
  *     (n rows).  The branch is supported for every fmt but INT8_ROW.
  *   y: m x n device, fp32 or bf16 (fp32 result rounded once, RNE).
  * Constraints: K % 64 == 0 (NVFP4, MXFP4), K % g == 0 (INT4_Gg) or
- * K % 32 == 0 (8-bit); K > 0; device pointers 16-byte aligned.
+ * K % 32 == 0 (8-bit); K > 0; ceil(m/128) * ceil(n/128) * K/16 < 2^31;
+ * device pointers 16-byte aligned.
  * Errors: MXQ_EINVAL, MXQ_EUNSUPPORTED (format pair / branch), MXQ_ECUDA.
  * A pipeline wait that runs out is reported by mxq_check(). */
 mxq_status mxq_qlinear(const mxq_qtensor *xq, const mxq_qtensor *wq, const void *tp, const void *l2p,

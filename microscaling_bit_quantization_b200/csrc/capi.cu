@@ -379,6 +379,8 @@ mxq_status mxq_qlinear_w4a16(const void *x, int64_t m, int64_t k, const mxq_qten
     if (wq->fmt != MXQ_INT4_G32 && wq->fmt != MXQ_INT4_G64) return MXQ_EUNSUPPORTED;
     if (wq->layout != MXQ_LAYOUT_CANONICAL || wq->cols != k || wq->rows < 0) return MXQ_EINVAL;
     if (m >= ((int64_t)1 << 31) || wq->rows >= ((int64_t)1 << 31) || k >= ((int64_t)1 << 31)) return MXQ_EINVAL;
+    // the kernel counts 128 x 128 tiles and their 64-column stages in 32-bit integers
+    if (((m + 127) / 128) * ((wq->rows + 127) / 128) * (k / 64) >= ((int64_t)1 << 31)) return MXQ_EINVAL;
     if (m > 0 && wq->rows > 0 && (!x || !y || !wq->codes || !wq->scales || !aligned16(x) || !aligned16(wq->codes)))
         return MXQ_EINVAL;
     return from_cuda(launch_w4a16(x, m, k, (const uint8_t *)wq->codes, (const float *)wq->scales, wq->rows,
@@ -402,6 +404,8 @@ mxq_status mxq_qlinear(const mxq_qtensor *xq, const mxq_qtensor *wq, const void 
     if (wq->cols != k || k <= 0 || m < 0 || n < 0) return MXQ_EINVAL;
     if (k % (igroup ? fmt_block(fmt) : fmt_is4(fmt) ? 64 : 32)) return MXQ_EINVAL;
     if (!valid_shape(fmt, m, k) || !valid_shape(fmt, n, k)) return MXQ_EINVAL;
+    // the kernels count output tiles and their K stages in 32-bit integers
+    if (((m + 127) / 128) * ((n + 127) / 128) * (k / 16) >= ((int64_t)1 << 31)) return MXQ_EINVAL;
     if (m > 0 && n > 0) {
         if (!xq->codes || !wq->codes || !aligned16(xq->codes) || !aligned16(wq->codes) || !aligned16(y))
             return MXQ_EINVAL;

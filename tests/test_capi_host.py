@@ -151,6 +151,8 @@ def test_w4a16_argument_checks(mxq):
     assert call(qt(mxq.INT4_G64, 0, 8, 96), k=96) == 1    # k % 64
     assert call(qt(mxq.INT4_G64, 0, 8, 192), k=128) == 1  # cols != k
     assert call(qt(mxq.INT4_G32, 0, 8, 128), yd=7) == 1   # bad output dtype
+    big = qt(mxq.INT4_G64, 0, (1 << 31) - 1, 1 << 20)
+    assert L.mxq_qlinear_w4a16(d, (1 << 31) - 1, 1 << 20, ctypes.byref(big), d, 1, None) == 1   # stage count
 
 
 def test_qlinear_argument_checks(mxq):
@@ -170,6 +172,9 @@ def test_qlinear_argument_checks(mxq):
     assert L.mxq_qlinear(ctypes.byref(i4), ctypes.byref(i4), None, None, y, 0, None) == 1   # layout
     a = Q(mxq.NVFP4, mxq.MMA, 64, 96, 256, 256, 256)
     assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(a), None, None, y, 0, None) == 1   # K % 64
+    big_a = Q(mxq.MXFP8, mxq.MMA, 1 << 26, 32, 256, 256, 0)
+    big_b = Q(mxq.MXFP8, mxq.MMA, 1 << 26, 32, 256, 256, 0)
+    assert L.mxq_qlinear(ctypes.byref(big_a), ctypes.byref(big_b), None, None, y, 0, None) == 1   # tile count
     i8 = Q(mxq.INT8_ROW, mxq.MMA, 64, 256, 256, 256, 0)
     t = ctypes.c_void_p(256)
     assert L.mxq_qlinear(ctypes.byref(i8), ctypes.byref(i8), t, t, y, 0, None) == 2       # branch on INT8
