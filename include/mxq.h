@@ -120,7 +120,8 @@ mxq_status mxq_check(void *stream);
  * completes; the bound runs out and the thread latches the device error word
  * exactly as a stuck wait in the library's kernels would, then returns, so
  * the next mxq_check returns MXQ_ETIMEOUT and the context stays usable.
- * Asynchronous on `stream`. */
+ * Asynchronous on `stream`.  Errors: MXQ_EINVAL (wait_us out of range),
+ * MXQ_ECUDA. */
 mxq_status mxq_selftest_wait_timeout(uint32_t wait_us, void *stream);
 
 /* ---------------------------------------------------------------------- */
@@ -238,7 +239,9 @@ mxq_status mxq_quantize_mse_workspace_bytes(int64_t rows, int64_t cols, size_t *
  *   workspace: device scratch of mxq_quantize_mse_workspace_bytes, 256-byte
  *     aligned; clobbered.
  * Constraints as mxq_quantize (cols % 16 == 0, 16-byte aligned w and
- * codes); rows * cols / 16 < 2^31.  Bit-identical from run to run. */
+ * codes); rows * cols / 16 < 2^31.  Bit-identical from run to run.
+ * Errors: MXQ_EINVAL (shape / pointer / iters < 0 / workspace alignment),
+ * MXQ_EUNSUPPORTED (fmt), MXQ_ENOSPACE (workspace), MXQ_ECUDA. */
 mxq_status mxq_quantize_mse(const void *w, int32_t wdtype, int64_t rows, int64_t cols, int32_t fmt,
                             int32_t iters, int32_t layout, void *codes, void *scales,
                             float *tensor_scale, double *sse, void *workspace,
@@ -253,7 +256,8 @@ mxq_status mxq_quantize_mse(const void *w, int32_t wdtype, int64_t rows, int64_t
  * exact); g = 1 is mxq_quantize's OCP rule, g = 4/3 the rule under which
  * E2M1 never clips.  Elements, scales and layouts as mxq_quantize.
  *   fmt: MXQ_MXFP4 or MXQ_MXFP8 (others MXQ_EUNSUPPORTED); g outside [1, 2]:
- *     MXQ_EINVAL.  Other arguments and constraints as mxq_quantize. */
+ *     MXQ_EINVAL.  Other arguments and constraints as mxq_quantize.
+ * Errors: MXQ_EINVAL, MXQ_EUNSUPPORTED, MXQ_ECUDA. */
 mxq_status mxq_quantize_mx_grid(const void *x, int32_t xdtype, int64_t rows, int64_t cols, int32_t fmt,
                                 int32_t hadamard_b, float grid_scale, int32_t layout, void *codes,
                                 void *scales, void *stream);
@@ -273,7 +277,9 @@ mxq_status mxq_fit_mx_grid_workspace_bytes(int64_t rows, int64_t cols, int32_t n
  *   sse: device double[n].
  *   workspace: device scratch of mxq_fit_mx_grid_workspace_bytes, 256-byte
  *     aligned; clobbered.
- * Other arguments and constraints as mxq_quantize_mx_grid. */
+ * Other arguments and constraints as mxq_quantize_mx_grid.
+ * Errors: MXQ_EINVAL (shape / pointer / candidates / workspace alignment),
+ * MXQ_EUNSUPPORTED (fmt), MXQ_ENOSPACE (workspace), MXQ_ECUDA. */
 mxq_status mxq_fit_mx_grid(const void *w, int32_t wdtype, int64_t rows, int64_t cols, int32_t fmt,
                            int32_t hadamard_b, const float *grid_scales, int32_t n, double *sse,
                            void *workspace, size_t workspace_bytes, void *stream);
@@ -298,7 +304,9 @@ mxq_status mxq_fit_mx_grid(const void *w, int32_t wdtype, int64_t rows, int64_t 
  * above).  Zero the accumulators before an entry's first activation.
  *   candidates: host array of 1..8 mxq_fmt values; cols % 64 == 0.
  *   workspace: device scratch of mxq_calibrate_workspace_bytes, 256-byte
- *     aligned; clobbered. */
+ *     aligned; clobbered.
+ * Errors: MXQ_EINVAL (shape / pointer / candidates / workspace alignment),
+ * MXQ_ENOSPACE (workspace), MXQ_ECUDA. */
 mxq_status mxq_calibrate_workspace_bytes(int64_t rows, int64_t cols, int32_t ncand, size_t *bytes);
 mxq_status mxq_calibrate_activation(const void *x, int32_t xdtype, int64_t rows, int64_t cols,
                                     const int32_t *candidates, int32_t ncand, double *sse_accum,
@@ -307,7 +315,8 @@ mxq_status mxq_calibrate_activation(const void *x, int32_t xdtype, int64_t rows,
 
 /* Writes one table entry (device uint8): forced_fmt when >= 0 (layers the
  * article pins to MXFP8), else the candidate with the least sse_accum
- * (device double[ncand]), ties to the lower candidate index. */
+ * (device double[ncand]), ties to the lower candidate index.
+ * Errors: MXQ_EINVAL (pointers / candidates / forced_fmt), MXQ_ECUDA. */
 mxq_status mxq_calibrate_pick(const double *sse_accum, const int32_t *candidates, int32_t ncand,
                               int32_t forced_fmt, uint8_t *entry, void *stream);
 
@@ -398,7 +407,9 @@ mxq_status mxq_quantize_lowrank_noalloc(const void *x, int32_t xdtype, int64_t m
  *   canonical layout (mxq_quantize), wq->cols == k; y: m x wq->rows device,
  *   ydtype MXQ_BF16 or MXQ_F32.
  * Constraints: k % 64 == 0; ceil(m/128) * ceil(n/128) * k/64 < 2^31.
- * Other formats: MXQ_EUNSUPPORTED. */
+ * Errors: MXQ_EINVAL (shape / layout / pointer / ydtype), MXQ_EUNSUPPORTED
+ * (formats other than INT4_G32 / INT4_G64), MXQ_ECUDA; a pipeline wait that
+ * runs out is reported by mxq_check(). */
 mxq_status mxq_qlinear_w4a16(const void *x, int64_t m, int64_t k, const mxq_qtensor *wq, void *y,
                              int32_t ydtype, void *stream);
 
