@@ -30,6 +30,12 @@
  *     errors are detected on the host before any launch.  A device-side
  *     bounded wait that runs out is latched in a device error word and
  *     reported by mxq_check().
+ *   - The library keeps state per device for the life of the process: the
+ *     device addresses of its own device variables (the error word, the
+ *     scratch array of the allocation-free entry point) and the kernels'
+ *     shared-memory opt-ins, set up on a device's first use.  A
+ *     cudaDeviceReset() discards what that state refers to, so the library
+ *     must not be used on a device after the device has been reset.
  *   - Stream order holds as usual.  The kernels of the activation -> GEMM
  *     chain (low-rank down projection, quantizer, GEMM) are launched with
  *     programmatic dependent launch: each may start its setup while the
@@ -455,6 +461,59 @@ mxq_status mxq_qlinear(const mxq_qtensor *xq, const mxq_qtensor *wq, const void 
  * -1 for out-of-range arguments.  Host only, no CUDA call. */
 int32_t mxq_route(const uint8_t *table, int32_t n_layers, int32_t n_intervals, int32_t layer,
                   int32_t step, int32_t n_steps);
+
+/* One linear layer prepared for routed execution: its weight quantized
+ * once, in the MMA layout, in every format its row of the format table can
+ * name, and the optional low-rank branch.
+ *   w[f]: the weight (N x K) in format f (w[f].fmt == f, layout MMA), or
+ *     w[f].codes == NULL when the layer is never routed to f.  All prepared
+ *     entries have the same rows (N) and cols (K).
+ *   l1: K x r bf16 device, the down projection (NULL: no branch, r = 0);
+ *   l2p: the packed up projection (mxq_lowrank_pack_l2, N rows).
+ *   hadamard_b: 0, or the block-diagonal rotation size the weights were
+ *     quantized with; the activation is rotated the same way. */
+typedef struct mxq_layer {
+    mxq_qtensor w[MXQ_NUM_FMT];
+    const void *l1;
+    const void *l2p;
+    int32_t r;
+    int32_t hadamard_b;
+} mxq_layer;
+
+/* Scratch bytes mxq_qlinear_routed needs for an m x k activation and rank
+ * r (0 without branch): the quantized activation in the largest format,
+ * its scales and tensor scale, the low-rank operands and the tensor-amax
+ * words, each at a 256-byte boundary. */
+mxq_status mxq_qlinear_routed_workspace_bytes(int64_t m, int64_t k, int32_t r, size_t *bytes);
+
+/* The routed quantized linear layer (Chameleon article, sections "the format
+ * is chosen by the value distribution" and "calibration, not acceleration,
+ * is planned": the trajectory is cut into intervals, and at generation time
+ * each layer reads the activation format of the current interval from a
+ * table computed in advance; Nunchaku/Diffusers article: the low-rank
+ * branch beside the low-bit residual).  One call:
+ *   fmt = fmt_table[layer][floor(step * n_intervals / n_steps)]  (host read,
+ *     as mxq_route),
+ *   xq  = x quantized in fmt (MMA layout; after the rotation when
+ *     layer_w->hadamard_b > 0), into the workspace,
+ *   y   = deq(xq) . deq(layer_w->w[fmt])^T (+ (bf16(x) . l1) . l2)
+ * with the kernels of mxq_quantize / mxq_quantize_lowrank and mxq_qlinear.
+ *   x: m x k fp32/bf16 device, 16-byte aligned; k == the weights' cols.
+ *   fmt_table: host uint8[n_layers][n_intervals] of mxq_fmt.
+ *   y: m x N device, ydtype MXQ_BF16 or MXQ_F32.
+ *   fmt_used: host int32 receiving the routed format, or NULL.
+ *   workspace: device scratch of mxq_qlinear_routed_workspace_bytes(m, k,
+ *     layer_w->r), 256-byte aligned; clobbered.
+ * Errors: MXQ_EINVAL (table arguments out of range, as mxq_route; the
+ * weight not prepared in the routed format; shapes, pointers, workspace
+ * alignment), MXQ_ENOSPACE (workspace), MXQ_EUNSUPPORTED (a branch with an
+ * INT8_ROW entry), MXQ_ECUDA; the argument rules of mxq_quantize and
+ * mxq_qlinear apply.  Everything but the table read runs asynchronously on
+ * `stream`. */
+mxq_status mxq_qlinear_routed(const void *x, int32_t xdtype, int64_t m, int64_t k, const mxq_layer *layer_w,
+                              const uint8_t *fmt_table, int32_t n_layers, int32_t n_intervals, int32_t layer,
+                              int32_t step, int32_t n_steps, void *y, int32_t ydtype, int32_t *fmt_used,
+                              void *workspace, size_t workspace_bytes, void *stream);
 
 #ifdef __cplusplus
 }

@@ -37,7 +37,8 @@ EXPORTS = ("mxq_status_string", "mxq_last_cuda_error_string", "mxq_device_suppor
            "mxq_calibrate_workspace_bytes", "mxq_calibrate_activation", "mxq_calibrate_pick",
            "mxq_lowrank_down", "mxq_lowrank_packed_bytes",
            "mxq_lowrank_down_packed", "mxq_lowrank_pack_t", "mxq_lowrank_pack_l2", "mxq_qlinear", "mxq_qlinear_w4a16", "mxq_route",
-           "mxq_quantize_lowrank_workspace_bytes", "mxq_quantize_lowrank", "mxq_quantize_lowrank_noalloc")
+           "mxq_quantize_lowrank_workspace_bytes", "mxq_quantize_lowrank", "mxq_quantize_lowrank_noalloc",
+           "mxq_qlinear_routed_workspace_bytes", "mxq_qlinear_routed")
 
 
 class MxqError(RuntimeError):
@@ -53,6 +54,11 @@ class _QTensorC(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int32), ("layout", ctypes.c_int32), ("rows", ctypes.c_int64),
                 ("cols", ctypes.c_int64), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("tensor_scale", ctypes.c_void_p)]
+
+
+class _LayerC(ctypes.Structure):
+    _fields_ = [("w", _QTensorC * 7), ("l1", ctypes.c_void_p), ("l2p", ctypes.c_void_p), ("r", ctypes.c_int32),
+                ("hadamard_b", ctypes.c_int32)]
 
 
 def _load():
@@ -95,6 +101,9 @@ def _load():
         "mxq_quantize_lowrank_workspace_bytes": (i32, [i64, i32, psz]),
         "mxq_quantize_lowrank": (i32, [P, i32, i64, i64, i32, i32, P, i32, P, P, P, P, P, P, sz, P]),
         "mxq_quantize_lowrank_noalloc": (i32, [P, i32, i64, i64, i32, i32, P, i32, P, P, P, P, P, P]),
+        "mxq_qlinear_routed_workspace_bytes": (i32, [i64, i64, i32, psz]),
+        "mxq_qlinear_routed": (i32, [P, i32, i64, i64, ctypes.POINTER(_LayerC), P, i32, i32, i32, i32, i32, P, i32,
+                                     ctypes.POINTER(ctypes.c_int32), P, sz, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -454,6 +463,66 @@ def route(table, layer: int, step: int, n_steps: int) -> int:
     tab = np.ascontiguousarray(np.asarray(table, dtype=np.uint8))
     n_layers, n_int = tab.shape
     return _lib.mxq_route(tab.ctypes.data_as(ctypes.c_void_p), n_layers, n_int, layer, step, n_steps)
+
+
+@dataclass
+class RoutedLayer:
+    """A linear layer prepared for routed execution: its weight quantized (MMA
+    layout) in every format its table row names, and the optional low-rank
+    branch (l1: K x r bf16, l2p: packed up projection)."""
+    weights: dict
+    l1: Optional[torch.Tensor] = None
+    l2p: Optional[torch.Tensor] = None
+    hadamard_b: int = 0
+
+    def c(self) -> _LayerC:
+        lay = _LayerC()
+        for f, q in self.weights.items():
+            lay.w[f] = q.c()
+        lay.l1 = _ptr(self.l1)
+        lay.l2p = _ptr(self.l2p)
+        lay.r = self.l1.shape[1] if self.l1 is not None else 0
+        lay.hadamard_b = self.hadamard_b
+        return lay
+
+
+def prepare_routed_layer(w: torch.Tensor, formats: Sequence[int], l1: torch.Tensor = None, l2: torch.Tensor = None,
+                         hadamard_b: int = 0, stream=None) -> RoutedLayer:
+    """Quantizes the weight w (N x K) once in each of `formats` (MMA layout)
+    and packs the low-rank up projection l2 (r x N bf16) when given."""
+    ws = {int(f): quantize(w, int(f), hadamard_b, MMA, stream=stream) for f in sorted(set(int(f) for f in formats))}
+    l2p = lowrank_pack_l2(l2, stream=stream) if l2 is not None else None
+    return RoutedLayer(ws, l1.contiguous() if l1 is not None else None, l2p, hadamard_b)
+
+
+def qlinear_routed_workspace_bytes(m: int, k: int, r: int = 0) -> int:
+    return _size(_lib.mxq_qlinear_routed_workspace_bytes, m, k, r)
+
+
+def qlinear_routed(x: torch.Tensor, layer_w: RoutedLayer, table, layer: int, step: int, n_steps: int,
+                   out_dtype=torch.bfloat16, out: torch.Tensor = None, workspace: torch.Tensor = None,
+                   stream=None):
+    """The routed linear layer: reads layer's format for `step` from the host
+    table [layers][intervals], quantizes x in it and runs the GEMM against the
+    weight prepared in that format.  Returns (y, routed format id)."""
+    import numpy as np
+    _require_cuda(x)
+    x = x.contiguous()
+    m, k = x.shape
+    n = next(iter(layer_w.weights.values())).rows
+    y = out if out is not None else torch.empty((m, n), dtype=out_dtype, device=x.device)
+    r = layer_w.l1.shape[1] if layer_w.l1 is not None else 0
+    wsb = qlinear_routed_workspace_bytes(m, k, r)
+    if workspace is None:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=x.device)
+    tab = np.ascontiguousarray(np.asarray(table, dtype=np.uint8))
+    n_layers, n_int = tab.shape
+    used = ctypes.c_int32(-1)
+    lay = layer_w.c()
+    _ok(_lib.mxq_qlinear_routed(_ptr(x), _dtype_code(x), m, k, ctypes.byref(lay), tab.ctypes.data_as(ctypes.c_void_p),
+                                n_layers, n_int, layer, step, n_steps, _ptr(y), _dtype_code(y), ctypes.byref(used),
+                                _ptr(workspace), workspace.numel(), _stream(stream)), "mxq_qlinear_routed")
+    return y, used.value
 
 
 def check(stream=None) -> int:

@@ -44,6 +44,21 @@ mxq_status from_cuda(cudaError_t e) {
 
 int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 
+// Arguments of mxq_quantize_lowrank other than the workspace.
+mxq_status check_quantize_lowrank(const void *x, int32_t xdtype, int64_t m, int64_t k, int32_t fmt,
+                                  int32_t hadamard_b, const void *l1, int32_t r, const float *w_tensor_scale,
+                                  const void *codes, const void *scales, const float *tensor_scale, const void *tp) {
+    if (!valid_fmt(fmt) || !valid_dtype(xdtype) || !valid_shape(fmt, m, k) || !valid_hadamard(hadamard_b, k))
+        return MXQ_EINVAL;
+    if (fmt == MXQ_INT8_ROW) return MXQ_EUNSUPPORTED;   // its GEMM takes no branch
+    if (k <= 0 || r < 1 || r > 32) return MXQ_EINVAL;
+    if (fmt_tensor_scaled(fmt) && (!tensor_scale || !w_tensor_scale)) return MXQ_EINVAL;
+    if (m > 0 && (!x || !codes || !tp || !l1 || !aligned16(x) || !aligned16(codes) || !aligned16(tp)))
+        return MXQ_EINVAL;
+    if (m > 0 && fmt != MXQ_FP8_TENSOR && !scales) return MXQ_EINVAL;
+    return MXQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -328,15 +343,10 @@ mxq_status mxq_quantize_lowrank(const void *x, int32_t xdtype, int64_t m, int64_
                                 const void *l1, int32_t r, const float *w_tensor_scale, void *codes, void *scales,
                                 float *tensor_scale, void *tp, void *workspace, size_t workspace_bytes,
                                 void *stream) {
-    if (!valid_fmt(fmt) || !valid_dtype(xdtype) || !valid_shape(fmt, m, k) || !valid_hadamard(hadamard_b, k))
-        return MXQ_EINVAL;
-    if (fmt == MXQ_INT8_ROW) return MXQ_EUNSUPPORTED;   // its GEMM takes no branch
-    if (k <= 0 || r < 1 || r > 32) return MXQ_EINVAL;
+    const mxq_status chk = check_quantize_lowrank(x, xdtype, m, k, fmt, hadamard_b, l1, r, w_tensor_scale, codes,
+                                                  scales, tensor_scale, tp);
+    if (chk != MXQ_OK) return chk;
     const bool ts = fmt_tensor_scaled(fmt);
-    if (ts && (!tensor_scale || !w_tensor_scale)) return MXQ_EINVAL;
-    if (m > 0 && (!x || !codes || !tp || !l1 || !aligned16(x) || !aligned16(codes) || !aligned16(tp)))
-        return MXQ_EINVAL;
-    if (m > 0 && fmt != MXQ_FP8_TENSOR && !scales) return MXQ_EINVAL;
     size_t need = 0, sb = 0;
     mxq_quantize_lowrank_workspace_bytes(m, r, &need);
     if (!workspace) return MXQ_EINVAL;
@@ -379,8 +389,11 @@ mxq_status mxq_qlinear_w4a16(const void *x, int64_t m, int64_t k, const mxq_qten
     if (wq->fmt != MXQ_INT4_G32 && wq->fmt != MXQ_INT4_G64) return MXQ_EUNSUPPORTED;
     if (wq->layout != MXQ_LAYOUT_CANONICAL || wq->cols != k || wq->rows < 0) return MXQ_EINVAL;
     if (m >= ((int64_t)1 << 31) || wq->rows >= ((int64_t)1 << 31) || k >= ((int64_t)1 << 31)) return MXQ_EINVAL;
-    // the kernel counts 128 x 128 tiles and their 64-column stages in 32-bit integers
-    if (((m + 127) / 128) * ((wq->rows + 127) / 128) * (k / 64) >= ((int64_t)1 << 31)) return MXQ_EINVAL;
+    // the kernel counts 128 x 128 tiles and their 64-column stages in 32-bit integers; each factor
+    // is below 2^24 here, so the tile count (< 2^48) is exact, and the product is formed only once
+    // the tile count is known to be below 2^31
+    const int64_t wa_tiles = ((m + 127) / 128) * ((wq->rows + 127) / 128);
+    if (wa_tiles >= ((int64_t)1 << 31) || wa_tiles * (k / 64) >= ((int64_t)1 << 31)) return MXQ_EINVAL;
     if (m > 0 && wq->rows > 0 && (!x || !y || !wq->codes || !wq->scales || !aligned16(x) || !aligned16(wq->codes)))
         return MXQ_EINVAL;
     return from_cuda(launch_w4a16(x, m, k, (const uint8_t *)wq->codes, (const float *)wq->scales, wq->rows,
@@ -474,6 +487,11 @@ mxq_status mxq_quantize_lowrank_noalloc(const void *x, int32_t xdtype, int64_t m
                                         int32_t hadamard_b, const void *l1, int32_t r,
                                         const float *w_tensor_scale, void *codes, void *scales,
                                         float *tensor_scale, void *tp, void *stream) {
+    // every argument is checked before the device array is looked up, so a
+    // rejected call makes no CUDA call at all
+    const mxq_status chk = check_quantize_lowrank(x, xdtype, m, k, fmt, hadamard_b, l1, r, w_tensor_scale, codes,
+                                                  scales, tensor_scale, tp);
+    if (chk != MXQ_OK) return chk;
     size_t need = 0;
     if (mxq_quantize_lowrank_workspace_bytes(m, r, &need) != MXQ_OK) return MXQ_EINVAL;
     if (need > kNoAllocScratchBytes) return MXQ_ENOSPACE;
@@ -490,6 +508,97 @@ int32_t mxq_route(const uint8_t *table, int32_t n_layers, int32_t n_intervals, i
     if (layer < 0 || layer >= n_layers || step < 0 || step >= n_steps) return -1;
     const int64_t interval = (int64_t)step * n_intervals / n_steps;
     return table[(int64_t)layer * n_intervals + interval];
+}
+
+}  // extern "C"
+
+namespace {
+
+// Workspace of mxq_qlinear_routed, each part at a 256-byte boundary: the
+// workspace of mxq_quantize_lowrank (the amax words, then t), the codes and
+// scales of the quantized activation in the largest format, its tensor
+// scale, and the packed low-rank operand.
+struct RoutedLayout {
+    size_t lowrank, codes, scales, tscale, tp, total;
+};
+
+RoutedLayout routed_layout(int64_t m, int64_t k, int32_t r) {
+    RoutedLayout L;
+    size_t off = 0;
+    auto take = [&off](size_t bytes) {
+        const size_t at = off;
+        off += (bytes + 255) / 256 * 256;
+        return at;
+    };
+    L.lowrank = take(kLrHeader + (size_t)(m * (r > 0 ? r : 0) * 4));
+    L.codes = take((size_t)(m * k));                                  // 8-bit codes, or INT4 as bytes
+    const size_t nv = (size_t)(round_up(m, 128) * round_up(k / 16, 16));   // NVFP4 scales bound the MX ones
+    const size_t ig = (size_t)(m * (k / 32) * 4);                        // INT4_G32 fp32 group scales
+    size_t sc = nv > ig ? nv : ig;
+    if ((size_t)(m * 4) > sc) sc = (size_t)(m * 4);                      // INT8_ROW row scales
+    L.scales = take(sc);
+    L.tscale = take(4);
+    L.tp = take(r > 0 ? (size_t)(m * 64 * 2) : 0);
+    L.total = off;
+    return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+mxq_status mxq_qlinear_routed_workspace_bytes(int64_t m, int64_t k, int32_t r, size_t *bytes) {
+    if (m < 0 || k < 0 || k % 16 || r < 0 || r > 32 || !bytes) return MXQ_EINVAL;
+    if (m > ((int64_t)1 << 31) || k > ((int64_t)1 << 31) || m * (k / 16) >= ((int64_t)1 << 31)) return MXQ_EINVAL;
+    *bytes = routed_layout(m, k, r).total;
+    return MXQ_OK;
+}
+
+mxq_status mxq_qlinear_routed(const void *x, int32_t xdtype, int64_t m, int64_t k, const mxq_layer *layer_w,
+                              const uint8_t *fmt_table, int32_t n_layers, int32_t n_intervals, int32_t layer,
+                              int32_t step, int32_t n_steps, void *y, int32_t ydtype, int32_t *fmt_used,
+                              void *workspace, size_t workspace_bytes, void *stream) {
+    if (!layer_w || !valid_dtype(xdtype) || !valid_dtype(ydtype)) return MXQ_EINVAL;
+    const int32_t fmt = mxq_route(fmt_table, n_layers, n_intervals, layer, step, n_steps);
+    if (!valid_fmt(fmt)) return MXQ_EINVAL;
+    if (fmt_used) *fmt_used = fmt;
+    const mxq_qtensor *wq = &layer_w->w[fmt];
+    if (!wq->codes || wq->fmt != fmt || wq->layout != MXQ_LAYOUT_MMA || wq->cols != k) return MXQ_EINVAL;
+    const int32_t r = layer_w->r;
+    if (r < 0 || r > 32 || (r > 0 && (!layer_w->l1 || !layer_w->l2p))) return MXQ_EINVAL;
+    if (r > 0 && fmt == MXQ_INT8_ROW) return MXQ_EUNSUPPORTED;   // the INT8 GEMM takes no branch
+    size_t need = 0;
+    if (mxq_qlinear_routed_workspace_bytes(m, k, r, &need) != MXQ_OK) return MXQ_EINVAL;
+    if (!workspace) return MXQ_EINVAL;
+    if (workspace_bytes < need) return MXQ_ENOSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MXQ_EINVAL;
+    const RoutedLayout L = routed_layout(m, k, r);
+    uint8_t *ws = (uint8_t *)workspace;
+    size_t cb = 0, sb = 0;
+    if (mxq_codes_bytes(fmt, m, k, MXQ_LAYOUT_MMA, &cb) != MXQ_OK ||
+        mxq_scales_bytes(fmt, m, k, MXQ_LAYOUT_MMA, &sb) != MXQ_OK)
+        return MXQ_EINVAL;   // k not a whole number of the routed format's blocks
+    mxq_qtensor xq;
+    xq.fmt = fmt;
+    xq.layout = MXQ_LAYOUT_MMA;
+    xq.rows = m;
+    xq.cols = k;
+    xq.codes = ws + L.codes;
+    xq.scales = sb ? ws + L.scales : nullptr;
+    xq.tensor_scale = fmt_tensor_scaled(fmt) ? (const float *)(ws + L.tscale) : nullptr;
+    mxq_status st;
+    void *tp = nullptr;
+    if (r > 0) {
+        tp = ws + L.tp;
+        st = mxq_quantize_lowrank(x, xdtype, m, k, fmt, layer_w->hadamard_b, layer_w->l1, r, wq->tensor_scale,
+                                  (void *)xq.codes, (void *)xq.scales, (float *)xq.tensor_scale, tp, ws + L.lowrank,
+                                  L.codes - L.lowrank, stream);
+    } else {
+        st = mxq_quantize(x, xdtype, m, k, fmt, layer_w->hadamard_b, MXQ_LAYOUT_MMA, (void *)xq.codes,
+                          (void *)xq.scales, (float *)xq.tensor_scale, ws + L.lowrank, L.codes - L.lowrank, stream);
+    }
+    if (st != MXQ_OK) return st;
+    return mxq_qlinear(&xq, wq, tp, r > 0 ? layer_w->l2p : nullptr, y, ydtype, stream);
 }
 
 }  // extern "C"

@@ -599,12 +599,10 @@ namespace {
 
 template <int KIND>
 cudaError_t launch_kind(const GemmParams &p, int grid, cudaStream_t s) {
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(k_gemm<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static PerDeviceOnce smem_opt_in;
+    cudaError_t e = smem_opt_in.run(
+        [] { return cudaFuncSetAttribute(k_gemm<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES); });
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3((unsigned)grid, 1, 1);   // clusters of 2 from __cluster_dims__
@@ -667,13 +665,7 @@ cudaError_t launch_qlinear(const GemmOperands &op, cudaStream_t s) {
     p.n_tiles = (int)((op.n + BN - 1) / BN);
     p.sfa_tiles = (int)((op.m + 127) / 128);
     p.wait_ns = 2000000000ull;   // 2 s
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms <= 0) sms = 148;
-    }
+    const int sms = sm_count();
     const int tiles = p.m_tiles * p.n_tiles;
     const int clusters = tiles < sms / 2 ? tiles : sms / 2;
     const int grid = 2 * clusters;

@@ -365,12 +365,10 @@ __global__ void __launch_bounds__(IG_THREADS, 1) k_gemm_igroup(const __grid_cons
 
 template <int GROUP>
 cudaError_t launch_group(const IGroupParams &p, int grid, cudaStream_t s) {
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(k_gemm_igroup<GROUP>, cudaFuncAttributeMaxDynamicSharedMemorySize, IG_SMEM);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static PerDeviceOnce smem_opt_in;
+    cudaError_t e = smem_opt_in.run(
+        [] { return cudaFuncSetAttribute(k_gemm_igroup<GROUP>, cudaFuncAttributeMaxDynamicSharedMemorySize, IG_SMEM); });
+    if (e != cudaSuccess) return e;
     k_gemm_igroup<GROUP><<<grid, IG_THREADS, IG_SMEM, s>>>(p);
     return cudaGetLastError();
 }
@@ -407,13 +405,7 @@ cudaError_t launch_qlinear_igroup(const GemmOperands &op, cudaStream_t s) {
     p.m_tiles = (int)((op.m + IG_BM - 1) / IG_BM);
     p.n_tiles = (int)((op.n + IG_BN - 1) / IG_BN);
     p.wait_ns = 2000000000ull;   // 2 s
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms <= 0) sms = 148;
-    }
+    const int sms = sm_count();
     const int tiles = p.m_tiles * p.n_tiles;
     const int grid = tiles < sms ? tiles : sms;
     return g == 32 ? launch_group<32>(p, grid, s) : launch_group<64>(p, grid, s);

@@ -329,13 +329,19 @@ cudaError_t launch_lowrank_down(const void *x, bool bf16, int64_t m, int64_t k, 
     const __nv_bfloat16 *l = (const __nv_bfloat16 *)l1;
     __nv_bfloat16 *tpb = (__nv_bfloat16 *)tp;
     if (bf16 && k % 64 == 0 && r % 8 == 0 && (reinterpret_cast<uintptr_t>(l1) & 15u) == 0) {
-        static bool configured = false;
-        if (!configured) {
-            cudaFuncSetAttribute(k_lowrank_staged<kLrT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kLsSmem);
-            cudaFuncSetAttribute(k_lowrank_staged<kLrPacked>, cudaFuncAttributeMaxDynamicSharedMemorySize, kLsSmem);
-            cudaFuncSetAttribute(k_lowrank_staged<kLrTAmax>, cudaFuncAttributeMaxDynamicSharedMemorySize, kLsSmem);
-            configured = true;
-        }
+        static PerDeviceOnce smem_opt_in;
+        const cudaError_t se = smem_opt_in.run([] {
+            cudaError_t e = cudaFuncSetAttribute(k_lowrank_staged<kLrT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 kLsSmem);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(k_lowrank_staged<kLrPacked>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kLsSmem);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(k_lowrank_staged<kLrTAmax>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kLsSmem);
+            return e;
+        });
+        if (se != cudaSuccess) return se;
         const __nv_bfloat16 *xb = (const __nv_bfloat16 *)x;
         if (mode == kLrT) k_lowrank_staged<kLrT><<<grid, kLsThreads, kLsSmem, s>>>(xb, m, k, l, r, t, xs, ws, tpb, amax_word);
         else if (mode == kLrPacked)

@@ -430,24 +430,29 @@ cudaError_t launch_lowrank_tc(const void *x, int64_t m, int64_t k, const void *l
     p.r = r;
     p.row_tiles = (int)((m + 127) / 128);
     p.kb_total = (int)((k + 63) / 64);
-    static bool configured = false;
-    if (!configured) {
+    static PerDeviceOnce smem_opt_in;
+    const cudaError_t se = smem_opt_in.run([] {
         for (auto fn : {k_lowrank_tc<1>, k_lowrank_tc<2>, k_lowrank_tc<4>, k_lowrank_tc<8>}) {
             cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, LT_SMEM_MAX);
             if (e != cudaSuccess) return e;
         }
-        configured = true;
-    }
+        return cudaSuccess;
+    });
+    if (se != cudaSuccess) return se;
+    const int dev = current_device_index();
+    if (dev < 0) return cudaErrorInvalidDevice;
     // cluster size: fewest rounds x k-blocks per CTA, then the smaller cluster; the
     // number of clusters that fit on the GPU at once comes from the occupancy query
-    static int max_clusters[4] = {-1, -1, -1, -1};
+    // co-resident clusters per cluster size, per device (0: not yet queried; else the count + 1)
+    static std::atomic<int> max_clusters_cache[kMaxDevices][4];
     int best_s = 0, best_clusters = 0;
     int64_t best_cost = 0;
     for (int li = 0, S = 1; S <= 8; li++, S *= 2) {
         if (S > p.kb_total) break;
         const int kb_max = (p.kb_total + S - 1) / S;
         if (lt_smem_bytes(kb_max) > LT_SMEM_MAX) continue;
-        if (max_clusters[li] < 0) {
+        int max_clusters = max_clusters_cache[dev][li].load(std::memory_order_relaxed) - 1;
+        if (max_clusters < 0) {
             cudaLaunchConfig_t q;
             memset(&q, 0, sizeof(q));
             q.gridDim = dim3((unsigned)S, 1, 1);
@@ -469,9 +474,10 @@ cudaError_t launch_lowrank_tc(const void *x, int64_t m, int64_t k, const void *l
                 cudaGetLastError();
                 n = 0;
             }
-            max_clusters[li] = n;
+            max_clusters = n;
+            max_clusters_cache[dev][li].store(n + 1, std::memory_order_relaxed);
         }
-        const int clusters = p.row_tiles < max_clusters[li] ? p.row_tiles : max_clusters[li];
+        const int clusters = p.row_tiles < max_clusters ? p.row_tiles : max_clusters;
         if (clusters < 1) continue;
         const int64_t cost = (int64_t)((p.row_tiles + clusters - 1) / clusters) * kb_max;
         if (!best_s || cost < best_cost) {

@@ -7,9 +7,53 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace mxq {
 
 constexpr int kMaxCandidates = 8;
+
+// Launch state that belongs to a device: a kernel's dynamic shared memory
+// opt-in (cudaFuncSetAttribute) is set per device, and SM counts and
+// occupancy differ between devices, so launchers keep such state per device
+// index.  Devices 0 .. kMaxDevices-1 are supported.
+constexpr int kMaxDevices = 64;
+
+// Index of the current device, or -1 when it cannot be read or is out of range.
+inline int current_device_index() {
+    int d = -1;
+    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) return -1;
+    return d;
+}
+
+// SM count of the current device (148 when it cannot be read), cached per device.
+inline int sm_count() {
+    static std::atomic<int> cache[kMaxDevices];
+    const int d = current_device_index();
+    if (d < 0) return 148;
+    int c = cache[d].load(std::memory_order_relaxed);
+    if (c <= 0) {
+        if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || c <= 0) c = 148;
+        cache[d].store(c, std::memory_order_relaxed);
+    }
+    return c;
+}
+
+// Runs `setup` (returning cudaError_t) once per device, on the current device;
+// a setup that fails is retried on the next call.  Two threads may both run
+// it the first time, which is harmless for attribute settings.
+struct PerDeviceOnce {
+    std::atomic<bool> done[kMaxDevices];
+    template <typename F>
+    cudaError_t run(F &&setup) {
+        const int d = current_device_index();
+        if (d < 0) return cudaErrorInvalidDevice;
+        if (done[d].load(std::memory_order_acquire)) return cudaSuccess;
+        const cudaError_t e = setup();
+        if (e == cudaSuccess) done[d].store(true, std::memory_order_release);
+        return e;
+    }
+};
 
 // Launch attribute of the kernels on the activation -> GEMM chain
 // (k_lowrank_tc, k_quantize, k_gemm): the kernel may be scheduled while

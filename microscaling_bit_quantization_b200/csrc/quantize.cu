@@ -634,16 +634,7 @@ __global__ void __launch_bounds__(kThreads) k_select(const T *__restrict__ w, Se
 
 // ====================================================================== host
 
-static int sm_count_cached() {
-    static int count = 0;
-    if (!count) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev);
-        if (count <= 0) count = 148;
-    }
-    return count;
-}
+static int sm_count_cached() { return sm_count(); }
 
 template <typename T, int F>
 static void launch_qf(const T *x, const QuantArgs &a, cudaStream_t s);

@@ -341,19 +341,10 @@ cudaError_t launch_w4a16(const void *x, int64_t m, int64_t k, const uint8_t *cod
     p.wait_ns = 2000000000ull;   // 2 s
     cudaError_t e = error_word_address(&p.err);
     if (e != cudaSuccess) return e;
-    static bool configured = false;
-    if (!configured) {
-        e = cudaFuncSetAttribute(k_w4a16, cudaFuncAttributeMaxDynamicSharedMemorySize, WA_SMEM);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms <= 0) sms = 148;
-    }
+    static PerDeviceOnce smem_opt_in;
+    e = smem_opt_in.run([] { return cudaFuncSetAttribute(k_w4a16, cudaFuncAttributeMaxDynamicSharedMemorySize, WA_SMEM); });
+    if (e != cudaSuccess) return e;
+    const int sms = sm_count();
     const int tiles = p.m_tiles * p.n_tiles;
     const int grid = tiles < sms ? tiles : sms;
     k_w4a16<<<grid, WA_THREADS, WA_SMEM, s>>>(p);

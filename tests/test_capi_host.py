@@ -153,6 +153,10 @@ def test_w4a16_argument_checks(mxq):
     assert call(qt(mxq.INT4_G32, 0, 8, 128), yd=7) == 1   # bad output dtype
     big = qt(mxq.INT4_G64, 0, (1 << 31) - 1, 1 << 20)
     assert L.mxq_qlinear_w4a16(d, (1 << 31) - 1, 1 << 20, ctypes.byref(big), d, 1, None) == 1   # stage count
+    # every factor at its largest: the product of tiles and stages (about 2^73) must not wrap around
+    kmax = (1 << 31) - 64
+    huge = qt(mxq.INT4_G64, 0, (1 << 31) - 1, kmax)
+    assert L.mxq_qlinear_w4a16(d, (1 << 31) - 1, kmax, ctypes.byref(huge), d, 1, None) == 1
 
 
 def test_qlinear_argument_checks(mxq):
@@ -181,6 +185,66 @@ def test_qlinear_argument_checks(mxq):
     a = Q(mxq.NVFP4, mxq.MMA, 64, 256, 256, 256, 256)
     assert L.mxq_qlinear(ctypes.byref(a), ctypes.byref(a), t, None, y, 0, None) == 1      # branch without l2p
     assert L.mxq_lowrank_down_packed(t, 1, 4, 64, t, 8, t, None, t, None) == 1             # one tensor scale
+
+
+def test_noalloc_rejects_arguments_before_any_cuda_call(mxq):
+    """The allocation-free entry point checks every argument before it looks
+    up its device array: on this GPU-less host a CUDA call would fail, so a
+    plain MXQ_EINVAL / MXQ_EUNSUPPORTED shows that none was made."""
+    L, P = mxq.lib(), ctypes.c_void_p
+    d = P(256)
+    call = L.mxq_quantize_lowrank_noalloc
+    assert call(d, 1, 64, 256, 9, 0, d, 32, d, d, d, d, d, None) == 1          # bad format
+    assert call(d, 1, 64, 256, mxq.NVFP4, 3, d, 32, d, d, d, d, d, None) == 1  # bad rotation size
+    assert call(d, 1, 64, 256, mxq.NVFP4, 0, d, 33, d, d, d, d, d, None) == 1  # rank above 32
+    assert call(d, 1, 64, 256, mxq.NVFP4, 0, d, 32, None, d, d, d, d, None) == 1   # no weight tensor scale
+    assert call(None, 1, 64, 256, mxq.NVFP4, 0, d, 32, d, d, d, d, d, None) == 1   # no input
+    assert call(d, 1, 64, 256, mxq.INT8_ROW, 0, d, 32, d, d, d, d, d, None) == 2   # no branch on INT8
+    assert call(d, 1, 40000, 512, mxq.NVFP4, 0, d, 32, d, d, d, d, d, None) == 5   # beyond the 4 MiB array
+
+
+def _routed_layout(m, k, r):
+    up = lambda b: (b + 255) // 256 * 256
+    rnd = lambda a, b: (a + b - 1) // b * b
+    total = up(4096 + 4 * m * r) + up(m * k)
+    total += up(max(rnd(m, 128) * rnd(k // 16, 16), m * (k // 32) * 4, 4 * m)) + up(4)
+    return total + (up(128 * m) if r else 0)
+
+
+def test_routed_workspace_and_argument_checks(mxq):
+    L, P = mxq.lib(), ctypes.c_void_p
+    size = ctypes.c_size_t(0)
+    for m, k, r in ((8192, 1152, 0), (8192, 4608, 0), (4096, 3072, 32), (1, 16, 8), (0, 64, 0)):
+        assert L.mxq_qlinear_routed_workspace_bytes(m, k, r, ctypes.byref(size)) == 0
+        assert size.value == _routed_layout(m, k, r), (m, k, r)
+    assert L.mxq_qlinear_routed_workspace_bytes(4, 40, 0, ctypes.byref(size)) == 1      # k % 16
+    assert L.mxq_qlinear_routed_workspace_bytes(4, 64, 33, ctypes.byref(size)) == 1     # rank
+    Q = mxq._QTensorC
+    m, k, n = 64, 256, 128
+    lay = mxq._LayerC()
+    lay.w[mxq.MXFP8] = Q(mxq.MXFP8, mxq.MMA, n, k, 256, 256, None)
+    lay.w[mxq.INT8_ROW] = Q(mxq.INT8_ROW, mxq.MMA, n, k, 256, 256, None)
+    table = np.array([[mxq.MXFP8, mxq.INT8_ROW, mxq.NVFP4]], np.uint8)
+    tp = table.ctypes.data_as(P)
+    d = P(256)
+    ws = P(1 << 20)
+    used = ctypes.c_int32(-1)
+
+    def call(step=0, n_steps=3, layer=0, lay=lay, ws=ws, wsb=1 << 24, x=d):
+        return L.mxq_qlinear_routed(x, 1, m, k, ctypes.byref(lay), tp, 1, 3, layer, step, n_steps, d, 1,
+                                    ctypes.byref(used), ws, wsb, None)
+
+    assert call(step=3) == 1                     # step out of range
+    assert call(layer=1) == 1                    # layer out of range
+    assert call(n_steps=0) == 1
+    assert call(step=2) == 1 and used.value == mxq.NVFP4   # routed to a format the layer was not prepared in
+    assert call(wsb=1024) == 5                   # workspace too small
+    assert call(ws=P((1 << 20) + 16)) == 1       # workspace not 256-byte aligned
+    assert call(x=None) == 1                     # the quantizer's own checks apply
+    lay.r, lay.l1, lay.l2p = 8, 256, 256
+    assert call(step=1) == 2 and used.value == mxq.INT8_ROW   # a branch on an INT8 entry
+    lay.w[mxq.MXFP8].cols = 512
+    assert call(step=0) == 1                     # weight K differs from x
 
 
 def test_route_matches_oracle(mxq, orc):

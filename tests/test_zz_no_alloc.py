@@ -34,14 +34,15 @@ def _inputs(seed, m, k, n, r):
     return x.to(bf).cuda(), w.to(bf).cuda(), l1.to(bf).cuda(), l2.to(bf).cuda()
 
 
-def _noalloc_call(mxq, x, fmt, l1, wq):
+def _noalloc_call(mxq, x, fmt, l1, wq, hadamard_b=0):
     """Direct call through the C ABI (no workspace argument)."""
     m, k = x.shape
     q = mxq.alloc_qtensor(fmt, m, k, mxq.MMA, x.device)
     tp = torch.empty((m, 64), dtype=torch.bfloat16, device=x.device)
     P = ctypes.c_void_p
+    xdt = mxq.BF16 if x.dtype == torch.bfloat16 else mxq.F32
     st = mxq.lib().mxq_quantize_lowrank_noalloc(
-        P(x.data_ptr()), mxq.BF16, m, k, fmt, 0, P(l1.data_ptr()), l1.shape[1],
+        P(x.data_ptr()), xdt, m, k, fmt, hadamard_b, P(l1.data_ptr()), l1.shape[1],
         P(wq.tensor_scale.data_ptr()) if wq.tensor_scale is not None else None,
         P(q.codes.data_ptr()), P(q.scales.data_ptr()) if q.scales is not None else None,
         P(q.tensor_scale.data_ptr()) if q.tensor_scale is not None else None, P(tp.data_ptr()),
@@ -71,6 +72,31 @@ def test_noalloc_matches_workspace_entry_point(mxq, fmt):
         err = np.abs(y - y_ref)
         assert np.linalg.norm(y - y_ref) <= 1e-4 * np.linalg.norm(y_ref)
         assert err.max() <= 1e-4 * np.abs(y_ref).max()
+
+
+@pytest.mark.parametrize("x_fp32,hadamard_b", [(True, 0), (False, 128), (True, 128)])
+def test_noalloc_cleared_amax_route(mxq, x_fp32, hadamard_b):
+    """NVFP4 with fp32 input or with the rotation takes the route that clears
+    the amax word in the shared array and folds every CTA's maximum into it:
+    two calls in a row (the second on a different input, so a stale maximum
+    would show) equal the workspace entry point bit for bit."""
+    fmt = 2
+    for call, seed in enumerate((21, 22)):
+        x, w, l1, _ = _inputs(seed + 7 * hadamard_b, 260 + 64 * call, 512, 384, 32)
+        if x_fp32:
+            x = x.float()
+        if call == 1:
+            x = x * 0.25   # a smaller tensor amax than the first call's
+        wq = mxq.quantize(w, fmt, hadamard_b, mxq.MMA)
+        ref_q, ref_tp = mxq.quantize_lowrank(x, fmt, l1, wq, hadamard_b)
+        st, q, tp = _noalloc_call(mxq, x, fmt, l1, wq, hadamard_b)
+        assert st == 0
+        torch.cuda.synchronize()
+        assert mxq.check() == 0
+        assert torch.equal(q.codes, ref_q.codes)
+        assert torch.equal(q.scales, ref_q.scales)
+        assert torch.equal(q.tensor_scale, ref_q.tensor_scale)
+        assert torch.equal(tp.view(torch.int16), ref_tp.view(torch.int16))
 
 
 def test_noalloc_rejects_sizes_beyond_the_array(mxq):

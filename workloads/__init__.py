@@ -164,3 +164,20 @@ def dit_forced_column_factors(seed: int, layer: int, in_features: int):
 
 def dit_weight(seed: int, layer: int, in_features: int, out_features: int):
     return normal(seed, "w.%d" % layer, (out_features, in_features), 0.02)
+
+
+def dit_layer_shape(layer: int):
+    """(in_features, out_features) of stack layer `layer` (4 linears per block)."""
+    _, kin, nout = DIT_LINEARS[layer % len(DIT_LINEARS)]
+    return kin, nout
+
+
+def dit_layer_input(seed: int, step: int, layer: int, forced, m: int = DIT_TOKENS):
+    """Input of stack layer `layer` at `step`: the step's shared activation of
+    that width, and for a forced layer its columns times the layer's factors
+    (log-uniform in [1, 163]), rounded once more to bf16."""
+    kin, _ = dit_layer_shape(layer)
+    x = dit_activation(seed, step, kin, m)
+    if layer in set(int(f) for f in forced):
+        x = to_bf16_values(x * dit_forced_column_factors(seed, layer, kin)[None, :])
+    return x
