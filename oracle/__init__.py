@@ -390,6 +390,32 @@ def w4a16(x, wq: QTensor, rows=None) -> np.ndarray:
     return xb @ w4a16_weights(wq).astype(np.float64).T
 
 
+# ---------------------------------------------------------------- per-channel mixed weight formats
+
+def qlinear_mixed(x, w, choice, rows=None) -> np.ndarray:
+    """Linear layer whose weight keeps a format per output channel (Chameleon
+    article, section "the format is chosen by the value distribution": each
+    output channel of a weight takes the format with the least reconstruction
+    error; its W8A8 / W4A8 settings quantize activations to 8 bits, here
+    MXFP8).  Y[m, n] = sum_k deq(MXFP8(X))[m, k] * deq_f(W)[n, k] with
+    f = choice[n], in binary64 over exactly dequantized operands.  Each
+    weight format quantizes the whole W, so a tensor-scaled format (NVFP4)
+    takes the tensor scale of the whole weight, as the selection measures it.
+    `rows` restricts the result to those rows of X."""
+    x, w = _f32(x), _f32(w)
+    choice = np.asarray(choice, dtype=np.uint8)
+    if choice.shape != (w.shape[0],):
+        raise OracleError("one format per output channel")
+    wd = np.zeros(w.shape, np.float64)
+    for f in np.unique(choice):
+        sel = choice == f
+        wd[sel] = quantize(w, int(f)).dequantize()[sel]
+    xd = quantize(x, MXFP8).dequantize()
+    if rows is not None:
+        xd = xd[np.asarray(rows)]
+    return xd @ wd.T
+
+
 # ---------------------------------------------------------------- routing
 
 def route(table, n_layers: int, n_intervals: int, layer: int, step: int, n_steps: int) -> int:

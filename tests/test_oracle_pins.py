@@ -801,3 +801,95 @@ def test_route_table_read(orc):
     # uneven split: 7 intervals over 20 steps -> floor(step * 7 / 20)
     t7 = np.arange(7, dtype=np.uint8)[None, :]
     assert [orc.route(t7, 1, 7, 0, s, 20) for s in range(20)] == [s * 7 // 20 for s in range(20)]
+
+
+# ------------------------------------------------------------------ per-channel mixed weight formats
+
+def _e2m1_grid(rng, shape, scale):
+    """Values of the E2M1 grid times `scale` (exact in binary32)."""
+    mags = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float64)
+    return (mags[rng.integers(0, 8, size=shape)] * rng.choice([-1.0, 1.0], size=shape) * scale)
+
+
+def test_qlinear_mixed_exact_operands(orc):
+    """Operands built to be exactly representable -- X in MXFP8, each weight row
+    in the format it is given (MXFP4: E2M1 values times a power of two per
+    32-block with the block maximum 6 times it; INT4-g32: integers in [-7, 7]
+    times a power of two with a 7 in every block; NVFP4: E2M1 values times an
+    E4M3 block scale per 16-block whose maximum is 6 times it, and one element
+    2688 = 6 * 448 so the tensor scale is exactly 1) -- make the mixed product
+    equal the plain product of the unquantized operands, which math.fsum gives
+    independently of the oracle.  Routing a row to another format breaks the
+    equality."""
+    rng = np.random.default_rng(41)
+    m, k = 5, 64
+    x = np.zeros((m, k), np.float64)
+    e4m3_vals = np.array([orc.e4m3_value(c) for c in range(0x7F)], np.float64)   # non-negative codes
+    for i in range(m):
+        for b in range(k // 32):
+            e = int(rng.integers(-6, 6))
+            blk = e4m3_vals[rng.integers(0, 0x7F, size=32)] * rng.choice([-1.0, 1.0], size=32)
+            blk[int(rng.integers(0, 32))] = 448.0 * rng.choice([-1.0, 1.0])   # floor(log2 amax) - 8 = 0
+            x[i, b * 32:(b + 1) * 32] = blk * 2.0 ** e
+    choice = np.array([1, 3, 2, 2, 3, 1, 2], np.uint8)   # MXFP4, INT4-g32, NVFP4
+    n = len(choice)
+    w = np.zeros((n, k), np.float64)
+    for r, f in enumerate(choice):
+        if f == 1:
+            for b in range(k // 32):
+                j = int(rng.integers(-8, 0))
+                blk = _e2m1_grid(rng, 32, 2.0 ** j)
+                blk[int(rng.integers(0, 32))] = 6.0 * 2.0 ** j
+                w[r, b * 32:(b + 1) * 32] = blk
+        elif f == 3:
+            for b in range(k // 32):
+                j = int(rng.integers(-8, 0))
+                blk = rng.integers(-7, 8, size=32).astype(np.float64) * 2.0 ** j
+                blk[int(rng.integers(0, 32))] = -7.0 * 2.0 ** j
+                w[r, b * 32:(b + 1) * 32] = blk
+        else:
+            for b in range(k // 16):
+                e4 = float(e4m3_vals[int(rng.integers(8, 0x60))])   # normal E4M3 scales up to 448 / 2
+                blk = _e2m1_grid(rng, 16, e4)
+                blk[int(rng.integers(0, 16))] = 6.0 * e4
+                w[r, b * 16:(b + 1) * 16] = blk
+    w[2, 0:16] = _e2m1_grid(rng, 16, 448.0)
+    w[2, 5] = 2688.0                                        # tensor amax: s_t = 2688 / 2688 = 1
+    x32, w32 = x.astype(np.float32), w.astype(np.float32)
+    assert np.array_equal(x32.astype(np.float64), x) and np.array_equal(w32.astype(np.float64), w)
+    y = orc.qlinear_mixed(x32, w32, choice)
+    for i in range(m):
+        for j in range(n):
+            ref = math.fsum(x[i, c] * w[j, c] for c in range(k))
+            assert abs(y[i, j] - ref) <= 1e-13 * (1.0 + math.fsum(abs(x[i, c] * w[j, c]) for c in range(k)))
+    # an NVFP4 row read as MXFP4 loses exactness somewhere
+    wrong = choice.copy()
+    wrong[2] = 1
+    y2 = orc.qlinear_mixed(x32, w32, wrong)
+    assert not np.allclose(y2[:, 2], y[:, 2], rtol=1e-9, atol=0)
+
+
+def test_qlinear_mixed_permutation_and_tensor_scale(orc):
+    """Permuting the output channels (weight rows with their formats) permutes
+    the columns of Y; and an NVFP4 channel uses the tensor scale of the whole
+    weight, not of the NVFP4 channels alone."""
+    rng = np.random.default_rng(42)
+    x = rng.standard_t(3, size=(6, 128)).astype(np.float32)
+    w = (rng.standard_normal((9, 128)) * 0.02).astype(np.float32)
+    w[4] *= 50.0                                             # the tensor maximum sits in an MXFP4 row
+    choice = np.array([2, 3, 1, 2, 1, 3, 2, 1, 2], np.uint8)
+    y = orc.qlinear_mixed(x, w, choice)
+    perm = rng.permutation(9)
+    yp = orc.qlinear_mixed(x, w[perm], choice[perm])
+    np.testing.assert_array_equal(yp, y[:, perm])
+    # column 0 (NVFP4) recomputed by brute force from the whole weight's NVFP4 quantization
+    xd = orc.quantize(x, orc.MXFP8).dequantize()
+    wq = orc.quantize(w, orc.NVFP4)
+    assert wq.tensor_scale == orc.quantize(w[[4]], orc.NVFP4).tensor_scale   # set by the MXFP4 row
+    wd = wq.dequantize()
+    for i in range(6):
+        ref = math.fsum(xd[i, c] * wd[0, c] for c in range(128))
+        assert abs(y[i, 0] - ref) <= 1e-12 * (1 + abs(ref))
+    # the NVFP4 rows alone would have had a different tensor scale
+    alone = orc.quantize(w[choice == 2], orc.NVFP4)
+    assert alone.tensor_scale != wq.tensor_scale
