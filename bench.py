@@ -561,6 +561,9 @@ def run_ours(args, world, rank, local):
         pass
 
     rows = {}
+    if args.rows == "none":   # the contract line only (e.g. under a profiler)
+        return finish(args, world, rank, ms, value, clocks, gemm_tflops, fp4_peak, peaks, profiles_traffic, gemm_ms,
+                      gemm_flops, rows, stream, sets, step, x_host, launches_per_step, torch, mxq)
     rows["activation_side"] = {"kernel": "k_lowrank_tc (T + tensor amax) + k_quantize<NVFP4> (codes, scales, "
                                          "packed T), X 4096 x 3072 bf16, graph replay of 100 launches",
                                "us": 1e3 * quant_ms, "bytes": quant_bytes, "GB/s": quant_gbs,
@@ -589,7 +592,22 @@ def run_ours(args, world, rank, local):
     x2_ms = timer.flushed_ms(lambda i: mxq.quantize(x2, mxq.MXFP8, 0, mxq.MMA, out=q2))
     rows["quantize_mxfp8_workload2_x"] = _hbm_row("k_quantize<MXFP8>, X 4096 x 3072 bf16 Student-t(3)", x2_ms,
                                                   x2.numel() * (2 + 1) + x2.numel() // 32, peaks)
-    del q2, x2
+    # the per-channel mixed-format linear layer on the selection's choices: X (MXFP8) . W^T
+    choice, _ = mxq.select_weight_format(wsel, cands, want_sse=False)
+    mw = mxq.prepare_mixed_weight(wsel, choice)
+    y2 = torch.empty((x2.shape[0], wsel.shape[0]), dtype=torch.bfloat16, device=dev)
+    ws2 = torch.empty(mxq.qlinear_mixed_workspace_bytes(x2.shape[0], mw), dtype=torch.uint8, device=dev)
+    mix_ms = timer.graph_ms(lambda i: mxq.qlinear_mixed(q2, mw, out=y2, workspace=ws2), n=10, reps=5)
+    mix_step_ms = timer.graph_ms(lambda i: (mxq.quantize(x2, mxq.MXFP8, 0, mxq.MMA, out=q2),
+                                            mxq.qlinear_mixed(q2, mw, out=y2, workspace=ws2)), n=10, reps=5)
+    f2 = 2 * x2.shape[0] * wsel.shape[0] * wsel.shape[1]
+    rows["mixed_format_linear_workload2"] = {
+        "kernels": "k_gemm<MXFP8> on the MXFP4 rows (E4M3 bytes), k_gemm_igroup<32> on the INT4-g32 rows, "
+                   "k_gemm<bf16> on the NVFP4 rows (x dequantized to bf16), scale conversion, dequantize, scatter",
+        "channels_mxfp4_int4g32_nvfp4": list(mw.n_group), "us": 1e3 * mix_ms,
+        "TFLOP/s": f2 / (mix_ms * 1e-3) / 1e12, "frac_of_fp8_peak": f2 / (mix_ms * 1e-3) / 1e12 / int8_peak,
+        "with_mxfp8_quantize_us": 1e3 * mix_step_ms}
+    del q2, x2, mw, y2, ws2
 
     # ---- workload 4: MXFP4 GEMM 8192 x 4096 x 4096, without and with the 128-wide rotation
     f4 = 2 * 8192 * 4096 * 4096
@@ -701,6 +719,14 @@ def run_ours(args, world, rank, local):
                                 "int8_peak": int8_peak}
     del wq4, xq4, tp4, w
     assert mxq.check() == 0
+    return finish(args, world, rank, ms, value, clocks, gemm_tflops, fp4_peak, peaks, profiles_traffic, gemm_ms,
+                  gemm_flops, rows, stream, sets, step, x_host, launches_per_step, torch, mxq)
+
+
+def finish(args, world, rank, ms, value, clocks, gemm_tflops, fp4_peak, peaks, profiles_traffic, gemm_ms, gemm_flops,
+           rows, stream, sets, step, x_host, launches_per_step, torch, mxq):
+    """End-to-end measurement, the oracle on the host cores, and the JSON line."""
+    dev = sets[0]["x"].device
 
     # ---- end to end through the public API with host buffers: each step copies its X in from
     # pinned memory and its Y out; the copies run on their own streams, overlapping the previous /
@@ -797,6 +823,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)   # ~0.3 s timed: a few clock samples
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--rows", default="all", choices=["all", "none"],
+                    help="'none': only the timed steps, the dominant kernel's timing, e2e and the CPU baseline")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

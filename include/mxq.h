@@ -451,6 +451,88 @@ mxq_status mxq_qlinear(const mxq_qtensor *xq, const mxq_qtensor *wq, const void 
                        void *y, int32_t ydtype, void *stream);
 
 /* ---------------------------------------------------------------------- */
+/* Per-channel mixed weight formats against MXFP8 activations.             */
+/* ---------------------------------------------------------------------- */
+
+/* A weight whose output channels keep the formats mxq_select_weight_format
+ * chose for them among MXFP4, INT4_G32 and NVFP4 (Chameleon article, section
+ * "the format is chosen by the value distribution"), laid out for the
+ * tensor cores as three groups of rows -- group 0 MXFP4, group 1 INT4_G32,
+ * group 2 NVFP4, each in channel order:
+ *   rows, cols: N output channels, K inputs (K % 32 == 0).
+ *   n_group[g]: channels in group g.
+ *   choice: device uint8[N], each channel's format; group_index: device
+ *     int32[N], each channel's row within its group (from mxq_mixed_plan).
+ *   mx_codes: device n_group[0] x K bytes, the E4M3 encoding of each E2M1
+ *     code (exact; zero as +0); mx_scales: their E8M0 block scales in the MMA
+ *     layout of mxq_quantize (n_group[0] rows).
+ *   i4_codes: device n_group[1] x K bytes, the E4M3 encoding of each integer
+ *     code; i4_scales: device fp32 [K/32][n_group[1]] group scales.
+ *   nv_values: device bf16 n_group[2] x K, each E2M1 code value times its
+ *     E4M3 block scale (exact in bf16); nv_tensor_scale: device fp32, the
+ *     NVFP4 tensor scale, that of the whole weight as in the selection.
+ * Buffers with a zero count may be NULL. */
+typedef struct mxq_mixed_weight {
+    int64_t rows, cols;
+    int64_t n_group[3];
+    const uint8_t *choice;
+    const int32_t *group_index;
+    void *mx_codes;
+    void *mx_scales;
+    void *i4_codes;
+    float *i4_scales;
+    void *nv_values;
+    const float *nv_tensor_scale;
+} mxq_mixed_weight;
+
+/* Host only: the grouping of channels by their chosen format.
+ *   choice: host uint8[n] of MXQ_MXFP4 / MXQ_INT4_G32 / MXQ_NVFP4.
+ *   n_group: host int64[3] receiving the group sizes; group_index: host
+ *     int32[n] receiving each channel's row within its group (channels keep
+ *     their order inside a group).
+ * Errors: MXQ_EINVAL (a format outside the three, n < 0 or >= 2^31, null). */
+mxq_status mxq_mixed_plan(const uint8_t *choice, int64_t n, int64_t n_group[3], int32_t *group_index);
+
+/* Host only: bytes of the five group buffers of mxq_mixed_weight, in the
+ * order mx_codes, mx_scales, i4_codes, i4_scales, nv_values. */
+mxq_status mxq_mixed_weight_bytes(const int64_t n_group[3], int64_t k, size_t bytes[5]);
+
+/* Lays the weight out as mxq_mixed_weight from its quantization in each of
+ * the three formats.
+ *   w_mxfp4, w_int4, w_nvfp4: the WHOLE weight (N x K) quantized by
+ *     mxq_quantize in MXQ_MXFP4, MXQ_INT4_G32 and MXQ_NVFP4, canonical layout.
+ *   out: rows, cols, n_group, choice, group_index filled by the caller (from
+ *     mxq_mixed_plan, choice and group_index copied to the device), the group
+ *     buffers allocated with mxq_mixed_weight_bytes; they are written here
+ *     (nv_tensor_scale may point at w_nvfp4->tensor_scale).
+ * Errors: MXQ_EINVAL (shapes, formats, layouts, pointers), MXQ_ECUDA. */
+mxq_status mxq_mixed_prepare(const mxq_qtensor *w_mxfp4, const mxq_qtensor *w_int4, const mxq_qtensor *w_nvfp4,
+                             const mxq_mixed_weight *out, void *stream);
+
+/* Scratch bytes mxq_qlinear_mixed needs for m activation rows: the
+ * activation's block scales as fp32 (INT4 group), the activation dequantized
+ * to bf16 (NVFP4 group) and one m x n_group[g] output per group, each at a
+ * 256-byte boundary. */
+mxq_status mxq_qlinear_mixed_workspace_bytes(int64_t m, const mxq_mixed_weight *w, int32_t ydtype, size_t *bytes);
+
+/* y = deq(xq) . deq_f(W)^T, each output channel n dequantized in its own
+ * format f = choice[n]: the MXFP4 group on kind::mxf8f6f4 block-scaled MMAs
+ * against the MXFP8 codes, the INT4_G32 group on the group GEMM of
+ * mxq_qlinear (each 32-element product of codes times the activation's 2^e
+ * and the weight's group scale), the NVFP4 group on bf16 kind::f16 MMAs
+ * against the activation dequantized to bf16 (exact while the block
+ * exponents stay inside the bf16 range), times the tensor scale; then the
+ * group outputs are scattered to channel order.  fp32 accumulation.
+ *   xq: MXQ_MXFP8, MMA layout, cols == w->cols.
+ *   y: m x N device, ydtype MXQ_BF16 or MXQ_F32.
+ *   workspace: device scratch of mxq_qlinear_mixed_workspace_bytes,
+ *     256-byte aligned; clobbered.
+ * Errors: MXQ_EINVAL, MXQ_ENOSPACE, MXQ_ECUDA; a pipeline wait that runs out
+ * is reported by mxq_check(). */
+mxq_status mxq_qlinear_mixed(const mxq_qtensor *xq, const mxq_mixed_weight *w, void *y, int32_t ydtype,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/* ---------------------------------------------------------------------- */
 /* a8: per-layer, per-timestep-interval format table.                      */
 /* ---------------------------------------------------------------------- */
 

@@ -38,7 +38,8 @@ EXPORTS = ("mxq_status_string", "mxq_last_cuda_error_string", "mxq_device_suppor
            "mxq_lowrank_down", "mxq_lowrank_packed_bytes",
            "mxq_lowrank_down_packed", "mxq_lowrank_pack_t", "mxq_lowrank_pack_l2", "mxq_qlinear", "mxq_qlinear_w4a16", "mxq_route",
            "mxq_quantize_lowrank_workspace_bytes", "mxq_quantize_lowrank", "mxq_quantize_lowrank_noalloc",
-           "mxq_qlinear_routed_workspace_bytes", "mxq_qlinear_routed")
+           "mxq_qlinear_routed_workspace_bytes", "mxq_qlinear_routed", "mxq_mixed_plan", "mxq_mixed_weight_bytes",
+           "mxq_mixed_prepare", "mxq_qlinear_mixed_workspace_bytes", "mxq_qlinear_mixed")
 
 
 class MxqError(RuntimeError):
@@ -59,6 +60,13 @@ class _QTensorC(ctypes.Structure):
 class _LayerC(ctypes.Structure):
     _fields_ = [("w", _QTensorC * 7), ("l1", ctypes.c_void_p), ("l2p", ctypes.c_void_p), ("r", ctypes.c_int32),
                 ("hadamard_b", ctypes.c_int32)]
+
+
+class _MixedC(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("n_group", ctypes.c_int64 * 3),
+                ("choice", ctypes.c_void_p), ("group_index", ctypes.c_void_p), ("mx_codes", ctypes.c_void_p),
+                ("mx_scales", ctypes.c_void_p), ("i4_codes", ctypes.c_void_p), ("i4_scales", ctypes.c_void_p),
+                ("nv_values", ctypes.c_void_p), ("nv_tensor_scale", ctypes.c_void_p)]
 
 
 def _load():
@@ -102,6 +110,12 @@ def _load():
         "mxq_quantize_lowrank": (i32, [P, i32, i64, i64, i32, i32, P, i32, P, P, P, P, P, P, sz, P]),
         "mxq_quantize_lowrank_noalloc": (i32, [P, i32, i64, i64, i32, i32, P, i32, P, P, P, P, P, P]),
         "mxq_qlinear_routed_workspace_bytes": (i32, [i64, i64, i32, psz]),
+        "mxq_mixed_plan": (i32, [P, i64, ctypes.POINTER(i64), P]),
+        "mxq_mixed_weight_bytes": (i32, [ctypes.POINTER(i64), i64, psz]),
+        "mxq_mixed_prepare": (i32, [ctypes.POINTER(_QTensorC), ctypes.POINTER(_QTensorC), ctypes.POINTER(_QTensorC),
+                                    ctypes.POINTER(_MixedC), P]),
+        "mxq_qlinear_mixed_workspace_bytes": (i32, [i64, ctypes.POINTER(_MixedC), i32, psz]),
+        "mxq_qlinear_mixed": (i32, [ctypes.POINTER(_QTensorC), ctypes.POINTER(_MixedC), P, i32, P, sz, P]),
         "mxq_qlinear_routed": (i32, [P, i32, i64, i64, ctypes.POINTER(_LayerC), P, i32, i32, i32, i32, i32, P, i32,
                                      ctypes.POINTER(ctypes.c_int32), P, sz, P]),
     }
@@ -523,6 +537,78 @@ def qlinear_routed(x: torch.Tensor, layer_w: RoutedLayer, table, layer: int, ste
                                 n_layers, n_int, layer, step, n_steps, _ptr(y), _dtype_code(y), ctypes.byref(used),
                                 _ptr(workspace), workspace.numel(), _stream(stream)), "mxq_qlinear_routed")
     return y, used.value
+
+
+@dataclass
+class MixedWeight:
+    """A weight whose output channels keep their own format among MXFP4,
+    INT4-g32 and NVFP4, laid out as three groups of rows (mxq_mixed_weight)."""
+    rows: int
+    cols: int
+    n_group: tuple
+    choice: torch.Tensor
+    group_index: torch.Tensor
+    mx_codes: torch.Tensor
+    mx_scales: torch.Tensor
+    i4_codes: torch.Tensor
+    i4_scales: torch.Tensor
+    nv_values: torch.Tensor
+    nv_tensor_scale: torch.Tensor
+
+    def c(self) -> _MixedC:
+        return _MixedC(self.rows, self.cols, (ctypes.c_int64 * 3)(*self.n_group), _ptr(self.choice),
+                       _ptr(self.group_index), _ptr(self.mx_codes), _ptr(self.mx_scales), _ptr(self.i4_codes),
+                       _ptr(self.i4_scales), _ptr(self.nv_values), _ptr(self.nv_tensor_scale))
+
+
+def prepare_mixed_weight(w: torch.Tensor, choice: torch.Tensor, stream=None) -> MixedWeight:
+    """Lays out w (N x K) with each output channel in the format `choice`
+    (device or host uint8[N] of MXFP4 / INT4_G32 / NVFP4, e.g. from
+    select_weight_format) names: the channel grouping from mxq_mixed_plan,
+    the whole weight quantized in each format, then mxq_mixed_prepare."""
+    import numpy as np
+    _require_cuda(w)
+    w = w.contiguous()
+    n, k = w.shape
+    ch = np.ascontiguousarray(choice.cpu().numpy() if isinstance(choice, torch.Tensor) else choice, dtype=np.uint8)
+    n_group = (ctypes.c_int64 * 3)()
+    gidx = np.zeros(max(n, 1), np.int32)
+    _ok(_lib.mxq_mixed_plan(ch.ctypes.data_as(ctypes.c_void_p), n, n_group, gidx.ctypes.data_as(ctypes.c_void_p)),
+        "mxq_mixed_plan")
+    sizes = (ctypes.c_size_t * 5)()
+    _ok(_lib.mxq_mixed_weight_bytes(n_group, k, sizes), "mxq_mixed_weight_bytes")
+    dev = w.device
+    buf = [torch.empty(max(int(b), 1), dtype=torch.uint8, device=dev) for b in sizes]
+    q = {f: quantize(w, f, stream=stream) for f in (MXFP4, INT4_G32, NVFP4)}
+    mw = MixedWeight(n, k, tuple(n_group), torch.from_numpy(ch).to(dev), torch.from_numpy(gidx[:n]).to(dev),
+                     buf[0], buf[1], buf[2], buf[3].view(torch.float32) if sizes[3] else buf[3], buf[4],
+                     q[NVFP4].tensor_scale)
+    mc = mw.c()
+    qc = [q[f].c() for f in (MXFP4, INT4_G32, NVFP4)]
+    _ok(_lib.mxq_mixed_prepare(ctypes.byref(qc[0]), ctypes.byref(qc[1]), ctypes.byref(qc[2]), ctypes.byref(mc),
+                               _stream(stream)), "mxq_mixed_prepare")
+    mw._keep = q   # the NVFP4 tensor scale lives in the NVFP4 quantization
+    return mw
+
+
+def qlinear_mixed_workspace_bytes(m: int, mw: MixedWeight, out_dtype=torch.bfloat16) -> int:
+    mc = mw.c()
+    return _size(_lib.mxq_qlinear_mixed_workspace_bytes, m, ctypes.byref(mc), BF16 if out_dtype == torch.bfloat16 else F32)
+
+
+def qlinear_mixed(xq: QTensor, mw: MixedWeight, out_dtype=torch.bfloat16, out: torch.Tensor = None,
+                  workspace: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """y = deq(xq) . deq(W)^T for an MXFP8 (MMA layout) activation and a
+    weight with per-channel formats."""
+    m = xq.rows
+    y = out if out is not None else torch.empty((m, mw.rows), dtype=out_dtype, device=xq.codes.device)
+    mc, xc = mw.c(), xq.c()
+    wsb = _size(_lib.mxq_qlinear_mixed_workspace_bytes, m, ctypes.byref(mc), _dtype_code(y))
+    if workspace is None:
+        workspace = torch.empty(max(wsb, 1), dtype=torch.uint8, device=xq.codes.device)
+    _ok(_lib.mxq_qlinear_mixed(ctypes.byref(xc), ctypes.byref(mc), _ptr(y), _dtype_code(y), _ptr(workspace),
+                               workspace.numel(), _stream(stream)), "mxq_qlinear_mixed")
+    return y
 
 
 def check(stream=None) -> int:

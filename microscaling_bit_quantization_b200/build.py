@@ -10,7 +10,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libmxq.so")
-SOURCES = ["quantize.cu", "mse.cu", "lowrank.cu", "lowrank_tc.cu", "gemm.cu", "gemm_igroup.cu", "w4a16.cu", "capi.cu"]
+SOURCES = ["quantize.cu", "mse.cu", "lowrank.cu", "lowrank_tc.cu", "gemm.cu", "gemm_igroup.cu", "w4a16.cu", "mixed.cu",
+           "capi.cu"]
 HEADERS = ["mxq_formats.cuh", "mxq_internal.h", "tc_ptx.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

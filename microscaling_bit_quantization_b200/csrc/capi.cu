@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "../../include/mxq.h"
@@ -175,7 +176,7 @@ mxq_status mxq_cast(const float *x, int64_t n, int32_t elem, uint8_t *out, void 
 
 mxq_status mxq_select_workspace_bytes(const int32_t *candidates, int32_t ncand, size_t *bytes) {
     if (!candidates || ncand < 1 || ncand > kMaxCandidates || !bytes) return MXQ_EINVAL;
-    *bytes = 16;
+    *bytes = kLrHeader;   // the amax word, or per-CTA maxima from byte 256
     return MXQ_OK;
 }
 
@@ -191,7 +192,11 @@ mxq_status mxq_select_weight_format(const void *w, int32_t wdtype, int64_t n, in
     }
     if (n > 0 && (!w || !fmt_per_channel || !aligned16(w))) return MXQ_EINVAL;
     if (!workspace) return MXQ_EINVAL;
-    if (workspace_bytes < 16) return MXQ_ENOSPACE;
+    if (workspace_bytes < kLrHeader) return MXQ_ENOSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MXQ_EINVAL;
+    const cudaError_t e = launch_select_fixed(w, wdtype == MXQ_BF16, n, k, cands, ncand, fmt_per_channel, sse,
+                                              (float *)((char *)workspace + 256), (cudaStream_t)stream);
+    if (e != cudaErrorNotSupported) return from_cuda(e);
     return from_cuda(launch_select(w, wdtype == MXQ_BF16, n, k, cands, ncand, fmt_per_channel, sse,
                                    (unsigned int *)workspace, (cudaStream_t)stream));
 }
@@ -599,6 +604,189 @@ mxq_status mxq_qlinear_routed(const void *x, int32_t xdtype, int64_t m, int64_t 
     }
     if (st != MXQ_OK) return st;
     return mxq_qlinear(&xq, wq, tp, r > 0 ? layer_w->l2p : nullptr, y, ydtype, stream);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Per-channel mixed weight formats (mixed.cu).
+namespace {
+
+int mixed_group(int32_t f) { return f == MXQ_MXFP4 ? 0 : f == MXQ_INT4_G32 ? 1 : f == MXQ_NVFP4 ? 2 : -1; }
+
+bool valid_mixed_weight(const mxq_mixed_weight *w) {
+    if (!w || w->rows < 0 || w->cols <= 0 || w->cols % 32 || w->rows >= ((int64_t)1 << 31)) return false;
+    if (w->rows * (w->cols / 16) >= ((int64_t)1 << 31)) return false;
+    int64_t total = 0;
+    for (int g = 0; g < 3; g++) {
+        if (w->n_group[g] < 0) return false;
+        total += w->n_group[g];
+    }
+    if (total != w->rows) return false;
+    if (w->rows > 0 && (!w->choice || !w->group_index)) return false;
+    if (w->n_group[0] > 0 && (!w->mx_codes || !w->mx_scales || !aligned16(w->mx_codes))) return false;
+    if (w->n_group[1] > 0 && (!w->i4_codes || !w->i4_scales || !aligned16(w->i4_codes))) return false;
+    if (w->n_group[2] > 0 && (!w->nv_values || !w->nv_tensor_scale || !aligned16(w->nv_values))) return false;
+    return true;
+}
+
+struct MixedLayout {
+    size_t sx, abf, y[3], total;
+};
+
+MixedLayout mixed_layout(int64_t m, const mxq_mixed_weight *w, int32_t ydtype) {
+    MixedLayout L;
+    size_t off = 0;
+    auto take = [&off](size_t bytes) {
+        const size_t at = off;
+        off += (bytes + 255) / 256 * 256;
+        return at;
+    };
+    const int64_t k = w->cols;
+    L.sx = take(w->n_group[1] > 0 ? (size_t)(m * (k / 32) * 4) : 0);
+    L.abf = take(w->n_group[2] > 0 ? (size_t)(m * k * 2) : 0);
+    const size_t esz = ydtype == MXQ_BF16 ? 2 : 4;
+    for (int g = 0; g < 3; g++) L.y[g] = take((size_t)(m * w->n_group[g]) * esz);
+    L.total = off;
+    return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+mxq_status mxq_mixed_plan(const uint8_t *choice, int64_t n, int64_t n_group[3], int32_t *group_index) {
+    if (!n_group || n < 0 || n >= ((int64_t)1 << 31) || (n > 0 && (!choice || !group_index))) return MXQ_EINVAL;
+    int64_t cnt[3] = {0, 0, 0};
+    for (int64_t i = 0; i < n; i++) {
+        const int g = mixed_group(choice[i]);
+        if (g < 0) return MXQ_EINVAL;
+        group_index[i] = (int32_t)cnt[g]++;
+    }
+    for (int g = 0; g < 3; g++) n_group[g] = cnt[g];
+    return MXQ_OK;
+}
+
+mxq_status mxq_mixed_weight_bytes(const int64_t n_group[3], int64_t k, size_t bytes[5]) {
+    if (!n_group || !bytes || k <= 0 || k % 32) return MXQ_EINVAL;
+    for (int g = 0; g < 3; g++)
+        if (n_group[g] < 0 || n_group[g] * (k / 16) >= ((int64_t)1 << 31)) return MXQ_EINVAL;
+    bytes[0] = (size_t)(n_group[0] * k);
+    if (mxq_scales_bytes(MXQ_MXFP8, n_group[0], k, MXQ_LAYOUT_MMA, &bytes[1]) != MXQ_OK) return MXQ_EINVAL;
+    bytes[2] = (size_t)(n_group[1] * k);
+    bytes[3] = (size_t)(n_group[1] * (k / 32) * 4);
+    bytes[4] = (size_t)(n_group[2] * k * 2);
+    return MXQ_OK;
+}
+
+mxq_status mxq_mixed_prepare(const mxq_qtensor *w_mxfp4, const mxq_qtensor *w_int4, const mxq_qtensor *w_nvfp4,
+                             const mxq_mixed_weight *out, void *stream) {
+    if (!w_mxfp4 || !w_int4 || !w_nvfp4 || !valid_mixed_weight(out)) return MXQ_EINVAL;
+    const mxq_qtensor *ws[3] = {w_mxfp4, w_int4, w_nvfp4};
+    const int32_t fmts[3] = {MXQ_MXFP4, MXQ_INT4_G32, MXQ_NVFP4};
+    for (int g = 0; g < 3; g++) {
+        const mxq_qtensor *q = ws[g];
+        if (q->fmt != fmts[g] || q->layout != MXQ_LAYOUT_CANONICAL || q->rows != out->rows || q->cols != out->cols)
+            return MXQ_EINVAL;
+        if (out->rows > 0 && (!q->codes || !q->scales)) return MXQ_EINVAL;
+    }
+    if (out->rows > 0 && !w_nvfp4->tensor_scale) return MXQ_EINVAL;
+    size_t bytes[5];
+    if (mxq_mixed_weight_bytes(out->n_group, out->cols, bytes) != MXQ_OK) return MXQ_EINVAL;
+    MixedPrep q;
+    q.n = out->rows;
+    q.k = out->cols;
+    for (int g = 0; g < 3; g++) q.n_group[g] = out->n_group[g];
+    q.choice = out->choice;
+    q.group_index = out->group_index;
+    q.mx_codes_c = w_mxfp4->codes;
+    q.mx_scales_c = w_mxfp4->scales;
+    q.i4_codes_c = w_int4->codes;
+    q.i4_scales_c = (const float *)w_int4->scales;
+    q.nv_codes_c = w_nvfp4->codes;
+    q.nv_scales_c = w_nvfp4->scales;
+    q.mx_codes = out->mx_codes;
+    q.mx_scales = out->mx_scales;
+    q.mx_scales_bytes = out->n_group[0] > 0 ? bytes[1] : 0;
+    q.i4_codes = out->i4_codes;
+    q.i4_scales = out->i4_scales;
+    q.nv_vals = out->nv_values;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = launch_mixed_prep(q, s);
+    if (e == cudaSuccess && out->n_group[2] > 0 && out->nv_tensor_scale != w_nvfp4->tensor_scale)
+        e = cudaMemcpyAsync((void *)out->nv_tensor_scale, w_nvfp4->tensor_scale, sizeof(float),
+                            cudaMemcpyDeviceToDevice, s);
+    return from_cuda(e);
+}
+
+mxq_status mxq_qlinear_mixed_workspace_bytes(int64_t m, const mxq_mixed_weight *w, int32_t ydtype, size_t *bytes) {
+    if (!bytes || m < 0 || m >= ((int64_t)1 << 31) || !valid_dtype(ydtype) || !valid_mixed_weight(w)) return MXQ_EINVAL;
+    *bytes = mixed_layout(m, w, ydtype).total;
+    return MXQ_OK;
+}
+
+mxq_status mxq_qlinear_mixed(const mxq_qtensor *xq, const mxq_mixed_weight *w, void *y, int32_t ydtype,
+                             void *workspace, size_t workspace_bytes, void *stream) {
+    if (!xq || !valid_dtype(ydtype) || !valid_mixed_weight(w)) return MXQ_EINVAL;
+    if (xq->fmt != MXQ_MXFP8 || xq->layout != MXQ_LAYOUT_MMA || xq->cols != w->cols) return MXQ_EINVAL;
+    const int64_t m = xq->rows, n = w->rows, k = w->cols;
+    if (!valid_shape(MXQ_MXFP8, m, k) || m >= ((int64_t)1 << 31)) return MXQ_EINVAL;
+    // the GEMM kernels count output tiles and their K stages in 32-bit integers
+    const int64_t tiles = ((m + 127) / 128) * ((n + 127) / 128);
+    if (tiles >= ((int64_t)1 << 31) || tiles * (k / 16) >= ((int64_t)1 << 31)) return MXQ_EINVAL;
+    if (m == 0 || n == 0) return MXQ_OK;
+    if (!y || !aligned16(y) || !xq->codes || !xq->scales || !aligned16(xq->codes)) return MXQ_EINVAL;
+    size_t need = 0;
+    mxq_qlinear_mixed_workspace_bytes(m, w, ydtype, &need);
+    if (!workspace) return MXQ_EINVAL;
+    if (workspace_bytes < need) return MXQ_ENOSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MXQ_EINVAL;
+    const MixedLayout L = mixed_layout(m, w, ydtype);
+    uint8_t *ws = (uint8_t *)workspace;
+    cudaStream_t s = (cudaStream_t)stream;
+    const bool ybf = ydtype == MXQ_BF16;
+    cudaError_t e = cudaSuccess;
+    const void *ybuf[3] = {ws + L.y[0], ws + L.y[1], ws + L.y[2]};
+    auto operands = [&](int fmt, int64_t rows_b, int g) {
+        GemmOperands op;
+        memset(&op, 0, sizeof(op));
+        op.fmt = fmt;
+        op.m = m;
+        op.n = rows_b;
+        op.k = k;
+        op.y = (void *)ybuf[g];
+        op.y_bf16 = ybf;
+        return op;
+    };
+    if (w->n_group[0] > 0) {   // MXFP4 rows as E4M3 against the MXFP8 codes, block scales on the tensor cores
+        GemmOperands op = operands(MXQ_MXFP8, w->n_group[0], 0);
+        op.a_codes = xq->codes;
+        op.a_scales = xq->scales;
+        op.b_codes = w->mx_codes;
+        op.b_scales = w->mx_scales;
+        e = launch_qlinear(op, s);
+    }
+    if (e == cudaSuccess && w->n_group[1] > 0) {   // INT4-g32 rows: per-group products, scales in the epilogue
+        float *sx = (float *)(ws + L.sx);
+        e = launch_mx_scales_f32(xq->scales, m, k, sx, s);
+        GemmOperands op = operands(MXQ_INT4_G32, w->n_group[1], 1);
+        op.a_codes = xq->codes;
+        op.a_scales = sx;
+        op.b_codes = w->i4_codes;
+        op.b_scales = w->i4_scales;
+        if (e == cudaSuccess) e = launch_qlinear_igroup(op, s);
+    }
+    if (e == cudaSuccess && w->n_group[2] > 0) {   // NVFP4 rows as bf16 against the bf16 activation
+        void *abf = ws + L.abf;
+        e = launch_dequantize(MXQ_MXFP8, MXQ_LAYOUT_MMA, m, k, xq->codes, xq->scales, nullptr, abf, true, s);
+        GemmOperands op = operands(MXQ_NVFP4, w->n_group[2], 2);
+        op.a_codes = abf;
+        op.b_codes = w->nv_values;
+        op.b_tensor_scale = w->nv_tensor_scale;
+        if (e == cudaSuccess) e = launch_gemm_bf16(op, s);
+    }
+    if (e == cudaSuccess) e = launch_mixed_scatter(ybuf, w->n_group, w->choice, w->group_index, y, ybf, m, n, s);
+    return from_cuda(e);
 }
 
 }  // extern "C"

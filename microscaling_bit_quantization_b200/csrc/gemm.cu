@@ -79,6 +79,7 @@ constexpr uint32_t TMEM_COLS = 512;
 #ifndef MXQ_SF_GROUPS
 #define MXQ_SF_GROUPS 2
 #endif
+
 constexpr uint32_t SF_GROUPS = MXQ_SF_GROUPS;
 constexpr uint32_t SF_SLOT_COLS = 12, SF_GROUP_COLS = 48;
 constexpr uint32_t TMEM_SF = TMEM_COLS - SF_GROUPS * SF_GROUP_COLS;
@@ -86,7 +87,9 @@ constexpr uint32_t ACC_STAGE1 = (TMEM_SF - 256) & ~31u;    // 32-column aligned
 constexpr uint32_t OVL_CHUNKS = (256 - ACC_STAGE1) / 32;   // shared 32-column chunks
 static_assert(ACC_STAGE1 + 256 <= TMEM_SF && OVL_CHUNKS >= 1 && OVL_CHUNKS <= 8, "TMEM budget");
 
-enum Kind : int { kKindNVFP4 = 0, kKindMXFP4 = 1, kKindMXFP8 = 2, kKindFP8 = 3, kKindINT8 = 4 };
+// kKindBF16: bf16 x bf16 operands on kind::f16 (no block scales), the
+// epilogue scale the B operand's tensor scale when it has one.
+enum Kind : int { kKindNVFP4 = 0, kKindMXFP4 = 1, kKindMXFP8 = 2, kKindFP8 = 3, kKindINT8 = 4, kKindBF16 = 5 };
 
 constexpr unsigned int kErrTimeoutProducer = 1u, kErrTimeoutMma = 2u, kErrTimeoutEpilogue = 4u;
 
@@ -370,6 +373,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                                 const uint32_t id = (uint32_t)ks;
                                 mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>() | (id << 29) | (id << 4),
                                                        accum, base, base + 4);
+                            } else if (KIND == kKindBF16) {
+                                mma_bf16(acc_addr, ad, bd, idesc_bf16(), accum);
                             } else {
                                 mma_plain<KIND>(acc_addr, ad, bd, idesc_main<KIND>(), accum);
                             }
@@ -461,6 +466,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + (st ? ACC_STAGE1 : 0u);
             float alpha = 1.0f, ra = 0.0f;
             if (KIND == kKindNVFP4 || KIND == kKindFP8) alpha = __fmul_rn(__ldg(p.a_ts), __ldg(p.b_ts));
+            if (KIND == kKindBF16 && p.b_ts) alpha = __ldg(p.b_ts);
             const bool row_ok = row < p.m;
             if (KIND == kKindINT8 && row_ok) ra = __ldg(p.a_row_scale + row);
             // The shared columns (the last OVL_CHUNKS chunks of stage 0, the first OVL_CHUNKS of
@@ -617,18 +623,18 @@ cudaError_t launch_kind(const GemmParams &p, int grid, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_qlinear(const GemmOperands &op, cudaStream_t s) {
+static cudaError_t launch_gemm_common(const GemmOperands &op, bool bf16_operands, cudaStream_t s) {
     if (op.m == 0 || op.n == 0) return cudaSuccess;
     GemmParams p;
     memset(&p, 0, sizeof(p));
-    const bool is4 = op.fmt == kMXFP4 || op.fmt == kNVFP4;
-    const int64_t kbytes = is4 ? op.k / 2 : op.k;
+    const bool is4 = !bf16_operands && (op.fmt == kMXFP4 || op.fmt == kNVFP4);
+    const int64_t kbytes = bf16_operands ? op.k * 2 : is4 ? op.k / 2 : op.k;
     const auto SW128 = CU_TENSOR_MAP_SWIZZLE_128B, NOSW = CU_TENSOR_MAP_SWIZZLE_NONE;
     if (!encode_2d(&p.tma_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, op.a_codes, kbytes, op.m, kbytes, BKB, BM, SW128) ||
         !encode_2d(&p.tma_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, op.b_codes, kbytes, op.n, kbytes, BKB, BNH, SW128))
         return cudaErrorInvalidValue;
     const int blk = fmt_block(op.fmt);
-    const bool byte_sf = fmt_byte_scales(op.fmt);
+    const bool byte_sf = !bf16_operands && fmt_byte_scales(op.fmt);
     if (byte_sf) {
         // scale atoms as rows of 64 x 8-byte elements: (row tile, scale-column group) -> atom index
         const int64_t s_pad = ((op.k / blk) + 15) / 16 * 16;
@@ -669,6 +675,7 @@ cudaError_t launch_qlinear(const GemmOperands &op, cudaStream_t s) {
     const int tiles = p.m_tiles * p.n_tiles;
     const int clusters = tiles < sms / 2 ? tiles : sms / 2;
     const int grid = 2 * clusters;
+    if (bf16_operands) return launch_kind<kKindBF16>(p, grid, s);
     switch (op.fmt) {
     case kNVFP4: return launch_kind<kKindNVFP4>(p, grid, s);
     case kMXFP4: return launch_kind<kKindMXFP4>(p, grid, s);
@@ -678,6 +685,10 @@ cudaError_t launch_qlinear(const GemmOperands &op, cudaStream_t s) {
     default: return cudaErrorInvalidValue;
     }
 }
+
+cudaError_t launch_qlinear(const GemmOperands &op, cudaStream_t s) { return launch_gemm_common(op, false, s); }
+
+cudaError_t launch_gemm_bf16(const GemmOperands &op, cudaStream_t s) { return launch_gemm_common(op, true, s); }
 
 namespace {
 constexpr unsigned int kErrSelfTest = 64u;

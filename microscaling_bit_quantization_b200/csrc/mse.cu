@@ -397,9 +397,15 @@ cudaError_t launch_fit_mx_grid(const void *w, bool bf16, int64_t rows, int64_t c
     return cudaGetLastError();
 }
 
-size_t calib_workspace_bytes(int64_t rows, int64_t cols, int ncand) {
+// Layout: the amax word at 0, per-row errors from 256, the row choices, the
+// moment partials (16-byte aligned), row and group sums; then, at a 256-byte
+// boundary, the per-CTA maxima of the fixed-set selection.
+static size_t calib_base_bytes(int64_t rows, int64_t cols, int ncand) {
     return 256 + (size_t)rows * ncand * 8 + (size_t)rows + 15 + (size_t)(rows * (cols / 16)) * 16 +
            (size_t)rows * 16 + (size_t)((rows + kMseGroup - 1) / kMseGroup) * 16 + 64;
+}
+size_t calib_workspace_bytes(int64_t rows, int64_t cols, int ncand) {
+    return (calib_base_bytes(rows, cols, ncand) + 255) / 256 * 256 + kLrHeader;
 }
 
 cudaError_t launch_calibrate(const void *x, bool bf16, int64_t rows, int64_t cols, const int *cands, int ncand,
@@ -412,7 +418,9 @@ cudaError_t launch_calibrate(const void *x, bool bf16, int64_t rows, int64_t col
     const int64_t chunks = rows * (cols / 16);
     double *row_sums = mom + 2 * chunks;
     double *grp_sums = row_sums + 2 * rows;
-    cudaError_t e = launch_select(x, bf16, rows, cols, cands, ncand, choice, sse_rows, amax, s);
+    float *slots = (float *)((char *)workspace + (calib_base_bytes(rows, cols, ncand) + 255) / 256 * 256);
+    cudaError_t e = launch_select_fixed(x, bf16, rows, cols, cands, ncand, choice, sse_rows, slots, s);
+    if (e == cudaErrorNotSupported) e = launch_select(x, bf16, rows, cols, cands, ncand, choice, sse_rows, amax, s);
     if (e != cudaSuccess) return e;
     for (int j = 0; j < ncand; j++)
         launch_sums<1, kFinAccumulate>(sse_rows + j, ncand, rows, 1, rows, row_sums, grp_sums, nullptr,

@@ -115,6 +115,13 @@ cudaError_t launch_hadamard(const void *x, void *y, bool bf16, int64_t rows, int
 cudaError_t launch_cast(const float *x, int64_t n, int elem, uint8_t *out, cudaStream_t s);
 cudaError_t launch_select(const void *w, bool bf16, int64_t n, int64_t k, const int *cands, int ncand,
                           uint8_t *choice, double *sse, unsigned int *amax_word, cudaStream_t s);
+// The same selection for the fixed candidate sets {MXFP4, NVFP4, INT4_G32}
+// and {MXFP8, INT8_ROW, FP8_TENSOR} (any order) with k % 64 == 0, by a kernel
+// specialized to the set; amax_slots: room for 2 x SM-count floats (the
+// per-CTA maxima of the tensor-amax pass).  Returns cudaErrorNotSupported,
+// launching nothing, for other sets and shapes.
+cudaError_t launch_select_fixed(const void *w, bool bf16, int64_t n, int64_t k, const int *cands, int ncand,
+                                uint8_t *choice, double *sse, float *amax_slots, cudaStream_t s);
 
 // t (m x r fp32) when tp is null; else the packed GEMM operand tp (m x 64
 // bf16, [hi | lo] of t / (xs * ws), xs = ws = null meaning 1).  With
@@ -149,6 +156,10 @@ struct GemmOperands {
     bool y_bf16;
 };
 cudaError_t launch_qlinear(const GemmOperands &op, cudaStream_t s);
+// bf16 x bf16 operands (a_codes m x k, b_codes n x k, k % 16 == 0) on the
+// same kernel with kind::f16 MMAs; y = acc * (*b_tensor_scale, or 1 when
+// null); no low-rank branch (tp must be null).
+cudaError_t launch_gemm_bf16(const GemmOperands &op, cudaStream_t s);
 // INT4_G32 / INT4_G64 operands (E4M3 code bytes, transposed fp32 group scales).
 cudaError_t launch_qlinear_igroup(const GemmOperands &op, cudaStream_t s);
 
@@ -156,6 +167,29 @@ cudaError_t launch_qlinear_igroup(const GemmOperands &op, cudaStream_t s);
 // driver entry point; false when the driver rejects it.
 bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
                uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
+
+// Per-channel mixed weight formats (mixed.cu).  Groups in the order MXFP4,
+// INT4_G32, NVFP4; group_index[n] is channel n's row in its group.
+struct MixedPrep {
+    int64_t n, k, n_group[3];
+    const uint8_t *choice;                  // device uint8[n]
+    const int32_t *group_index;             // device int32[n]
+    const void *mx_codes_c, *mx_scales_c;   // the whole weight in canonical MXFP4
+    const void *i4_codes_c;                 // ... in canonical INT4_G32
+    const float *i4_scales_c;
+    const void *nv_codes_c, *nv_scales_c;   // ... in canonical NVFP4
+    void *mx_codes, *mx_scales;             // outputs (see mxq_mixed_weight in mxq.h)
+    size_t mx_scales_bytes;
+    void *i4_codes;
+    float *i4_scales;
+    void *nv_vals;
+};
+cudaError_t launch_mixed_prep(const MixedPrep &q, cudaStream_t s);
+// E8M0 scales (MMA layout) of an m x k MX tensor as fp32 [k/32][m].
+cudaError_t launch_mx_scales_f32(const void *scales_mma, int64_t m, int64_t k, float *out, cudaStream_t s);
+cudaError_t launch_mixed_scatter(const void *const ybuf[3], const int64_t n_group[3], const uint8_t *choice,
+                                 const int32_t *group_index, void *y, bool y_bf16, int64_t m, int64_t n,
+                                 cudaStream_t s);
 
 // Device error word (bounded waits that ran out); read-and-clear, and its
 // device address on the current device (for kernels of other files).

@@ -630,6 +630,255 @@ __global__ void __launch_bounds__(kThreads) k_select(const T *__restrict__ w, Se
     }
 }
 
+// ------------------------------------------------------------------ selection over a fixed format set
+//
+// The same errors for the candidate sets the library is used with -- the
+// Chameleon weight set {MXFP4, NVFP4, INT4-g32} and the W8A8 activation set
+// {MXFP8, INT8 per row, FP8 per tensor} -- with the formats fixed at compile
+// time (MASK, one bit per format), codes taken by the bracketed-reciprocal
+// codecs of the quantizer instead of an IEEE division per element, and the
+// next chunk of the row prefetched while the current one is scored.  Each
+// error term is formed exactly: for the MX formats d = v - q 2^e is exact in
+// fp32 (q 2^e has at most 4 significant bits and, unless q = 0 where d = v,
+// lies within a few binades of v, so d is a multiple of v's last place below
+// 2^24 of them); for the others d = v - q S (S the exact binary64 product of
+// the scales) is one binary64 FMA, exact because q S and v are within a few
+// binades of each other.  The square is added with one binary64 FMA.  The
+// caller's candidate order only decides the reported order and ties.
+
+constexpr uint32_t kSelSetW4 = (1u << kMXFP4) | (1u << kNVFP4) | (1u << kINT4G32);
+constexpr uint32_t kSelSetA8 = (1u << kMXFP8) | (1u << kINT8Row) | (1u << kFP8Tensor);
+constexpr int kSelThreads = 256;
+
+__host__ __device__ constexpr int sel_slot(uint32_t mask, int f) {
+    int n = 0;
+    for (int i = 0; i < f; i++) n += (mask >> i) & 1u;
+    return n;
+}
+__host__ __device__ constexpr int sel_count(uint32_t mask) { return sel_slot(mask, kNumFmt); }
+
+struct SelectSetArgs {
+    int64_t n, k;
+    int ncand;
+    int slot[kMaxCandidates];        // slot of caller's candidate j in the kernel's format order
+    int cand[kMaxCandidates];
+    const float *amax_slots;         // tensor amax = max of n_slots values
+    int n_slots;
+    uint8_t *choice;
+    double *sse;                     // may be null
+};
+
+// E2M1 code (sign in bit 3) as fp32 / binary64, from its bits.
+__device__ __forceinline__ float e2m1_bits_f32(uint32_t c) {
+    const uint32_t m = c & 7u;
+    const uint32_t b = m >= 2u ? (m + 252u) << 22 : (m ? 0x3F000000u : 0u);
+    return __uint_as_float(b | ((c & 8u) << 28));
+}
+__device__ __forceinline__ double e2m1_bits_f64(uint32_t c) {
+    const uint32_t m = c & 7u;
+    const uint32_t hi = m >= 2u ? (m + 2044u) << 19 : (m ? 0x3FE00000u : 0u);
+    return __hiloint2double((int)(hi | ((c & 8u) << 28)), 0);
+}
+// Four E4M3 codes (bytes of c) as fp32 (exact: every E4M3 value is an fp16 value).
+__device__ __forceinline__ void e4m3x4_f32(uint32_t c, float *o) {
+    uint32_t h0, h1;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, lo;\n\tcvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+        : "=r"(h0), "=r"(h1)
+        : "r"(c));
+    o[0] = __half2float(__ushort_as_half((unsigned short)(h0 & 0xFFFFu)));
+    o[1] = __half2float(__ushort_as_half((unsigned short)(h0 >> 16)));
+    o[2] = __half2float(__ushort_as_half((unsigned short)(h1 & 0xFFFFu)));
+    o[3] = __half2float(__ushort_as_half((unsigned short)(h1 >> 16)));
+}
+
+// acc += sum (v - q 2^e)^2 over one chunk of an MX block with maximum amax.
+template <int F>
+__device__ __forceinline__ void sel_err_mx(const float (&v)[16], float amax, double &acc) {
+    if (!(amax > 0.0f)) return;   // all values are +-0 and all codes zero
+    float inv;
+    const int e = (int)mx_scale(amax, F == kMXFP8 ? 8 : 2, inv) - 127;
+    const float X = exp2i_f32(e);
+    float u[16];
+    mul8(v, inv, u);
+    mul8(v + 8, inv, u + 8);
+    if (F == kMXFP4) {
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+            const uint32_t c = cvt_e2m1x8(u[8 * h], u[8 * h + 1], u[8 * h + 2], u[8 * h + 3], u[8 * h + 4],
+                                          u[8 * h + 5], u[8 * h + 6], u[8 * h + 7]);
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                const float d = __fmaf_rn(-e2m1_bits_f32(c >> (4 * i)), X, v[8 * h + i]);
+                const double dd = (double)d;
+                acc = __fma_rn(dd, dd, acc);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int h = 0; h < 4; h++) {
+            float q[4];
+            e4m3x4_f32(cvt_e4m3x4(u[4 * h], u[4 * h + 1], u[4 * h + 2], u[4 * h + 3]), q);
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const float d = __fmaf_rn(-q[i], X, v[4 * h + i]);
+                const double dd = (double)d;
+                acc = __fma_rn(dd, dd, acc);
+            }
+        }
+    }
+}
+
+// acc += sum (v - q e4 s_t)^2 over one NVFP4 block.
+__device__ __forceinline__ void sel_err_nvfp4(const float (&v)[16], const double (&vd)[16], float amax,
+                                              const TensorRecip &tr, double st, double &acc) {
+    float dsc;
+    const uint32_t e4 = nvfp4_block_scale_fast(amax, tr, dsc);
+    if (!e4) {   // all codes zero
+#pragma unroll
+        for (int i = 0; i < 16; i++) acc = __fma_rn(vd[i], vd[i], acc);
+        return;
+    }
+    const Recip r = recip_of(dsc);
+    const uint32_t c0 = e2m1x8_quot(v, r), c1 = e2m1x8_quot(v + 8, r);
+    const double S = __dmul_rn((double)e4m3_to_f32(e4), st);   // exact: 4 x 24 significant bits
+#pragma unroll
+    for (int i = 0; i < 16; i++) {
+        const double d = __fma_rn(-e2m1_bits_f64((i < 8 ? c0 : c1) >> (4 * (i & 7))), S, vd[i]);
+        acc = __fma_rn(d, d, acc);
+    }
+}
+
+// acc += sum (v - q s)^2 for symmetric integer codes with scale s.
+__device__ __forceinline__ void sel_err_int(const float (&v)[16], const double (&vd)[16], float s, int qmax,
+                                            double &acc) {
+    if (s == 0.0f) {   // all codes zero
+#pragma unroll
+        for (int i = 0; i < 16; i++) acc = __fma_rn(vd[i], vd[i], acc);
+        return;
+    }
+    const Recip r = recip_of(s);
+    const double sd = (double)s;
+#pragma unroll
+    for (int h = 0; h < 4; h++) {
+        const uint32_t b = int_x4_quot(v + 4 * h, r, qmax);
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const double q = (double)(int)(int8_t)(uint8_t)(b >> (8 * i));
+            const double d = __fma_rn(-q, sd, vd[4 * h + i]);
+            acc = __fma_rn(d, d, acc);
+        }
+    }
+}
+
+// acc += sum (v - q s)^2 for E4M3 codes of v / s (FP8 per tensor).
+__device__ __forceinline__ void sel_err_fp8t(const float (&v)[16], const double (&vd)[16], const Recip &rt, double sd,
+                                             double &acc) {
+#pragma unroll
+    for (int h = 0; h < 4; h++) {
+        float q[4];
+        e4m3x4_f32(e4m3x4_quot(v + 4 * h, rt), q);
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const double d = __fma_rn(-(double)q[i], sd, vd[4 * h + i]);
+            acc = __fma_rn(d, d, acc);
+        }
+    }
+}
+
+template <typename T, uint32_t MASK>
+__global__ void __launch_bounds__(kSelThreads) k_select_set(const T *__restrict__ w, SelectSetArgs a) {
+    constexpr int NS = sel_count(MASK);
+    constexpr bool kTensor = (MASK & ((1u << kNVFP4) | (1u << kFP8Tensor))) != 0;
+    constexpr bool kRow = (MASK & (1u << kINT8Row)) != 0;
+    constexpr bool kNeedVd = (MASK & ~((1u << kMXFP4) | (1u << kMXFP8))) != 0;
+    const int lane = lane_id();
+    const int64_t warp = ((int64_t)blockIdx.x * kSelThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * kSelThreads) >> 5;
+    const int cpr = (int)(a.k >> 4);
+    // launched right after the tensor-amax pass: nothing global is read before it completes
+    pdl_wait();
+    pdl_launch_dependents();
+    float tamax = 0.0f;
+    if (kTensor) tamax = cta_max_of<kSelThreads>(a.amax_slots, a.n_slots);
+    const float st_nv = nvfp4_tensor_scale(tamax), st_f8 = fp8_tensor_scale(tamax);
+    const TensorRecip tr = tensor_recip_of(st_nv);
+    const Recip rf8 = recip_of(st_f8);
+    for (int64_t row = warp; row < a.n; row += nwarps) {
+        const T *wr = w + row * a.k;
+        float rowamax = 0.0f;
+        if (kRow) {
+            for (int c = lane; c < cpr; c += 32) {
+                float v[16];
+                load16(wr + (int64_t)c * 16, v);
+                rowamax = fmaxf(rowamax, amax16(v));
+            }
+            rowamax = group_max<32>(rowamax);
+        }
+        const float s_row = __fdiv_rn(rowamax, 127.0f);
+        double acc[NS];
+#pragma unroll
+        for (int j = 0; j < NS; j++) acc[j] = 0.0;
+        RawChunk<T> pre;
+        if (lane < cpr) raw_load(pre, wr + (int64_t)lane * 16);
+        for (int c0 = 0; c0 < cpr; c0 += 32) {
+            const int c = c0 + lane;
+            float v[16];
+            if (c < cpr) raw_unpack(pre, v);
+            else {
+#pragma unroll
+                for (int i = 0; i < 16; i++) v[i] = 0.0f;
+            }
+            if (c + 32 < cpr) raw_load(pre, wr + (int64_t)(c + 32) * 16);
+            // lanes past the row end hold zeros: their blocks (whole groups of
+            // lanes, since k % 64 == 0) add nothing
+            const float m1 = amax16(v);
+            const float m2 = group_max<2>(m1);
+            double vd[16];
+            if (kNeedVd) {
+#pragma unroll
+                for (int i = 0; i < 16; i++) vd[i] = (double)v[i];
+            }
+            if (MASK & (1u << kMXFP8)) sel_err_mx<kMXFP8>(v, m2, acc[sel_slot(MASK, kMXFP8)]);
+            if (MASK & (1u << kMXFP4)) sel_err_mx<kMXFP4>(v, m2, acc[sel_slot(MASK, kMXFP4)]);
+            if (MASK & (1u << kNVFP4)) sel_err_nvfp4(v, vd, m1, tr, (double)st_nv, acc[sel_slot(MASK, kNVFP4)]);
+            if (MASK & (1u << kINT4G32)) sel_err_int(v, vd, __fdiv_rn(m2, 7.0f), 7, acc[sel_slot(MASK, kINT4G32)]);
+            if (MASK & (1u << kINT4G64))
+                sel_err_int(v, vd, __fdiv_rn(group_max<4>(m2), 7.0f), 7, acc[sel_slot(MASK, kINT4G64)]);
+            if (MASK & (1u << kINT8Row)) sel_err_int(v, vd, s_row, 127, acc[sel_slot(MASK, kINT8Row)]);
+            if (MASK & (1u << kFP8Tensor)) sel_err_fp8t(v, vd, rf8, (double)st_f8, acc[sel_slot(MASK, kFP8Tensor)]);
+        }
+#pragma unroll
+        for (int j = 0; j < NS; j++) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc[j] = __dadd_rn(acc[j], __shfl_xor_sync(0xFFFFFFFFu, acc[j], o));
+        }
+        if (lane == 0) {
+            int best = 0;
+            double bestv = 0.0;
+#pragma unroll
+            for (int j = 0; j < kMaxCandidates; j++) {
+                if (j < a.ncand) {
+                    double s = 0.0;
+#pragma unroll
+                    for (int t = 0; t < NS; t++)
+                        if (t == a.slot[j]) s = acc[t];
+                    if (a.sse) a.sse[row * a.ncand + j] = s;
+                    if (j == 0 || s < bestv) {
+                        best = j;
+                        bestv = s;
+                    }
+                }
+            }
+            int fmt = a.cand[0];
+#pragma unroll
+            for (int j = 1; j < kMaxCandidates; j++)
+                if (j == best) fmt = a.cand[j];
+            a.choice[row] = (uint8_t)fmt;
+        }
+    }
+}
+
 }  // namespace
 
 // ====================================================================== host
@@ -814,6 +1063,64 @@ cudaError_t launch_cast(const float *x, int64_t n, int elem, uint8_t *out, cudaS
     int64_t ctas = (n + kThreads - 1) / kThreads;
     int grid = (int)(ctas > (int64_t)sm_count_cached() * 16 ? (int64_t)sm_count_cached() * 16 : ctas);
     k_cast<<<grid, kThreads, 0, s>>>(x, n, elem, out);
+    return cudaGetLastError();
+}
+
+// The candidate set as a format mask when it is one of the fixed sets with
+// distinct formats (0 otherwise).
+static uint32_t select_set_of(const int *cands, int ncand) {
+    uint32_t mask = 0;
+    for (int j = 0; j < ncand; j++) {
+        if (mask & (1u << cands[j])) return 0;   // repeated format
+        mask |= 1u << cands[j];
+    }
+    return (mask == kSelSetW4 || mask == kSelSetA8) ? mask : 0u;
+}
+
+template <typename T, uint32_t MASK>
+static void launch_select_set(const T *w, const SelectSetArgs &a, cudaStream_t s) {
+    const int64_t ctas = (a.n + kSelThreads / 32 - 1) / (kSelThreads / 32);
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)(ctas < 1 ? 1 : ctas), 1, 1);
+    cfg.blockDim = dim3(kSelThreads, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1] = {pdl_attribute()};
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, k_select_set<T, MASK>, w, a);
+}
+
+cudaError_t launch_select_fixed(const void *w, bool bf16, int64_t n, int64_t k, const int *cands, int ncand,
+                                uint8_t *choice, double *sse, float *amax_slots, cudaStream_t s) {
+    const uint32_t mask = select_set_of(cands, ncand);
+    if (!mask || k % 64 || n * (k / 16) >= ((int64_t)1 << 31)) return cudaErrorNotSupported;
+    SelectSetArgs a;
+    memset(&a, 0, sizeof(a));
+    a.n = n;
+    a.k = k;
+    a.ncand = ncand;
+    for (int j = 0; j < ncand; j++) {
+        a.cand[j] = cands[j];
+        a.slot[j] = sel_slot(mask, cands[j]);
+    }
+    a.choice = choice;
+    a.sse = sse;
+    if (mask & ((1u << kNVFP4) | (1u << kFP8Tensor))) {
+        // per-CTA maxima of |w| (every slot written, no clearing), read by the
+        // selection kernel launched right behind it
+        cudaError_t e = launch_amax_slots(w, bf16, n, k, 0, amax_slots, &a.n_slots, s);
+        if (e != cudaSuccess) return e;
+        a.amax_slots = amax_slots;
+    }
+    if (n == 0) return cudaSuccess;
+    if (mask == kSelSetW4) {
+        if (bf16) launch_select_set<__nv_bfloat16, kSelSetW4>((const __nv_bfloat16 *)w, a, s);
+        else launch_select_set<float, kSelSetW4>((const float *)w, a, s);
+    } else {
+        if (bf16) launch_select_set<__nv_bfloat16, kSelSetA8>((const __nv_bfloat16 *)w, a, s);
+        else launch_select_set<float, kSelSetA8>((const float *)w, a, s);
+    }
     return cudaGetLastError();
 }
 

@@ -247,6 +247,33 @@ def test_routed_workspace_and_argument_checks(mxq):
     assert call(step=0) == 1                     # weight K differs from x
 
 
+def test_mixed_plan_and_sizes(mxq):
+    L = mxq.lib()
+    ch = np.array([1, 2, 3, 2, 1, 1, 3, 2, 2], np.uint8)
+    ng = (ctypes.c_int64 * 3)()
+    gi = np.zeros(len(ch), np.int32)
+    assert L.mxq_mixed_plan(ch.ctypes.data_as(ctypes.c_void_p), len(ch), ng, gi.ctypes.data_as(ctypes.c_void_p)) == 0
+    assert list(ng) == [3, 2, 4]
+    assert gi.tolist() == [0, 0, 0, 1, 1, 2, 1, 2, 3]
+    bad = np.array([1, 0], np.uint8)   # MXFP8 is not a weight candidate
+    assert L.mxq_mixed_plan(bad.ctypes.data_as(ctypes.c_void_p), 2, ng, gi.ctypes.data_as(ctypes.c_void_p)) == 1
+    sizes = (ctypes.c_size_t * 5)()
+    g3 = (ctypes.c_int64 * 3)(3, 2, 4)
+    assert L.mxq_mixed_weight_bytes(g3, 256, sizes) == 0
+    assert list(sizes) == [3 * 256, 128 * 16, 2 * 256, 2 * 8 * 4, 4 * 256 * 2]
+    assert L.mxq_mixed_weight_bytes(g3, 48, sizes) == 1    # k % 32
+    mw = mxq._MixedC(9, 256, (ctypes.c_int64 * 3)(3, 2, 4), 256, 256, 256, 256, 256, 256, 256, 256)
+    size = ctypes.c_size_t(0)
+    assert L.mxq_qlinear_mixed_workspace_bytes(100, ctypes.byref(mw), 1, ctypes.byref(size)) == 0
+    up = lambda b: (b + 255) // 256 * 256
+    assert size.value == up(100 * 8 * 4) + up(100 * 256 * 2) + up(100 * 3 * 2) + up(100 * 2 * 2) + up(100 * 4 * 2)
+    wrong = mxq._MixedC(9, 256, (ctypes.c_int64 * 3)(3, 2, 3), 256, 256, 256, 256, 256, 256, 256, 256)
+    assert L.mxq_qlinear_mixed_workspace_bytes(100, ctypes.byref(wrong), 1, ctypes.byref(size)) == 1   # counts != N
+    xq = mxq._QTensorC(mxq.NVFP4, mxq.MMA, 100, 256, 256, 256, 256)
+    assert L.mxq_qlinear_mixed(ctypes.byref(xq), ctypes.byref(mw), ctypes.c_void_p(256), 1, ctypes.c_void_p(256),
+                               1 << 30, None) == 1        # activation must be MXFP8
+
+
 def test_route_matches_oracle(mxq, orc):
     rng = np.random.default_rng(3)
     for n_layers, n_int, n_steps in ((112, 10, 20), (7, 3, 11), (1, 1, 1)):
