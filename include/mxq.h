@@ -511,8 +511,8 @@ mxq_status mxq_mixed_prepare(const mxq_qtensor *w_mxfp4, const mxq_qtensor *w_in
 
 /* Scratch bytes mxq_qlinear_mixed needs for m activation rows: the
  * activation's block scales as fp32 (INT4 group), the activation dequantized
- * to bf16 (NVFP4 group) and one m x n_group[g] output per group, each at a
- * 256-byte boundary. */
+ * to bf16 (NVFP4 group) and one m x n_group[g] output per group (none when
+ * one group holds every channel), each at a 256-byte boundary. */
 mxq_status mxq_qlinear_mixed_workspace_bytes(int64_t m, const mxq_mixed_weight *w, int32_t ydtype, size_t *bytes);
 
 /* y = deq(xq) . deq_f(W)^T, each output channel n dequantized in its own
@@ -522,7 +522,9 @@ mxq_status mxq_qlinear_mixed_workspace_bytes(int64_t m, const mxq_mixed_weight *
  * and the weight's group scale), the NVFP4 group on bf16 kind::f16 MMAs
  * against the activation dequantized to bf16 (exact while the block
  * exponents stay inside the bf16 range), times the tensor scale; then the
- * group outputs are scattered to channel order.  fp32 accumulation.
+ * group outputs are scattered to channel order (when one group holds every
+ * channel, its GEMM writes y directly: channel n is row n of the group, as
+ * mxq_mixed_plan numbers them).  fp32 accumulation.
  *   xq: MXQ_MXFP8, MMA layout, cols == w->cols.
  *   y: m x N device, ydtype MXQ_BF16 or MXQ_F32.
  *   workspace: device scratch of mxq_qlinear_mixed_workspace_bytes,

@@ -634,6 +634,15 @@ struct MixedLayout {
     size_t sx, abf, y[3], total;
 };
 
+// The group that holds every channel, or -1: channel n is then row n of that
+// group (mxq_mixed_plan keeps the channel order inside a group), so its GEMM
+// writes y directly and nothing is scattered.
+int mixed_single_group(const mxq_mixed_weight *w) {
+    for (int g = 0; g < 3; g++)
+        if (w->n_group[g] == w->rows && w->rows > 0) return g;
+    return -1;
+}
+
 MixedLayout mixed_layout(int64_t m, const mxq_mixed_weight *w, int32_t ydtype) {
     MixedLayout L;
     size_t off = 0;
@@ -646,7 +655,8 @@ MixedLayout mixed_layout(int64_t m, const mxq_mixed_weight *w, int32_t ydtype) {
     L.sx = take(w->n_group[1] > 0 ? (size_t)(m * (k / 32) * 4) : 0);
     L.abf = take(w->n_group[2] > 0 ? (size_t)(m * k * 2) : 0);
     const size_t esz = ydtype == MXQ_BF16 ? 2 : 4;
-    for (int g = 0; g < 3; g++) L.y[g] = take((size_t)(m * w->n_group[g]) * esz);
+    const int single = mixed_single_group(w);
+    for (int g = 0; g < 3; g++) L.y[g] = take(single >= 0 ? 0 : (size_t)(m * w->n_group[g]) * esz);
     L.total = off;
     return L;
 }
@@ -746,7 +756,9 @@ mxq_status mxq_qlinear_mixed(const mxq_qtensor *xq, const mxq_mixed_weight *w, v
     cudaStream_t s = (cudaStream_t)stream;
     const bool ybf = ydtype == MXQ_BF16;
     cudaError_t e = cudaSuccess;
+    const int single = mixed_single_group(w);
     const void *ybuf[3] = {ws + L.y[0], ws + L.y[1], ws + L.y[2]};
+    if (single >= 0) ybuf[single] = y;
     auto operands = [&](int fmt, int64_t rows_b, int g) {
         GemmOperands op;
         memset(&op, 0, sizeof(op));
@@ -785,7 +797,8 @@ mxq_status mxq_qlinear_mixed(const mxq_qtensor *xq, const mxq_mixed_weight *w, v
         op.b_tensor_scale = w->nv_tensor_scale;
         if (e == cudaSuccess) e = launch_gemm_bf16(op, s);
     }
-    if (e == cudaSuccess) e = launch_mixed_scatter(ybuf, w->n_group, w->choice, w->group_index, y, ybf, m, n, s);
+    if (e == cudaSuccess && single < 0)
+        e = launch_mixed_scatter(ybuf, w->n_group, w->choice, w->group_index, y, ybf, m, n, s);
     return from_cuda(e);
 }
 

@@ -22,8 +22,8 @@
 //               that issues the MMAs, committing to both CTAs' barriers
 //   warps 2-5   epilogue: TMEM -> registers -> scaling -> swizzled shared
 //               staging -> TMA bulk stores
-//   warps 6-7   in the first CTA, two threads that copy each stage's scale
-//               factors to TMEM (tcgen05.cp, even / odd atoms) and signal
+//   warps 6-    in the first CTA, kSfWarps threads that copy each stage's scale
+//               factors to TMEM (tcgen05.cp) and signal
 //               the MMA thread
 // The kernel is persistent: clusters walk the tiles, the TMA ring runs on
 // across tiles, and tiles alternate between two TMEM accumulator stages
@@ -66,7 +66,13 @@ constexpr int EPI_BUF = 4096;           // one 32-row x 128-byte staging buffer
 constexpr int EPI_BYTES = 4 * 2 * EPI_BUF;                  // 4 warps x 2 buffers
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
-constexpr int kGemmThreads = 256;   // 8 warps
+// Warps that copy scale factors to TMEM (warps 6 .. 6 + kSfWarps - 1), one
+// k-step's atoms (SFA and the one or two SFB atoms) per warp in turn: a
+// tcgen05.cp stalls the thread that issues it, so a stage's copies are
+// spread over several threads (NVFP4, workload 3: 2 warps 95.8 us, 4 warps
+// 93.7 us; dealing single copies round-robin instead was slower).
+constexpr int kSfWarps = 4;
+constexpr int kGemmThreads = 32 * (6 + kSfWarps);
 constexpr uint32_t TMEM_COLS = 512;
 // TMEM columns: accumulator stage 0 at [0, 256), stage 1 at
 // [ACC_STAGE1, ACC_STAGE1 + 256) (the two stages share 256 - ACC_STAGE1
@@ -251,7 +257,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
         mbar_init(ovlf, 8);
         mbar_init(drain, 1);
-        for (int i = 0; i < STAGES; i++) mbar_init(sfready + i, 2);   // one arrival per scale-factor warp
+        for (int i = 0; i < STAGES; i++) mbar_init(sfready + i, kSfWarps);   // one arrival per scale-factor warp
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -398,8 +404,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     } else if (warp >= 6) {
         // ---------------------------------------------------------- scale-factor copies (first CTA)
         // Issued apart from the MMA thread: a tcgen05.cp stalls the thread that
-        // issues it, but runs alongside the MMAs in the tensor pipe.  Two warps
-        // share the atoms of a stage (even / odd atoms).
+        // issues it, but runs alongside the MMAs in the tensor pipe.  The atoms
+        // of a stage are dealt to the kSfWarps warps in turn.
         const int par = warp - 6;
         if (NSF && lane == 0 && rank == 0) {
             int it = 0;
@@ -425,7 +431,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                         const uint8_t *sf = smem + s * STAGE_BYTES + A_STAGE + B_STAGE;
                         const uint32_t group = tmem + TMEM_SF + SF_GROUP_COLS * ((uint32_t)it % SF_GROUPS);
                         tc_fence_after();
-                        for (int a = par; a < natoms; a += 2) {
+                        for (int a = par; a < natoms; a += kSfWarps) {
                             const uint32_t base = group + SF_SLOT_COLS * (uint32_t)a;
                             tc_cp_pair(base, sdesc_sf(sf + 512 * a));
                             tc_cp_pair(base + 4, sdesc_sf(sf + 2048 + 512 * a));

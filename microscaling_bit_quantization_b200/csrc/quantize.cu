@@ -668,16 +668,21 @@ struct SelectSetArgs {
     double *sse;                     // may be null
 };
 
-// E2M1 code (sign in bit 3) as fp32 / binary64, from its bits.
-__device__ __forceinline__ float e2m1_bits_f32(uint32_t c) {
-    const uint32_t m = c & 7u;
-    const uint32_t b = m >= 2u ? (m + 252u) << 22 : (m ? 0x3F000000u : 0u);
-    return __uint_as_float(b | ((c & 8u) << 28));
+// The eight E2M1 codes packed in a word (element i in nibble i) as fp16
+// values (exact: every E2M1 value is an fp16 value), through the hardware
+// conversion.
+__device__ __forceinline__ void e2m1x8_to_half(uint32_t c, __half (&h)[8]) {
+#pragma unroll
+    for (int b = 0; b < 4; b++) {
+        const __half2_raw r = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)((c >> (8 * b)) & 0xFFu), __NV_E2M1);
+        h[2 * b] = __ushort_as_half(r.x);
+        h[2 * b + 1] = __ushort_as_half(r.y);
+    }
 }
-__device__ __forceinline__ double e2m1_bits_f64(uint32_t c) {
-    const uint32_t m = c & 7u;
-    const uint32_t hi = m >= 2u ? (m + 2044u) << 19 : (m ? 0x3FE00000u : 0u);
-    return __hiloint2double((int)(hi | ((c & 8u) << 28)), 0);
+__device__ __forceinline__ double half_to_f64(__half h) {
+    double d;
+    asm("cvt.f64.f16 %0, %1;" : "=d"(d) : "h"(__half_as_ushort(h)));
+    return d;
 }
 // Four E4M3 codes (bytes of c) as fp32 (exact: every E4M3 value is an fp16 value).
 __device__ __forceinline__ void e4m3x4_f32(uint32_t c, float *o) {
@@ -705,11 +710,13 @@ __device__ __forceinline__ void sel_err_mx(const float (&v)[16], float amax, dou
     if (F == kMXFP4) {
 #pragma unroll
         for (int h = 0; h < 2; h++) {
-            const uint32_t c = cvt_e2m1x8(u[8 * h], u[8 * h + 1], u[8 * h + 2], u[8 * h + 3], u[8 * h + 4],
-                                          u[8 * h + 5], u[8 * h + 6], u[8 * h + 7]);
+            __half q[8];
+            e2m1x8_to_half(cvt_e2m1x8(u[8 * h], u[8 * h + 1], u[8 * h + 2], u[8 * h + 3], u[8 * h + 4],
+                                      u[8 * h + 5], u[8 * h + 6], u[8 * h + 7]),
+                           q);
 #pragma unroll
             for (int i = 0; i < 8; i++) {
-                const float d = __fmaf_rn(-e2m1_bits_f32(c >> (4 * i)), X, v[8 * h + i]);
+                const float d = __fmaf_rn(-__half2float(q[i]), X, v[8 * h + i]);
                 const double dd = (double)d;
                 acc = __fma_rn(dd, dd, acc);
             }
@@ -740,12 +747,16 @@ __device__ __forceinline__ void sel_err_nvfp4(const float (&v)[16], const double
         return;
     }
     const Recip r = recip_of(dsc);
-    const uint32_t c0 = e2m1x8_quot(v, r), c1 = e2m1x8_quot(v + 8, r);
     const double S = __dmul_rn((double)e4m3_to_f32(e4), st);   // exact: 4 x 24 significant bits
 #pragma unroll
-    for (int i = 0; i < 16; i++) {
-        const double d = __fma_rn(-e2m1_bits_f64((i < 8 ? c0 : c1) >> (4 * (i & 7))), S, vd[i]);
-        acc = __fma_rn(d, d, acc);
+    for (int h = 0; h < 2; h++) {
+        __half q[8];
+        e2m1x8_to_half(e2m1x8_quot(v + 8 * h, r), q);
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const double d = __fma_rn(-half_to_f64(q[i]), S, vd[8 * h + i]);
+            acc = __fma_rn(d, d, acc);
+        }
     }
 }
 
@@ -759,15 +770,29 @@ __device__ __forceinline__ void sel_err_int(const float (&v)[16], const double (
     }
     const Recip r = recip_of(s);
     const double sd = (double)s;
+    // the codes as floats: RN(t + 1.5 * 2^23) - 1.5 * 2^23 is RNE(t) for |t| < 2^22 (the quantizer's
+    // rounding), taken from both ends of the quotient bracket; any group of four whose ends disagree
+    // is coded with exact divisions
+    float q[16];
+    bool same = r.fast;
 #pragma unroll
-    for (int h = 0; h < 4; h++) {
-        const uint32_t b = int_x4_quot(v + 4 * h, r, qmax);
+    for (int i = 0; i < 16; i++) {
+        const float lo = __fmaf_rn(v[i], r.lo, kRoundMagic), hi = __fmaf_rn(v[i], r.hi, kRoundMagic);
+        same = same && lo == hi;
+        q[i] = __fsub_rn(lo, kRoundMagic);
+    }
+    if (!same) {
 #pragma unroll
-        for (int i = 0; i < 4; i++) {
-            const double q = (double)(int)(int8_t)(uint8_t)(b >> (8 * i));
-            const double d = __fma_rn(-q, sd, vd[4 * h + i]);
-            acc = __fma_rn(d, d, acc);
+        for (int i = 0; i < 16; i++) {
+            int c = __float2int_rn(__fdiv_rn(v[i], s));
+            c = c > qmax ? qmax : (c < -qmax ? -qmax : c);
+            q[i] = (float)c;
         }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; i++) {
+        const double d = __fma_rn(-(double)q[i], sd, vd[i]);
+        acc = __fma_rn(d, d, acc);
     }
 }
 
@@ -787,7 +812,7 @@ __device__ __forceinline__ void sel_err_fp8t(const float (&v)[16], const double 
 }
 
 template <typename T, uint32_t MASK>
-__global__ void __launch_bounds__(kSelThreads) k_select_set(const T *__restrict__ w, SelectSetArgs a) {
+__global__ void __launch_bounds__(kSelThreads, 3) k_select_set(const T *__restrict__ w, SelectSetArgs a) {
     constexpr int NS = sel_count(MASK);
     constexpr bool kTensor = (MASK & ((1u << kNVFP4) | (1u << kFP8Tensor))) != 0;
     constexpr bool kRow = (MASK & (1u << kINT8Row)) != 0;

@@ -267,6 +267,9 @@ def test_mixed_plan_and_sizes(mxq):
     assert L.mxq_qlinear_mixed_workspace_bytes(100, ctypes.byref(mw), 1, ctypes.byref(size)) == 0
     up = lambda b: (b + 255) // 256 * 256
     assert size.value == up(100 * 8 * 4) + up(100 * 256 * 2) + up(100 * 3 * 2) + up(100 * 2 * 2) + up(100 * 4 * 2)
+    single = mxq._MixedC(9, 256, (ctypes.c_int64 * 3)(0, 0, 9), 256, 256, 256, 256, 256, 256, 256, 256)
+    assert L.mxq_qlinear_mixed_workspace_bytes(100, ctypes.byref(single), 1, ctypes.byref(size)) == 0
+    assert size.value == up(100 * 256 * 2)          # the bf16 activation only: the GEMM writes y itself
     wrong = mxq._MixedC(9, 256, (ctypes.c_int64 * 3)(3, 2, 3), 256, 256, 256, 256, 256, 256, 256, 256)
     assert L.mxq_qlinear_mixed_workspace_bytes(100, ctypes.byref(wrong), 1, ctypes.byref(size)) == 1   # counts != N
     xq = mxq._QTensorC(mxq.NVFP4, mxq.MMA, 100, 256, 256, 256, 256)

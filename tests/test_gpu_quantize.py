@@ -190,6 +190,21 @@ def test_select_constructed_rows(mxq, orc):
         np.testing.assert_array_equal(sse.cpu().numpy() == 0, ref_sse == 0)
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_select_fixed_sets_small(mxq, orc, dtype):
+    """The two candidate sets with a specialised kernel ({MXFP4, NVFP4,
+    INT4-g32} and {MXFP8, INT8 row, FP8 tensor}), in two orders each, on the
+    nasty inputs: errors to 1e-12 relative, choices up to near-ties."""
+    x = host_values(_moderate(nasty_matrix(401, 70, 320)), dtype)
+    for cands in ([mxq.INT4_G32, mxq.NVFP4, mxq.MXFP4], [mxq.MXFP4, mxq.INT4_G32, mxq.NVFP4],
+                  [mxq.INT8_ROW, mxq.FP8_TENSOR, mxq.MXFP8], [mxq.MXFP8, mxq.INT8_ROW, mxq.FP8_TENSOR]):
+        ch, sse = mxq.select_weight_format(dev(x, dtype), cands)
+        ref_ch, ref_sse = orc.select_weight_format(x, cands)
+        np.testing.assert_allclose(sse.cpu().numpy(), ref_sse, rtol=1e-12, atol=0)
+        np.testing.assert_array_equal(sse.cpu().numpy() == 0, ref_sse == 0)
+        _near_tie_ok(ch.cpu().numpy(), ref_ch, ref_sse, cands)
+
+
 def test_select_full_size(mxq, orc):
     """Workload 2: W 3072 x 3072 bf16 Student-t, candidates {INT4-g32, NVFP4, MXFP4}."""
     w = workloads.chameleon_selection()["w"]
