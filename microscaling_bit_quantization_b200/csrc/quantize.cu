@@ -384,6 +384,48 @@ __global__ void __launch_bounds__(kThreads) k_quantize_int8_row(const T *__restr
     }
 }
 
+// INT8 per row with the whole row in registers (rows of at most 32 * NC
+// chunks): one warp per row issues all of its loads at once, reduces the
+// row maximum and codes from the registers, so the row is read once.
+template <typename T, int NC>
+__global__ void __launch_bounds__(kThreads) k_quantize_int8_row_reg(const T *__restrict__ x, QuantArgs a) {
+    const int lane = lane_id();
+    const int64_t warp = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * kThreads) >> 5;
+    const int cpr = (int)(a.cols >> 4);
+    for (int64_t row = warp; row < a.rows; row += nwarps) {
+        const T *xr = x + row * a.cols;
+        RawChunk<T> raw[NC];
+#pragma unroll
+        for (int j = 0; j < NC; j++)
+            if (lane + 32 * j < cpr) raw_load(raw[j], xr + (int64_t)(lane + 32 * j) * 16);
+        float m = 0.0f;
+#pragma unroll
+        for (int j = 0; j < NC; j++) {
+            if (lane + 32 * j < cpr) {
+                float v[16];
+                raw_unpack(raw[j], v);
+                m = fmaxf(m, amax16(v));
+            }
+        }
+        m = group_max<32>(m);
+        const float s = __fdiv_rn(m, 127.0f);
+        const Recip rs = recip_of(s);
+#pragma unroll
+        for (int j = 0; j < NC; j++) {
+            const int c = lane + 32 * j;
+            if (c < cpr) {
+                float v[16];
+                raw_unpack(raw[j], v);
+                *reinterpret_cast<uint4 *>(a.codes + (row * cpr + c) * 16) =
+                    make_uint4(int_x4_quot(v, rs, 127), int_x4_quot(v + 4, rs, 127), int_x4_quot(v + 8, rs, 127),
+                               int_x4_quot(v + 12, rs, 127));
+            }
+        }
+        if (lane == 0) reinterpret_cast<float *>(a.scales)[row] = s;
+    }
+}
+
 // ------------------------------------------------------------------ dequantize
 
 struct DequantArgs {
@@ -982,7 +1024,14 @@ static void launch_q(int fmt, int grid, const T *x, const QuantArgs &a, cudaStre
     case kFP8Tensor: launch_qf<T, kFP8Tensor>(x, a, s); break;
     case kINT8Row: {
         int g = grid_for(a.rows, sm_count_cached());
-        k_quantize_int8_row<T><<<g, kThreads, 0, s>>>(x, a);
+        const int64_t cpr = a.cols >> 4;
+        if (a.hadamard_b == 0 && cpr <= 32) k_quantize_int8_row_reg<T, 1><<<g, kThreads, 0, s>>>(x, a);
+        else if (a.hadamard_b == 0 && cpr <= 64) k_quantize_int8_row_reg<T, 2><<<g, kThreads, 0, s>>>(x, a);
+        else if (a.hadamard_b == 0 && cpr <= 128) k_quantize_int8_row_reg<T, 4><<<g, kThreads, 0, s>>>(x, a);
+        else if (a.hadamard_b == 0 && cpr <= 256) k_quantize_int8_row_reg<T, 8><<<g, kThreads, 0, s>>>(x, a);
+        else if (a.hadamard_b == 0 && cpr <= 384 && sizeof(T) == 2)   // bf16 rows up to 6144 elements
+            k_quantize_int8_row_reg<T, sizeof(T) == 2 ? 12 : 1><<<g, kThreads, 0, s>>>(x, a);
+        else k_quantize_int8_row<T><<<g, kThreads, 0, s>>>(x, a);
         break;
     }
     }

@@ -77,26 +77,32 @@ def test_quantize_full_size_workloads(mxq, orc):
     del w3
     w4 = workloads.mxfp4_hadamard_gemm()
     for hb in (0, 128):
-        q = mxq.quantize(dev(w4["x"], "bf16"), mxq.MXFP4, hb, mxq.MMA)
-        assert_qtensor_equal(q, orc.quantize(w4["x"], mxq.MXFP4, hb), layout_mma=True)
+        for name in ("x", "w"):   # activations and the weight, with and without the rotation
+            q = mxq.quantize(dev(w4[name], "bf16"), mxq.MXFP4, hb, mxq.MMA)
+            assert_qtensor_equal(q, orc.quantize(w4[name], mxq.MXFP4, hb), layout_mma=True)
     w1 = workloads.tiny_nvfp4_linear()
     q = mxq.quantize(dev(w1["x"], "f32"), mxq.NVFP4)
     assert_qtensor_equal(q, orc.quantize(w1["x"], mxq.NVFP4))
 
 
 def test_quantize_dit_activations(mxq, orc):
-    """Workload 5 activations: every step's tail index, the three formats, a
-    forced layer's 163x column spread."""
+    """Workload 5 activations at full size (M = 8192, both widths): the tail
+    index of the first, middle and last steps, the three routed formats, and a
+    forced layer's input with its 163x column spread; every element."""
     seed = 5
+    table, forced = workloads.dit_format_table(seed)
     for step in (0, 9, 19):
-        x = workloads.dit_activation(seed, step, workloads.DIT_HIDDEN, m=1024)
-        for fmt in (mxq.INT8_ROW, mxq.FP8_TENSOR, mxq.MXFP8):
-            q = mxq.quantize(dev(x, "bf16"), fmt, 0, mxq.MMA)
-            assert_qtensor_equal(q, orc.quantize(x, fmt), layout_mma=True)
-    f = workloads.dit_forced_column_factors(seed, 3, workloads.DIT_MLP)
-    x = workloads.to_bf16_values(workloads.dit_activation(seed, 4, workloads.DIT_MLP, m=512) * f[None, :])
-    q = mxq.quantize(dev(x, "bf16"), mxq.MXFP8, 0, mxq.MMA)
-    assert_qtensor_equal(q, orc.quantize(x, mxq.MXFP8), layout_mma=True)
+        for width in (workloads.DIT_HIDDEN, workloads.DIT_MLP):
+            x = workloads.dit_activation(seed, step, width)
+            xd = dev(x, "bf16")
+            for fmt in (mxq.INT8_ROW, mxq.FP8_TENSOR, mxq.MXFP8):
+                q = mxq.quantize(xd, fmt, 0, mxq.MMA)
+                assert_qtensor_equal(q, orc.quantize(x, fmt), layout_mma=True)
+            del xd, q
+    for layer in forced[:2]:
+        x = workloads.dit_layer_input(seed, 4, int(layer), forced)
+        q = mxq.quantize(dev(x, "bf16"), mxq.MXFP8, 0, mxq.MMA)
+        assert_qtensor_equal(q, orc.quantize(x, mxq.MXFP8), layout_mma=True)
 
 
 @pytest.mark.parametrize("fmt", ALL_FMTS)
