@@ -404,20 +404,32 @@ mxq_status mxq_quantize_lowrank_noalloc(const void *x, int32_t xdtype, int64_t m
                                         const float *w_tensor_scale, void *codes, void *scales,
                                         float *tensor_scale, void *tp, void *stream);
 
+/* Scratch bytes mxq_qlinear_w4a16 can use for an m x k activation and an
+ * n x k weight: n * k * 2 (the unpacked bf16 weight) when m >= 512, where
+ * unpacking the weight once per call costs less than converting it in
+ * every 128-row tile of x; else 0. */
+mxq_status mxq_qlinear_w4a16_workspace_bytes(int64_t m, int64_t n, int64_t k, size_t *bytes);
+
 /* W4A16 linear (Nunchaku/Diffusers article, awq_w4a16: 4-bit per-group
  * weights against 16-bit activations): y = bf16(x) . W16^T with
  * W16 = bf16(RN32(q s)), q the signed INT4 code and s its group's fp32
- * scale, fp32 accumulation on tcgen05 tensor cores; the weights are
- * dequantized in shared memory, stage by stage, never written out.
+ * scale, fp32 accumulation on tcgen05 tensor cores.  Two routes, the same
+ * products:
+ *   - workspace of at least mxq_qlinear_w4a16_workspace_bytes (> 0): W16 is
+ *     written once into the workspace (mxq_dequantize's kernel) and a bf16
+ *     kind::f16 GEMM (the block-scaled GEMM's bf16 variant) multiplies it;
+ *   - otherwise (workspace NULL or the query 0): the weights are dequantized
+ *     in shared memory, stage by stage, by the converter warps of one fused
+ *     kernel, never written out (the memory-light route for small m).
  *   x: m x k bf16 device (16-byte aligned); wq: INT4_G32 or INT4_G64 in the
  *   canonical layout (mxq_quantize), wq->cols == k; y: m x wq->rows device,
- *   ydtype MXQ_BF16 or MXQ_F32.
+ *   ydtype MXQ_BF16 or MXQ_F32; workspace: device, 16-byte aligned, or NULL.
  * Constraints: k % 64 == 0; ceil(m/128) * ceil(n/128) * k/64 < 2^31.
  * Errors: MXQ_EINVAL (shape / layout / pointer / ydtype), MXQ_EUNSUPPORTED
  * (formats other than INT4_G32 / INT4_G64), MXQ_ECUDA; a pipeline wait that
  * runs out is reported by mxq_check(). */
 mxq_status mxq_qlinear_w4a16(const void *x, int64_t m, int64_t k, const mxq_qtensor *wq, void *y,
-                             int32_t ydtype, void *stream);
+                             int32_t ydtype, void *workspace, size_t workspace_bytes, void *stream);
 
 /* Re-lays the up-projection l2 (r x n bf16, device) as the GEMM operand
  * l2p (n x 64 bf16, device): row j of l2p holds l2[0..r-1][j], zeros up to

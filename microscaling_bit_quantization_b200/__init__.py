@@ -36,7 +36,8 @@ EXPORTS = ("mxq_status_string", "mxq_last_cuda_error_string", "mxq_device_suppor
            "mxq_quantize_mse", "mxq_quantize_mx_grid", "mxq_fit_mx_grid_workspace_bytes", "mxq_fit_mx_grid",
            "mxq_calibrate_workspace_bytes", "mxq_calibrate_activation", "mxq_calibrate_pick",
            "mxq_lowrank_down", "mxq_lowrank_packed_bytes",
-           "mxq_lowrank_down_packed", "mxq_lowrank_pack_t", "mxq_lowrank_pack_l2", "mxq_qlinear", "mxq_qlinear_w4a16", "mxq_route",
+           "mxq_lowrank_down_packed", "mxq_lowrank_pack_t", "mxq_lowrank_pack_l2", "mxq_qlinear", "mxq_qlinear_w4a16",
+           "mxq_qlinear_w4a16_workspace_bytes", "mxq_route",
            "mxq_quantize_lowrank_workspace_bytes", "mxq_quantize_lowrank", "mxq_quantize_lowrank_noalloc",
            "mxq_qlinear_routed_workspace_bytes", "mxq_qlinear_routed", "mxq_mixed_plan", "mxq_mixed_weight_bytes",
            "mxq_mixed_prepare", "mxq_qlinear_mixed_workspace_bytes", "mxq_qlinear_mixed")
@@ -104,7 +105,8 @@ def _load():
         "mxq_lowrank_pack_t": (i32, [P, i32, i64, P, P, P, P]),
         "mxq_lowrank_pack_l2": (i32, [P, i32, i64, P, P]),
         "mxq_qlinear": (i32, [ctypes.POINTER(_QTensorC), ctypes.POINTER(_QTensorC), P, P, P, i32, P]),
-        "mxq_qlinear_w4a16": (i32, [P, i64, i64, ctypes.POINTER(_QTensorC), P, i32, P]),
+        "mxq_qlinear_w4a16": (i32, [P, i64, i64, ctypes.POINTER(_QTensorC), P, i32, P, sz, P]),
+        "mxq_qlinear_w4a16_workspace_bytes": (i32, [i64, i64, i64, psz]),
         "mxq_route": (i32, [P, i32, i32, i32, i32, i32]),
         "mxq_quantize_lowrank_workspace_bytes": (i32, [i64, i32, psz]),
         "mxq_quantize_lowrank": (i32, [P, i32, i64, i64, i32, i32, P, i32, P, P, P, P, P, P, sz, P]),
@@ -457,16 +459,30 @@ def qlinear(xq: QTensor, wq: QTensor, tp: torch.Tensor = None, l2p: torch.Tensor
     return y
 
 
+def qlinear_w4a16_workspace_bytes(m: int, n: int, k: int) -> int:
+    return _size(_lib.mxq_qlinear_w4a16_workspace_bytes, m, n, k)
+
+
 def qlinear_w4a16(x: torch.Tensor, wq: QTensor, out_dtype=torch.bfloat16, out: torch.Tensor = None,
-                  stream=None) -> torch.Tensor:
-    """y = bf16(x) . bf16(q s)^T for an INT4-g32/g64 weight in the canonical layout."""
+                  workspace: torch.Tensor = None, fused: bool = False, stream=None) -> torch.Tensor:
+    """y = bf16(x) . bf16(q s)^T for an INT4-g32/g64 weight in the canonical
+    layout.  With a workspace (allocated here when the library asks for one
+    and `fused` is false) the weight is unpacked once and multiplied by the
+    bf16 GEMM; otherwise the fused kernel converts it in shared memory."""
     _require_cuda(x)
     assert x.dtype == torch.bfloat16
     x = x.contiguous()
     m, k = x.shape
     y = out if out is not None else torch.empty((m, wq.rows), dtype=out_dtype, device=x.device)
+    if fused:
+        workspace = None
+    elif workspace is None:
+        wsb = qlinear_w4a16_workspace_bytes(m, wq.rows, k)
+        if wsb:
+            workspace = torch.empty(wsb, dtype=torch.uint8, device=x.device)
     wc = wq.c()
-    _ok(_lib.mxq_qlinear_w4a16(_ptr(x), m, k, ctypes.byref(wc), _ptr(y), _dtype_code(y), _stream(stream)),
+    _ok(_lib.mxq_qlinear_w4a16(_ptr(x), m, k, ctypes.byref(wc), _ptr(y), _dtype_code(y), _ptr(workspace),
+                               workspace.numel() if workspace is not None else 0, _stream(stream)),
         "mxq_qlinear_w4a16")
     return y
 

@@ -388,8 +388,15 @@ mxq_status mxq_quantize_lowrank(const void *x, int32_t xdtype, int64_t m, int64_
                                      amax, s, &pack, amax_ready, 1.0f, slots, n_slots));
 }
 
+mxq_status mxq_qlinear_w4a16_workspace_bytes(int64_t m, int64_t n, int64_t k, size_t *bytes) {
+    if (!bytes || m < 0 || n < 0 || k <= 0 || k % 64 || n >= ((int64_t)1 << 31) || k >= ((int64_t)1 << 31))
+        return MXQ_EINVAL;
+    *bytes = m >= 512 ? (size_t)(n * k * 2) : 0;   // below that, the fused kernel is the faster route
+    return MXQ_OK;
+}
+
 mxq_status mxq_qlinear_w4a16(const void *x, int64_t m, int64_t k, const mxq_qtensor *wq, void *y, int32_t ydtype,
-                             void *stream) {
+                             void *workspace, size_t workspace_bytes, void *stream) {
     if (!wq || !valid_dtype(ydtype) || m < 0 || k <= 0 || k % 64) return MXQ_EINVAL;
     if (wq->fmt != MXQ_INT4_G32 && wq->fmt != MXQ_INT4_G64) return MXQ_EUNSUPPORTED;
     if (wq->layout != MXQ_LAYOUT_CANONICAL || wq->cols != k || wq->rows < 0) return MXQ_EINVAL;
@@ -401,6 +408,29 @@ mxq_status mxq_qlinear_w4a16(const void *x, int64_t m, int64_t k, const mxq_qten
     if (wa_tiles >= ((int64_t)1 << 31) || wa_tiles * (k / 64) >= ((int64_t)1 << 31)) return MXQ_EINVAL;
     if (m > 0 && wq->rows > 0 && (!x || !y || !wq->codes || !wq->scales || !aligned16(x) || !aligned16(wq->codes)))
         return MXQ_EINVAL;
+    size_t need = 0;
+    mxq_qlinear_w4a16_workspace_bytes(m, wq->rows, k, &need);
+    if (workspace && need > 0 && workspace_bytes >= need && m > 0 && wq->rows > 0) {
+        if (!aligned16(workspace)) return MXQ_EINVAL;
+        // the bf16 GEMM counts 256-row x 256-column tiles and their 64-element stages in 32-bit integers
+        if (((m + 255) / 256) * ((wq->rows + 255) / 256) * (k / 64) >= ((int64_t)1 << 31)) return MXQ_EINVAL;
+        cudaStream_t s = (cudaStream_t)stream;
+        // W16 = bf16(RN32(q s)), the dequantizer's rounding, written once
+        cudaError_t e = launch_dequantize(wq->fmt, MXQ_LAYOUT_CANONICAL, wq->rows, k, wq->codes, wq->scales, nullptr,
+                                          workspace, true, s);
+        if (e != cudaSuccess) return from_cuda(e);
+        GemmOperands op;
+        memset(&op, 0, sizeof(op));
+        op.fmt = wq->fmt;
+        op.m = m;
+        op.n = wq->rows;
+        op.k = k;
+        op.a_codes = x;
+        op.b_codes = workspace;
+        op.y = y;
+        op.y_bf16 = ydtype == MXQ_BF16;
+        return from_cuda(launch_gemm_bf16(op, s));
+    }
     return from_cuda(launch_w4a16(x, m, k, (const uint8_t *)wq->codes, (const float *)wq->scales, wq->rows,
                                   wq->fmt == MXQ_INT4_G32 ? 32 : 64, y, ydtype == MXQ_BF16, (cudaStream_t)stream));
 }

@@ -145,18 +145,23 @@ def test_w4a16_argument_checks(mxq):
     def qt(fmt, layout, rows, cols):
         return mxq._QTensorC(fmt, layout, rows, cols, 256, 256, None)
 
-    call = lambda q, k=128, yd=1: L.mxq_qlinear_w4a16(d, 4, k, ctypes.byref(q), d, yd, None)
+    call = lambda q, k=128, yd=1: L.mxq_qlinear_w4a16(d, 4, k, ctypes.byref(q), d, yd, None, 0, None)
     assert call(qt(mxq.NVFP4, 0, 8, 128)) == 2            # INT4 groups only
     assert call(qt(mxq.INT4_G64, 1, 8, 128)) == 1         # canonical layout only
     assert call(qt(mxq.INT4_G64, 0, 8, 96), k=96) == 1    # k % 64
     assert call(qt(mxq.INT4_G64, 0, 8, 192), k=128) == 1  # cols != k
     assert call(qt(mxq.INT4_G32, 0, 8, 128), yd=7) == 1   # bad output dtype
     big = qt(mxq.INT4_G64, 0, (1 << 31) - 1, 1 << 20)
-    assert L.mxq_qlinear_w4a16(d, (1 << 31) - 1, 1 << 20, ctypes.byref(big), d, 1, None) == 1   # stage count
+    assert L.mxq_qlinear_w4a16(d, (1 << 31) - 1, 1 << 20, ctypes.byref(big), d, 1, None, 0, None) == 1   # stage count
     # every factor at its largest: the product of tiles and stages (about 2^73) must not wrap around
     kmax = (1 << 31) - 64
     huge = qt(mxq.INT4_G64, 0, (1 << 31) - 1, kmax)
-    assert L.mxq_qlinear_w4a16(d, (1 << 31) - 1, kmax, ctypes.byref(huge), d, 1, None) == 1
+    assert L.mxq_qlinear_w4a16(d, (1 << 31) - 1, kmax, ctypes.byref(huge), d, 1, None, 0, None) == 1
+    size = ctypes.c_size_t(0)
+    assert L.mxq_qlinear_w4a16_workspace_bytes(4096, 12288, 3072, ctypes.byref(size)) == 0
+    assert size.value == 12288 * 3072 * 2   # large m: the unpacked bf16 weight
+    assert L.mxq_qlinear_w4a16_workspace_bytes(64, 12288, 3072, ctypes.byref(size)) == 0 and size.value == 0
+    assert L.mxq_qlinear_w4a16_workspace_bytes(64, 128, 96, ctypes.byref(size)) == 1   # k % 64
 
 
 def test_qlinear_argument_checks(mxq):

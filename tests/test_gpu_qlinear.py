@@ -295,6 +295,23 @@ def test_w4a16_small(mxq, orc, fmt, shape):
         gemm_close(y.float().cpu().numpy(), ref, bf16_out=out_dtype == torch.bfloat16)
 
 
+@pytest.mark.parametrize("fmt", [4, 3])
+def test_w4a16_both_routes(mxq, orc, fmt):
+    """m = 600 (above the size where the library asks for a workspace): the
+    unpacked-weight route and the fused kernel, every element against the
+    oracle, fp32 and bf16 out."""
+    m, n, k = 600, 392, 320
+    d = _inputs(95 + fmt, m, n, k)
+    assert mxq.qlinear_w4a16_workspace_bytes(m, n, k) == n * k * 2
+    wq = mxq.quantize(dev(d["w"], "bf16"), fmt)
+    ref = orc.w4a16(host_values(d["x"], "bf16"), orc.quantize(host_values(d["w"], "bf16"), fmt))
+    for fused in (False, True):
+        for out_dtype in (torch.float32, torch.bfloat16):
+            y = mxq.qlinear_w4a16(dev(d["x"], "bf16"), wq, out_dtype=out_dtype, fused=fused)
+            assert mxq.check() == 0
+            gemm_close(y.float().cpu().numpy(), ref, bf16_out=out_dtype == torch.bfloat16)
+
+
 def test_w4a16_full_size(mxq, orc):
     """Workload 3's shape with its residual weight as INT4-g64: 256 sampled
     rows (all 12288 columns) against the oracle."""
