@@ -788,6 +788,8 @@ def finish(args, world, rank, ms, value, clocks, gemm_tflops, fp4_peak, peaks, p
         sec_all = o.timed(6, threads=n_cores)
         cpu = {"value": o.flops / sec / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
                "sample": o.desc + "; 6 steps on 1 thread",
+               "extrapolated_full_step_s": sec * M / o.rows,
+               "extrapolation": "the sample's time per step x %d / %d token rows (linear in M)" % (M, o.rows),
                "all_cores": {"value": o.flops / sec_all / 1e12, "unit": "TFLOP/s", "cores": n_cores,
                              "sample": "the same sample with numpy's BLAS on all host cores (the C steps stay on "
                                        "one thread)"}}

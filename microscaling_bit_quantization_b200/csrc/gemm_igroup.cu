@@ -14,7 +14,10 @@
 // formed on its own: the codes are stored as E4M3 bytes (every integer in
 // [-7, 7] is an E4M3 value), a kind::f8f6f4 MMA gives P_g exactly in fp32
 // (|P_g| <= 64 * 49), and the epilogue folds it into fp32 running sums held
-// in registers, acc += P_g * (sx * sw).  Those two ALU operations per output
+// in registers, acc += P_g * (sx * sw).  The mixed-format linear layer runs
+// the same kernel with MXFP8 activations (E4M3 codes, sx = 2^e of the
+// 32-element block) against INT4-g32 weights; P_g then sums 32 products of
+// E4M3 values and integers, each exact, in fp32.  Those two ALU operations per output
 // element and group bound the kernel; the MMAs of a group take less than half
 // as long and run up to three groups ahead in a ring of four TMEM buffers.
 //
