@@ -224,6 +224,30 @@ __device__ __forceinline__ void scale_chunk(const uint32_t (&r)[32], float (&v)[
     }
 }
 
+// One k-step (32 bytes of K) of the main product: an NVFP4 scale atom serves
+// one k-step, an MXFP4 atom two, an MXFP8 atom four (the MX kinds select the
+// atom's scale column through the instruction descriptor).
+template <int KIND>
+__device__ __forceinline__ void mma_kstep(uint32_t acc_addr, uint64_t ad, uint64_t bd, uint32_t accum, uint32_t group,
+                                          int ks) {
+    constexpr int NSF = sf_atoms<KIND>();
+    const int a = NSF == 4 ? ks : NSF == 2 ? (ks >> 1) : 0;
+    const uint32_t base = group + SF_SLOT_COLS * (uint32_t)a;
+    if (KIND == kKindNVFP4) {
+        mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>(), accum, base, base + 4);
+    } else if (KIND == kKindMXFP4) {
+        const uint32_t id = (uint32_t)((ks & 1) * 2);
+        mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>() | (id << 29) | (id << 4), accum, base, base + 4);
+    } else if (KIND == kKindMXFP8) {
+        const uint32_t id = (uint32_t)ks;
+        mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>() | (id << 29) | (id << 4), accum, base, base + 4);
+    } else if (KIND == kKindBF16) {
+        mma_bf16(acc_addr, ad, bd, idesc_bf16(), accum);
+    } else {
+        mma_plain<KIND>(acc_addr, ad, bd, idesc_main<KIND>(), accum);
+    }
+}
+
 template <int KIND>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     k_gemm(const __grid_constant__ GemmParams p) {
@@ -330,9 +354,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer (first CTA)
+        // This one thread's latency per k-tile (barrier wait, set-up, four MMA
+        // issues, commit) is what keeps the tensor pipe fed, so the loop is
+        // lean: stage and phase are counters, a stage's descriptors are the
+        // stage-0 descriptors plus constants, and a whole k-tile's four
+        // k-steps are unrolled.
         if (lane == 0 && rank == 0) {
             bool issued_any = false;
-            int it = 0, tcount = 0;
+            int it = 0, tcount = 0, s = 0;
+            uint32_t ph = 0;
+            const uint64_t ad0 = sdesc_sw128(smem), bd0 = sdesc_sw128(smem + A_STAGE);
+            const int nk_full = p.kbytes / BKB;   // k-tiles with all four k-steps
             for (int tile = cid; tile < num_tiles && !*abort_flag; tile += ncl, tcount++) {
                 const int st = tcount & 1;
                 const uint32_t acc_addr = tmem + (st ? ACC_STAGE1 : 0u);
@@ -346,8 +378,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 }
                 tc_fence_after();
                 for (int kt = 0; kt < nsteps; kt++, it++) {
-                    const int s = it % STAGES;
-                    const uint32_t ph = (it / STAGES) & 1;
                     // block-scaled kinds: the scale-factor warp has copied this stage's atoms to TMEM
                     // (and seen the stage full); other kinds wait for the stage itself
                     if (!mbar_wait(NSF ? sfready + s : full + s, ph, p.wait_ns)) {
@@ -355,43 +385,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                         *abort_flag = 1;
                         break;
                     }
-                    if (*abort_flag) break;
                     tc_fence_after();
-                    uint8_t *sa = smem + s * STAGE_BYTES;
-                    uint8_t *sb = sa + A_STAGE;
-                    if (kt < p.num_k_tiles) {
-                        const int rem = (p.kbytes - kt * BKB) >> 5;
-                        const int nks = rem < 4 ? rem : 4;
-                        const uint32_t group = tmem + TMEM_SF + SF_GROUP_COLS * ((uint32_t)it % SF_GROUPS);
-                        for (int ks = 0; ks < nks; ks++) {
-                            const uint64_t ad = sdesc_sw128(sa + ks * 32), bd = sdesc_sw128(sb + ks * 32);
-                            const uint32_t accum = (kt > 0 || ks > 0) ? 1u : 0u;
-                            // an NVFP4 atom serves one k-step, an MXFP4 atom two, an MXFP8 atom four
-                            const int a = NSF == 4 ? ks : NSF == 2 ? (ks >> 1) : 0;
-                            const uint32_t base = group + SF_SLOT_COLS * (uint32_t)a;
-                            if (KIND == kKindNVFP4) {
-                                mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>(), accum, base, base + 4);
-                            } else if (KIND == kKindMXFP4) {
-                                const uint32_t id = (uint32_t)((ks & 1) * 2);
-                                mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>() | (id << 29) | (id << 4),
-                                                       accum, base, base + 4);
-                            } else if (KIND == kKindMXFP8) {
-                                const uint32_t id = (uint32_t)ks;
-                                mma_block_scaled<KIND>(acc_addr, ad, bd, idesc_main<KIND>() | (id << 29) | (id << 4),
-                                                       accum, base, base + 4);
-                            } else if (KIND == kKindBF16) {
-                                mma_bf16(acc_addr, ad, bd, idesc_bf16(), accum);
-                            } else {
-                                mma_plain<KIND>(acc_addr, ad, bd, idesc_main<KIND>(), accum);
-                            }
-                        }
-                    } else {
+                    const uint64_t soff = (uint64_t)(s * (STAGE_BYTES >> 4));
+                    const uint64_t ad = ad0 + soff, bd = bd0 + soff;   // +2 per 32-byte k-step
+                    const uint32_t group = tmem + TMEM_SF + SF_GROUP_COLS * ((uint32_t)it % SF_GROUPS);
+                    if (kt < nk_full) {
 #pragma unroll
                         for (int ks = 0; ks < 4; ks++)
-                            mma_bf16(acc_addr, sdesc_sw128(sa + ks * 32), sdesc_sw128(sb + ks * 32), idesc_bf16(), 1u);
+                            mma_kstep<KIND>(acc_addr, ad + 2 * ks, bd + 2 * ks, (kt | ks) != 0 ? 1u : 0u, group, ks);
+                    } else if (kt < p.num_k_tiles) {
+                        const int nks = (p.kbytes - kt * BKB) >> 5;   // 1..3 k-steps in the last k-tile
+                        for (int ks = 0; ks < nks; ks++)
+                            mma_kstep<KIND>(acc_addr, ad + 2 * ks, bd + 2 * ks, (kt | ks) != 0 ? 1u : 0u, group, ks);
+                    } else {
+#pragma unroll
+                        for (int ks = 0; ks < 4; ks++) mma_bf16(acc_addr, ad + 2 * ks, bd + 2 * ks, idesc_bf16(), 1u);
                     }
                     issued_any = true;
                     tc_commit_pair(empty + s);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
                 if (*abort_flag) break;
                 tc_commit_pair(accf + st);

@@ -85,14 +85,16 @@ def test_qlinear_short_k(mxq, orc, fmt):
 
 
 @pytest.mark.parametrize("fmt", GEMM_FMTS)
-def test_qlinear_partial_last_round(mxq, orc, fmt):
-    """81 output tiles of 256 x 256 on 74 clusters (a partly filled last round
-    of the persistent walk), ragged M and N (the last tiles are 152 rows and
-    152 columns), with the low-rank branch where the format takes it; every
-    output element checked."""
-    m, n, k = 2200, 2200, 512
+@pytest.mark.parametrize("shape", [(2200, 2200, 512), (2560, 1000, 512)])
+def test_qlinear_partial_last_round(mxq, orc, fmt, shape):
+    """Rounds of the persistent walk over 74 clusters, with ragged edges and
+    the low-rank branch where the format takes it; every output element
+    checked.  2200 x 2200: 81 tiles of 256 x 256, a partly filled second
+    round (the last tiles are 152 rows and 152 columns).  2560 x 1000: 40
+    tiles in one round, the last column tile 232 wide."""
+    m, n, k = shape
     r = 32 if fmt in LOWRANK_FMTS else 0
-    d = _inputs(60 + fmt, m, n, k, r)
+    d = _inputs(60 + fmt + (m % 7), m, n, k, r)
     ref, _, _ = _ref(orc, fmt, d, r)
     for out_dtype in (torch.float32, torch.bfloat16):
         y, _, _ = _run(mxq, fmt, d, r, out_dtype)
