@@ -369,8 +369,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 const int st = tcount & 1;
                 const uint32_t acc_addr = tmem + (st ? ACC_STAGE1 : 0u);
                 // this stage drained (tile tcount-2) and the shared columns (tile tcount-1), in both CTAs
-                bool ok = mbar_wait<true>(acce + st, ((tcount >> 1) & 1) ^ 1, p.wait_ns);
-                if (ok && tcount > 0) ok = mbar_wait<true>(ovlf, (tcount - 1) & 1, p.wait_ns);
+                bool ok = mbar_wait_spin<true>(acce + st, ((tcount >> 1) & 1) ^ 1, p.wait_ns);
+                if (ok && tcount > 0) ok = mbar_wait_spin<true>(ovlf, (tcount - 1) & 1, p.wait_ns);
                 if (!ok) {
                     latch_error(kErrTimeoutMma);
                     *abort_flag = 1;
@@ -380,7 +380,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 for (int kt = 0; kt < nsteps; kt++, it++) {
                     // block-scaled kinds: the scale-factor warp has copied this stage's atoms to TMEM
                     // (and seen the stage full); other kinds wait for the stage itself
-                    if (!mbar_wait(NSF ? sfready + s : full + s, ph, p.wait_ns)) {
+                    if (!mbar_wait_spin(NSF ? sfready + s : full + s, ph, p.wait_ns)) {
                         latch_error(kErrTimeoutMma);
                         *abort_flag = 1;
                         break;
@@ -470,6 +470,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const uint32_t acce_leader0 = map_to_rank(acce, 0), acce_leader1 = map_to_rank(acce + 1, 0);
         uint8_t *stage_buf = epi + q * 2 * EPI_BUF;
         const bool vec = p.y_bf16 ? (p.n % 8 == 0) : (p.n % 4 == 0);
+        // the tensor scales hold for the whole launch: read once, outside the tile loop
+        float alpha = 1.0f;
+        if (KIND == kKindNVFP4 || KIND == kKindFP8) alpha = __fmul_rn(__ldg(p.a_ts), __ldg(p.b_ts));
+        if (KIND == kKindBF16 && p.b_ts) alpha = __ldg(p.b_ts);
         int tcount = 0, sub = 0;
         for (int tile = cid; tile < num_tiles; tile += ncl, tcount++) {
             const int pm0 = (tile / p.n_tiles) * 256, n0 = (tile % p.n_tiles) * BN;
@@ -485,11 +489,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             }
             tc_fence_after();
             const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + (st ? ACC_STAGE1 : 0u);
-            float alpha = 1.0f, ra = 0.0f;
-            if (KIND == kKindNVFP4 || KIND == kKindFP8) alpha = __fmul_rn(__ldg(p.a_ts), __ldg(p.b_ts));
-            if (KIND == kKindBF16 && p.b_ts) alpha = __ldg(p.b_ts);
+            float ra = 0.0f;   // INT8 row scale, read once the shared columns are released
             const bool row_ok = row < p.m;
-            if (KIND == kKindINT8 && row_ok) ra = __ldg(p.a_row_scale + row);
             // The shared columns (the last OVL_CHUNKS chunks of stage 0, the first OVL_CHUNKS of
             // stage 1) go to registers first and are released at once, so the next tile's MMAs
             // wait only for these loads; then every chunk is scaled, staged and stored.
@@ -566,7 +567,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             for (int i = 0; i + 1 < (int)OVL_CHUNKS; i++) tmem_reg_tie(ro[i]);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_remote(ovl_leader);
+            if (lane == 0) mbar_arrive_remote_relaxed(ovl_leader);
+            if (KIND == kKindINT8 && row_ok) ra = __ldg(p.a_row_scale + row);
 #pragma unroll
             for (int i = 0; i < (int)OVL_CHUNKS; i++) process(st ? i : 8 - (int)OVL_CHUNKS + i, ro[i]);
 #pragma unroll 1
@@ -577,7 +579,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 if (i == BN / 32 - 1) {   // the whole stage is drained
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive_remote(st ? acce_leader1 : acce_leader0);
+                    if (lane == 0) mbar_arrive_remote_relaxed(st ? acce_leader1 : acce_leader0);
                 }
                 process(c, r);
             }

@@ -42,6 +42,13 @@ __device__ __forceinline__ uint32_t map_to_rank(const void *p, uint32_t rank) {
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
+// Arrival on a barrier of a CTA of the cluster that publishes no data: the
+// arriving thread reports only that operations it has already waited for are
+// complete (tensor-memory loads after tcgen05.wait::ld), so it needs no release
+// ordering, which at cluster scope held the arrival back by some 500 ns.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
 
 // ---- mbarriers, copies, tcgen05
 
@@ -79,6 +86,40 @@ __device__ __forceinline__ uint64_t global_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
+}
+template <bool CLUSTER>
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    if (CLUSTER)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+    return ok != 0;
+}
+// Bounded wait that polls without suspending the thread, for the thread
+// whose latency feeds the tensor pipe (it resumes sooner than a thread
+// suspended in try_wait).
+template <bool CLUSTER = false>
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t *bar, uint32_t parity, unsigned long long limit_ns) {
+    if (mbar_test_wait<CLUSTER>(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        for (int i = 0; i < 32; i++)
+            if (mbar_test_wait<CLUSTER>(bar, parity)) return true;
+        if (global_ns() - t0 > limit_ns) return false;
+    }
 }
 // Bounded wait for the phase of parity `parity` to complete.
 template <bool CLUSTER = false>
