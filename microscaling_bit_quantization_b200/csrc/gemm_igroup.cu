@@ -269,23 +269,27 @@ __global__ void __launch_bounds__(IG_THREADS, 1) k_gemm_igroup(const __grid_cons
                 tc_fence_after();
                 return w;
             };
-            // acc[j] += P[j] * (sx * sw[j]) for the 32 columns of one half; factor 1 for the branch
-            float acc[IG_EPI_COLS];
+            // acc[j] += P[j] * (sx * sw[j]) for the 32 columns of one half; factor 1 for the branch.
+            // Two columns per packed fp32x2 operation, each lane rounded like the scalar operation.
+            float2 acc[IG_EPI_COLS / 2];
 #pragma unroll
-            for (int j = 0; j < IG_EPI_COLS; j++) acc[j] = 0.0f;
-            auto fold = [&](const uint32_t (&r)[32], float *accp, const float *sw, float sxv, bool lr) {
+            for (int j = 0; j < IG_EPI_COLS / 2; j++) acc[j] = make_float2(0.0f, 0.0f);
+            auto fold = [&](const uint32_t (&r)[32], float2 *accp, const float *sw, float sxv, bool lr) {
                 if (lr) {
 #pragma unroll
-                    for (int j = 0; j < 32; j++) accp[j] = __fadd_rn(accp[j], __uint_as_float(r[j]));
+                    for (int j = 0; j < 16; j++)
+                        accp[j] = __fadd2_rn(accp[j], make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])));
                 } else {
+                    const float2 sx2 = make_float2(sxv, sxv);
                     const float4 *sw4 = reinterpret_cast<const float4 *>(sw);
 #pragma unroll
                     for (int jj = 0; jj < 8; jj++) {
                         const float4 w4 = sw4[jj];
-                        accp[4 * jj] = __fmaf_rn(__uint_as_float(r[4 * jj]), __fmul_rn(sxv, w4.x), accp[4 * jj]);
-                        accp[4 * jj + 1] = __fmaf_rn(__uint_as_float(r[4 * jj + 1]), __fmul_rn(sxv, w4.y), accp[4 * jj + 1]);
-                        accp[4 * jj + 2] = __fmaf_rn(__uint_as_float(r[4 * jj + 2]), __fmul_rn(sxv, w4.z), accp[4 * jj + 2]);
-                        accp[4 * jj + 3] = __fmaf_rn(__uint_as_float(r[4 * jj + 3]), __fmul_rn(sxv, w4.w), accp[4 * jj + 3]);
+                        accp[2 * jj] = __ffma2_rn(make_float2(__uint_as_float(r[4 * jj]), __uint_as_float(r[4 * jj + 1])),
+                                                  __fmul2_rn(sx2, make_float2(w4.x, w4.y)), accp[2 * jj]);
+                        accp[2 * jj + 1] =
+                            __ffma2_rn(make_float2(__uint_as_float(r[4 * jj + 2]), __uint_as_float(r[4 * jj + 3])),
+                                       __fmul2_rn(sx2, make_float2(w4.z, w4.w)), accp[2 * jj + 1]);
                     }
                 }
             };
@@ -311,12 +315,12 @@ __global__ void __launch_bounds__(IG_THREADS, 1) k_gemm_igroup(const __grid_cons
                 tmem_ld_wait(rb);
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_local(bempty + b);   // the MMAs may reuse this buffer
+                if (lane == 0) mbar_arrive_local_relaxed(bempty + b);   // the MMAs may reuse this buffer
                 if (gi + 1 < ngroups) {
                     ok = wait_group(gc + 1);
                     if (ok) tmem_ld_32x32b_x32_async(lane_base + ((gc + 1) % IG_NBUF) * IG_BN, ra);   // next first half
                 }
-                fold(rb, acc + 32, slot + 64, sxv, lr);
+                fold(rb, acc + 16, slot + 64, sxv, lr);
                 tmem_ld_wait(ra);
             }
             cp_async_wait<0>();
@@ -329,14 +333,16 @@ __global__ void __launch_bounds__(IG_THREADS, 1) k_gemm_igroup(const __grid_cons
                         const int c = col0 + 8 * jj;
                         if (p.y_vec && c + 8 <= p.n) {
                             reinterpret_cast<uint4 *>(yr)[jj] =
-                                make_uint4(pack_bf16x2(acc[8 * jj], acc[8 * jj + 1]),
-                                           pack_bf16x2(acc[8 * jj + 2], acc[8 * jj + 3]),
-                                           pack_bf16x2(acc[8 * jj + 4], acc[8 * jj + 5]),
-                                           pack_bf16x2(acc[8 * jj + 6], acc[8 * jj + 7]));
+                                make_uint4(pack_bf16x2(acc[4 * jj].x, acc[4 * jj].y),
+                                           pack_bf16x2(acc[4 * jj + 1].x, acc[4 * jj + 1].y),
+                                           pack_bf16x2(acc[4 * jj + 2].x, acc[4 * jj + 2].y),
+                                           pack_bf16x2(acc[4 * jj + 3].x, acc[4 * jj + 3].y));
                         } else {
 #pragma unroll
                             for (int t = 0; t < 8; t++)
-                                if (c + t < p.n) yr[8 * jj + t] = __float2bfloat16_rn(acc[8 * jj + t]);
+                                if (c + t < p.n)
+                                    yr[8 * jj + t] = __float2bfloat16_rn((t & 1) ? acc[4 * jj + (t >> 1)].y
+                                                                                  : acc[4 * jj + (t >> 1)].x);
                         }
                     }
                 } else {
@@ -346,11 +352,11 @@ __global__ void __launch_bounds__(IG_THREADS, 1) k_gemm_igroup(const __grid_cons
                         const int c = col0 + 4 * jj;
                         if (p.y_vec && c + 4 <= p.n) {
                             reinterpret_cast<float4 *>(yr)[jj] =
-                                make_float4(acc[4 * jj], acc[4 * jj + 1], acc[4 * jj + 2], acc[4 * jj + 3]);
+                                make_float4(acc[2 * jj].x, acc[2 * jj].y, acc[2 * jj + 1].x, acc[2 * jj + 1].y);
                         } else {
 #pragma unroll
                             for (int t = 0; t < 4; t++)
-                                if (c + t < p.n) yr[4 * jj + t] = acc[4 * jj + t];
+                                if (c + t < p.n) yr[4 * jj + t] = (t & 1) ? acc[2 * jj + (t >> 1)].y : acc[2 * jj + (t >> 1)].x;
                         }
                     }
                 }

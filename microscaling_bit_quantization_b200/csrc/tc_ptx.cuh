@@ -148,6 +148,13 @@ __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::
 __device__ __forceinline__ void mbar_arrive_local(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
+// The same arrival without release ordering, for a thread that publishes no
+// data but reports operations it has already waited for (tensor-memory loads
+// after tcgen05.wait::ld): a release arrival waits for the thread's earlier
+// global stores.
+__device__ __forceinline__ void mbar_arrive_local_relaxed(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 
 // Shared-memory matrix descriptor, K-major, 128-byte swizzle: 8-row x 128 B
 // core groups 1024 B apart (stride byte offset), descriptor version 1.
