@@ -18,20 +18,23 @@
 // the same kernel with MXFP8 activations (E4M3 codes, sx = 2^e of the
 // 32-element block) against INT4-g32 weights; P_g then sums 32 products of
 // E4M3 values and integers, each exact, in fp32.  Those two ALU operations per output
-// element and group bound the kernel; the MMAs of a group take less than half
-// as long and run up to three groups ahead in a ring of four TMEM buffers.
+// element and group (one packed fp32x2 multiply and FMA per two columns) and
+// the latency of fetching each group's sums from TMEM bound the kernel; the
+// MMAs of a group run up to three groups ahead in a ring of four TMEM buffers.
 //
 // Per CTA (one per SM, persistent over 128 x 128 output tiles):
 //   warp 0      TMA producer into a 6-stage ring (A and B tiles of
 //               128 rows x 128 B, 128-byte swizzle)
 //   warp 1      TMEM allocation (4 group buffers x 128 columns) and the
 //               thread that issues the MMAs (cta_group::1)
-//   warps 2-9   epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 (its 32
-//               rows) and one half of the 128 columns ((w - 2) / 4), keeps
-//               64 running sums per thread and stores its rows of Y.  TMEM
-//               loads run one half-group (32 columns) ahead of the arithmetic,
-//               and each warp's group scales arrive by cp.async in a ring of
-//               shared-memory slots IG_SCALE_AHEAD groups ahead of their use
+//   warps 2-17  epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 (its 32
+//               rows) and one quarter of the 128 columns ((w - 2) / 4), keeps
+//               32 running sums per thread and stores its rows of Y.  Each
+//               group's 32 columns are loaded, the buffer released at once,
+//               then folded: four epilogue warps per scheduler hide the load
+//               latency of one another.  Each warp's group scales arrive by
+//               cp.async in a ring of shared-memory slots IG_SCALE_AHEAD
+//               groups ahead of their use
 // The low-rank branch is one more group with scale 1: a bf16 kind::f16 MMA
 // of the packed activation [T_hi | T_lo] against [L2^T | L2^T].
 // Every wait is bounded; a wait that runs out latches the error word and
@@ -55,9 +58,9 @@ constexpr int IG_A = IG_BM * IG_BKB, IG_B = IG_BN * IG_BKB;   // 16 KB each
 constexpr int IG_STAGE = IG_A + IG_B;
 constexpr int IG_NBUF = 4;                                    // TMEM group buffers
 constexpr uint32_t IG_TMEM_COLS = IG_NBUF * IG_BN;            // 512
-constexpr int IG_EPI_WARPS = 8;
-constexpr int IG_EPI_COLS = IG_BN / (IG_EPI_WARPS / 4);        // 64 columns per epilogue warp
-constexpr int IG_THREADS = 64 + 32 * IG_EPI_WARPS;            // 320
+constexpr int IG_EPI_WARPS = 16;
+constexpr int IG_EPI_COLS = IG_BN / (IG_EPI_WARPS / 4);        // 32 columns per epilogue warp
+constexpr int IG_THREADS = 64 + 32 * IG_EPI_WARPS;            // 576
 constexpr int IG_SCALE_SLOTS = 8, IG_SCALE_AHEAD = 6;          // per-warp scale ring: slots, groups in flight
 constexpr int IG_SLOT_FLOATS = 32 + IG_EPI_COLS;              // sx of the warp's 32 rows, sw of its columns
 constexpr int IG_WSCALE_BYTES = IG_EPI_WARPS * IG_SCALE_SLOTS * IG_SLOT_FLOATS * 4;
@@ -247,81 +250,64 @@ __global__ void __launch_bounds__(IG_THREADS, 1) k_gemm_igroup(const __grid_cons
             const int row = m0 + q * 32 + lane;
             const int col0 = n0 + cq * IG_EPI_COLS;
             const bool row_ok = row < p.m;
-            // group g's scales into slot g % IG_SCALE_SLOTS: sx of this lane's row, sw of columns
-            // col0 + lane and col0 + 32 + lane (zeros past the matrix); one commit group per group
+            // group g's scales into slot g % IG_SCALE_SLOTS: sx of this lane's row, sw of column
+            // col0 + lane (zeros past the matrix); one commit group per group
             auto fetch_scales = [&](int g) {
                 if (g < p.groups) {
                     float *slot = ring + (g % IG_SCALE_SLOTS) * IG_SLOT_FLOATS;
-                    const int c0 = col0 + lane, c1 = col0 + 32 + lane;
+                    const int c0 = col0 + lane;
                     cp_async4(slot + lane, p.sx + (int64_t)g * p.m + (row_ok ? row : 0), row_ok ? 4u : 0u);
                     cp_async4(slot + 32 + lane, p.sw + (int64_t)g * p.n + (c0 < p.n ? c0 : 0), c0 < p.n ? 4u : 0u);
-                    cp_async4(slot + 64 + lane, p.sw + (int64_t)g * p.n + (c1 < p.n ? c1 : 0), c1 < p.n ? 4u : 0u);
                 }
                 cp_async_commit();
             };
-            auto wait_group = [&](uint32_t g) {
-                bool w = !*abort_flag && mbar_wait(bfull + g % IG_NBUF, (g / IG_NBUF) & 1, p.wait_ns);
-                w = __all_sync(0xFFFFFFFFu, w);
-                if (!w) {
-                    if (lane == 0 && !*abort_flag) atomicOr(p.err, kErrIgEpilogue);
-                    *abort_flag = 1;
-                }
-                tc_fence_after();
-                return w;
-            };
-            // acc[j] += P[j] * (sx * sw[j]) for the 32 columns of one half; factor 1 for the branch.
+            // acc[j] += P[j] * (sx * sw[j]) over the warp's 32 columns; factor 1 for the branch.
             // Two columns per packed fp32x2 operation, each lane rounded like the scalar operation.
             float2 acc[IG_EPI_COLS / 2];
 #pragma unroll
             for (int j = 0; j < IG_EPI_COLS / 2; j++) acc[j] = make_float2(0.0f, 0.0f);
-            auto fold = [&](const uint32_t (&r)[32], float2 *accp, const float *sw, float sxv, bool lr) {
-                if (lr) {
-#pragma unroll
-                    for (int j = 0; j < 16; j++)
-                        accp[j] = __fadd2_rn(accp[j], make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])));
-                } else {
-                    const float2 sx2 = make_float2(sxv, sxv);
-                    const float4 *sw4 = reinterpret_cast<const float4 *>(sw);
-#pragma unroll
-                    for (int jj = 0; jj < 8; jj++) {
-                        const float4 w4 = sw4[jj];
-                        accp[2 * jj] = __ffma2_rn(make_float2(__uint_as_float(r[4 * jj]), __uint_as_float(r[4 * jj + 1])),
-                                                  __fmul2_rn(sx2, make_float2(w4.x, w4.y)), accp[2 * jj]);
-                        accp[2 * jj + 1] =
-                            __ffma2_rn(make_float2(__uint_as_float(r[4 * jj + 2]), __uint_as_float(r[4 * jj + 3])),
-                                       __fmul2_rn(sx2, make_float2(w4.z, w4.w)), accp[2 * jj + 1]);
-                    }
-                }
-            };
             for (int g = 0; g < IG_SCALE_AHEAD; g++) fetch_scales(g);
-            bool ok = wait_group(gc);
-            uint32_t ra[32], rb[32];
-#pragma unroll
-            for (int j = 0; j < 32; j++) ra[j] = 0u;
-            if (ok) tmem_ld_32x32b_x32_async(lane_base + (gc % IG_NBUF) * IG_BN, ra);
-            tmem_ld_wait(ra);
+            bool ok = true;
 #pragma unroll 1
             for (int gi = 0; ok && gi < ngroups; gi++, gc++) {
                 const bool lr = gi >= p.groups;
-                // slot gi + AHEAD was last read by group gi + AHEAD - SLOTS < gi, before the previous __syncwarp
+                // slot gi + AHEAD was last read by group gi + AHEAD - SLOTS < gi, before an earlier __syncwarp
                 fetch_scales(gi + IG_SCALE_AHEAD);
-                cp_async_wait<IG_SCALE_AHEAD>();   // this group's copies (all but the newest AHEAD) have landed
-                __syncwarp();                      // ... for every lane of the warp
-                const float *slot = ring + (gi % IG_SCALE_SLOTS) * IG_SLOT_FLOATS;
-                const float sxv = lr ? 1.0f : slot[lane];
                 const uint32_t b = gc % IG_NBUF;
-                tmem_ld_32x32b_x32_async(lane_base + b * IG_BN + 32, rb);   // second half, in flight
-                fold(ra, acc, slot + 32, sxv, lr);
-                tmem_ld_wait(rb);
+                ok = !*abort_flag && mbar_wait(bfull + b, (gc / IG_NBUF) & 1, p.wait_ns);
+                ok = __all_sync(0xFFFFFFFFu, ok);
+                if (!ok) {
+                    if (lane == 0 && !*abort_flag) atomicOr(p.err, kErrIgEpilogue);
+                    *abort_flag = 1;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(lane_base + b * IG_BN, r);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_local_relaxed(bempty + b);   // the MMAs may reuse this buffer
-                if (gi + 1 < ngroups) {
-                    ok = wait_group(gc + 1);
-                    if (ok) tmem_ld_32x32b_x32_async(lane_base + ((gc + 1) % IG_NBUF) * IG_BN, ra);   // next first half
+                cp_async_wait<IG_SCALE_AHEAD>();   // this group's copies (all but the newest AHEAD) have landed
+                __syncwarp();                      // ... for every lane of the warp
+                const float *slot = ring + (gi % IG_SCALE_SLOTS) * IG_SLOT_FLOATS;
+                if (lr) {
+#pragma unroll
+                    for (int j = 0; j < 16; j++)
+                        acc[j] = __fadd2_rn(acc[j], make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])));
+                } else {
+                    const float sxv = slot[lane];
+                    const float2 sx2 = make_float2(sxv, sxv);
+                    const float4 *sw4 = reinterpret_cast<const float4 *>(slot + 32);
+#pragma unroll
+                    for (int jj = 0; jj < 8; jj++) {
+                        const float4 w4 = sw4[jj];
+                        acc[2 * jj] = __ffma2_rn(make_float2(__uint_as_float(r[4 * jj]), __uint_as_float(r[4 * jj + 1])),
+                                                 __fmul2_rn(sx2, make_float2(w4.x, w4.y)), acc[2 * jj]);
+                        acc[2 * jj + 1] =
+                            __ffma2_rn(make_float2(__uint_as_float(r[4 * jj + 2]), __uint_as_float(r[4 * jj + 3])),
+                                       __fmul2_rn(sx2, make_float2(w4.z, w4.w)), acc[2 * jj + 1]);
+                    }
                 }
-                fold(rb, acc + 16, slot + 64, sxv, lr);
-                tmem_ld_wait(ra);
             }
             cp_async_wait<0>();
             if (!ok) break;
