@@ -46,20 +46,30 @@ constexpr uint32_t LT_TMEM_COLS = 64;
 constexpr int LT_SMEM_MAX = 232448;     // 227 KB per CTA
 constexpr unsigned int kErrLt = 16u;
 
-// M = 128, N = 32, bf16 x bf16 -> fp32, K-major A and B.
+// M = 128, N = 32, bf16 x bf16 -> fp32, K-major A and B; the same with B
+// MN-major (bit 16) for B tiles that are L1's own rows.
 constexpr uint32_t kLtIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((32u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t kLtIdescBmn = kLtIdesc | (1u << 16);
+
+// Shared-memory descriptor of an MN-major operand with 64-byte swizzle: rows
+// of 64 B (the 32 columns of L1), 8-row groups 512 B apart.
+__device__ __forceinline__ uint64_t sdesc_mn_sw64(const void *p) {
+    const uint64_t a = (smem_u32(p) >> 4) & 0x3FFFu;
+    return a | (1ull << 16) | (32ull << 32) | (1ull << 46) | (4ull << 61);
+}
 
 inline int lt_smem_bytes(int kb_max) { return LT_STAGES * LT_X + kb_max * LT_B + 2 * LT_RED + LT_BAR + 1024; }
 
 struct LrTcParams {
     CUtensorMap tma_x;
+    CUtensorMap tma_l1;        // L1 rows (r = 32), 64-row boxes, 64-byte swizzle; used when b_tma
     const __nv_bfloat16 *l1;   // k x r
     float *t;                  // m x r (T output) or null
     __nv_bfloat16 *tp;         // m x 64 (packed output) or null
     const float *xs, *ws;      // packed output divisor s_x * s_w; null: 1
     float *amax_slots;         // null: no amax; else warp w (2-5) of CTA b writes slot 4 b + w - 2
     unsigned int *err;
-    int m, k, r, kb_total, kb_max, row_tiles, S;
+    int m, k, r, kb_total, kb_max, row_tiles, S, b_tma;
     unsigned long long wait_ns;
 };
 
@@ -70,11 +80,11 @@ __device__ __forceinline__ void tma_load_x(const CUtensorMap *map, void *dst, ui
         "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar))
         : "memory");
 }
-__device__ __forceinline__ void mma_lt(uint32_t d, uint64_t a, uint64_t b, uint32_t acc) {
+__device__ __forceinline__ void mma_lt(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-        "l"(a), "l"(b), "r"(kLtIdesc), "r"(acc));
+        "l"(a), "l"(b), "r"(idesc), "r"(acc));
 }
 __device__ __forceinline__ void commit_lt(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -117,7 +127,8 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
     uint64_t *redfree = redf + 2;   // every receiver has consumed buffer (remote arrivals)
     uint64_t *sumdone = redfree + 2;   // the four reducing warps are done with my buffer
     uint64_t *drain = sumdone + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    uint64_t *bfull = drain + 1;    // the B tiles loaded by TMA (b_tma)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bfull + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -146,6 +157,7 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
             mbar_init(sumdone + i, 4);
         }
         mbar_init(drain, 1);
+        mbar_init(bfull, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         if (S > 1) {   // the bytes of the first two row tiles are expected before any sender may start
@@ -180,8 +192,16 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
             }
         }
     };
-    // B tile j, row n, 16-byte unit c holds L1[(kb0 + j) 64 + 8 c + t][n], t = 0..7 (128B swizzle)
-    if (p.r % 8 == 0 && (reinterpret_cast<uintptr_t>(p.l1) & 15u) == 0) {
+    if (p.b_tma) {
+        // B tile j is rows (kb0 + j) 64 .. + 63 of L1 as they are (MN-major, 64-byte swizzle,
+        // zeros past K): no transpose
+        if (warp == 0 && lane == 0) {
+            mbar_arrive_expect_tx(bfull, (uint32_t)(nkb * LT_B));
+            for (int j = 0; j < nkb; j++) tma_load_x(&p.tma_l1, btile + j * LT_B, bfull, 0, (kb0 + j) * 64);
+        }
+        prefetch_x();
+    } else if (p.r % 8 == 0 && (reinterpret_cast<uintptr_t>(p.l1) & 15u) == 0) {
+        // B tile j, row n, 16-byte unit c holds L1[(kb0 + j) 64 + 8 c + t][n], t = 0..7 (128B swizzle)
         // 8 x 8 blocks: eight independent 16-byte row loads, a transpose by byte permutes, eight stores
         auto load_block = [&](int idx, uint4 (&rv)[8]) {
             const int j = idx >> 5, c = (idx >> 2) & 7, n0 = 8 * (idx & 3);
@@ -264,6 +284,12 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
         if (lane == 0) {
             int u = 0;
             bool any = false;
+            const bool bmn = p.b_tma != 0;
+            const uint32_t idesc = bmn ? kLtIdescBmn : kLtIdesc;
+            if (bmn && ntiles > 0 && !mbar_wait(bfull, 0, p.wait_ns)) {
+                atomicOr(p.err, kErrLt);
+                *abort_flag = 1;
+            }
             for (int tc = 0; tc < ntiles && !*abort_flag; tc++) {
                 const uint32_t slot = (uint32_t)(tc & 1);
                 bool ok = mbar_wait(acce + slot, ((tc >> 1) & 1) ^ 1, p.wait_ns);
@@ -274,9 +300,10 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll
-                    for (int ks = 0; ks < 4; ks++)
+                    for (int ks = 0; ks < 4; ks++)   // K = 16 per MMA: 32 bytes of a K-major row, 16 rows of an MN-major tile
                         mma_lt(tmem + slot * 32, sdesc_sw128(xst + s * LT_X + ks * 32),
-                               sdesc_sw128(btile + j * LT_B + ks * 32), (j > 0 || ks > 0) ? 1u : 0u);
+                               bmn ? sdesc_mn_sw64(btile + j * LT_B + ks * 1024) : sdesc_sw128(btile + j * LT_B + ks * 32),
+                               idesc, (j > 0 || ks > 0) ? 1u : 0u);
                     commit_lt(empty + s);
                     any = true;
                 }
@@ -318,8 +345,9 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
                 }
                 if (!ok) break;
             }
+            // the waits of this phase poll: the stream is over, so nothing else needs the issue slots
             const uint32_t slot = (uint32_t)(tc & 1);
-            bool w = !*abort_flag && mbar_wait(accf + slot, (tc >> 1) & 1, p.wait_ns);
+            bool w = !*abort_flag && mbar_wait_spin(accf + slot, (tc >> 1) & 1, p.wait_ns);
             if (!__all_sync(0xFFFFFFFFu, w)) {
                 ok = false;
                 break;
@@ -333,7 +361,7 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
 
             // send this thread's row (row q*32 + lane of the tile) to the CTA that owns it
             const uint32_t pb = (uint32_t)(tc & 1);
-            w = mbar_wait<true>(redfree + pb, ((tc >> 1) & 1) ^ 1, p.wait_ns);
+            w = mbar_wait_spin<true>(redfree + pb, ((tc >> 1) & 1) ^ 1, p.wait_ns);
             if (!__all_sync(0xFFFFFFFFu, w)) {
                 ok = false;
                 break;
@@ -354,7 +382,7 @@ __global__ void __launch_bounds__(LT_THREADS, 1) k_lowrank_tc(const __grid_const
             }
 
             // receive rows [rank R, rank R + R) from every CTA, add in rank order, write
-            w = mbar_wait<true>(redf + pb, (tc >> 1) & 1, p.wait_ns);
+            w = mbar_wait_spin<true>(redf + pb, (tc >> 1) & 1, p.wait_ns);
             if (!__all_sync(0xFFFFFFFFu, w)) {
                 ok = false;
                 break;
@@ -503,6 +531,10 @@ cudaError_t launch_lowrank_tc(const void *x, int64_t m, int64_t k, const void *l
     if (!encode_2d(&p.tma_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)k, (uint64_t)m, (uint64_t)k * 2, 64, 128,
                    CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
+    // rank 32: the B tiles are L1's rows loaded as they are (else built by a transpose in the kernel)
+    p.b_tma = r == 32 && (reinterpret_cast<uintptr_t>(l1) & 15u) == 0 &&
+              encode_2d(&p.tma_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, l1, 32, (uint64_t)k, 64, 32, 64,
+                        CU_TENSOR_MAP_SWIZZLE_64B);
     const int smem = lt_smem_bytes(p.kb_max);
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
