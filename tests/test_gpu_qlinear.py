@@ -123,6 +123,21 @@ def test_lowrank_down(mxq, orc):
     assert np.abs(t - ref).max() <= 1e-5 * np.abs(ref).max()
 
 
+@pytest.mark.parametrize("m,k,r", [(300, 208, 32), (129, 80, 32), (257, 1104, 32), (300, 208, 24), (64, 16, 32)])
+def test_lowrank_down_ragged(mxq, orc, m, k, r):
+    """T = bf16(X) . L1 with K not a multiple of the 64-column k-block (the
+    rank-32 path loads L1's rows by TMA and the rows past K read as zeros; the
+    other ranks build the tiles in the kernel) and M not a multiple of 128;
+    every element against the oracle's binary64 T."""
+    rng = np.random.default_rng(70 + k + r)
+    x = workloads.to_bf16_values(rng.standard_t(4, size=(m, k)).astype(np.float32))
+    l1 = workloads.to_bf16_values((rng.standard_normal((k, r)) * 0.05).astype(np.float32))
+    t = mxq.lowrank_down(dev(x, "bf16"), dev(l1, "bf16")).cpu().numpy().astype(np.float64)
+    ref = orc.lowrank_down(x, l1)
+    assert t.shape == ref.shape
+    assert np.abs(t - ref).max() <= 1e-5 * max(np.abs(ref).max(), 1e-30)
+
+
 def test_tiny_nvfp4_linear_full(mxq, orc):
     """Workload 1 end to end, every output: fp32 X, NVFP4, rank-8 branch."""
     w1 = workloads.tiny_nvfp4_linear()
