@@ -426,6 +426,171 @@ __global__ void __launch_bounds__(kThreads) k_quantize_int8_row_reg(const T *__r
     }
 }
 
+// INT8 per row for bf16 rows of more than 2048 elements, staged in shared
+// memory: each CTA walks blocks of kRowBlk consecutive rows; one bulk copy
+// brings a block into one of two stages while the CTA codes the one before.
+// kI8Parts warps share a row: thread (part, lane) owns the 16-byte words
+// part * 32 + lane + 128 j of it (a warp reads 512 consecutive bytes), keeps
+// them in registers, forms their maximum, and after the parts' maxima meet
+// in shared memory codes them.  The arithmetic is that of
+// k_quantize_int8_row_reg; on long rows this kernel keeps more of the input
+// in flight than one warp per row can hold in registers.
+constexpr int kRowBlk = 4;            // rows per block
+constexpr int kI8Parts = 4;           // warps per row
+constexpr int kI8RowThreads = 32 * kRowBlk * kI8Parts;
+constexpr int kI8CtasPerSm = 2;       // so that one CTA codes while the other waits at a barrier
+constexpr int kI8Stages = 2;          // a block is coded while the next one loads
+constexpr int kI8SmemCap = 113664;    // dynamic shared memory opt-in per CTA: two CTAs fit on an SM
+constexpr unsigned int kErrI8Row = 32u;   // error-word bit of a wait on a block's copy that ran out
+
+__device__ __forceinline__ void bulk_load_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4 &w, float v[8]) {
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        v[2 * j] = __uint_as_float(u[j] << 16);
+        v[2 * j + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
+    }
+}
+
+template <int NQ>
+__global__ void __launch_bounds__(kI8RowThreads, kI8CtasPerSm)
+    k_quantize_int8_row_staged(const __nv_bfloat16 *__restrict__ x, QuantArgs a, unsigned int *err,
+                               unsigned long long wait_ns) {
+    constexpr int nst = kI8Stages;
+    extern __shared__ __align__(128) uint8_t sx[];
+    __shared__ float part_max[kRowBlk][kI8Parts];
+    __shared__ int abort_flag;
+    const int lane = lane_id(), warp = (int)(threadIdx.x >> 5);
+    const int rw = warp / kI8Parts, part = warp % kI8Parts;
+    const int words = (int)(a.cols >> 3);
+    const uint32_t row_bytes = (uint32_t)(a.cols * 2);
+    const uint32_t stage_bytes = row_bytes * kRowBlk;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sx + (size_t)nst * stage_bytes);
+    const int64_t nblk = (a.rows + kRowBlk - 1) / kRowBlk;
+    if (threadIdx.x == 0) {
+        for (int j = 0; j < nst; j++) mbar_init(full + j, 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    auto issue = [&](int64_t b, int st) {
+        const int64_t r0 = b * kRowBlk;
+        const uint32_t nr = (uint32_t)(a.rows - r0 < kRowBlk ? a.rows - r0 : kRowBlk);
+        mbar_arrive_expect_tx(full + st, row_bytes * nr);
+        bulk_load_g2s(sx + (size_t)st * stage_bytes, x + r0 * a.cols, row_bytes * nr, full + st);
+    };
+    int64_t issued = 0;
+    if (threadIdx.x == 0) {
+        for (int j = 0; j < nst; j++) {
+            const int64_t b = blockIdx.x + (int64_t)j * gridDim.x;
+            if (b < nblk) {
+                issue(b, j);
+                issued++;
+            }
+        }
+    }
+    int st = 0;
+    uint32_t ph = 0;
+    int64_t it = 0;
+    for (int64_t b = blockIdx.x; b < nblk; b += gridDim.x, it++) {
+        if (!mbar_wait(full + st, ph, wait_ns)) {
+            if (lane == 0) atomicOr(err, kErrI8Row);
+            abort_flag = 1;
+        }
+        const int64_t row = b * kRowBlk + rw;
+        const bool live = row < a.rows;
+        const uint4 *src = reinterpret_cast<const uint4 *>(sx + (size_t)st * stage_bytes + (size_t)rw * row_bytes);
+        uint4 w[NQ];
+        float m = 0.0f;
+#pragma unroll
+        for (int j = 0; j < NQ; j++) {
+            const int q = part * 32 + lane + 128 * j;
+            w[j] = make_uint4(0u, 0u, 0u, 0u);
+            if (live && q < words) w[j] = src[q];
+            float v[8];
+            unpack_bf16x8(w[j], v);
+#pragma unroll
+            for (int e = 0; e < 8; e++) m = fmaxf(m, fabsf(v[e]));
+        }
+        m = group_max<32>(m);
+        if (lane == 0) part_max[rw][part] = m;
+        __syncthreads();   // the parts' maxima are in; an expired wait anywhere ends every thread here
+        if (abort_flag) break;
+        if (live) {
+            float rm = part_max[rw][0];
+#pragma unroll
+            for (int j = 1; j < kI8Parts; j++) rm = fmaxf(rm, part_max[rw][j]);
+            const float sc = __fdiv_rn(rm, 127.0f);
+            const Recip rs = recip_of(sc);
+            uint8_t *dst = a.codes + row * a.cols;
+#pragma unroll
+            for (int j = 0; j < NQ; j++) {
+                const int q = part * 32 + lane + 128 * j;
+                if (q < words) {
+                    float v[8];
+                    unpack_bf16x8(w[j], v);
+                    *reinterpret_cast<uint2 *>(dst + (int64_t)q * 8) =
+                        make_uint2(int_x4_quot(v, rs, 127), int_x4_quot(v + 4, rs, 127));
+                }
+            }
+            if (lane == 0 && part == 0) reinterpret_cast<float *>(a.scales)[row] = sc;
+        }
+        __syncthreads();   // stage st and part_max are free: thread 0 refills the stage
+        if (threadIdx.x == 0) {
+            const int64_t b2 = b + (int64_t)nst * gridDim.x;
+            if (b2 < nblk) {
+                issue(b2, st);
+                issued++;
+            }
+        }
+        if (++st == nst) {
+            st = 0;
+            ph ^= 1u;
+        }
+    }
+    if (threadIdx.x == 0 && abort_flag) {   // let the copies in flight land before the CTA exits
+        for (int64_t j = it; j < issued; j++) mbar_wait(full + (int)(j % nst), (uint32_t)((j / nst) & 1), wait_ns);
+    }
+}
+
+// One launch of k_quantize_int8_row_staged<NQ>, after its one-time opt-in
+// to the large shared-memory carve-out on this device.
+template <int NQ>
+bool launch_int8_row_staged_nq(const __nv_bfloat16 *x, const QuantArgs &a, int grid, size_t smem, unsigned int *err,
+                               cudaStream_t s) {
+    static PerDeviceOnce opt_in;
+    if (opt_in.run([] {
+            return cudaFuncSetAttribute(k_quantize_int8_row_staged<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        kI8SmemCap);
+        }) != cudaSuccess)
+        return false;
+    k_quantize_int8_row_staged<NQ><<<grid, kI8RowThreads, smem, s>>>(x, a, err, 2000000000ull);
+    return true;
+}
+
+// Launches k_quantize_int8_row_staged when it takes the shape (bf16 rows of
+// at most 5120 elements, a multiple of 8, starting 16-byte aligned: two
+// stages of 4 rows take at most 80 KB); false (nothing launched) otherwise.
+bool launch_int8_row_staged(const __nv_bfloat16 *x, const QuantArgs &a, cudaStream_t s) {
+    const int64_t words = a.cols >> 3;
+    if (a.rows <= 0 || a.cols % 8 || words > 128 * 5 || (reinterpret_cast<uintptr_t>(x) & 15u)) return false;
+    const size_t smem = (size_t)kI8Stages * kRowBlk * a.cols * 2 + 8 * kI8Stages;
+    unsigned int *err = nullptr;
+    if (error_word_address(&err) != cudaSuccess) return false;
+    const int64_t nblk = (a.rows + kRowBlk - 1) / kRowBlk;
+    const int64_t cap = (int64_t)sm_count() * kI8CtasPerSm;
+    const int grid = (int)(nblk < cap ? nblk : cap);
+    if (words <= 128 * 4) return launch_int8_row_staged_nq<4>(x, a, grid, smem, err, s);
+    return launch_int8_row_staged_nq<5>(x, a, grid, smem, err, s);
+}
+
 // ------------------------------------------------------------------ dequantize
 
 struct DequantArgs {
@@ -1023,6 +1188,9 @@ static void launch_q(int fmt, int grid, const T *x, const QuantArgs &a, cudaStre
     case kINT4G64: launch_qf<T, kINT4G64>(x, a, s); break;
     case kFP8Tensor: launch_qf<T, kFP8Tensor>(x, a, s); break;
     case kINT8Row: {
+        if (sizeof(T) == 2 && a.hadamard_b == 0 && a.cols > 2048 &&
+            launch_int8_row_staged(reinterpret_cast<const __nv_bfloat16 *>(x), a, s))
+            break;
         int g = grid_for(a.rows, sm_count_cached());
         const int64_t cpr = a.cols >> 4;
         if (a.hadamard_b == 0 && cpr <= 32) k_quantize_int8_row_reg<T, 1><<<g, kThreads, 0, s>>>(x, a);

@@ -44,6 +44,21 @@ def test_quantize_small_ragged(mxq, orc, fmt, dtype, hadamard_b):
         assert_qtensor_equal(q, ref, layout_mma=layout == mxq.MMA)
 
 
+@pytest.mark.parametrize("rows,cols", [(4097, 2064), (5, 5120), (3, 2560), (1, 4096), (1027, 4608), (6, 5136),
+                                       (2, 2048)])
+def test_quantize_int8_row_long_rows(mxq, orc, rows, cols):
+    """INT8 per row over bf16 rows longer than 2048 elements, where rows are
+    coded in blocks of 4 staged in shared memory: ragged last blocks, single
+    rows, the longest row that path takes (5120) and rows just outside it on
+    both sides; every code and scale."""
+    x = nasty_matrix(300 + rows % 97 + cols % 89, rows, cols)
+    ref = orc.quantize(host_values(x, "bf16"), mxq.INT8_ROW)
+    for layout in (mxq.CANONICAL, mxq.MMA):
+        q = mxq.quantize(dev(x, "bf16"), mxq.INT8_ROW, 0, layout)
+        torch.cuda.synchronize()
+        assert_qtensor_equal(q, ref, layout_mma=layout == mxq.MMA)
+
+
 @pytest.mark.parametrize("fmt", ALL_FMTS)
 def test_quantize_edge_shapes(mxq, orc, fmt):
     blk = {0: 32, 1: 32, 2: 16, 3: 32, 4: 64, 5: 16, 6: 16}[fmt]
