@@ -204,6 +204,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16() { return idesc_common() | (1
 // Scale-factor atoms (512 B) per stage for 128 rows.
 template <int KIND>
 __host__ __device__ constexpr int sf_atoms() { return KIND == kKindNVFP4 ? 4 : KIND == kKindMXFP4 ? 2 : KIND == kKindMXFP8 ? 1 : 0; }
+// Accumulator stage 1 and the columns it shares with stage 0: the kinds
+// without block scales leave the scale-factor slots empty, so their two
+// stages are disjoint ([0, 256) and [256, 512)) and a tile's MMAs wait only
+// for the drain of the tile two before.
+template <int KIND>
+__host__ __device__ constexpr uint32_t acc_stage1() { return sf_atoms<KIND>() ? ACC_STAGE1 : 256u; }
+template <int KIND>
+__host__ __device__ constexpr int ovl_chunks() { return sf_atoms<KIND>() ? (int)OVL_CHUNKS : 0; }
 
 __device__ __forceinline__ void latch_error(unsigned int code) { atomicOr(&g_error_word, code); }
 
@@ -367,10 +375,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             const int nk_full = p.kbytes / BKB;   // k-tiles with all four k-steps
             for (int tile = cid; tile < num_tiles && !*abort_flag; tile += ncl, tcount++) {
                 const int st = tcount & 1;
-                const uint32_t acc_addr = tmem + (st ? ACC_STAGE1 : 0u);
+                const uint32_t acc_addr = tmem + (st ? acc_stage1<KIND>() : 0u);
                 // this stage drained (tile tcount-2) and the shared columns (tile tcount-1), in both CTAs
                 bool ok = mbar_wait_spin<true>(acce + st, ((tcount >> 1) & 1) ^ 1, p.wait_ns);
-                if (ok && tcount > 0) ok = mbar_wait_spin<true>(ovlf, (tcount - 1) & 1, p.wait_ns);
+                if (ovl_chunks<KIND>() > 0 && ok && tcount > 0)
+                    ok = mbar_wait_spin<true>(ovlf, (tcount - 1) & 1, p.wait_ns);
                 if (!ok) {
                     latch_error(kErrTimeoutMma);
                     *abort_flag = 1;
@@ -488,8 +497,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 break;
             }
             tc_fence_after();
-            const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + (st ? ACC_STAGE1 : 0u);
-            float ra = 0.0f;   // INT8 row scale, read once the shared columns are released
+            const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16) + (st ? acc_stage1<KIND>() : 0u);
+            constexpr int OVL = ovl_chunks<KIND>();
+            static_assert(KIND != kKindINT8 || OVL == 0, "the INT8 row scale is read before any chunk");
+            float ra = 0.0f;   // INT8 row scale
             const bool row_ok = row < p.m;
             // The shared columns (the last OVL_CHUNKS chunks of stage 0, the first OVL_CHUNKS of
             // stage 1) go to registers first and are released at once, so the next tile's MMAs
@@ -558,22 +569,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                         }
                     }
             };
-            uint32_t ro[OVL_CHUNKS][32];
+            if constexpr (OVL > 0) {
+                uint32_t ro[OVL][32];
 #pragma unroll
-            for (int i = 0; i < (int)OVL_CHUNKS; i++)
-                tmem_ld_32x32b_x32_async(lane_base + (uint32_t)((st ? i : 8 - (int)OVL_CHUNKS + i) * 32), ro[i]);
-            tmem_ld_wait(ro[OVL_CHUNKS - 1]);
+                for (int i = 0; i < OVL; i++)
+                    tmem_ld_32x32b_x32_async(lane_base + (uint32_t)((st ? i : 8 - OVL + i) * 32), ro[i]);
+                tmem_ld_wait(ro[OVL - 1]);
 #pragma unroll
-            for (int i = 0; i + 1 < (int)OVL_CHUNKS; i++) tmem_reg_tie(ro[i]);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_remote_relaxed(ovl_leader);
-            if (KIND == kKindINT8 && row_ok) ra = __ldg(p.a_row_scale + row);
+                for (int i = 0; i + 1 < OVL; i++) tmem_reg_tie(ro[i]);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote_relaxed(ovl_leader);
 #pragma unroll
-            for (int i = 0; i < (int)OVL_CHUNKS; i++) process(st ? i : 8 - (int)OVL_CHUNKS + i, ro[i]);
+                for (int i = 0; i < OVL; i++) process(st ? i : 8 - OVL + i, ro[i]);
+            }
+            if (KIND == kKindINT8 && row_ok) ra = __ldg(p.a_row_scale + row);   // INT8 has no shared columns
 #pragma unroll 1
-            for (int i = (int)OVL_CHUNKS; i < BN / 32; i++) {
-                const int c = st ? i : i - (int)OVL_CHUNKS;
+            for (int i = OVL; i < BN / 32; i++) {
+                const int c = st ? i : i - OVL;
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(lane_base + (uint32_t)(c * 32), r);
                 if (i == BN / 32 - 1) {   // the whole stage is drained

@@ -265,10 +265,13 @@ __device__ __forceinline__ uint32_t e2m1x8_quot(const float *v, const Recip &r) 
 // E4M3 codes of RN(v[i] / d) for four values, packed like cvt_e4m3x4.
 __device__ __forceinline__ uint32_t e4m3x4_quot(const float *v, const Recip &r) {
     if (r.fast) {
-        const uint32_t lo = cvt_e4m3x4(__fmul_rn(v[0], r.lo), __fmul_rn(v[1], r.lo), __fmul_rn(v[2], r.lo),
-                                       __fmul_rn(v[3], r.lo));
-        const uint32_t hi = cvt_e4m3x4(__fmul_rn(v[0], r.hi), __fmul_rn(v[1], r.hi), __fmul_rn(v[2], r.hi),
-                                       __fmul_rn(v[3], r.hi));
+        // packed two-wide products, each lane rounded like __fmul_rn
+        const float2 v01 = make_float2(v[0], v[1]), v23 = make_float2(v[2], v[3]);
+        const float2 lo2 = make_float2(r.lo, r.lo), hi2 = make_float2(r.hi, r.hi);
+        const float2 l01 = __fmul2_rn(v01, lo2), l23 = __fmul2_rn(v23, lo2);
+        const float2 h01 = __fmul2_rn(v01, hi2), h23 = __fmul2_rn(v23, hi2);
+        const uint32_t lo = cvt_e4m3x4(l01.x, l01.y, l23.x, l23.y);
+        const uint32_t hi = cvt_e4m3x4(h01.x, h01.y, h23.x, h23.y);
         if (lo == hi) return lo;
     }
     return cvt_e4m3x4(__fdiv_rn(v[0], r.d), __fdiv_rn(v[1], r.d), __fdiv_rn(v[2], r.d), __fdiv_rn(v[3], r.d));
@@ -303,6 +306,24 @@ __device__ __forceinline__ uint32_t int_x4_quot(const float *v, const Recip &r, 
         out |= ((uint32_t)q & 0xFFu) << (8 * i);
     }
     return out;
+}
+
+// int_x4_quot with the bracket FMAs packed two-wide (each lane rounded like
+// __fmaf_rn): fewer instructions, two more live registers, so it is used
+// where registers are not the limit (the staged INT8 per-row kernel).
+__device__ __forceinline__ uint32_t int_x4_quot_packed(const float *v, const Recip &r, int qmax) {
+    if (r.d == 0.0f) return 0u;
+    if (r.fast) {
+        const float2 lo2 = make_float2(r.lo, r.lo), hi2 = make_float2(r.hi, r.hi);
+        const float2 mg = make_float2(kRoundMagic, kRoundMagic);
+        const float2 v01 = make_float2(v[0], v[1]), v23 = make_float2(v[2], v[3]);
+        const float2 l01 = __ffma2_rn(v01, lo2, mg), l23 = __ffma2_rn(v23, lo2, mg);
+        const float2 h01 = __ffma2_rn(v01, hi2, mg), h23 = __ffma2_rn(v23, hi2, mg);
+        if (l01.x == h01.x && l01.y == h01.y && l23.x == h23.x && l23.y == h23.y)
+            return __byte_perm(__byte_perm(__float_as_uint(l01.x), __float_as_uint(l01.y), 0x0040),
+                               __byte_perm(__float_as_uint(l23.x), __float_as_uint(l23.y), 0x0040), 0x5410);
+    }
+    return int_x4_quot(v, Recip{r.d, r.lo, r.hi, false}, qmax);   // exact divisions
 }
 
 // The same integer codes as E4M3 bytes (element i in byte i).  Every integer

@@ -537,7 +537,7 @@ __global__ void __launch_bounds__(kI8RowThreads, kI8CtasPerSm)
                     float v[8];
                     unpack_bf16x8(w[j], v);
                     *reinterpret_cast<uint2 *>(dst + (int64_t)q * 8) =
-                        make_uint2(int_x4_quot(v, rs, 127), int_x4_quot(v + 4, rs, 127));
+                        make_uint2(int_x4_quot_packed(v, rs, 127), int_x4_quot_packed(v + 4, rs, 127));
                 }
             }
             if (lane == 0 && part == 0) reinterpret_cast<float *>(a.scales)[row] = sc;
