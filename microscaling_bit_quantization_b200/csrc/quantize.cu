@@ -212,11 +212,25 @@ __device__ __forceinline__ void encode_chunk(const float (&v)[16], float amax, u
         }
     } else if (F == kFP8Tensor) {
         if (!valid) return;
-        uint4 w;
-        w.x = e4m3x4_quot(v, rt);
-        w.y = e4m3x4_quot(v + 4, rt);
-        w.z = e4m3x4_quot(v + 8, rt);
-        w.w = e4m3x4_quot(v + 12, rt);
+        // both ends of the four brackets without branches; one test sends the
+        // chunk to e4m3x4_quot (same codes) when any pair disagrees
+        const float2 lo2 = make_float2(rt.lo, rt.lo), hi2 = make_float2(rt.hi, rt.hi);
+        uint32_t lo[4], hi[4];
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            const float2 v01 = make_float2(v[4 * k], v[4 * k + 1]), v23 = make_float2(v[4 * k + 2], v[4 * k + 3]);
+            const float2 l01 = __fmul2_rn(v01, lo2), l23 = __fmul2_rn(v23, lo2);
+            const float2 h01 = __fmul2_rn(v01, hi2), h23 = __fmul2_rn(v23, hi2);
+            lo[k] = cvt_e4m3x4(l01.x, l01.y, l23.x, l23.y);
+            hi[k] = cvt_e4m3x4(h01.x, h01.y, h23.x, h23.y);
+        }
+        uint4 w = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        if (!(rt.fast && lo[0] == hi[0] && lo[1] == hi[1] && lo[2] == hi[2] && lo[3] == hi[3])) {
+            w.x = e4m3x4_quot(v, rt);
+            w.y = e4m3x4_quot(v + 4, rt);
+            w.z = e4m3x4_quot(v + 8, rt);
+            w.w = e4m3x4_quot(v + 12, rt);
+        }
         *reinterpret_cast<uint4 *>(a.codes + (int64_t)c * 16) = w;
     }
 }
