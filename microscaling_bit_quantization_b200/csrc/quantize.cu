@@ -1153,6 +1153,45 @@ cudaError_t launch_amax(const void *x, bool bf16, int64_t rows, int64_t cols, in
     return cudaGetLastError();
 }
 
+// The tensor amax of an unrotated tensor as per-CTA maxima: a grid-stride
+// stream of 16-byte words, kAmaxWords of them in flight per thread, each
+// CTA writing the max |x| of its words to out[blockIdx.x].  The maximum is
+// exact and independent of the order it is taken in (fmaxf: a NaN never
+// wins), so it is the same value the chunk loop of k_quantize would give.
+constexpr int kAmaxWords = 8;   // 128 B in flight per thread, 128 KB per SM
+__device__ __forceinline__ float amax_word(const uint4 &w, bool bf16) {
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+    float m = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        if (bf16) {
+            m = fmaxf(m, fabsf(__uint_as_float(u[j] << 16)));
+            m = fmaxf(m, fabsf(__uint_as_float(u[j] & 0xFFFF0000u)));
+        } else {
+            m = fmaxf(m, fabsf(__uint_as_float(u[j])));
+        }
+    }
+    return m;
+}
+template <bool BF16>
+__global__ void __launch_bounds__(kQThreads, 2) k_amax_words(const uint4 *__restrict__ x, int64_t words, float *out) {
+    pdl_wait();   // nothing is read before the previous kernel has completed
+    pdl_launch_dependents();
+    const int64_t stride = (int64_t)gridDim.x * kQThreads;
+    int64_t i = (int64_t)blockIdx.x * kQThreads + threadIdx.x;
+    float m = 0.0f;
+    for (; i + (kAmaxWords - 1) * stride < words; i += kAmaxWords * stride) {
+        uint4 w[kAmaxWords];
+#pragma unroll
+        for (int u = 0; u < kAmaxWords; u++) w[u] = __ldg(x + i + u * stride);
+#pragma unroll
+        for (int u = 0; u < kAmaxWords; u++) m = fmaxf(m, amax_word(w[u], BF16));
+    }
+    for (; i < words; i += stride) m = fmaxf(m, amax_word(__ldg(x + i), BF16));
+    const float r = cta_reduce_max<kQThreads>(m);
+    if (threadIdx.x == 0) out[blockIdx.x] = r;
+}
+
 // The tensor amax as per-CTA maxima (no clearing, no atomics): slots must
 // hold 2 x SM-count floats; *n_slots gets the count written.
 static cudaError_t launch_amax_slots(const void *x, bool bf16, int64_t rows, int64_t cols, int hadamard_b,
@@ -1168,8 +1207,26 @@ static cudaError_t launch_amax_slots(const void *x, bool bf16, int64_t rows, int
     a.cpr = make_fastdiv((uint32_t)(cols / 16 > 0 ? cols / 16 : 1));
     a.hadamard_b = hadamard_b;
     a.amax_out = slots;
-    const int64_t steps = (chunks + kQThreads - 1) / kQThreads;
     const int64_t cap = (int64_t)sm_count_cached() * 2;
+    if (hadamard_b == 0) {
+        const int64_t words = chunks * (bf16 ? 2 : 4);
+        const int64_t per_cta = (int64_t)kQThreads * kAmaxWords;
+        const int64_t want = (words + per_cta - 1) / per_cta;
+        const int grid = (int)(want < cap ? want : cap);
+        *n_slots = grid;
+        cudaLaunchConfig_t cfg;
+        memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3((unsigned)grid, 1, 1);
+        cfg.blockDim = dim3(kQThreads, 1, 1);
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1] = {pdl_attribute()};
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (bf16) cudaLaunchKernelEx(&cfg, k_amax_words<true>, (const uint4 *)x, words, slots);
+        else cudaLaunchKernelEx(&cfg, k_amax_words<false>, (const uint4 *)x, words, slots);
+        return cudaGetLastError();
+    }
+    const int64_t steps = (chunks + kQThreads - 1) / kQThreads;
     *n_slots = (int)(steps < cap ? steps : cap);
     if (bf16) launch_qf<__nv_bfloat16, kNumFmt>((const __nv_bfloat16 *)x, a, s);
     else launch_qf<float, kNumFmt>((const float *)x, a, s);
