@@ -657,8 +657,8 @@ def run_ours(args, world, rank, local):
         b.record(stream)
         torch.cuda.synchronize()
     rows["tiny_nvfp4_latency"] = {
-        "workload": "X 64 x 256 fp32, W 128 x 256, NVFP4, rank 8, fp32 out: memset + k_lowrank (fp32 X) + "
-                    "k_quantize + k_gemm",
+        "workload": "X 64 x 256 fp32, W 128 x 256, NVFP4, rank 8, fp32 out: k_lowrank (fp32 X, per-CTA amax "
+                    "slots) + k_quantize + k_gemm",
         "eager_us_median_of_50": 1e3 * statistics.median(a.elapsed_time(b) for a, b in evs),
         "graph_replay_us": 1e3 * timer.graph_ms(tiny, n=20, reps=5)}
     del x1, wq1, xq1, tp1, ws1, y1

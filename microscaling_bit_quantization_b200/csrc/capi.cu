@@ -368,12 +368,17 @@ mxq_status mxq_quantize_lowrank(const void *x, int32_t xdtype, int64_t m, int64_
     int n_slots = 0;
     if (ts && hadamard_b == 0) {
         // one read of x from HBM gives both the tensor amax and t: the
-        // tensor-core kernel writes per-warp maxima (no clearing needed, so
-        // the three kernels follow each other with no memset between); the
-        // other kernels fold into a zeroed word
+        // tensor-core kernel writes per-warp maxima and the mma.sync kernels
+        // per-CTA maxima (every slot written, so no clearing: the kernels
+        // follow each other with no memset between); only a grid with more
+        // CTAs than slots folds into a zeroed word
         e = bf ? launch_lowrank_tc(x, m, k, l1, r, t, nullptr, nullptr, nullptr, slots, &n_slots, s)
                : cudaErrorNotSupported;
-        if (e == cudaErrorNotSupported) {
+        if (e == cudaErrorNotSupported) {   // the mma.sync kernels: one maximum per CTA, still no clearing
+            n_slots = 0;
+            e = launch_lowrank_down(x, bf, m, k, l1, r, t, nullptr, nullptr, nullptr, s, nullptr, slots, &n_slots);
+        }
+        if (e == cudaErrorNotSupported) {   // more CTAs than slots: fold into a cleared word
             n_slots = 0;
             e = cudaMemsetAsync(amax, 0, sizeof(unsigned int), s);
             if (e == cudaSuccess) e = launch_lowrank_down(x, bf, m, k, l1, r, t, nullptr, nullptr, nullptr, s, amax);

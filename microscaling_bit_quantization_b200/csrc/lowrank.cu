@@ -47,12 +47,14 @@ constexpr int kLrWarps = 8, kLrUnroll = 8;
 // eight partial tiles are summed in a fixed order through shared memory.
 //   kLrT      t (m x r fp32)
 //   kLrPacked the GEMM operand tp (m x 64 bf16, [hi | lo] of t / (xs * ws))
-//   kLrTAmax  t, and max |x| over the whole tensor into *amax_word
+//   kLrTAmax  t, and max |x| over the whole tensor: each CTA's maximum into
+//             amax_slots[blockIdx.x], or folded into *amax_word
 template <typename T, int MODE>
 __global__ void __launch_bounds__(kLrWarps * 32) k_lowrank(const T *__restrict__ x, int64_t m, int64_t k,
                                                          const __nv_bfloat16 *__restrict__ l1, int r,
                                                          float *__restrict__ t, const float *xs, const float *ws,
-                                                         __nv_bfloat16 *__restrict__ tp, unsigned int *amax_word) {
+                                                         __nv_bfloat16 *__restrict__ tp, unsigned int *amax_word,
+                                                         float *amax_slots) {
     __shared__ float red[kLrWarps][16][33];
     __shared__ float wmax[kLrWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -115,7 +117,8 @@ __global__ void __launch_bounds__(kLrWarps * 32) k_lowrank(const T *__restrict__
     if (MODE == kLrTAmax && threadIdx.x == 0) {
         float v = 0.0f;
         for (int w = 0; w < kLrWarps; w++) v = fmaxf(v, wmax[w]);
-        if (v > 0.0f) atomicMax(amax_word, __float_as_uint(v));
+        if (amax_slots) amax_slots[blockIdx.x] = v;   // every CTA writes its slot: no clearing
+        else if (v > 0.0f) atomicMax(amax_word, __float_as_uint(v));
     }
     float alpha = 1.0f;
     if (MODE == kLrPacked && xs) alpha = __fmul_rn(*xs, *ws);
@@ -204,7 +207,8 @@ template <int MODE>
 __global__ void __launch_bounds__(kLsThreads) k_lowrank_staged(const __nv_bfloat16 *__restrict__ x, int64_t m, int64_t k,
                                                               const __nv_bfloat16 *__restrict__ l1, int r,
                                                               float *__restrict__ t, const float *xs, const float *ws,
-                                                              __nv_bfloat16 *__restrict__ tp, unsigned int *amax_word) {
+                                                              __nv_bfloat16 *__restrict__ tp, unsigned int *amax_word,
+                                                              float *amax_slots) {
     extern __shared__ __align__(128) uint8_t ls_smem[];
     __shared__ float red[4][16][33];
     __shared__ float wmax[4];
@@ -286,7 +290,8 @@ __global__ void __launch_bounds__(kLsThreads) k_lowrank_staged(const __nv_bfloat
     __syncthreads();
     if (MODE == kLrTAmax && tid == 0) {
         const float v = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
-        if (v > 0.0f) atomicMax(amax_word, __float_as_uint(v));
+        if (amax_slots) amax_slots[blockIdx.x] = v;   // every CTA writes its slot: no clearing
+        else if (v > 0.0f) atomicMax(amax_word, __float_as_uint(v));
     }
     float alpha = 1.0f;
     if (MODE == kLrPacked && xs) alpha = __fmul_rn(*xs, *ws);
@@ -310,22 +315,28 @@ __global__ void __launch_bounds__(kLsThreads) k_lowrank_staged(const __nv_bfloat
 
 template <typename T>
 static void launch_lr(int mode, int grid, const T *x, int64_t m, int64_t k, const __nv_bfloat16 *l1, int r, float *t,
-                      const float *xs, const float *ws, __nv_bfloat16 *tp, unsigned int *amax, cudaStream_t s) {
+                      const float *xs, const float *ws, __nv_bfloat16 *tp, unsigned int *amax, float *slots,
+                      cudaStream_t s) {
     const int threads = kLrWarps * 32;
-    if (mode == kLrT) k_lowrank<T, kLrT><<<grid, threads, 0, s>>>(x, m, k, l1, r, t, xs, ws, tp, amax);
-    else if (mode == kLrPacked) k_lowrank<T, kLrPacked><<<grid, threads, 0, s>>>(x, m, k, l1, r, t, xs, ws, tp, amax);
-    else k_lowrank<T, kLrTAmax><<<grid, threads, 0, s>>>(x, m, k, l1, r, t, xs, ws, tp, amax);
+    if (mode == kLrT) k_lowrank<T, kLrT><<<grid, threads, 0, s>>>(x, m, k, l1, r, t, xs, ws, tp, amax, slots);
+    else if (mode == kLrPacked)
+        k_lowrank<T, kLrPacked><<<grid, threads, 0, s>>>(x, m, k, l1, r, t, xs, ws, tp, amax, slots);
+    else k_lowrank<T, kLrTAmax><<<grid, threads, 0, s>>>(x, m, k, l1, r, t, xs, ws, tp, amax, slots);
 }
 
 cudaError_t launch_lowrank_down(const void *x, bool bf16, int64_t m, int64_t k, const void *l1, int r, float *t,
-                                const float *xs, const float *ws, void *tp, cudaStream_t s, unsigned int *amax_word) {
+                                const float *xs, const float *ws, void *tp, cudaStream_t s, unsigned int *amax_word,
+                                float *amax_slots, int *n_slots) {
     if (m == 0) return cudaSuccess;
-    if (bf16 && !amax_word) {   // the tensor-core path when it takes the shape (its amax goes to slots)
+    if (bf16 && !amax_word && !amax_slots) {   // the tensor-core path when it takes the shape (its amax goes to slots)
         const cudaError_t e = launch_lowrank_tc(x, m, k, l1, r, tp ? nullptr : t, tp, xs, ws, nullptr, nullptr, s);
         if (e != cudaErrorNotSupported) return e;
     }
-    const int grid = (int)((m + 15) / 16);
-    const int mode = tp ? kLrPacked : (amax_word ? kLrTAmax : kLrT);
+    const int64_t grid64 = (m + 15) / 16;
+    if (amax_slots && (tp || grid64 > kAmaxSlots)) return cudaErrorNotSupported;   // one slot per CTA
+    const int grid = (int)grid64;
+    const int mode = tp ? kLrPacked : ((amax_word || amax_slots) ? kLrTAmax : kLrT);
+    if (amax_slots) *n_slots = grid;
     const __nv_bfloat16 *l = (const __nv_bfloat16 *)l1;
     __nv_bfloat16 *tpb = (__nv_bfloat16 *)tp;
     if (bf16 && k % 64 == 0 && r % 8 == 0 && (reinterpret_cast<uintptr_t>(l1) & 15u) == 0) {
@@ -343,14 +354,18 @@ cudaError_t launch_lowrank_down(const void *x, bool bf16, int64_t m, int64_t k, 
         });
         if (se != cudaSuccess) return se;
         const __nv_bfloat16 *xb = (const __nv_bfloat16 *)x;
-        if (mode == kLrT) k_lowrank_staged<kLrT><<<grid, kLsThreads, kLsSmem, s>>>(xb, m, k, l, r, t, xs, ws, tpb, amax_word);
+        if (mode == kLrT)
+            k_lowrank_staged<kLrT><<<grid, kLsThreads, kLsSmem, s>>>(xb, m, k, l, r, t, xs, ws, tpb, amax_word, amax_slots);
         else if (mode == kLrPacked)
-            k_lowrank_staged<kLrPacked><<<grid, kLsThreads, kLsSmem, s>>>(xb, m, k, l, r, t, xs, ws, tpb, amax_word);
-        else k_lowrank_staged<kLrTAmax><<<grid, kLsThreads, kLsSmem, s>>>(xb, m, k, l, r, t, xs, ws, tpb, amax_word);
+            k_lowrank_staged<kLrPacked><<<grid, kLsThreads, kLsSmem, s>>>(xb, m, k, l, r, t, xs, ws, tpb, amax_word,
+                                                                         amax_slots);
+        else
+            k_lowrank_staged<kLrTAmax><<<grid, kLsThreads, kLsSmem, s>>>(xb, m, k, l, r, t, xs, ws, tpb, amax_word,
+                                                                        amax_slots);
         return cudaGetLastError();
     }
-    if (bf16) launch_lr(mode, grid, (const __nv_bfloat16 *)x, m, k, l, r, t, xs, ws, tpb, amax_word, s);
-    else launch_lr(mode, grid, (const float *)x, m, k, l, r, t, xs, ws, tpb, amax_word, s);
+    if (bf16) launch_lr(mode, grid, (const __nv_bfloat16 *)x, m, k, l, r, t, xs, ws, tpb, amax_word, amax_slots, s);
+    else launch_lr(mode, grid, (const float *)x, m, k, l, r, t, xs, ws, tpb, amax_word, amax_slots, s);
     return cudaGetLastError();
 }
 

@@ -126,10 +126,15 @@ cudaError_t launch_select_fixed(const void *w, bool bf16, int64_t n, int64_t k, 
 // t (m x r fp32) when tp is null; else the packed GEMM operand tp (m x 64
 // bf16, [hi | lo] of t / (xs * ws), xs = ws = null meaning 1).  With
 // amax_word (and tp null) the max |x| of the whole tensor is also
-// atomically folded into *amax_word (which must be zeroed beforehand).
+// atomically folded into *amax_word (which must be zeroed beforehand); with
+// amax_slots instead, one maximum per CTA is written to amax_slots (every
+// slot written, *n_slots of them, so nothing needs clearing), or
+// cudaErrorNotSupported (nothing launched) when more than kAmaxSlots CTAs
+// would be needed.
 cudaError_t launch_lowrank_down(const void *x, bool bf16, int64_t m, int64_t k, const void *l1, int r,
                                 float *t, const float *xs, const float *ws, void *tp, cudaStream_t s,
-                                unsigned int *amax_word = nullptr);
+                                unsigned int *amax_word = nullptr, float *amax_slots = nullptr,
+                                int *n_slots = nullptr);
 // Tensor-core down-projection of bf16 x (one pass over x): writes t (m x r
 // fp32) or, when t is null, the packed operand tp (as launch_lowrank_down);
 // with amax_word (zeroed beforehand) also folds in max |x|.  Returns

@@ -207,10 +207,15 @@ def test_dit_layers_full_size(mxq, orc, fmt):
 @pytest.mark.parametrize("fmt", LOWRANK_FMTS)
 @pytest.mark.parametrize("hadamard_b", [0, 64])
 @pytest.mark.parametrize("x_dtype", ["bf16", "f32"])
-def test_quantize_lowrank_fused(mxq, orc, fmt, hadamard_b, x_dtype):
+@pytest.mark.parametrize("shape", [(77, 300, 512, 24), (16448, 64, 64, 16)], ids=["small", "tall"])
+def test_quantize_lowrank_fused(mxq, orc, fmt, hadamard_b, x_dtype, shape):
     """The fused activation path equals quantize + lowrank_down_packed bit for
-    bit, and its codes/scales equal the oracle's."""
-    d = _inputs(40 + fmt, 77, 300, 512, 24)
+    bit, and its codes/scales equal the oracle's.  The tall shape takes, for
+    the tensor-scaled formats, the route that folds every CTA's maximum into
+    a cleared word (more 16-row CTAs than amax slots); the small one the
+    per-CTA slots."""
+    m, n, k, r = shape
+    d = _inputs(40 + fmt, m, n, k, r)
     x = dev(d["x"], x_dtype)
     wq = mxq.quantize(dev(d["w"], "bf16"), fmt, hadamard_b, mxq.MMA)
     l1 = dev(d["l1"], "bf16")

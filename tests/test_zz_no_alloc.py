@@ -74,15 +74,17 @@ def test_noalloc_matches_workspace_entry_point(mxq, fmt):
         assert err.max() <= 1e-4 * np.abs(y_ref).max()
 
 
-@pytest.mark.parametrize("x_fp32,hadamard_b", [(True, 0), (False, 128), (True, 128)])
-def test_noalloc_cleared_amax_route(mxq, x_fp32, hadamard_b):
-    """NVFP4 with fp32 input or with the rotation takes the route that clears
-    the amax word in the shared array and folds every CTA's maximum into it:
-    two calls in a row (the second on a different input, so a stale maximum
-    would show) equal the workspace entry point bit for bit."""
+@pytest.mark.parametrize("x_fp32,hadamard_b,m0,k", [(True, 0, 260, 512), (False, 128, 260, 512),
+                                                    (True, 128, 260, 512), (True, 0, 16384, 64)])
+def test_noalloc_amax_routes(mxq, x_fp32, hadamard_b, m0, k):
+    """NVFP4 through the other amax routes in the shared array: per-CTA
+    maxima of the mma.sync low-rank kernel (fp32 input), of the amax pass
+    (with the rotation), and, past 960 16-row CTAs, the amax word cleared and
+    folded into: two calls in a row (the second on a different input, so a
+    stale maximum would show) equal the workspace entry point bit for bit."""
     fmt = 2
     for call, seed in enumerate((21, 22)):
-        x, w, l1, _ = _inputs(seed + 7 * hadamard_b, 260 + 64 * call, 512, 384, 32)
+        x, w, l1, _ = _inputs(seed + 7 * hadamard_b, m0 + 64 * call, k, 384, 32)
         if x_fp32:
             x = x.float()
         if call == 1:
