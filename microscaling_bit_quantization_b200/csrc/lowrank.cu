@@ -6,8 +6,11 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <cstring>
+
 #include "mxq_formats.cuh"
 #include "mxq_internal.h"
+#include "tc_ptx.cuh"
 
 namespace mxq {
 
@@ -57,6 +60,10 @@ __global__ void __launch_bounds__(kLrWarps * 32) k_lowrank(const T *__restrict__
                                                          float *amax_slots) {
     __shared__ float red[kLrWarps][16][33];
     __shared__ float wmax[kLrWarps];
+    // launched with programmatic serialization: nothing global is touched
+    // before the previous kernel has completed
+    pdl_wait();
+    pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, tq = lane & 3;
     const int64_t row0 = (int64_t)blockIdx.x * 16;
@@ -212,6 +219,8 @@ __global__ void __launch_bounds__(kLsThreads) k_lowrank_staged(const __nv_bfloat
     extern __shared__ __align__(128) uint8_t ls_smem[];
     __shared__ float red[4][16][33];
     __shared__ float wmax[4];
+    pdl_wait();   // as in k_lowrank
+    pdl_launch_dependents();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t row0 = (int64_t)blockIdx.x * 16;
     const int nchunks = (int)(k >> 6);
@@ -313,15 +322,28 @@ __global__ void __launch_bounds__(kLsThreads) k_lowrank_staged(const __nv_bfloat
 
 }  // namespace
 
+// One launch with the programmatic-serialization attribute.
+template <typename... P, typename... A>
+static cudaError_t launch_pdl(void (*kern)(P...), int grid, int threads, size_t smem, cudaStream_t s, A... args) {
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3((unsigned)threads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1] = {pdl_attribute()};
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 template <typename T>
-static void launch_lr(int mode, int grid, const T *x, int64_t m, int64_t k, const __nv_bfloat16 *l1, int r, float *t,
-                      const float *xs, const float *ws, __nv_bfloat16 *tp, unsigned int *amax, float *slots,
-                      cudaStream_t s) {
+static cudaError_t launch_lr(int mode, int grid, const T *x, int64_t m, int64_t k, const __nv_bfloat16 *l1, int r,
+                             float *t, const float *xs, const float *ws, __nv_bfloat16 *tp, unsigned int *amax,
+                             float *slots, cudaStream_t s) {
     const int threads = kLrWarps * 32;
-    if (mode == kLrT) k_lowrank<T, kLrT><<<grid, threads, 0, s>>>(x, m, k, l1, r, t, xs, ws, tp, amax, slots);
-    else if (mode == kLrPacked)
-        k_lowrank<T, kLrPacked><<<grid, threads, 0, s>>>(x, m, k, l1, r, t, xs, ws, tp, amax, slots);
-    else k_lowrank<T, kLrTAmax><<<grid, threads, 0, s>>>(x, m, k, l1, r, t, xs, ws, tp, amax, slots);
+    auto kern = mode == kLrT ? k_lowrank<T, kLrT> : mode == kLrPacked ? k_lowrank<T, kLrPacked> : k_lowrank<T, kLrTAmax>;
+    return launch_pdl(kern, grid, threads, 0, s, x, m, k, l1, r, t, xs, ws, tp, amax, slots);
 }
 
 cudaError_t launch_lowrank_down(const void *x, bool bf16, int64_t m, int64_t k, const void *l1, int r, float *t,
@@ -354,19 +376,13 @@ cudaError_t launch_lowrank_down(const void *x, bool bf16, int64_t m, int64_t k, 
         });
         if (se != cudaSuccess) return se;
         const __nv_bfloat16 *xb = (const __nv_bfloat16 *)x;
-        if (mode == kLrT)
-            k_lowrank_staged<kLrT><<<grid, kLsThreads, kLsSmem, s>>>(xb, m, k, l, r, t, xs, ws, tpb, amax_word, amax_slots);
-        else if (mode == kLrPacked)
-            k_lowrank_staged<kLrPacked><<<grid, kLsThreads, kLsSmem, s>>>(xb, m, k, l, r, t, xs, ws, tpb, amax_word,
-                                                                         amax_slots);
-        else
-            k_lowrank_staged<kLrTAmax><<<grid, kLsThreads, kLsSmem, s>>>(xb, m, k, l, r, t, xs, ws, tpb, amax_word,
-                                                                        amax_slots);
-        return cudaGetLastError();
+        auto kern = mode == kLrT ? k_lowrank_staged<kLrT>
+                  : mode == kLrPacked ? k_lowrank_staged<kLrPacked> : k_lowrank_staged<kLrTAmax>;
+        return launch_pdl(kern, grid, kLsThreads, (size_t)kLsSmem, s, xb, m, k, l, r, t, xs, ws, tpb, amax_word,
+                          amax_slots);
     }
-    if (bf16) launch_lr(mode, grid, (const __nv_bfloat16 *)x, m, k, l, r, t, xs, ws, tpb, amax_word, amax_slots, s);
-    else launch_lr(mode, grid, (const float *)x, m, k, l, r, t, xs, ws, tpb, amax_word, amax_slots, s);
-    return cudaGetLastError();
+    if (bf16) return launch_lr(mode, grid, (const __nv_bfloat16 *)x, m, k, l, r, t, xs, ws, tpb, amax_word, amax_slots, s);
+    return launch_lr(mode, grid, (const float *)x, m, k, l, r, t, xs, ws, tpb, amax_word, amax_slots, s);
 }
 
 cudaError_t launch_pack_l2(const void *l2, int r, int64_t n, void *l2p, cudaStream_t s) {
