@@ -463,7 +463,7 @@ def routed_stack_row(mxq, torch, dev, timer, peaks):
             "frac_of_fp8_int8_peak": total_flop / (pass_ms * 1e-3) / 1e12 / fp8_peak, "fp8_int8_peak": fp8_peak,
             "per_format": split,
             "launches_per_layer_call": "2 (k_quantize or k_quantize_int8_row, k_gemm) + 1 for FP8 per tensor "
-                                       "(amax pass) + a memset of the scale padding for MXFP8 at K = 1152"}
+                                       "(amax pass)"}
 
 
 def run_ours(args, world, rank, local):

@@ -339,6 +339,26 @@ __global__ void __launch_bounds__(kQThreads, 2) k_quantize(const T *__restrict__
         }
         return;
     }
+    if (fmt_block(F) && (F == kMXFP8 || F == kMXFP4 || F == kNVFP4) && a.layout == 1) {
+        // the MMA layout's padding (columns S .. s_pad - 1 of every row, and
+        // every column of the rows up to the next multiple of 128) holds zero
+        // scales, which this grid writes: no clearing of the buffer first.
+        // Disjoint from the scales written above, so no ordering is needed.
+        const uint32_t S = (uint32_t)(a.cols / BLK), sp = (uint32_t)a.s_pad;
+        const uint32_t rows = (uint32_t)a.rows, rows_pad = (rows + 127u) & ~127u;
+        const uint32_t n1 = rows * (sp - S), n = n1 + (rows_pad - rows) * sp;
+        for (uint32_t i = blockIdx.x * kQThreads + threadIdx.x; i < n; i += gridDim.x * kQThreads) {
+            uint32_t r, sc;
+            if (i < n1) {
+                r = i / (sp - S);
+                sc = S + (i - r * (sp - S));
+            } else {
+                r = rows + (i - n1) / sp;
+                sc = (i - n1) % sp;
+            }
+            reinterpret_cast<uint8_t *>(a.scales)[mma_scale_offset32(r, sc, s_pad4)] = 0;
+        }
+    }
     if (a.tp) {
         // packed low-rank operand, one row per warp, one value per lane:
         // u = t / alpha, hi = bf16(u), lo = bf16(u - hi), zeros past r
@@ -1307,13 +1327,10 @@ cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols
     a.r = pack ? pack->r : 0;
     a.w_ts = pack ? pack->w_ts : nullptr;
     a.tp = pack ? (__nv_bfloat16 *)pack->tp : nullptr;
-    if (layout == 1 && fmt_byte_scales(fmt)) {
+    (void)scales_bytes;   // the whole buffer: k_quantize writes every byte of it, padding included
+    if (layout == 1 && fmt_byte_scales(fmt)) {   // k_quantize writes the padding's zero scales itself
         int64_t S = cols / fmt_block(fmt);
         a.s_pad = (S + 15) / 16 * 16;
-        if (a.s_pad != S || rows % 128) {   // padding bytes must read as 0
-            e = cudaMemsetAsync(scales, 0, scales_bytes, s);
-            if (e != cudaSuccess) return e;
-        }
     }
     if (a.total_chunks == 0) {
         if (fmt_tensor_scaled(fmt)) {   // empty tensor: amax 0 -> scale 1

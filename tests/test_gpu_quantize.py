@@ -44,6 +44,25 @@ def test_quantize_small_ragged(mxq, orc, fmt, dtype, hadamard_b):
         assert_qtensor_equal(q, ref, layout_mma=layout == mxq.MMA)
 
 
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+@pytest.mark.parametrize("rows,cols", [(37, 1088), (300, 1152), (128, 1152), (1, 64)])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_quantize_mma_scale_padding(mxq, orc, fmt, rows, cols, dtype):
+    """The MMA layout pads the byte scales to 16 columns and 128 rows; the
+    quantizer writes those padding bytes as zero itself, so a scale buffer
+    that held 0xFF (a NaN E8M0 scale) before the call reads as the oracle's
+    scales plus zero padding after it."""
+    x = nasty_matrix(500 + fmt + rows, rows, cols)
+    ref = orc.quantize(host_values(x, dtype), fmt)
+    q = mxq.alloc_qtensor(fmt, rows, cols, mxq.MMA)
+    for _ in range(2):   # the second call writes over its own output
+        q.codes.fill_(0xFF)
+        q.scales.fill_(0xFF)
+        mxq.quantize(dev(x, dtype), fmt, 0, mxq.MMA, out=q)
+        torch.cuda.synchronize()
+        assert_qtensor_equal(q, ref, layout_mma=True)
+
+
 @pytest.mark.parametrize("rows,cols", [(4097, 2064), (5, 5120), (3, 2560), (1, 4096), (1027, 4608), (6, 5136),
                                        (2, 2048)])
 def test_quantize_int8_row_long_rows(mxq, orc, rows, cols):
