@@ -2,12 +2,15 @@
 // block-diagonal Hadamard + block-scaled quantization, dequantization,
 // standalone Hadamard, element casts, and per-channel format selection.
 //
-// Work mapping shared by all kernels: a row of `cols` elements is cut into
+// Work mapping of the chunk kernels: a row of `cols` elements is cut into
 // 16-element chunks; lane i of a warp owns chunk (32*w + i), so a warp reads
 // 32 consecutive chunks (1 KB of bf16) and every quantization block (16, 32
 // or 64 elements) or Hadamard block (<= 256 elements) lies in aligned lanes
 // of one warp.  Block maxima and cross-lane butterflies use warp shuffles.
-// Loads are 16-byte vectors; codes are stored as 8- or 16-byte vectors.
+// Loads are 16-byte vectors; codes are stored as 8- or 16-byte vectors.  Two
+// kernels that need no block structure work on 16-byte words instead: the
+// tensor-amax pass of unrotated tensors (`k_amax_words`) and INT8 per row
+// over long rows staged in shared memory (`k_quantize_int8_row_staged`).
 #include <cuda_runtime.h>
 
 #include <cstring>
