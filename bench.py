@@ -16,7 +16,13 @@ same layer on its own batch (data parallel over tokens, no collective on the
 data path: weak scaling); the timed region is bracketed by a barrier and a
 device synchronize, and the time is the max over ranks.  Inputs and outputs
 rotate over 4 device-resident sets (about 620 MB > 126 MB L2), so every step
-reads its operands from HBM.
+reads its operands from HBM.  The timed steps replay CUDA graphs of 20
+consecutive steps (and of the K mod 20 left), captured before timing: the
+host issues one launch per 20 steps instead of two Python API calls per step,
+whose cost (~40-90 us per step through ctypes) would otherwise pace the
+device, and the programmatic edges between kernels hold across steps.  The
+same steps launched eagerly are timed after (`ms_per_step_eager`), and the
+end-to-end leg stays eager.
 
 After the timed steps the same process measures, on the same stream: the
 dominant kernel (the GEMM) and the activation side by CUDA-graph replay of
@@ -521,6 +527,37 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     assert mxq.check() == 0
 
+    # Consecutive steps are captured once as CUDA graphs (each step's three kernels and the
+    # programmatic edges between all of them, across steps too): a graph of G = 20 steps (five
+    # rounds of the rotating sets) and one of the K mod G left over; the timed region replays the
+    # first K // G times and the second once -- exactly K steps, one host launch per 20, so the
+    # number is the device's, not the Python submission's.  The same steps launched eagerly are
+    # timed after, for reference (ms_per_step_eager).
+    G = 20 if args.steps >= 20 else max(args.steps, 1)
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for i in range(N_SETS):
+            step(i)
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+
+    def capture(n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(n):
+                step(i)
+        return g
+
+    g_full = capture(G)
+    rem = args.steps % G
+    g_rem = capture(rem) if rem else None
+    g_full.replay()
+    if g_rem is not None:
+        g_rem.replay()
+    torch.cuda.synchronize()
+    assert mxq.check() == 0
+
     # ---- timed region: exactly K steps between a pair of events on the launching stream
     sampler = ClockSampler(local)
     sampler.start()
@@ -529,14 +566,28 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
-    for i in range(args.steps):
-        step(i)
+    for _ in range(args.steps // G):
+        g_full.replay()   # steps i .. i + G - 1 use the sets in the same rotation (G % N_SETS == 0)
+    if g_rem is not None:
+        g_rem.replay()
     end.record(stream)
     torch.cuda.synchronize()
     _barrier(world)
     clocks = sampler.stop()
     ms_local = start.elapsed_time(end) / args.steps
     ms, value = job_throughput(ms_local, world, FLOP_STEP)
+    assert mxq.check() == 0
+    del g_full, g_rem
+
+    # the same K steps launched eagerly through the Python API (two calls per step)
+    _barrier(world)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(args.steps):
+        step(i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    args.ms_eager = _max_over_ranks(start.elapsed_time(end) / args.steps, world)
     assert mxq.check() == 0
 
     peaks = _peaks()
@@ -799,12 +850,16 @@ def finish(args, world, rank, ms, value, clocks, gemm_tflops, fp4_peak, peaks, p
         line = {
             "metric": "qlinear TFLOPS (NVFP4 W4A4 + rank-32 low-rank), whole step",
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "ms_per_step": ms, "ms_per_step_eager": args.ms_eager,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "nvfp4(e2m1+ue4m3)xnvfp4->f32 acc, bf16 out", "data": "synthetic",
             "config": {"workload": WORKLOAD, "m": M, "k": K, "n": N, "rank": RANK, "out": "bf16",
                        "l2": "4 rotating input/output sets (~620 MB > 126 MB L2), no flush in the step loop; "
                              "bandwidth rows flushed (256 MiB read) before each launch",
-                       "parallelism": "dp%d (independent batch per GPU)" % world},
+                       "parallelism": "dp%d (independent batch per GPU)" % world,
+                       "launch": "the timed steps replay CUDA graphs of 20 consecutive steps (60 kernels with "
+                                 "programmatic edges, captured once before timing) and of the K mod 20 left; "
+                                 "ms_per_step_eager: the same steps launched eagerly through the Python API"},
             "roofline": {"bound": "tensor", "kernel": "k_gemm<NVFP4> (main + low-rank up MMAs, fused epilogue)",
                          "achieved": gemm_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
                          "frac": gemm_tflops / fp4_peak, "traffic": profiles_traffic,
