@@ -381,8 +381,8 @@ mxq_status mxq_quantize_lowrank(const void *x, int32_t xdtype, int64_t m, int64_
                                 size_t workspace_bytes, void *stream);
 
 /* Same as mxq_quantize_lowrank, but without a workspace argument: the
- * scratch it needs (the tensor-amax word and the m x r fp32 low-rank
- * activation, 4096 + 4*m*r bytes) lives in a 4 MiB array that the library
+ * scratch it needs (the tensor-amax word and per-CTA maxima, and the m x r
+ * fp32 low-rank activation, 4096 + 4*m*r bytes) lives in a 4 MiB array that the library
  * keeps in device memory, one per GPU that loads it, until the process
  * exits.  The pages describe no such call; it exists for callers that
  * cannot allocate device memory themselves: code embedded in a host
@@ -395,8 +395,9 @@ mxq_status mxq_quantize_lowrank(const void *x, int32_t xdtype, int64_t m, int64_
  *     that device current); make that first call before any stream capture.
  *   All calls share the array: calls whose work overlaps on the GPU (other
  *     streams, other host threads) race on it and must be ordered by the
- *     caller.  The amax word is cleared on every call; nothing else in the
- *     array needs to start at zero.
+ *     caller.  Every per-CTA maximum a call reads is written by that call,
+ *     and a call that folds into the amax word clears it first: nothing in
+ *     the array needs to start at zero.
  *   The call itself allocates and frees nothing.
  * Other arguments, results and errors as mxq_quantize_lowrank. */
 mxq_status mxq_quantize_lowrank_noalloc(const void *x, int32_t xdtype, int64_t m, int64_t k,
