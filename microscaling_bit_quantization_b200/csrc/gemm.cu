@@ -645,8 +645,7 @@ cudaError_t launch_kind(const GemmParams &p, int grid, cudaStream_t s) {
     cudaError_t e = smem_opt_in.run(
         [] { return cudaFuncSetAttribute(k_gemm<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES); });
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid, 1, 1);   // clusters of 2 from __cluster_dims__
     cfg.blockDim = dim3(kGemmThreads, 1, 1);
     cfg.dynamicSmemBytes = SMEM_BYTES;

@@ -325,8 +325,7 @@ __global__ void __launch_bounds__(kLsThreads) k_lowrank_staged(const __nv_bfloat
 // One launch with the programmatic-serialization attribute.
 template <typename... P, typename... A>
 static cudaError_t launch_pdl(void (*kern)(P...), int grid, int threads, size_t smem, cudaStream_t s, A... args) {
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid, 1, 1);
     cfg.blockDim = dim3((unsigned)threads, 1, 1);
     cfg.dynamicSmemBytes = smem;

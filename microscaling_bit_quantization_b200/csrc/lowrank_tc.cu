@@ -481,8 +481,7 @@ cudaError_t launch_lowrank_tc(const void *x, int64_t m, int64_t k, const void *l
         if (lt_smem_bytes(kb_max) > LT_SMEM_MAX) continue;
         int max_clusters = max_clusters_cache[dev][li].load(std::memory_order_relaxed) - 1;
         if (max_clusters < 0) {
-            cudaLaunchConfig_t q;
-            memset(&q, 0, sizeof(q));
+            cudaLaunchConfig_t q = {};
             q.gridDim = dim3((unsigned)S, 1, 1);
             q.blockDim = dim3(LT_THREADS, 1, 1);
             q.dynamicSmemBytes = (size_t)LT_SMEM_MAX;
@@ -536,8 +535,7 @@ cudaError_t launch_lowrank_tc(const void *x, int64_t m, int64_t k, const void *l
               encode_2d(&p.tma_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, l1, 32, (uint64_t)k, 64, 32, 64,
                         CU_TENSOR_MAP_SWIZZLE_64B);
     const int smem = lt_smem_bytes(p.kb_max);
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(best_clusters * best_s), 1, 1);
     cfg.blockDim = dim3(LT_THREADS, 1, 1);
     cfg.dynamicSmemBytes = (size_t)smem;

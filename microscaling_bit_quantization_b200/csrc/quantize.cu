@@ -1237,8 +1237,7 @@ static cudaError_t launch_amax_slots(const void *x, bool bf16, int64_t rows, int
         const int64_t want = (words + per_cta - 1) / per_cta;
         const int grid = (int)(want < cap ? want : cap);
         *n_slots = grid;
-        cudaLaunchConfig_t cfg;
-        memset(&cfg, 0, sizeof(cfg));
+        cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)grid, 1, 1);
         cfg.blockDim = dim3(kQThreads, 1, 1);
         cfg.stream = s;
@@ -1261,8 +1260,7 @@ static void launch_qf(const T *x, const QuantArgs &a, cudaStream_t s) {
     const int64_t steps = (a.total_chunks + kQThreads - 1) / kQThreads;
     const int64_t cap = (int64_t)sm_count_cached() * 2;   // two 512-thread CTAs per SM
     const int grid = (int)(steps < cap ? steps : cap);
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid, 1, 1);
     cfg.blockDim = dim3(kQThreads, 1, 1);
     cfg.stream = s;
@@ -1273,7 +1271,7 @@ static void launch_qf(const T *x, const QuantArgs &a, cudaStream_t s) {
 }
 
 template <typename T>
-static void launch_q(int fmt, int grid, const T *x, const QuantArgs &a, cudaStream_t s) {
+static void launch_q(int fmt, const T *x, const QuantArgs &a, cudaStream_t s) {
     switch (fmt) {
     case kMXFP8: launch_qf<T, kMXFP8>(x, a, s); break;
     case kMXFP4: launch_qf<T, kMXFP4>(x, a, s); break;
@@ -1342,9 +1340,8 @@ cudaError_t launch_quantize(const void *x, bool bf16, int64_t rows, int64_t cols
         }
         return cudaSuccess;
     }
-    int grid = grid_for((a.total_chunks + 31) / 32, sm_count_cached());
-    if (bf16) launch_q<__nv_bfloat16>(fmt, grid, (const __nv_bfloat16 *)x, a, s);
-    else launch_q<float>(fmt, grid, (const float *)x, a, s);
+    if (bf16) launch_q<__nv_bfloat16>(fmt, (const __nv_bfloat16 *)x, a, s);
+    else launch_q<float>(fmt, (const float *)x, a, s);
     return cudaGetLastError();
 }
 
@@ -1413,8 +1410,7 @@ static uint32_t select_set_of(const int *cands, int ncand) {
 template <typename T, uint32_t MASK>
 static void launch_select_set(const T *w, const SelectSetArgs &a, cudaStream_t s) {
     const int64_t ctas = (a.n + kSelThreads / 32 - 1) / (kSelThreads / 32);
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(ctas < 1 ? 1 : ctas), 1, 1);
     cfg.blockDim = dim3(kSelThreads, 1, 1);
     cfg.stream = s;
