@@ -462,33 +462,64 @@ __device__ __forceinline__ float group_max(float a) {
 // a row in consecutive lanes.  Butterfly stage h pairs elements i and i+h
 // (bit h of i clear) into (a+c, a-c); stages h < 16 stay inside the lane,
 // stages h >= 16 pair lanes that differ in bit h/16.  Then every element is
-// multiplied by RN(1/sqrt(b)).  All lanes of the warp must call this.
-__device__ __forceinline__ void hadamard_chunk(float v[16], int b, int lane) {
+// multiplied by norm = RN(1/sqrt(b)) (hadamard_chunk computes it; a loop over
+// many chunks passes it in).  All lanes of the warp must call this.
+__device__ __forceinline__ void hadamard_chunk_n(float v[16], int b, int lane, float norm) {
+    // stage h = 1 inside the lane, element pairs (i, i + 1)
+    if (b > 1) {
 #pragma unroll
-    for (int h = 1; h < 16; h <<= 1) {
+        for (int i = 0; i < 16; i += 2) {
+            const float a = v[i], c = v[i + 1];
+            v[i] = __fadd_rn(a, c);
+            v[i + 1] = __fsub_rn(a, c);
+        }
+    }
+    // stages h = 2, 4, 8 inside the lane on adjacent pairs, two-wide: a + c,
+    // and a - c as the FMA c * (-1) + a (exact product, one rounding: the
+    // same value as the subtraction)
+#pragma unroll
+    for (int h = 2; h < 16; h <<= 1) {
         if (h < b) {
 #pragma unroll
-            for (int i = 0; i < 16; i++) {
+            for (int i = 0; i < 16; i += 2) {
                 if (!(i & h)) {
-                    float a = v[i], c = v[i + h];
-                    v[i] = __fadd_rn(a, c);
-                    v[i + h] = __fsub_rn(a, c);
+                    const float2 a = make_float2(v[i], v[i + 1]), c = make_float2(v[i + h], v[i + h + 1]);
+                    const float2 sum = __fadd2_rn(a, c), dif = __ffma2_rn(c, make_float2(-1.0f, -1.0f), a);
+                    v[i] = sum.x;
+                    v[i + 1] = sum.y;
+                    v[i + h] = dif.x;
+                    v[i + h + 1] = dif.y;
                 }
             }
         }
     }
-    for (int h = 16; h < b; h <<= 1) {
-        int lm = h >> 4;
-        bool upper = (lane & lm) != 0;
+    // stages h = 16 lm across lanes that differ in bit lm: the lower lane
+    // keeps v + p, the upper p - v, both as the FMA (+-1) * v + p
 #pragma unroll
-        for (int i = 0; i < 16; i++) {
-            float p = __shfl_xor_sync(0xFFFFFFFFu, v[i], lm);
-            v[i] = upper ? __fsub_rn(p, v[i]) : __fadd_rn(v[i], p);
+    for (int lm = 1; lm < 16; lm <<= 1) {
+        if (16 * lm < b) {
+            const float sg = (lane & lm) ? -1.0f : 1.0f;
+            const float2 sg2 = make_float2(sg, sg);
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+                const float p0 = __shfl_xor_sync(0xFFFFFFFFu, v[i], lm);
+                const float p1 = __shfl_xor_sync(0xFFFFFFFFu, v[i + 1], lm);
+                const float2 r = __ffma2_rn(sg2, make_float2(v[i], v[i + 1]), make_float2(p0, p1));
+                v[i] = r.x;
+                v[i + 1] = r.y;
+            }
         }
     }
-    float norm = __frsqrt_rn((float)b);
+    const float2 n2 = make_float2(norm, norm);
 #pragma unroll
-    for (int i = 0; i < 16; i++) v[i] = __fmul_rn(v[i], norm);
+    for (int i = 0; i < 16; i += 2) {
+        const float2 r = __fmul2_rn(make_float2(v[i], v[i + 1]), n2);
+        v[i] = r.x;
+        v[i + 1] = r.y;
+    }
+}
+__device__ __forceinline__ void hadamard_chunk(float v[16], int b, int lane) {
+    hadamard_chunk_n(v, b, lane, __frsqrt_rn((float)b));
 }
 
 // Byte offset of scale (row r, scale column s) in the MMA scale layout:

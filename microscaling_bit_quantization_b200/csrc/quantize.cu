@@ -269,6 +269,7 @@ __global__ void __launch_bounds__(kQThreads, 2) k_quantize(const T *__restrict__
         else rt = recip_of(s_t);
     }
 
+    const float hnorm = a.hadamard_b ? __frsqrt_rn((float)a.hadamard_b) : 1.0f;   // RN(1/sqrt(b))
     // this thread's chunk c = (row, colc), advanced by kQThreads chunks a step
     uint32_t c = c_begin + threadIdx.x;
     uint32_t row = fdiv(c, a.cpr);
@@ -310,7 +311,7 @@ __global__ void __launch_bounds__(kQThreads, 2) k_quantize(const T *__restrict__
                 } else {
                     if (cn < c_end) raw_load(pre[j], x + (int64_t)cn * 16);
                 }
-                if (a.hadamard_b) hadamard_chunk(v, a.hadamard_b, lane);
+                if (a.hadamard_b) hadamard_chunk_n(v, a.hadamard_b, lane, hnorm);
                 float amax = amax16(v);
                 if (F == kNumFmt) {   // tensor-amax pass only
                     tensor_max = fmaxf(tensor_max, amax);
