@@ -457,8 +457,9 @@ __device__ __forceinline__ float group_max(float a) {
 
 // ----------------------------------------------------------------- Hadamard
 
-// Block-diagonal Hadamard rotation of size b ("Bridging the Gap ...",
-// item 3) over 16-element chunks, one chunk per lane, consecutive chunks of
+// Block-diagonal Hadamard rotation of size b (a power of two in [2, 256]:
+// the callers check it) ("Bridging the Gap ...", item 3) over 16-element
+// chunks, one chunk per lane, consecutive chunks of
 // a row in consecutive lanes.  Butterfly stage h pairs elements i and i+h
 // (bit h of i clear) into (a+c, a-c); stages h < 16 stay inside the lane,
 // stages h >= 16 pair lanes that differ in bit h/16.  Then every element is
