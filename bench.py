@@ -296,7 +296,7 @@ class Timer:
         self.stream.wait_stream(side)
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
             for i in range(n):
                 fn(i)
         g.replay()
@@ -429,7 +429,7 @@ def routed_stack_row(mxq, torch, dev, timer, peaks):
         timer.stream.wait_stream(side)
         torch.cuda.synchronize()
         gr = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gr):
+        with torch.cuda.graph(gr, capture_error_mode="thread_local"):
             for layer, step in pairs:
                 call(layer, step)
         return gr
@@ -542,9 +542,9 @@ def run_ours(args, world, rank, local):
     stream.wait_stream(side)
     torch.cuda.synchronize()
 
-    def capture(n):
+    def capture(n):   # thread_local: under torchrun the NCCL watchdog thread may query events meanwhile
         g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
             for i in range(n):
                 step(i)
         return g
